@@ -1,0 +1,187 @@
+/*
+ * ts_verify.h -- C ABI of libtsverify.so, the B200 (sm_100a) implementation
+ * of TokenSwift's per-step verification path.
+ *
+ * TokenSwift accelerates ultra-long generation by drafting several tokens,
+ * verifying them in one tree-structured pass over the full KV cache, keeping
+ * the longest valid candidate, penalising recently generated tokens, and
+ * drafting over a partial KV cache that keeps the initial tokens plus the
+ * most important ones ("TokenSwift - A framework for accelerating the
+ * generation of ultra-long text", aiboss88.com, section "TokenSwift's
+ * technical principles"; "From Hours to Minutes: Lossless Acceleration of
+ * Ultra-Long Sequence Generation up to 100K Tokens", arxivlens.com,
+ * "Technical Contribution").  This library implements the three kernels of
+ * that step; the model around them (projections, LM head, draft heads) is
+ * the caller's.
+ *
+ * Conventions for every entry point
+ *  - Memory: the caller owns every buffer.  The library never allocates,
+ *    frees or synchronises (except ts_workspace_status, which says so).
+ *    "device" pointers are CUDA device memory on the current device.
+ *  - Streams: `stream` is a cudaStream_t passed as void*; NULL is the legacy
+ *    default stream.  Calls are asynchronous with respect to the host.
+ *  - Errors: arguments are validated on the host before anything is
+ *    launched; an invalid call returns a non-zero ts_status and launches
+ *    nothing.  A launch failure returns TS_ERR_CUDA.  Conditions that only
+ *    the device can see (a window id outside the vocabulary, an expired
+ *    bounded wait) are recorded in the workspace's status word, read by
+ *    ts_workspace_status().
+ *  - Workspace: sized by the matching *_workspace_size() call, at least
+ *    256-byte aligned, zero-filled once by the caller before first use
+ *    (every call leaves it zero-filled again apart from the status word).
+ *    Concurrent calls need distinct workspaces.
+ *  - bf16 tensors are raw IEEE bfloat16 bit patterns; every device pointer
+ *    must be 16-byte aligned.
+ *  - No C++ exception crosses this interface.
+ */
+#ifndef TS_VERIFY_H
+#define TS_VERIFY_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    TS_OK = 0,
+    TS_ERR_INVALID_ARG = 1, /* a host-checked argument is invalid */
+    TS_ERR_UNSUPPORTED = 2, /* valid, but outside what this build supports */
+    TS_ERR_WORKSPACE = 3,   /* workspace missing, too small or misaligned */
+    TS_ERR_CUDA = 4,        /* a CUDA runtime call or launch failed */
+    TS_ERR_TIMEOUT = 5,     /* device: a bounded wait expired (status word) */
+    TS_ERR_DEVICE_ARG = 6   /* device: invalid data seen on the device (status word) */
+} ts_status;
+
+/* Largest draft tree, in nodes (ancestor sets are 64-bit masks). */
+#define TS_MAX_TREE 64
+
+/* Static description of a status code; never NULL. */
+const char *ts_status_string(int status);
+
+/* Library ABI version (major * 100 + minor). */
+int ts_version(void);
+
+/*
+ * Tree-masked attention of the draft-tree queries over the full KV cache.
+ *
+ * Source: tree-based multi-candidate verification ("TokenSwift's technical
+ * principles", aiboss88.com; tencent article, parallel-verification figure:
+ * candidates go through the model with the full KV cache under tree-based
+ * attention; arxivlens "Technical Contribution": a 3-ary tree).
+ *
+ * For tree node i and query head h (KV head g = h / (Hq / Hkv)):
+ *   out[i,h,:] = sum_j softmax_j(scale * q[i,h,:] . k[g,j,:]) v[g,j,:]
+ * over j in [0, n_ctx) and j = n_ctx + a for every node a on the root path
+ * of i (i included).  The tree tail rows [n_ctx, n_ctx + n_tree) of the
+ * cache hold the tree nodes' own K/V, node a at row n_ctx + a.
+ *
+ *  q            device bf16 [n_tree, Hq, D], contiguous (node-major).
+ *  k_cache      device bf16 [Hkv, kv_cap, D], contiguous; rows [0, n_ctx)
+ *               context, [n_ctx, n_ctx + n_tree) the tree tail, rows beyond
+ *               are not read.
+ *  v_cache      same layout as k_cache.
+ *  kv_cap       rows per KV head in the cache, >= n_ctx + n_tree.
+ *  n_heads_q, n_heads_kv, head_dim
+ *               Hq % Hkv == 0; head_dim is 64 or 128.
+ *  n_ctx        context length, >= 0 (0: the tree attends only to itself).
+ *  n_tree       tree nodes, 1 .. TS_MAX_TREE.
+ *  parent       HOST int32 [n_tree]: parent[0] = -1, 0 <= parent[i] < i
+ *               (BFS/topological order).  Read before the call returns.
+ *  softmax_scale  finite, usually 1/sqrt(D).
+ *  out          device fp32 [n_tree, Hq, D], written entirely.
+ *  workspace    device, >= ts_tree_verify_attn_workspace_size(...) bytes.
+ */
+size_t ts_tree_verify_attn_workspace_size(int n_heads_q, int n_heads_kv, int head_dim,
+                                          int n_ctx, int n_tree);
+int ts_tree_verify_attn(const void *q, const void *k_cache, const void *v_cache, int64_t kv_cap,
+                        int n_heads_q, int n_heads_kv, int head_dim, int n_ctx, int n_tree,
+                        const int32_t *parent, float softmax_scale, float *out,
+                        void *workspace, size_t workspace_bytes, void *stream);
+
+/*
+ * Dynamic partial-KV update: importance scores, sink + top-budget selection
+ * and the gather into the compact draft cache.
+ *
+ * Source: "TokenSwift's technical principles" (aiboss88.com): the initial
+ * KV cache is retained and the rest is replaced in order of token
+ * importance; tencent article 动态KV缓存更新: the partial cache is updated
+ * dynamically to cut KV load time; the draft model is the target model run
+ * with that partial cache (无损的输出质量).
+ *
+ *   score[g,n] = (1/G) sum_{h in group g} softmax_n(scale * q_last[h] . k[g,n])
+ * over n in [0, n_ctx).  Per KV head g the kept set is [0, n_sink) plus the
+ * `budget` highest scores of [n_sink, n_ctx) (equal scores: lower position
+ * first), listed in ascending position; n_keep = min(n_ctx, n_sink+budget).
+ *
+ *  q_last       device bf16 [Hq, D] (the root node's query rows).
+ *  k_cache, v_cache, kv_cap, n_heads_q, n_heads_kv, head_dim
+ *               as for ts_tree_verify_attn; only rows [0, n_ctx) are read.
+ *  n_ctx        >= 1.   n_sink, budget >= 0.
+ *  softmax_scale  finite.
+ *  scores_out   device fp32 [Hkv, n_ctx], or NULL (not returned).
+ *  idx_out      device int32 [Hkv, n_keep], ascending positions.
+ *  k_partial, v_partial
+ *               device bf16 [Hkv, partial_cap, D]; rows [0, n_keep) are
+ *               written with the kept rows, in idx_out order.
+ *  partial_cap  >= n_keep.
+ */
+size_t ts_kv_importance_select_workspace_size(int n_heads_q, int n_heads_kv, int head_dim,
+                                              int n_ctx);
+int ts_kv_importance_select(const void *q_last, const void *k_cache, const void *v_cache,
+                            int64_t kv_cap, int n_heads_q, int n_heads_kv, int head_dim,
+                            int n_ctx, int n_sink, int budget, float softmax_scale,
+                            float *scores_out, int32_t *idx_out, void *k_partial,
+                            void *v_partial, int64_t partial_cap, void *workspace,
+                            size_t workspace_bytes, void *stream);
+
+/*
+ * Contextual penalty, per-node target argmax and the longest accepted path.
+ *
+ * Source: "TokenSwift's technical principles" (aiboss88.com): a penalty on
+ * recently generated tokens; the longest valid candidate is the output;
+ * tencent article 上下文惩罚 and the figure text (the longest valid sequence,
+ * e.g. "is the father of", is kept).
+ *
+ * For every id in the window (a set), a positive logit is divided by
+ * `penalty` and a non-positive one multiplied by it (binary32,
+ * round-to-nearest).  argmax[i] is the largest penalised logit of node i,
+ * ties to the lowest id, NaN counted as -inf.  The root is valid; a draft
+ * node is valid when its parent is valid and its token equals the argmax at
+ * its parent (it is what greedy decoding would have produced).  The accepted
+ * path is the root path of the deepest valid node, equal depths going to
+ * the lowest node index.
+ *
+ *  logits       device fp32 [n_tree, vocab]; not modified.
+ *  n_tree       1 .. TS_MAX_TREE.   vocab >= 1.
+ *  window       device int32 [window_len] (may be NULL when window_len is
+ *               0); ids outside [0, vocab) are ignored and flagged as
+ *               TS_ERR_DEVICE_ARG in the status word.
+ *  penalty      finite, > 0.
+ *  parent       HOST int32 [n_tree], as for ts_tree_verify_attn.
+ *  tree_tokens  device int32 [n_tree]; tree_tokens[0] (the root) is unused.
+ *  argmax_out   device int32 [n_tree], or NULL.
+ *  accept_out   device int32 [2 + n_tree]: {L, bonus, path[0..L]} where L
+ *               is the number of accepted draft nodes, path[0] = 0 is the
+ *               root, and bonus = argmax at path[L]; entries past path[L]
+ *               are set to -1.
+ */
+size_t ts_penalize_accept_workspace_size(int n_tree, int vocab);
+int ts_penalize_accept(const float *logits, int n_tree, int vocab, const int32_t *window,
+                       int window_len, float penalty, const int32_t *parent,
+                       const int32_t *tree_tokens, int32_t *argmax_out, int32_t *accept_out,
+                       void *workspace, size_t workspace_bytes, void *stream);
+
+/*
+ * Reads the status word of a workspace after the work queued on `stream`
+ * has finished (this call synchronises `stream`).  Returns TS_OK or the
+ * first device-side error recorded since the last clear; clears the word
+ * when `clear` is non-zero.  Returns TS_ERR_CUDA if the copy fails.
+ */
+int ts_workspace_status(const void *workspace, void *stream, int clear);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* TS_VERIFY_H */
