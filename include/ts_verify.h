@@ -40,6 +40,12 @@
 #include <stddef.h>
 #include <stdint.h>
 
+#if defined(__GNUC__)
+#define TS_API __attribute__((visibility("default")))
+#else
+#define TS_API
+#endif
+
 #ifdef __cplusplus
 extern "C" {
 #endif
@@ -58,10 +64,10 @@ typedef enum {
 #define TS_MAX_TREE 64
 
 /* Static description of a status code; never NULL. */
-const char *ts_status_string(int status);
+TS_API const char *ts_status_string(int status);
 
 /* Library ABI version (major * 100 + minor). */
-int ts_version(void);
+TS_API int ts_version(void);
 
 /*
  * Tree-masked attention of the draft-tree queries over the full KV cache.
@@ -93,9 +99,9 @@ int ts_version(void);
  *  out          device fp32 [n_tree, Hq, D], written entirely.
  *  workspace    device, >= ts_tree_verify_attn_workspace_size(...) bytes.
  */
-size_t ts_tree_verify_attn_workspace_size(int n_heads_q, int n_heads_kv, int head_dim,
+TS_API size_t ts_tree_verify_attn_workspace_size(int n_heads_q, int n_heads_kv, int head_dim,
                                           int n_ctx, int n_tree);
-int ts_tree_verify_attn(const void *q, const void *k_cache, const void *v_cache, int64_t kv_cap,
+TS_API int ts_tree_verify_attn(const void *q, const void *k_cache, const void *v_cache, int64_t kv_cap,
                         int n_heads_q, int n_heads_kv, int head_dim, int n_ctx, int n_tree,
                         const int32_t *parent, float softmax_scale, float *out,
                         void *workspace, size_t workspace_bytes, void *stream);
@@ -127,9 +133,9 @@ int ts_tree_verify_attn(const void *q, const void *k_cache, const void *v_cache,
  *               written with the kept rows, in idx_out order.
  *  partial_cap  >= n_keep.
  */
-size_t ts_kv_importance_select_workspace_size(int n_heads_q, int n_heads_kv, int head_dim,
+TS_API size_t ts_kv_importance_select_workspace_size(int n_heads_q, int n_heads_kv, int head_dim,
                                               int n_ctx);
-int ts_kv_importance_select(const void *q_last, const void *k_cache, const void *v_cache,
+TS_API int ts_kv_importance_select(const void *q_last, const void *k_cache, const void *v_cache,
                             int64_t kv_cap, int n_heads_q, int n_heads_kv, int head_dim,
                             int n_ctx, int n_sink, int budget, float softmax_scale,
                             float *scores_out, int32_t *idx_out, void *k_partial,
@@ -167,8 +173,8 @@ int ts_kv_importance_select(const void *q_last, const void *k_cache, const void 
  *               root, and bonus = argmax at path[L]; entries past path[L]
  *               are set to -1.
  */
-size_t ts_penalize_accept_workspace_size(int n_tree, int vocab);
-int ts_penalize_accept(const float *logits, int n_tree, int vocab, const int32_t *window,
+TS_API size_t ts_penalize_accept_workspace_size(int n_tree, int vocab);
+TS_API int ts_penalize_accept(const float *logits, int n_tree, int vocab, const int32_t *window,
                        int window_len, float penalty, const int32_t *parent,
                        const int32_t *tree_tokens, int32_t *argmax_out, int32_t *accept_out,
                        void *workspace, size_t workspace_bytes, void *stream);
@@ -179,7 +185,7 @@ int ts_penalize_accept(const float *logits, int n_tree, int vocab, const int32_t
  * first device-side error recorded since the last clear; clears the word
  * when `clear` is non-zero.  Returns TS_ERR_CUDA if the copy fails.
  */
-int ts_workspace_status(const void *workspace, void *stream, int clear);
+TS_API int ts_workspace_status(const void *workspace, void *stream, int clear);
 
 #ifdef __cplusplus
 }

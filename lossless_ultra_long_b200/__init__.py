@@ -1,0 +1,236 @@
+"""B200-native TokenSwift verification path: thin ctypes binding of libtsverify.so.
+
+The three calls mirror the C ABI in ``include/ts_verify.h``; every step of
+the path runs in the library's CUDA kernels.  This module only checks
+tensor dtypes/devices, passes raw pointers and the current CUDA stream, and
+turns non-zero status codes into exceptions.  torch supplies device memory
+and streams.  There is no CPU fallback: if the library is not built, every
+call raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libtsverify.so")
+
+TS_MAX_TREE = 64
+STATUS = {0: "TS_OK", 1: "TS_ERR_INVALID_ARG", 2: "TS_ERR_UNSUPPORTED", 3: "TS_ERR_WORKSPACE",
+          4: "TS_ERR_CUDA", 5: "TS_ERR_TIMEOUT", 6: "TS_ERR_DEVICE_ARG"}
+
+EXPORTS = ("ts_status_string", "ts_version", "ts_tree_verify_attn_workspace_size",
+           "ts_tree_verify_attn", "ts_kv_importance_select_workspace_size",
+           "ts_kv_importance_select", "ts_penalize_accept_workspace_size", "ts_penalize_accept",
+           "ts_workspace_status")
+
+
+class TsError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {STATUS.get(status, status)} "
+                         f"({_lib().ts_status_string(status).decode()})")
+
+
+_LIB = None
+
+
+def _lib():
+    global _LIB
+    if _LIB is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"libtsverify.so is not built ({LIB_PATH}); run "
+                               "`python -m lossless_ultra_long_b200.build`")
+        lib = ctypes.CDLL(LIB_PATH)
+        P, i32, i64, f32, sz = (ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_float,
+                                ctypes.c_size_t)
+        lib.ts_status_string.restype = ctypes.c_char_p
+        lib.ts_status_string.argtypes = [i32]
+        lib.ts_version.restype = i32
+        lib.ts_tree_verify_attn_workspace_size.restype = sz
+        lib.ts_tree_verify_attn_workspace_size.argtypes = [i32, i32, i32, i32, i32]
+        lib.ts_tree_verify_attn.restype = i32
+        lib.ts_tree_verify_attn.argtypes = [P, P, P, i64, i32, i32, i32, i32, i32, P, f32, P, P,
+                                            sz, P]
+        lib.ts_kv_importance_select_workspace_size.restype = sz
+        lib.ts_kv_importance_select_workspace_size.argtypes = [i32, i32, i32, i32]
+        lib.ts_kv_importance_select.restype = i32
+        lib.ts_kv_importance_select.argtypes = [P, P, P, i64, i32, i32, i32, i32, i32, i32, f32,
+                                                P, P, P, P, i64, P, sz, P]
+        lib.ts_penalize_accept_workspace_size.restype = sz
+        lib.ts_penalize_accept_workspace_size.argtypes = [i32, i32]
+        lib.ts_penalize_accept.restype = i32
+        lib.ts_penalize_accept.argtypes = [P, i32, i32, P, i32, f32, P, P, P, P, P, sz, P]
+        lib.ts_workspace_status.restype = i32
+        lib.ts_workspace_status.argtypes = [P, P, i32]
+        _LIB = lib
+    return _LIB
+
+
+def library():
+    """The loaded ctypes handle (raises if the library is not built)."""
+    return _lib()
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _check_dev(name, t, dtype):
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+def _host_i32(a):
+    import numpy as np
+    arr = np.ascontiguousarray(a.cpu().numpy() if isinstance(a, torch.Tensor) else a,
+                               dtype=np.int32)
+    return arr, arr.ctypes.data_as(ctypes.c_void_p)
+
+
+def _raise(rc, where):
+    if rc != 0:
+        raise TsError(rc, where)
+
+
+def new_workspace(nbytes: int, device=None) -> torch.Tensor:
+    """A zero-filled uint8 device buffer (torch allocations are 512-byte aligned)."""
+    return torch.zeros(max(int(nbytes), 256), dtype=torch.uint8,
+                       device=device if device is not None else "cuda")
+
+
+# ----------------------------------------------------------- attention
+def tree_verify_attn_workspace_size(n_heads_q, n_heads_kv, head_dim, n_ctx, n_tree) -> int:
+    return int(_lib().ts_tree_verify_attn_workspace_size(n_heads_q, n_heads_kv, head_dim, n_ctx,
+                                                         n_tree))
+
+
+def tree_verify_attn(q, k_cache, v_cache, n_ctx: int, parent, out=None, workspace=None,
+                     softmax_scale: float | None = None, stream=None):
+    """Tree-masked attention (``ts_tree_verify_attn``).
+
+    q: bf16 [T, Hq, D]; k_cache, v_cache: bf16 [Hkv, kv_cap, D]; parent: host
+    int32 [T].  Returns fp32 [T, Hq, D].
+    """
+    _check_dev("q", q, torch.bfloat16)
+    _check_dev("k_cache", k_cache, torch.bfloat16)
+    _check_dev("v_cache", v_cache, torch.bfloat16)
+    t, hq, d = q.shape
+    hkv, cap, d2 = k_cache.shape
+    if v_cache.shape != k_cache.shape or d2 != d:
+        raise ValueError("k_cache / v_cache / q shapes disagree")
+    if out is None:
+        out = torch.empty((t, hq, d), dtype=torch.float32, device=q.device)
+    _check_dev("out", out, torch.float32)
+    if workspace is None:
+        workspace = new_workspace(tree_verify_attn_workspace_size(hq, hkv, d, n_ctx, t), q.device)
+    par, par_p = _host_i32(parent)
+    if len(par) != t:
+        raise ValueError("parent must have one entry per tree node")
+    scale = float(d) ** -0.5 if softmax_scale is None else float(softmax_scale)
+    rc = _lib().ts_tree_verify_attn(_ptr(q), _ptr(k_cache), _ptr(v_cache), cap, hq, hkv, d,
+                                    int(n_ctx), t, par_p, scale, _ptr(out), _ptr(workspace),
+                                    workspace.numel() * workspace.element_size(), _stream(stream))
+    _raise(rc, "ts_tree_verify_attn")
+    return out
+
+
+# ------------------------------------------------------------ selection
+def kv_importance_select_workspace_size(n_heads_q, n_heads_kv, head_dim, n_ctx) -> int:
+    return int(_lib().ts_kv_importance_select_workspace_size(n_heads_q, n_heads_kv, head_dim,
+                                                             n_ctx))
+
+
+def kv_importance_select(q_last, k_cache, v_cache, n_ctx: int, n_sink: int, budget: int,
+                         k_partial=None, v_partial=None, idx_out=None, scores_out=None,
+                         workspace=None, softmax_scale: float | None = None, stream=None,
+                         want_scores: bool = False):
+    """Sink + top-budget partial-KV update (``ts_kv_importance_select``).
+
+    Returns ``(idx [Hkv, n_keep] int32, k_partial, v_partial, scores or None)``.
+    """
+    _check_dev("q_last", q_last, torch.bfloat16)
+    _check_dev("k_cache", k_cache, torch.bfloat16)
+    _check_dev("v_cache", v_cache, torch.bfloat16)
+    hq, d = q_last.shape
+    hkv, cap, d2 = k_cache.shape
+    n_keep = min(n_ctx, n_sink + budget)
+    dev = q_last.device
+    if k_partial is None:
+        k_partial = torch.empty((hkv, n_keep, d), dtype=torch.bfloat16, device=dev)
+    if v_partial is None:
+        v_partial = torch.empty_like(k_partial)
+    if idx_out is None:
+        idx_out = torch.empty((hkv, n_keep), dtype=torch.int32, device=dev)
+    if want_scores and scores_out is None:
+        scores_out = torch.empty((hkv, n_ctx), dtype=torch.float32, device=dev)
+    for name, t, dt in (("k_partial", k_partial, torch.bfloat16),
+                        ("v_partial", v_partial, torch.bfloat16),
+                        ("idx_out", idx_out, torch.int32)):
+        _check_dev(name, t, dt)
+    if scores_out is not None:
+        _check_dev("scores_out", scores_out, torch.float32)
+    if workspace is None:
+        workspace = new_workspace(kv_importance_select_workspace_size(hq, hkv, d, n_ctx), dev)
+    scale = float(d) ** -0.5 if softmax_scale is None else float(softmax_scale)
+    rc = _lib().ts_kv_importance_select(
+        _ptr(q_last), _ptr(k_cache), _ptr(v_cache), cap, hq, hkv, d, int(n_ctx), int(n_sink),
+        int(budget), scale, _ptr(scores_out), _ptr(idx_out), _ptr(k_partial), _ptr(v_partial),
+        k_partial.shape[1], _ptr(workspace), workspace.numel(), _stream(stream))
+    _raise(rc, "ts_kv_importance_select")
+    return idx_out, k_partial, v_partial, scores_out
+
+
+# ------------------------------------------------------ penalty + accept
+def penalize_accept_workspace_size(n_tree, vocab) -> int:
+    return int(_lib().ts_penalize_accept_workspace_size(n_tree, vocab))
+
+
+def penalize_accept(logits, window, penalty: float, parent, tree_tokens, argmax_out=None,
+                    accept_out=None, workspace=None, stream=None, want_argmax: bool = True):
+    """Contextual penalty + per-node argmax + longest accepted path (``ts_penalize_accept``).
+
+    Returns ``(accept [2 + T] int32, argmax [T] int32 or None)``.
+    """
+    _check_dev("logits", logits, torch.float32)
+    _check_dev("tree_tokens", tree_tokens, torch.int32)
+    t, vocab = logits.shape
+    dev = logits.device
+    if window is not None and window.numel() > 0:
+        _check_dev("window", window, torch.int32)
+        wlen, wptr = window.numel(), _ptr(window)
+    else:
+        wlen, wptr = 0, None
+    if accept_out is None:
+        accept_out = torch.empty(2 + t, dtype=torch.int32, device=dev)
+    if want_argmax and argmax_out is None:
+        argmax_out = torch.empty(t, dtype=torch.int32, device=dev)
+    _check_dev("accept_out", accept_out, torch.int32)
+    if argmax_out is not None:
+        _check_dev("argmax_out", argmax_out, torch.int32)
+    if workspace is None:
+        workspace = new_workspace(penalize_accept_workspace_size(t, vocab), dev)
+    par, par_p = _host_i32(parent)
+    if len(par) != t:
+        raise ValueError("parent must have one entry per tree node")
+    rc = _lib().ts_penalize_accept(_ptr(logits), t, vocab, wptr, wlen, float(penalty), par_p,
+                                   _ptr(tree_tokens), _ptr(argmax_out), _ptr(accept_out),
+                                   _ptr(workspace), workspace.numel(), _stream(stream))
+    _raise(rc, "ts_penalize_accept")
+    return accept_out, argmax_out
+
+
+def workspace_status(workspace, clear: bool = True, stream=None) -> int:
+    """Device-side status word of a workspace (synchronises the stream)."""
+    return int(_lib().ts_workspace_status(_ptr(workspace), _stream(stream), int(clear)))

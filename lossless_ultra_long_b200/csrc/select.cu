@@ -1,0 +1,481 @@
+// select.cu -- dynamic partial-KV update: importance score, sink + top-budget
+// selection, and the gather into the compact draft cache.
+//
+// TokenSwift (aiboss88.com), "TokenSwift's technical principles": the
+// initial KV cache is kept and the rest is replaced in order of token
+// importance; tencent article 动态KV缓存更新: the partial cache is refreshed
+// during generation; 无损的输出质量: the draft model is the target model with
+// that partial cache.
+//
+// Pass 1 (grid: chunks x Hkv): s[h,n] = log2(e) * scale * q_last[h] . k[g,n]
+//   for the G query heads of KV head g.  Each lane loads 16 bytes of a key
+//   row (a row is D/8 lanes), forms the partial dots of several rows and
+//   heads, and a transpose-reduce across the row's lanes leaves one finished
+//   (row, head) dot per lane: one shuffle per dot instead of log2(D/8).
+//   Writes s (fp32 [Hq, n_ctx]) and a running (max, sum 2^(s-max)) per head
+//   and chunk.  K is read once: Hkv * n_ctx * D * 2 bytes.
+// Pass 2 (one 8-CTA cluster per KV head): merges the chunk partials into
+//   the softmax max / normaliser of each head, forms
+//   score[n] = (1/G) sum_h 2^(s[h,n] - M_h) / Z_h for its slice of
+//   positions, keeps the order-preserving bit pattern of every score in
+//   shared memory, and finds the budget-th largest candidate exactly with a
+//   4 x 8-bit radix select whose histograms are summed over the cluster
+//   through distributed shared memory.  Positions are then compacted in
+//   ascending order (sinks, every key above the threshold, and the first
+//   keys equal to it in position order, so equal scores go to the lower
+//   position) and the kept K/V rows are copied with 16-byte loads.
+#include <cooperative_groups.h>
+#include <math.h>
+
+#include "ts_internal.cuh"
+
+namespace cg = cooperative_groups;
+
+namespace ts {
+namespace {
+
+constexpr int kP1Threads = 256;
+constexpr int kClusterCtas = 8;
+constexpr int kP2Threads = 512;
+constexpr int kMaxSlice = 48 * 1024;   // positions per CTA held in shared memory
+constexpr int kMaxGroup = 8;
+
+// ------------------------------------------------------------------ pass 1
+template <int D, int GP>
+__global__ void __launch_bounds__(kP1Threads)
+score_logits_kernel(SelectArgs a, int chunk, int n_chunks)
+{
+    constexpr int LPR = D / 8;          // lanes per key row (16 bytes each)
+    constexpr int NV = LPR;             // values per lane before the reduce
+    constexpr int RL = NV / GP;         // rows per lane group per step
+    constexpr int GROUPS = 32 / LPR;    // lane groups per warp
+    constexpr int ROWS_PER_WARP = GROUPS * RL;
+
+    const int g = blockIdx.y;
+    const int c = blockIdx.x;
+    const int G = a.n_heads_q / a.n_heads_kv;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int li = lane % LPR, grp = lane / LPR;
+    const int n0 = c * chunk;
+    const int n1 = min(n0 + chunk, a.n_ctx);
+
+    float qf[GP][8];
+#pragma unroll
+    for (int h = 0; h < GP; ++h) {
+        if (h < G) {
+            const uint4 raw = *reinterpret_cast<const uint4 *>(
+                a.q_last + (int64_t)(g * G + h) * D + li * 8);
+            const __nv_bfloat162 *p2 = reinterpret_cast<const __nv_bfloat162 *>(&raw);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const float2 f = __bfloat1622float2(p2[e]);
+                qf[h][2 * e] = f.x * a.scale_log2;
+                qf[h][2 * e + 1] = f.y * a.scale_log2;
+            }
+        } else {
+#pragma unroll
+            for (int e = 0; e < 8; ++e)
+                qf[h][e] = 0.f;
+        }
+    }
+    // this lane's finished value is always head (li % GP), row slot li / GP
+    const int my_h = li % GP, my_j = li / GP;
+    float run_m = -INFINITY, run_l = 0.f;
+
+    const __nv_bfloat16 *kh = a.k + (int64_t)g * a.kv_cap * D;
+    float *s_out = reinterpret_cast<float *>(reinterpret_cast<char *>(a.workspace) + kHeaderBytes);
+    const int nwarps = kP1Threads / 32;
+    for (int base = n0 + warp * ROWS_PER_WARP; base < n1; base += nwarps * ROWS_PER_WARP) {
+        uint4 kr[RL];
+#pragma unroll
+        for (int j = 0; j < RL; ++j) {
+            const int n = base + grp * RL + j;
+            kr[j] = n < n1 ? __ldcs(reinterpret_cast<const uint4 *>(kh + (int64_t)n * D + li * 8))
+                           : make_uint4(0u, 0u, 0u, 0u);
+        }
+        float v[NV];
+#pragma unroll
+        for (int j = 0; j < RL; ++j) {
+            const __nv_bfloat162 *p2 = reinterpret_cast<const __nv_bfloat162 *>(&kr[j]);
+            float kf[8];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const float2 f = __bfloat1622float2(p2[e]);
+                kf[2 * e] = f.x;
+                kf[2 * e + 1] = f.y;
+            }
+#pragma unroll
+            for (int h = 0; h < GP; ++h) {
+                float acc = 0.f;
+#pragma unroll
+                for (int e = 0; e < 8; ++e)
+                    acc = fmaf(qf[h][e], kf[e], acc);
+                v[j * GP + h] = acc;
+            }
+        }
+        // transpose-reduce across the LPR lanes of the row group
+#pragma unroll
+        for (int o = NV / 2; o >= 1; o >>= 1) {
+            const bool upper = (li & o) != 0;
+#pragma unroll
+            for (int t = 0; t < o; ++t) {
+                const float send = upper ? v[t] : v[t + o];
+                const float keep = upper ? v[t + o] : v[t];
+                v[t] = keep + __shfl_xor_sync(0xffffffffu, send, o);
+            }
+        }
+        const int n = base + grp * RL + my_j;
+        if (my_h < G && n < n1) {
+            const float s = v[0];
+            s_out[(int64_t)(g * G + my_h) * a.n_ctx + n] = s;
+            const float m_new = fmaxf(run_m, s);
+            run_l = run_l * exp2f(run_m - m_new) + exp2f(s - m_new);
+            run_m = m_new;
+        }
+    }
+
+    // merge the running (max, sum) of every lane that holds head h
+    __shared__ float sm_m[kP1Threads], sm_l[kP1Threads];
+    sm_m[threadIdx.x] = run_m;
+    sm_l[threadIdx.x] = run_l;
+    __syncthreads();
+    if (threadIdx.x < G) {
+        const int h = threadIdx.x;
+        float M = -INFINITY;
+        for (int t = 0; t < kP1Threads; ++t)
+            if (((t & 31) % LPR) % GP == h)
+                M = fmaxf(M, sm_m[t]);
+        float L = 0.f;
+        for (int t = 0; t < kP1Threads; ++t)
+            if (((t & 31) % LPR) % GP == h && sm_m[t] != -INFINITY)
+                L += sm_l[t] * exp2f(sm_m[t] - M);
+        float *part = s_out + (size_t)a.n_heads_q * a.n_ctx;
+        float2 *pp = reinterpret_cast<float2 *>(part);
+        pp[(size_t)(g * G + h) * n_chunks + c] = make_float2(M, L);
+    }
+}
+
+// ------------------------------------------------------------------ pass 2
+__device__ __forceinline__ uint32_t order_key(float f)
+{
+    const uint32_t b = __float_as_uint(f);
+    return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
+}
+
+// exclusive scan of one int per thread over the block; returns the total
+__device__ int block_exclusive_scan(int x, int *scratch, int &excl)
+{
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    int incl = x;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o)
+            incl += y;
+    }
+    if (lane == 31)
+        scratch[warp] = incl;
+    __syncthreads();
+    if (warp == 0) {
+        const int nw = blockDim.x / 32;
+        int w = lane < nw ? scratch[lane] : 0;
+        int wi = w;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int y = __shfl_up_sync(0xffffffffu, wi, o);
+            if (lane >= o)
+                wi += y;
+        }
+        if (lane < nw)
+            scratch[32 + lane] = wi - w;
+        if (lane == nw - 1)
+            scratch[64] = wi;
+    }
+    __syncthreads();
+    excl = scratch[32 + warp] + incl - x;
+    const int total = scratch[64];
+    __syncthreads();
+    return total;
+}
+
+struct P2Shared {
+    int hist[256];
+    int scan[72];
+    float head_w[kMaxGroup];   // 1 / (G * Z_h)
+    float head_m[kMaxGroup];
+    int counts[4];             // [0] equal-to-threshold, [1] kept
+    int bcast[4];
+};
+
+template <int D>
+__global__ void __launch_bounds__(kP2Threads, 1)
+select_gather_kernel(SelectArgs a, int n_chunks, int slice)
+{
+    cg::cluster_group cluster = cg::this_cluster();
+    extern __shared__ __align__(16) unsigned char dsm[];
+    P2Shared &sh = *reinterpret_cast<P2Shared *>(dsm);
+    uint32_t *keys = reinterpret_cast<uint32_t *>(dsm + sizeof(P2Shared));
+
+    const int rank = (int)cluster.block_rank();
+    const int g = blockIdx.y;
+    const int G = a.n_heads_q / a.n_heads_kv;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int N = a.n_ctx;
+    const int p0 = min(rank * slice, N), p1 = min(p0 + slice, N);
+    const int64_t want = (int64_t)a.n_sink + a.budget;
+    const bool keep_all = want >= N;
+    const int n_keep = keep_all ? N : (int)want;
+
+    const float *s_all = reinterpret_cast<const float *>(
+        reinterpret_cast<const char *>(a.workspace) + kHeaderBytes);
+    const float2 *part = reinterpret_cast<const float2 *>(s_all + (size_t)a.n_heads_q * N);
+
+    // softmax max / normaliser per head of the group
+    if (warp < G) {
+        const float2 *pp = part + (size_t)(g * G + warp) * n_chunks;
+        float M = -INFINITY;
+        for (int c = lane; c < n_chunks; c += 32)
+            M = fmaxf(M, pp[c].x);
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1)
+            M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+        float L = 0.f;
+        for (int c = lane; c < n_chunks; c += 32)
+            if (pp[c].x != -INFINITY)
+                L += pp[c].y * exp2f(pp[c].x - M);
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1)
+            L += __shfl_xor_sync(0xffffffffu, L, o);
+        if (lane == 0) {
+            sh.head_m[warp] = M;
+            sh.head_w[warp] = 1.f / ((float)G * L);
+        }
+    }
+    __syncthreads();
+
+    // scores of this slice -> order-preserving keys in shared memory
+    for (int n = p0 + tid; n < p1; n += kP2Threads) {
+        float sc = 0.f;
+        for (int h = 0; h < G; ++h)
+            sc += exp2f(s_all[(size_t)(g * G + h) * N + n] - sh.head_m[h]) * sh.head_w[h];
+        keys[n - p0] = order_key(sc);
+        if (a.scores_out)
+            a.scores_out[(size_t)g * N + n] = sc;
+    }
+    __syncthreads();
+
+    // exact radix select of the budget-th largest key over [n_sink, N)
+    uint32_t prefix = 0u, pmask = 0u;
+    int need = a.budget;
+    const bool do_select = !keep_all && a.budget > 0;
+    if (do_select) {
+        const int c0 = max(p0, a.n_sink);
+        for (int pass = 0; pass < 4; ++pass) {
+            const int shift = 24 - 8 * pass;
+            for (int b = tid; b < 256; b += kP2Threads)
+                sh.hist[b] = 0;
+            __syncthreads();
+            for (int n = c0 + tid; n < p1; n += kP2Threads) {
+                const uint32_t key = keys[n - p0];
+                if ((key & pmask) == prefix)
+                    atomicAdd(&sh.hist[(key >> shift) & 255u], 1);
+            }
+            cluster.sync();
+            // Thread t looks at bin b = 255 - t; an inclusive scan over t is
+            // then a suffix sum over bins.  The digit is the bin with
+            // (keys in higher bins) < need <= (that count + its own keys).
+            const int b = 255 - tid;
+            int x = 0;
+            if (tid < 256)
+                for (int r = 0; r < kClusterCtas; ++r)
+                    x += cluster.map_shared_rank(&sh.hist[0], r)[b];
+            int above;
+            block_exclusive_scan(x, sh.scan, above);
+            if (tid < 256 && above < need && need <= above + x) {
+                sh.bcast[0] = b;
+                sh.bcast[1] = above;
+            }
+            cluster.sync();   // every CTA has read the histograms; digit is in bcast
+            const int d = sh.bcast[0];
+            need -= sh.bcast[1];
+            prefix |= (uint32_t)d << shift;
+            pmask |= 255u << shift;
+            __syncthreads();
+        }
+    }
+    // prefix is now the threshold key; `need` keys equal to it are kept
+
+    // positions of this slice: how many equal the threshold (candidates only)
+    const int per_thread = (p1 - p0 + kP2Threads - 1) / kP2Threads;
+    const int q0 = p0 + tid * per_thread, q1 = min(q0 + per_thread, p1);
+    int my_eq = 0;
+    if (do_select)
+        for (int n = max(q0, a.n_sink); n < q1; ++n)
+            my_eq += keys[n - p0] == prefix;
+    int eq_excl;
+    const int eq_total = block_exclusive_scan(my_eq, sh.scan, eq_excl);
+    if (tid == 0)
+        sh.counts[0] = eq_total;
+    cluster.sync();
+    int eq_before = 0;
+    for (int r = 0; r < rank; ++r)
+        eq_before += *cluster.map_shared_rank(&sh.counts[0], r);
+
+    // kept flags -> counts -> ascending slots
+    auto kept = [&](int n, int &eq_rank) -> bool {
+        if (keep_all || n < a.n_sink)
+            return true;
+        if (!do_select)
+            return false;
+        const uint32_t key = keys[n - p0];
+        if (key > prefix)
+            return true;
+        if (key == prefix)
+            return eq_rank++ < need;
+        return false;
+    };
+    int my_kept = 0;
+    {
+        int eq_rank = eq_before + eq_excl;
+        for (int n = q0; n < q1; ++n)
+            my_kept += kept(n, eq_rank);
+    }
+    int kept_excl;
+    const int kept_total = block_exclusive_scan(my_kept, sh.scan, kept_excl);
+    if (tid == 0)
+        sh.counts[1] = kept_total;
+    cluster.sync();
+    int kept_before = 0;
+    for (int r = 0; r < rank; ++r)
+        kept_before += *cluster.map_shared_rank(&sh.counts[1], r);
+    cluster.sync();   // no CTA may exit while others read its shared memory
+
+    // write indices; reuse the key slots of kept positions to list them
+    int32_t *idx = a.idx_out + (size_t)g * n_keep;
+    {
+        int eq_rank = eq_before + eq_excl;
+        int slot = kept_before + kept_excl;
+        for (int n = q0; n < q1; ++n)
+            if (kept(n, eq_rank)) {
+                if (slot < n_keep)
+                    idx[slot] = n;
+                else
+                    record_status(reinterpret_cast<WorkspaceHeader *>(a.workspace),
+                                  TS_ERR_DEVICE_ARG);
+                ++slot;
+            }
+    }
+    __syncthreads();
+
+    // gather: kept rows of this slice are idx[kept_before .. kept_before + kept_total)
+    constexpr int LPR = D / 8;   // lanes per row, 16 bytes each
+    const __nv_bfloat16 *kh = a.k + (int64_t)g * a.kv_cap * D;
+    const __nv_bfloat16 *vh = a.v + (int64_t)g * a.kv_cap * D;
+    __nv_bfloat16 *kp = a.k_partial + (int64_t)g * a.partial_cap * D;
+    __nv_bfloat16 *vp = a.v_partial + (int64_t)g * a.partial_cap * D;
+    const int rows_per_pass = kP2Threads / LPR;
+    const int li = tid % LPR;
+    __threadfence_block();
+    const int my_rows = min(kept_total, n_keep - kept_before);
+    for (int t = tid / LPR; t < my_rows; t += rows_per_pass) {
+        const int slot = kept_before + t;
+        const int n = __ldcg(&idx[slot]);
+        if (n < 0 || n >= N)
+            continue;
+        const uint4 kv = *reinterpret_cast<const uint4 *>(kh + (int64_t)n * D + li * 8);
+        const uint4 vv = *reinterpret_cast<const uint4 *>(vh + (int64_t)n * D + li * 8);
+        *reinterpret_cast<uint4 *>(kp + (int64_t)slot * D + li * 8) = kv;
+        *reinterpret_cast<uint4 *>(vp + (int64_t)slot * D + li * 8) = vv;
+    }
+}
+
+struct SelPlan {
+    int chunk, n_chunks, slice;
+};
+
+SelPlan make_sel_plan(int n_heads_kv, int n_ctx, int num_sms)
+{
+    SelPlan p;
+    int want = (num_sms * 4 + n_heads_kv - 1) / n_heads_kv;
+    const int min_chunk = 512;
+    int chunk = (n_ctx + want - 1) / want;
+    chunk = chunk < min_chunk ? min_chunk : chunk;
+    p.chunk = chunk;
+    p.n_chunks = (n_ctx + chunk - 1) / chunk;
+    p.slice = (n_ctx + kClusterCtas - 1) / kClusterCtas;
+    return p;
+}
+
+template <int D, int GP>
+cudaError_t launch_p1(const SelectArgs &a, const SelPlan &p, cudaStream_t stream)
+{
+    dim3 grid(p.n_chunks, a.n_heads_kv);
+    score_logits_kernel<D, GP><<<grid, kP1Threads, 0, stream>>>(a, p.chunk, p.n_chunks);
+    return cudaGetLastError();
+}
+
+template <int D>
+cudaError_t launch_d(const SelectArgs &a, const SelPlan &p, cudaStream_t stream)
+{
+    const int G = a.n_heads_q / a.n_heads_kv;
+    cudaError_t e;
+    if (G == 1)
+        e = launch_p1<D, 1>(a, p, stream);
+    else if (G == 2)
+        e = launch_p1<D, 2>(a, p, stream);
+    else if (G <= 4)
+        e = launch_p1<D, 4>(a, p, stream);
+    else
+        e = launch_p1<D, 8>(a, p, stream);
+    if (e != cudaSuccess)
+        return e;
+
+    const size_t smem = sizeof(P2Shared) + (size_t)p.slice * sizeof(uint32_t);
+    e = cudaFuncSetAttribute(select_gather_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)smem);
+    if (e != cudaSuccess)
+        return e;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(kClusterCtas, a.n_heads_kv, 1);
+    cfg.blockDim = dim3(kP2Threads, 1, 1);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = kClusterCtas;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, select_gather_kernel<D>, a, p.n_chunks, p.slice);
+}
+
+}  // namespace
+
+int select_supported(int n_heads_q, int n_heads_kv, int head_dim, int n_ctx)
+{
+    const int G = n_heads_q / n_heads_kv;
+    if (G > kMaxGroup)
+        return 0;
+    if (head_dim == 64 && G > 8)
+        return 0;
+    return (n_ctx + kClusterCtas - 1) / kClusterCtas <= kMaxSlice;
+}
+
+size_t select_workspace_bytes(int n_heads_q, int n_heads_kv, int head_dim, int n_ctx,
+                              int num_sms)
+{
+    (void)head_dim;
+    const SelPlan p = make_sel_plan(n_heads_kv, n_ctx, num_sms);
+    const size_t s_bytes = (size_t)n_heads_q * n_ctx * sizeof(float);
+    const size_t part = (size_t)n_heads_q * p.n_chunks * 2 * sizeof(float);
+    return kHeaderBytes + align_up(s_bytes + part, 256);
+}
+
+cudaError_t select_launch(const SelectArgs &a, int num_sms, cudaStream_t stream)
+{
+    const SelPlan p = make_sel_plan(a.n_heads_kv, a.n_ctx, num_sms);
+    return a.head_dim == 128 ? launch_d<128>(a, p, stream) : launch_d<64>(a, p, stream);
+}
+
+}  // namespace ts

@@ -1,0 +1,100 @@
+// ts_internal.cuh -- shared definitions of the libtsverify kernels (not part
+// of the public interface; the C ABI is include/ts_verify.h).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+#include <stdint.h>
+
+#include "ts_verify.h"
+
+namespace ts {
+
+// ---------------------------------------------------------------- workspace
+// Every workspace starts with this header.  `status` collects device-side
+// errors (ts_status codes, first one wins); the tickets serve "last CTA does
+// the epilogue" hand-offs and are returned to zero by the CTA that takes
+// the last ticket.
+struct WorkspaceHeader {
+    uint32_t status;
+    uint32_t tickets[63];
+};
+static_assert(sizeof(WorkspaceHeader) == 256, "header is one 256-byte line");
+constexpr size_t kHeaderBytes = sizeof(WorkspaceHeader);
+
+inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+__device__ __forceinline__ void record_status(WorkspaceHeader *ws, uint32_t code)
+{
+    atomicCAS(&ws->status, 0u, code);
+}
+
+// Ancestor sets of the draft tree, bit a of anc[i] set iff node a is on the
+// root path of node i (i included).  Passed by value as a kernel parameter.
+struct TreeMasks {
+    unsigned long long anc[TS_MAX_TREE];
+};
+
+struct TreeParents {
+    int8_t parent[TS_MAX_TREE];
+};
+
+// ------------------------------------------------------------ launch entry
+struct AttnArgs {
+    const __nv_bfloat16 *q;
+    const __nv_bfloat16 *k;
+    const __nv_bfloat16 *v;
+    float *out;
+    int64_t kv_cap;
+    int n_heads_q, n_heads_kv, head_dim;
+    int n_ctx, n_tree;
+    float scale_log2;   // softmax_scale * log2(e)
+    void *workspace;
+    size_t workspace_bytes;
+};
+
+size_t attn_workspace_bytes(int n_heads_q, int n_heads_kv, int head_dim, int n_ctx, int n_tree,
+                            int num_sms);
+cudaError_t attn_launch(const AttnArgs &a, const TreeMasks &masks, int num_sms,
+                        cudaStream_t stream);
+
+struct SelectArgs {
+    const __nv_bfloat16 *q_last;
+    const __nv_bfloat16 *k;
+    const __nv_bfloat16 *v;
+    int64_t kv_cap;
+    int n_heads_q, n_heads_kv, head_dim;
+    int n_ctx, n_sink, budget;
+    float scale_log2;
+    float *scores_out;
+    int32_t *idx_out;
+    __nv_bfloat16 *k_partial;
+    __nv_bfloat16 *v_partial;
+    int64_t partial_cap;
+    void *workspace;
+    size_t workspace_bytes;
+};
+
+size_t select_workspace_bytes(int n_heads_q, int n_heads_kv, int head_dim, int n_ctx,
+                              int num_sms);
+int select_supported(int n_heads_q, int n_heads_kv, int head_dim, int n_ctx);
+cudaError_t select_launch(const SelectArgs &a, int num_sms, cudaStream_t stream);
+
+struct PenalizeArgs {
+    const float *logits;
+    int n_tree, vocab;
+    const int32_t *window;
+    int window_len;
+    float penalty;
+    const int32_t *tree_tokens;
+    int32_t *argmax_out;
+    int32_t *accept_out;
+    void *workspace;
+    size_t workspace_bytes;
+};
+
+size_t penalize_workspace_bytes(int n_tree, int vocab);
+cudaError_t penalize_launch(const PenalizeArgs &a, const TreeParents &parents,
+                            cudaStream_t stream);
+
+}  // namespace ts

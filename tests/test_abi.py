@@ -1,0 +1,108 @@
+"""C-ABI boundary checks that need no GPU: the library loads, exports every
+symbol the public header declares, and rejects invalid arguments on the
+host before touching the device."""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "ts_verify.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from lossless_ultra_long_b200 import build
+    build.build()
+    import lossless_ultra_long_b200 as L
+    return L.library()
+
+
+def declared_symbols():
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"^TS_API[^(;]*?\b(ts_\w+)\s*\(", text, flags=re.M)))
+
+
+def test_header_declares_the_three_calls():
+    syms = declared_symbols()
+    for name in ("ts_tree_verify_attn", "ts_kv_importance_select", "ts_penalize_accept"):
+        assert name in syms
+
+
+def test_every_declared_symbol_is_exported(lib):
+    for name in declared_symbols():
+        assert hasattr(lib, name), name
+
+
+def test_binding_export_list_matches_header():
+    import lossless_ultra_long_b200 as L
+    assert set(L.EXPORTS) <= set(declared_symbols())
+
+
+def test_status_strings(lib):
+    for code in range(7):
+        assert lib.ts_status_string(code)
+    assert lib.ts_version() >= 100
+
+
+def _attn_call(lib, **over):
+    args = dict(q=1 << 20, k=1 << 20, v=1 << 20, kv_cap=100, hq=8, hkv=2, d=64, n_ctx=50, t=4,
+                parent=np.array([-1, 0, 0, 1], np.int32), scale=0.125, out=1 << 20,
+                ws=1 << 20, ws_bytes=1 << 30)
+    args.update(over)
+    P = ctypes.c_void_p
+    par = args["parent"]
+    return lib.ts_tree_verify_attn(P(args["q"]), P(args["k"]), P(args["v"]), args["kv_cap"],
+                                   args["hq"], args["hkv"], args["d"], args["n_ctx"], args["t"],
+                                   par.ctypes.data_as(P) if par is not None else None,
+                                   args["scale"], P(args["out"]), P(args["ws"]),
+                                   args["ws_bytes"], None)
+
+
+@pytest.mark.parametrize("over,code", [
+    (dict(q=0), 1),
+    (dict(hq=6, hkv=4), 1),
+    (dict(parent=np.array([0, 0, 0, 1], np.int32)), 1),
+    (dict(parent=np.array([-1, 0, 2, 1], np.int32)), 1),
+    (dict(parent=None), 1),
+    (dict(t=65, parent=np.array([-1] + list(range(64)), np.int32)), 1),
+    (dict(kv_cap=53), 1),
+    (dict(scale=float("nan")), 1),
+    (dict(q=(1 << 20) + 8), 1),
+    (dict(d=96), 2),
+    (dict(ws=0), 3),
+    (dict(ws=(1 << 20) + 128), 3),
+    (dict(ws_bytes=16), 3),
+])
+def test_attention_rejects_on_host(lib, over, code):
+    assert _attn_call(lib, **over) == code
+
+
+def test_select_and_penalize_reject_on_host(lib):
+    P = ctypes.c_void_p
+    a = P(1 << 20)
+    # partial_cap smaller than n_sink + budget
+    assert lib.ts_kv_importance_select(a, a, a, 1000, 8, 2, 64, 1000, 16, 240, 0.125, None, a, a,
+                                       a, 100, a, 1 << 30, None) == 1
+    # group larger than supported
+    assert lib.ts_kv_importance_select(a, a, a, 1000, 64, 2, 64, 1000, 16, 240, 0.125, None, a, a,
+                                       a, 256, a, 1 << 30, None) == 2
+    par = np.array([-1, 0], np.int32)
+    pp = par.ctypes.data_as(P)
+    assert lib.ts_penalize_accept(a, 2, 100, a, 4, ctypes.c_float(0.0), pp, a, None, a, a,
+                                  1 << 20, None) == 1
+    assert lib.ts_penalize_accept(a, 2, 100, None, 4, ctypes.c_float(1.2), pp, a, None, a, a,
+                                  1 << 20, None) == 1
+    assert lib.ts_penalize_accept(a, 2, 100, a, 4, ctypes.c_float(1.2), pp, a, None, a, a,
+                                  8, None) == 3
+
+
+def test_workspace_sizes_are_positive_and_zero_for_invalid(lib):
+    import lossless_ultra_long_b200 as L
+    assert L.tree_verify_attn_workspace_size(32, 8, 128, 102400, 40) > 0
+    assert L.tree_verify_attn_workspace_size(32, 8, 96, 1024, 40) == 0
+    assert L.kv_importance_select_workspace_size(32, 8, 128, 102400) > 0
+    assert L.penalize_accept_workspace_size(40, 128256) > 0
+    assert L.penalize_accept_workspace_size(0, 128256) == 0
