@@ -1,0 +1,484 @@
+#!/usr/bin/env python
+"""Benchmark of the TokenSwift verification hot path on B200.
+
+One step = one pass of the whole per-step hot path on the LLaMA3.1-8B
+100K-context workload (Hq=32, Hkv=8, D=128, n_ctx=102400, 40-node 3-ary
+tree):
+  1. ts_tree_verify_attn over the full cache (the headline call),
+  2. ts_kv_importance_select: 64 sinks + top-4032 into the partial cache,
+  3. the draft pass: ts_tree_verify_attn of a 4-node chain over that
+     4096-row partial cache,
+  4. ts_penalize_accept over fp32 logits [40, 128256], window 1024.
+The metric counts tree-verify calls: each step holds exactly one.
+
+Prints ONE JSON line (rank 0).  ``--impl reference`` times the fp64 CPU
+oracle on a bounded sample of the same step instead.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "tree-verify attn calls/s @100K ctx (LLaMA-8B GQA shape); % of HBM/tensor roofline"
+UNIT = "calls/s"
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--e2e-steps", type=int, default=50)
+    return ap.parse_args()
+
+
+def dist_env():
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return rank, world, local
+
+
+def workload():
+    from lossless_ultra_long_b200 import inputs as I
+    return I.LLAMA8B_100K
+
+
+def attn_bytes(hq, hkv, d, n_ctx, t):
+    """Algorithmic HBM bytes of one tree-verify call: K+V (context + tail, bf16),
+    Q (bf16) and O (fp32)."""
+    return 4 * hkv * d * (n_ctx + t) + 2 * t * hq * d + 4 * t * hq * d
+
+
+def attn_flops(hq, d, n_ctx, t):
+    return 4 * hq * t * d * (n_ctx + t)
+
+
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            j = json.load(f)
+        return float(j["hbm_gbs"]), float(j["bf16_tflops"]), "measured"
+    return 6650.0, 1590.0, "fallback"
+
+
+def attn_traffic_record():
+    """DRAM bytes per launch of the attention call from a committed ncu capture,
+    valid only while the kernel sources are unchanged since that capture."""
+    p = os.path.join(ROOT, "profiles", "attn_traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        rec = json.load(f)
+    h = hashlib.sha256()
+    for rel in rec.get("sources", []):
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            h.update(f.read())
+    if h.hexdigest() != rec.get("sources_sha256"):
+        return None
+    return float(rec["dram_bytes_per_call"])
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled during the timed region."""
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_bench_{os.getpid()}.csv")
+
+    def __enter__(self):
+        os.makedirs(os.path.dirname(self.path), exist_ok=True)
+        q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+        try:
+            self.fh = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={q}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=self.fh, stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+            self.fh.close()
+
+    def summary(self):
+        if self.proc is None or not os.path.exists(self.path):
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+        sm, smax, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        with open(self.path) as f:
+            for line in f:
+                parts = [x.strip() for x in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    sm.append(float(parts[1]))
+                    smax = float(parts[2])
+                except ValueError:
+                    continue
+                for name, val in zip(names, parts[5:9]):
+                    if val.lower() == "active":
+                        reasons.add(name)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": smax,
+                "samples": len(sm), "reasons": sorted(reasons)}
+
+
+# --------------------------------------------------------------------- ours
+class Step:
+    """Device-resident buffers and the four ABI calls of one verification step."""
+
+    def __init__(self, torch, L, I, w, dev):
+        from_bits = lambda b: torch.from_numpy(np.ascontiguousarray(b).view(np.int16)).view(
+            torch.bfloat16).to(dev)
+        self.torch, self.L, self.w = torch, L, w
+        self.parent = w.parent()
+        self.draft_parent = I.chain_tree(w.draft_tree)
+        q = I.gen_q(w)
+        k, v = I.gen_kv(w)
+        self.q = from_bits(q)
+        self.k, self.v = from_bits(k), from_bits(v)
+        del k, v
+        lg = I.gen_logits(w)
+        tokens, lg = I.gen_tree_tokens(w, self.parent, lg)
+        self.logits = torch.from_numpy(lg).to(dev)
+        self.window = torch.from_numpy(I.gen_window(w)).to(dev)
+        self.tokens = torch.from_numpy(tokens).to(dev)
+        hq, hkv, d = w.n_heads_q, w.n_heads_kv, w.head_dim
+        self.n_keep = w.n_sink + w.budget
+        cap = self.n_keep + w.draft_tree
+        self.kp = torch.zeros((hkv, cap, d), dtype=torch.bfloat16, device=dev)
+        self.vp = torch.zeros_like(self.kp)
+        # the draft chain's own K/V rows sit after the kept rows
+        dk = I.gen_q(w.with_(seed=w.seed + 100), n_nodes=w.draft_tree)   # any seeded bf16 rows
+        self.kp[:, self.n_keep:] = from_bits(dk[:, :hkv, :].transpose(1, 0, 2))
+        self.vp[:, self.n_keep:] = from_bits(dk[:, hkv:2 * hkv, :].transpose(1, 0, 2))
+        self.dq = from_bits(I.gen_draft_q(w))
+        self.idx = torch.empty((hkv, self.n_keep), dtype=torch.int32, device=dev)
+        self.out = torch.empty((w.n_tree, hq, d), dtype=torch.float32, device=dev)
+        self.dout = torch.empty((w.draft_tree, hq, d), dtype=torch.float32, device=dev)
+        self.accept = torch.empty(2 + w.n_tree, dtype=torch.int32, device=dev)
+        self.argmax = torch.empty(w.n_tree, dtype=torch.int32, device=dev)
+        self.ws_attn = L.new_workspace(L.tree_verify_attn_workspace_size(hq, hkv, d, w.n_ctx,
+                                                                         w.n_tree), dev)
+        self.ws_draft = L.new_workspace(L.tree_verify_attn_workspace_size(
+            hq, hkv, d, self.n_keep, w.draft_tree), dev)
+        self.ws_sel = L.new_workspace(L.kv_importance_select_workspace_size(hq, hkv, d, w.n_ctx),
+                                      dev)
+        self.ws_pen = L.new_workspace(L.penalize_accept_workspace_size(w.n_tree, w.vocab), dev)
+
+    def attn(self):
+        self.L.tree_verify_attn(self.q, self.k, self.v, self.w.n_ctx, self.parent, out=self.out,
+                                workspace=self.ws_attn)
+
+    def rest(self):
+        w, L = self.w, self.L
+        L.kv_importance_select(self.q[0], self.k, self.v, w.n_ctx, w.n_sink, w.budget,
+                               k_partial=self.kp, v_partial=self.vp, idx_out=self.idx,
+                               workspace=self.ws_sel)
+        L.tree_verify_attn(self.dq, self.kp, self.vp, self.n_keep, self.draft_parent,
+                           out=self.dout, workspace=self.ws_draft)
+        L.penalize_accept(self.logits, self.window, w.penalty, self.parent, self.tokens,
+                          argmax_out=self.argmax, accept_out=self.accept, workspace=self.ws_pen)
+
+    def step(self):
+        self.attn()
+        self.rest()
+
+
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+    import lossless_ultra_long_b200 as L
+    from lossless_ultra_long_b200 import inputs as I
+
+    rank, world, local = dist_env()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=dev)
+    L.library()
+    w = workload()
+    st = Step(torch, L, I, w, dev)
+    stream = torch.cuda.Stream(device=dev)
+
+    # warm-up eagerly (sets kernel attributes), then capture two graphs:
+    # the headline attention call and the rest of the step
+    with torch.cuda.stream(stream):
+        for _ in range(max(args.warmup, 3)):
+            st.step()
+    stream.synchronize()
+    g_attn, g_rest = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g_attn, stream=stream, capture_error_mode="thread_local"):
+        st.attn()
+    with torch.cuda.graph(g_rest, stream=stream, capture_error_mode="thread_local"):
+        st.rest()
+    with torch.cuda.stream(stream):
+        for _ in range(max(args.warmup, 3)):
+            g_attn.replay()
+            g_rest.replay()
+    stream.synchronize()
+
+    launches_per_step = None
+    c0 = L.kernel_launch_count()
+    with torch.cuda.stream(stream):
+        st.step()
+    stream.synchronize()
+    launches_per_step = L.kernel_launch_count() - c0
+
+    K = args.steps
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(K)]
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clk:
+        with torch.cuda.stream(stream):
+            t0.record(stream)
+            for i in range(K):
+                ev[i][0].record(stream)
+                g_attn.replay()
+                ev[i][1].record(stream)
+                g_rest.replay()
+            t1.record(stream)
+        torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    ms_total = t0.elapsed_time(t1)
+    attn_ms = [a.elapsed_time(b) for a, b in ev]
+    ms_t = torch.tensor([ms_total], device=dev)
+    if world > 1:
+        dist.all_reduce(ms_t, op=dist.ReduceOp.MAX)
+    ms_max = float(ms_t.item())
+
+    # end to end through the public API: per step, pinned host inputs are
+    # copied in, the four calls run, and the results are read back
+    e2e = run_e2e(torch, L, st, w, dev, stream, args.e2e_steps)
+    e2e_t = torch.tensor([e2e["ms_per_step"]], device=dev)
+    if world > 1:
+        dist.all_reduce(e2e_t, op=dist.ReduceOp.MAX)
+
+    out = None
+    if rank == 0:
+        hbm, tflops, src = measured_peaks()
+        attn_avg_s = statistics.mean(attn_ms) / 1e3
+        byts = attn_bytes(w.n_heads_q, w.n_heads_kv, w.head_dim, w.n_ctx, w.n_tree)
+        flops = attn_flops(w.n_heads_q, w.head_dim, w.n_ctx, w.n_tree)
+        achieved = byts / attn_avg_s / 1e9
+        value = world * K / (ms_max / 1e3)
+        e2e_value = world * 1e3 / float(e2e_t.item())
+        out = {
+            "metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": world,
+            "steps": K, "warmup": args.warmup, "ms_per_step": round(ms_max / K, 5),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic",
+            "config": {"workload": w.name, "n_heads_q": w.n_heads_q, "n_heads_kv": w.n_heads_kv,
+                       "head_dim": w.head_dim, "n_ctx": w.n_ctx, "n_tree": w.n_tree,
+                       "tree": "3-ary BFS depth 3", "step": "verify attn + importance select "
+                       "(64+4032) + 4-node draft attn over the partial cache + penalty/accept "
+                       "(V=128256, W=1024)", "l2": "inputs larger than L2 (420 MB KV per step)",
+                       "parallelism": f"replicas x{world}", "graphs": True},
+            "attn_call_us": round(attn_avg_s * 1e6, 2),
+            "attn_only_calls_per_s": round(1.0 / attn_avg_s, 1),
+            "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": hbm,
+                         "unit": "GB/s", "frac": round(achieved / hbm, 4),
+                         "peak_source": src, "traffic": attn_traffic_record(),
+                         "algorithmic_bytes": byts,
+                         "tensor_frac": round(flops / attn_avg_s / 1e12 / tflops, 4)},
+            "e2e": {"value": round(e2e_value, 2), "unit": UNIT,
+                    "h2d_bytes_per_step": e2e["h2d"], "d2h_bytes_per_step": e2e["d2h"]},
+            "gpu_launches": int(launches_per_step * K),
+            "clocks": clk.summary(),
+        }
+        if not args.no_cpu_baseline:
+            out["cpu_baseline"] = cpu_baseline(w)
+    if world > 1:
+        dist.barrier()
+        del g_attn, g_rest
+        dist.destroy_process_group()
+    return out
+
+
+def run_e2e(torch, L, st, w, dev, stream, steps):
+    """The same step through the Python API with host buffers: H2D of the
+    step's new inputs (queries, the tree's own K/V rows, logits, window,
+    tree tokens, draft queries) from pinned memory, the four calls, D2H of
+    the results (outputs, accept, kept indices)."""
+    hq, hkv, d, t = w.n_heads_q, w.n_heads_kv, w.head_dim, w.n_tree
+    pin = lambda x: x.cpu().pin_memory()
+    h_q, h_dq = pin(st.q), pin(st.dq)
+    h_kt = pin(st.k[:, w.n_ctx:w.n_ctx + t])
+    h_vt = pin(st.v[:, w.n_ctx:w.n_ctx + t])
+    h_lg, h_win, h_tok = pin(st.logits), pin(st.window), pin(st.tokens)
+    o_out = torch.empty_like(st.out, device="cpu").pin_memory()
+    o_dout = torch.empty_like(st.dout, device="cpu").pin_memory()
+    o_acc = torch.empty_like(st.accept, device="cpu").pin_memory()
+    o_idx = torch.empty_like(st.idx, device="cpu").pin_memory()
+    h2d = sum(x.numel() * x.element_size() for x in (h_q, h_dq, h_kt, h_vt, h_lg, h_win, h_tok))
+    d2h = sum(x.numel() * x.element_size() for x in (o_out, o_dout, o_acc, o_idx))
+
+    def one():
+        st.q.copy_(h_q, non_blocking=True)
+        st.dq.copy_(h_dq, non_blocking=True)
+        st.k[:, w.n_ctx:w.n_ctx + t].copy_(h_kt, non_blocking=True)
+        st.v[:, w.n_ctx:w.n_ctx + t].copy_(h_vt, non_blocking=True)
+        st.logits.copy_(h_lg, non_blocking=True)
+        st.window.copy_(h_win, non_blocking=True)
+        st.tokens.copy_(h_tok, non_blocking=True)
+        st.step()
+        o_out.copy_(st.out, non_blocking=True)
+        o_dout.copy_(st.dout, non_blocking=True)
+        o_acc.copy_(st.accept, non_blocking=True)
+        o_idx.copy_(st.idx, non_blocking=True)
+        stream.synchronize()
+
+    with torch.cuda.stream(stream):
+        for _ in range(3):
+            one()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(steps):
+            one()
+        e1.record(stream)
+    torch.cuda.synchronize()
+    return {"ms_per_step": e0.elapsed_time(e1) / steps, "h2d": h2d, "d2h": d2h}
+
+
+# ----------------------------------------------------------- the oracle
+class OracleSample:
+    """The fp64 oracle on a bounded sample of one step, scaled to a full step.
+
+    attn_rows of the T*Hq verify-attention rows, the importance select of KV
+    head 0 over the first sel_positions context positions, draft_rows of the
+    draft pass's rows, pen_nodes of the tree nodes' penalty/argmax, and the
+    acceptance walk; each part's time is scaled by the share it sampled."""
+
+    def __init__(self, w, attn_rows, sel_positions, draft_rows, pen_nodes):
+        import oracle
+        from lossless_ultra_long_b200 import inputs as I
+        oracle.build()
+        self.o, self.w = oracle, w
+        self.attn_rows, self.sel_positions = attn_rows, min(sel_positions, w.n_ctx)
+        self.draft_rows, self.pen_nodes = draft_rows, pen_nodes
+        self.q = I.gen_q(w)
+        self.k, self.v = I.gen_kv(w)
+        self.parent = w.parent()
+        self.n_keep = w.n_sink + w.budget
+        self.dq = I.gen_draft_q(w)
+        self.kp = np.ascontiguousarray(self.k[:, : self.n_keep + w.draft_tree])
+        self.vp = np.ascontiguousarray(self.v[:, : self.n_keep + w.draft_tree])
+        self.dparent = I.chain_tree(w.draft_tree)
+        lg = I.gen_logits(w)
+        self.tokens, self.lg = I.gen_tree_tokens(w, self.parent, lg)
+        self.win = I.gen_window(w)
+        self.rng = np.random.default_rng(0)
+        self.sample = (f"{attn_rows} of {w.n_tree * w.n_heads_q} verify-attention rows; "
+                       f"importance select of KV head 0 over {self.sel_positions} of "
+                       f"{w.n_ctx} positions (x{w.n_heads_kv} heads); {draft_rows} of "
+                       f"{w.draft_tree * w.n_heads_q} draft-pass rows; penalty/argmax of "
+                       f"{pen_nodes} of {w.n_tree} nodes; acceptance; scaled to one step")
+
+    def seconds_per_step(self):
+        o, w = self.o, self.w
+        rows_total = w.n_tree * w.n_heads_q
+        sel = self.rng.choice(rows_total, size=self.attn_rows, replace=False)
+        t0 = time.perf_counter()
+        o.tree_verify_attn_rows(self.q, self.k, self.v, w.n_ctx, self.parent,
+                                (sel // w.n_heads_q).astype(np.int32),
+                                (sel % w.n_heads_q).astype(np.int32))
+        t_attn = (time.perf_counter() - t0) * rows_total / self.attn_rows
+        g, n = w.group, self.sel_positions
+        t0 = time.perf_counter()
+        sc = o.importance_scores(self.q[0, :g], self.k[:1], n, g)
+        idx = o.select_topk(sc, w.n_sink, w.budget)
+        o.gather_rows(self.k[:1], idx)
+        o.gather_rows(self.v[:1], idx)
+        t_sel = (time.perf_counter() - t0) * w.n_heads_kv * w.n_ctx / n
+        drows = w.draft_tree * w.n_heads_q
+        dsel = self.rng.choice(drows, size=self.draft_rows, replace=False)
+        t0 = time.perf_counter()
+        o.tree_verify_attn_rows(self.dq, self.kp, self.vp, self.n_keep, self.dparent,
+                                (dsel // w.n_heads_q).astype(np.int32),
+                                (dsel % w.n_heads_q).astype(np.int32))
+        t_draft = (time.perf_counter() - t0) * drows / self.draft_rows
+        t0 = time.perf_counter()
+        am = o.penalize_argmax(self.lg[: self.pen_nodes], self.win, w.penalty)
+        t_pen = (time.perf_counter() - t0) * w.n_tree / self.pen_nodes
+        am_full = np.resize(am, w.n_tree).astype(np.int32)
+        t0 = time.perf_counter()
+        o.accept_longest(self.parent, self.tokens, am_full)
+        t_acc = time.perf_counter() - t0
+        return t_attn + t_sel + t_draft + t_pen + t_acc
+
+
+def oracle_threads():
+    return int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
+
+
+def cpu_baseline(w):
+    """About 10-30 s of oracle work on the host cores (rank 0, N = 1 leg)."""
+    smp = OracleSample(w, attn_rows=160, sel_positions=w.n_ctx, draft_rows=128, pen_nodes=40)
+    per_step = smp.seconds_per_step()
+    return {"value": round(1.0 / per_step, 6), "unit": UNIT, "cores": oracle_threads(),
+            "kind": "oracle", "sample": smp.sample, "seconds_per_step": round(per_step, 3)}
+
+
+def run_reference(args):
+    rank, world, _ = dist_env()
+    if rank != 0:
+        return None
+    w = workload()
+    K = max(1, args.steps)
+    smp = OracleSample(w, attn_rows=2, sel_positions=12800, draft_rows=4, pen_nodes=2)
+    for _ in range(min(args.warmup, 1)):
+        smp.seconds_per_step()
+    secs = [smp.seconds_per_step() for _ in range(K)]
+    per_step = statistics.mean(secs)
+    val = round(1.0 / per_step, 6)
+    return {"metric": METRIC, "value": val, "unit": UNIT, "n_gpus": world, "steps": K,
+            "warmup": args.warmup, "ms_per_step": round(per_step * 1e3, 3),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "impl": "reference",
+            "config": {"workload": w.name, "n_heads_q": w.n_heads_q, "n_heads_kv": w.n_heads_kv,
+                       "head_dim": w.head_dim, "n_ctx": w.n_ctx, "n_tree": w.n_tree},
+            "cpu_baseline": {"value": val, "unit": UNIT, "cores": oracle_threads(),
+                             "kind": "oracle", "sample": smp.sample},
+            "e2e": {"value": val, "unit": UNIT, "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+
+
+def main():
+    args = parse()
+    out = run_reference(args) if args.impl == "reference" else run_ours(args)
+    if out is not None:
+        print(json.dumps(out), flush=True)
+
+
+if __name__ == "__main__":
+    main()

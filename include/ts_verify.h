@@ -180,6 +180,12 @@ TS_API int ts_penalize_accept(const float *logits, int n_tree, int vocab, const 
                        void *workspace, size_t workspace_bytes, void *stream);
 
 /*
+ * Number of kernels this library has launched in this process (all
+ * devices, all entry points); a diagnostic for counting launches.
+ */
+TS_API unsigned long long ts_kernel_launch_count(void);
+
+/*
  * Reads the status word of a workspace after the work queued on `stream`
  * has finished (this call synchronises `stream`).  Returns TS_OK or the
  * first device-side error recorded since the last clear; clears the word

@@ -24,7 +24,7 @@ STATUS = {0: "TS_OK", 1: "TS_ERR_INVALID_ARG", 2: "TS_ERR_UNSUPPORTED", 3: "TS_E
 EXPORTS = ("ts_status_string", "ts_version", "ts_tree_verify_attn_workspace_size",
            "ts_tree_verify_attn", "ts_kv_importance_select_workspace_size",
            "ts_kv_importance_select", "ts_penalize_accept_workspace_size", "ts_penalize_accept",
-           "ts_workspace_status")
+           "ts_workspace_status", "ts_kernel_launch_count")
 
 
 class TsError(RuntimeError):
@@ -63,6 +63,8 @@ def _lib():
         lib.ts_penalize_accept_workspace_size.argtypes = [i32, i32]
         lib.ts_penalize_accept.restype = i32
         lib.ts_penalize_accept.argtypes = [P, i32, i32, P, i32, f32, P, P, P, P, P, sz, P]
+        lib.ts_kernel_launch_count.restype = ctypes.c_ulonglong
+        lib.ts_kernel_launch_count.argtypes = []
         lib.ts_workspace_status.restype = i32
         lib.ts_workspace_status.argtypes = [P, P, i32]
         _LIB = lib
@@ -229,6 +231,11 @@ def penalize_accept(logits, window, penalty: float, parent, tree_tokens, argmax_
                                    _ptr(workspace), workspace.numel(), _stream(stream))
     _raise(rc, "ts_penalize_accept")
     return accept_out, argmax_out
+
+
+def kernel_launch_count() -> int:
+    """Kernels the library has launched in this process."""
+    return int(_lib().ts_kernel_launch_count())
 
 
 def workspace_status(workspace, clear: bool = True, stream=None) -> int:

@@ -12,7 +12,8 @@
 // all G*T rows that share the head stream its K/V exactly once per split.
 // K/V tiles are staged in shared memory by cp.async (16-byte, XOR-swizzled
 // rows) in a three-stage ring; QK^T and PV run on mma.m16n8k16 bf16 with
-// fp32 accumulators; the softmax is the online (running max / sum) form in
+// fp32 accumulators (P enters PV as two bf16 parts, so PV keeps ~16
+// significant bits of P); the softmax is the online (running max / sum) form in
 // base 2.  Only tiles that reach the tree tail evaluate the ancestor mask.
 // Each split writes an unnormalised partial (acc, m, l) that a combine
 // kernel merges across splits with a log-sum-exp rescale; a single-split
@@ -67,10 +68,14 @@ __device__ __forceinline__ void mma_bf16(float (&c)[4], const uint32_t (&a)[4], 
         : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 
-__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi)
+// (lo, hi) floats -> bf16x2 of their rounding, and bf16x2 of the remainders
+__device__ __forceinline__ void split_bf16(float lo, float hi, uint32_t &big, uint32_t &small)
 {
     __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
-    return *reinterpret_cast<uint32_t *>(&h);
+    const float2 back = __bfloat1622float2(h);
+    __nv_bfloat162 r = __floats2bfloat162_rn(lo - back.x, hi - back.y);
+    big = *reinterpret_cast<uint32_t *>(&h);
+    small = *reinterpret_cast<uint32_t *>(&r);
 }
 
 // byte offset of 16-byte chunk `c` of tile row `r` (rows of D bf16)
@@ -243,14 +248,15 @@ attn_split_kernel(AttnArgs a, TreeMasks masks, int tiles_per_split, int n_split)
             o[dt][3] *= corr[1];
         }
 
-        // O += P V
+        // O += P V, with P = P_hi + P_lo (two bf16 parts, ~16 significant
+        // bits) so that few, large weights keep fp32-level accuracy
 #pragma unroll
         for (int kt = 0; kt < kTile / 16; ++kt) {
-            uint32_t pa[4];
-            pa[0] = pack_bf16(s[2 * kt][0], s[2 * kt][1]);
-            pa[1] = pack_bf16(s[2 * kt][2], s[2 * kt][3]);
-            pa[2] = pack_bf16(s[2 * kt + 1][0], s[2 * kt + 1][1]);
-            pa[3] = pack_bf16(s[2 * kt + 1][2], s[2 * kt + 1][3]);
+            uint32_t pa[4], pl[4];
+            split_bf16(s[2 * kt][0], s[2 * kt][1], pa[0], pl[0]);
+            split_bf16(s[2 * kt][2], s[2 * kt][3], pa[1], pl[1]);
+            split_bf16(s[2 * kt + 1][0], s[2 * kt + 1][1], pa[2], pl[2]);
+            split_bf16(s[2 * kt + 1][2], s[2 * kt + 1][3], pa[3], pl[3]);
 #pragma unroll
             for (int dp = 0; dp < D / 16; ++dp) {
                 uint32_t b0, b1, b2, b3;
@@ -258,6 +264,8 @@ attn_split_kernel(AttnArgs a, TreeMasks masks, int tiles_per_split, int n_split)
                 ldsm_x4_t(vs + swz<D>(tok, dp * 2 + (mat >> 1)), b0, b1, b2, b3);
                 mma_bf16(o[2 * dp], pa, b0, b1);
                 mma_bf16(o[2 * dp + 1], pa, b2, b3);
+                mma_bf16(o[2 * dp], pl, b0, b1);
+                mma_bf16(o[2 * dp + 1], pl, b2, b3);
             }
         }
     }
@@ -367,15 +375,18 @@ cudaError_t launch_d(const AttnArgs &a, const TreeMasks &masks, const SplitPlan 
                      cudaStream_t stream)
 {
     const int smem = Plan<D>::kSmem;
-    cudaError_t e = cudaFuncSetAttribute(attn_split_kernel<D>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-    if (e != cudaSuccess)
-        return e;
+    static const cudaError_t attr = cudaFuncSetAttribute(
+        attn_split_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (attr != cudaSuccess)
+        return attr;
     dim3 grid(p.n_split, a.n_heads_kv, p.row_blocks);
     attn_split_kernel<D><<<grid, p.warps * 32, smem, stream>>>(a, masks, p.tiles_per_split,
                                                                p.n_split);
-    e = cudaGetLastError();
-    if (e != cudaSuccess || p.n_split == 1)
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess)
+        return e;
+    count_launches(1);
+    if (p.n_split == 1)
         return e;
     const int rows_all = a.n_tree * a.n_heads_q;
     const float *ws_o = reinterpret_cast<const float *>(
@@ -383,7 +394,10 @@ cudaError_t launch_d(const AttnArgs &a, const TreeMasks &masks, const SplitPlan 
     const float *ws_ml = ws_o + (size_t)p.n_split * rows_all * D;
     attn_combine_kernel<D><<<(rows_all + 7) / 8, 256, 0, stream>>>(ws_o, ws_ml, a.out, rows_all,
                                                                    p.n_split);
-    return cudaGetLastError();
+    e = cudaGetLastError();
+    if (e == cudaSuccess)
+        count_launches(1);
+    return e;
 }
 
 }  // namespace

@@ -154,6 +154,9 @@ penalize_accept_kernel(PenalizeArgs a, TreeParents tree, int n_chunks)
                 a.argmax_out[n] = c.i;
         }
     }
+    __shared__ int tok[TS_MAX_TREE];
+    for (int i = tid; i < a.n_tree; i += kThreads)
+        tok[i] = a.tree_tokens[i];
     __syncthreads();
     if (tid == 0) {
         // valid[i]: parent valid and token == argmax at the parent
@@ -164,7 +167,7 @@ penalize_accept_kernel(PenalizeArgs a, TreeParents tree, int n_chunks)
         for (int i = 1; i < a.n_tree; ++i) {
             const int pa = tree.parent[i];
             depth[i] = depth[pa] + 1;
-            const bool ok = ((valid >> pa) & 1ull) && a.tree_tokens[i] == am[pa];
+            const bool ok = ((valid >> pa) & 1ull) && tok[i] == am[pa];
             if (ok) {
                 valid |= 1ull << i;
                 if (depth[i] > depth[best])
@@ -200,7 +203,10 @@ cudaError_t penalize_launch(const PenalizeArgs &a, const TreeParents &parents,
     const int n_chunks = (a.vocab + kChunk - 1) / kChunk;
     dim3 grid(n_chunks, a.n_tree);
     penalize_accept_kernel<<<grid, kThreads, 0, stream>>>(a, parents, n_chunks);
-    return cudaGetLastError();
+    const cudaError_t e = cudaGetLastError();
+    if (e == cudaSuccess)
+        count_launches(1);
+    return e;
 }
 
 }  // namespace ts

@@ -275,10 +275,20 @@ select_gather_kernel(SelectArgs a, int n_chunks, int slice)
             for (int b = tid; b < 256; b += kP2Threads)
                 sh.hist[b] = 0;
             __syncthreads();
-            for (int n = c0 + tid; n < p1; n += kP2Threads) {
-                const uint32_t key = keys[n - p0];
-                if ((key & pmask) == prefix)
-                    atomicAdd(&sh.hist[(key >> shift) & 255u], 1);
+            // positive scores share their leading bytes, so most lanes hit
+            // the same bin: lanes with equal bins add once, by their leader
+            for (int nb = c0 - (c0 - p0) % 32; nb < p1; nb += kP2Threads) {
+                const int n = nb + tid;
+                const bool in = n >= c0 && n < p1;
+                const uint32_t key = in ? keys[n - p0] : 0u;
+                const bool hit = in && (key & pmask) == prefix;
+                const unsigned act = __ballot_sync(0xffffffffu, hit);
+                if (hit) {
+                    const uint32_t bin = (key >> shift) & 255u;
+                    const unsigned same = __match_any_sync(act, bin);
+                    if ((lane) == __ffs(same) - 1)
+                        atomicAdd(&sh.hist[bin], __popc(same));
+                }
             }
             cluster.sync();
             // Thread t looks at bin b = 255 - t; an inclusive scan over t is
@@ -411,7 +421,10 @@ cudaError_t launch_p1(const SelectArgs &a, const SelPlan &p, cudaStream_t stream
 {
     dim3 grid(p.n_chunks, a.n_heads_kv);
     score_logits_kernel<D, GP><<<grid, kP1Threads, 0, stream>>>(a, p.chunk, p.n_chunks);
-    return cudaGetLastError();
+    const cudaError_t e = cudaGetLastError();
+    if (e == cudaSuccess)
+        count_launches(1);
+    return e;
 }
 
 template <int D>
@@ -431,10 +444,11 @@ cudaError_t launch_d(const SelectArgs &a, const SelPlan &p, cudaStream_t stream)
         return e;
 
     const size_t smem = sizeof(P2Shared) + (size_t)p.slice * sizeof(uint32_t);
-    e = cudaFuncSetAttribute(select_gather_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)smem);
-    if (e != cudaSuccess)
-        return e;
+    static const cudaError_t attr_ok = cudaFuncSetAttribute(
+        select_gather_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        (int)(sizeof(P2Shared) + (size_t)kMaxSlice * sizeof(uint32_t)));
+    if (attr_ok != cudaSuccess)
+        return attr_ok;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(kClusterCtas, a.n_heads_kv, 1);
     cfg.blockDim = dim3(kP2Threads, 1, 1);
@@ -447,7 +461,10 @@ cudaError_t launch_d(const SelectArgs &a, const SelPlan &p, cudaStream_t stream)
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, select_gather_kernel<D>, a, p.n_chunks, p.slice);
+    e = cudaLaunchKernelEx(&cfg, select_gather_kernel<D>, a, p.n_chunks, p.slice);
+    if (e == cudaSuccess)
+        count_launches(1);
+    return e;
 }
 
 }  // namespace

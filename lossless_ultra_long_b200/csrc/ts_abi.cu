@@ -4,7 +4,14 @@
 #include <math.h>
 #include <string.h>
 
+#include <atomic>
+
 #include "ts_internal.cuh"
+
+namespace ts {
+static std::atomic<unsigned long long> g_launches{0};
+void count_launches(unsigned n) { g_launches.fetch_add(n, std::memory_order_relaxed); }
+}  // namespace ts
 
 namespace {
 
@@ -65,6 +72,8 @@ const char *ts_status_string(int status)
 }
 
 int ts_version(void) { return 100; }
+
+unsigned long long ts_kernel_launch_count(void) { return ts::g_launches.load(); }
 
 size_t ts_tree_verify_attn_workspace_size(int n_heads_q, int n_heads_kv, int head_dim, int n_ctx,
                                           int n_tree)

@@ -24,6 +24,9 @@ constexpr size_t kHeaderBytes = sizeof(WorkspaceHeader);
 
 inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
+// Host-side count of kernel launches issued by the library.
+void count_launches(unsigned n);
+
 __device__ __forceinline__ void record_status(WorkspaceHeader *ws, uint32_t code)
 {
     atomicCAS(&ws->status, 0u, code);
