@@ -57,7 +57,8 @@ typedef enum {
     TS_ERR_WORKSPACE = 3,   /* workspace missing, too small or misaligned */
     TS_ERR_CUDA = 4,        /* a CUDA runtime call or launch failed */
     TS_ERR_TIMEOUT = 5,     /* device: a bounded wait expired (status word) */
-    TS_ERR_DEVICE_ARG = 6   /* device: invalid data seen on the device (status word) */
+    TS_ERR_DEVICE_ARG = 6,  /* device: invalid data seen on the device (status word) */
+    TS_ERR_SCRATCH_LIMIT = 7 /* needs more scratch than ts_tree_verify_attn_noalloc holds */
 } ts_status;
 
 /* Largest draft tree, in nodes (ancestor sets are 64-bit masks). */
@@ -105,6 +106,39 @@ TS_API int ts_tree_verify_attn(const void *q, const void *k_cache, const void *v
                         int n_heads_q, int n_heads_kv, int head_dim, int n_ctx, int n_tree,
                         const int32_t *parent, float softmax_scale, float *out,
                         void *workspace, size_t workspace_bytes, void *stream);
+
+/*
+ * ts_tree_verify_attn without a workspace argument, for callers that cannot
+ * allocate device memory (the TokenSwift pages have no counterpart; this is
+ * an interface convenience).  Some callers may not call cudaMalloc where
+ * they run attention: code whose device memory is all owned by another
+ * runtime's allocator or a fixed, pre-planned budget, or code that must not
+ * block on an allocation.  They pass inputs and outputs as for
+ * ts_tree_verify_attn; the split-KV scratch comes from a static device array
+ * of TS_NOALLOC_SCRATCH_BYTES inside the library, taken on each device that
+ * calls this entry point and held until the process exits.  Nothing is
+ * allocated and no allocating routine is called.
+ *
+ *  - Limit: a problem whose ts_tree_verify_attn_workspace_size() exceeds
+ *    TS_NOALLOC_SCRATCH_BYTES is rejected with TS_ERR_SCRATCH_LIMIT before
+ *    anything is launched (16 MiB covers, e.g., 32/8 heads, D 128, a 40-node
+ *    tree at any context length).
+ *  - Set-up: the first call on a device looks up the array's device address
+ *    (cudaGetSymbolAddress) and caches it; make that first call outside any
+ *    stream capture.
+ *  - Sharing: every call on a device uses the same array and it keeps the
+ *    last call's contents; each call clears the part that must start at
+ *    zero.  Calls whose work overlaps on the GPU (different streams, no
+ *    ordering between them) race on the array and give wrong results:
+ *    order them, or use ts_tree_verify_attn with separate workspaces.
+ *  - Errors: as ts_tree_verify_attn, plus TS_ERR_SCRATCH_LIMIT.
+ */
+#define TS_NOALLOC_SCRATCH_BYTES (16u << 20)
+TS_API int ts_tree_verify_attn_noalloc(const void *q, const void *k_cache, const void *v_cache,
+                                       int64_t kv_cap, int n_heads_q, int n_heads_kv,
+                                       int head_dim, int n_ctx, int n_tree,
+                                       const int32_t *parent, float softmax_scale, float *out,
+                                       void *stream);
 
 /*
  * Dynamic partial-KV update: importance scores, sink + top-budget selection

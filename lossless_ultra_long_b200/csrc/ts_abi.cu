@@ -67,6 +67,7 @@ const char *ts_status_string(int status)
     case TS_ERR_CUDA: return "CUDA runtime error";
     case TS_ERR_TIMEOUT: return "device wait timed out";
     case TS_ERR_DEVICE_ARG: return "invalid data seen on the device";
+    case TS_ERR_SCRATCH_LIMIT: return "problem needs more scratch than the no-alloc entry point holds";
     default: return "unknown status";
     }
 }
