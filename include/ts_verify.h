@@ -181,7 +181,7 @@ TS_API int ts_kv_importance_select(const void *q_last, const void *k_cache, cons
  *
  * Source: "TokenSwift's technical principles" (aiboss88.com): a penalty on
  * recently generated tokens; the longest valid candidate is the output;
- * tencent article 上下文惩罚 and the figure text (the longest valid sequence,
+ * tencent article 上下文惩罚 and the figure text (the longest valid candidate,
  * e.g. "is the father of", is kept).
  *
  * For every id in the window (a set), a positive logit is divided by

@@ -4,7 +4,7 @@
 // TokenSwift (aiboss88.com), "TokenSwift's technical principles": a penalty
 // on recently generated tokens; the longest valid candidate of the tree is
 // kept.  Tencent article: 上下文惩罚 and the parallel-verification figure
-// ("is the father of" is the longest valid sequence).
+// (the worked example keeps "is the father of", the longest valid candidate).
 //
 // Grid (vocab chunks, tree nodes).  Each CTA marks the window ids that fall
 // in its chunk in a shared-memory bitmap, streams its slice of the logits

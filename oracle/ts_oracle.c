@@ -347,7 +347,7 @@ int tso_penalize_argmax(const float *logits, int n_tree, int vocab, const int32_
 
 /*
  * Longest accepted path (aiboss88 "technical principles": the longest valid
- * candidate is kept; tencent figure text: the longest valid sequence, e.g.
+ * candidate is kept; tencent figure text: the longest valid candidate, e.g.
  * "is the father of", is the output).  Greedy reading: the root is valid; a
  * draft node is valid when its parent is valid and its token equals the
  * target argmax at its parent, so a valid path is exactly what ordinary
