@@ -1,0 +1,38 @@
+// attn_common.cuh -- pieces shared by the two tree-verify attention kernels
+// (tcgen05 and mma.sync) and the dispatch between them.
+#pragma once
+
+#include "ts_internal.cuh"
+
+namespace ts {
+
+struct AttnPlan {
+    int n_split;          // KV splits per head
+    int tiles_per_split;  // KV tiles each split streams
+};
+
+// The tcgen05 kernel feeds P to the PV product as one bf16 value; that is
+// exact enough (<= 1e-4 class) once attention is spread over thousands of
+// positions.  Shorter contexts, where a few weights can dominate, go to the
+// mma.sync kernel, which splits P into two bf16 parts.
+constexpr int kTcMinContext = 2048;
+
+// Split partials share one layout: acc fp32 [n_split, T*Hq, D] after the
+// workspace header, then (m, l) fp32 [n_split, T*Hq, 2]; m is in log2 units.
+inline size_t attn_partial_bytes(int n_split, int n_heads_q, int head_dim, int n_tree)
+{
+    return (size_t)n_split * n_tree * n_heads_q * (head_dim + 2) * sizeof(float);
+}
+cudaError_t attn_combine_launch(const AttnArgs &a, int n_split, cudaStream_t stream);
+
+size_t attn_mma_workspace_bytes(int n_heads_q, int n_heads_kv, int head_dim, int n_ctx,
+                                int n_tree, int num_sms);
+cudaError_t attn_mma_launch(const AttnArgs &a, const TreeMasks &masks, int num_sms,
+                            cudaStream_t stream);
+
+bool attn_tc_eligible(int n_heads_q, int n_heads_kv, int head_dim, int n_ctx, int n_tree);
+AttnPlan attn_tc_plan(int n_heads_q, int n_heads_kv, int n_ctx, int n_tree, int num_sms);
+cudaError_t attn_tc_launch(const AttnArgs &a, const TreeMasks &masks, int num_sms,
+                           cudaStream_t stream);
+
+}  // namespace ts

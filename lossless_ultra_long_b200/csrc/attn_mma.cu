@@ -20,7 +20,7 @@
 // launch normalises in place instead.
 #include <math.h>
 
-#include "ts_internal.cuh"
+#include "attn_common.cuh"
 
 namespace ts {
 namespace {
@@ -388,31 +388,38 @@ cudaError_t launch_d(const AttnArgs &a, const TreeMasks &masks, const SplitPlan 
     count_launches(1);
     if (p.n_split == 1)
         return e;
+    return attn_combine_launch(a, p.n_split, stream);
+}
+
+}  // namespace
+
+cudaError_t attn_combine_launch(const AttnArgs &a, int n_split, cudaStream_t stream)
+{
     const int rows_all = a.n_tree * a.n_heads_q;
     const float *ws_o = reinterpret_cast<const float *>(
         reinterpret_cast<const char *>(a.workspace) + kHeaderBytes);
-    const float *ws_ml = ws_o + (size_t)p.n_split * rows_all * D;
-    attn_combine_kernel<D><<<(rows_all + 7) / 8, 256, 0, stream>>>(ws_o, ws_ml, a.out, rows_all,
-                                                                   p.n_split);
-    e = cudaGetLastError();
+    const float *ws_ml = ws_o + (size_t)n_split * rows_all * a.head_dim;
+    if (a.head_dim == 128)
+        attn_combine_kernel<128><<<(rows_all + 7) / 8, 256, 0, stream>>>(ws_o, ws_ml, a.out,
+                                                                         rows_all, n_split);
+    else
+        attn_combine_kernel<64><<<(rows_all + 7) / 8, 256, 0, stream>>>(ws_o, ws_ml, a.out,
+                                                                        rows_all, n_split);
+    const cudaError_t e = cudaGetLastError();
     if (e == cudaSuccess)
         count_launches(1);
     return e;
 }
 
-}  // namespace
-
-size_t attn_workspace_bytes(int n_heads_q, int n_heads_kv, int head_dim, int n_ctx, int n_tree,
-                            int num_sms)
+size_t attn_mma_workspace_bytes(int n_heads_q, int n_heads_kv, int head_dim, int n_ctx,
+                                int n_tree, int num_sms)
 {
     const SplitPlan p = make_plan(n_heads_q, n_heads_kv, n_ctx, n_tree, num_sms);
-    const size_t rows_all = (size_t)n_tree * n_heads_q;
-    const size_t bytes = (size_t)p.n_split * rows_all * (head_dim + 2) * sizeof(float);
-    return kHeaderBytes + align_up(bytes, 256);
+    return kHeaderBytes + align_up(attn_partial_bytes(p.n_split, n_heads_q, head_dim, n_tree), 256);
 }
 
-cudaError_t attn_launch(const AttnArgs &a, const TreeMasks &masks, int num_sms,
-                        cudaStream_t stream)
+cudaError_t attn_mma_launch(const AttnArgs &a, const TreeMasks &masks, int num_sms,
+                            cudaStream_t stream)
 {
     const SplitPlan p = make_plan(a.n_heads_q, a.n_heads_kv, a.n_ctx, a.n_tree, num_sms);
     return a.head_dim == 128 ? launch_d<128>(a, masks, p, stream)

@@ -76,6 +76,16 @@ def test_attn_max_tree_and_irregular(oracle_mod):
     _attn_full(oracle_mod, w, parent=parent)
 
 
+@pytest.mark.parametrize("n_ctx", [2047, 2048, 2049, 2111, 9000])
+@pytest.mark.parametrize("hq,hkv,t", [(8, 2, 13), (32, 8, 40), (40, 8, 40), (32, 32, 40),
+                                      (64, 8, 32), (16, 1, 16), (32, 8, 4), (32, 8, 1)])
+def test_attn_dispatch_threshold_and_row_blocks(oracle_mod, n_ctx, hq, hkv, t):
+    """Both sides of the kernel switch at 2048 positions, one and two 128-row
+    blocks (up to the 256-row limit), ragged tails."""
+    w = I.Workload("tc", hq, hkv, 128, n_ctx, t, seed=n_ctx * 3 + hq + t)
+    _attn_sampled(oracle_mod, w, count=24)
+
+
 def test_attn_chain_equals_sequential_decode():
     """GPU chain verification == T GPU single-node decodes with a growing cache."""
     w = I.Workload("chain", 32, 8, 128, 5000, 8, tree="chain", seed=77)
