@@ -31,6 +31,8 @@ cudaError_t attn_mma_launch(const AttnArgs &a, const TreeMasks &masks, int num_s
                             cudaStream_t stream);
 
 bool attn_tc_eligible(int n_heads_q, int n_heads_kv, int head_dim, int n_ctx, int n_tree);
+// (the tcgen05 kernel also needs softmax_scale > 0: it takes the row max on
+// unscaled scores)
 AttnPlan attn_tc_plan(int n_heads_q, int n_heads_kv, int n_ctx, int n_tree, int num_sms);
 cudaError_t attn_tc_launch(const AttnArgs &a, const TreeMasks &masks, int num_sms,
                            cudaStream_t stream);

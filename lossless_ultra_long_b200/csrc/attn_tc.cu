@@ -5,33 +5,39 @@
 // full KV cache, each node seeing the context plus its own root path
 // (TokenSwift, aiboss88.com, "TokenSwift's technical principles"; tencent
 // article, parallel-verification figure; arxivlens "Technical
-// Contribution": a 3-ary tree).  For one KV head the G*T query rows
-// (node-major, then the group's heads) form one or two 128-row blocks that
-// every KV tile of the split serves, so K/V are streamed from HBM once.
+// Contribution": a 3-ary tree).  For one KV head the R = G*T query rows
+// (node-major, then the group's heads) share every KV tile, so K/V are
+// streamed from HBM once per split.
+//
+// The two products run in the orientations the tensor core executes at
+// full rate (an MMA instruction costs about the same below N = 128, and an
+// MN-major B operand runs at about half rate):
+//   S_b  = Q_b K^T      rows on M (128-row blocks b), N = 64 positions,
+//                       both operands K-major in shared memory;
+//   O^T += V^T P^T      head dim on M, all R rows on N (padded to 16),
+//                       V^T is the TMA tile read MN-major, P^T K-major.
+// P^T is written to shared memory by the softmax threads, one row each.
 //
 // CTA = (split, KV head), 12 warps, one CTA per SM:
-//   warp 0      TMA producer: K and V tiles of 64 positions (two 64-column
-//               boxes each, 128-byte swizzle) into a ring of stages.  The
+//   warps 0, 2  TMA producers for K and for V: 64-position tiles (two
+//               64-column boxes each, 128-byte swizzle) into two rings.  The
 //               tensor map's row extent is n_ctx + T, so rows past the tree
 //               tail arrive as zeros.
-//   warp 1      allocates TMEM; one lane issues every tcgen05.mma:
-//                 S_b(t)  = Q_b K(t)^T   (M 128, N 64,  K 128; smem x smem)
-//                 O_b    += P_b(t) V(t)  (M 128, N 128, K 64;  tmem x smem)
-//               S is double-buffered so QK of tile t+1 overlaps the
-//               softmax of tile t.
-//   warps 4-11  softmax, one thread per query row (TMEM lane): loads S,
-//               scales to base 2, applies the ancestor mask on tiles that
-//               reach the tree tail, exponentiates against a per-row
-//               reference max and writes P as bf16 back over S for the PV
-//               product.  The reference only moves (rescaling O and l in
-//               place) when a tile's max exceeds it by more than 2^8, so
-//               the common tile needs no O traffic; l sums the bf16-rounded
-//               P so the normalisation matches what PV used.
-// TMEM columns: O_b at [128 b, 128 b + 128); S_b(buf) at 128 NB + 64 (2b + buf).
+//   warp 1      allocates TMEM; one lane issues every tcgen05.mma.  S is
+//               double-buffered so QK of tile t+1 overlaps the softmax of t.
+//   warps 4..   softmax, one thread per query row (TMEM lane of its block):
+//               scale to base 2, ancestor mask on tiles that reach the tree
+//               tail, exponentiate against a per-row reference max, write
+//               the bf16 P^T row.  The reference only moves when a tile's
+//               max exceeds it by more than 2^8; then warps 4-7 (which
+//               between them see all 128 TMEM lanes, i.e. all of D) rescale
+//               the affected O^T columns before the next PV.  l sums the
+//               bf16-rounded P so the normalisation matches what PV used.
+// TMEM: O^T in columns [0, R_pad); S_b(buf) at kSCol0 + 64 (2b + buf).
 // Each split leaves an unnormalised partial (acc, m, l) for the combine
 // kernel, or normalises in place when it is the only split.
 //
-// Every wait on an mbarrier is bounded (about a second): on expiry the
+// Every wait is on an mbarrier and bounded (about a second): on expiry the
 // kernel records TS_ERR_TIMEOUT in the workspace status word, all roles
 // leave their loops, and TMEM is freed before the CTA exits.
 #include <cuda.h>
@@ -50,44 +56,103 @@ using namespace sm100;
 
 constexpr int kD = 128;
 constexpr int kTileN = 64;                      // KV positions per tile
-constexpr int kBlockM = 128;                    // query rows per MMA block
+constexpr int kBlockM = 128;                    // query rows per QK block
 constexpr int kBoxBytes = kTileN * 64 * 2;      // one 64-column box of a tile: 8 KB
-constexpr int kStageBytes = 4 * kBoxBytes;      // K lo, K hi, V lo, V hi
+constexpr int kHalfStageBytes = 2 * kBoxBytes;  // K (or V) of a tile: lo and hi boxes
 constexpr int kQBlockBytes = kBlockM * kD * 2;  // 32 KB
 constexpr int kThreads = 384;
 constexpr int kFirstSoftmaxWarp = 4;
-
-template <int NB>
-struct TcCfg {
-    static constexpr int kStages = NB == 2 ? 4 : 5;
-    static constexpr int kTmemCols = NB == 2 ? 512 : 256;
-    static constexpr int kSCol0 = 128 * NB;
-    static constexpr size_t kSmemBytes =
-        1024 + (size_t)NB * kQBlockBytes + (size_t)kStages * kStageBytes + 256;
-};
+constexpr int kMaxStages = 8;
+constexpr int kMaxRows = 256;
+constexpr size_t kSmemLimit = 232448;           // dynamic shared memory per CTA
 
 struct TcBarriers {
-    uint64_t full[5];
-    uint64_t empty[5];
-    uint64_t s_full[2][2];
-    uint64_t p_full[2][2];
-    uint64_t o_done[2];
-    uint64_t o_final[2];
+    uint64_t full_k[kMaxStages];
+    uint64_t empty_k[kMaxStages];
+    uint64_t full_v[kMaxStages];
+    uint64_t empty_v[kMaxStages];
+    uint64_t s_full[2][2];     // QK of a block landed in S(buf)
+    uint64_t sm_sync[2];       // every softmax warp finished a tile
+    uint64_t p_full[2];        // P^T(buf) written and O^T corrected
+    uint64_t o_done;           // one commit per PV
+    uint64_t o_final;          // committed once, after the last PV
     uint64_t drain;
     uint32_t tmem_base;
     uint32_t abort;
+    int32_t rescale_tile[2];   // tile index + 1 when that tile moved a row's max
 };
-static_assert(sizeof(TcBarriers) <= 256, "barrier block");
 
-constexpr uint32_t kIdescQK = idesc_bf16(kBlockM, kTileN, 0, 0);
-constexpr uint32_t kIdescPV = idesc_bf16(kBlockM, kD, 0, 1);
+struct TcAux {
+    float factor[2][kMaxRows];  // per-row O^T rescale factor of the tile
+    float l[kMaxRows];
+    float m[kMaxRows];
+    TcBarriers bar;
+};
+constexpr size_t kAuxBytes = (sizeof(TcAux) + 1023) / 1024 * 1024;
 
-__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi, float &sum)
+struct TcLayout {
+    int r_pad;       // rows rounded up to 16: N of the PV product
+    int stages_k, stages_v;
+    size_t p_off, k_off, v_off, aux_off, smem_bytes;
+};
+
+__host__ __device__ inline TcLayout tc_layout(int nb, int rows)
 {
-    __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
-    const float2 back = __bfloat1622float2(h);
-    sum += back.x + back.y;
-    return *reinterpret_cast<uint32_t *>(&h);
+    TcLayout L;
+    L.r_pad = (rows + 15) / 16 * 16;
+    L.p_off = (size_t)nb * kQBlockBytes;
+    L.k_off = L.p_off + 2 * (size_t)L.r_pad * 128;
+    const size_t fixed = 1024 + L.k_off + kAuxBytes;
+    int halves = (int)((kSmemLimit - fixed) / kHalfStageBytes);
+    halves = halves > 2 * kMaxStages ? 2 * kMaxStages : halves;
+    // V is consumed one softmax later than K, but both need a tile or two of
+    // look-ahead beyond the one in use
+    L.stages_v = halves * 3 / 7 < 2 ? 2 : halves * 3 / 7;
+    L.stages_k = halves - L.stages_v;
+    L.stages_k = L.stages_k > kMaxStages ? kMaxStages : L.stages_k;
+    L.v_off = L.k_off + (size_t)L.stages_k * kHalfStageBytes;
+    L.aux_off = L.v_off + (size_t)L.stages_v * kHalfStageBytes;
+    L.smem_bytes = 1024 + L.aux_off + kAuxBytes;
+    return L;
+}
+
+// P = 2^(x * scale - m) for the 64 scores of one row, packed to bf16 pairs;
+// returns the sum of the rounded values (what the PV product will use).
+// POLY: one pair in four goes through the FMA-pipe polynomial instead of
+// MUFU ex2 (masked tiles, whose -inf scores the polynomial clamps instead of
+// zeroing, use MUFU only).
+template <bool POLY>
+__device__ __forceinline__ float exp_pack_tile(const float (&x)[64], float scale, float neg_m,
+                                               uint32_t (&pk)[32])
+{
+    const uint64_t sc2 = pack2(scale, scale);
+    const uint64_t nm2 = pack2(neg_m, neg_m);
+    uint64_t y[32];
+#pragma unroll
+    for (int j = 0; j < 32; ++j)
+        y[j] = fma2(pack2(x[2 * j], x[2 * j + 1]), sc2, nm2);
+    uint64_t ls2[4] = {0ull, 0ull, 0ull, 0ull};
+#pragma unroll
+    for (int j = 0; j < 32; ++j) {
+        float e0, e1;
+        if (POLY && (j & 3) == 3) {
+            unpack2(exp2_poly2(y[j]), e0, e1);
+        } else {
+            float y0, y1;
+            unpack2(y[j], y0, y1);
+            e0 = ex2(y0);
+            e1 = ex2(y1);
+        }
+        __nv_bfloat162 h = __floats2bfloat162_rn(e0, e1);
+        const uint32_t hb = *reinterpret_cast<uint32_t *>(&h);
+        pk[j] = hb;
+        ls2[j & 3] = add2(ls2[j & 3],
+                          pack2(__uint_as_float(hb << 16), __uint_as_float(hb & 0xFFFF0000u)));
+    }
+    const uint64_t s01 = add2(add2(ls2[0], ls2[1]), add2(ls2[2], ls2[3]));
+    float a0, a1;
+    unpack2(s01, a0, a1);
+    return a0 + a1;
 }
 
 template <int NB>
@@ -95,53 +160,64 @@ __global__ void __launch_bounds__(kThreads, 1)
 attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_constant__ CUtensorMap tmap_v,
                AttnArgs a, TreeMasks masks, int tiles_per_split, int n_split)
 {
-    using Cfg = TcCfg<NB>;
-    constexpr int S = Cfg::kStages;
+    constexpr int kSCol0 = NB == 2 ? 256 : 128;
+    constexpr int kTmemCols = NB == 2 ? 512 : 256;
+    constexpr int kSoftmaxWarps = 4 * NB;
+
+    const int G = a.n_heads_q / a.n_heads_kv;
+    const int R = G * a.n_tree;
+    const TcLayout lay = tc_layout(NB, R);
+    const int SK = lay.stages_k, SV = lay.stages_v, r_pad = lay.r_pad;
+
     extern __shared__ unsigned char smem_raw[];
     unsigned char *base = reinterpret_cast<unsigned char *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     unsigned char *sQ = base;
-    unsigned char *sKV = base + NB * kQBlockBytes;
-    TcBarriers *bar = reinterpret_cast<TcBarriers *>(sKV + S * kStageBytes);
+    unsigned char *sP = base + lay.p_off;
+    unsigned char *sK = base + lay.k_off;
+    unsigned char *sV = base + lay.v_off;
+    TcAux *aux = reinterpret_cast<TcAux *>(base + lay.aux_off);
+    TcBarriers *bar = &aux->bar;
     WorkspaceHeader *hdr = reinterpret_cast<WorkspaceHeader *>(a.workspace);
     volatile uint32_t *abort = &bar->abort;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int split = blockIdx.x, g = blockIdx.y;
-    const int G = a.n_heads_q / a.n_heads_kv;
-    const int R = G * a.n_tree;
     const int total = a.n_ctx + a.n_tree;
     const int n_tiles_all = (total + kTileN - 1) / kTileN;
     const int t_begin = split * tiles_per_split;
     const int n_tiles = min(t_begin + tiles_per_split, n_tiles_all) - t_begin;
 
-    // softmax warps with at least one real row, per block
-    int active_warps[2];
-#pragma unroll
-    for (int b = 0; b < 2; ++b) {
-        const int rows = min(max(R - b * kBlockM, 0), kBlockM);
-        active_warps[b] = (rows + 31) / 32;
-    }
+    // softmax warps that take part in the per-tile sync: those with rows,
+    // and warps 4-7, which rescale and write out O^T
+    int sync_warps = 0;
+    for (int w = 0; w < kSoftmaxWarps; ++w)
+        sync_warps += (w < 4) || ((w / 4) * kBlockM + (w % 4) * 32 < R);
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < S; ++s) {
-            mbar_init(smem_addr(&bar->full[s]), 1);
-            mbar_init(smem_addr(&bar->empty[s]), 1);
+        for (int s = 0; s < SK; ++s) {
+            mbar_init(smem_addr(&bar->full_k[s]), 1);
+            mbar_init(smem_addr(&bar->empty_k[s]), 1);
         }
-        for (int b = 0; b < NB; ++b) {
-            for (int u = 0; u < 2; ++u) {
+        for (int s = 0; s < SV; ++s) {
+            mbar_init(smem_addr(&bar->full_v[s]), 1);
+            mbar_init(smem_addr(&bar->empty_v[s]), 1);
+        }
+        for (int u = 0; u < 2; ++u) {
+            for (int b = 0; b < NB; ++b)
                 mbar_init(smem_addr(&bar->s_full[b][u]), 1);
-                mbar_init(smem_addr(&bar->p_full[b][u]), active_warps[b]);
-            }
-            mbar_init(smem_addr(&bar->o_done[b]), 1);
-            mbar_init(smem_addr(&bar->o_final[b]), 1);
+            mbar_init(smem_addr(&bar->sm_sync[u]), sync_warps);
+            mbar_init(smem_addr(&bar->p_full[u]), 4);
+            bar->rescale_tile[u] = 0;
         }
+        mbar_init(smem_addr(&bar->o_done), 1);
+        mbar_init(smem_addr(&bar->o_final), 1);
         mbar_init(smem_addr(&bar->drain), 1);
         bar->abort = 0u;
         fence_mbar_init();
     }
     if (warp == 1) {
-        tmem_alloc(smem_addr(&bar->tmem_base), Cfg::kTmemCols);
+        tmem_alloc(smem_addr(&bar->tmem_base), kTmemCols);
         tmem_relinquish();
     }
     if (warp == 0 && lane == 0) {
@@ -170,210 +246,262 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_constant
     tc_fence_after();
     const uint32_t tmem = bar->tmem_base;
 
-    if (warp == 0) {
-        // ------------------------------------------------------ TMA producer
+    if (warp == 0 || warp == 2) {
+        // ----------------------------------------- TMA producers (K, V)
         if (lane == 0) {
+            const bool is_k = warp == 0;
+            const int ns = is_k ? SK : SV;
+            uint64_t *full = is_k ? bar->full_k : bar->full_v;
+            uint64_t *empty = is_k ? bar->empty_k : bar->empty_v;
+            unsigned char *ring = is_k ? sK : sV;
+            const void *tmap = is_k ? static_cast<const void *>(&tmap_k)
+                                    : static_cast<const void *>(&tmap_v);
             int issued = 0;
             for (int t = 0; t < n_tiles; ++t) {
-                const int s = t % S;
-                if (t >= S &&
-                    !wait_bounded(smem_addr(&bar->empty[s]), ((t / S) & 1) ^ 1, abort, hdr))
+                const int s = t % ns;
+                if (t >= ns &&
+                    !wait_bounded(smem_addr(&empty[s]), ((t / ns) & 1) ^ 1, abort, hdr))
                     break;
-                const uint32_t fb = smem_addr(&bar->full[s]);
-                mbar_arrive_expect_tx(fb, kStageBytes);
-                const uint32_t dst = smem_addr(sKV + s * kStageBytes);
+                const uint32_t fb = smem_addr(&full[s]);
+                mbar_arrive_expect_tx(fb, kHalfStageBytes);
+                const uint32_t dst = smem_addr(ring + s * kHalfStageBytes);
                 const int pos0 = (t_begin + t) * kTileN;
-                tma_load_3d(dst, &tmap_k, 0, pos0, g, fb);
-                tma_load_3d(dst + kBoxBytes, &tmap_k, 64, pos0, g, fb);
-                tma_load_3d(dst + 2 * kBoxBytes, &tmap_v, 0, pos0, g, fb);
-                tma_load_3d(dst + 3 * kBoxBytes, &tmap_v, 64, pos0, g, fb);
+                tma_load_3d(dst, tmap, 0, pos0, g, fb);
+                tma_load_3d(dst + kBoxBytes, tmap, 64, pos0, g, fb);
                 issued = t + 1;
             }
             if (*abort) {
                 // let our own copies land before the CTA exits
-                for (int t = max(0, issued - S); t < issued; ++t)
-                    wait_drain(smem_addr(&bar->full[t % S]), (t / S) & 1);
+                for (int t = max(0, issued - ns); t < issued; ++t)
+                    wait_drain(smem_addr(&full[t % ns]), (t / ns) & 1);
             }
         }
     } else if (warp == 1) {
         // ------------------------------------------------------- MMA issuer
         if (lane == 0) {
-            const uint32_t q_base = smem_addr(sQ);
+            constexpr uint32_t idesc_qk = idesc_bf16(kBlockM, kTileN, 0, 0);
+            const uint32_t idesc_pv = idesc_bf16(kD, r_pad, 1, 0);
+            // Descriptors are built once; per MMA only the start-address
+            // field moves (address / 16 in the low bits, no carry out of it
+            // inside shared memory).
+            uint64_t qd[NB][8];
+#pragma unroll
+            for (int b = 0; b < NB; ++b)
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk)
+                    qd[b][kk] = sdesc_sw128(smem_addr(sQ) + b * kQBlockBytes +
+                                                (kk >> 2) * (kBlockM * 128) + (kk & 3) * 32,
+                                            16, 1024);
+            const uint64_t kd0 = sdesc_sw128(smem_addr(sK), 16, 1024);
+            const uint64_t vd0 = sdesc_sw128(smem_addr(sV), kBoxBytes, 1024);
+            const uint64_t pd0 = sdesc_sw128(smem_addr(sP), 16, 1024);
+            constexpr uint64_t kStageStep = kHalfStageBytes >> 4;
             bool ok = true;
             for (int t = 0; t <= n_tiles && ok; ++t) {
                 if (t < n_tiles) {
-                    const int s = t % S;
-                    if (!wait_bounded(smem_addr(&bar->full[s]), (t / S) & 1, abort, hdr)) {
+                    const int s = t % SK;
+                    if (!wait_bounded(smem_addr(&bar->full_k[s]), (t / SK) & 1, abort, hdr)) {
                         ok = false;
                         break;
                     }
                     tc_fence_after();
-                    const uint32_t k_base = smem_addr(sKV + s * kStageBytes);
+                    const uint64_t kd = kd0 + (uint64_t)s * kStageStep;
 #pragma unroll
                     for (int b = 0; b < NB; ++b) {
-                        const uint32_t d_col = tmem + Cfg::kSCol0 + 64 * (2 * b + (t & 1));
+                        const uint32_t d_col = tmem + kSCol0 + 64 * (2 * b + (t & 1));
+                        mma_ss_c<0>(d_col, qd[b][0], kd, idesc_qk);
 #pragma unroll
-                        for (int kk = 0; kk < kD / 16; ++kk) {
-                            const uint32_t koff = (kk >> 2) * kBoxBytes + (kk & 3) * 32;
-                            const uint32_t qoff = b * kQBlockBytes + (kk >> 2) * (kBlockM * 128) +
-                                                  (kk & 3) * 32;
-                            mma_ss(d_col, sdesc_sw128(q_base + qoff, 16, 1024),
-                                   sdesc_sw128(k_base + koff, 16, 1024), kIdescQK, kk > 0);
-                        }
+                        for (int kk = 1; kk < kD / 16; ++kk)
+                            mma_ss_c<1>(d_col, qd[b][kk],
+                                        kd + (((kk >> 2) * kBoxBytes + (kk & 3) * 32) >> 4),
+                                        idesc_qk);
                         mma_commit(smem_addr(&bar->s_full[b][t & 1]));
                     }
+                    mma_commit(smem_addr(&bar->empty_k[s]));
                 }
                 if (t >= 1) {
-                    const int u = t - 1, s = u % S;
-                    const uint32_t v_base = smem_addr(sKV + s * kStageBytes + 2 * kBoxBytes);
-#pragma unroll
-                    for (int b = 0; b < NB; ++b) {
-                        if (!wait_bounded(smem_addr(&bar->p_full[b][u & 1]), (u >> 1) & 1, abort,
-                                          hdr)) {
-                            ok = false;
-                            break;
-                        }
-                        tc_fence_after();
-                        const uint32_t o_col = tmem + 128 * b;
-                        const uint32_t p_col = tmem + Cfg::kSCol0 + 64 * (2 * b + (u & 1));
-#pragma unroll
-                        for (int kk = 0; kk < kTileN / 16; ++kk)
-                            mma_ts(o_col, p_col + kk * 8,
-                                   sdesc_sw128(v_base + kk * 2048, kBoxBytes, 1024), kIdescPV,
-                                   (u > 0 || kk > 0) ? 1u : 0u);
-                        mma_commit(smem_addr(&bar->o_done[b]));
-                        if (u == n_tiles - 1)
-                            mma_commit(smem_addr(&bar->o_final[b]));
+                    const int u = t - 1, s = u % SV;
+                    if (!wait_bounded(smem_addr(&bar->full_v[s]), (u / SV) & 1, abort, hdr) ||
+                        !wait_bounded(smem_addr(&bar->p_full[u & 1]), (u >> 1) & 1, abort, hdr)) {
+                        ok = false;
+                        break;
                     }
-                    if (ok)
-                        mma_commit(smem_addr(&bar->empty[s]));
+                    tc_fence_after();
+                    const uint64_t vd = vd0 + (uint64_t)s * kStageStep;
+                    const uint64_t pd = pd0 + (uint64_t)((u & 1) * r_pad * 128 >> 4);
+                    if (u == 0)
+                        mma_ss_c<0>(tmem, vd, pd, idesc_pv);
+                    else
+                        mma_ss_c<1>(tmem, vd, pd, idesc_pv);
+#pragma unroll
+                    for (int kk = 1; kk < kTileN / 16; ++kk)
+                        mma_ss_c<1>(tmem, vd + kk * (2048 >> 4), pd + kk * (32 >> 4), idesc_pv);
+                    mma_commit(smem_addr(&bar->o_done));
+                    if (u == n_tiles - 1)
+                        mma_commit(smem_addr(&bar->o_final));
+                    mma_commit(smem_addr(&bar->empty_v[s]));
                 }
             }
             // every MMA issued above has finished before TMEM is released
             mma_commit(smem_addr(&bar->drain));
             wait_drain(smem_addr(&bar->drain), 0);
         }
-    } else if (warp >= kFirstSoftmaxWarp) {
+    } else if (warp >= kFirstSoftmaxWarp && warp < kFirstSoftmaxWarp + kSoftmaxWarps &&
+               ((warp - kFirstSoftmaxWarp) < 4 ||
+                (warp - kFirstSoftmaxWarp) / 4 * kBlockM + (warp & 3) * 32 < R)) {
         // ---------------------------------------------------------- softmax
         const int b = (warp - kFirstSoftmaxWarp) / 4;
         const int quarter = warp & 3;
-        if (b < NB && quarter < active_warps[b]) {
-            const int lane_row = quarter * 32 + lane;
-            const int r = b * kBlockM + lane_row;
-            const bool valid = r < R;
-            const int rr = valid ? r : 0;
-            const int node = rr / G, h = g * G + rr % G;
-            const unsigned long long anc = masks.anc[node];
-            const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
-            const uint32_t o_addr = tmem + lane_off + 128 * b;
-            float m_ref = -INFINITY, l = 0.f;
-            bool ok = true;
-            for (int t = 0; t < n_tiles; ++t) {
-                const int buf = t & 1;
+        const bool corrector = b == 0;   // warps 4-7: all 128 lanes between them
+        const bool active = b * kBlockM + quarter * 32 < R;
+        const int r = b * kBlockM + quarter * 32 + lane;
+        const int rr = r < R ? r : 0;
+        const int node = rr / G;
+        const unsigned long long anc = masks.anc[node];
+        const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
+        float m_ref = -INFINITY, l = 0.f;
+        bool ok = true;
+        for (int t = 0; t < n_tiles; ++t) {
+            const int buf = t & 1;
+            if (active) {
                 if (!warp_wait_bounded(smem_addr(&bar->s_full[b][buf]), (t >> 1) & 1, abort,
                                        hdr)) {
                     ok = false;
                     break;
                 }
                 tc_fence_after();
-                const uint32_t s_addr = tmem + lane_off + Cfg::kSCol0 + 64 * (2 * b + buf);
-                uint32_t raw[2][32];
-                tmem_ld32(s_addr, raw[0]);
-                tmem_ld32(s_addr + 32, raw[1]);
+                uint32_t raw[64];
+                tmem_ld64(tmem + lane_off + kSCol0 + 64 * (2 * b + buf), raw);
+                // raw scores; the scale (> 0) is applied inside the exponent
                 float x[64];
-                float mx = -INFINITY;
                 const int pos0 = (t_begin + t) * kTileN;
-                if (pos0 + kTileN <= a.n_ctx) {
+                const bool edge = pos0 + kTileN > a.n_ctx;
+                if (!edge) {
 #pragma unroll
-                    for (int j = 0; j < 64; ++j) {
-                        x[j] = __uint_as_float(raw[j >> 5][j & 31]) * a.scale_log2;
-                        mx = fmaxf(mx, x[j]);
-                    }
+                    for (int j = 0; j < 64; ++j)
+                        x[j] = __uint_as_float(raw[j]);
                 } else {
 #pragma unroll
                     for (int j = 0; j < 64; ++j) {
                         const int pos = pos0 + j;
-                        float v = __uint_as_float(raw[j >> 5][j & 31]) * a.scale_log2;
-                        if (pos >= total)
-                            v = -INFINITY;
-                        else if (pos >= a.n_ctx && !((anc >> (pos - a.n_ctx)) & 1ull))
-                            v = -INFINITY;
-                        x[j] = v;
-                        mx = fmaxf(mx, v);
+                        const bool seen = pos < total &&
+                                          (pos < a.n_ctx || ((anc >> (pos - a.n_ctx)) & 1ull));
+                        x[j] = seen ? __uint_as_float(raw[j]) : -INFINITY;
                     }
                 }
+                float pm[8];
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    pm[e] = max3f(x[e], x[e + 8], x[e + 16]);
+                    pm[e] = max3f(pm[e], x[e + 24], x[e + 32]);
+                    pm[e] = max3f(pm[e], x[e + 40], x[e + 48]);
+                    pm[e] = fmaxf(pm[e], x[e + 56]);
+                }
+                const float mx = max3f(max3f(pm[0], pm[1], pm[2]), max3f(pm[3], pm[4], pm[5]),
+                                       fmaxf(pm[6], pm[7])) *
+                                 a.scale_log2;
                 // move the reference max only when this tile exceeds it by > 2^8
+                float f = 1.f;
                 const bool need = mx > m_ref + 8.0f;
-                if (__any_sync(0xffffffffu, need)) {
-                    const float m_new = need ? mx : m_ref;
-                    const float f = (m_ref == -INFINITY) ? 0.f : exp2f(m_ref - m_new);
+                if (need) {
+                    f = (m_ref == -INFINITY) ? 0.f : ex2(m_ref - mx);
+                    m_ref = mx;
                     l *= f;
-                    if (t > 0) {
-                        // S(t) is committed after PV(t-2) was issued, so
-                        // o_done has completed t-1 or t phases here: parity
-                        // (t-1) tells them apart
-                        if (!warp_wait_bounded(smem_addr(&bar->o_done[b]), (t - 1) & 1, abort,
-                                               hdr)) {
-                            ok = false;
-                            break;
-                        }
-                        tc_fence_after();
-#pragma unroll
-                        for (int c = 0; c < 4; ++c) {
-                            uint32_t o[32];
-                            tmem_ld32(o_addr + 32 * c, o);
-#pragma unroll
-                            for (int j = 0; j < 32; ++j)
-                                o[j] = __float_as_uint(__uint_as_float(o[j]) * f);
-                            tmem_st32(o_addr + 32 * c, o);
-                        }
-                        tmem_st_wait();
-                    }
-                    m_ref = m_new;
                 }
-                const float m_use = m_ref == -INFINITY ? 0.f : m_ref;
+                aux->factor[buf][r] = f;
+                if (__any_sync(0xffffffffu, need) && lane == 0)
+                    bar->rescale_tile[buf] = t + 1;
+                const float neg_m = m_ref == -INFINITY ? 0.f : -m_ref;
                 uint32_t pk[32];
+                // the choice of exponent paths is hoisted out of the unrolled
+                // loop so that each version is straight-line code
+                if (edge)
+                    l += exp_pack_tile<false>(x, a.scale_log2, neg_m, pk);
+                else
+                    l += exp_pack_tile<true>(x, a.scale_log2, neg_m, pk);
+                // P^T row r: 64 bf16 = one 128-byte swizzled row of the K-major tile
+                unsigned char *prow = sP + buf * r_pad * 128 + (r >> 3) * 1024 + (r & 7) * 128;
+                if (r < r_pad) {
 #pragma unroll
-                for (int j = 0; j < 32; ++j)
-                    pk[j] = pack_bf16x2(exp2f(x[2 * j] - m_use), exp2f(x[2 * j + 1] - m_use), l);
-                tmem_st32(s_addr, pk);
-                tmem_st_wait();
+                    for (int c = 0; c < 8; ++c)
+                        *reinterpret_cast<uint4 *>(prow + ((c ^ (r & 7)) << 4)) =
+                            make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
+                }
+                fence_proxy_async_smem();
+            }
+            __syncwarp();
+            if (lane == 0)
+                mbar_arrive(smem_addr(&bar->sm_sync[buf]));
+            if (corrector) {
+                if (!warp_wait_bounded(smem_addr(&bar->sm_sync[buf]), (t >> 1) & 1, abort, hdr)) {
+                    ok = false;
+                    break;
+                }
+                if (t > 0 && bar->rescale_tile[buf] == t + 1) {
+                    // S(t) was committed after PV(t-2) was issued, so o_done has
+                    // completed t-1 or t phases: parity (t-1) tells them apart
+                    if (!warp_wait_bounded(smem_addr(&bar->o_done), (t - 1) & 1, abort, hdr)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    for (int c = 0; c < r_pad; c += 32) {
+                        uint32_t o[32];
+                        tmem_ld32(tmem + lane_off + c, o);
+#pragma unroll
+                        for (int j = 0; j < 32; ++j)
+                            o[j] = __float_as_uint(__uint_as_float(o[j]) *
+                                                   aux->factor[buf][c + j]);
+                        tmem_st32(tmem + lane_off + c, o);
+                    }
+                    tmem_st_wait();
+                }
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0)
-                    mbar_arrive(smem_addr(&bar->p_full[b][buf]));
+                    mbar_arrive(smem_addr(&bar->p_full[buf]));
             }
-            // o_done alone cannot say whether the last PV has landed: when the
-            // softmax finishes its last tile, PV(n-2) may still be queued
-            // (QK of a tile is issued before PV of the previous one), and a
-            // parity wait cannot tell n-2 completions from n.  o_final is
-            // committed once, after the last PV of this block.
-            if (ok && n_tiles > 0 &&
-                warp_wait_bounded(smem_addr(&bar->o_final[b]), 0, abort, hdr)) {
-                tc_fence_after();
-                const int rows_all = a.n_tree * a.n_heads_q;
-                const int orow = node * a.n_heads_q + h;
-                float *ws_o = reinterpret_cast<float *>(reinterpret_cast<char *>(a.workspace) +
-                                                        kHeaderBytes);
-                float *ws_ml = ws_o + (size_t)n_split * rows_all * kD;
-                const float inv = (n_split == 1 && l > 0.f) ? 1.f / l : 1.f;
-                float *dst = n_split == 1 ? a.out + (size_t)orow * kD
-                                          : ws_o + ((size_t)split * rows_all + orow) * kD;
-#pragma unroll
-                for (int c = 0; c < 4; ++c) {
-                    uint32_t o[32];
-                    tmem_ld32(o_addr + 32 * c, o);
-                    if (valid) {
-#pragma unroll
-                        for (int j = 0; j < 32; j += 4)
-                            *reinterpret_cast<float4 *>(dst + 32 * c + j) = make_float4(
-                                __uint_as_float(o[j]) * inv, __uint_as_float(o[j + 1]) * inv,
-                                __uint_as_float(o[j + 2]) * inv, __uint_as_float(o[j + 3]) * inv);
-                    }
-                }
-                if (valid && n_split > 1)
+        }
+
+        // ---- epilogue: row owners publish (m, l); warps 4-7 write O^T out
+        if (ok) {
+            const int rows_all = a.n_tree * a.n_heads_q;
+            float *ws_o =
+                reinterpret_cast<float *>(reinterpret_cast<char *>(a.workspace) + kHeaderBytes);
+            float *ws_ml = ws_o + (size_t)n_split * rows_all * kD;
+            if (active && r < R) {
+                aux->l[r] = l;
+                if (n_split > 1) {
+                    const int orow = node * a.n_heads_q + g * G + r % G;
                     *reinterpret_cast<float2 *>(ws_ml + ((size_t)split * rows_all + orow) * 2) =
                         make_float2(m_ref, l);
+                }
+            }
+            __syncwarp();
+            if (lane == 0)
+                mbar_arrive(smem_addr(&bar->sm_sync[n_tiles & 1]));
+            if (corrector &&
+                warp_wait_bounded(smem_addr(&bar->sm_sync[n_tiles & 1]), (n_tiles >> 1) & 1,
+                                  abort, hdr) &&
+                warp_wait_bounded(smem_addr(&bar->o_final), 0, abort, hdr)) {
+                tc_fence_after();
+                const int d = quarter * 32 + lane;
+                for (int c = 0; c < r_pad; c += 32) {
+                    uint32_t o[32];
+                    tmem_ld32(tmem + lane_off + c, o);
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) {
+                        const int rw = c + j;
+                        if (rw < R) {
+                            const int orow = (rw / G) * a.n_heads_q + g * G + rw % G;
+                            const float v = __uint_as_float(o[j]);
+                            if (n_split == 1)
+                                a.out[(size_t)orow * kD + d] = v / aux->l[rw];
+                            else
+                                ws_o[((size_t)split * rows_all + orow) * kD + d] = v;
+                        }
+                    }
+                }
             }
         }
     }
@@ -382,7 +510,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_constant
     __syncthreads();
     if (warp == 1) {
         tc_fence_after();
-        tmem_dealloc(tmem, Cfg::kTmemCols);
+        tmem_dealloc(tmem, kTmemCols);
     }
 }
 
@@ -430,9 +558,10 @@ cudaError_t launch_nb(const AttnArgs &a, const TreeMasks &masks, const AttnPlan 
     if (!encode_kv_map(&mk, a.k, rows, a.kv_cap, a.n_heads_kv) ||
         !encode_kv_map(&mv, a.v, rows, a.kv_cap, a.n_heads_kv))
         return cudaErrorInvalidValue;
-    const size_t smem = TcCfg<NB>::kSmemBytes;
+    const TcLayout lay = tc_layout(NB, (a.n_heads_q / a.n_heads_kv) * a.n_tree);
+    const size_t smem = lay.smem_bytes;
     static const cudaError_t attr = cudaFuncSetAttribute(
-        attn_tc_kernel<NB>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        attn_tc_kernel<NB>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemLimit);
     if (attr != cudaSuccess)
         return attr;
     attn_tc_kernel<NB><<<dim3(p.n_split, a.n_heads_kv), kThreads, smem, stream>>>(
@@ -451,7 +580,7 @@ cudaError_t launch_nb(const AttnArgs &a, const TreeMasks &masks, const AttnPlan 
 bool attn_tc_eligible(int n_heads_q, int n_heads_kv, int head_dim, int n_ctx, int n_tree)
 {
     const int rows = (n_heads_q / n_heads_kv) * n_tree;
-    return head_dim == kD && rows <= 2 * kBlockM && n_ctx >= kTcMinContext;
+    return head_dim == kD && rows <= kMaxRows && n_ctx >= kTcMinContext;
 }
 
 AttnPlan attn_tc_plan(int n_heads_q, int n_heads_kv, int n_ctx, int n_tree, int num_sms)
