@@ -317,28 +317,45 @@ attn_combine_kernel(const float *__restrict__ ws_o, const float *__restrict__ ws
         return;
     float M = -INFINITY;
     for (int s = 0; s < n_split; ++s)
-        M = fmaxf(M, ws_ml[((size_t)s * rows_all + row) * 2]);
+        M = fmaxf(M, __ldcg(ws_ml + ((size_t)s * rows_all + row) * 2));
     constexpr int PER = D / 32;
     float acc[PER];
 #pragma unroll
     for (int e = 0; e < PER; ++e)
         acc[e] = 0.f;
     float L = 0.f;
-    for (int s = 0; s < n_split; ++s) {
-        const float2 ml = *reinterpret_cast<const float2 *>(ws_ml + ((size_t)s * rows_all + row) * 2);
-        const float w = ml.x == -INFINITY ? 0.f : exp2f(ml.x - M);
-        L += w * ml.y;
-        const float *src = ws_o + ((size_t)s * rows_all + row) * D + lane * PER;
-        if constexpr (PER == 4) {
-            const float4 x = *reinterpret_cast<const float4 *>(src);
-            acc[0] += w * x.x;
-            acc[1] += w * x.y;
-            acc[2] += w * x.z;
-            acc[3] += w * x.w;
-        } else {
-            const float2 x = *reinterpret_cast<const float2 *>(src);
-            acc[0] += w * x.x;
-            acc[1] += w * x.y;
+    // splits in batches of kB: the batch's loads are in flight together
+    constexpr int kB = 6;
+    for (int s0 = 0; s0 < n_split; s0 += kB) {
+        float2 ml[kB];
+        float x[kB][PER];
+#pragma unroll
+        for (int u = 0; u < kB; ++u) {
+            const int s = s0 + u;
+            if (s < n_split) {
+                ml[u] = __ldcg(reinterpret_cast<const float2 *>(ws_ml + ((size_t)s * rows_all + row) * 2));
+                const float *src = ws_o + ((size_t)s * rows_all + row) * D + lane * PER;
+                if constexpr (PER == 4) {
+                    const float4 v = __ldcg(reinterpret_cast<const float4 *>(src));
+                    x[u][0] = v.x; x[u][1] = v.y; x[u][2] = v.z; x[u][3] = v.w;
+                } else {
+                    const float2 v = __ldcg(reinterpret_cast<const float2 *>(src));
+                    x[u][0] = v.x; x[u][1] = v.y;
+                }
+            } else {
+                ml[u] = make_float2(-INFINITY, 0.f);
+#pragma unroll
+                for (int e = 0; e < PER; ++e)
+                    x[u][e] = 0.f;
+            }
+        }
+#pragma unroll
+        for (int u = 0; u < kB; ++u) {
+            const float w = ml[u].x == -INFINITY ? 0.f : exp2f(ml[u].x - M);
+            L += w * ml[u].y;
+#pragma unroll
+            for (int e = 0; e < PER; ++e)
+                acc[e] += w * x[u][e];
         }
     }
     const float inv = 1.f / L;

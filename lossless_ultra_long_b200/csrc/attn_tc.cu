@@ -12,28 +12,38 @@
 // The two products run in the orientations the tensor core executes at
 // full rate (an MMA instruction costs about the same below N = 128, and an
 // MN-major B operand runs at about half rate):
-//   S_b  = Q_b K^T      rows on M (128-row blocks b), N = 64 positions,
-//                       both operands K-major in shared memory;
+//   S_b  = Q_b K^T      rows on M (128-row blocks b), N = 64 positions;
+//                       Q_b is held in TMEM (loaded once), K is K-major in
+//                       shared memory;
 //   O^T += V^T P^T      head dim on M, all R rows on N (padded to 16),
 //                       V^T is the TMA tile read MN-major, P^T K-major.
 // P^T is written to shared memory by the softmax threads, one row each.
+// Shared-memory bandwidth (about 128 B/clk for tensor-core operand reads)
+// is the scarce resource at these shapes, which is why Q lives in TMEM
+// rather than being re-read from shared memory by every QK instruction.
 //
-// CTA = (split, KV head), 12 warps, one CTA per SM:
+// CTA = (split, KV head), 15 warps, one CTA per SM:
 //   warps 0, 2  TMA producers for K and for V: 64-position tiles (two
 //               64-column boxes each, 128-byte swizzle) into two rings.  The
 //               tensor map's row extent is n_ctx + T, so rows past the tree
 //               tail arrive as zeros.
-//   warp 1      allocates TMEM; one lane issues every tcgen05.mma.  S is
-//               double-buffered so QK of tile t+1 overlaps the softmax of t.
-//   warps 4..   softmax, one thread per query row (TMEM lane of its block):
+//   warp 1      allocates TMEM; one lane issues every tcgen05.mma.  A
+//               block's S is released as soon as its softmax warps have
+//               loaded it into registers, so QK of tile t+1 overlaps the
+//               softmax arithmetic of tile t.
+//   warps 4-7, 12-14  softmax, one thread per query row (a TMEM lane of
+//               its block; block 0 rows on warps 4-7, block 1 rows on 12-14):
 //               scale to base 2, ancestor mask on tiles that reach the tree
 //               tail, exponentiate against a per-row reference max, write
-//               the bf16 P^T row.  The reference only moves when a tile's
-//               max exceeds it by more than 2^8; then warps 4-7 (which
-//               between them see all 128 TMEM lanes, i.e. all of D) rescale
-//               the affected O^T columns before the next PV.  l sums the
-//               bf16-rounded P so the normalisation matches what PV used.
-// TMEM: O^T in columns [0, R_pad); S_b(buf) at kSCol0 + 64 (2b + buf).
+//               the bf16 P^T row.  l sums the bf16-rounded P so the
+//               normalisation matches what PV used.
+//   warps 8-11  correctors: between them they see all 128 TMEM lanes, i.e.
+//               all of D.  After every softmax warp has finished a tile they
+//               release it to PV; when a row's reference max moved (only
+//               when a tile's max exceeds it by more than 2^8) they first
+//               rescale that row's O^T column.  At the end they write O^T.
+// TMEM: O^T in [0, kOCols), Q_b in 64 columns from kQCol0, S_b in 64
+// columns from kSCol0.
 // Each split leaves an unnormalised partial (acc, m, l) for the combine
 // kernel, or normalises in place when it is the only split.
 //
@@ -59,11 +69,9 @@ constexpr int kTileN = 64;                      // KV positions per tile
 constexpr int kBlockM = 128;                    // query rows per QK block
 constexpr int kBoxBytes = kTileN * 64 * 2;      // one 64-column box of a tile: 8 KB
 constexpr int kHalfStageBytes = 2 * kBoxBytes;  // K (or V) of a tile: lo and hi boxes
-constexpr int kQBlockBytes = kBlockM * kD * 2;  // 32 KB
-constexpr int kThreads = 384;
-constexpr int kFirstSoftmaxWarp = 4;
+constexpr int kThreads = 480;    // 15 warps
 constexpr int kMaxStages = 8;
-constexpr int kMaxRows = 256;
+constexpr int kMaxRows = 224;    // block 1 has softmax warps 12-14 only
 constexpr size_t kSmemLimit = 232448;           // dynamic shared memory per CTA
 
 struct TcBarriers {
@@ -71,21 +79,22 @@ struct TcBarriers {
     uint64_t empty_k[kMaxStages];
     uint64_t full_v[kMaxStages];
     uint64_t empty_v[kMaxStages];
-    uint64_t s_full[2][2];     // QK of a block landed in S(buf)
+    uint64_t s_full[2];        // QK of a block landed in its S
+    uint64_t s_free[2];        // that block's softmax warps hold S in registers
     uint64_t sm_sync[2];       // every softmax warp finished a tile
     uint64_t p_full[2];        // P^T(buf) written and O^T corrected
-    uint64_t o_done;           // one commit per PV
+    uint64_t pv_done[2];       // PV of a tile whose P^T sat in buffer (t & 1) finished
     uint64_t o_final;          // committed once, after the last PV
-    uint64_t drain;
+    uint64_t drain[2];         // each issuing thread's own MMAs, before TMEM is freed
     uint32_t tmem_base;
     uint32_t abort;
     int32_t rescale_tile[2];   // tile index + 1 when that tile moved a row's max
 };
 
 struct TcAux {
-    float factor[2][kMaxRows];  // per-row O^T rescale factor of the tile
-    float l[kMaxRows];
-    float m[kMaxRows];
+    float factor[2][256];  // per-row O^T rescale factor of the tile (32-column reads)
+    float l[256];
+    float m[256];
     TcBarriers bar;
 };
 constexpr size_t kAuxBytes = (sizeof(TcAux) + 1023) / 1024 * 1024;
@@ -100,7 +109,8 @@ __host__ __device__ inline TcLayout tc_layout(int nb, int rows)
 {
     TcLayout L;
     L.r_pad = (rows + 15) / 16 * 16;
-    L.p_off = (size_t)nb * kQBlockBytes;
+    (void)nb;
+    L.p_off = 0;
     L.k_off = L.p_off + 2 * (size_t)L.r_pad * 128;
     const size_t fixed = 1024 + L.k_off + kAuxBytes;
     int halves = (int)((kSmemLimit - fixed) / kHalfStageBytes);
@@ -160,9 +170,10 @@ __global__ void __launch_bounds__(kThreads, 1)
 attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_constant__ CUtensorMap tmap_v,
                AttnArgs a, TreeMasks masks, int tiles_per_split, int n_split)
 {
-    constexpr int kSCol0 = NB == 2 ? 256 : 128;
+    constexpr int kOCols = NB == 2 ? 256 : 128;
+    constexpr int kQCol0 = kOCols;
+    constexpr int kSCol0 = kQCol0 + 64 * NB;
     constexpr int kTmemCols = NB == 2 ? 512 : 256;
-    constexpr int kSoftmaxWarps = 4 * NB;
 
     const int G = a.n_heads_q / a.n_heads_kv;
     const int R = G * a.n_tree;
@@ -172,7 +183,6 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_constant
     extern __shared__ unsigned char smem_raw[];
     unsigned char *base = reinterpret_cast<unsigned char *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    unsigned char *sQ = base;
     unsigned char *sP = base + lay.p_off;
     unsigned char *sK = base + lay.k_off;
     unsigned char *sV = base + lay.v_off;
@@ -188,11 +198,14 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_constant
     const int t_begin = split * tiles_per_split;
     const int n_tiles = min(t_begin + tiles_per_split, n_tiles_all) - t_begin;
 
-    // softmax warps that take part in the per-tile sync: those with rows,
-    // and warps 4-7, which rescale and write out O^T
-    int sync_warps = 0;
-    for (int w = 0; w < kSoftmaxWarps; ++w)
-        sync_warps += (w < 4) || ((w / 4) * kBlockM + (w % 4) * 32 < R);
+    // softmax warps with rows: they arrive once per tile on sm_sync, and on
+    // their block's s_free
+    int sync_warps = 0, block_warps[2] = {0, 0};
+    for (int w = 0; w < 4 * NB && w < 7; ++w) {
+        const int has = (w / 4) * kBlockM + (w % 4) * 32 < R;
+        sync_warps += has;
+        block_warps[w / 4] += has;
+    }
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < SK; ++s) {
@@ -203,16 +216,20 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_constant
             mbar_init(smem_addr(&bar->full_v[s]), 1);
             mbar_init(smem_addr(&bar->empty_v[s]), 1);
         }
+        for (int b = 0; b < NB; ++b) {
+            mbar_init(smem_addr(&bar->s_full[b]), 1);
+            mbar_init(smem_addr(&bar->s_free[b]), block_warps[b]);
+        }
         for (int u = 0; u < 2; ++u) {
-            for (int b = 0; b < NB; ++b)
-                mbar_init(smem_addr(&bar->s_full[b][u]), 1);
             mbar_init(smem_addr(&bar->sm_sync[u]), sync_warps);
             mbar_init(smem_addr(&bar->p_full[u]), 4);
             bar->rescale_tile[u] = 0;
         }
-        mbar_init(smem_addr(&bar->o_done), 1);
+        mbar_init(smem_addr(&bar->pv_done[0]), 1);
+        mbar_init(smem_addr(&bar->pv_done[1]), 1);
         mbar_init(smem_addr(&bar->o_final), 1);
-        mbar_init(smem_addr(&bar->drain), 1);
+        mbar_init(smem_addr(&bar->drain[0]), 1);
+        mbar_init(smem_addr(&bar->drain[1]), 1);
         bar->abort = 0u;
         fence_mbar_init();
     }
@@ -225,26 +242,47 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_constant
         prefetch_tmap(&tmap_v);
     }
 
-    // Q rows of this KV head into 128-byte-swizzled K-major blocks:
-    // row r (node r / G, head g*G + r % G), 16-byte chunk c of the row.
-    for (int idx = threadIdx.x; idx < NB * kBlockM * (kD / 8); idx += kThreads) {
-        const int r = idx / (kD / 8), c = idx % (kD / 8);
-        uint4 val = make_uint4(0u, 0u, 0u, 0u);
-        if (r < R) {
-            const int node = r / G, h = g * G + r % G;
-            val = *reinterpret_cast<const uint4 *>(a.q + ((int64_t)node * a.n_heads_q + h) * kD +
-                                                   c * 8);
-        }
-        const int blk = r / kBlockM, rr = r % kBlockM, half = c / 8, cc = c % 8;
-        unsigned char *dst = sQ + blk * kQBlockBytes + half * (kBlockM * 128) + rr * 128 +
-                             ((cc ^ (rr & 7)) << 4);
-        *reinterpret_cast<uint4 *>(dst) = val;
-    }
-    fence_proxy_async_smem();
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = bar->tmem_base;
+
+    // Q rows of this KV head into TMEM, as the A operand of QK: the thread
+    // owning query row r (node r / G, head g*G + r % G) writes its 128 bf16
+    // as 64 packed columns of its block's lane.
+    if ((warp >= 4 && warp < 8) || (NB == 2 && warp >= 12)) {
+        const int b = warp < 8 ? 0 : 1;
+        const int quarter = warp & 3;
+        if (b * kBlockM + quarter * 32 < R) {
+            const int r = b * kBlockM + quarter * 32 + lane;
+            uint32_t qv[64];
+            if (r < R) {
+                const uint4 *src = reinterpret_cast<const uint4 *>(
+                    a.q + ((int64_t)(r / G) * a.n_heads_q + g * G + r % G) * kD);
+#pragma unroll
+                for (int c = 0; c < 16; ++c) {
+                    const uint4 u = src[c];
+                    qv[4 * c] = u.x;
+                    qv[4 * c + 1] = u.y;
+                    qv[4 * c + 2] = u.z;
+                    qv[4 * c + 3] = u.w;
+                }
+            } else {
+#pragma unroll
+                for (int c = 0; c < 64; ++c)
+                    qv[c] = 0u;
+            }
+            const uint32_t qa = tmem + ((uint32_t)(quarter * 32) << 16) + kQCol0 + 64 * b;
+            uint32_t (&q0)[32] = *reinterpret_cast<uint32_t (*)[32]>(&qv[0]);
+            uint32_t (&q1)[32] = *reinterpret_cast<uint32_t (*)[32]>(&qv[32]);
+            tmem_st32(qa, q0);
+            tmem_st32(qa + 32, q1);
+            tmem_st_wait();
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
 
     if (warp == 0 || warp == 2) {
         // ----------------------------------------- TMA producers (K, V)
@@ -276,102 +314,104 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_constant
                     wait_drain(smem_addr(&full[t % ns]), (t / ns) & 1);
             }
         }
-    } else if (warp == 1) {
-        // ------------------------------------------------------- MMA issuer
+    } else if (warp == 1 || warp == 3) {
+        // --------------------------------------------- MMA issuers: QK, PV
+        // Two threads feed the tensor core, so that one issues while the
+        // other waits; each commits (and at the end drains) its own MMAs.
         if (lane == 0) {
-            constexpr uint32_t idesc_qk = idesc_bf16(kBlockM, kTileN, 0, 0);
-            const uint32_t idesc_pv = idesc_bf16(kD, r_pad, 1, 0);
             // Descriptors are built once; per MMA only the start-address
             // field moves (address / 16 in the low bits, no carry out of it
             // inside shared memory).
-            uint64_t qd[NB][8];
-#pragma unroll
-            for (int b = 0; b < NB; ++b)
-#pragma unroll
-                for (int kk = 0; kk < 8; ++kk)
-                    qd[b][kk] = sdesc_sw128(smem_addr(sQ) + b * kQBlockBytes +
-                                                (kk >> 2) * (kBlockM * 128) + (kk & 3) * 32,
-                                            16, 1024);
-            const uint64_t kd0 = sdesc_sw128(smem_addr(sK), 16, 1024);
-            const uint64_t vd0 = sdesc_sw128(smem_addr(sV), kBoxBytes, 1024);
-            const uint64_t pd0 = sdesc_sw128(smem_addr(sP), 16, 1024);
             constexpr uint64_t kStageStep = kHalfStageBytes >> 4;
-            bool ok = true;
-            for (int t = 0; t <= n_tiles && ok; ++t) {
-                if (t < n_tiles) {
+            if (warp == 1) {
+                constexpr uint32_t idesc_qk = idesc_bf16(kBlockM, kTileN, 0, 0);
+                const uint64_t kd0 = sdesc_sw128(smem_addr(sK), 16, 1024);
+                for (int t = 0; t < n_tiles; ++t) {
                     const int s = t % SK;
-                    if (!wait_bounded(smem_addr(&bar->full_k[s]), (t / SK) & 1, abort, hdr)) {
-                        ok = false;
+                    if (!wait_bounded(smem_addr(&bar->full_k[s]), (t / SK) & 1, abort, hdr))
                         break;
-                    }
                     tc_fence_after();
                     const uint64_t kd = kd0 + (uint64_t)s * kStageStep;
+                    bool ok = true;
 #pragma unroll
                     for (int b = 0; b < NB; ++b) {
-                        const uint32_t d_col = tmem + kSCol0 + 64 * (2 * b + (t & 1));
-                        mma_ss_c<0>(d_col, qd[b][0], kd, idesc_qk);
+                        // S_b is reused: its softmax warps must hold S(t-1)
+                        if (t > 0 &&
+                            !wait_bounded(smem_addr(&bar->s_free[b]), (t - 1) & 1, abort, hdr)) {
+                            ok = false;
+                            break;
+                        }
+                        tc_fence_after();
+                        const uint32_t d_col = tmem + kSCol0 + 64 * b;
+                        const uint32_t q_col = tmem + kQCol0 + 64 * b;
+                        mma_ts_c<0>(d_col, q_col, kd, idesc_qk);
 #pragma unroll
                         for (int kk = 1; kk < kD / 16; ++kk)
-                            mma_ss_c<1>(d_col, qd[b][kk],
+                            mma_ts_c<1>(d_col, q_col + kk * 8,
                                         kd + (((kk >> 2) * kBoxBytes + (kk & 3) * 32) >> 4),
                                         idesc_qk);
-                        mma_commit(smem_addr(&bar->s_full[b][t & 1]));
+                        mma_commit(smem_addr(&bar->s_full[b]));
                     }
+                    if (!ok)
+                        break;
                     mma_commit(smem_addr(&bar->empty_k[s]));
                 }
-                if (t >= 1) {
-                    const int u = t - 1, s = u % SV;
-                    if (!wait_bounded(smem_addr(&bar->full_v[s]), (u / SV) & 1, abort, hdr) ||
-                        !wait_bounded(smem_addr(&bar->p_full[u & 1]), (u >> 1) & 1, abort, hdr)) {
-                        ok = false;
+            } else {
+                const uint32_t idesc_pv = idesc_bf16(kD, r_pad, 1, 0);
+                const uint64_t vd0 = sdesc_sw128(smem_addr(sV), kBoxBytes, 1024);
+                const uint64_t pd0 = sdesc_sw128(smem_addr(sP), 16, 1024);
+                for (int t = 0; t < n_tiles; ++t) {
+                    const int s = t % SV;
+                    if (!wait_bounded(smem_addr(&bar->full_v[s]), (t / SV) & 1, abort, hdr) ||
+                        !wait_bounded(smem_addr(&bar->p_full[t & 1]), (t >> 1) & 1, abort, hdr))
                         break;
-                    }
                     tc_fence_after();
                     const uint64_t vd = vd0 + (uint64_t)s * kStageStep;
-                    const uint64_t pd = pd0 + (uint64_t)((u & 1) * r_pad * 128 >> 4);
-                    if (u == 0)
+                    const uint64_t pd = pd0 + (uint64_t)((t & 1) * r_pad * 128 >> 4);
+                    if (t == 0)
                         mma_ss_c<0>(tmem, vd, pd, idesc_pv);
                     else
                         mma_ss_c<1>(tmem, vd, pd, idesc_pv);
 #pragma unroll
                     for (int kk = 1; kk < kTileN / 16; ++kk)
                         mma_ss_c<1>(tmem, vd + kk * (2048 >> 4), pd + kk * (32 >> 4), idesc_pv);
-                    mma_commit(smem_addr(&bar->o_done));
-                    if (u == n_tiles - 1)
+                    mma_commit(smem_addr(&bar->pv_done[t & 1]));
+                    if (t == n_tiles - 1)
                         mma_commit(smem_addr(&bar->o_final));
                     mma_commit(smem_addr(&bar->empty_v[s]));
                 }
             }
-            // every MMA issued above has finished before TMEM is released
-            mma_commit(smem_addr(&bar->drain));
-            wait_drain(smem_addr(&bar->drain), 0);
+            // every MMA this thread issued has finished before TMEM is released
+            const int dn = warp == 1 ? 0 : 1;
+            mma_commit(smem_addr(&bar->drain[dn]));
+            wait_drain(smem_addr(&bar->drain[dn]), 0);
         }
-    } else if (warp >= kFirstSoftmaxWarp && warp < kFirstSoftmaxWarp + kSoftmaxWarps &&
-               ((warp - kFirstSoftmaxWarp) < 4 ||
-                (warp - kFirstSoftmaxWarp) / 4 * kBlockM + (warp & 3) * 32 < R)) {
+    } else if ((warp >= 4 && warp < 8) || (NB == 2 && warp >= 12)) {
         // ---------------------------------------------------------- softmax
-        const int b = (warp - kFirstSoftmaxWarp) / 4;
+        const int b = warp < 8 ? 0 : 1;
         const int quarter = warp & 3;
-        const bool corrector = b == 0;   // warps 4-7: all 128 lanes between them
-        const bool active = b * kBlockM + quarter * 32 < R;
         const int r = b * kBlockM + quarter * 32 + lane;
-        const int rr = r < R ? r : 0;
-        const int node = rr / G;
-        const unsigned long long anc = masks.anc[node];
-        const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
-        float m_ref = -INFINITY, l = 0.f;
-        bool ok = true;
-        for (int t = 0; t < n_tiles; ++t) {
-            const int buf = t & 1;
-            if (active) {
-                if (!warp_wait_bounded(smem_addr(&bar->s_full[b][buf]), (t >> 1) & 1, abort,
-                                       hdr)) {
+        if (b * kBlockM + quarter * 32 < R) {
+            const int rr = r < R ? r : 0;
+            const int node = rr / G;
+            const unsigned long long anc = masks.anc[node];
+            const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
+            float m_ref = -INFINITY, l = 0.f;
+            bool ok = true;
+            for (int t = 0; t < n_tiles; ++t) {
+                const int buf = t & 1;
+                if (!warp_wait_bounded(smem_addr(&bar->s_full[b]), t & 1, abort, hdr)) {
                     ok = false;
                     break;
                 }
                 tc_fence_after();
                 uint32_t raw[64];
-                tmem_ld64(tmem + lane_off + kSCol0 + 64 * (2 * b + buf), raw);
+                tmem_ld64(tmem + lane_off + kSCol0 + 64 * b, raw);
+                // S is in registers: QK of the next tile may overwrite it
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0)
+                    mbar_arrive(smem_addr(&bar->s_free[b]));
                 // raw scores; the scale (> 0) is applied inside the exponent
                 float x[64];
                 const int pos0 = (t_begin + t) * kTileN;
@@ -413,12 +453,17 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_constant
                     bar->rescale_tile[buf] = t + 1;
                 const float neg_m = m_ref == -INFINITY ? 0.f : -m_ref;
                 uint32_t pk[32];
-                // the choice of exponent paths is hoisted out of the unrolled
-                // loop so that each version is straight-line code
-                if (edge)
-                    l += exp_pack_tile<false>(x, a.scale_log2, neg_m, pk);
-                else
-                    l += exp_pack_tile<true>(x, a.scale_log2, neg_m, pk);
+                l += exp_pack_tile<false>(x, a.scale_log2, neg_m, pk);
+                // P^T(t) reuses the buffer of P^T(t-2): PV(t-2) must be done.
+                // PV(t-4), the buffer's previous user, finished before this
+                // warp wrote P^T(t-2), so pv_done[buf] has exactly one phase
+                // that can still be open
+                if (t >= 2 &&
+                    !warp_wait_bounded(smem_addr(&bar->pv_done[buf]), ((t - 2) >> 1) & 1, abort,
+                                       hdr)) {
+                    ok = false;
+                    break;
+                }
                 // P^T row r: 64 bf16 = one 128-byte swizzled row of the K-major tile
                 unsigned char *prow = sP + buf * r_pad * 128 + (r >> 3) * 1024 + (r & 7) * 128;
                 if (r < r_pad) {
@@ -428,78 +473,89 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_constant
                             make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
                 }
                 fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0)
+                    mbar_arrive(smem_addr(&bar->sm_sync[buf]));
             }
-            __syncwarp();
-            if (lane == 0)
-                mbar_arrive(smem_addr(&bar->sm_sync[buf]));
-            if (corrector) {
-                if (!warp_wait_bounded(smem_addr(&bar->sm_sync[buf]), (t >> 1) & 1, abort, hdr)) {
+            // publish (m, l) for the correctors' epilogue
+            if (ok) {
+                const int rows_all = a.n_tree * a.n_heads_q;
+                float *ws_ml = reinterpret_cast<float *>(reinterpret_cast<char *>(a.workspace) +
+                                                         kHeaderBytes) +
+                               (size_t)n_split * rows_all * kD;
+                if (r < R) {
+                    aux->l[r] = l;
+                    if (n_split > 1) {
+                        const int orow = node * a.n_heads_q + g * G + r % G;
+                        *reinterpret_cast<float2 *>(ws_ml +
+                                                    ((size_t)split * rows_all + orow) * 2) =
+                            make_float2(m_ref, l);
+                    }
+                }
+                __syncwarp();
+                if (lane == 0)
+                    mbar_arrive(smem_addr(&bar->sm_sync[n_tiles & 1]));
+            }
+        }
+    } else if (warp >= 8 && warp < 12) {
+        // -------------------------------------------------------- correctors
+        const int quarter = warp & 3;
+        const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
+        bool ok = true;
+        for (int t = 0; t < n_tiles; ++t) {
+            const int buf = t & 1;
+            if (!warp_wait_bounded(smem_addr(&bar->sm_sync[buf]), (t >> 1) & 1, abort, hdr)) {
+                ok = false;
+                break;
+            }
+            if (t > 0 && bar->rescale_tile[buf] == t + 1) {
+                // PV(t-1) must be done.  Every softmax warp waited for
+                // PV(t-2) before writing P^T(t), and PV runs in order, so
+                // PV(t-3) is done too: pv_done[(t-1) & 1] has one open phase
+                if (!warp_wait_bounded(smem_addr(&bar->pv_done[(t - 1) & 1]), ((t - 1) >> 1) & 1,
+                                       abort, hdr)) {
                     ok = false;
                     break;
                 }
-                if (t > 0 && bar->rescale_tile[buf] == t + 1) {
-                    // S(t) was committed after PV(t-2) was issued, so o_done has
-                    // completed t-1 or t phases: parity (t-1) tells them apart
-                    if (!warp_wait_bounded(smem_addr(&bar->o_done), (t - 1) & 1, abort, hdr)) {
-                        ok = false;
-                        break;
-                    }
-                    tc_fence_after();
-                    for (int c = 0; c < r_pad; c += 32) {
-                        uint32_t o[32];
-                        tmem_ld32(tmem + lane_off + c, o);
-#pragma unroll
-                        for (int j = 0; j < 32; ++j)
-                            o[j] = __float_as_uint(__uint_as_float(o[j]) *
-                                                   aux->factor[buf][c + j]);
-                        tmem_st32(tmem + lane_off + c, o);
-                    }
-                    tmem_st_wait();
-                }
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0)
-                    mbar_arrive(smem_addr(&bar->p_full[buf]));
-            }
-        }
-
-        // ---- epilogue: row owners publish (m, l); warps 4-7 write O^T out
-        if (ok) {
-            const int rows_all = a.n_tree * a.n_heads_q;
-            float *ws_o =
-                reinterpret_cast<float *>(reinterpret_cast<char *>(a.workspace) + kHeaderBytes);
-            float *ws_ml = ws_o + (size_t)n_split * rows_all * kD;
-            if (active && r < R) {
-                aux->l[r] = l;
-                if (n_split > 1) {
-                    const int orow = node * a.n_heads_q + g * G + r % G;
-                    *reinterpret_cast<float2 *>(ws_ml + ((size_t)split * rows_all + orow) * 2) =
-                        make_float2(m_ref, l);
-                }
-            }
-            __syncwarp();
-            if (lane == 0)
-                mbar_arrive(smem_addr(&bar->sm_sync[n_tiles & 1]));
-            if (corrector &&
-                warp_wait_bounded(smem_addr(&bar->sm_sync[n_tiles & 1]), (n_tiles >> 1) & 1,
-                                  abort, hdr) &&
-                warp_wait_bounded(smem_addr(&bar->o_final), 0, abort, hdr)) {
                 tc_fence_after();
-                const int d = quarter * 32 + lane;
                 for (int c = 0; c < r_pad; c += 32) {
                     uint32_t o[32];
                     tmem_ld32(tmem + lane_off + c, o);
 #pragma unroll
-                    for (int j = 0; j < 32; ++j) {
-                        const int rw = c + j;
-                        if (rw < R) {
-                            const int orow = (rw / G) * a.n_heads_q + g * G + rw % G;
-                            const float v = __uint_as_float(o[j]);
-                            if (n_split == 1)
-                                a.out[(size_t)orow * kD + d] = v / aux->l[rw];
-                            else
-                                ws_o[((size_t)split * rows_all + orow) * kD + d] = v;
-                        }
+                    for (int j = 0; j < 32; ++j)
+                        o[j] = __float_as_uint(__uint_as_float(o[j]) * aux->factor[buf][c + j]);
+                    tmem_st32(tmem + lane_off + c, o);
+                }
+                tmem_st_wait();
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0)
+                mbar_arrive(smem_addr(&bar->p_full[buf]));
+        }
+        // ---- epilogue: O^T (D on lanes, query rows on columns) to out / partials
+        if (ok &&
+            warp_wait_bounded(smem_addr(&bar->sm_sync[n_tiles & 1]), (n_tiles >> 1) & 1, abort,
+                              hdr) &&
+            warp_wait_bounded(smem_addr(&bar->o_final), 0, abort, hdr)) {
+            tc_fence_after();
+            const int rows_all = a.n_tree * a.n_heads_q;
+            float *ws_o =
+                reinterpret_cast<float *>(reinterpret_cast<char *>(a.workspace) + kHeaderBytes);
+            const int d = quarter * 32 + lane;
+            for (int c = 0; c < r_pad; c += 32) {
+                uint32_t o[32];
+                tmem_ld32(tmem + lane_off + c, o);
+#pragma unroll
+                for (int j = 0; j < 32; ++j) {
+                    const int rw = c + j;
+                    if (rw < R) {
+                        const int orow = (rw / G) * a.n_heads_q + g * G + rw % G;
+                        const float v = __uint_as_float(o[j]);
+                        if (n_split == 1)
+                            a.out[(size_t)orow * kD + d] = v / aux->l[rw];
+                        else
+                            ws_o[((size_t)split * rows_all + orow) * kD + d] = v;
                     }
                 }
             }

@@ -99,10 +99,22 @@ penalize_accept_kernel(PenalizeArgs a, TreeParents tree, int n_chunks)
     const float p = a.penalty;
     Best b{-INFINITY, INT_MAX};
     if ((a.vocab & 3) == 0) {
-        for (int v = v0 + tid * 4; v < v1; v += kThreads * 4) {
-            const float4 x4 = __ldcs(reinterpret_cast<const float4 *>(row + v));
+        // all of this thread's 16-byte loads are issued before any is used
+        constexpr int kPer = kChunk / (kThreads * 4);
+        float4 x4[kPer];
+#pragma unroll
+        for (int u = 0; u < kPer; ++u) {
+            const int v = v0 + (u * kThreads + tid) * 4;
+            x4[u] = v < v1 ? __ldcs(reinterpret_cast<const float4 *>(row + v))
+                           : make_float4(-INFINITY, -INFINITY, -INFINITY, -INFINITY);
+        }
+#pragma unroll
+        for (int u = 0; u < kPer; ++u) {
+            const int v = v0 + (u * kThreads + tid) * 4;
+            if (v >= v1)
+                continue;
             const uint32_t word = bits[(v - v0) >> 5] >> ((v - v0) & 31);
-            float x[4] = {x4.x, x4.y, x4.z, x4.w};
+            float x[4] = {x4[u].x, x4[u].y, x4[u].z, x4[u].w};
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
                 float y = ((word >> e) & 1u) ? penalise(x[e], p) : x[e];

@@ -8,7 +8,9 @@
 // that partial cache.
 //
 // Pass 1 (grid: chunks x Hkv): s[h,n] = log2(e) * scale * q_last[h] . k[g,n]
-//   for the G query heads of KV head g.  Each lane loads 16 bytes of a key
+//   for the G query heads of KV head g.  A CTA streams its chunk of key rows
+//   (contiguous for one head) through a 4-stage shared-memory ring filled by
+//   1-D bulk async copies of 64 rows.  Each lane takes 16 bytes of a key
 //   row (a row is D/8 lanes), forms the partial dots of several rows and
 //   heads, and a transpose-reduce across the row's lanes leaves one finished
 //   (row, head) dot per lane: one shuffle per dot instead of log2(D/8).
@@ -27,6 +29,7 @@
 #include <cooperative_groups.h>
 #include <math.h>
 
+#include "sm100.cuh"
 #include "ts_internal.cuh"
 
 namespace cg = cooperative_groups;
@@ -41,15 +44,34 @@ constexpr int kMaxSlice = 48 * 1024;   // positions per CTA held in shared memor
 constexpr int kMaxGroup = 8;
 
 // ------------------------------------------------------------------ pass 1
+constexpr int kP1Rows = 64;     // key rows per pipeline stage
+constexpr int kP1Stages = 4;
+
+__device__ __forceinline__ void bulk_load(uint32_t dst, const void *src, uint32_t bytes,
+                                          uint32_t bar)
+{
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];\n"
+        ::"r"(dst), "l"(src), "r"(bytes), "r"(bar)
+        : "memory");
+}
+
 template <int D, int GP>
 __global__ void __launch_bounds__(kP1Threads)
 score_logits_kernel(SelectArgs a, int chunk, int n_chunks)
 {
+    using namespace sm100;
     constexpr int LPR = D / 8;          // lanes per key row (16 bytes each)
     constexpr int NV = LPR;             // values per lane before the reduce
     constexpr int RL = NV / GP;         // rows per lane group per step
     constexpr int GROUPS = 32 / LPR;    // lane groups per warp
     constexpr int ROWS_PER_WARP = GROUPS * RL;
+    constexpr int kStageBytes = kP1Rows * D * 2;
+
+    extern __shared__ __align__(128) unsigned char ring_raw[];
+    unsigned char(*ring)[kStageBytes] = reinterpret_cast<unsigned char(*)[kStageBytes]>(ring_raw);
+    __shared__ uint64_t full[kP1Stages];
+    __shared__ uint32_t abort_flag;
 
     const int g = blockIdx.y;
     const int c = blockIdx.x;
@@ -58,6 +80,27 @@ score_logits_kernel(SelectArgs a, int chunk, int n_chunks)
     const int li = lane % LPR, grp = lane / LPR;
     const int n0 = c * chunk;
     const int n1 = min(n0 + chunk, a.n_ctx);
+    const int n_tiles = (n1 - n0 + kP1Rows - 1) / kP1Rows;
+    const __nv_bfloat16 *kh = a.k + (int64_t)g * a.kv_cap * D;
+    WorkspaceHeader *hdr = reinterpret_cast<WorkspaceHeader *>(a.workspace);
+
+    // rows of one KV head are contiguous: each tile is one bulk copy
+    auto issue = [&](int t) {
+        const int r0 = n0 + t * kP1Rows;
+        const uint32_t bytes = (uint32_t)min(kP1Rows, n1 - r0) * D * 2;
+        const uint32_t fb = smem_addr(&full[t % kP1Stages]);
+        mbar_arrive_expect_tx(fb, bytes);
+        bulk_load(smem_addr(ring[t % kP1Stages]), kh + (int64_t)r0 * D, bytes, fb);
+    };
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kP1Stages; ++s)
+            mbar_init(smem_addr(&full[s]), 1);
+        abort_flag = 0u;
+        fence_mbar_init();
+        fence_proxy_async_smem();
+        for (int t = 0; t < min(kP1Stages, n_tiles); ++t)
+            issue(t);
+    }
 
     float qf[GP][8];
 #pragma unroll
@@ -78,61 +121,71 @@ score_logits_kernel(SelectArgs a, int chunk, int n_chunks)
                 qf[h][e] = 0.f;
         }
     }
+    __syncthreads();
+
     // this lane's finished value is always head (li % GP), row slot li / GP
     const int my_h = li % GP, my_j = li / GP;
     float run_m = -INFINITY, run_l = 0.f;
-
-    const __nv_bfloat16 *kh = a.k + (int64_t)g * a.kv_cap * D;
     float *s_out = reinterpret_cast<float *>(reinterpret_cast<char *>(a.workspace) + kHeaderBytes);
     const int nwarps = kP1Threads / 32;
-    for (int base = n0 + warp * ROWS_PER_WARP; base < n1; base += nwarps * ROWS_PER_WARP) {
-        uint4 kr[RL];
+    for (int t = 0; t < n_tiles; ++t) {
+        const bool ok = wait_bounded(smem_addr(&full[t % kP1Stages]), (t / kP1Stages) & 1,
+                                     &abort_flag, hdr);
+        if (__syncthreads_or(!ok))   // leave the loop together
+            break;
+        const unsigned char *stage = ring[t % kP1Stages];
+        const int rows = min(kP1Rows, n1 - (n0 + t * kP1Rows));
+        for (int base = warp * ROWS_PER_WARP; base < rows; base += nwarps * ROWS_PER_WARP) {
+            float v[NV];
 #pragma unroll
-        for (int j = 0; j < RL; ++j) {
-            const int n = base + grp * RL + j;
-            kr[j] = n < n1 ? __ldcs(reinterpret_cast<const uint4 *>(kh + (int64_t)n * D + li * 8))
-                           : make_uint4(0u, 0u, 0u, 0u);
-        }
-        float v[NV];
+            for (int j = 0; j < RL; ++j) {
+                const int r = base + grp * RL + j;
+                const uint4 kr = r < rows ? *reinterpret_cast<const uint4 *>(stage + r * D * 2 + li * 16)
+                                          : make_uint4(0u, 0u, 0u, 0u);
+                const __nv_bfloat162 *p2 = reinterpret_cast<const __nv_bfloat162 *>(&kr);
+                float kf[8];
 #pragma unroll
-        for (int j = 0; j < RL; ++j) {
-            const __nv_bfloat162 *p2 = reinterpret_cast<const __nv_bfloat162 *>(&kr[j]);
-            float kf[8];
+                for (int e = 0; e < 4; ++e) {
+                    const float2 f = __bfloat1622float2(p2[e]);
+                    kf[2 * e] = f.x;
+                    kf[2 * e + 1] = f.y;
+                }
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                const float2 f = __bfloat1622float2(p2[e]);
-                kf[2 * e] = f.x;
-                kf[2 * e + 1] = f.y;
+                for (int h = 0; h < GP; ++h) {
+                    float acc = 0.f;
+#pragma unroll
+                    for (int e = 0; e < 8; ++e)
+                        acc = fmaf(qf[h][e], kf[e], acc);
+                    v[j * GP + h] = acc;
+                }
             }
+            // transpose-reduce across the LPR lanes of the row group
 #pragma unroll
-            for (int h = 0; h < GP; ++h) {
-                float acc = 0.f;
+            for (int o = NV / 2; o >= 1; o >>= 1) {
+                const bool upper = (li & o) != 0;
 #pragma unroll
-                for (int e = 0; e < 8; ++e)
-                    acc = fmaf(qf[h][e], kf[e], acc);
-                v[j * GP + h] = acc;
+                for (int q = 0; q < o; ++q) {
+                    const float send = upper ? v[q] : v[q + o];
+                    const float keep = upper ? v[q + o] : v[q];
+                    v[q] = keep + __shfl_xor_sync(0xffffffffu, send, o);
+                }
+            }
+            const int r = base + grp * RL + my_j;
+            if (my_h < G && r < rows) {
+                const float sv = v[0];
+                s_out[(int64_t)(g * G + my_h) * a.n_ctx + n0 + t * kP1Rows + r] = sv;
+                const float m_new = fmaxf(run_m, sv);
+                run_l = run_l * exp2f(run_m - m_new) + exp2f(sv - m_new);
+                run_m = m_new;
             }
         }
-        // transpose-reduce across the LPR lanes of the row group
-#pragma unroll
-        for (int o = NV / 2; o >= 1; o >>= 1) {
-            const bool upper = (li & o) != 0;
-#pragma unroll
-            for (int t = 0; t < o; ++t) {
-                const float send = upper ? v[t] : v[t + o];
-                const float keep = upper ? v[t + o] : v[t];
-                v[t] = keep + __shfl_xor_sync(0xffffffffu, send, o);
-            }
-        }
-        const int n = base + grp * RL + my_j;
-        if (my_h < G && n < n1) {
-            const float s = v[0];
-            s_out[(int64_t)(g * G + my_h) * a.n_ctx + n] = s;
-            const float m_new = fmaxf(run_m, s);
-            run_l = run_l * exp2f(run_m - m_new) + exp2f(s - m_new);
-            run_m = m_new;
-        }
+        __syncthreads();   // every warp is done with this stage
+        if (threadIdx.x == 0 && t + kP1Stages < n_tiles)
+            issue(t + kP1Stages);
     }
+    if (abort_flag && threadIdx.x == 0)
+        for (int t = max(0, n_tiles - kP1Stages); t < n_tiles; ++t)
+            wait_drain(smem_addr(&full[t % kP1Stages]), (t / kP1Stages) & 1);
 
     // merge the running (max, sum) of every lane that holds head h
     __shared__ float sm_m[kP1Threads], sm_l[kP1Threads];
@@ -253,14 +306,35 @@ select_gather_kernel(SelectArgs a, int n_chunks, int slice)
     }
     __syncthreads();
 
-    // scores of this slice -> order-preserving keys in shared memory
-    for (int n = p0 + tid; n < p1; n += kP2Threads) {
-        float sc = 0.f;
-        for (int h = 0; h < G; ++h)
-            sc += exp2f(s_all[(size_t)(g * G + h) * N + n] - sh.head_m[h]) * sh.head_w[h];
-        keys[n - p0] = order_key(sc);
-        if (a.scores_out)
-            a.scores_out[(size_t)g * N + n] = sc;
+    // scores of this slice -> order-preserving keys in shared memory; four
+    // positions per thread per step so their loads are in flight together
+    constexpr int kU = 4;
+    for (int nb = p0 + tid; nb < p1; nb += kP2Threads * kU) {
+        float sc[kU];
+#pragma unroll
+        for (int u = 0; u < kU; ++u)
+            sc[u] = 0.f;
+        for (int h = 0; h < G; ++h) {
+            const float *row = s_all + (size_t)(g * G + h) * N;
+            float sv[kU];
+#pragma unroll
+            for (int u = 0; u < kU; ++u) {
+                const int n = nb + u * kP2Threads;
+                sv[u] = n < p1 ? __ldcg(row + n) : 0.f;
+            }
+#pragma unroll
+            for (int u = 0; u < kU; ++u)
+                sc[u] += exp2f(sv[u] - sh.head_m[h]) * sh.head_w[h];
+        }
+#pragma unroll
+        for (int u = 0; u < kU; ++u) {
+            const int n = nb + u * kP2Threads;
+            if (n < p1) {
+                keys[n - p0] = order_key(sc[u]);
+                if (a.scores_out)
+                    a.scores_out[(size_t)g * N + n] = sc[u];
+            }
+        }
     }
     __syncthreads();
 
@@ -387,15 +461,28 @@ select_gather_kernel(SelectArgs a, int n_chunks, int slice)
     const int li = tid % LPR;
     __threadfence_block();
     const int my_rows = min(kept_total, n_keep - kept_before);
-    for (int t = tid / LPR; t < my_rows; t += rows_per_pass) {
-        const int slot = kept_before + t;
-        const int n = __ldcg(&idx[slot]);
-        if (n < 0 || n >= N)
-            continue;
-        const uint4 kv = *reinterpret_cast<const uint4 *>(kh + (int64_t)n * D + li * 8);
-        const uint4 vv = *reinterpret_cast<const uint4 *>(vh + (int64_t)n * D + li * 8);
-        *reinterpret_cast<uint4 *>(kp + (int64_t)slot * D + li * 8) = kv;
-        *reinterpret_cast<uint4 *>(vp + (int64_t)slot * D + li * 8) = vv;
+    // four rows per thread per step: their K and V loads are in flight together
+    constexpr int kG = 4;
+    for (int t0 = tid / LPR; t0 < my_rows; t0 += rows_per_pass * kG) {
+        uint4 kv[kG], vv[kG];
+        int slot[kG];
+        bool ok[kG];
+#pragma unroll
+        for (int u = 0; u < kG; ++u) {
+            const int t = t0 + u * rows_per_pass;
+            slot[u] = kept_before + t;
+            const int n = t < my_rows ? __ldcg(&idx[slot[u]]) : -1;
+            ok[u] = n >= 0 && n < N;
+            const int nn = ok[u] ? n : 0;
+            kv[u] = *reinterpret_cast<const uint4 *>(kh + (int64_t)nn * D + li * 8);
+            vv[u] = *reinterpret_cast<const uint4 *>(vh + (int64_t)nn * D + li * 8);
+        }
+#pragma unroll
+        for (int u = 0; u < kG; ++u)
+            if (ok[u]) {
+                *reinterpret_cast<uint4 *>(kp + (int64_t)slot[u] * D + li * 8) = kv[u];
+                *reinterpret_cast<uint4 *>(vp + (int64_t)slot[u] * D + li * 8) = vv[u];
+            }
     }
 }
 
@@ -406,7 +493,8 @@ struct SelPlan {
 SelPlan make_sel_plan(int n_heads_kv, int n_ctx, int num_sms)
 {
     SelPlan p;
-    int want = (num_sms * 4 + n_heads_kv - 1) / n_heads_kv;
+    // three 64 KB-ring CTAs fit an SM: one wave of them over all heads
+    int want = (num_sms * 3 + n_heads_kv - 1) / n_heads_kv;
     const int min_chunk = 512;
     int chunk = (n_ctx + want - 1) / want;
     chunk = chunk < min_chunk ? min_chunk : chunk;
@@ -419,8 +507,13 @@ SelPlan make_sel_plan(int n_heads_kv, int n_ctx, int num_sms)
 template <int D, int GP>
 cudaError_t launch_p1(const SelectArgs &a, const SelPlan &p, cudaStream_t stream)
 {
+    constexpr int smem = kP1Stages * kP1Rows * D * 2;
+    static const cudaError_t attr = cudaFuncSetAttribute(
+        score_logits_kernel<D, GP>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (attr != cudaSuccess)
+        return attr;
     dim3 grid(p.n_chunks, a.n_heads_kv);
-    score_logits_kernel<D, GP><<<grid, kP1Threads, 0, stream>>>(a, p.chunk, p.n_chunks);
+    score_logits_kernel<D, GP><<<grid, kP1Threads, smem, stream>>>(a, p.chunk, p.n_chunks);
     const cudaError_t e = cudaGetLastError();
     if (e == cudaSuccess)
         count_launches(1);

@@ -195,6 +195,20 @@ __device__ __forceinline__ void mma_ts(uint32_t d, uint32_t a_tmem, uint64_t b, 
         : "memory");
 }
 
+// D(tmem) (+)= A(tmem) * B(smem desc), accumulate flag fixed at compile time.
+template <int ACC>
+__device__ __forceinline__ void mma_ts_c(uint32_t d, uint32_t a_tmem, uint64_t b, uint32_t idesc)
+{
+    asm volatile(
+        "{\n"
+        " .reg .pred p;\n"
+        " setp.ne.b32 p, %4, 0;\n"
+        " tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n"
+        "}\n" ::"r"(d),
+        "r"(a_tmem), "l"(b), "r"(idesc), "n"(ACC)
+        : "memory");
+}
+
 // Arrive once on `bar` when every tcgen05 operation this thread issued so
 // far has completed.
 __device__ __forceinline__ void mma_commit(uint32_t bar)
