@@ -2,6 +2,9 @@
 // (tcgen05 and mma.sync) and the dispatch between them.
 #pragma once
 
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
 #include "ts_internal.cuh"
 
 namespace ts {
@@ -30,11 +33,24 @@ size_t attn_mma_workspace_bytes(int n_heads_q, int n_heads_kv, int head_dim, int
 cudaError_t attn_mma_launch(const AttnArgs &a, const TreeMasks &masks, int num_sms,
                             cudaStream_t stream);
 
+// Tensor map over a bf16 [Hkv, kv_cap, 128] cache viewed as 3-D (d,
+// position, head), 128-byte swizzle, boxes of 64 columns x box_rows
+// positions; positions at or past `rows` read as zeros.
+bool encode_kv_map(CUtensorMap *m, const void *ptr, int rows, int64_t kv_cap, int n_heads_kv,
+                   int box_rows);
+
 bool attn_tc_eligible(int n_heads_q, int n_heads_kv, int head_dim, int n_ctx, int n_tree);
 // (the tcgen05 kernel also needs softmax_scale > 0: it takes the row max on
 // unscaled scores)
 AttnPlan attn_tc_plan(int n_heads_q, int n_heads_kv, int n_ctx, int n_tree, int num_sms);
 cudaError_t attn_tc_launch(const AttnArgs &a, const TreeMasks &masks, int num_sms,
                            cudaStream_t stream);
+
+// 128-position tiles, softmax spread over the four SM sub-partitions; up to
+// 192 query rows per KV head.
+bool attn_t128_eligible(int n_heads_q, int n_heads_kv, int head_dim, int n_ctx, int n_tree);
+AttnPlan attn_t128_plan(int n_heads_q, int n_heads_kv, int n_ctx, int n_tree, int num_sms);
+cudaError_t attn_t128_launch(const AttnArgs &a, const TreeMasks &masks, int num_sms,
+                             cudaStream_t stream);
 
 }  // namespace ts

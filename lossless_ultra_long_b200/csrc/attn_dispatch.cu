@@ -1,10 +1,11 @@
 // attn_dispatch.cu -- picks the tree-verify attention kernel for a shape.
 //
-// head_dim 128, at most 256 query rows per KV head (G * T) and a context of
-// at least kTcMinContext positions and a positive softmax scale run on the
-// tcgen05 kernel; everything else (head_dim 64, larger groups or trees,
-// short contexts) on the general mma.sync kernel.  The workspace size
-// covers whichever kernel a launch picks.
+// head_dim 128, a context of at least kTcMinContext positions and a
+// positive softmax scale run on a tcgen05 kernel: the 128-position-tile one
+// up to 192 query rows per KV head (G * T), the 64-position-tile one up to
+// 224.  Everything else (head_dim 64, larger groups or trees, short
+// contexts) runs on the general mma.sync kernel.  The workspace size covers
+// whichever kernel a launch picks.
 #include "attn_common.cuh"
 
 namespace ts {
@@ -14,21 +15,27 @@ size_t attn_workspace_bytes(int n_heads_q, int n_heads_kv, int head_dim, int n_c
 {
     // large enough for whichever kernel the launch picks
     size_t bytes = attn_mma_workspace_bytes(n_heads_q, n_heads_kv, head_dim, n_ctx, n_tree, num_sms);
-    if (attn_tc_eligible(n_heads_q, n_heads_kv, head_dim, n_ctx, n_tree)) {
-        const AttnPlan p = attn_tc_plan(n_heads_q, n_heads_kv, n_ctx, n_tree, num_sms);
+    auto take = [&](const AttnPlan &p) {
         const size_t tc = kHeaderBytes +
                           align_up(attn_partial_bytes(p.n_split, n_heads_q, head_dim, n_tree), 256);
         bytes = tc > bytes ? tc : bytes;
-    }
+    };
+    if (attn_t128_eligible(n_heads_q, n_heads_kv, head_dim, n_ctx, n_tree))
+        take(attn_t128_plan(n_heads_q, n_heads_kv, n_ctx, n_tree, num_sms));
+    if (attn_tc_eligible(n_heads_q, n_heads_kv, head_dim, n_ctx, n_tree))
+        take(attn_tc_plan(n_heads_q, n_heads_kv, n_ctx, n_tree, num_sms));
     return bytes;
 }
 
 cudaError_t attn_launch(const AttnArgs &a, const TreeMasks &masks, int num_sms,
                         cudaStream_t stream)
 {
-    if (attn_tc_eligible(a.n_heads_q, a.n_heads_kv, a.head_dim, a.n_ctx, a.n_tree) &&
-        a.scale_log2 > 0.f)
-        return attn_tc_launch(a, masks, num_sms, stream);
+    if (a.scale_log2 > 0.f) {
+        if (attn_t128_eligible(a.n_heads_q, a.n_heads_kv, a.head_dim, a.n_ctx, a.n_tree))
+            return attn_t128_launch(a, masks, num_sms, stream);
+        if (attn_tc_eligible(a.n_heads_q, a.n_heads_kv, a.head_dim, a.n_ctx, a.n_tree))
+            return attn_tc_launch(a, masks, num_sms, stream);
+    }
     return attn_mma_launch(a, masks, num_sms, stream);
 }
 

@@ -1,0 +1,666 @@
+// attn_t128.cu -- split-KV tree-verify attention on the 5th-generation tensor
+// cores with 128-position KV tiles and the softmax spread evenly over the
+// four SM sub-partitions.
+//
+// Tree-based verification runs every draft-tree node's query against the
+// full KV cache, each node seeing the context plus its own root path
+// (TokenSwift, aiboss88.com, "TokenSwift's technical principles"; tencent
+// article, parallel-verification figure; arxivlens "Technical
+// Contribution": a 3-ary tree).  For one KV head the R = G*T query rows
+// (node-major, then the group's heads) share every KV tile, so K/V are
+// streamed from HBM once per split.
+//
+// Products (orientations the tensor core runs at full rate):
+//   S_b  = Q_b K^T     query rows on M (128-lane blocks b), N = 128 positions.
+//                      Block 0's Q sits in TMEM; block 1's (rows 128..R-1)
+//                      in shared memory.
+//   O^T += V^T P^T     head dim on M, the R rows on N (padded to 16); V^T is
+//                      the TMA tile read MN-major, P^T is K-major.
+// An MMA below N = 128 costs about as much as one at N = 128, so a 128-wide
+// tile needs half the QK instructions of a 64-wide one.
+//
+// Query rows are spread over the TMEM lane quarters: block b's rows are cut
+// into four runs of rq_b = ceil(R_b / 4); run q sits in lanes 32q..32q+rq_b-1.
+// A warp can only reach its own lane quarter (its sub-partition), so this
+// gives every sub-partition the same share of the exponentials.  A softmax
+// warp owns a unit of 16 lanes of one block and reads it with the 16x256b
+// TMEM shape: four threads per row, 32 of the tile's 128 scores each, two
+// rows per thread (lanes t/4 and 8 + t/4 of the unit).
+//
+// CTA = (split, KV head), 16 warps, one CTA per SM:
+//   warp 0, 3   TMA producers of K and of V (two 64-column boxes of 128
+//               positions per tile, 128-byte swizzle).  The map's row extent
+//               is n_ctx + T, so rows past the tree tail arrive as zeros.
+//   warp 1      allocates TMEM; one lane issues the QK MMAs.  A block's S is
+//               released as soon as its softmax warps hold it in registers.
+//   warp 2      one lane issues the PV MMAs.
+//   warps 4-15  softmax, unit j = (warp - 4) / 4 of lane quarter warp % 4:
+//               scale to base 2, ancestor mask on tiles that reach the tree
+//               tail, exponentiate against a per-row reference max, write
+//               the bf16 P^T rows.  l sums the bf16-rounded P so the
+//               normalisation matches what PV used.  The reference max only
+//               moves when a tile exceeds it by more than 2^8; then the
+//               softmax warps rescale the O^T columns of the moved rows
+//               themselves (their lane quarters together cover all of D)
+//               before PV of the tile.  At the end they write O^T.
+// TMEM: O^T in [0, 192), Q_0 in [192, 256), S_0 in [256, 384), S_1 in
+// [384, 512).
+// Each split leaves an unnormalised partial (acc, m, l) for the combine
+// kernel, or normalises in place when it is the only split.
+//
+// Every wait is on an mbarrier and bounded (about a second): on expiry the
+// kernel records TS_ERR_TIMEOUT in the workspace status word, all roles
+// leave their loops, and TMEM is freed before the CTA exits.
+#include <math.h>
+
+#include "attn_common.cuh"
+#include "sm100.cuh"
+
+namespace ts {
+namespace {
+
+using namespace sm100;
+
+constexpr int kD = 128;
+constexpr int kTileN = 128;                  // KV positions per tile
+constexpr int kBlockM = 128;                 // query rows per QK block (TMEM lanes)
+constexpr int kBoxBytes = kTileN * 64 * 2;   // one 64-column box of a tile: 16 KB
+constexpr int kStageBytes = 2 * kBoxBytes;   // K (or V) of a tile
+constexpr int kThreads = 512;                // 16 warps
+constexpr int kMaxStages = 4;
+constexpr int kMaxRows = 192;
+constexpr int kQCol = 192;                   // Q of block 0: 128 bf16 = 64 columns per lane
+constexpr int kSCol = 256;                   // S_b: 128 columns from kSCol + 128 b
+constexpr int kTmemCols = 512;
+constexpr int kQ1Bytes = kBlockM * kD * 2;   // Q of block 1 in shared memory: 32 KB
+constexpr float kMoveLog2 = 8.f;             // reference max moves past this headroom
+constexpr size_t kSmemLimit = 232448;        // dynamic shared memory per CTA
+
+struct Bars {
+    uint64_t full_k[kMaxStages];
+    uint64_t empty_k[kMaxStages];
+    uint64_t full_v[kMaxStages];
+    uint64_t empty_v[kMaxStages];
+    uint64_t s_full[2];   // QK of block b landed in S_b
+    uint64_t s_free[2];   // block b's softmax warps hold S_b in registers
+    uint64_t decided;     // every softmax warp has published the tile's factors
+    uint64_t sm_done;     // every softmax warp wrote its P^T rows (O^T rescaled)
+    uint64_t pv_done;     // one commit per PV
+    uint64_t l_ready;     // every softmax warp published its final l
+    uint64_t o_final;     // committed once, after the last PV
+    uint64_t drain[2];    // each issuing thread's own MMAs, before TMEM is freed
+    uint32_t tmem_base;
+    uint32_t abort;
+    int32_t moved[2];     // tile index + 1 when that tile moved some row's max
+};
+
+struct Aux {
+    float factor[2][256];  // per-row O^T rescale factor of tile t in [t & 1]
+    float l[256];
+    Bars bar;
+};
+constexpr size_t kAuxBytes = (sizeof(Aux) + 1023) / 1024 * 1024;
+
+struct Layout {
+    int r_pad;  // rows rounded up to 16: N of the PV product
+    int stages_k, stages_v;
+    size_t q1_off, p_off, k_off, v_off, aux_off, smem_bytes;
+};
+
+__host__ __device__ inline Layout t128_layout(int rows)
+{
+    Layout L;
+    L.r_pad = (rows + 15) / 16 * 16;
+    L.q1_off = 0;
+    L.p_off = rows > kBlockM ? kQ1Bytes : 0;
+    // P^T: positions 0-63 then 64-127, each r_pad rows of 128 bytes
+    L.k_off = L.p_off + (size_t)L.r_pad * 256;
+    const size_t fixed = 1024 + L.k_off + kAuxBytes;
+    int stages = (int)((kSmemLimit - fixed) / kStageBytes);
+    stages = stages > 2 * kMaxStages ? 2 * kMaxStages : stages;
+    L.stages_v = 2;
+    L.stages_k = stages - 2 > kMaxStages ? kMaxStages : stages - 2;
+    L.v_off = L.k_off + (size_t)L.stages_k * kStageBytes;
+    L.aux_off = L.v_off + (size_t)L.stages_v * kStageBytes;
+    L.smem_bytes = 1024 + L.aux_off + kAuxBytes;
+    return L;
+}
+
+// P = 2^(x * scale - m) for the 32 scores a thread holds of row A
+// (registers r[4j], r[4j + 1], j = 0..15) and, when TWO, of row B
+// (r[4j + 2], r[4j + 3]), packed to bf16 pairs; adds the sums of the rounded
+// values (what the PV product will use) to lA and lB.  Both rows advance
+// together, so each score register is dead once its pair is packed.
+template <bool TWO>
+__device__ __forceinline__ void exp_pack_rows(const uint32_t (&r)[64], float scale, float neg_mA,
+                                              float neg_mB, uint32_t (&pA)[16],
+                                              uint32_t (&pB)[16], float &lA, float &lB)
+{
+    const uint64_t sc2 = pack2(scale, scale);
+    const uint64_t nA2 = pack2(neg_mA, neg_mA);
+    const uint64_t nB2 = pack2(neg_mB, neg_mB);
+    uint64_t sA = 0ull, sB = 0ull;
+#pragma unroll
+    for (int j = 0; j < 16; ++j) {
+#pragma unroll
+        for (int h = 0; h < (TWO ? 2 : 1); ++h) {
+            const uint64_t y = fma2(pack2(__uint_as_float(r[4 * j + 2 * h]),
+                                          __uint_as_float(r[4 * j + 2 * h + 1])),
+                                    sc2, h ? nB2 : nA2);
+            float y0, y1;
+            unpack2(y, y0, y1);
+            __nv_bfloat162 hv = __floats2bfloat162_rn(ex2(y0), ex2(y1));
+            const uint32_t hb = *reinterpret_cast<uint32_t *>(&hv);
+            const uint64_t e2 =
+                pack2(__uint_as_float(hb << 16), __uint_as_float(hb & 0xFFFF0000u));
+            if (h) {
+                pB[j] = hb;
+                sB = add2(sB, e2);
+            } else {
+                pA[j] = hb;
+                sA = add2(sA, e2);
+            }
+        }
+    }
+    float a0, a1;
+    unpack2(sA, a0, a1);
+    lA += a0 + a1;
+    if (TWO) {
+        unpack2(sB, a0, a1);
+        lB += a0 + a1;
+    }
+}
+
+// Row maximum of the 32 scores a thread holds of one row.
+__device__ __forceinline__ float row_max(const uint32_t (&r)[64], int e)
+{
+    float m[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+        m[u] = max3f(__uint_as_float(r[4 * u + e]), __uint_as_float(r[4 * u + e + 1]),
+                     __uint_as_float(r[4 * (u + 4) + e]));
+        m[u] = max3f(m[u], __uint_as_float(r[4 * (u + 4) + e + 1]),
+                     __uint_as_float(r[4 * (u + 8) + e]));
+        m[u] = max3f(m[u], __uint_as_float(r[4 * (u + 8) + e + 1]),
+                     __uint_as_float(r[4 * (u + 12) + e]));
+        m[u] = fmaxf(m[u], __uint_as_float(r[4 * (u + 12) + e + 1]));
+    }
+    return fmaxf(max3f(m[0], m[1], m[2]), m[3]);
+}
+
+// One row's 32 bf16 pairs into the K-major, 128-byte-swizzled P^T tile:
+// pair j covers positions 8j + c0, +1 (c0 = 2 * (lane % 4)).
+__device__ __forceinline__ void store_p_row(unsigned char *sP, int n, int r_pad, int lane,
+                                            const uint32_t (&pk)[16])
+{
+    unsigned char *row = sP + (n >> 3) * 1024 + (n & 7) * 128 + 4 * (lane & 3);
+#pragma unroll
+    for (int j = 0; j < 16; ++j)
+        *reinterpret_cast<uint32_t *>(row + (j >> 3) * (r_pad * 128) +
+                                      (((j & 7) ^ (n & 7)) << 4)) = pk[j];
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+attn_t128_kernel(const __grid_constant__ CUtensorMap tmap_k,
+                 const __grid_constant__ CUtensorMap tmap_v, AttnArgs a, TreeMasks masks,
+                 int tiles_per_split, int n_split)
+{
+    const int G = a.n_heads_q / a.n_heads_kv;
+    const int R = G * a.n_tree;
+    const int NB = R > kBlockM ? 2 : 1;
+    const int R0 = R < kBlockM ? R : kBlockM, R1 = R - R0;
+    const int rq0 = (R0 + 3) / 4, rq1 = (R1 + 3) / 4;  // rows per lane quarter
+    const int u0 = (rq0 + 15) / 16, u1 = (rq1 + 15) / 16;
+    const int U = u0 + u1;  // softmax warps per lane quarter (at most 3)
+    const Layout lay = t128_layout(R);
+    const int SK = lay.stages_k, SV = lay.stages_v, r_pad = lay.r_pad;
+
+    extern __shared__ unsigned char smem_raw[];
+    unsigned char *base = reinterpret_cast<unsigned char *>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    unsigned char *sQ1 = base + lay.q1_off;
+    unsigned char *sP = base + lay.p_off;
+    unsigned char *sK = base + lay.k_off;
+    unsigned char *sV = base + lay.v_off;
+    Aux *aux = reinterpret_cast<Aux *>(base + lay.aux_off);
+    Bars *bar = &aux->bar;
+    WorkspaceHeader *hdr = reinterpret_cast<WorkspaceHeader *>(a.workspace);
+    volatile uint32_t *abort = &bar->abort;
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int split = blockIdx.x, g = blockIdx.y;
+    const int total = a.n_ctx + a.n_tree;
+    const int n_tiles_all = (total + kTileN - 1) / kTileN;
+    const int t_begin = split * tiles_per_split;
+    const int n_tiles = min(t_begin + tiles_per_split, n_tiles_all) - t_begin;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < SK; ++s) {
+            mbar_init(smem_addr(&bar->full_k[s]), 1);
+            mbar_init(smem_addr(&bar->empty_k[s]), 1);
+        }
+        for (int s = 0; s < SV; ++s) {
+            mbar_init(smem_addr(&bar->full_v[s]), 1);
+            mbar_init(smem_addr(&bar->empty_v[s]), 1);
+        }
+        mbar_init(smem_addr(&bar->s_full[0]), 1);
+        mbar_init(smem_addr(&bar->s_full[1]), 1);
+        mbar_init(smem_addr(&bar->s_free[0]), 4 * u0);
+        mbar_init(smem_addr(&bar->s_free[1]), u1 > 0 ? 4 * u1 : 1);
+        mbar_init(smem_addr(&bar->decided), 4 * U);
+        mbar_init(smem_addr(&bar->sm_done), 4 * U);
+        mbar_init(smem_addr(&bar->pv_done), 1);
+        mbar_init(smem_addr(&bar->l_ready), 4 * U);
+        mbar_init(smem_addr(&bar->o_final), 1);
+        mbar_init(smem_addr(&bar->drain[0]), 1);
+        mbar_init(smem_addr(&bar->drain[1]), 1);
+        bar->abort = 0u;
+        bar->moved[0] = bar->moved[1] = 0;
+        fence_mbar_init();
+    }
+    if (warp == 1) {
+        tmem_alloc(smem_addr(&bar->tmem_base), kTmemCols);
+        tmem_relinquish();
+    }
+    if (warp == 0 && lane == 0) {
+        prefetch_tmap(&tmap_k);
+        prefetch_tmap(&tmap_v);
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = bar->tmem_base;
+
+    // Query rows of this KV head into place: row n = node * G + (head - g*G).
+    // Block 0 (rows 0..R0-1) into TMEM lanes (warps 4-7, 32x32b stores);
+    // block 1 (rows 128..R-1) into the shared-memory A tile (warps 8-11).
+    auto q_row = [&](int n) {
+        return reinterpret_cast<const uint4 *>(
+            a.q + ((int64_t)(n / G) * a.n_heads_q + g * G + n % G) * kD);
+    };
+    if (warp >= 4 && warp < 8) {
+        const int q = warp & 3;
+        const int n = q * rq0 + lane;
+        const bool valid = lane < rq0 && n < R0;
+        uint32_t qv[64];
+        if (valid) {
+            const uint4 *src = q_row(n);
+#pragma unroll
+            for (int c = 0; c < 16; ++c) {
+                const uint4 u = src[c];
+                qv[4 * c] = u.x;
+                qv[4 * c + 1] = u.y;
+                qv[4 * c + 2] = u.z;
+                qv[4 * c + 3] = u.w;
+            }
+        } else {
+#pragma unroll
+            for (int c = 0; c < 64; ++c)
+                qv[c] = 0u;
+        }
+        const uint32_t qa = tmem + ((uint32_t)(q * 32) << 16) + kQCol;
+        uint32_t (&q0)[32] = *reinterpret_cast<uint32_t (*)[32]>(&qv[0]);
+        uint32_t (&q1)[32] = *reinterpret_cast<uint32_t (*)[32]>(&qv[32]);
+        tmem_st32(qa, q0);
+        tmem_st32(qa + 32, q1);
+        tmem_st_wait();
+    } else if (NB == 2 && warp >= 8 && warp < 12) {
+        const int q = warp & 3;
+        const int m = q * 32 + lane;  // A-tile row = TMEM lane of S_1
+        const int n = kBlockM + q * rq1 + lane;
+        const bool valid = lane < rq1 && n < R;
+        const uint4 *src = valid ? q_row(n) : nullptr;
+#pragma unroll
+        for (int c = 0; c < 16; ++c) {
+            const uint4 u = valid ? src[c] : make_uint4(0u, 0u, 0u, 0u);
+            *reinterpret_cast<uint4 *>(sQ1 + (c >> 3) * kBoxBytes + (m >> 3) * 1024 +
+                                       (m & 7) * 128 + (((c & 7) ^ (m & 7)) << 4)) = u;
+        }
+        fence_proxy_async_smem();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+
+    if (warp == 0 || warp == 3) {
+        // ----------------------------------------- TMA producers (K, V)
+        if (lane == 0) {
+            const bool is_k = warp == 0;
+            const int ns = is_k ? SK : SV;
+            uint64_t *full = is_k ? bar->full_k : bar->full_v;
+            uint64_t *empty = is_k ? bar->empty_k : bar->empty_v;
+            unsigned char *ring = is_k ? sK : sV;
+            const void *tmap = is_k ? static_cast<const void *>(&tmap_k)
+                                    : static_cast<const void *>(&tmap_v);
+            int issued = 0;
+            for (int t = 0; t < n_tiles; ++t) {
+                const int s = t % ns;
+                if (t >= ns &&
+                    !wait_bounded(smem_addr(&empty[s]), ((t / ns) & 1) ^ 1, abort, hdr))
+                    break;
+                const uint32_t fb = smem_addr(&full[s]);
+                mbar_arrive_expect_tx(fb, kStageBytes);
+                const uint32_t dst = smem_addr(ring + s * kStageBytes);
+                const int pos0 = (t_begin + t) * kTileN;
+                tma_load_3d(dst, tmap, 0, pos0, g, fb);
+                tma_load_3d(dst + kBoxBytes, tmap, 64, pos0, g, fb);
+                issued = t + 1;
+            }
+            if (*abort) {
+                // let our own copies land before the CTA exits
+                for (int t = max(0, issued - ns); t < issued; ++t)
+                    wait_drain(smem_addr(&full[t % ns]), (t / ns) & 1);
+            }
+        }
+    } else if (warp == 1 || warp == 2) {
+        // --------------------------------------------- MMA issuers: QK, PV
+        if (lane == 0) {
+            constexpr uint64_t kStageStep = kStageBytes >> 4;
+            if (warp == 1) {
+                const uint32_t idesc = idesc_bf16(kBlockM, kTileN, 0, 0);
+                const uint64_t kd0 = sdesc_sw128(smem_addr(sK), 16, 1024);
+                const uint64_t qd0 = sdesc_sw128(smem_addr(sQ1), 16, 1024);
+                for (int t = 0; t < n_tiles; ++t) {
+                    const int s = t % SK;
+                    if (!wait_bounded(smem_addr(&bar->full_k[s]), (t / SK) & 1, abort, hdr))
+                        break;
+                    const uint64_t kd = kd0 + (uint64_t)s * kStageStep;
+                    bool ok = true;
+                    for (int b = 0; b < NB; ++b) {
+                        // S_b is reused: its softmax warps must hold S_b(t-1)
+                        if (t > 0 &&
+                            !wait_bounded(smem_addr(&bar->s_free[b]), (t - 1) & 1, abort, hdr)) {
+                            ok = false;
+                            break;
+                        }
+                        tc_fence_after();
+                        const uint32_t d_col = tmem + kSCol + 128 * b;
+                        if (b == 0) {
+                            mma_ts_c<0>(d_col, tmem + kQCol, kd, idesc);
+#pragma unroll
+                            for (int kk = 1; kk < kD / 16; ++kk)
+                                mma_ts_c<1>(d_col, tmem + kQCol + kk * 8,
+                                            kd + (((kk >> 2) * kBoxBytes + (kk & 3) * 32) >> 4),
+                                            idesc);
+                        } else {
+                            mma_ss_c<0>(d_col, qd0, kd, idesc);
+#pragma unroll
+                            for (int kk = 1; kk < kD / 16; ++kk) {
+                                const uint64_t off = ((kk >> 2) * kBoxBytes + (kk & 3) * 32) >> 4;
+                                mma_ss_c<1>(d_col, qd0 + off, kd + off, idesc);
+                            }
+                        }
+                        mma_commit(smem_addr(&bar->s_full[b]));
+                    }
+                    if (!ok)
+                        break;
+                    mma_commit(smem_addr(&bar->empty_k[s]));
+                }
+            } else {
+                const uint32_t idesc = idesc_bf16(kD, r_pad, 1, 0);
+                const uint64_t vd0 = sdesc_sw128(smem_addr(sV), kBoxBytes, 1024);
+                const uint64_t pd0 = sdesc_sw128(smem_addr(sP), 16, 1024);
+                const uint32_t p_half = (uint32_t)r_pad * 128;
+                for (int t = 0; t < n_tiles; ++t) {
+                    const int s = t % SV;
+                    if (!wait_bounded(smem_addr(&bar->full_v[s]), (t / SV) & 1, abort, hdr) ||
+                        !wait_bounded(smem_addr(&bar->sm_done), t & 1, abort, hdr))
+                        break;
+                    tc_fence_after();
+                    const uint64_t vd = vd0 + (uint64_t)s * kStageStep;
+                    if (t == 0)
+                        mma_ss_c<0>(tmem, vd, pd0, idesc);
+                    else
+                        mma_ss_c<1>(tmem, vd, pd0, idesc);
+#pragma unroll
+                    for (int kk = 1; kk < kTileN / 16; ++kk)
+                        mma_ss_c<1>(tmem, vd + ((kk * 2048) >> 4),
+                                    pd0 + (((kk >> 2) * p_half + (kk & 3) * 32) >> 4), idesc);
+                    mma_commit(smem_addr(&bar->pv_done));
+                    if (t == n_tiles - 1)
+                        mma_commit(smem_addr(&bar->o_final));
+                    mma_commit(smem_addr(&bar->empty_v[s]));
+                }
+            }
+            // every MMA this thread issued has finished before TMEM is released
+            const int dn = warp - 1;
+            mma_commit(smem_addr(&bar->drain[dn]));
+            wait_drain(smem_addr(&bar->drain[dn]), 0);
+        }
+    } else if (warp >= 4 && (warp - 4) / 4 < U) {
+        // ---------------------------------------------------------- softmax
+        const int q = warp & 3, j = (warp - 4) >> 2;
+        const int b = j < u0 ? 0 : 1;
+        const int lb = 16 * (b == 0 ? j : j - u0);  // unit's first lane in the quarter
+        const int Rb = b == 0 ? R0 : R1, rqb = b == 0 ? rq0 : rq1;
+        const int iA = lb + (lane >> 2), iB = iA + 8;
+        const bool vA = iA < rqb && q * rqb + iA < Rb;
+        const bool vB = iB < rqb && q * rqb + iB < Rb;
+        const bool hasA = __any_sync(0xffffffffu, vA), hasB = __any_sync(0xffffffffu, vB);
+        const int nA = kBlockM * b + q * rqb + iA, nB = nA + 8;
+        const uint32_t s_addr = tmem + ((uint32_t)(32 * q + lb) << 16) + kSCol + 128 * b;
+        const uint32_t o_lane = (uint32_t)(32 * q) << 16;
+        const int c0 = 2 * (lane & 3);
+        volatile int32_t *moved = bar->moved;
+        float mA = -INFINITY, mB = -INFINITY, lA = 0.f, lB = 0.f;
+        bool ok = true;
+        for (int t = 0; t < n_tiles; ++t) {
+            const int buf = t & 1;
+            if (!warp_wait_bounded(smem_addr(&bar->s_full[b]), t & 1, abort, hdr)) {
+                ok = false;
+                break;
+            }
+            tc_fence_after();
+            uint32_t r[64];
+            tmem_ld16x256_x16(s_addr, r);
+            // S is in registers: QK of the next tile may overwrite it
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0)
+                mbar_arrive(smem_addr(&bar->s_free[b]));
+            // raw scores; the scale (> 0) is applied inside the exponent
+            const int pos0 = (t_begin + t) * kTileN;
+            if (pos0 + kTileN > a.n_ctx) {
+                // visibility of this thread's 32 positions (entry k = 2 jj + e
+                // is position pos0 + 8 jj + c0 + e) for its two rows
+                const unsigned long long ancA = masks.anc[vA ? nA / G : 0];
+                const unsigned long long ancB = masks.anc[vB ? nB / G : 0];
+                uint32_t visA = 0u, visB = 0u;
+#pragma unroll 1
+                for (int k = 0; k < 32; ++k) {
+                    const int pos = pos0 + 8 * (k >> 1) + c0 + (k & 1);
+                    const int tp = pos - a.n_ctx;
+                    const bool in = pos < total;
+                    visA |= (uint32_t)(in && (tp < 0 || ((ancA >> tp) & 1ull))) << k;
+                    visB |= (uint32_t)(in && (tp < 0 || ((ancB >> tp) & 1ull))) << k;
+                }
+#pragma unroll
+                for (int k = 0; k < 32; ++k) {
+                    if (!((visA >> k) & 1u))
+                        r[4 * (k >> 1) + (k & 1)] = __float_as_uint(-INFINITY);
+                    if (!((visB >> k) & 1u))
+                        r[4 * (k >> 1) + 2 + (k & 1)] = __float_as_uint(-INFINITY);
+                }
+            }
+            float xA = row_max(r, 0), xB = row_max(r, 2);
+            xA = fmaxf(xA, __shfl_xor_sync(0xffffffffu, xA, 1));
+            xB = fmaxf(xB, __shfl_xor_sync(0xffffffffu, xB, 1));
+            xA = fmaxf(xA, __shfl_xor_sync(0xffffffffu, xA, 2)) * a.scale_log2;
+            xB = fmaxf(xB, __shfl_xor_sync(0xffffffffu, xB, 2)) * a.scale_log2;
+            // move a row's reference max only when this tile exceeds it by > 2^8
+            float fA = 1.f, fB = 1.f;
+            const bool needA = xA > mA + kMoveLog2, needB = xB > mB + kMoveLog2;
+            if (needA) {
+                fA = (mA == -INFINITY) ? 0.f : ex2(mA - xA);
+                mA = xA;
+                lA *= fA;
+            }
+            if (needB) {
+                fB = (mB == -INFINITY) ? 0.f : ex2(mB - xB);
+                mB = xB;
+                lB *= fB;
+            }
+            if ((lane & 3) == 0) {
+                if (vA)
+                    aux->factor[buf][nA] = fA;
+                if (vB)
+                    aux->factor[buf][nB] = fB;
+            }
+            if (__any_sync(0xffffffffu, (needA && vA) || (needB && vB)) && lane == 0)
+                moved[buf] = t + 1;
+            __syncwarp();
+            if (lane == 0)
+                mbar_arrive(smem_addr(&bar->decided));
+
+            uint32_t pA[16], pB[16];
+            {
+                const float nmA = mA == -INFINITY ? 0.f : -mA;
+                const float nmB = mB == -INFINITY ? 0.f : -mB;
+                if (hasB)
+                    exp_pack_rows<true>(r, a.scale_log2, nmA, nmB, pA, pB, lA, lB);
+                else if (hasA)
+                    exp_pack_rows<false>(r, a.scale_log2, nmA, nmB, pA, pB, lA, lB);
+            }
+
+            // every warp's factors are in place; P^T and O^T are free once
+            // PV(t-1) is done.  This warp saw PV(t-2) done before writing
+            // P^T(t-1), and PV(t) waits for this warp, so pv_done has one
+            // open phase here.
+            if (!warp_wait_bounded(smem_addr(&bar->decided), t & 1, abort, hdr) ||
+                (t > 0 &&
+                 !warp_wait_bounded(smem_addr(&bar->pv_done), (t - 1) & 1, abort, hdr))) {
+                ok = false;
+                break;
+            }
+            if (hasA && vA)
+                store_p_row(sP, nA, r_pad, lane, pA);
+            if (hasB && vB)
+                store_p_row(sP, nB, r_pad, lane, pB);
+            if (t > 0 && moved[buf] == t + 1) {
+                // some row's max moved: scale this quarter's D lanes of O^T,
+                // 32-column chunks j, j + U, ...
+                tc_fence_after();
+                for (int c = 32 * j; c < r_pad; c += 32 * U) {
+#pragma unroll
+                    for (int h = 0; h < 32; h += 16) {
+                        uint32_t o[16];
+                        tmem_ld16(tmem + o_lane + c + h, o);
+#pragma unroll
+                        for (int jj = 0; jj < 16; ++jj)
+                            o[jj] = __float_as_uint(__uint_as_float(o[jj]) *
+                                                    aux->factor[buf][c + h + jj]);
+                        tmem_st16(tmem + o_lane + c + h, o);
+                    }
+                }
+                tmem_st_wait();
+            }
+            fence_proxy_async_smem();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0)
+                mbar_arrive(smem_addr(&bar->sm_done));
+        }
+        // ---- final l of each row (four threads' partial sums), then O^T out
+        lA += __shfl_xor_sync(0xffffffffu, lA, 1);
+        lB += __shfl_xor_sync(0xffffffffu, lB, 1);
+        lA += __shfl_xor_sync(0xffffffffu, lA, 2);
+        lB += __shfl_xor_sync(0xffffffffu, lB, 2);
+        const int rows_all = a.n_tree * a.n_heads_q;
+        float *ws_o =
+            reinterpret_cast<float *>(reinterpret_cast<char *>(a.workspace) + kHeaderBytes);
+        float *ws_ml = ws_o + (size_t)n_split * rows_all * kD;
+        auto orow_of = [&](int n) { return (n / G) * a.n_heads_q + g * G + n % G; };
+        if (ok && (lane & 3) == 0) {
+            if (vA) {
+                aux->l[nA] = lA;
+                if (n_split > 1)
+                    *reinterpret_cast<float2 *>(ws_ml + ((size_t)split * rows_all + orow_of(nA)) *
+                                                            2) = make_float2(mA, lA);
+            }
+            if (vB) {
+                aux->l[nB] = lB;
+                if (n_split > 1)
+                    *reinterpret_cast<float2 *>(ws_ml + ((size_t)split * rows_all + orow_of(nB)) *
+                                                            2) = make_float2(mB, lB);
+            }
+        }
+        __syncwarp();
+        if (ok && lane == 0)
+            mbar_arrive(smem_addr(&bar->l_ready));
+        if (ok && warp_wait_bounded(smem_addr(&bar->l_ready), 0, abort, hdr) &&
+            warp_wait_bounded(smem_addr(&bar->o_final), 0, abort, hdr)) {
+            tc_fence_after();
+            const int d = 32 * q + lane;
+            for (int c = 32 * j; c < r_pad; c += 32 * U) {
+                uint32_t o[32];
+                tmem_ld32(tmem + o_lane + c, o);
+#pragma unroll
+                for (int jj = 0; jj < 32; ++jj) {
+                    const int n = c + jj;
+                    if (n < R) {
+                        const float v = __uint_as_float(o[jj]);
+                        if (n_split == 1)
+                            a.out[(size_t)orow_of(n) * kD + d] = v / aux->l[n];
+                        else
+                            ws_o[((size_t)split * rows_all + orow_of(n)) * kD + d] = v;
+                    }
+                }
+            }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem, kTmemCols);
+    }
+}
+
+}  // namespace
+
+bool attn_t128_eligible(int n_heads_q, int n_heads_kv, int head_dim, int n_ctx, int n_tree)
+{
+    const int rows = (n_heads_q / n_heads_kv) * n_tree;
+    return head_dim == kD && rows <= kMaxRows && n_ctx >= kTcMinContext;
+}
+
+AttnPlan attn_t128_plan(int n_heads_q, int n_heads_kv, int n_ctx, int n_tree, int num_sms)
+{
+    AttnPlan p;
+    const int n_tiles = (n_ctx + n_tree + kTileN - 1) / kTileN;
+    int want = num_sms / n_heads_kv;
+    want = want < 1 ? 1 : (want > n_tiles ? n_tiles : want);
+    p.tiles_per_split = (n_tiles + want - 1) / want;
+    p.n_split = (n_tiles + p.tiles_per_split - 1) / p.tiles_per_split;
+    (void)n_heads_q;
+    return p;
+}
+
+cudaError_t attn_t128_launch(const AttnArgs &a, const TreeMasks &masks, int num_sms,
+                             cudaStream_t stream)
+{
+    const AttnPlan p = attn_t128_plan(a.n_heads_q, a.n_heads_kv, a.n_ctx, a.n_tree, num_sms);
+    CUtensorMap mk, mv;
+    const int rows = a.n_ctx + a.n_tree;
+    if (!encode_kv_map(&mk, a.k, rows, a.kv_cap, a.n_heads_kv, kTileN) ||
+        !encode_kv_map(&mv, a.v, rows, a.kv_cap, a.n_heads_kv, kTileN))
+        return cudaErrorInvalidValue;
+    const Layout lay = t128_layout((a.n_heads_q / a.n_heads_kv) * a.n_tree);
+    static const cudaError_t attr = cudaFuncSetAttribute(
+        attn_t128_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemLimit);
+    if (attr != cudaSuccess)
+        return attr;
+    attn_t128_kernel<<<dim3(p.n_split, a.n_heads_kv), kThreads, lay.smem_bytes, stream>>>(
+        mk, mv, a, masks, p.tiles_per_split, p.n_split);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess)
+        return e;
+    count_launches(1);
+    if (p.n_split == 1)
+        return cudaSuccess;
+    return attn_combine_launch(a, p.n_split, stream);
+}
+
+}  // namespace ts

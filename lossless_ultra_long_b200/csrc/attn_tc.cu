@@ -571,48 +571,14 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_constant
 }
 
 // ------------------------------------------------------------------- host
-PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder()
-{
-    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-    static std::once_flag once;
-    std::call_once(once, [] {
-        cudaDriverEntryPointQueryResult q;
-        void *p = nullptr;
-        if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000,
-                                             cudaEnableDefault, &q) == cudaSuccess &&
-            q == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
-        else
-            cudaGetLastError();
-    });
-    return fn;
-}
-
-// [Hkv, kv_cap, D] bf16 viewed as 3-D (d, position, head); positions past
-// `rows` read as zeros.
-bool encode_kv_map(CUtensorMap *m, const void *ptr, int rows, int64_t kv_cap, int n_heads_kv)
-{
-    auto enc = tensor_map_encoder();
-    if (!enc)
-        return false;
-    const cuuint64_t dims[3] = {(cuuint64_t)kD, (cuuint64_t)rows, (cuuint64_t)n_heads_kv};
-    const cuuint64_t strides[2] = {(cuuint64_t)kD * 2, (cuuint64_t)kv_cap * kD * 2};
-    const cuuint32_t box[3] = {64, (cuuint32_t)kTileN, 1};
-    const cuuint32_t estr[3] = {1, 1, 1};
-    return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(ptr), dims, strides, box,
-               estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-               CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
 template <int NB>
 cudaError_t launch_nb(const AttnArgs &a, const TreeMasks &masks, const AttnPlan &p,
                       cudaStream_t stream)
 {
     CUtensorMap mk, mv;
     const int rows = a.n_ctx + a.n_tree;
-    if (!encode_kv_map(&mk, a.k, rows, a.kv_cap, a.n_heads_kv) ||
-        !encode_kv_map(&mv, a.v, rows, a.kv_cap, a.n_heads_kv))
+    if (!encode_kv_map(&mk, a.k, rows, a.kv_cap, a.n_heads_kv, kTileN) ||
+        !encode_kv_map(&mv, a.v, rows, a.kv_cap, a.n_heads_kv, kTileN))
         return cudaErrorInvalidValue;
     const TcLayout lay = tc_layout(NB, (a.n_heads_q / a.n_heads_kv) * a.n_tree);
     const size_t smem = lay.smem_bytes;
@@ -632,6 +598,39 @@ cudaError_t launch_nb(const AttnArgs &a, const TreeMasks &masks, const AttnPlan 
 }
 
 }  // namespace
+
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder()
+{
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        cudaDriverEntryPointQueryResult q;
+        void *p = nullptr;
+        if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000,
+                                             cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+        else
+            cudaGetLastError();
+    });
+    return fn;
+}
+
+bool encode_kv_map(CUtensorMap *m, const void *ptr, int rows, int64_t kv_cap, int n_heads_kv,
+                   int box_rows)
+{
+    auto enc = tensor_map_encoder();
+    if (!enc)
+        return false;
+    const cuuint64_t dims[3] = {(cuuint64_t)kD, (cuuint64_t)rows, (cuuint64_t)n_heads_kv};
+    const cuuint64_t strides[2] = {(cuuint64_t)kD * 2, (cuuint64_t)kv_cap * kD * 2};
+    const cuuint32_t box[3] = {64, (cuuint32_t)box_rows, 1};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(ptr), dims, strides, box,
+               estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
 
 bool attn_tc_eligible(int n_heads_q, int n_heads_kv, int head_dim, int n_ctx, int n_tree)
 {

@@ -78,10 +78,14 @@ def test_attn_max_tree_and_irregular(oracle_mod):
 
 @pytest.mark.parametrize("n_ctx", [2047, 2048, 2049, 2111, 9000])
 @pytest.mark.parametrize("hq,hkv,t", [(8, 2, 13), (32, 8, 40), (40, 8, 40), (32, 32, 40),
-                                      (64, 8, 32), (16, 1, 16), (32, 8, 4), (32, 8, 1)])
+                                      (64, 8, 32), (16, 1, 16), (32, 8, 4), (32, 8, 1),
+                                      (32, 8, 32), (24, 8, 43), (32, 8, 36), (32, 8, 44),
+                                      (32, 8, 48), (20, 4, 20), (8, 8, 61)])
 def test_attn_dispatch_threshold_and_row_blocks(oracle_mod, n_ctx, hq, hkv, t):
-    """Both sides of the kernel switch at 2048 positions, one and two 128-row
-    blocks (up to the 256-row limit), ragged tails."""
+    """Both sides of the kernel switch at 2048 positions; G*T query rows per
+    KV head from 1 to 256: one and two 128-row blocks, uneven runs per lane
+    quarter, the 192-row limit of the 128-position-tile kernel and the
+    224-row limit of the 64-position-tile one; ragged tails."""
     w = I.Workload("tc", hq, hkv, 128, n_ctx, t, seed=n_ctx * 3 + hq + t)
     _attn_sampled(oracle_mod, w, count=24)
 
@@ -129,6 +133,28 @@ def test_attn_mha7b_100k(oracle_mod):
 @pytest.mark.parametrize("t", I.SWEEP_TREE)
 def test_attn_14b_sweep(oracle_mod, n_ctx, t):
     _attn_sampled(oracle_mod, I.sweep14b(n_ctx, t), count=8)
+
+
+@pytest.mark.parametrize("hq,hkv,t", [(128, 32, 40), (32, 32, 40), (160, 32, 40)])
+def test_attn_rising_scores_move_the_reference_max(oracle_mod, hq, hkv, t):
+    """Scores rise in plateaus: every query row has 4.0 in dimension 0 and
+    every key 16 * (position // 512) there, so each 512-position block sits
+    about 2^8.2 above the one before (softmax scale 1/sqrt(128)) while the
+    weight inside a block stays spread over its positions.  Each row's
+    reference max therefore moves every block and the accumulated output is
+    rescaled again and again; sampled rows against the oracle."""
+    w = I.Workload("rise", hq, hkv, 128, 12000, t, seed=40 + hq + t)
+    q = I.gen_q(w)
+    k, v = I.gen_kv(w)
+    q[:, :, 0] = I.f32_to_bf16_bits(np.float32(4.0))
+    pos = np.arange(k.shape[1])
+    k[:, :, 0] = I.f32_to_bf16_bits(16.0 * (pos // 512).astype(np.float32))[None, :]
+    got = run_attn(q, k, v, w.n_ctx, w.parent())
+    nodes, heads = sample_rows(w.n_tree, w.n_heads_q, 24, w.seed)
+    want = oracle_mod.tree_verify_attn_rows(q, k, v, w.n_ctx, w.parent(), nodes, heads)
+    err = np.abs(got[nodes, heads] - want).max()
+    assert err <= ATTN_TOL, f"{w.name}: max abs err {err}"
+    assert np.isfinite(got).all()
 
 
 def test_attn_draft_pass_over_partial_cache(oracle_mod):
