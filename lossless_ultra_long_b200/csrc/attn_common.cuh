@@ -50,6 +50,7 @@ cudaError_t attn_tc_launch(const AttnArgs &a, const TreeMasks &masks, int num_sm
 // 192 query rows per KV head.
 bool attn_t128_eligible(int n_heads_q, int n_heads_kv, int head_dim, int n_ctx, int n_tree);
 AttnPlan attn_t128_plan(int n_heads_q, int n_heads_kv, int n_ctx, int n_tree, int num_sms);
+size_t attn_t128_workspace_bytes(int n_heads_q, int n_heads_kv, int n_ctx, int n_tree, int num_sms);
 cudaError_t attn_t128_launch(const AttnArgs &a, const TreeMasks &masks, int num_sms,
                              cudaStream_t stream);
 

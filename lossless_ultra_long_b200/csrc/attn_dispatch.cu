@@ -20,8 +20,10 @@ size_t attn_workspace_bytes(int n_heads_q, int n_heads_kv, int head_dim, int n_c
                           align_up(attn_partial_bytes(p.n_split, n_heads_q, head_dim, n_tree), 256);
         bytes = tc > bytes ? tc : bytes;
     };
-    if (attn_t128_eligible(n_heads_q, n_heads_kv, head_dim, n_ctx, n_tree))
-        take(attn_t128_plan(n_heads_q, n_heads_kv, n_ctx, n_tree, num_sms));
+    if (attn_t128_eligible(n_heads_q, n_heads_kv, head_dim, n_ctx, n_tree)) {
+        const size_t t128 = attn_t128_workspace_bytes(n_heads_q, n_heads_kv, n_ctx, n_tree, num_sms);
+        bytes = t128 > bytes ? t128 : bytes;
+    }
     if (attn_tc_eligible(n_heads_q, n_heads_kv, head_dim, n_ctx, n_tree))
         take(attn_tc_plan(n_heads_q, n_heads_kv, n_ctx, n_tree, num_sms));
     return bytes;

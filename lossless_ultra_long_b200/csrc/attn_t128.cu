@@ -38,15 +38,23 @@
 //               scale to base 2, ancestor mask on tiles that reach the tree
 //               tail, exponentiate against a per-row reference max, write
 //               the bf16 P^T rows.  l sums the bf16-rounded P so the
-//               normalisation matches what PV used.  The reference max only
-//               moves when a tile exceeds it by more than 2^8; then the
-//               softmax warps rescale the O^T columns of the moved rows
-//               themselves (their lane quarters together cover all of D)
-//               before PV of the tile.  At the end they write O^T.
+//               normalisation matches what PV used.  At the end they write
+//               O^T (their lane quarters together cover all of D).
 // TMEM: O^T in [0, 192), Q_0 in [192, 256), S_0 in [256, 384), S_1 in
 // [384, 512).
-// Each split leaves an unnormalised partial (acc, m, l) for the combine
-// kernel, or normalises in place when it is the only split.
+//
+// The reference max of a row is fixed at the first tile where the row sees
+// anything, and never moves: fp32 accumulation has room for weights up to
+// 2^64 (times the head dim, the values and the split length), so nothing
+// has to be rescaled while a row's scores stay within 64 (base-2) above
+// its first tile's maximum -- which takes a score jump of about 44 nats
+// inside one split.  This keeps the softmax warps free of any per-tile
+// agreement with each other.  A split in which some row does exceed the
+// headroom raises a flag; the combine kernel then recomputes that split's
+// partial for the affected head exactly (fp32, online softmax on CUDA
+// cores) instead of reading it.
+// Each split leaves an unnormalised partial (acc, m, l) and its flag; the
+// combine kernel always runs.
 //
 // Every wait is on an mbarrier and bounded (about a second): on expiry the
 // kernel records TS_ERR_TIMEOUT in the workspace status word, all roles
@@ -73,7 +81,7 @@ constexpr int kQCol = 192;                   // Q of block 0: 128 bf16 = 64 colu
 constexpr int kSCol = 256;                   // S_b: 128 columns from kSCol + 128 b
 constexpr int kTmemCols = 512;
 constexpr int kQ1Bytes = kBlockM * kD * 2;   // Q of block 1 in shared memory: 32 KB
-constexpr float kMoveLog2 = 8.f;             // reference max moves past this headroom
+constexpr float kHeadroomLog2 = 64.f;        // weights stay below 2^64 of the reference
 constexpr size_t kSmemLimit = 232448;        // dynamic shared memory per CTA
 
 struct Bars {
@@ -83,20 +91,16 @@ struct Bars {
     uint64_t empty_v[kMaxStages];
     uint64_t s_full[2];   // QK of block b landed in S_b
     uint64_t s_free[2];   // block b's softmax warps hold S_b in registers
-    uint64_t decided;     // every softmax warp has published the tile's factors
-    uint64_t sm_done;     // every softmax warp wrote its P^T rows (O^T rescaled)
+    uint64_t sm_done;     // every softmax warp wrote its P^T rows
     uint64_t pv_done;     // one commit per PV
-    uint64_t l_ready;     // every softmax warp published its final l
     uint64_t o_final;     // committed once, after the last PV
     uint64_t drain[2];    // each issuing thread's own MMAs, before TMEM is freed
     uint32_t tmem_base;
     uint32_t abort;
-    int32_t moved[2];     // tile index + 1 when that tile moved some row's max
+    int32_t overflow;     // some row exceeded its reference max by the headroom
 };
 
 struct Aux {
-    float factor[2][256];  // per-row O^T rescale factor of tile t in [t & 1]
-    float l[256];
     Bars bar;
 };
 constexpr size_t kAuxBytes = (sizeof(Aux) + 1023) / 1024 * 1024;
@@ -203,7 +207,7 @@ __device__ __forceinline__ void store_p_row(unsigned char *sP, int n, int r_pad,
 __global__ void __launch_bounds__(kThreads, 1)
 attn_t128_kernel(const __grid_constant__ CUtensorMap tmap_k,
                  const __grid_constant__ CUtensorMap tmap_v, AttnArgs a, TreeMasks masks,
-                 int tiles_per_split, int n_split)
+                 int tiles_per_split, int n_split, int32_t *flags)
 {
     const int G = a.n_heads_q / a.n_heads_kv;
     const int R = G * a.n_tree;
@@ -247,15 +251,13 @@ attn_t128_kernel(const __grid_constant__ CUtensorMap tmap_k,
         mbar_init(smem_addr(&bar->s_full[1]), 1);
         mbar_init(smem_addr(&bar->s_free[0]), 4 * u0);
         mbar_init(smem_addr(&bar->s_free[1]), u1 > 0 ? 4 * u1 : 1);
-        mbar_init(smem_addr(&bar->decided), 4 * U);
         mbar_init(smem_addr(&bar->sm_done), 4 * U);
         mbar_init(smem_addr(&bar->pv_done), 1);
-        mbar_init(smem_addr(&bar->l_ready), 4 * U);
         mbar_init(smem_addr(&bar->o_final), 1);
         mbar_init(smem_addr(&bar->drain[0]), 1);
         mbar_init(smem_addr(&bar->drain[1]), 1);
         bar->abort = 0u;
-        bar->moved[0] = bar->moved[1] = 0;
+        bar->overflow = 0;
         fence_mbar_init();
     }
     if (warp == 1) {
@@ -442,11 +444,9 @@ attn_t128_kernel(const __grid_constant__ CUtensorMap tmap_k,
         const uint32_t s_addr = tmem + ((uint32_t)(32 * q + lb) << 16) + kSCol + 128 * b;
         const uint32_t o_lane = (uint32_t)(32 * q) << 16;
         const int c0 = 2 * (lane & 3);
-        volatile int32_t *moved = bar->moved;
         float mA = -INFINITY, mB = -INFINITY, lA = 0.f, lB = 0.f;
-        bool ok = true;
+        bool over = false, ok = true;
         for (int t = 0; t < n_tiles; ++t) {
-            const int buf = t & 1;
             if (!warp_wait_bounded(smem_addr(&bar->s_full[b]), t & 1, abort, hdr)) {
                 ok = false;
                 break;
@@ -483,35 +483,22 @@ attn_t128_kernel(const __grid_constant__ CUtensorMap tmap_k,
                         r[4 * (k >> 1) + 2 + (k & 1)] = __float_as_uint(-INFINITY);
                 }
             }
-            float xA = row_max(r, 0), xB = row_max(r, 2);
-            xA = fmaxf(xA, __shfl_xor_sync(0xffffffffu, xA, 1));
-            xB = fmaxf(xB, __shfl_xor_sync(0xffffffffu, xB, 1));
-            xA = fmaxf(xA, __shfl_xor_sync(0xffffffffu, xA, 2)) * a.scale_log2;
-            xB = fmaxf(xB, __shfl_xor_sync(0xffffffffu, xB, 2)) * a.scale_log2;
-            // move a row's reference max only when this tile exceeds it by > 2^8
-            float fA = 1.f, fB = 1.f;
-            const bool needA = xA > mA + kMoveLog2, needB = xB > mB + kMoveLog2;
-            if (needA) {
-                fA = (mA == -INFINITY) ? 0.f : ex2(mA - xA);
-                mA = xA;
-                lA *= fA;
+            // this thread's part of each row's tile max, in base-2 units
+            const float xA = row_max(r, 0) * a.scale_log2;
+            const float xB = row_max(r, 2) * a.scale_log2;
+            // a row that has seen nothing yet takes this tile's max as its
+            // reference (its O^T column and l are still zero)
+            if (__any_sync(0xffffffffu, mA == -INFINITY || mB == -INFINITY)) {
+                float yA = fmaxf(xA, __shfl_xor_sync(0xffffffffu, xA, 1));
+                float yB = fmaxf(xB, __shfl_xor_sync(0xffffffffu, xB, 1));
+                yA = fmaxf(yA, __shfl_xor_sync(0xffffffffu, yA, 2));
+                yB = fmaxf(yB, __shfl_xor_sync(0xffffffffu, yB, 2));
+                if (mA == -INFINITY)
+                    mA = yA;
+                if (mB == -INFINITY)
+                    mB = yB;
             }
-            if (needB) {
-                fB = (mB == -INFINITY) ? 0.f : ex2(mB - xB);
-                mB = xB;
-                lB *= fB;
-            }
-            if ((lane & 3) == 0) {
-                if (vA)
-                    aux->factor[buf][nA] = fA;
-                if (vB)
-                    aux->factor[buf][nB] = fB;
-            }
-            if (__any_sync(0xffffffffu, (needA && vA) || (needB && vB)) && lane == 0)
-                moved[buf] = t + 1;
-            __syncwarp();
-            if (lane == 0)
-                mbar_arrive(smem_addr(&bar->decided));
+            over |= (vA && xA > mA + kHeadroomLog2) || (vB && xB > mB + kHeadroomLog2);
 
             uint32_t pA[16], pB[16];
             {
@@ -522,14 +509,11 @@ attn_t128_kernel(const __grid_constant__ CUtensorMap tmap_k,
                 else if (hasA)
                     exp_pack_rows<false>(r, a.scale_log2, nmA, nmB, pA, pB, lA, lB);
             }
-
-            // every warp's factors are in place; P^T and O^T are free once
-            // PV(t-1) is done.  This warp saw PV(t-2) done before writing
-            // P^T(t-1), and PV(t) waits for this warp, so pv_done has one
-            // open phase here.
-            if (!warp_wait_bounded(smem_addr(&bar->decided), t & 1, abort, hdr) ||
-                (t > 0 &&
-                 !warp_wait_bounded(smem_addr(&bar->pv_done), (t - 1) & 1, abort, hdr))) {
+            // P^T is free once PV(t-1) is done.  This warp saw PV(t-2) done
+            // before writing P^T(t-1), and PV(t) waits for this warp, so
+            // pv_done has one open phase here.
+            if (t > 0 &&
+                !warp_wait_bounded(smem_addr(&bar->pv_done), (t - 1) & 1, abort, hdr)) {
                 ok = false;
                 break;
             }
@@ -537,31 +521,14 @@ attn_t128_kernel(const __grid_constant__ CUtensorMap tmap_k,
                 store_p_row(sP, nA, r_pad, lane, pA);
             if (hasB && vB)
                 store_p_row(sP, nB, r_pad, lane, pB);
-            if (t > 0 && moved[buf] == t + 1) {
-                // some row's max moved: scale this quarter's D lanes of O^T,
-                // 32-column chunks j, j + U, ...
-                tc_fence_after();
-                for (int c = 32 * j; c < r_pad; c += 32 * U) {
-#pragma unroll
-                    for (int h = 0; h < 32; h += 16) {
-                        uint32_t o[16];
-                        tmem_ld16(tmem + o_lane + c + h, o);
-#pragma unroll
-                        for (int jj = 0; jj < 16; ++jj)
-                            o[jj] = __float_as_uint(__uint_as_float(o[jj]) *
-                                                    aux->factor[buf][c + h + jj]);
-                        tmem_st16(tmem + o_lane + c + h, o);
-                    }
-                }
-                tmem_st_wait();
-            }
             fence_proxy_async_smem();
-            tc_fence_before();
             __syncwarp();
             if (lane == 0)
                 mbar_arrive(smem_addr(&bar->sm_done));
         }
-        // ---- final l of each row (four threads' partial sums), then O^T out
+        if (__any_sync(0xffffffffu, over) && lane == 0)
+            bar->overflow = 1;
+        // ---- (m, l) of each row (four threads' partial sums), then O^T
         lA += __shfl_xor_sync(0xffffffffu, lA, 1);
         lB += __shfl_xor_sync(0xffffffffu, lB, 1);
         lA += __shfl_xor_sync(0xffffffffu, lA, 2);
@@ -572,24 +539,14 @@ attn_t128_kernel(const __grid_constant__ CUtensorMap tmap_k,
         float *ws_ml = ws_o + (size_t)n_split * rows_all * kD;
         auto orow_of = [&](int n) { return (n / G) * a.n_heads_q + g * G + n % G; };
         if (ok && (lane & 3) == 0) {
-            if (vA) {
-                aux->l[nA] = lA;
-                if (n_split > 1)
-                    *reinterpret_cast<float2 *>(ws_ml + ((size_t)split * rows_all + orow_of(nA)) *
-                                                            2) = make_float2(mA, lA);
-            }
-            if (vB) {
-                aux->l[nB] = lB;
-                if (n_split > 1)
-                    *reinterpret_cast<float2 *>(ws_ml + ((size_t)split * rows_all + orow_of(nB)) *
-                                                            2) = make_float2(mB, lB);
-            }
+            if (vA)
+                *reinterpret_cast<float2 *>(ws_ml + ((size_t)split * rows_all + orow_of(nA)) * 2) =
+                    make_float2(mA, lA);
+            if (vB)
+                *reinterpret_cast<float2 *>(ws_ml + ((size_t)split * rows_all + orow_of(nB)) * 2) =
+                    make_float2(mB, lB);
         }
-        __syncwarp();
-        if (ok && lane == 0)
-            mbar_arrive(smem_addr(&bar->l_ready));
-        if (ok && warp_wait_bounded(smem_addr(&bar->l_ready), 0, abort, hdr) &&
-            warp_wait_bounded(smem_addr(&bar->o_final), 0, abort, hdr)) {
+        if (ok && warp_wait_bounded(smem_addr(&bar->o_final), 0, abort, hdr)) {
             tc_fence_after();
             const int d = 32 * q + lane;
             for (int c = 32 * j; c < r_pad; c += 32 * U) {
@@ -598,13 +555,9 @@ attn_t128_kernel(const __grid_constant__ CUtensorMap tmap_k,
 #pragma unroll
                 for (int jj = 0; jj < 32; ++jj) {
                     const int n = c + jj;
-                    if (n < R) {
-                        const float v = __uint_as_float(o[jj]);
-                        if (n_split == 1)
-                            a.out[(size_t)orow_of(n) * kD + d] = v / aux->l[n];
-                        else
-                            ws_o[((size_t)split * rows_all + orow_of(n)) * kD + d] = v;
-                    }
+                    if (n < R)
+                        ws_o[((size_t)split * rows_all + orow_of(n)) * kD + d] =
+                            __uint_as_float(o[jj]);
                 }
             }
         }
@@ -616,9 +569,172 @@ attn_t128_kernel(const __grid_constant__ CUtensorMap tmap_k,
         tc_fence_after();
         tmem_dealloc(tmem, kTmemCols);
     }
+    if (threadIdx.x == 0)
+        flags[split * a.n_heads_kv + g] = bar->overflow;
+}
+
+// One split's partial (m, l, acc) of one query row, recomputed exactly in
+// fp32 from K and V by an online softmax over the split's visible
+// positions.  One warp; lane holds head dims 4 lane .. 4 lane + 3.  Used
+// only for splits whose flag says the kernel's fixed reference max ran out
+// of headroom.
+__device__ void split_partial_exact(const AttnArgs &a, unsigned long long anc, int g,
+                                    const float (&q4)[4], int p0, int p1, float &m, float &l,
+                                    float (&acc)[4])
+{
+    const int lane = threadIdx.x & 31;
+    const __nv_bfloat16 *kh = a.k + (size_t)g * a.kv_cap * kD + 4 * lane;
+    const __nv_bfloat16 *vh = a.v + (size_t)g * a.kv_cap * kD + 4 * lane;
+    m = -INFINITY;
+    l = 0.f;
+#pragma unroll
+    for (int e = 0; e < 4; ++e)
+        acc[e] = 0.f;
+    for (int pos = p0; pos < p1; ++pos) {
+        const int tp = pos - a.n_ctx;
+        if (tp >= 0 && !((anc >> tp) & 1ull))
+            continue;
+        const uint2 kb = *reinterpret_cast<const uint2 *>(kh + (size_t)pos * kD);
+        const float2 k01 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&kb.x));
+        const float2 k23 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&kb.y));
+        float dot = q4[0] * k01.x + q4[1] * k01.y + q4[2] * k23.x + q4[3] * k23.y;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1)
+            dot += __shfl_xor_sync(0xffffffffu, dot, o);
+        const float sc = dot * a.scale_log2;
+        if (sc > m) {
+            const float f = exp2f(m - sc);
+            l *= f;
+#pragma unroll
+            for (int e = 0; e < 4; ++e)
+                acc[e] *= f;
+            m = sc;
+        }
+        const float pw = exp2f(sc - m);
+        const uint2 vb = *reinterpret_cast<const uint2 *>(vh + (size_t)pos * kD);
+        const float2 v01 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&vb.x));
+        const float2 v23 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&vb.y));
+        l += pw;
+        acc[0] += pw * v01.x;
+        acc[1] += pw * v01.y;
+        acc[2] += pw * v23.x;
+        acc[3] += pw * v23.y;
+    }
+}
+
+// One warp per output row: out = sum_s 2^(m_s - M) acc_s / sum_s 2^(m_s - M) l_s
+// over the splits' partials, with flagged splits recomputed exactly.
+__global__ void __launch_bounds__(256)
+attn_t128_combine_kernel(AttnArgs a, TreeMasks masks, int n_split, int tiles_per_split,
+                         const int32_t *__restrict__ flags)
+{
+    const int rows_all = a.n_tree * a.n_heads_q;
+    const int row = blockIdx.x * 8 + (threadIdx.x >> 5);
+    const int lane = threadIdx.x & 31;
+    if (row >= rows_all)
+        return;
+    const int head = row % a.n_heads_q, node = row / a.n_heads_q;
+    const int g = head / (a.n_heads_q / a.n_heads_kv);
+    const float *ws_o =
+        reinterpret_cast<const float *>(reinterpret_cast<const char *>(a.workspace) + kHeaderBytes);
+    const float *ws_ml = ws_o + (size_t)n_split * rows_all * kD;
+    bool any = false;
+    for (int s = lane; s < n_split; s += 32)
+        any |= flags[s * a.n_heads_kv + g] != 0;
+    any = __any_sync(0xffffffffu, any);
+
+    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+    float L = 0.f;
+    if (!any) {
+        float M = -INFINITY;
+        for (int s = 0; s < n_split; ++s)
+            M = fmaxf(M, __ldcg(ws_ml + ((size_t)s * rows_all + row) * 2));
+        // splits in batches of kB: the batch's loads are in flight together
+        constexpr int kB = 6;
+        for (int s0 = 0; s0 < n_split; s0 += kB) {
+            float2 ml[kB];
+            float4 x[kB];
+#pragma unroll
+            for (int u = 0; u < kB; ++u) {
+                const int s = s0 + u;
+                if (s < n_split) {
+                    ml[u] = __ldcg(
+                        reinterpret_cast<const float2 *>(ws_ml + ((size_t)s * rows_all + row) * 2));
+                    x[u] = __ldcg(reinterpret_cast<const float4 *>(
+                        ws_o + ((size_t)s * rows_all + row) * kD + 4 * lane));
+                } else {
+                    ml[u] = make_float2(-INFINITY, 0.f);
+                    x[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+                }
+            }
+#pragma unroll
+            for (int u = 0; u < kB; ++u) {
+                const float w = ml[u].x == -INFINITY ? 0.f : exp2f(ml[u].x - M);
+                L += w * ml[u].y;
+                acc[0] += w * x[u].x;
+                acc[1] += w * x[u].y;
+                acc[2] += w * x[u].z;
+                acc[3] += w * x[u].w;
+            }
+        }
+    } else {
+        // fold the splits one by one into a running (M, L, acc)
+        const uint2 qb = *reinterpret_cast<const uint2 *>(a.q + (size_t)row * kD + 4 * lane);
+        const float2 q01 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&qb.x));
+        const float2 q23 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&qb.y));
+        const float q4[4] = {q01.x, q01.y, q23.x, q23.y};
+        const int total = a.n_ctx + a.n_tree;
+        float M = -INFINITY;
+        for (int s = 0; s < n_split; ++s) {
+            float ms, ls, as[4];
+            if (flags[s * a.n_heads_kv + g]) {
+                const int p0 = s * tiles_per_split * kTileN;
+                const int p1 = min(p0 + tiles_per_split * kTileN, total);
+                split_partial_exact(a, masks.anc[node], g, q4, p0, p1, ms, ls, as);
+            } else {
+                const float2 ml = __ldcg(
+                    reinterpret_cast<const float2 *>(ws_ml + ((size_t)s * rows_all + row) * 2));
+                const float4 x = __ldcg(reinterpret_cast<const float4 *>(
+                    ws_o + ((size_t)s * rows_all + row) * kD + 4 * lane));
+                ms = ml.x;
+                ls = ml.y;
+                as[0] = x.x;
+                as[1] = x.y;
+                as[2] = x.z;
+                as[3] = x.w;
+            }
+            if (ms == -INFINITY)
+                continue;
+            const float Mn = fmaxf(M, ms);
+            const float fa = M == -INFINITY ? 0.f : exp2f(M - Mn);
+            const float fb = exp2f(ms - Mn);
+            L = L * fa + ls * fb;
+#pragma unroll
+            for (int e = 0; e < 4; ++e)
+                acc[e] = acc[e] * fa + as[e] * fb;
+            M = Mn;
+        }
+    }
+    const float inv = 1.f / L;
+    *reinterpret_cast<float4 *>(a.out + (size_t)row * kD + 4 * lane) =
+        make_float4(acc[0] * inv, acc[1] * inv, acc[2] * inv, acc[3] * inv);
+}
+
+// Split partials (acc, m, l) after the header, then one int32 overflow flag
+// per (split, KV head).
+size_t flags_offset(int n_split, int n_heads_q, int n_tree)
+{
+    return kHeaderBytes + align_up(attn_partial_bytes(n_split, n_heads_q, kD, n_tree), 256);
 }
 
 }  // namespace
+
+size_t attn_t128_workspace_bytes(int n_heads_q, int n_heads_kv, int n_ctx, int n_tree, int num_sms)
+{
+    const AttnPlan p = attn_t128_plan(n_heads_q, n_heads_kv, n_ctx, n_tree, num_sms);
+    return flags_offset(p.n_split, n_heads_q, n_tree) +
+           align_up((size_t)p.n_split * n_heads_kv * sizeof(int32_t), 256);
+}
 
 bool attn_t128_eligible(int n_heads_q, int n_heads_kv, int head_dim, int n_ctx, int n_tree)
 {
@@ -652,15 +768,21 @@ cudaError_t attn_t128_launch(const AttnArgs &a, const TreeMasks &masks, int num_
         attn_t128_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemLimit);
     if (attr != cudaSuccess)
         return attr;
+    int32_t *flags = reinterpret_cast<int32_t *>(
+        reinterpret_cast<char *>(a.workspace) + flags_offset(p.n_split, a.n_heads_q, a.n_tree));
     attn_t128_kernel<<<dim3(p.n_split, a.n_heads_kv), kThreads, lay.smem_bytes, stream>>>(
-        mk, mv, a, masks, p.tiles_per_split, p.n_split);
+        mk, mv, a, masks, p.tiles_per_split, p.n_split, flags);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess)
         return e;
     count_launches(1);
-    if (p.n_split == 1)
-        return cudaSuccess;
-    return attn_combine_launch(a, p.n_split, stream);
+    const int rows_all = a.n_tree * a.n_heads_q;
+    attn_t128_combine_kernel<<<(rows_all + 7) / 8, 256, 0, stream>>>(a, masks, p.n_split,
+                                                                      p.tiles_per_split, flags);
+    e = cudaGetLastError();
+    if (e == cudaSuccess)
+        count_launches(1);
+    return e;
 }
 
 }  // namespace ts

@@ -157,6 +157,28 @@ def test_attn_rising_scores_move_the_reference_max(oracle_mod, hq, hkv, t):
     assert np.isfinite(got).all()
 
 
+@pytest.mark.parametrize("hq,hkv,t", [(32, 8, 40), (32, 32, 40)])
+def test_attn_score_jump_past_headroom(oracle_mod, hq, hkv, t):
+    """Two context positions whose K is 120.0 in every dimension: rows with a
+    positive query sum see a score about 15 * sum(q) (base 2) above
+    everything else -- far past the 64 of headroom the tcgen05 kernel keeps
+    above a row's first-tile max, and past the fp32 range for many rows.
+    Those splits must come out exact all the same (they are recomputed);
+    sampled rows, plus every row of node 0, against the oracle."""
+    w = I.Workload("jump", hq, hkv, 128, 12000, t, seed=70 + hq)
+    q = I.gen_q(w)
+    k, v = I.gen_kv(w)
+    k[:, [5000, 9001], :] = I.f32_to_bf16_bits(np.float32(120.0))
+    got = run_attn(q, k, v, w.n_ctx, w.parent())
+    nodes, heads = sample_rows(w.n_tree, w.n_heads_q, 24, w.seed)
+    nodes = np.concatenate([nodes, np.zeros(hq, np.int32)])
+    heads = np.concatenate([heads, np.arange(hq, dtype=np.int32)])
+    want = oracle_mod.tree_verify_attn_rows(q, k, v, w.n_ctx, w.parent(), nodes, heads)
+    err = np.abs(got[nodes, heads] - want).max()
+    assert err <= ATTN_TOL, f"{w.name}: max abs err {err}"
+    assert np.isfinite(got).all()
+
+
 def test_attn_draft_pass_over_partial_cache(oracle_mod):
     """Draft pass: a 4-node chain over a 4096-row compact cache (64 sinks + 4032)."""
     w = I.Workload("draft", 32, 8, 128, 4096, 4, tree="chain", seed=12)
