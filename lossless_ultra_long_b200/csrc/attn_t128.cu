@@ -117,8 +117,9 @@ __host__ __device__ inline Layout t128_layout(int rows)
     L.r_pad = (rows + 15) / 16 * 16;
     L.q1_off = 0;
     L.p_off = rows > kBlockM ? kQ1Bytes : 0;
-    // P^T: positions 0-63 then 64-127, each r_pad rows of 128 bytes
-    L.k_off = L.p_off + (size_t)L.r_pad * 256;
+    // P^T: positions 0-63 then 64-127, each r_pad rows of 128 bytes; then
+    // 1 KB that rows past the query rows are written to
+    L.k_off = L.p_off + (size_t)L.r_pad * 256 + 1024;
     const size_t fixed = 1024 + L.k_off + kAuxBytes;
     int stages = (int)((kSmemLimit - fixed) / kStageBytes);
     stages = stages > 2 * kMaxStages ? 2 * kMaxStages : stages;
@@ -192,16 +193,28 @@ __device__ __forceinline__ float row_max(const uint32_t (&r)[64], int e)
     return fmaxf(max3f(m[0], m[1], m[2]), m[3]);
 }
 
-// One row's 32 bf16 pairs into the K-major, 128-byte-swizzled P^T tile:
-// pair j covers positions 8j + c0, +1 (c0 = 2 * (lane % 4)).
-__device__ __forceinline__ void store_p_row(unsigned char *sP, int n, int r_pad, int lane,
-                                            const uint32_t (&pk)[16])
+// Eight rows' P (one half of a 16-lane unit: rows nbase + r, r = 0..7, of
+// which the first n_valid are query rows) into the K-major,
+// 128-byte-swizzled P^T tile.  pk[j] of thread t holds positions
+// 8j + 2(t%4), +1 of row t/4: the m8n8 fragment of matrix j, so four
+// stmatrix instructions write the 16 matrices, each row a 16-byte chunk.
+// Rows past n_valid go to the scratch kilobyte instead, so they cannot land
+// on another lane quarter's rows.
+__device__ __forceinline__ void store_p_half(uint32_t p_addr, uint32_t scratch, int nbase,
+                                             int n_valid, int r_pad, int lane,
+                                             const uint32_t (&pk)[16])
 {
-    unsigned char *row = sP + (n >> 3) * 1024 + (n & 7) * 128 + 4 * (lane & 3);
+    const int r = lane & 7, n = nbase + r;
+    const bool valid = r < n_valid;
+    const uint32_t row = p_addr + (uint32_t)((n >> 3) * 1024 + (n & 7) * 128);
 #pragma unroll
-    for (int j = 0; j < 16; ++j)
-        *reinterpret_cast<uint32_t *>(row + (j >> 3) * (r_pad * 128) +
-                                      (((j & 7) ^ (n & 7)) << 4)) = pk[j];
+    for (int m = 0; m < 4; ++m) {
+        const int j = 4 * m + (lane >> 3);
+        const uint32_t addr = valid ? row + (uint32_t)((j >> 3) * (r_pad * 128) +
+                                                       (((j & 7) ^ (n & 7)) << 4))
+                                    : scratch + (uint32_t)(lane << 4);
+        stmatrix_x4(addr, pk[4 * m], pk[4 * m + 1], pk[4 * m + 2], pk[4 * m + 3]);
+    }
 }
 
 __global__ void __launch_bounds__(kThreads, 1)
@@ -444,6 +457,13 @@ attn_t128_kernel(const __grid_constant__ CUtensorMap tmap_k,
         const uint32_t s_addr = tmem + ((uint32_t)(32 * q + lb) << 16) + kSCol + 128 * b;
         const uint32_t o_lane = (uint32_t)(32 * q) << 16;
         const int c0 = 2 * (lane & 3);
+        // P^T rows of this unit: half A is nbase + 0..7, half B nbase + 8..15;
+        // the valid ones are those inside the quarter's run and the block
+        const int nbase = kBlockM * b + q * rqb + lb;
+        const int nvA = max(0, min(8, min(rqb - lb, Rb - q * rqb - lb)));
+        const int nvB = max(0, min(8, min(rqb - lb - 8, Rb - q * rqb - lb - 8)));
+        const uint32_t p_addr = smem_addr(sP);
+        const uint32_t p_scratch = p_addr + (uint32_t)r_pad * 256;
         float mA = -INFINITY, mB = -INFINITY, lA = 0.f, lB = 0.f;
         bool over = false, ok = true;
         for (int t = 0; t < n_tiles; ++t) {
@@ -517,10 +537,10 @@ attn_t128_kernel(const __grid_constant__ CUtensorMap tmap_k,
                 ok = false;
                 break;
             }
-            if (hasA && vA)
-                store_p_row(sP, nA, r_pad, lane, pA);
-            if (hasB && vB)
-                store_p_row(sP, nB, r_pad, lane, pB);
+            if (hasA)
+                store_p_half(p_addr, p_scratch, nbase, nvA, r_pad, lane, pA);
+            if (hasB)
+                store_p_half(p_addr, p_scratch, nbase + 8, nvB, r_pad, lane, pB);
             fence_proxy_async_smem();
             __syncwarp();
             if (lane == 0)

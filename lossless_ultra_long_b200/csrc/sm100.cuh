@@ -312,6 +312,17 @@ __device__ __forceinline__ void tmem_st_wait()
     asm volatile("tcgen05.wait::st.sync.aligned;\n" ::: "memory");
 }
 
+// Four 8x8 b16 matrices to shared memory: register i of thread t holds
+// row t/4, elements 2(t%4) and 2(t%4)+1 of matrix i; thread t gives the
+// 16-byte-aligned address of row t%8 of matrix t/8.
+__device__ __forceinline__ void stmatrix_x4(uint32_t addr, uint32_t r0, uint32_t r1, uint32_t r2,
+                                            uint32_t r3)
+{
+    asm volatile("stmatrix.sync.aligned.m8n8.x4.shared.b16 [%0], {%1, %2, %3, %4};\n" ::"r"(addr),
+                 "r"(r0), "r"(r1), "r"(r2), "r"(r3)
+                 : "memory");
+}
+
 // 2^x by the MUFU ex2 instruction, subnormal results flushed to zero.
 __device__ __forceinline__ float ex2(float x)
 {
