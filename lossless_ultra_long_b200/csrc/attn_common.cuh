@@ -33,11 +33,11 @@ size_t attn_mma_workspace_bytes(int n_heads_q, int n_heads_kv, int head_dim, int
 cudaError_t attn_mma_launch(const AttnArgs &a, const TreeMasks &masks, int num_sms,
                             cudaStream_t stream);
 
-// Tensor map over a bf16 [Hkv, kv_cap, 128] cache viewed as 3-D (d,
+// Tensor map over a bf16 [Hkv, kv_cap, head_dim] cache viewed as 3-D (d,
 // position, head), 128-byte swizzle, boxes of 64 columns x box_rows
 // positions; positions at or past `rows` read as zeros.
 bool encode_kv_map(CUtensorMap *m, const void *ptr, int rows, int64_t kv_cap, int n_heads_kv,
-                   int box_rows);
+                   int box_rows, int head_dim = 128);
 
 bool attn_tc_eligible(int n_heads_q, int n_heads_kv, int head_dim, int n_ctx, int n_tree);
 // (the tcgen05 kernel also needs softmax_scale > 0: it takes the row max on

@@ -617,13 +617,13 @@ PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder()
 }
 
 bool encode_kv_map(CUtensorMap *m, const void *ptr, int rows, int64_t kv_cap, int n_heads_kv,
-                   int box_rows)
+                   int box_rows, int head_dim)
 {
     auto enc = tensor_map_encoder();
     if (!enc)
         return false;
-    const cuuint64_t dims[3] = {(cuuint64_t)kD, (cuuint64_t)rows, (cuuint64_t)n_heads_kv};
-    const cuuint64_t strides[2] = {(cuuint64_t)kD * 2, (cuuint64_t)kv_cap * kD * 2};
+    const cuuint64_t dims[3] = {(cuuint64_t)head_dim, (cuuint64_t)rows, (cuuint64_t)n_heads_kv};
+    const cuuint64_t strides[2] = {(cuuint64_t)head_dim * 2, (cuuint64_t)kv_cap * head_dim * 2};
     const cuuint32_t box[3] = {64, (cuuint32_t)box_rows, 1};
     const cuuint32_t estr[3] = {1, 1, 1};
     return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(ptr), dims, strides, box,

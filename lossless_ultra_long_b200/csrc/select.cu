@@ -8,14 +8,14 @@
 // that partial cache.
 //
 // Pass 1 (grid: chunks x Hkv): s[h,n] = log2(e) * scale * q_last[h] . k[g,n]
-//   for the G query heads of KV head g.  A CTA streams its chunk of key rows
-//   (contiguous for one head) through a 4-stage shared-memory ring filled by
-//   1-D bulk async copies of 64 rows.  Each lane takes 16 bytes of a key
-//   row (a row is D/8 lanes), forms the partial dots of several rows and
-//   heads, and a transpose-reduce across the row's lanes leaves one finished
-//   (row, head) dot per lane: one shuffle per dot instead of log2(D/8).
-//   Writes s (fp32 [Hq, n_ctx]) and a running (max, sum 2^(s-max)) per head
-//   and chunk.  K is read once: Hkv * n_ctx * D * 2 bytes.
+//   for the G query heads of KV head g, on the tensor cores: per 16 keys a
+//   warp runs D/16 mma.sync m16n8k16 (bf16 in, fp32 accumulate) with the
+//   keys as the 16 rows of A, read from a 128-byte-swizzled TMA tile with
+//   ldmatrix, and the group's query rows as the 8 columns of B, held in
+//   registers.  A CTA streams its chunk of key rows through a 4-stage ring
+//   of 64-row tiles (one producer lane, four MMA warps).  Writes s (fp32
+//   [Hq, n_ctx]) and a running (max, sum 2^(s-max)) per head and chunk.
+//   K is read once: Hkv * n_ctx * D * 2 bytes.
 // Pass 2 (one 8-CTA cluster per KV head): merges the chunk partials into
 //   the softmax max / normaliser of each head, forms
 //   score[n] = (1/G) sum_h 2^(s[h,n] - M_h) / Z_h for its slice of
@@ -29,6 +29,7 @@
 #include <cooperative_groups.h>
 #include <math.h>
 
+#include "attn_common.cuh"
 #include "sm100.cuh"
 #include "ts_internal.cuh"
 
@@ -37,7 +38,6 @@ namespace cg = cooperative_groups;
 namespace ts {
 namespace {
 
-constexpr int kP1Threads = 256;
 constexpr int kClusterCtas = 8;
 constexpr int kP2Threads = 512;
 constexpr int kMaxSlice = 48 * 1024;   // positions per CTA held in shared memory
@@ -46,164 +46,153 @@ constexpr int kMaxGroup = 8;
 // ------------------------------------------------------------------ pass 1
 constexpr int kP1Rows = 64;     // key rows per pipeline stage
 constexpr int kP1Stages = 4;
+constexpr int kP1Warps = 4;     // MMA warps, 16 keys of a tile each; warp 4 loads
+constexpr int kP1Threads = 32 * (kP1Warps + 1);
+constexpr int kP1BoxBytes = kP1Rows * 128;   // 64 rows x 64 columns of bf16
 
-__device__ __forceinline__ void bulk_load(uint32_t dst, const void *src, uint32_t bytes,
-                                          uint32_t bar)
+__device__ __forceinline__ void ldmatrix_x4(uint32_t addr, uint32_t (&r)[4])
 {
-    asm volatile(
-        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];\n"
-        ::"r"(dst), "l"(src), "r"(bytes), "r"(bar)
-        : "memory");
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];\n"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+                 : "r"(addr));
 }
 
-template <int D, int GP>
+// d += a (16x16, row-major) * b (16x8, column-major), bf16 in, fp32 accumulate
+__device__ __forceinline__ void mma_16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0,
+                                          uint32_t b1)
+{
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, "
+        "{%4, %5, %6, %7}, {%8, %9}, {%0, %1, %2, %3};\n"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+template <int D>
 __global__ void __launch_bounds__(kP1Threads)
-score_logits_kernel(SelectArgs a, int chunk, int n_chunks)
+score_logits_kernel(const __grid_constant__ CUtensorMap tmap_k, SelectArgs a, int chunk,
+                    int n_chunks)
 {
     using namespace sm100;
-    constexpr int LPR = D / 8;          // lanes per key row (16 bytes each)
-    constexpr int NV = LPR;             // values per lane before the reduce
-    constexpr int RL = NV / GP;         // rows per lane group per step
-    constexpr int GROUPS = 32 / LPR;    // lane groups per warp
-    constexpr int ROWS_PER_WARP = GROUPS * RL;
-    constexpr int kStageBytes = kP1Rows * D * 2;
+    constexpr int kBoxes = D / 64;
+    constexpr int kStageBytes = kBoxes * kP1BoxBytes;
 
-    extern __shared__ __align__(128) unsigned char ring_raw[];
-    unsigned char(*ring)[kStageBytes] = reinterpret_cast<unsigned char(*)[kStageBytes]>(ring_raw);
-    __shared__ uint64_t full[kP1Stages];
+    extern __shared__ unsigned char p1_raw[];
+    unsigned char *ring = reinterpret_cast<unsigned char *>(
+        (reinterpret_cast<uintptr_t>(p1_raw) + 1023) & ~uintptr_t(1023));
+    __shared__ uint64_t full[kP1Stages], empty[kP1Stages];
     __shared__ uint32_t abort_flag;
+    __shared__ float red_m[kP1Warps * 32][2], red_l[kP1Warps * 32][2];
 
     const int g = blockIdx.y;
     const int c = blockIdx.x;
     const int G = a.n_heads_q / a.n_heads_kv;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    const int li = lane % LPR, grp = lane / LPR;
     const int n0 = c * chunk;
     const int n1 = min(n0 + chunk, a.n_ctx);
     const int n_tiles = (n1 - n0 + kP1Rows - 1) / kP1Rows;
-    const __nv_bfloat16 *kh = a.k + (int64_t)g * a.kv_cap * D;
     WorkspaceHeader *hdr = reinterpret_cast<WorkspaceHeader *>(a.workspace);
+    float *s_out = reinterpret_cast<float *>(reinterpret_cast<char *>(a.workspace) + kHeaderBytes);
 
-    // rows of one KV head are contiguous: each tile is one bulk copy
-    auto issue = [&](int t) {
-        const int r0 = n0 + t * kP1Rows;
-        const uint32_t bytes = (uint32_t)min(kP1Rows, n1 - r0) * D * 2;
-        const uint32_t fb = smem_addr(&full[t % kP1Stages]);
-        mbar_arrive_expect_tx(fb, bytes);
-        bulk_load(smem_addr(ring[t % kP1Stages]), kh + (int64_t)r0 * D, bytes, fb);
-    };
     if (threadIdx.x == 0) {
-        for (int s = 0; s < kP1Stages; ++s)
+        for (int s = 0; s < kP1Stages; ++s) {
             mbar_init(smem_addr(&full[s]), 1);
+            mbar_init(smem_addr(&empty[s]), kP1Warps);
+        }
         abort_flag = 0u;
         fence_mbar_init();
-        fence_proxy_async_smem();
-        for (int t = 0; t < min(kP1Stages, n_tiles); ++t)
-            issue(t);
     }
+    __syncthreads();
 
-    float qf[GP][8];
+    if (warp == kP1Warps) {
+        // ------------------------------------------------------- producer
+        if (lane == 0) {
+            int issued = 0;
+            for (int t = 0; t < n_tiles; ++t) {
+                const int s = t % kP1Stages;
+                if (t >= kP1Stages && !wait_bounded(smem_addr(&empty[s]),
+                                                    ((t / kP1Stages) & 1) ^ 1, &abort_flag, hdr))
+                    break;
+                const uint32_t fb = smem_addr(&full[s]);
+                mbar_arrive_expect_tx(fb, kStageBytes);
 #pragma unroll
-    for (int h = 0; h < GP; ++h) {
-        if (h < G) {
-            const uint4 raw = *reinterpret_cast<const uint4 *>(
-                a.q_last + (int64_t)(g * G + h) * D + li * 8);
-            const __nv_bfloat162 *p2 = reinterpret_cast<const __nv_bfloat162 *>(&raw);
+                for (int b = 0; b < kBoxes; ++b)
+                    tma_load_3d(smem_addr(ring + s * kStageBytes + b * kP1BoxBytes), &tmap_k, 64 * b,
+                                n0 + t * kP1Rows, g, fb);
+                issued = t + 1;
+            }
+            if (abort_flag)
+                for (int t = max(0, issued - kP1Stages); t < issued; ++t)
+                    wait_drain(smem_addr(&full[t % kP1Stages]), (t / kP1Stages) & 1);
+        }
+    } else {
+        // ------------------------------------------------------ MMA warps
+        // B = Q_group^T: column n = query head g*G + n (zero past G); the
+        // fragment of k-step kk holds q[n][16kk + 2(lane%4) + {0,1}] and
+        // q[n][16kk + 8 + 2(lane%4) + {0,1}] for n = lane / 4
+        const int hq = lane >> 2;
+        uint32_t bq[D / 16][2];
+        const uint32_t *qrow = reinterpret_cast<const uint32_t *>(
+            a.q_last + (int64_t)(g * G + (hq < G ? hq : 0)) * D);
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+            bq[kk][0] = hq < G ? qrow[8 * kk + (lane & 3)] : 0u;
+            bq[kk][1] = hq < G ? qrow[8 * kk + 4 + (lane & 3)] : 0u;
+        }
+        // this lane's ldmatrix row (of the warp's 16 keys) and 8-column half
+        const int lr = warp * 16 + (lane & 7) + 8 * ((lane >> 3) & 1);
+        const int lh = lane >> 4;
+        // accumulator (key, head) of this lane: keys lane/4 and lane/4 + 8,
+        // heads 2(lane%4) and 2(lane%4) + 1
+        const int h0 = 2 * (lane & 3);
+        float run_m[2] = {-INFINITY, -INFINITY}, run_l[2] = {0.f, 0.f};
+        for (int t = 0; t < n_tiles; ++t) {
+            const int s = t % kP1Stages;
+            if (!warp_wait_bounded(smem_addr(&full[s]), (t / kP1Stages) & 1, &abort_flag, hdr))
+                break;
+            const uint32_t stage = smem_addr(ring + s * kStageBytes);
+            float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+            for (int kk = 0; kk < D / 16; ++kk) {
+                const int ch = (kk & 3) * 2 + lh;   // 16-byte chunk within the 128-byte row
+                uint32_t af[4];
+                ldmatrix_x4(stage + (kk >> 2) * kP1BoxBytes + lr * 128 + ((ch ^ (lr & 7)) << 4), af);
+                mma_16816(acc, af, bq[kk][0], bq[kk][1]);
+            }
+            __syncwarp();
+            if (lane == 0)
+                mbar_arrive(smem_addr(&empty[s]));
+            const int nk = n0 + t * kP1Rows + warp * 16 + (lane >> 2);
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
-                const float2 f = __bfloat1622float2(p2[e]);
-                qf[h][2 * e] = f.x * a.scale_log2;
-                qf[h][2 * e + 1] = f.y * a.scale_log2;
+                const int n = nk + 8 * (e >> 1), h = h0 + (e & 1);
+                if (h < G && n < n1) {
+                    const float sv = acc[e] * a.scale_log2;
+                    s_out[(int64_t)(g * G + h) * a.n_ctx + n] = sv;
+                    const float m_new = fmaxf(run_m[e & 1], sv);
+                    run_l[e & 1] = run_l[e & 1] * exp2f(run_m[e & 1] - m_new) + exp2f(sv - m_new);
+                    run_m[e & 1] = m_new;
+                }
             }
-        } else {
-#pragma unroll
-            for (int e = 0; e < 8; ++e)
-                qf[h][e] = 0.f;
         }
+        red_m[threadIdx.x][0] = run_m[0];
+        red_m[threadIdx.x][1] = run_m[1];
+        red_l[threadIdx.x][0] = run_l[0];
+        red_l[threadIdx.x][1] = run_l[1];
     }
     __syncthreads();
-
-    // this lane's finished value is always head (li % GP), row slot li / GP
-    const int my_h = li % GP, my_j = li / GP;
-    float run_m = -INFINITY, run_l = 0.f;
-    float *s_out = reinterpret_cast<float *>(reinterpret_cast<char *>(a.workspace) + kHeaderBytes);
-    const int nwarps = kP1Threads / 32;
-    for (int t = 0; t < n_tiles; ++t) {
-        const bool ok = wait_bounded(smem_addr(&full[t % kP1Stages]), (t / kP1Stages) & 1,
-                                     &abort_flag, hdr);
-        if (__syncthreads_or(!ok))   // leave the loop together
-            break;
-        const unsigned char *stage = ring[t % kP1Stages];
-        const int rows = min(kP1Rows, n1 - (n0 + t * kP1Rows));
-        for (int base = warp * ROWS_PER_WARP; base < rows; base += nwarps * ROWS_PER_WARP) {
-            float v[NV];
-#pragma unroll
-            for (int j = 0; j < RL; ++j) {
-                const int r = base + grp * RL + j;
-                const uint4 kr = r < rows ? *reinterpret_cast<const uint4 *>(stage + r * D * 2 + li * 16)
-                                          : make_uint4(0u, 0u, 0u, 0u);
-                const __nv_bfloat162 *p2 = reinterpret_cast<const __nv_bfloat162 *>(&kr);
-                float kf[8];
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const float2 f = __bfloat1622float2(p2[e]);
-                    kf[2 * e] = f.x;
-                    kf[2 * e + 1] = f.y;
-                }
-#pragma unroll
-                for (int h = 0; h < GP; ++h) {
-                    float acc = 0.f;
-#pragma unroll
-                    for (int e = 0; e < 8; ++e)
-                        acc = fmaf(qf[h][e], kf[e], acc);
-                    v[j * GP + h] = acc;
-                }
-            }
-            // transpose-reduce across the LPR lanes of the row group
-#pragma unroll
-            for (int o = NV / 2; o >= 1; o >>= 1) {
-                const bool upper = (li & o) != 0;
-#pragma unroll
-                for (int q = 0; q < o; ++q) {
-                    const float send = upper ? v[q] : v[q + o];
-                    const float keep = upper ? v[q + o] : v[q];
-                    v[q] = keep + __shfl_xor_sync(0xffffffffu, send, o);
-                }
-            }
-            const int r = base + grp * RL + my_j;
-            if (my_h < G && r < rows) {
-                const float sv = v[0];
-                s_out[(int64_t)(g * G + my_h) * a.n_ctx + n0 + t * kP1Rows + r] = sv;
-                const float m_new = fmaxf(run_m, sv);
-                run_l = run_l * exp2f(run_m - m_new) + exp2f(sv - m_new);
-                run_m = m_new;
-            }
-        }
-        __syncthreads();   // every warp is done with this stage
-        if (threadIdx.x == 0 && t + kP1Stages < n_tiles)
-            issue(t + kP1Stages);
-    }
-    if (abort_flag && threadIdx.x == 0)
-        for (int t = max(0, n_tiles - kP1Stages); t < n_tiles; ++t)
-            wait_drain(smem_addr(&full[t % kP1Stages]), (t / kP1Stages) & 1);
-
     // merge the running (max, sum) of every lane that holds head h
-    __shared__ float sm_m[kP1Threads], sm_l[kP1Threads];
-    sm_m[threadIdx.x] = run_m;
-    sm_l[threadIdx.x] = run_l;
-    __syncthreads();
     if (threadIdx.x < G) {
-        const int h = threadIdx.x;
+        const int h = threadIdx.x, e = h & 1;
         float M = -INFINITY;
-        for (int t = 0; t < kP1Threads; ++t)
-            if (((t & 31) % LPR) % GP == h)
-                M = fmaxf(M, sm_m[t]);
+        for (int t = 0; t < kP1Warps * 32; ++t)
+            if (2 * (t & 3) == (h & ~1))
+                M = fmaxf(M, red_m[t][e]);
         float L = 0.f;
-        for (int t = 0; t < kP1Threads; ++t)
-            if (((t & 31) % LPR) % GP == h && sm_m[t] != -INFINITY)
-                L += sm_l[t] * exp2f(sm_m[t] - M);
-        float *part = s_out + (size_t)a.n_heads_q * a.n_ctx;
-        float2 *pp = reinterpret_cast<float2 *>(part);
+        for (int t = 0; t < kP1Warps * 32; ++t)
+            if (2 * (t & 3) == (h & ~1) && red_m[t][e] != -INFINITY)
+                L += red_l[t][e] * exp2f(red_m[t][e] - M);
+        float2 *pp = reinterpret_cast<float2 *>(s_out + (size_t)a.n_heads_q * a.n_ctx);
         pp[(size_t)(g * G + h) * n_chunks + c] = make_float2(M, L);
     }
 }
@@ -504,16 +493,19 @@ SelPlan make_sel_plan(int n_heads_kv, int n_ctx, int num_sms)
     return p;
 }
 
-template <int D, int GP>
+template <int D>
 cudaError_t launch_p1(const SelectArgs &a, const SelPlan &p, cudaStream_t stream)
 {
-    constexpr int smem = kP1Stages * kP1Rows * D * 2;
+    CUtensorMap mk;
+    if (!encode_kv_map(&mk, a.k, a.n_ctx, a.kv_cap, a.n_heads_kv, kP1Rows, D))
+        return cudaErrorInvalidValue;
+    constexpr int smem = 1024 + kP1Stages * (D / 64) * kP1BoxBytes;
     static const cudaError_t attr = cudaFuncSetAttribute(
-        score_logits_kernel<D, GP>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+        score_logits_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (attr != cudaSuccess)
         return attr;
     dim3 grid(p.n_chunks, a.n_heads_kv);
-    score_logits_kernel<D, GP><<<grid, kP1Threads, smem, stream>>>(a, p.chunk, p.n_chunks);
+    score_logits_kernel<D><<<grid, kP1Threads, smem, stream>>>(mk, a, p.chunk, p.n_chunks);
     const cudaError_t e = cudaGetLastError();
     if (e == cudaSuccess)
         count_launches(1);
@@ -523,16 +515,7 @@ cudaError_t launch_p1(const SelectArgs &a, const SelPlan &p, cudaStream_t stream
 template <int D>
 cudaError_t launch_d(const SelectArgs &a, const SelPlan &p, cudaStream_t stream)
 {
-    const int G = a.n_heads_q / a.n_heads_kv;
-    cudaError_t e;
-    if (G == 1)
-        e = launch_p1<D, 1>(a, p, stream);
-    else if (G == 2)
-        e = launch_p1<D, 2>(a, p, stream);
-    else if (G <= 4)
-        e = launch_p1<D, 4>(a, p, stream);
-    else
-        e = launch_p1<D, 8>(a, p, stream);
+    cudaError_t e = launch_p1<D>(a, p, stream);
     if (e != cudaSuccess)
         return e;
 
