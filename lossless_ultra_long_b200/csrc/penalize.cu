@@ -6,24 +6,41 @@
 // kept.  Tencent article: 上下文惩罚 and the parallel-verification figure
 // (the worked example keeps "is the father of", the longest valid candidate).
 //
-// Grid (vocab chunks, tree nodes).  Each CTA marks the window ids that fall
-// in its chunk in a shared-memory bitmap, streams its slice of the logits
-// row with 16-byte loads, penalises marked ids (binary32 divide / multiply,
-// round-to-nearest) and reduces (value, id) with warp shuffles, ties to the
-// lower id.  Its result goes to the workspace; the CTA that takes the last
-// ticket reduces every node's chunks, writes the argmax, and walks the tree.
-// The logits are read exactly once; HBM traffic is T * V * 4 bytes.
+// Grid (vocab splits, tree nodes), sized to one wave of resident CTAs.  Each
+// CTA starts one bulk asynchronous copy of its slice of the logits row into
+// shared memory, marks the window ids that fall in the slice in a
+// shared-memory bitmap while it is in flight, then penalises marked ids
+// (binary32 divide / multiply, round-to-nearest) and reduces (value, id)
+// with warp shuffles, ties to the lower id.  Its result goes to the workspace; the CTA that
+// takes the last ticket reduces every node's splits, writes the argmax, and
+// walks the tree.  The logits are read exactly once: T * V * 4 bytes.
 #include <float.h>
 #include <limits.h>
 
+#include "sm100.cuh"
 #include "ts_internal.cuh"
 
 namespace ts {
 namespace {
 
 constexpr int kThreads = 256;
-constexpr int kChunk = 8192;            // vocab entries per CTA
-constexpr int kBitWords = kChunk / 32;
+constexpr int kMaxChunk = 16384;               // vocab entries per CTA, at most (64 KB)
+constexpr int kBitWords = kMaxChunk / 32;
+constexpr int kMaxSplits = 1024;
+
+// Vocab entries per CTA (a multiple of 4): enough splits per node for one
+// wave of resident CTAs (ctas_per_sm on each SM), no more than kMaxChunk
+// entries each.
+int penalize_chunk(int n_tree, int vocab, int num_sms, int ctas_per_sm)
+{
+    int splits = (ctas_per_sm * num_sms) / (n_tree > 0 ? n_tree : 1);
+    const int need = (vocab + kMaxChunk - 1) / kMaxChunk;
+    splits = splits < need ? need : splits;
+    splits = splits > kMaxSplits ? kMaxSplits : (splits < 1 ? 1 : splits);
+    int chunk = (vocab + splits - 1) / splits;
+    chunk = (chunk + 3) / 4 * 4;
+    return chunk < 4 ? 4 : chunk;
+}
 
 struct Best {
     float v;
@@ -59,27 +76,61 @@ __device__ __forceinline__ Best warp_best(Best b)
     return b;
 }
 
+// 64-bit key ordered like beats(): order-preserving bits of the value
+// (NaN already mapped to -inf by consider, zero's sign dropped), then the
+// complemented id
+__device__ __forceinline__ unsigned long long best_key(Best b)
+{
+    // -0 and +0 compare equal, so they must share one key (ties by id)
+    const uint32_t u = b.v == 0.f ? 0u : __float_as_uint(b.v);
+    const uint32_t ord = (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+    return ((unsigned long long)ord << 32) | (uint32_t)~(uint32_t)b.i;
+}
+
 __device__ __forceinline__ float penalise(float x, float p)
 {
     return x > 0.0f ? __fdiv_rn(x, p) : __fmul_rn(x, p);
 }
 
-__global__ void __launch_bounds__(kThreads)
-penalize_accept_kernel(PenalizeArgs a, TreeParents tree, int n_chunks)
+__device__ __forceinline__ void bulk_load(uint32_t dst, const void *src, uint32_t bytes,
+                                          uint32_t bar)
 {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];\n"
+        ::"r"(dst), "l"(src), "r"(bytes), "r"(bar)
+        : "memory");
+}
+
+__global__ void __launch_bounds__(kThreads)
+penalize_accept_kernel(PenalizeArgs a, TreeParents tree, int chunk, int n_chunks)
+{
+    extern __shared__ __align__(16) float xs[];   // this CTA's slice of the logits row
     __shared__ uint32_t bits[kBitWords];
     __shared__ Best warp_res[kThreads / 32];
     __shared__ int am[TS_MAX_TREE];
     __shared__ int is_last;
+    __shared__ uint64_t landed;
+    __shared__ uint32_t abort_flag;
 
     WorkspaceHeader *hdr = reinterpret_cast<WorkspaceHeader *>(a.workspace);
     Best *part = reinterpret_cast<Best *>(reinterpret_cast<char *>(a.workspace) + kHeaderBytes);
 
     const int tid = threadIdx.x;
     const int node = blockIdx.y;
-    const int v0 = blockIdx.x * kChunk;
-    const int v1 = min(v0 + kChunk, a.vocab);
+    const int v0 = blockIdx.x * chunk;
+    const int v1 = min(v0 + chunk, a.vocab);
+    const float *row = a.logits + (int64_t)node * a.vocab;
+    // rows and slices start on 16-byte boundaries and end on whole vectors
+    const bool vec = (a.vocab & 3) == 0 && (reinterpret_cast<uintptr_t>(a.logits) & 15) == 0;
 
+    if (vec && tid == 0) {
+        sm100::mbar_init(sm100::smem_addr(&landed), 1);
+        abort_flag = 0u;
+        sm100::fence_mbar_init();
+        const uint32_t bytes = (uint32_t)(v1 - v0) * 4u;
+        sm100::mbar_arrive_expect_tx(sm100::smem_addr(&landed), bytes);
+        bulk_load(sm100::smem_addr(xs), row + v0, bytes, sm100::smem_addr(&landed));
+    }
     for (int w = tid; w < kBitWords; w += kThreads)
         bits[w] = 0u;
     __syncthreads();
@@ -95,31 +146,26 @@ penalize_accept_kernel(PenalizeArgs a, TreeParents tree, int n_chunks)
     }
     __syncthreads();
 
-    const float *row = a.logits + (int64_t)node * a.vocab;
     const float p = a.penalty;
     Best b{-INFINITY, INT_MAX};
-    if ((a.vocab & 3) == 0) {
-        // all of this thread's 16-byte loads are issued before any is used
-        constexpr int kPer = kChunk / (kThreads * 4);
-        float4 x4[kPer];
+    if (vec) {
+        if (sm100::wait_bounded(sm100::smem_addr(&landed), 0, &abort_flag, hdr)) {
+            // two independent running bests (even and odd lanes of each
+            // vector) halve the compare chain
+            const float4 *x4 = reinterpret_cast<const float4 *>(xs);
+            Best b2{-INFINITY, INT_MAX};
+            for (int u = tid; u < (v1 - v0) / 4; u += kThreads) {
+                const float4 q = x4[u];
+                const uint32_t word = bits[u >> 3] >> ((u & 7) * 4);
+                const float x[4] = {q.x, q.y, q.z, q.w};
 #pragma unroll
-        for (int u = 0; u < kPer; ++u) {
-            const int v = v0 + (u * kThreads + tid) * 4;
-            x4[u] = v < v1 ? __ldcs(reinterpret_cast<const float4 *>(row + v))
-                           : make_float4(-INFINITY, -INFINITY, -INFINITY, -INFINITY);
-        }
-#pragma unroll
-        for (int u = 0; u < kPer; ++u) {
-            const int v = v0 + (u * kThreads + tid) * 4;
-            if (v >= v1)
-                continue;
-            const uint32_t word = bits[(v - v0) >> 5] >> ((v - v0) & 31);
-            float x[4] = {x4[u].x, x4[u].y, x4[u].z, x4[u].w};
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                float y = ((word >> e) & 1u) ? penalise(x[e], p) : x[e];
-                consider(b, y, v + e);
+                for (int e = 0; e < 4; ++e) {
+                    const float y = ((word >> e) & 1u) ? penalise(x[e], p) : x[e];
+                    consider(e & 1 ? b2 : b, y, v0 + 4 * u + e);
+                }
             }
+            if (beats(b2.v, b2.i, b.v, b.i))
+                b = b2;
         }
     } else {
         for (int v = v0 + tid; v < v1; v += kThreads) {
@@ -149,44 +195,76 @@ penalize_accept_kernel(PenalizeArgs a, TreeParents tree, int n_chunks)
 
     // ---- epilogue: the last CTA sees every chunk's result
     __threadfence();
-    const int warp = tid >> 5, lane = tid & 31;
-    for (int n = warp; n < a.n_tree; n += kThreads / 32) {
-        Best c{-INFINITY, INT_MAX};
-        for (int ch = lane; ch < n_chunks; ch += 32) {
-            Best q;
-            q.v = __ldcg(&part[n * n_chunks + ch].v);
-            q.i = __ldcg(&part[n * n_chunks + ch].i);
-            if (beats(q.v, q.i, c.v, c.i))
-                c = q;
-        }
-        c = warp_best(c);
-        if (lane == 0) {
-            am[n] = c.i;
-            if (a.argmax_out)
-                a.argmax_out[n] = c.i;
-        }
-    }
-    __shared__ int tok[TS_MAX_TREE];
-    for (int i = tid; i < a.n_tree; i += kThreads)
-        tok[i] = a.tree_tokens[i];
+    // every (node, split) result is loaded in one round and folded into its
+    // node with a 64-bit max whose order is that of beats(): the float's
+    // order-preserving bits above the complemented id (larger value, then
+    // lower id)
+    __shared__ unsigned long long node_key[TS_MAX_TREE];
+    for (int n = tid; n < a.n_tree; n += kThreads)
+        node_key[n] = 0ull;
     __syncthreads();
-    if (tid == 0) {
-        // valid[i]: parent valid and token == argmax at the parent
-        unsigned long long valid = 1ull;
-        int depth[TS_MAX_TREE];
-        depth[0] = 0;
-        int best = 0;
-        for (int i = 1; i < a.n_tree; ++i) {
-            const int pa = tree.parent[i];
-            depth[i] = depth[pa] + 1;
-            const bool ok = ((valid >> pa) & 1ull) && tok[i] == am[pa];
-            if (ok) {
-                valid |= 1ull << i;
-                if (depth[i] > depth[best])
-                    best = i;
+    {
+        const int total = a.n_tree * n_chunks;
+        constexpr int kL = 8;   // results per thread in flight
+        for (int base = 0; base < total; base += kThreads * kL) {
+            Best q[kL];
+#pragma unroll
+            for (int u = 0; u < kL; ++u) {
+                const int k = base + u * kThreads + tid;
+                if (k < total) {
+                    q[u].v = __ldcg(&part[k].v);
+                    q[u].i = __ldcg(&part[k].i);
+                }
+            }
+#pragma unroll
+            for (int u = 0; u < kL; ++u) {
+                const int k = base + u * kThreads + tid;
+                if (k < total)
+                    atomicMax(&node_key[k / n_chunks], best_key(q[u]));
             }
         }
-        const int len = depth[best];
+    }
+    __syncthreads();
+    for (int n = tid; n < a.n_tree; n += kThreads) {
+        const int id = (int)~(uint32_t)node_key[n];
+        am[n] = id;
+        if (a.argmax_out)
+            a.argmax_out[n] = id;
+    }
+    __shared__ int tok[TS_MAX_TREE], par[TS_MAX_TREE];
+    for (int i = tid; i < a.n_tree; i += kThreads) {
+        tok[i] = a.tree_tokens[i];
+        par[i] = tree.parent[i];
+    }
+    __syncthreads();
+    // Each node checks its own root path: valid when every node on it
+    // carries the argmax at its parent.  The kept node is the deepest valid
+    // one, ties to the lowest index: the largest (depth << 8 | 255 - i).
+    __shared__ int best_key[2];
+    if (tid < 2 * 32) {
+        int key = -1;
+        if (tid < a.n_tree) {
+            int i = tid, d = 0;
+            bool ok = true;
+            while (i != 0) {
+                const int pa = par[i];
+                ok = ok && tok[i] == am[pa];
+                i = pa;
+                ++d;
+            }
+            if (ok)
+                key = (d << 8) | (255 - tid);
+        }
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1)
+            key = max(key, __shfl_xor_sync(0xffffffffu, key, off));
+        if ((tid & 31) == 0)
+            best_key[tid >> 5] = key;
+    }
+    __syncthreads();
+    if (tid == 0) {
+        const int key = max(best_key[0], best_key[1]);
+        const int best = 255 - (key & 255), len = key >> 8;
         int32_t *out = a.accept_out;
         out[0] = len;
         out[1] = am[best];
@@ -195,7 +273,7 @@ penalize_accept_kernel(PenalizeArgs a, TreeParents tree, int n_chunks)
         int nd = best;
         for (int t = len; t >= 0; --t) {
             out[2 + t] = nd;
-            nd = tree.parent[nd];
+            nd = par[nd];
         }
         hdr->tickets[0] = 0u;
     }
@@ -205,16 +283,33 @@ penalize_accept_kernel(PenalizeArgs a, TreeParents tree, int n_chunks)
 
 size_t penalize_workspace_bytes(int n_tree, int vocab)
 {
-    const size_t n_chunks = (size_t)(vocab + kChunk - 1) / kChunk;
-    return kHeaderBytes + align_up(n_chunks * (size_t)n_tree * sizeof(Best), 256);
+    // room for the most splits any device gives (per-split results)
+    return kHeaderBytes + align_up((size_t)kMaxSplits * n_tree * sizeof(Best), 256);
 }
 
-cudaError_t penalize_launch(const PenalizeArgs &a, const TreeParents &parents,
+cudaError_t penalize_launch(const PenalizeArgs &a, const TreeParents &parents, int num_sms,
                             cudaStream_t stream)
 {
-    const int n_chunks = (a.vocab + kChunk - 1) / kChunk;
+    static int per_sm = 0;
+    if (per_sm == 0) {
+        int n = 0;
+        if (cudaFuncSetAttribute(penalize_accept_kernel,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 kMaxChunk * (int)sizeof(float)) != cudaSuccess ||
+            cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, penalize_accept_kernel, kThreads,
+                                                          kMaxChunk * sizeof(float)) !=
+                cudaSuccess ||
+            n < 1) {
+            cudaGetLastError();
+            n = 1;
+        }
+        per_sm = n;
+    }
+    const int chunk = penalize_chunk(a.n_tree, a.vocab, num_sms, per_sm);
+    const int n_chunks = (a.vocab + chunk - 1) / chunk;
     dim3 grid(n_chunks, a.n_tree);
-    penalize_accept_kernel<<<grid, kThreads, 0, stream>>>(a, parents, n_chunks);
+    penalize_accept_kernel<<<grid, kThreads, (size_t)chunk * sizeof(float), stream>>>(
+        a, parents, chunk, n_chunks);
     const cudaError_t e = cudaGetLastError();
     if (e == cudaSuccess)
         count_launches(1);

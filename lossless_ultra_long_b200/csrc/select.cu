@@ -259,6 +259,7 @@ select_gather_kernel(SelectArgs a, int n_chunks, int slice)
     uint32_t *keys = reinterpret_cast<uint32_t *>(dsm + sizeof(P2Shared));
 
     const int rank = (int)cluster.block_rank();
+    const int n_ranks = (int)cluster.num_blocks();
     const int g = blockIdx.y;
     const int G = a.n_heads_q / a.n_heads_kv;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -295,9 +296,9 @@ select_gather_kernel(SelectArgs a, int n_chunks, int slice)
     }
     __syncthreads();
 
-    // scores of this slice -> order-preserving keys in shared memory; four
+    // scores of this slice -> order-preserving keys in shared memory; eight
     // positions per thread per step so their loads are in flight together
-    constexpr int kU = 4;
+    constexpr int kU = 8;
     for (int nb = p0 + tid; nb < p1; nb += kP2Threads * kU) {
         float sc[kU];
 #pragma unroll
@@ -360,7 +361,7 @@ select_gather_kernel(SelectArgs a, int n_chunks, int slice)
             const int b = 255 - tid;
             int x = 0;
             if (tid < 256)
-                for (int r = 0; r < kClusterCtas; ++r)
+                for (int r = 0; r < n_ranks; ++r)
                     x += cluster.map_shared_rank(&sh.hist[0], r)[b];
             int above;
             block_exclusive_scan(x, sh.scan, above);
@@ -450,8 +451,8 @@ select_gather_kernel(SelectArgs a, int n_chunks, int slice)
     const int li = tid % LPR;
     __threadfence_block();
     const int my_rows = min(kept_total, n_keep - kept_before);
-    // four rows per thread per step: their K and V loads are in flight together
-    constexpr int kG = 4;
+    // eight rows per thread per step: their K and V loads are in flight together
+    constexpr int kG = 8;
     for (int t0 = tid / LPR; t0 < my_rows; t0 += rows_per_pass * kG) {
         uint4 kv[kG], vv[kG];
         int slot[kG];
@@ -483,7 +484,9 @@ SelPlan make_sel_plan(int n_heads_kv, int n_ctx, int num_sms)
 {
     SelPlan p;
     // three 64 KB-ring CTAs fit an SM: one wave of them over all heads
-    int want = (num_sms * 3 + n_heads_kv - 1) / n_heads_kv;
+    // (rounded down, so that no CTA waits for a second wave)
+    int want = (num_sms * 3) / n_heads_kv;
+    want = want < 1 ? 1 : want;
     const int min_chunk = 512;
     int chunk = (n_ctx + want - 1) / want;
     chunk = chunk < min_chunk ? min_chunk : chunk;

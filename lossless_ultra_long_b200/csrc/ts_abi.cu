@@ -232,7 +232,8 @@ int ts_penalize_accept(const float *logits, int n_tree, int vocab, const int32_t
     a.accept_out = accept_out;
     a.workspace = workspace;
     a.workspace_bytes = workspace_bytes;
-    const cudaError_t e = ts::penalize_launch(a, tp, static_cast<cudaStream_t>(stream));
+    const cudaError_t e =
+        ts::penalize_launch(a, tp, current_num_sms(), static_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? TS_OK : TS_ERR_CUDA;
 }
 

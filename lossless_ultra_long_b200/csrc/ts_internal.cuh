@@ -97,7 +97,7 @@ struct PenalizeArgs {
 };
 
 size_t penalize_workspace_bytes(int n_tree, int vocab);
-cudaError_t penalize_launch(const PenalizeArgs &a, const TreeParents &parents,
+cudaError_t penalize_launch(const PenalizeArgs &a, const TreeParents &parents, int num_sms,
                             cudaStream_t stream);
 
 }  // namespace ts

@@ -331,12 +331,19 @@ def test_penalize_unplanted_logits_and_penalty_flips(oracle_mod):
 
 
 def test_penalize_edges(oracle_mod):
-    # exact ties across chunks, NaN, -inf, a single-node tree, T = 64
+    # exact ties across chunks, NaN, -inf, signed zeros, a single-node tree, T = 64
     lg = np.full((64, 20000), -np.inf, np.float32)
     lg[:, 19999] = 3.0
     lg[:, 8192] = 3.0
     lg[3, :] = np.nan
     lg[5, 17] = 3.0
+    # signed zeros tie (-0 == +0): the lower id wins either way round
+    lg[7, :] = -1.0
+    lg[7, 9000] = -0.0
+    lg[7, 12] = 0.0
+    lg[9, :] = -1.0
+    lg[9, 30] = -0.0
+    lg[9, 15000] = 0.0
     win = np.array([19999, 19999, 0], np.int32)
     parent = I.bfs_tree(64)
     _, am = run_pen(lg, win, 1.0, parent, np.zeros(64, np.int32))
