@@ -240,8 +240,8 @@ __device__ int block_exclusive_scan(int x, int *scratch, int &excl)
     return total;
 }
 
-struct P2Shared {
-    int hist[256];
+struct alignas(16) P2Shared {
+    int hist[2][256];          // pass p uses hist[p & 1]
     int scan[72];
     float head_w[kMaxGroup];   // 1 / (G * Z_h)
     float head_m[kMaxGroup];
@@ -296,33 +296,61 @@ select_gather_kernel(SelectArgs a, int n_chunks, int slice)
     }
     __syncthreads();
 
-    // scores of this slice -> order-preserving keys in shared memory; eight
-    // positions per thread per step so their loads are in flight together
-    constexpr int kU = 8;
-    for (int nb = p0 + tid; nb < p1; nb += kP2Threads * kU) {
-        float sc[kU];
+    // scores of this slice -> order-preserving keys in shared memory
+    if ((N & 3) == 0) {
+        // four consecutive positions per thread, one 16-byte load per head
+        // (the slice is a multiple of 4, so p0 and p1 are too)
+        for (int nb = p0 + 4 * tid; nb < p1; nb += 4 * kP2Threads) {
+            float4 sv[kMaxGroup];
 #pragma unroll
-        for (int u = 0; u < kU; ++u)
-            sc[u] = 0.f;
-        for (int h = 0; h < G; ++h) {
-            const float *row = s_all + (size_t)(g * G + h) * N;
-            float sv[kU];
+            for (int h = 0; h < kMaxGroup; ++h)
+                if (h < G)
+                    sv[h] = __ldcg(reinterpret_cast<const float4 *>(
+                        s_all + (size_t)(g * G + h) * N + nb));
+            float sc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+            for (int h = 0; h < kMaxGroup; ++h)
+                if (h < G) {
+                    const float m = sh.head_m[h], wgt = sh.head_w[h];
+                    sc[0] += exp2f(sv[h].x - m) * wgt;
+                    sc[1] += exp2f(sv[h].y - m) * wgt;
+                    sc[2] += exp2f(sv[h].z - m) * wgt;
+                    sc[3] += exp2f(sv[h].w - m) * wgt;
+                }
+            *reinterpret_cast<uint4 *>(&keys[nb - p0]) =
+                make_uint4(order_key(sc[0]), order_key(sc[1]), order_key(sc[2]), order_key(sc[3]));
+            if (a.scores_out)
+                *reinterpret_cast<float4 *>(a.scores_out + (size_t)g * N + nb) =
+                    make_float4(sc[0], sc[1], sc[2], sc[3]);
+        }
+    } else {
+        // eight positions per thread per step so their loads are in flight together
+        constexpr int kU = 8;
+        for (int nb = p0 + tid; nb < p1; nb += kP2Threads * kU) {
+            float sc[kU];
+#pragma unroll
+            for (int u = 0; u < kU; ++u)
+                sc[u] = 0.f;
+            for (int h = 0; h < G; ++h) {
+                const float *row = s_all + (size_t)(g * G + h) * N;
+                float sv[kU];
+#pragma unroll
+                for (int u = 0; u < kU; ++u) {
+                    const int n = nb + u * kP2Threads;
+                    sv[u] = n < p1 ? __ldcg(row + n) : 0.f;
+                }
+#pragma unroll
+                for (int u = 0; u < kU; ++u)
+                    sc[u] += exp2f(sv[u] - sh.head_m[h]) * sh.head_w[h];
+            }
 #pragma unroll
             for (int u = 0; u < kU; ++u) {
                 const int n = nb + u * kP2Threads;
-                sv[u] = n < p1 ? __ldcg(row + n) : 0.f;
-            }
-#pragma unroll
-            for (int u = 0; u < kU; ++u)
-                sc[u] += exp2f(sv[u] - sh.head_m[h]) * sh.head_w[h];
-        }
-#pragma unroll
-        for (int u = 0; u < kU; ++u) {
-            const int n = nb + u * kP2Threads;
-            if (n < p1) {
-                keys[n - p0] = order_key(sc[u]);
-                if (a.scores_out)
-                    a.scores_out[(size_t)g * N + n] = sc[u];
+                if (n < p1) {
+                    keys[n - p0] = order_key(sc[u]);
+                    if (a.scores_out)
+                        a.scores_out[(size_t)g * N + n] = sc[u];
+                }
             }
         }
     }
@@ -336,8 +364,11 @@ select_gather_kernel(SelectArgs a, int n_chunks, int slice)
         const int c0 = max(p0, a.n_sink);
         for (int pass = 0; pass < 4; ++pass) {
             const int shift = 24 - 8 * pass;
+            // this buffer was last read by other CTAs two passes ago, before
+            // they reached the previous pass's cluster barrier
+            int *hist = sh.hist[pass & 1];
             for (int b = tid; b < 256; b += kP2Threads)
-                sh.hist[b] = 0;
+                hist[b] = 0;
             __syncthreads();
             // positive scores share their leading bytes, so most lanes hit
             // the same bin: lanes with equal bins add once, by their leader
@@ -351,7 +382,7 @@ select_gather_kernel(SelectArgs a, int n_chunks, int slice)
                     const uint32_t bin = (key >> shift) & 255u;
                     const unsigned same = __match_any_sync(act, bin);
                     if ((lane) == __ffs(same) - 1)
-                        atomicAdd(&sh.hist[bin], __popc(same));
+                        atomicAdd(&hist[bin], __popc(same));
                 }
             }
             cluster.sync();
@@ -362,14 +393,14 @@ select_gather_kernel(SelectArgs a, int n_chunks, int slice)
             int x = 0;
             if (tid < 256)
                 for (int r = 0; r < n_ranks; ++r)
-                    x += cluster.map_shared_rank(&sh.hist[0], r)[b];
+                    x += cluster.map_shared_rank(hist, r)[b];
             int above;
             block_exclusive_scan(x, sh.scan, above);
             if (tid < 256 && above < need && need <= above + x) {
                 sh.bcast[0] = b;
                 sh.bcast[1] = above;
             }
-            cluster.sync();   // every CTA has read the histograms; digit is in bcast
+            __syncthreads();   // the digit is in bcast
             const int d = sh.bcast[0];
             need -= sh.bcast[1];
             prefix |= (uint32_t)d << shift;
@@ -492,7 +523,7 @@ SelPlan make_sel_plan(int n_heads_kv, int n_ctx, int num_sms)
     chunk = chunk < min_chunk ? min_chunk : chunk;
     p.chunk = chunk;
     p.n_chunks = (n_ctx + chunk - 1) / chunk;
-    p.slice = (n_ctx + kClusterCtas - 1) / kClusterCtas;
+    p.slice = ((n_ctx + kClusterCtas - 1) / kClusterCtas + 3) / 4 * 4;
     return p;
 }
 
@@ -555,7 +586,7 @@ int select_supported(int n_heads_q, int n_heads_kv, int head_dim, int n_ctx)
         return 0;
     if (head_dim == 64 && G > 8)
         return 0;
-    return (n_ctx + kClusterCtas - 1) / kClusterCtas <= kMaxSlice;
+    return ((n_ctx + kClusterCtas - 1) / kClusterCtas + 3) / 4 * 4 <= kMaxSlice;
 }
 
 size_t select_workspace_bytes(int n_heads_q, int n_heads_kv, int head_dim, int n_ctx,
