@@ -93,6 +93,7 @@ struct Bars {
     uint64_t s_free[2];   // block b's softmax warps hold S_b in registers
     uint64_t sm_done;     // every softmax warp wrote its P^T rows
     uint64_t pv_done;     // one commit per PV
+    uint64_t pv_issued[2];  // PV(t) is in the tensor queue (slot t & 1)
     uint64_t o_final;     // committed once, after the last PV
     uint64_t drain[2];    // each issuing thread's own MMAs, before TMEM is freed
     uint32_t tmem_base;
@@ -266,6 +267,8 @@ attn_t128_kernel(const __grid_constant__ CUtensorMap tmap_k,
         mbar_init(smem_addr(&bar->s_free[1]), u1 > 0 ? 4 * u1 : 1);
         mbar_init(smem_addr(&bar->sm_done), 4 * U);
         mbar_init(smem_addr(&bar->pv_done), 1);
+        mbar_init(smem_addr(&bar->pv_issued[0]), 1);
+        mbar_init(smem_addr(&bar->pv_issued[1]), 1);
         mbar_init(smem_addr(&bar->o_final), 1);
         mbar_init(smem_addr(&bar->drain[0]), 1);
         mbar_init(smem_addr(&bar->drain[1]), 1);
@@ -380,6 +383,13 @@ attn_t128_kernel(const __grid_constant__ CUtensorMap tmap_k,
                     const int s = t % SK;
                     if (!wait_bounded(smem_addr(&bar->full_k[s]), (t / SK) & 1, abort, hdr))
                         break;
+                    // QK(t) enters the tensor queue after PV(t-2): the softmax
+                    // warps wait for PV(t-2) before writing P^T(t-1), while
+                    // S(t) is only read after they finish tile t-1.  PV(t)
+                    // needs S(t), so slot t & 1 has one open phase here.
+                    if (t >= 2 && !wait_bounded(smem_addr(&bar->pv_issued[t & 1]),
+                                                ((t - 2) >> 1) & 1, abort, hdr))
+                        break;
                     const uint64_t kd = kd0 + (uint64_t)s * kStageStep;
                     bool ok = true;
                     for (int b = 0; b < NB; ++b) {
@@ -436,6 +446,7 @@ attn_t128_kernel(const __grid_constant__ CUtensorMap tmap_k,
                     if (t == n_tiles - 1)
                         mma_commit(smem_addr(&bar->o_final));
                     mma_commit(smem_addr(&bar->empty_v[s]));
+                    mbar_arrive(smem_addr(&bar->pv_issued[t & 1]));
                 }
             }
             // every MMA this thread issued has finished before TMEM is released
@@ -666,11 +677,10 @@ attn_t128_combine_kernel(AttnArgs a, TreeMasks masks, int n_split, int tiles_per
     float acc[4] = {0.f, 0.f, 0.f, 0.f};
     float L = 0.f;
     if (!any) {
+        // one pass: splits in batches of kB whose loads are in flight
+        // together, folded into a running (M, L, acc)
+        constexpr int kB = 9;
         float M = -INFINITY;
-        for (int s = 0; s < n_split; ++s)
-            M = fmaxf(M, __ldcg(ws_ml + ((size_t)s * rows_all + row) * 2));
-        // splits in batches of kB: the batch's loads are in flight together
-        constexpr int kB = 6;
         for (int s0 = 0; s0 < n_split; s0 += kB) {
             float2 ml[kB];
             float4 x[kB];
@@ -687,15 +697,27 @@ attn_t128_combine_kernel(AttnArgs a, TreeMasks masks, int n_split, int tiles_per
                     x[u] = make_float4(0.f, 0.f, 0.f, 0.f);
                 }
             }
+            float Mb = M;
+#pragma unroll
+            for (int u = 0; u < kB; ++u)
+                Mb = fmaxf(Mb, ml[u].x);
+            if (Mb == -INFINITY)
+                continue;
+            const float fa = M == -INFINITY ? 0.f : exp2f(M - Mb);
+            L *= fa;
+#pragma unroll
+            for (int e = 0; e < 4; ++e)
+                acc[e] *= fa;
 #pragma unroll
             for (int u = 0; u < kB; ++u) {
-                const float w = ml[u].x == -INFINITY ? 0.f : exp2f(ml[u].x - M);
+                const float w = ml[u].x == -INFINITY ? 0.f : exp2f(ml[u].x - Mb);
                 L += w * ml[u].y;
                 acc[0] += w * x[u].x;
                 acc[1] += w * x[u].y;
                 acc[2] += w * x[u].z;
                 acc[3] += w * x[u].w;
             }
+            M = Mb;
         }
     } else {
         // fold the splits one by one into a running (M, L, acc)
