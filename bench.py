@@ -52,6 +52,24 @@ def dist_env():
     return rank, world, local
 
 
+def max_over_ranks(x: float, world: int, device) -> float:
+    """The largest of every rank's x (a duration): the job is as slow as its
+    slowest replica.  Single process: x itself."""
+    if world <= 1:
+        return float(x)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(steps: int, world: int, ms_max: float) -> float:
+    """Whole-job steps/s: every rank ran `steps` steps of its own problem
+    (weak scaling) and the job took the slowest rank's ms_max."""
+    return world * steps / (ms_max / 1e3)
+
+
 def workload():
     from lossless_ultra_long_b200 import inputs as I
     return I.LLAMA8B_100K
@@ -346,17 +364,12 @@ def run_ours(args):
     ms_total = t0.elapsed_time(t1)
     # in-graph pairs: only the graphs the timed loop replayed
     attn_ms = [a.elapsed_time(b) for a, b in (ev_in[:min(K, kGraphs)] if in_graph else ev)]
-    ms_t = torch.tensor([ms_total], device=dev)
-    if world > 1:
-        dist.all_reduce(ms_t, op=dist.ReduceOp.MAX)
-    ms_max = float(ms_t.item())
+    ms_max = max_over_ranks(ms_total, world, dev)
 
     # end to end through the public API: per step, pinned host inputs are
     # copied in, the four calls run, and the results are read back
     e2e = run_e2e(torch, L, st, w, dev, stream, args.e2e_steps)
-    e2e_t = torch.tensor([e2e["ms_per_step"]], device=dev)
-    if world > 1:
-        dist.all_reduce(e2e_t, op=dist.ReduceOp.MAX)
+    e2e_ms = max_over_ranks(e2e["ms_per_step"], world, dev)
 
     out = None
     if rank == 0:
@@ -365,8 +378,8 @@ def run_ours(args):
         byts = attn_bytes(w.n_heads_q, w.n_heads_kv, w.head_dim, w.n_ctx, w.n_tree)
         flops = attn_flops(w.n_heads_q, w.head_dim, w.n_ctx, w.n_tree)
         achieved = byts / attn_avg_s / 1e9
-        value = world * K / (ms_max / 1e3)
-        e2e_value = world * 1e3 / float(e2e_t.item())
+        value = job_throughput(K, world, ms_max)
+        e2e_value = job_throughput(1, world, e2e_ms)
         out = {
             "metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": world,
             "steps": K, "warmup": args.warmup, "ms_per_step": round(ms_max / K, 5),
@@ -452,10 +465,14 @@ def run_e2e(torch, L, st, w, dev, stream, steps):
 class OracleSample:
     """The fp64 oracle on a bounded sample of one step, scaled to a full step.
 
-    attn_rows of the T*Hq verify-attention rows, the importance select of KV
-    head 0 over the first sel_positions context positions, draft_rows of the
-    draft pass's rows, pen_nodes of the tree nodes' penalty/argmax, and the
-    acceptance walk; each part's time is scaled by the share it sampled."""
+    attn_rows of the T*Hq verify-attention rows, the importance select of
+    every KV head over the first sel_positions context positions, draft_rows
+    of the draft pass's rows, pen_nodes of the tree nodes' penalty/argmax,
+    and the acceptance walk; each part's time is scaled by the share it
+    sampled.  The oracle spreads rows, heads and nodes over the host's
+    threads, so every sampled part keeps all of them busy (at least one row
+    or node per thread, all heads) and the scaling does not charge idle
+    threads to the full step."""
 
     def __init__(self, w, attn_rows, sel_positions, draft_rows, pen_nodes):
         import oracle
@@ -477,8 +494,8 @@ class OracleSample:
         self.win = I.gen_window(w)
         self.rng = np.random.default_rng(0)
         self.sample = (f"{attn_rows} of {w.n_tree * w.n_heads_q} verify-attention rows; "
-                       f"importance select of KV head 0 over {self.sel_positions} of "
-                       f"{w.n_ctx} positions (x{w.n_heads_kv} heads); {draft_rows} of "
+                       f"importance select of all {w.n_heads_kv} KV heads over "
+                       f"{self.sel_positions} of {w.n_ctx} positions; {draft_rows} of "
                        f"{w.draft_tree * w.n_heads_q} draft-pass rows; penalty/argmax of "
                        f"{pen_nodes} of {w.n_tree} nodes; acceptance; scaled to one step")
 
@@ -493,11 +510,11 @@ class OracleSample:
         t_attn = (time.perf_counter() - t0) * rows_total / self.attn_rows
         g, n = w.group, self.sel_positions
         t0 = time.perf_counter()
-        sc = o.importance_scores(self.q[0, :g], self.k[:1], n, g)
+        sc = o.importance_scores(self.q[0], self.k, n, w.n_heads_q)
         idx = o.select_topk(sc, w.n_sink, w.budget)
-        o.gather_rows(self.k[:1], idx)
-        o.gather_rows(self.v[:1], idx)
-        t_sel = (time.perf_counter() - t0) * w.n_heads_kv * w.n_ctx / n
+        o.gather_rows(self.k, idx)
+        o.gather_rows(self.v, idx)
+        t_sel = (time.perf_counter() - t0) * w.n_ctx / n
         drows = w.draft_tree * w.n_heads_q
         dsel = self.rng.choice(drows, size=self.draft_rows, replace=False)
         t0 = time.perf_counter()
@@ -533,7 +550,10 @@ def run_reference(args):
         return None
     w = workload()
     K = max(1, args.steps)
-    smp = OracleSample(w, attn_rows=2, sel_positions=12800, draft_rows=4, pen_nodes=2)
+    thr = oracle_threads()
+    smp = OracleSample(w, attn_rows=max(8, thr), sel_positions=8192,
+                       draft_rows=min(w.draft_tree * w.n_heads_q, max(8, thr)),
+                       pen_nodes=min(w.n_tree, max(8, thr)))
     for _ in range(min(args.warmup, 1)):
         smp.seconds_per_step()
     secs = [smp.seconds_per_step() for _ in range(K)]
