@@ -246,20 +246,31 @@ class Step:
         self.ws_sel = L.new_workspace(L.kv_importance_select_workspace_size(hq, hkv, d, w.n_ctx),
                                       dev)
         self.ws_pen = L.new_workspace(L.penalize_accept_workspace_size(w.n_tree, w.vocab), dev)
+        self.side = torch.cuda.Stream(device=dev)
 
     def attn(self):
         self.L.tree_verify_attn(self.q, self.k, self.v, self.w.n_ctx, self.parent, out=self.out,
                                 workspace=self.ws_attn)
 
     def rest(self):
-        w, L = self.w, self.L
+        """Select, then the draft pass over the partial cache it builds; the
+        penalty/accept call depends on neither and runs beside them on a
+        second stream (the select's cluster kernel leaves most SMs idle)."""
+        w, L, torch = self.w, self.L, self.torch
+        main = torch.cuda.current_stream()
+        self.side.wait_stream(main)   # fork: the side stream depends on what came before
         L.kv_importance_select(self.q[0], self.k, self.v, w.n_ctx, w.n_sink, w.budget,
                                k_partial=self.kp, v_partial=self.vp, idx_out=self.idx,
                                workspace=self.ws_sel)
+        # enqueued after the select so that the score pass's one-wave grid
+        # starts first and the penalty CTAs fill the SMs it leaves
+        with torch.cuda.stream(self.side):
+            L.penalize_accept(self.logits, self.window, w.penalty, self.parent, self.tokens,
+                              argmax_out=self.argmax, accept_out=self.accept,
+                              workspace=self.ws_pen)
         L.tree_verify_attn(self.dq, self.kp, self.vp, self.n_keep, self.draft_parent,
                            out=self.dout, workspace=self.ws_draft)
-        L.penalize_accept(self.logits, self.window, w.penalty, self.parent, self.tokens,
-                          argmax_out=self.argmax, accept_out=self.accept, workspace=self.ws_pen)
+        main.wait_stream(self.side)
 
     def step(self):
         self.attn()
@@ -389,7 +400,8 @@ def run_ours(args):
                        "head_dim": w.head_dim, "n_ctx": w.n_ctx, "n_tree": w.n_tree,
                        "tree": "3-ary BFS depth 3", "step": "verify attn + importance select "
                        "(64+4032) + 4-node draft attn over the partial cache + penalty/accept "
-                       "(V=128256, W=1024)", "l2": "inputs larger than L2 (420 MB KV per step)",
+                       "(V=128256, W=1024); penalty/accept on a second stream beside the "
+                       "select and draft pass", "l2": "inputs larger than L2 (420 MB KV per step)",
                        "parallelism": f"replicas x{world}", "graphs": True,
                        "attn_timing": ("events inside the step graph, last %d steps" % kGraphs
                                        if in_graph else "events around the attention graph")},
