@@ -128,10 +128,6 @@ __host__ __device__ inline TcLayout tc_layout(int nb, int rows)
 
 // P = 2^(x * scale - m) for the 64 scores of one row, packed to bf16 pairs;
 // returns the sum of the rounded values (what the PV product will use).
-// POLY: one pair in four goes through the FMA-pipe polynomial instead of
-// MUFU ex2 (masked tiles, whose -inf scores the polynomial clamps instead of
-// zeroing, use MUFU only).
-template <bool POLY>
 __device__ __forceinline__ float exp_pack_tile(const float (&x)[64], float scale, float neg_m,
                                                uint32_t (&pk)[32])
 {
@@ -144,16 +140,9 @@ __device__ __forceinline__ float exp_pack_tile(const float (&x)[64], float scale
     uint64_t ls2[4] = {0ull, 0ull, 0ull, 0ull};
 #pragma unroll
     for (int j = 0; j < 32; ++j) {
-        float e0, e1;
-        if (POLY && (j & 3) == 3) {
-            unpack2(exp2_poly2(y[j]), e0, e1);
-        } else {
-            float y0, y1;
-            unpack2(y[j], y0, y1);
-            e0 = ex2(y0);
-            e1 = ex2(y1);
-        }
-        __nv_bfloat162 h = __floats2bfloat162_rn(e0, e1);
+        float y0, y1;
+        unpack2(y[j], y0, y1);
+        __nv_bfloat162 h = __floats2bfloat162_rn(ex2(y0), ex2(y1));
         const uint32_t hb = *reinterpret_cast<uint32_t *>(&h);
         pk[j] = hb;
         ls2[j & 3] = add2(ls2[j & 3],
@@ -453,7 +442,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_constant
                     bar->rescale_tile[buf] = t + 1;
                 const float neg_m = m_ref == -INFINITY ? 0.f : -m_ref;
                 uint32_t pk[32];
-                l += exp_pack_tile<false>(x, a.scale_log2, neg_m, pk);
+                l += exp_pack_tile(x, a.scale_log2, neg_m, pk);
                 // P^T(t) reuses the buffer of P^T(t-2): PV(t-2) must be done.
                 // PV(t-4), the buffer's previous user, finished before this
                 // warp wrote P^T(t-2), so pv_done[buf] has exactly one phase

@@ -160,21 +160,7 @@ __device__ __forceinline__ void tc_fence_after()
     asm volatile("tcgen05.fence::after_thread_sync;\n" ::: "memory");
 }
 
-// D(tmem) (+)= A(smem desc) * B(smem desc)
-__device__ __forceinline__ void mma_ss(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc,
-                                       uint32_t accumulate)
-{
-    asm volatile(
-        "{\n"
-        " .reg .pred p;\n"
-        " setp.ne.b32 p, %4, 0;\n"
-        " tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n"
-        "}\n" ::"r"(d),
-        "l"(a), "l"(b), "r"(idesc), "r"(accumulate)
-        : "memory");
-}
-
-// Same, with the accumulate flag fixed at compile time.
+// D(tmem) (+)= A(smem desc) * B(smem desc), accumulate flag fixed at compile time.
 template <int ACC>
 __device__ __forceinline__ void mma_ss_c(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc)
 {
@@ -185,20 +171,6 @@ __device__ __forceinline__ void mma_ss_c(uint32_t d, uint64_t a, uint64_t b, uin
         " tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n"
         "}\n" ::"r"(d),
         "l"(a), "l"(b), "r"(idesc), "n"(ACC)
-        : "memory");
-}
-
-// D(tmem) (+)= A(tmem) * B(smem desc)
-__device__ __forceinline__ void mma_ts(uint32_t d, uint32_t a_tmem, uint64_t b, uint32_t idesc,
-                                       uint32_t accumulate)
-{
-    asm volatile(
-        "{\n"
-        " .reg .pred p;\n"
-        " setp.ne.b32 p, %4, 0;\n"
-        " tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n"
-        "}\n" ::"r"(d),
-        "r"(a_tmem), "l"(b), "r"(idesc), "r"(accumulate)
         : "memory");
 }
 
@@ -222,28 +194,6 @@ __device__ __forceinline__ void mma_commit(uint32_t bar)
 {
     asm volatile(
         "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n" ::"r"(bar)
-        : "memory");
-}
-
-// 16 consecutive 32-bit TMEM columns of this thread's lane; waits for them.
-__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16])
-{
-    asm volatile(
-        "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
-        "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];\n"
-        "tcgen05.wait::ld.sync.aligned;\n"
-        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
-        : "r"(taddr)
-        : "memory");
-}
-
-// 16 consecutive 32-bit TMEM columns of this thread's lane; not waited.
-__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16])
-{
-    asm volatile(
-        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
-        "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};\n" ::"r"(taddr),
-        "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
         : "memory");
 }
 
@@ -363,34 +313,6 @@ __device__ __forceinline__ uint64_t add2(uint64_t a, uint64_t b)
     uint64_t d;
     asm("add.rn.f32x2 %0, %1, %2;\n" : "=l"(d) : "l"(a), "l"(b));
     return d;
-}
-
-// 2^y for a pair, on the FMA pipe instead of the MUFU unit.  Cody-Waite
-// style split y = j + f with j = nearest integer (found by adding
-// 1.5 * 2^23, which leaves j in the low mantissa bits) and f in
-// [-1/2, 1/2]; 2^f by a degree-3 polynomial fitted here for minimum relative
-// error on that interval (max 7.5e-5, well below the bf16 rounding that
-// follows); 2^j by adding j to the exponent field.  y is clamped at -126,
-// so results below 2^-126 come out as tiny non-negative numbers.
-__device__ __forceinline__ uint64_t exp2_poly2(uint64_t y)
-{
-    constexpr float kRound = 12582912.0f;  // 1.5 * 2^23
-    constexpr float c0 = 0.99992805719f, c1 = 0.69326096773f, c2 = 0.24261115491f,
-                    c3 = 0.05517166853f;
-    float y0, y1;
-    unpack2(y, y0, y1);
-    const uint64_t yc = pack2(fmaxf(y0, -126.f), fmaxf(y1, -126.f));
-    const uint64_t t = add2(yc, pack2(kRound, kRound));
-    const uint64_t j = add2(t, pack2(-kRound, -kRound));
-    const uint64_t f = fma2(j, pack2(-1.f, -1.f), yc);
-    uint64_t p = fma2(f, pack2(c3, c3), pack2(c2, c2));
-    p = fma2(p, f, pack2(c1, c1));
-    p = fma2(p, f, pack2(c0, c0));
-    float p0, p1, t0, t1;
-    unpack2(p, p0, p1);
-    unpack2(t, t0, t1);
-    return pack2(__uint_as_float(__float_as_uint(p0) + (__float_as_uint(t0) << 23)),
-                 __uint_as_float(__float_as_uint(p1) + (__float_as_uint(t1) << 23)));
 }
 
 // Shared-memory matrix descriptor, 128-byte swizzle, sm_100 version bits.
