@@ -125,7 +125,8 @@ class ClockSampler:
         self.pci = pci_bus_id
         self.samples, self.reason_bits, self.max_mhz = [], 0, None
         self.thread = self.proc = None
-        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_bench_{os.getpid()}.csv")
+        import tempfile
+        self.path = os.path.join(tempfile.gettempdir(), f"clocks_bench_{os.getpid()}.csv")
 
     def _nvml_loop(self, nv, h):
         import time
