@@ -44,15 +44,15 @@
 // [384, 512).
 //
 // The reference max of a row is fixed at the first tile where the row sees
-// anything, and never moves: fp32 accumulation has room for weights up to
-// 2^64 (times the head dim, the values and the split length), so nothing
-// has to be rescaled while a row's scores stay within 64 (base-2) above
-// its first tile's maximum -- which takes a score jump of about 44 nats
-// inside one split.  This keeps the softmax warps free of any per-tile
-// agreement with each other.  A split in which some row does exceed the
-// headroom raises a flag; the combine kernel then recomputes that split's
-// partial for the affected head exactly (fp32, online softmax on CUDA
-// cores) instead of reading it.
+// anything, and never moves, so the softmax warps need no per-tile
+// agreement with each other and no per-tile maximum at all.  fp32 has room
+// for it: a row's weights are at most its sum l, and while l <= 2^80 the
+// accumulated O^T stays below 2^80 * max|V|, far from overflow (a score
+// rise of about 55 nats inside one split would be needed to exceed it).  A
+// split in which some row's l ends above 2^80 (or not a number) raises a
+// flag; the combine kernel then recomputes that split's partial for the
+// affected head exactly (fp32, online softmax on CUDA cores) instead of
+// reading it.
 // Each split leaves an unnormalised partial (acc, m, l) and its flag; the
 // combine kernel always runs.
 //
@@ -81,7 +81,7 @@ constexpr int kQCol = 192;                   // Q of block 0: 128 bf16 = 64 colu
 constexpr int kSCol = 256;                   // S_b: 128 columns from kSCol + 128 b
 constexpr int kTmemCols = 512;
 constexpr int kQ1Bytes = kBlockM * kD * 2;   // Q of block 1 in shared memory: 32 KB
-constexpr float kHeadroomLog2 = 64.f;        // weights stay below 2^64 of the reference
+constexpr float kMaxRowSum = 1.2089258196146292e24f;   // 2^80: bound on a row's weight sum
 constexpr size_t kSmemLimit = 232448;        // dynamic shared memory per CTA
 
 struct Bars {
@@ -476,7 +476,7 @@ attn_t128_kernel(const __grid_constant__ CUtensorMap tmap_k,
         const uint32_t p_addr = smem_addr(sP);
         const uint32_t p_scratch = p_addr + (uint32_t)r_pad * 256;
         float mA = -INFINITY, mB = -INFINITY, lA = 0.f, lB = 0.f;
-        bool over = false, ok = true;
+        bool ok = true;
         for (int t = 0; t < n_tiles; ++t) {
             if (!warp_wait_bounded(smem_addr(&bar->s_full[b]), t & 1, abort, hdr)) {
                 ok = false;
@@ -514,12 +514,12 @@ attn_t128_kernel(const __grid_constant__ CUtensorMap tmap_k,
                         r[4 * (k >> 1) + 2 + (k & 1)] = __float_as_uint(-INFINITY);
                 }
             }
-            // this thread's part of each row's tile max, in base-2 units
-            const float xA = row_max(r, 0) * a.scale_log2;
-            const float xB = row_max(r, 2) * a.scale_log2;
             // a row that has seen nothing yet takes this tile's max as its
-            // reference (its O^T column and l are still zero)
+            // reference (its O^T column and l are still zero); afterwards
+            // the maxima are not needed
             if (__any_sync(0xffffffffu, mA == -INFINITY || mB == -INFINITY)) {
+                const float xA = row_max(r, 0) * a.scale_log2;
+                const float xB = row_max(r, 2) * a.scale_log2;
                 float yA = fmaxf(xA, __shfl_xor_sync(0xffffffffu, xA, 1));
                 float yB = fmaxf(xB, __shfl_xor_sync(0xffffffffu, xB, 1));
                 yA = fmaxf(yA, __shfl_xor_sync(0xffffffffu, yA, 2));
@@ -529,7 +529,6 @@ attn_t128_kernel(const __grid_constant__ CUtensorMap tmap_k,
                 if (mB == -INFINITY)
                     mB = yB;
             }
-            over |= (vA && xA > mA + kHeadroomLog2) || (vB && xB > mB + kHeadroomLog2);
 
             uint32_t pA[16], pB[16];
             {
@@ -557,13 +556,16 @@ attn_t128_kernel(const __grid_constant__ CUtensorMap tmap_k,
             if (lane == 0)
                 mbar_arrive(smem_addr(&bar->sm_done));
         }
-        if (__any_sync(0xffffffffu, over) && lane == 0)
-            bar->overflow = 1;
         // ---- (m, l) of each row (four threads' partial sums), then O^T
         lA += __shfl_xor_sync(0xffffffffu, lA, 1);
         lB += __shfl_xor_sync(0xffffffffu, lB, 1);
         lA += __shfl_xor_sync(0xffffffffu, lA, 2);
         lB += __shfl_xor_sync(0xffffffffu, lB, 2);
+        // every weight of a row is at most its sum: a sum past 2^80 (or not a
+        // number) flags the split for the exact recompute
+        const bool over = (vA && !(lA <= kMaxRowSum)) || (vB && !(lB <= kMaxRowSum));
+        if (__any_sync(0xffffffffu, over) && lane == 0)
+            bar->overflow = 1;
         const int rows_all = a.n_tree * a.n_heads_q;
         float *ws_o =
             reinterpret_cast<float *>(reinterpret_cast<char *>(a.workspace) + kHeaderBytes);

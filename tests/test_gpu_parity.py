@@ -161,10 +161,11 @@ def test_attn_rising_scores_move_the_reference_max(oracle_mod, hq, hkv, t):
 def test_attn_score_jump_past_headroom(oracle_mod, hq, hkv, t):
     """Two context positions whose K is 120.0 in every dimension: rows with a
     positive query sum see a score about 15 * sum(q) (base 2) above
-    everything else -- far past the 64 of headroom the tcgen05 kernel keeps
-    above a row's first-tile max, and past the fp32 range for many rows.
-    Those splits must come out exact all the same (they are recomputed);
-    sampled rows, plus every row of node 0, against the oracle."""
+    everything else -- far past the 2^80 bound the tcgen05 kernel keeps on a
+    row's weight sum relative to its first-tile max, and past the fp32
+    range for many rows.  Those splits must come out exact all the same
+    (they are recomputed); sampled rows, plus every row of node 0, against
+    the oracle."""
     w = I.Workload("jump", hq, hkv, 128, 12000, t, seed=70 + hq)
     q = I.gen_q(w)
     k, v = I.gen_kv(w)
