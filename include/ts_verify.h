@@ -63,6 +63,8 @@ typedef enum {
 
 /* Largest draft tree, in nodes (ancestor sets are 64-bit masks). */
 #define TS_MAX_TREE 64
+/* query heads per KV head supported by the importance select */
+#define TS_MAX_SELECT_GROUP 8
 
 /* Static description of a status code; never NULL. */
 TS_API const char *ts_status_string(int status);
@@ -175,6 +177,43 @@ TS_API int ts_kv_importance_select(const void *q_last, const void *k_cache, cons
                             float *scores_out, int32_t *idx_out, void *k_partial,
                             void *v_partial, int64_t partial_cap, void *workspace,
                             size_t workspace_bytes, void *stream);
+
+/*
+ * The same verify attention, also leaving the root node's scores for the
+ * importance select: root_scores_out[h][n] = log2(e) * softmax_scale *
+ * q[0][h] . k[h / G][n] for n in [0, n_ctx), fp32 [n_heads_q, n_ctx]
+ * (device, 4-byte aligned; 16-byte aligned when n_ctx is a multiple of 4,
+ * for ts_kv_select_from_scores).  The root's query rows are the ones the
+ * importance score is defined on, and the verify pass computes these
+ * products anyway: handing them to ts_kv_select_from_scores spares the
+ * select's own pass over K.  G = n_heads_q / n_heads_kv must be at most
+ * TS_MAX_SELECT_GROUP (else TS_ERR_UNSUPPORTED).  Every other argument, the
+ * workspace and `out` are as for ts_tree_verify_attn, and `out` is the
+ * same.
+ */
+TS_API int ts_tree_verify_attn_root_scores(const void *q, const void *k_cache,
+                                           const void *v_cache, int64_t kv_cap, int n_heads_q,
+                                           int n_heads_kv, int head_dim, int n_ctx, int n_tree,
+                                           const int32_t *parent, float softmax_scale,
+                                           float *out, float *root_scores_out, void *workspace,
+                                           size_t workspace_bytes, void *stream);
+
+/*
+ * The partial-KV update of ts_kv_importance_select from root scores given
+ * by the caller (as left by ts_tree_verify_attn_root_scores): the group-mean
+ * softmax over [0, n_ctx) of root_scores (base 2), then the same sink +
+ * top-budget selection and gather.  root_scores: device fp32 [n_heads_q,
+ * n_ctx], read only.  The other arguments are as for
+ * ts_kv_importance_select (no query rows, no scale); the workspace needs
+ * ts_kv_select_from_scores_workspace_size() bytes.
+ */
+TS_API size_t ts_kv_select_from_scores_workspace_size(void);
+TS_API int ts_kv_select_from_scores(const float *root_scores, const void *k_cache,
+                                    const void *v_cache, int64_t kv_cap, int n_heads_q,
+                                    int n_heads_kv, int head_dim, int n_ctx, int n_sink,
+                                    int budget, float *scores_out, int32_t *idx_out,
+                                    void *k_partial, void *v_partial, int64_t partial_cap,
+                                    void *workspace, size_t workspace_bytes, void *stream);
 
 /*
  * Contextual penalty, per-node target argmax and the longest accepted path.

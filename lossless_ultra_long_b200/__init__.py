@@ -24,7 +24,8 @@ STATUS = {0: "TS_OK", 1: "TS_ERR_INVALID_ARG", 2: "TS_ERR_UNSUPPORTED", 3: "TS_E
 EXPORTS = ("ts_status_string", "ts_version", "ts_tree_verify_attn_workspace_size",
            "ts_tree_verify_attn", "ts_kv_importance_select_workspace_size",
            "ts_kv_importance_select", "ts_penalize_accept_workspace_size", "ts_penalize_accept",
-           "ts_workspace_status", "ts_kernel_launch_count")
+           "ts_workspace_status", "ts_kernel_launch_count", "ts_tree_verify_attn_root_scores",
+           "ts_kv_select_from_scores_workspace_size", "ts_kv_select_from_scores")
 
 
 class TsError(RuntimeError):
@@ -54,6 +55,14 @@ def _lib():
         lib.ts_tree_verify_attn.restype = i32
         lib.ts_tree_verify_attn.argtypes = [P, P, P, i64, i32, i32, i32, i32, i32, P, f32, P, P,
                                             sz, P]
+        lib.ts_tree_verify_attn_root_scores.restype = i32
+        lib.ts_tree_verify_attn_root_scores.argtypes = [P, P, P, i64, i32, i32, i32, i32, i32, P,
+                                                        f32, P, P, P, sz, P]
+        lib.ts_kv_select_from_scores_workspace_size.restype = sz
+        lib.ts_kv_select_from_scores_workspace_size.argtypes = []
+        lib.ts_kv_select_from_scores.restype = i32
+        lib.ts_kv_select_from_scores.argtypes = [P, P, P, i64, i32, i32, i32, i32, i32, i32, P, P,
+                                                 P, P, i64, P, sz, P]
         lib.ts_kv_importance_select_workspace_size.restype = sz
         lib.ts_kv_importance_select_workspace_size.argtypes = [i32, i32, i32, i32]
         lib.ts_kv_importance_select.restype = i32
@@ -119,11 +128,14 @@ def tree_verify_attn_workspace_size(n_heads_q, n_heads_kv, head_dim, n_ctx, n_tr
 
 
 def tree_verify_attn(q, k_cache, v_cache, n_ctx: int, parent, out=None, workspace=None,
-                     softmax_scale: float | None = None, stream=None):
+                     softmax_scale: float | None = None, stream=None, root_scores_out=None):
     """Tree-masked attention (``ts_tree_verify_attn``).
 
     q: bf16 [T, Hq, D]; k_cache, v_cache: bf16 [Hkv, kv_cap, D]; parent: host
-    int32 [T].  Returns fp32 [T, Hq, D].
+    int32 [T].  Returns fp32 [T, Hq, D].  With ``root_scores_out`` (fp32
+    [Hq, n_ctx]) it also leaves the root node's base-2 scores over the
+    context (``ts_tree_verify_attn_root_scores``), the input of
+    :func:`kv_select_from_scores`.
     """
     _check_dev("q", q, torch.bfloat16)
     _check_dev("k_cache", k_cache, torch.bfloat16)
@@ -141,10 +153,20 @@ def tree_verify_attn(q, k_cache, v_cache, n_ctx: int, parent, out=None, workspac
     if len(par) != t:
         raise ValueError("parent must have one entry per tree node")
     scale = float(d) ** -0.5 if softmax_scale is None else float(softmax_scale)
-    rc = _lib().ts_tree_verify_attn(_ptr(q), _ptr(k_cache), _ptr(v_cache), cap, hq, hkv, d,
-                                    int(n_ctx), t, par_p, scale, _ptr(out), _ptr(workspace),
-                                    workspace.numel() * workspace.element_size(), _stream(stream))
-    _raise(rc, "ts_tree_verify_attn")
+    ws_bytes = workspace.numel() * workspace.element_size()
+    if root_scores_out is None:
+        rc = _lib().ts_tree_verify_attn(_ptr(q), _ptr(k_cache), _ptr(v_cache), cap, hq, hkv, d,
+                                        int(n_ctx), t, par_p, scale, _ptr(out), _ptr(workspace),
+                                        ws_bytes, _stream(stream))
+        _raise(rc, "ts_tree_verify_attn")
+        return out
+    _check_dev("root_scores_out", root_scores_out, torch.float32)
+    if tuple(root_scores_out.shape) != (hq, int(n_ctx)):
+        raise ValueError("root_scores_out must be [Hq, n_ctx]")
+    rc = _lib().ts_tree_verify_attn_root_scores(
+        _ptr(q), _ptr(k_cache), _ptr(v_cache), cap, hq, hkv, d, int(n_ctx), t, par_p, scale,
+        _ptr(out), _ptr(root_scores_out), _ptr(workspace), ws_bytes, _stream(stream))
+    _raise(rc, "ts_tree_verify_attn_root_scores")
     return out
 
 
@@ -191,6 +213,51 @@ def kv_importance_select(q_last, k_cache, v_cache, n_ctx: int, n_sink: int, budg
         int(budget), scale, _ptr(scores_out), _ptr(idx_out), _ptr(k_partial), _ptr(v_partial),
         k_partial.shape[1], _ptr(workspace), workspace.numel(), _stream(stream))
     _raise(rc, "ts_kv_importance_select")
+    return idx_out, k_partial, v_partial, scores_out
+
+
+def kv_select_from_scores_workspace_size() -> int:
+    return int(_lib().ts_kv_select_from_scores_workspace_size())
+
+
+def kv_select_from_scores(root_scores, k_cache, v_cache, n_ctx: int, n_sink: int, budget: int,
+                          k_partial=None, v_partial=None, idx_out=None, scores_out=None,
+                          workspace=None, stream=None, want_scores: bool = False):
+    """The partial-KV update from root scores left by the verify attention
+    (``ts_kv_select_from_scores``).  root_scores: fp32 [Hq, n_ctx] (base 2).
+
+    Returns ``(idx [Hkv, n_keep] int32, k_partial, v_partial, scores or None)``.
+    """
+    _check_dev("root_scores", root_scores, torch.float32)
+    _check_dev("k_cache", k_cache, torch.bfloat16)
+    _check_dev("v_cache", v_cache, torch.bfloat16)
+    hq, n = root_scores.shape
+    if n != int(n_ctx):
+        raise ValueError("root_scores must be [Hq, n_ctx]")
+    hkv, cap, d = k_cache.shape
+    n_keep = min(n_ctx, n_sink + budget)
+    dev = root_scores.device
+    if k_partial is None:
+        k_partial = torch.empty((hkv, n_keep, d), dtype=torch.bfloat16, device=dev)
+    if v_partial is None:
+        v_partial = torch.empty_like(k_partial)
+    if idx_out is None:
+        idx_out = torch.empty((hkv, n_keep), dtype=torch.int32, device=dev)
+    if want_scores and scores_out is None:
+        scores_out = torch.empty((hkv, n_ctx), dtype=torch.float32, device=dev)
+    for name, t, dt in (("k_partial", k_partial, torch.bfloat16),
+                        ("v_partial", v_partial, torch.bfloat16),
+                        ("idx_out", idx_out, torch.int32)):
+        _check_dev(name, t, dt)
+    if scores_out is not None:
+        _check_dev("scores_out", scores_out, torch.float32)
+    if workspace is None:
+        workspace = new_workspace(kv_select_from_scores_workspace_size(), dev)
+    rc = _lib().ts_kv_select_from_scores(
+        _ptr(root_scores), _ptr(k_cache), _ptr(v_cache), cap, hq, hkv, d, int(n_ctx),
+        int(n_sink), int(budget), _ptr(scores_out), _ptr(idx_out), _ptr(k_partial),
+        _ptr(v_partial), k_partial.shape[1], _ptr(workspace), workspace.numel(), _stream(stream))
+    _raise(rc, "ts_kv_select_from_scores")
     return idx_out, k_partial, v_partial, scores_out
 
 

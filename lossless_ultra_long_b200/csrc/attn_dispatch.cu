@@ -32,13 +32,31 @@ size_t attn_workspace_bytes(int n_heads_q, int n_heads_kv, int head_dim, int n_c
 cudaError_t attn_launch(const AttnArgs &a, const TreeMasks &masks, int num_sms,
                         cudaStream_t stream)
 {
-    if (a.scale_log2 > 0.f) {
-        if (attn_t128_eligible(a.n_heads_q, a.n_heads_kv, a.head_dim, a.n_ctx, a.n_tree))
-            return attn_t128_launch(a, masks, num_sms, stream);
-        if (attn_tc_eligible(a.n_heads_q, a.n_heads_kv, a.head_dim, a.n_ctx, a.n_tree))
-            return attn_tc_launch(a, masks, num_sms, stream);
-    }
-    return attn_mma_launch(a, masks, num_sms, stream);
+    if (a.scale_log2 > 0.f &&
+        attn_t128_eligible(a.n_heads_q, a.n_heads_kv, a.head_dim, a.n_ctx, a.n_tree))
+        return attn_t128_launch(a, masks, num_sms, stream);   // leaves root scores itself
+    cudaError_t e;
+    if (a.scale_log2 > 0.f &&
+        attn_tc_eligible(a.n_heads_q, a.n_heads_kv, a.head_dim, a.n_ctx, a.n_tree))
+        e = attn_tc_launch(a, masks, num_sms, stream);
+    else
+        e = attn_mma_launch(a, masks, num_sms, stream);
+    if (e != cudaSuccess || a.root_scores == nullptr || a.n_ctx == 0)
+        return e;
+    // the other kernels do not leave root scores: the select's score pass does
+    SelectArgs sa = {};
+    sa.q_last = a.q;   // node 0's rows [Hq, D]
+    sa.k = a.k;
+    sa.v = a.v;
+    sa.kv_cap = a.kv_cap;
+    sa.n_heads_q = a.n_heads_q;
+    sa.n_heads_kv = a.n_heads_kv;
+    sa.head_dim = a.head_dim;
+    sa.n_ctx = a.n_ctx;
+    sa.scale_log2 = a.scale_log2;
+    sa.workspace = a.workspace;
+    sa.workspace_bytes = a.workspace_bytes;
+    return select_score_pass_launch(sa, a.root_scores, num_sms, stream);
 }
 
 }  // namespace ts

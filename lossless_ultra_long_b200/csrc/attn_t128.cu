@@ -109,10 +109,21 @@ constexpr size_t kAuxBytes = (sizeof(Aux) + 1023) / 1024 * 1024;
 struct Layout {
     int r_pad;  // rows rounded up to 16: N of the PV product
     int stages_k, stages_v;
-    size_t q1_off, p_off, k_off, v_off, aux_off, smem_bytes;
+    size_t q1_off, p_off, k_off, v_off, aux_off, rs_off, smem_bytes;
 };
 
-__host__ __device__ inline Layout t128_layout(int rows)
+// Shared memory that stages the root node's scores for bulk copies (two
+// tiles of the G root rows), when the call asks for them and every row of
+// them starts on a 16-byte boundary; 0 when they are stored directly.
+__host__ __device__ inline int t128_rs_bytes(const AttnArgs &a)
+{
+    const bool bulk = a.root_scores != nullptr &&
+                      (reinterpret_cast<uintptr_t>(a.root_scores) & 15) == 0 &&
+                      (a.n_ctx & 3) == 0;
+    return bulk ? 2 * (a.n_heads_q / a.n_heads_kv) * kTileN * 4 : 0;
+}
+
+__host__ __device__ inline Layout t128_layout(int rows, int rs_bytes)
 {
     Layout L;
     L.r_pad = (rows + 15) / 16 * 16;
@@ -121,14 +132,15 @@ __host__ __device__ inline Layout t128_layout(int rows)
     // P^T: positions 0-63 then 64-127, each r_pad rows of 128 bytes; then
     // 1 KB that rows past the query rows are written to
     L.k_off = L.p_off + (size_t)L.r_pad * 256 + 1024;
-    const size_t fixed = 1024 + L.k_off + kAuxBytes;
+    const size_t fixed = 1024 + L.k_off + kAuxBytes + rs_bytes;
     int stages = (int)((kSmemLimit - fixed) / kStageBytes);
     stages = stages > 2 * kMaxStages ? 2 * kMaxStages : stages;
     L.stages_v = 2;
     L.stages_k = stages - 2 > kMaxStages ? kMaxStages : stages - 2;
     L.v_off = L.k_off + (size_t)L.stages_k * kStageBytes;
     L.aux_off = L.v_off + (size_t)L.stages_v * kStageBytes;
-    L.smem_bytes = 1024 + L.aux_off + kAuxBytes;
+    L.rs_off = L.aux_off + kAuxBytes;
+    L.smem_bytes = 1024 + L.rs_off + rs_bytes;
     return L;
 }
 
@@ -230,7 +242,8 @@ attn_t128_kernel(const __grid_constant__ CUtensorMap tmap_k,
     const int rq0 = (R0 + 3) / 4, rq1 = (R1 + 3) / 4;  // rows per lane quarter
     const int u0 = (rq0 + 15) / 16, u1 = (rq1 + 15) / 16;
     const int U = u0 + u1;  // softmax warps per lane quarter (at most 3)
-    const Layout lay = t128_layout(R);
+    const int rs_bytes = t128_rs_bytes(a);
+    const Layout lay = t128_layout(R, rs_bytes);
     const int SK = lay.stages_k, SV = lay.stages_v, r_pad = lay.r_pad;
 
     extern __shared__ unsigned char smem_raw[];
@@ -476,6 +489,12 @@ attn_t128_kernel(const __grid_constant__ CUtensorMap tmap_k,
         const uint32_t p_addr = smem_addr(sP);
         const uint32_t p_scratch = p_addr + (uint32_t)r_pad * 256;
         float mA = -INFINITY, mB = -INFINITY, lA = 0.f, lB = 0.f;
+        // root rows (node 0: rows 0..G-1) held by this thread and this warp;
+        // the first lane of a row's quad copies its staged scores out
+        const bool rootA = vA && nA < G, rootB = vB && nB < G;
+        const bool rs_warp =
+            a.root_scores != nullptr && __any_sync(0xffffffffu, rootA || rootB);
+        const bool rs_issue = rs_bytes != 0 && (lane & 3) == 0 && (rootA || rootB);
         bool ok = true;
         for (int t = 0; t < n_tiles; ++t) {
             if (!warp_wait_bounded(smem_addr(&bar->s_full[b]), t & 1, abort, hdr)) {
@@ -492,6 +511,64 @@ attn_t128_kernel(const __grid_constant__ CUtensorMap tmap_k,
                 mbar_arrive(smem_addr(&bar->s_free[b]));
             // raw scores; the scale (> 0) is applied inside the exponent
             const int pos0 = (t_begin + t) * kTileN;
+            // the root node's rows (0..G-1) leave their context scores, base
+            // 2, for the importance select
+            if (rs_warp && pos0 < a.n_ctx) {
+                if (rs_bytes != 0) {
+                    // staged in shared memory (one buffer per tile parity)
+                    // and written out by bulk copies, so that no global
+                    // store sits ahead of this warp's barrier arrivals
+                    const uint32_t buf =
+                        smem_addr(base + lay.rs_off) + (uint32_t)((t & 1) * G * kTileN * 4);
+                    if (rs_issue)
+                        bulk_wait_read<1>();   // the copy out of this buffer two tiles ago
+                    __syncwarp();
+#pragma unroll
+                    for (int h = 0; h < 2; ++h) {
+                        if (h ? rootB : rootA) {
+                            const uint32_t row =
+                                buf + (uint32_t)((h ? nB : nA) * kTileN * 4 + c0 * 4);
+#pragma unroll
+                            for (int jj = 0; jj < 16; ++jj)
+                                st_shared_v2(row + 32 * jj,
+                                             __float_as_uint(__uint_as_float(r[4 * jj + 2 * h]) *
+                                                             a.scale_log2),
+                                             __float_as_uint(__uint_as_float(r[4 * jj + 2 * h + 1]) *
+                                                             a.scale_log2));
+                        }
+                    }
+                    fence_proxy_async_smem();
+                    __syncwarp();
+                    if (rs_issue) {
+                        const uint32_t bytes = (uint32_t)min(kTileN, a.n_ctx - pos0) * 4;
+#pragma unroll
+                        for (int h = 0; h < 2; ++h) {
+                            const int n = h ? nB : nA;
+                            if (h ? rootB : rootA)
+                                bulk_store(a.root_scores + (size_t)(g * G + n) * a.n_ctx + pos0,
+                                           buf + (uint32_t)(n * kTileN * 4), bytes);
+                        }
+                        bulk_commit();
+                    }
+                } else {
+#pragma unroll
+                    for (int h = 0; h < 2; ++h) {
+                        if (h ? rootB : rootA) {
+                            float *dst = a.root_scores + (size_t)(g * G + (h ? nB : nA)) * a.n_ctx;
+#pragma unroll
+                            for (int jj = 0; jj < 16; ++jj) {
+#pragma unroll
+                                for (int e = 0; e < 2; ++e) {
+                                    const int pos = pos0 + 8 * jj + c0 + e;
+                                    if (pos < a.n_ctx)
+                                        dst[pos] =
+                                            __uint_as_float(r[4 * jj + 2 * h + e]) * a.scale_log2;
+                                }
+                            }
+                        }
+                    }
+                }
+            }
             if (pos0 + kTileN > a.n_ctx) {
                 // visibility of this thread's 32 positions (entry k = 2 jj + e
                 // is position pos0 + 8 jj + c0 + e) for its two rows
@@ -556,6 +633,8 @@ attn_t128_kernel(const __grid_constant__ CUtensorMap tmap_k,
             if (lane == 0)
                 mbar_arrive(smem_addr(&bar->sm_done));
         }
+        if (rs_issue)
+            bulk_wait_all();   // shared memory must outlive the copies out of it
         // ---- (m, l) of each row (four threads' partial sums), then O^T
         lA += __shfl_xor_sync(0xffffffffu, lA, 1);
         lB += __shfl_xor_sync(0xffffffffu, lB, 1);
@@ -807,7 +886,7 @@ cudaError_t attn_t128_launch(const AttnArgs &a, const TreeMasks &masks, int num_
     if (!encode_kv_map(&mk, a.k, rows, a.kv_cap, a.n_heads_kv, kTileN) ||
         !encode_kv_map(&mv, a.v, rows, a.kv_cap, a.n_heads_kv, kTileN))
         return cudaErrorInvalidValue;
-    const Layout lay = t128_layout((a.n_heads_q / a.n_heads_kv) * a.n_tree);
+    const Layout lay = t128_layout((a.n_heads_q / a.n_heads_kv) * a.n_tree, t128_rs_bytes(a));
     static const cudaError_t attr = cudaFuncSetAttribute(
         attn_t128_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemLimit);
     if (attr != cudaSuccess)

@@ -41,7 +41,7 @@ namespace {
 constexpr int kClusterCtas = 8;
 constexpr int kP2Threads = 512;
 constexpr int kMaxSlice = 48 * 1024;   // positions per CTA held in shared memory
-constexpr int kMaxGroup = 8;
+constexpr int kMaxGroup = TS_MAX_SELECT_GROUP;
 
 // ------------------------------------------------------------------ pass 1
 constexpr int kP1Rows = 64;     // key rows per pipeline stage
@@ -71,7 +71,7 @@ __device__ __forceinline__ void mma_16816(float (&d)[4], const uint32_t (&a)[4],
 template <int D>
 __global__ void __launch_bounds__(kP1Threads)
 score_logits_kernel(const __grid_constant__ CUtensorMap tmap_k, SelectArgs a, int chunk,
-                    int n_chunks)
+                    int n_chunks, float *s_out, float2 *part_out)
 {
     using namespace sm100;
     constexpr int kBoxes = D / 64;
@@ -92,7 +92,6 @@ score_logits_kernel(const __grid_constant__ CUtensorMap tmap_k, SelectArgs a, in
     const int n1 = min(n0 + chunk, a.n_ctx);
     const int n_tiles = (n1 - n0 + kP1Rows - 1) / kP1Rows;
     WorkspaceHeader *hdr = reinterpret_cast<WorkspaceHeader *>(a.workspace);
-    float *s_out = reinterpret_cast<float *>(reinterpret_cast<char *>(a.workspace) + kHeaderBytes);
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < kP1Stages; ++s) {
@@ -182,7 +181,7 @@ score_logits_kernel(const __grid_constant__ CUtensorMap tmap_k, SelectArgs a, in
     }
     __syncthreads();
     // merge the running (max, sum) of every lane that holds head h
-    if (threadIdx.x < G) {
+    if (part_out != nullptr && threadIdx.x < G) {
         const int h = threadIdx.x, e = h & 1;
         float M = -INFINITY;
         for (int t = 0; t < kP1Warps * 32; ++t)
@@ -192,8 +191,7 @@ score_logits_kernel(const __grid_constant__ CUtensorMap tmap_k, SelectArgs a, in
         for (int t = 0; t < kP1Warps * 32; ++t)
             if (2 * (t & 3) == (h & ~1) && red_m[t][e] != -INFINITY)
                 L += red_l[t][e] * exp2f(red_m[t][e] - M);
-        float2 *pp = reinterpret_cast<float2 *>(s_out + (size_t)a.n_heads_q * a.n_ctx);
-        pp[(size_t)(g * G + h) * n_chunks + c] = make_float2(M, L);
+        part_out[(size_t)(g * G + h) * n_chunks + c] = make_float2(M, L);
     }
 }
 
@@ -245,13 +243,14 @@ struct alignas(16) P2Shared {
     int scan[72];
     float head_w[kMaxGroup];   // 1 / (G * Z_h)
     float head_m[kMaxGroup];
+    float2 slice_ml[kMaxGroup];  // this CTA's (max, sum) per head over its slice
     int counts[4];             // [0] equal-to-threshold, [1] kept
     int bcast[4];
 };
 
 template <int D>
 __global__ void __launch_bounds__(kP2Threads, 1)
-select_gather_kernel(SelectArgs a, int n_chunks, int slice)
+select_gather_kernel(SelectArgs a, int n_chunks, int slice, const float *__restrict__ s_all)
 {
     cg::cluster_group cluster = cg::this_cluster();
     extern __shared__ __align__(16) unsigned char dsm[];
@@ -269,12 +268,53 @@ select_gather_kernel(SelectArgs a, int n_chunks, int slice)
     const bool keep_all = want >= N;
     const int n_keep = keep_all ? N : (int)want;
 
-    const float *s_all = reinterpret_cast<const float *>(
-        reinterpret_cast<const char *>(a.workspace) + kHeaderBytes);
-    const float2 *part = reinterpret_cast<const float2 *>(s_all + (size_t)a.n_heads_q * N);
+    const float2 *part = reinterpret_cast<const float2 *>(
+        reinterpret_cast<const char *>(a.workspace) + kHeaderBytes +
+        (size_t)a.n_heads_q * N * sizeof(float));
 
-    // softmax max / normaliser per head of the group
-    if (warp < G) {
+    // softmax max / normaliser per head of the group: from the score pass's
+    // per-chunk partials, or, for scores given by the caller, from this
+    // cluster's own pass over them (each CTA its slice, summed across ranks)
+    if (a.root_scores != nullptr) {
+        if (warp < G) {
+            const float *row = s_all + (size_t)(g * G + warp) * N;
+            float m = -INFINITY;
+            for (int n = p0 + lane; n < p1; n += 32)
+                m = fmaxf(m, __ldcg(row + n));
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1)
+                m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+            float l = 0.f;
+            if (m != -INFINITY)
+                for (int n = p0 + lane; n < p1; n += 32)
+                    l += exp2f(__ldcg(row + n) - m);
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1)
+                l += __shfl_xor_sync(0xffffffffu, l, o);
+            if (lane == 0)
+                sh.slice_ml[warp] = make_float2(m, l);
+        }
+        cluster.sync();
+        if (warp < G) {
+            float M = -INFINITY;
+            float2 part_r[kClusterCtas];
+#pragma unroll
+            for (int r = 0; r < kClusterCtas; ++r) {
+                part_r[r] = r < n_ranks ? cluster.map_shared_rank(&sh.slice_ml[0], r)[warp]
+                                        : make_float2(-INFINITY, 0.f);
+                M = fmaxf(M, part_r[r].x);
+            }
+            float L = 0.f;
+#pragma unroll
+            for (int r = 0; r < kClusterCtas; ++r)
+                if (part_r[r].x != -INFINITY)
+                    L += part_r[r].y * exp2f(part_r[r].x - M);
+            if (lane == 0) {
+                sh.head_m[warp] = M;
+                sh.head_w[warp] = 1.f / ((float)G * L);
+            }
+        }
+    } else if (warp < G) {
         const float2 *pp = part + (size_t)(g * G + warp) * n_chunks;
         float M = -INFINITY;
         for (int c = lane; c < n_chunks; c += 32)
@@ -528,7 +568,8 @@ SelPlan make_sel_plan(int n_heads_kv, int n_ctx, int num_sms)
 }
 
 template <int D>
-cudaError_t launch_p1(const SelectArgs &a, const SelPlan &p, cudaStream_t stream)
+cudaError_t launch_p1(const SelectArgs &a, const SelPlan &p, float *s_out, float2 *part_out,
+                      cudaStream_t stream)
 {
     CUtensorMap mk;
     if (!encode_kv_map(&mk, a.k, a.n_ctx, a.kv_cap, a.n_heads_kv, kP1Rows, D))
@@ -539,7 +580,8 @@ cudaError_t launch_p1(const SelectArgs &a, const SelPlan &p, cudaStream_t stream
     if (attr != cudaSuccess)
         return attr;
     dim3 grid(p.n_chunks, a.n_heads_kv);
-    score_logits_kernel<D><<<grid, kP1Threads, smem, stream>>>(mk, a, p.chunk, p.n_chunks);
+    score_logits_kernel<D><<<grid, kP1Threads, smem, stream>>>(mk, a, p.chunk, p.n_chunks, s_out,
+                                                                part_out);
     const cudaError_t e = cudaGetLastError();
     if (e == cudaSuccess)
         count_launches(1);
@@ -549,9 +591,18 @@ cudaError_t launch_p1(const SelectArgs &a, const SelPlan &p, cudaStream_t stream
 template <int D>
 cudaError_t launch_d(const SelectArgs &a, const SelPlan &p, cudaStream_t stream)
 {
-    cudaError_t e = launch_p1<D>(a, p, stream);
-    if (e != cudaSuccess)
-        return e;
+    // scores from the caller, or the score pass into the workspace
+    const float *s_all = a.root_scores;
+    cudaError_t e = cudaSuccess;
+    if (s_all == nullptr) {
+        float *s_ws =
+            reinterpret_cast<float *>(reinterpret_cast<char *>(a.workspace) + kHeaderBytes);
+        e = launch_p1<D>(a, p, s_ws, reinterpret_cast<float2 *>(s_ws + (size_t)a.n_heads_q * a.n_ctx),
+                         stream);
+        if (e != cudaSuccess)
+            return e;
+        s_all = s_ws;
+    }
 
     const size_t smem = sizeof(P2Shared) + (size_t)p.slice * sizeof(uint32_t);
     static const cudaError_t attr_ok = cudaFuncSetAttribute(
@@ -571,13 +622,21 @@ cudaError_t launch_d(const SelectArgs &a, const SelPlan &p, cudaStream_t stream)
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    e = cudaLaunchKernelEx(&cfg, select_gather_kernel<D>, a, p.n_chunks, p.slice);
+    e = cudaLaunchKernelEx(&cfg, select_gather_kernel<D>, a, p.n_chunks, p.slice, s_all);
     if (e == cudaSuccess)
         count_launches(1);
     return e;
 }
 
 }  // namespace
+
+cudaError_t select_score_pass_launch(const SelectArgs &a, float *out, int num_sms,
+                                     cudaStream_t stream)
+{
+    const SelPlan p = make_sel_plan(a.n_heads_kv, a.n_ctx, num_sms);
+    return a.head_dim == 128 ? launch_p1<128>(a, p, out, nullptr, stream)
+                             : launch_p1<64>(a, p, out, nullptr, stream);
+}
 
 int select_supported(int n_heads_q, int n_heads_kv, int head_dim, int n_ctx)
 {

@@ -86,10 +86,12 @@ size_t ts_tree_verify_attn_workspace_size(int n_heads_q, int n_heads_kv, int hea
                                     current_num_sms());
 }
 
-int ts_tree_verify_attn(const void *q, const void *k_cache, const void *v_cache, int64_t kv_cap,
-                        int n_heads_q, int n_heads_kv, int head_dim, int n_ctx, int n_tree,
-                        const int32_t *parent, float softmax_scale, float *out,
-                        void *workspace, size_t workspace_bytes, void *stream)
+namespace {
+
+int attn_call(const void *q, const void *k_cache, const void *v_cache, int64_t kv_cap,
+              int n_heads_q, int n_heads_kv, int head_dim, int n_ctx, int n_tree,
+              const int32_t *parent, float softmax_scale, float *out, float *root_scores,
+              void *workspace, size_t workspace_bytes, void *stream)
 {
     if (!q || !k_cache || !v_cache || !out || !shape_ok(n_heads_q, n_heads_kv, head_dim))
         return TS_ERR_INVALID_ARG;
@@ -127,8 +129,36 @@ int ts_tree_verify_attn(const void *q, const void *k_cache, const void *v_cache,
     a.scale_log2 = softmax_scale * 1.4426950408889634f;
     a.workspace = workspace;
     a.workspace_bytes = workspace_bytes;
+    a.root_scores = root_scores;
     const cudaError_t e = ts::attn_launch(a, masks, sms, static_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? TS_OK : TS_ERR_CUDA;
+}
+
+}  // namespace
+
+int ts_tree_verify_attn(const void *q, const void *k_cache, const void *v_cache, int64_t kv_cap,
+                        int n_heads_q, int n_heads_kv, int head_dim, int n_ctx, int n_tree,
+                        const int32_t *parent, float softmax_scale, float *out,
+                        void *workspace, size_t workspace_bytes, void *stream)
+{
+    return attn_call(q, k_cache, v_cache, kv_cap, n_heads_q, n_heads_kv, head_dim, n_ctx,
+                     n_tree, parent, softmax_scale, out, nullptr, workspace, workspace_bytes,
+                     stream);
+}
+
+int ts_tree_verify_attn_root_scores(const void *q, const void *k_cache, const void *v_cache,
+                                    int64_t kv_cap, int n_heads_q, int n_heads_kv, int head_dim,
+                                    int n_ctx, int n_tree, const int32_t *parent,
+                                    float softmax_scale, float *out, float *root_scores_out,
+                                    void *workspace, size_t workspace_bytes, void *stream)
+{
+    if (!root_scores_out || !aligned(root_scores_out, 4))
+        return TS_ERR_INVALID_ARG;
+    if (shape_ok(n_heads_q, n_heads_kv, head_dim) && n_heads_q / n_heads_kv > TS_MAX_SELECT_GROUP)
+        return TS_ERR_UNSUPPORTED;
+    return attn_call(q, k_cache, v_cache, kv_cap, n_heads_q, n_heads_kv, head_dim, n_ctx,
+                     n_tree, parent, softmax_scale, out, root_scores_out, workspace,
+                     workspace_bytes, stream);
 }
 
 size_t ts_kv_importance_select_workspace_size(int n_heads_q, int n_heads_kv, int head_dim,
@@ -167,7 +197,7 @@ int ts_kv_importance_select(const void *q_last, const void *k_cache, const void 
     if (!workspace_ok(workspace, workspace_bytes, need))
         return TS_ERR_WORKSPACE;
 
-    ts::SelectArgs a;
+    ts::SelectArgs a = {};
     a.q_last = static_cast<const __nv_bfloat16 *>(q_last);
     a.k = static_cast<const __nv_bfloat16 *>(k_cache);
     a.v = static_cast<const __nv_bfloat16 *>(v_cache);
@@ -187,6 +217,60 @@ int ts_kv_importance_select(const void *q_last, const void *k_cache, const void 
     a.workspace = workspace;
     a.workspace_bytes = workspace_bytes;
     const cudaError_t e = ts::select_launch(a, sms, static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? TS_OK : TS_ERR_CUDA;
+}
+
+size_t ts_kv_select_from_scores_workspace_size(void) { return ts::kHeaderBytes; }
+
+int ts_kv_select_from_scores(const float *root_scores, const void *k_cache, const void *v_cache,
+                             int64_t kv_cap, int n_heads_q, int n_heads_kv, int head_dim,
+                             int n_ctx, int n_sink, int budget, float *scores_out,
+                             int32_t *idx_out, void *k_partial, void *v_partial,
+                             int64_t partial_cap, void *workspace, size_t workspace_bytes,
+                             void *stream)
+{
+    if (!root_scores || !k_cache || !v_cache || !idx_out || !k_partial || !v_partial)
+        return TS_ERR_INVALID_ARG;
+    if (!shape_ok(n_heads_q, n_heads_kv, head_dim) || n_ctx < 1 || n_sink < 0 || budget < 0)
+        return TS_ERR_INVALID_ARG;
+    if ((int64_t)n_ctx > kv_cap)
+        return TS_ERR_INVALID_ARG;
+    const int64_t want = (int64_t)n_sink + budget;
+    const int n_keep = want < n_ctx ? (int)want : n_ctx;
+    if (partial_cap < n_keep)
+        return TS_ERR_INVALID_ARG;
+    if (!aligned(root_scores, 4) || !aligned(k_cache, 16) || !aligned(v_cache, 16) ||
+        !aligned(k_partial, 16) || !aligned(v_partial, 16) || !aligned(idx_out, 4) ||
+        (scores_out && !aligned(scores_out, 4)))
+        return TS_ERR_INVALID_ARG;
+    // the score rows are read 16 bytes at a time when n_ctx is a multiple of 4
+    if ((n_ctx & 3) == 0 && !aligned(root_scores, 16))
+        return TS_ERR_INVALID_ARG;
+    if (!head_dim_supported(head_dim) || !ts::select_supported(n_heads_q, n_heads_kv, head_dim, n_ctx))
+        return TS_ERR_UNSUPPORTED;
+    if (!workspace_ok(workspace, workspace_bytes, ts::kHeaderBytes))
+        return TS_ERR_WORKSPACE;
+
+    ts::SelectArgs a = {};
+    a.k = static_cast<const __nv_bfloat16 *>(k_cache);
+    a.v = static_cast<const __nv_bfloat16 *>(v_cache);
+    a.kv_cap = kv_cap;
+    a.n_heads_q = n_heads_q;
+    a.n_heads_kv = n_heads_kv;
+    a.head_dim = head_dim;
+    a.n_ctx = n_ctx;
+    a.n_sink = n_sink;
+    a.budget = budget;
+    a.scores_out = scores_out;
+    a.idx_out = idx_out;
+    a.k_partial = static_cast<__nv_bfloat16 *>(k_partial);
+    a.v_partial = static_cast<__nv_bfloat16 *>(v_partial);
+    a.partial_cap = partial_cap;
+    a.workspace = workspace;
+    a.workspace_bytes = workspace_bytes;
+    a.root_scores = root_scores;
+    const cudaError_t e =
+        ts::select_launch(a, current_num_sms(), static_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? TS_OK : TS_ERR_CUDA;
 }
 

@@ -54,6 +54,9 @@ struct AttnArgs {
     float scale_log2;   // softmax_scale * log2(e)
     void *workspace;
     size_t workspace_bytes;
+    // optional: the root node's scores over the context, base 2
+    // (scale_log2 * q[0, h] . k[g, n]), fp32 [Hq, n_ctx]; null if not wanted
+    float *root_scores;
 };
 
 size_t attn_workspace_bytes(int n_heads_q, int n_heads_kv, int head_dim, int n_ctx, int n_tree,
@@ -76,12 +79,19 @@ struct SelectArgs {
     int64_t partial_cap;
     void *workspace;
     size_t workspace_bytes;
+    // optional: base-2 root scores fp32 [Hq, n_ctx] computed elsewhere (by
+    // the verify attention); when set, the score pass is skipped and q_last
+    // and scale_log2 are unused
+    const float *root_scores;
 };
 
 size_t select_workspace_bytes(int n_heads_q, int n_heads_kv, int head_dim, int n_ctx,
                               int num_sms);
 int select_supported(int n_heads_q, int n_heads_kv, int head_dim, int n_ctx);
 cudaError_t select_launch(const SelectArgs &a, int num_sms, cudaStream_t stream);
+// The score pass alone: base-2 root scores fp32 [Hq, n_ctx] into `out`.
+cudaError_t select_score_pass_launch(const SelectArgs &a, float *out, int num_sms,
+                                     cudaStream_t stream);
 
 struct PenalizeArgs {
     const float *logits;

@@ -225,6 +225,56 @@ def test_select_llama8b_100k_spiked(oracle_mod):
     print(f"indices differing from the fp64 ranking: {diff}")
 
 
+# ------------------------------- select from the verify attention's scores
+@pytest.mark.parametrize("hq,hkv,d,n_ctx,t,n_sink,budget", [
+    (32, 8, 128, 32768, 40, 64, 4032),   # 128-position tcgen05 kernel, 160 rows
+    (16, 16, 128, 9001, 13, 16, 500),    # same kernel, G = 1, odd context
+    (40, 8, 128, 6000, 40, 32, 1000),    # 64-position tcgen05 kernel (200 rows)
+    (8, 2, 64, 3000, 13, 16, 240),       # mma.sync kernel (head_dim 64)
+    (8, 2, 128, 1000, 4, 8, 100),        # mma.sync kernel (short context)
+])
+def test_select_from_verify_attention_scores(oracle_mod, hq, hkv, d, n_ctx, t, n_sink, budget):
+    """The verify attention leaves the root node's scores; the select run on
+    them gives the oracle's importance and selection (same bars as the
+    select's own score pass), and the attention output is unchanged."""
+    w = I.Workload("rs", hq, hkv, d, n_ctx, t, n_sink=n_sink, budget=budget,
+                   seed=n_ctx + hq + t)
+    q = I.gen_q(w)
+    k, v = I.gen_kv(w)
+    dq, dk, dv = dev_bf16(q), dev_bf16(k), dev_bf16(v)
+    plain = L.tree_verify_attn(dq, dk, dv, n_ctx, w.parent())
+    rs = torch.empty((hq, n_ctx), dtype=torch.float32, device="cuda")
+    fused = L.tree_verify_attn(dq, dk, dv, n_ctx, w.parent(), root_scores_out=rs)
+    idx, kp, vp, sc = L.kv_select_from_scores(rs, dk, dv, n_ctx, n_sink, budget,
+                                              want_scores=True)
+    torch.cuda.synchronize()
+    assert torch.equal(plain, fused)
+    # root scores: log2(e) * q[0,h] . k[g,n] / sqrt(D) at sampled positions
+    qf, kf = I.bf16_bits_to_f32(q).astype(np.float64), I.bf16_bits_to_f32(k).astype(np.float64)
+    rng = np.random.default_rng(n_ctx)
+    pos = np.concatenate([[0, n_ctx - 1], rng.integers(0, n_ctx, 64)])
+    g = np.arange(hq) // (hq // hkv)
+    want_rs = np.einsum("hd,hpd->hp", qf[0], kf[g][:, pos]) / np.sqrt(d) * np.log2(np.e)
+    got_rs = rs.cpu().numpy().astype(np.float64)[:, pos]
+    assert np.abs(got_rs - want_rs).max() <= 1e-3 * (1.0 + np.abs(want_rs).max())
+    idx, sc = idx.cpu().numpy(), sc.cpu().numpy()
+    want_sc = oracle_mod.importance_scores(q[0], k, n_ctx, hq)
+    rel = np.abs(sc - want_sc) / np.maximum(want_sc, 1e-30)
+    assert rel.max() <= SCORE_RTOL, f"score rel err {rel.max()}"
+    np.testing.assert_array_equal(idx, oracle_mod.select_topk(sc.astype(np.float64), n_sink, budget))
+    np.testing.assert_array_equal(host_bits(kp), oracle_mod.gather_rows(k, idx))
+    np.testing.assert_array_equal(host_bits(vp), oracle_mod.gather_rows(v, idx))
+
+
+def test_root_scores_reject_large_groups():
+    q = torch.zeros((2, 32, 128), dtype=torch.bfloat16, device="cuda")
+    k = torch.zeros((2, 3000, 128), dtype=torch.bfloat16, device="cuda")
+    rs = torch.empty((32, 2990), dtype=torch.float32, device="cuda")
+    with pytest.raises(L.TsError) as e:
+        L.tree_verify_attn(q, k, k, 2990, [-1, 0], root_scores_out=rs)
+    assert e.value.status == 2
+
+
 @pytest.mark.parametrize("n_ctx,n_sink,budget", [(300, 16, 240), (256, 16, 240), (257, 16, 240),
                                                  (5000, 0, 100), (5000, 64, 0), (9, 4, 2),
                                                  (33000, 64, 4032)])
