@@ -42,6 +42,9 @@ def parse():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=50)
+    ap.add_argument("--select-score-pass", action="store_true",
+                    help="the select scores the context with its own pass over K instead "
+                         "of taking the root node's scores from the verify attention")
     return ap.parse_args()
 
 
@@ -75,10 +78,12 @@ def workload():
     return I.LLAMA8B_100K
 
 
-def attn_bytes(hq, hkv, d, n_ctx, t):
+def attn_bytes(hq, hkv, d, n_ctx, t, root_scores=True):
     """Algorithmic HBM bytes of one tree-verify call: K+V (context + tail, bf16),
-    Q (bf16) and O (fp32)."""
-    return 4 * hkv * d * (n_ctx + t) + 2 * t * hq * d + 4 * t * hq * d
+    Q (bf16) and O (fp32), plus the root node's fp32 scores over the context
+    when the call leaves them for the select."""
+    return (4 * hkv * d * (n_ctx + t) + 2 * t * hq * d + 4 * t * hq * d +
+            (4 * hq * n_ctx if root_scores else 0))
 
 
 def attn_flops(hq, d, n_ctx, t):
@@ -209,7 +214,7 @@ class ClockSampler:
 class Step:
     """Device-resident buffers and the four ABI calls of one verification step."""
 
-    def __init__(self, torch, L, I, w, dev):
+    def __init__(self, torch, L, I, w, dev, fused=True):
         from_bits = lambda b: torch.from_numpy(np.ascontiguousarray(b).view(np.int16)).view(
             torch.bfloat16).to(dev)
         self.torch, self.L, self.w = torch, L, w
@@ -244,14 +249,22 @@ class Step:
                                                                          w.n_tree), dev)
         self.ws_draft = L.new_workspace(L.tree_verify_attn_workspace_size(
             hq, hkv, d, self.n_keep, w.draft_tree), dev)
-        self.ws_sel = L.new_workspace(L.kv_importance_select_workspace_size(hq, hkv, d, w.n_ctx),
-                                      dev)
+        # the root node's base-2 scores, left by the verify attention for the
+        # select (or, unfused, computed by the select's own score pass)
+        self.fused = fused
+        if fused:
+            self.rs = torch.empty((hq, w.n_ctx), dtype=torch.float32, device=dev)
+            self.ws_sel = L.new_workspace(L.kv_select_from_scores_workspace_size(), dev)
+        else:
+            self.rs = None
+            self.ws_sel = L.new_workspace(
+                L.kv_importance_select_workspace_size(hq, hkv, d, w.n_ctx), dev)
         self.ws_pen = L.new_workspace(L.penalize_accept_workspace_size(w.n_tree, w.vocab), dev)
         self.side = torch.cuda.Stream(device=dev)
 
     def attn(self):
         self.L.tree_verify_attn(self.q, self.k, self.v, self.w.n_ctx, self.parent, out=self.out,
-                                workspace=self.ws_attn)
+                                workspace=self.ws_attn, root_scores_out=self.rs)
 
     def rest(self):
         """Select, then the draft pass over the partial cache it builds; the
@@ -260,11 +273,16 @@ class Step:
         w, L, torch = self.w, self.L, self.torch
         main = torch.cuda.current_stream()
         self.side.wait_stream(main)   # fork: the side stream depends on what came before
-        L.kv_importance_select(self.q[0], self.k, self.v, w.n_ctx, w.n_sink, w.budget,
-                               k_partial=self.kp, v_partial=self.vp, idx_out=self.idx,
-                               workspace=self.ws_sel)
-        # enqueued after the select so that the score pass's one-wave grid
-        # starts first and the penalty CTAs fill the SMs it leaves
+        if self.fused:
+            L.kv_select_from_scores(self.rs, self.k, self.v, w.n_ctx, w.n_sink, w.budget,
+                                    k_partial=self.kp, v_partial=self.vp, idx_out=self.idx,
+                                    workspace=self.ws_sel)
+        else:
+            L.kv_importance_select(self.q[0], self.k, self.v, w.n_ctx, w.n_sink, w.budget,
+                                   k_partial=self.kp, v_partial=self.vp, idx_out=self.idx,
+                                   workspace=self.ws_sel)
+        # enqueued after the select so that its cluster kernel starts first
+        # and the penalty CTAs fill the SMs it leaves
         with torch.cuda.stream(self.side):
             L.penalize_accept(self.logits, self.window, w.penalty, self.parent, self.tokens,
                               argmax_out=self.argmax, accept_out=self.accept,
@@ -293,7 +311,7 @@ def run_ours(args):
                                 device_id=dev)
     L.library()
     w = workload()
-    st = Step(torch, L, I, w, dev)
+    st = Step(torch, L, I, w, dev, fused=not args.select_score_pass)
     stream = torch.cuda.Stream(device=dev)
 
     # warm-up eagerly (sets kernel attributes), then capture the step as CUDA
@@ -387,7 +405,8 @@ def run_ours(args):
     if rank == 0:
         hbm, tflops, src = measured_peaks()
         attn_avg_s = statistics.mean(attn_ms) / 1e3
-        byts = attn_bytes(w.n_heads_q, w.n_heads_kv, w.head_dim, w.n_ctx, w.n_tree)
+        byts = attn_bytes(w.n_heads_q, w.n_heads_kv, w.head_dim, w.n_ctx, w.n_tree,
+                          root_scores=st.fused)
         flops = attn_flops(w.n_heads_q, w.head_dim, w.n_ctx, w.n_tree)
         achieved = byts / attn_avg_s / 1e9
         value = job_throughput(K, world, ms_max)
@@ -399,8 +418,9 @@ def run_ours(args):
             "data": "synthetic",
             "config": {"workload": w.name, "n_heads_q": w.n_heads_q, "n_heads_kv": w.n_heads_kv,
                        "head_dim": w.head_dim, "n_ctx": w.n_ctx, "n_tree": w.n_tree,
-                       "tree": "3-ary BFS depth 3", "step": "verify attn + importance select "
-                       "(64+4032) + 4-node draft attn over the partial cache + penalty/accept "
+                       "tree": "3-ary BFS depth 3", "step": ("verify attn (leaving the root's scores) + importance "
+                                "select from them" if st.fused else "verify attn + importance "
+                                "select with its own score pass") + " (64+4032) + 4-node draft attn over the partial cache + penalty/accept "
                        "(V=128256, W=1024); penalty/accept on a second stream beside the "
                        "select and draft pass", "l2": "inputs larger than L2 (420 MB KV per step)",
                        "parallelism": f"replicas x{world}", "graphs": True,
