@@ -106,3 +106,70 @@ def test_workspace_sizes_are_positive_and_zero_for_invalid(lib):
     assert L.kv_importance_select_workspace_size(32, 8, 128, 102400) > 0
     assert L.penalize_accept_workspace_size(40, 128256) > 0
     assert L.penalize_accept_workspace_size(0, 128256) == 0
+
+
+def _root_scores_call(lib, rs=1 << 20, **over):
+    args = dict(q=1 << 20, k=1 << 20, v=1 << 20, kv_cap=100, hq=8, hkv=2, d=64, n_ctx=50, t=4,
+                parent=np.array([-1, 0, 0, 1], np.int32), scale=0.125, out=1 << 20,
+                ws=1 << 20, ws_bytes=1 << 30)
+    args.update(over)
+    P = ctypes.c_void_p
+    return lib.ts_tree_verify_attn_root_scores(
+        P(args["q"]), P(args["k"]), P(args["v"]), args["kv_cap"], args["hq"], args["hkv"],
+        args["d"], args["n_ctx"], args["t"], args["parent"].ctypes.data_as(P), args["scale"],
+        P(args["out"]), P(rs) if rs else None, P(args["ws"]), args["ws_bytes"], None)
+
+
+@pytest.mark.parametrize("rs,over,code", [
+    (0, {}, 1),                          # no scores buffer
+    ((1 << 20) + 2, {}, 1),              # scores not 4-byte aligned
+    (1 << 20, dict(hq=32, hkv=2), 2),    # group of 16 > TS_MAX_SELECT_GROUP
+    (1 << 20, dict(q=0), 1),             # the attention's own checks still apply
+    (1 << 20, dict(d=96), 2),
+    (1 << 20, dict(ws_bytes=16), 3),
+])
+def test_root_scores_attention_rejects_on_host(lib, rs, over, code):
+    assert _root_scores_call(lib, rs, **over) == code
+
+
+def _from_scores_call(lib, **over):
+    args = dict(rs=1 << 20, k=1 << 20, v=1 << 20, kv_cap=1000, hq=8, hkv=2, d=64, n_ctx=1000,
+                n_sink=16, budget=240, scores=None, idx=1 << 20, kp=1 << 20, vp=1 << 20,
+                cap=256, ws=1 << 20, ws_bytes=1 << 20)
+    args.update(over)
+    P = ctypes.c_void_p
+    p = lambda x: P(x) if x else None
+    return lib.ts_kv_select_from_scores(
+        p(args["rs"]), p(args["k"]), p(args["v"]), args["kv_cap"], args["hq"], args["hkv"],
+        args["d"], args["n_ctx"], args["n_sink"], args["budget"], p(args["scores"]),
+        p(args["idx"]), p(args["kp"]), p(args["vp"]), args["cap"], p(args["ws"]),
+        args["ws_bytes"], None)
+
+
+@pytest.mark.parametrize("over,code", [
+    (dict(rs=0), 1),
+    (dict(idx=0), 1),
+    (dict(cap=255), 1),                  # partial cache shorter than n_sink + budget
+    (dict(n_ctx=1001), 1),               # context past the cache capacity
+    (dict(n_sink=-1), 1),
+    (dict(rs=(1 << 20) + 4), 1),         # n_ctx % 4 == 0: rows read 16 bytes at a time
+    (dict(rs=(1 << 20) + 2), 1),
+    (dict(kp=(1 << 20) + 8), 1),
+    (dict(hq=6, hkv=4), 1),
+    (dict(hq=64, hkv=2), 2),             # group of 32
+    (dict(d=96), 2),
+    (dict(ws=0), 3),
+    (dict(ws_bytes=8), 3),
+])
+def test_select_from_scores_rejects_on_host(lib, over, code):
+    assert _from_scores_call(lib, **over) == code
+
+
+def test_select_from_scores_accepts_4_byte_rows_for_ragged_contexts(lib):
+    # n_ctx not a multiple of 4: scores need only 4-byte alignment, so the
+    # call passes every host check; it is not launched here (the workspace
+    # is one byte short of the header, the last check)
+    import lossless_ultra_long_b200 as L
+    need = L.kv_select_from_scores_workspace_size()
+    assert need > 0
+    assert _from_scores_call(lib, rs=(1 << 20) + 4, n_ctx=999, ws_bytes=need - 1) == 3
