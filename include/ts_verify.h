@@ -253,6 +253,63 @@ TS_API int ts_penalize_accept(const float *logits, int n_tree, int vocab, const 
                        void *workspace, size_t workspace_bytes, void *stream);
 
 /*
+ * n-gram reuse table.  TokenSwift drafts with the frequencies of the
+ * n-grams already generated: phrases that occurred often are retrieved and
+ * reused as draft candidates, and the table is updated with the tokens
+ * each verification accepts ("TokenSwift - A framework for accelerating
+ * the generation of ultra-long text", aiboss88.com, "Parallel generation
+ * of multiple tokens and token reuse"; "TokenSwift ... 从小时到分钟",
+ * cloud.tencent.com, the parallel-verification step of the method figure).
+ * The pages fix neither n nor the retrieval rule; this table counts every
+ * run of n consecutive tokens of the generated text (2 <= n <= 8) and
+ * returns, for a first token, its most frequent n-grams: count
+ * descending, ties by continuation in ascending token order.
+ *
+ * Host code on caller-owned HOST memory: one contiguous buffer of
+ * ts_ngram_table_bytes(n, capacity) bytes, 8-byte aligned, holding a
+ * header, `capacity` n-gram slots (open addressing, linear probing) and
+ * `capacity` first-token entries that chain the n-grams sharing a first
+ * token and keep the best 16 of them in order (a top-k of k <= 16 reads
+ * that list; a larger k walks the chain).  The table holds at most capacity - max(1, capacity/8) distinct
+ * n-grams.
+ * Calls on one table must not overlap (no internal locking).  Tokens are
+ * non-negative int32 ids.
+ *
+ *  ts_ngram_table_bytes  bytes for (n, capacity); 0 if n is outside [2, 8]
+ *                        or capacity is not a power of two in [2, 2^31].
+ *  ts_ngram_init         formats `table` (table_bytes must be at least the
+ *                        size above) as an empty table.
+ *  ts_ngram_update       counts the n-grams of `text` that END at one of its
+ *                        last n_new positions (text[0, text_len) is the
+ *                        tail of the generated text; pass at least the n-1
+ *                        tokens before the new ones so that n-grams which
+ *                        straddle them are counted).  All or nothing: if
+ *                        the distinct n-grams not yet present would exceed
+ *                        the fill limit, nothing changes and
+ *                        TS_ERR_WORKSPACE is returned.  A negative token in
+ *                        the scanned range is TS_ERR_INVALID_ARG.
+ *  ts_ngram_topk         the k (1 <= k <= 4096) most frequent n-grams that
+ *                        start with `first`: their n-1 continuation tokens
+ *                        into cont_out [k, n-1] and counts into count_out
+ *                        [k]; *n_found = how many exist (<= k); rows past
+ *                        that get tokens -1 and count 0.
+ *  ts_ngram_count        occurrences of one n-gram (gram[0..n)); 0 if absent.
+ *  ts_ngram_size         distinct n-grams held and total n-grams counted.
+ * Errors: TS_ERR_INVALID_ARG for NULL pointers, an unformatted table, a
+ * table_bytes smaller than the table, or out-of-range sizes.
+ */
+TS_API size_t ts_ngram_table_bytes(int n, int64_t capacity);
+TS_API int ts_ngram_init(void *table, size_t table_bytes, int n, int64_t capacity);
+TS_API int ts_ngram_update(void *table, size_t table_bytes, const int32_t *text,
+                           int64_t text_len, int64_t n_new);
+TS_API int ts_ngram_topk(const void *table, size_t table_bytes, int32_t first, int k,
+                         int32_t *cont_out, int64_t *count_out, int *n_found);
+TS_API int ts_ngram_count(const void *table, size_t table_bytes, const int32_t *gram,
+                          int64_t *count);
+TS_API int ts_ngram_size(const void *table, size_t table_bytes, int64_t *distinct,
+                         int64_t *total);
+
+/*
  * Number of kernels this library has launched in this process (all
  * devices, all entry points); a diagnostic for counting launches.
  */

@@ -25,7 +25,9 @@ EXPORTS = ("ts_status_string", "ts_version", "ts_tree_verify_attn_workspace_size
            "ts_tree_verify_attn", "ts_kv_importance_select_workspace_size",
            "ts_kv_importance_select", "ts_penalize_accept_workspace_size", "ts_penalize_accept",
            "ts_workspace_status", "ts_kernel_launch_count", "ts_tree_verify_attn_root_scores",
-           "ts_kv_select_from_scores_workspace_size", "ts_kv_select_from_scores")
+           "ts_kv_select_from_scores_workspace_size", "ts_kv_select_from_scores",
+           "ts_ngram_table_bytes", "ts_ngram_init", "ts_ngram_update", "ts_ngram_topk",
+           "ts_ngram_count", "ts_ngram_size")
 
 
 class TsError(RuntimeError):
@@ -76,6 +78,18 @@ def _lib():
         lib.ts_kernel_launch_count.argtypes = []
         lib.ts_workspace_status.restype = i32
         lib.ts_workspace_status.argtypes = [P, P, i32]
+        lib.ts_ngram_table_bytes.restype = sz
+        lib.ts_ngram_table_bytes.argtypes = [i32, i64]
+        lib.ts_ngram_init.restype = i32
+        lib.ts_ngram_init.argtypes = [P, sz, i32, i64]
+        lib.ts_ngram_update.restype = i32
+        lib.ts_ngram_update.argtypes = [P, sz, P, i64, i64]
+        lib.ts_ngram_topk.restype = i32
+        lib.ts_ngram_topk.argtypes = [P, sz, ctypes.c_int32, i32, P, P, P]
+        lib.ts_ngram_count.restype = i32
+        lib.ts_ngram_count.argtypes = [P, sz, P, P]
+        lib.ts_ngram_size.restype = i32
+        lib.ts_ngram_size.argtypes = [P, sz, P, P]
         _LIB = lib
     return _LIB
 
@@ -308,3 +322,54 @@ def kernel_launch_count() -> int:
 def workspace_status(workspace, clear: bool = True, stream=None) -> int:
     """Device-side status word of a workspace (synchronises the stream)."""
     return int(_lib().ts_workspace_status(_ptr(workspace), _stream(stream), int(clear)))
+
+
+# --------------------------------------------------------- n-gram reuse table
+class NgramTable:
+    """The n-gram reuse table (``ts_ngram_*``) in a host buffer this object
+    owns.  ``update(text, n_new)`` counts the n-grams of ``text`` that end
+    at its last ``n_new`` tokens; ``topk(first, k)`` returns the most
+    frequent ones starting with ``first`` as ``(continuations [m, n-1],
+    counts [m])``, count descending, ties by continuation ascending."""
+
+    def __init__(self, n: int, capacity: int):
+        import numpy as np
+        nbytes = int(_lib().ts_ngram_table_bytes(int(n), int(capacity)))
+        if nbytes == 0:
+            raise ValueError("n must be in [2, 8] and capacity a power of two >= 2")
+        self.n, self.capacity, self.nbytes = int(n), int(capacity), nbytes
+        self._buf = np.empty((nbytes + 7) // 8, dtype=np.uint64)   # 8-byte aligned
+        self._p = self._buf.ctypes.data_as(ctypes.c_void_p)
+        _raise(_lib().ts_ngram_init(self._p, nbytes, self.n, self.capacity), "ts_ngram_init")
+
+    def update(self, text, n_new: int | None = None) -> None:
+        arr, p = _host_i32(text)
+        n_new = len(arr) if n_new is None else int(n_new)
+        _raise(_lib().ts_ngram_update(self._p, self.nbytes, p, len(arr), n_new),
+               "ts_ngram_update")
+
+    def topk(self, first: int, k: int):
+        import numpy as np
+        cont = np.empty((int(k), self.n - 1), dtype=np.int32)
+        cnt = np.empty(int(k), dtype=np.int64)
+        found = ctypes.c_int(0)
+        _raise(_lib().ts_ngram_topk(self._p, self.nbytes, int(first), int(k),
+                                    cont.ctypes.data_as(ctypes.c_void_p),
+                                    cnt.ctypes.data_as(ctypes.c_void_p), ctypes.byref(found)),
+               "ts_ngram_topk")
+        return cont[:found.value], cnt[:found.value]
+
+    def count(self, gram) -> int:
+        arr, p = _host_i32(gram)
+        if len(arr) != self.n:
+            raise ValueError(f"an n-gram has {self.n} tokens")
+        c = ctypes.c_int64(0)
+        _raise(_lib().ts_ngram_count(self._p, self.nbytes, p, ctypes.byref(c)), "ts_ngram_count")
+        return int(c.value)
+
+    def size(self):
+        """(distinct n-grams held, n-grams counted)."""
+        d, t = ctypes.c_int64(0), ctypes.c_int64(0)
+        _raise(_lib().ts_ngram_size(self._p, self.nbytes, ctypes.byref(d), ctypes.byref(t)),
+               "ts_ngram_size")
+        return int(d.value), int(t.value)
