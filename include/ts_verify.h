@@ -262,17 +262,20 @@ TS_API int ts_penalize_accept(const float *logits, int n_tree, int vocab, const 
  * cloud.tencent.com, the parallel-verification step of the method figure).
  * The pages fix neither n nor the retrieval rule; this table counts every
  * run of n consecutive tokens of the generated text (2 <= n <= 8) and
- * returns, for a first token, its most frequent n-grams: count
- * descending, ties by continuation in ascending token order.
+ * returns, for a prefix of p tokens (1 <= p <= n-1), the most frequent
+ * n-grams that start with it: count descending, ties by continuation in
+ * ascending token order.  p = 1 gives whole-phrase continuations of a
+ * token; p = n-1 gives the next-token counts after the last n-1 tokens.
  *
  * Host code on caller-owned HOST memory: one contiguous buffer of
- * ts_ngram_table_bytes(n, capacity) bytes, 8-byte aligned, holding a
- * header, `capacity` n-gram slots (open addressing, linear probing) and
- * `capacity` first-token entries that chain the n-grams sharing a first
- * token and keep the best 16 of them in order (a top-k of k <= 16 reads
- * that list; a larger k walks the chain).  The table holds at most capacity - max(1, capacity/8) distinct
- * n-grams.
- * Calls on one table must not overlap (no internal locking).  Tokens are
+ * ts_ngram_table_bytes(n, capacity) = 64 + 216 * capacity bytes, 8-byte
+ * aligned, holding a header, `capacity` n-gram slots (open addressing,
+ * linear probing) and two indices of `capacity` entries each, which chain
+ * the n-grams by first token and by first n-1 tokens and keep each
+ * chain's best 16 in order.  A top-k with k <= 16 for p = 1 or p = n-1
+ * reads that list; a larger k, or another p, walks a chain.  The table
+ * holds at most capacity - max(1, capacity/8) distinct n-grams.  Calls on
+ * one table must not overlap (no internal locking).  Tokens are
  * non-negative int32 ids.
  *
  *  ts_ngram_table_bytes  bytes for (n, capacity); 0 if n is outside [2, 8]
@@ -288,11 +291,13 @@ TS_API int ts_penalize_accept(const float *logits, int n_tree, int vocab, const 
  *                        the fill limit, nothing changes and
  *                        TS_ERR_WORKSPACE is returned.  A negative token in
  *                        the scanned range is TS_ERR_INVALID_ARG.
- *  ts_ngram_topk         the k (1 <= k <= 4096) most frequent n-grams that
- *                        start with `first`: their n-1 continuation tokens
- *                        into cont_out [k, n-1] and counts into count_out
- *                        [k]; *n_found = how many exist (<= k); rows past
- *                        that get tokens -1 and count 0.
+ *  ts_ngram_topk_prefix  the k (1 <= k <= 4096) most frequent n-grams that
+ *                        start with prefix[0..p): their n-p continuation
+ *                        tokens into cont_out [k, n-p] and counts into
+ *                        count_out [k]; *n_found = how many exist (<= k);
+ *                        rows past that get tokens -1 and count 0.
+ *  ts_ngram_topk         ts_ngram_topk_prefix with the one-token prefix
+ *                        `first` (cont_out [k, n-1]).
  *  ts_ngram_count        occurrences of one n-gram (gram[0..n)); 0 if absent.
  *  ts_ngram_size         distinct n-grams held and total n-grams counted.
  * Errors: TS_ERR_INVALID_ARG for NULL pointers, an unformatted table, a
@@ -302,6 +307,9 @@ TS_API size_t ts_ngram_table_bytes(int n, int64_t capacity);
 TS_API int ts_ngram_init(void *table, size_t table_bytes, int n, int64_t capacity);
 TS_API int ts_ngram_update(void *table, size_t table_bytes, const int32_t *text,
                            int64_t text_len, int64_t n_new);
+TS_API int ts_ngram_topk_prefix(const void *table, size_t table_bytes, const int32_t *prefix,
+                                int p, int k, int32_t *cont_out, int64_t *count_out,
+                                int *n_found);
 TS_API int ts_ngram_topk(const void *table, size_t table_bytes, int32_t first, int k,
                          int32_t *cont_out, int64_t *count_out, int *n_found);
 TS_API int ts_ngram_count(const void *table, size_t table_bytes, const int32_t *gram,

@@ -27,6 +27,7 @@ EXPORTS = ("ts_status_string", "ts_version", "ts_tree_verify_attn_workspace_size
            "ts_workspace_status", "ts_kernel_launch_count", "ts_tree_verify_attn_root_scores",
            "ts_kv_select_from_scores_workspace_size", "ts_kv_select_from_scores",
            "ts_ngram_table_bytes", "ts_ngram_init", "ts_ngram_update", "ts_ngram_topk",
+           "ts_ngram_topk_prefix",
            "ts_ngram_count", "ts_ngram_size")
 
 
@@ -86,6 +87,8 @@ def _lib():
         lib.ts_ngram_update.argtypes = [P, sz, P, i64, i64]
         lib.ts_ngram_topk.restype = i32
         lib.ts_ngram_topk.argtypes = [P, sz, ctypes.c_int32, i32, P, P, P]
+        lib.ts_ngram_topk_prefix.restype = i32
+        lib.ts_ngram_topk_prefix.argtypes = [P, sz, P, i32, i32, P, P, P]
         lib.ts_ngram_count.restype = i32
         lib.ts_ngram_count.argtypes = [P, sz, P, P]
         lib.ts_ngram_size.restype = i32
@@ -330,7 +333,9 @@ class NgramTable:
     owns.  ``update(text, n_new)`` counts the n-grams of ``text`` that end
     at its last ``n_new`` tokens; ``topk(first, k)`` returns the most
     frequent ones starting with ``first`` as ``(continuations [m, n-1],
-    counts [m])``, count descending, ties by continuation ascending."""
+    counts [m])``, count descending, ties by continuation ascending;
+    ``topk_prefix(prefix, k)`` does the same for a prefix of 1 to n-1
+    tokens (n-1 tokens: the next-token counts)."""
 
     def __init__(self, n: int, capacity: int):
         import numpy as np
@@ -357,6 +362,21 @@ class NgramTable:
                                     cont.ctypes.data_as(ctypes.c_void_p),
                                     cnt.ctypes.data_as(ctypes.c_void_p), ctypes.byref(found)),
                "ts_ngram_topk")
+        return cont[:found.value], cnt[:found.value]
+
+    def topk_prefix(self, prefix, k: int):
+        """The k most frequent n-grams that start with ``prefix`` (1 to n-1
+        tokens): ``(continuations [m, n - len(prefix)], counts [m])``."""
+        import numpy as np
+        arr, p = _host_i32(prefix)
+        cont = np.empty((int(k), max(self.n - len(arr), 0)), dtype=np.int32)
+        cnt = np.empty(int(k), dtype=np.int64)
+        found = ctypes.c_int(0)
+        _raise(_lib().ts_ngram_topk_prefix(self._p, self.nbytes, p, len(arr), int(k),
+                                           cont.ctypes.data_as(ctypes.c_void_p),
+                                           cnt.ctypes.data_as(ctypes.c_void_p),
+                                           ctypes.byref(found)),
+               "ts_ngram_topk_prefix")
         return cont[:found.value], cnt[:found.value]
 
     def count(self, gram) -> int:

@@ -8,16 +8,18 @@
 // parallel-verification step of the method figure).  The table lives in one
 // caller-owned buffer:
 //
-//   Header | Slot[capacity] | Key[capacity]
+//   Header | Slot[capacity] | Key[capacity] (first token) | Key[capacity] ((n-1)-prefix)
 //
 // A Slot holds one n-gram and its count (count 0 = empty); slots are found
-// by open addressing with linear probing on a hash of the n tokens.  A Key
-// holds a first token, the head of the chain of slots whose n-gram starts
-// with it (head -1 = empty), and that chain's best kTop slots in retrieval
-// order.  Counts only grow, one at a time, so the best list stays exact when
+// by open addressing with linear probing on a hash of the n tokens.  Two
+// indices chain the slots: by first token (whole-phrase continuations of a
+// token) and by the first n-1 tokens (next-token counts after a prefix).  A
+// Key holds the head of one chain (-1 = empty entry; the key's tokens are
+// read from its head slot) and that chain's best kTop slots in retrieval
+// order.  Counts only grow, one at a time, so a best list stays exact when
 // each counted slot is moved up in it (or enters it past its last entry);
-// a retrieval of up to kTop n-grams then reads the list and never walks the
-// chain.  Nothing is ever removed.
+// a retrieval of up to kTop n-grams on an indexed prefix reads the list and
+// never walks the chain.  Nothing is ever removed.
 #include <stdint.h>
 #include <string.h>
 
@@ -29,10 +31,10 @@
 
 namespace {
 
-constexpr uint32_t kMagic = 0x4e475431u;   // "NGT1"
+constexpr uint32_t kMagic = 0x4e475432u;   // "NGT2"
 constexpr int kMaxN = 8;
 constexpr int kMaxK = 4096;
-constexpr int kTop = 16;                              // best n-grams kept per first token
+constexpr int kTop = 16;                              // best n-grams kept per key
 constexpr int64_t kMaxCapacity = int64_t(1) << 31;    // slot indices fit int32
 
 struct Header {
@@ -49,14 +51,14 @@ static_assert(sizeof(Header) == 64, "header is 64 bytes");
 struct Slot {
     int32_t tok[kMaxN];
     int64_t count;
-    int64_t next;    // next slot with the same first token, -1 at the end
+    int64_t next[2];   // next slot in the chain of index 0 / 1, -1 at the end
 };
-static_assert(sizeof(Slot) == 48, "slot is 48 bytes");
+static_assert(sizeof(Slot) == 56, "slot is 56 bytes");
 
 struct Key {
-    int32_t first;
-    int32_t n_top;       // entries of top[] in use
     int64_t head;        // -1: empty entry
+    int32_t n_top;       // entries of top[] in use
+    int32_t pad;
     int32_t top[kTop];   // best slots of the chain, retrieval order
 };
 static_assert(sizeof(Key) == 80, "key is 80 bytes");
@@ -67,7 +69,7 @@ size_t table_bytes(int n, int64_t capacity)
 {
     if (n < 2 || n > kMaxN || !capacity_ok(capacity))
         return 0;
-    return sizeof(Header) + (size_t)capacity * (sizeof(Slot) + sizeof(Key));
+    return sizeof(Header) + (size_t)capacity * (sizeof(Slot) + 2 * sizeof(Key));
 }
 
 // At least one slot stays empty, so every probe sequence ends.
@@ -91,9 +93,10 @@ uint64_t hash_tokens(const int32_t *t, int n)
 struct View {
     Header *hdr;
     Slot *slots;
-    Key *keys;
+    Key *keys[2];   // index 0: first token; index 1: first n-1 tokens
     int n;
     int64_t mask;
+    int plen(int idx) const { return idx == 0 ? 1 : n - 1; }
 };
 
 // The table in `p` if it is formatted and fits in `bytes`.
@@ -107,7 +110,8 @@ bool view_of(const void *p, size_t bytes, View &v)
         return false;
     v.hdr = h;
     v.slots = reinterpret_cast<Slot *>(h + 1);
-    v.keys = reinterpret_cast<Key *>(v.slots + h->capacity);
+    v.keys[0] = reinterpret_cast<Key *>(v.slots + h->capacity);
+    v.keys[1] = v.keys[0] + h->capacity;
     v.n = h->n;
     v.mask = h->capacity - 1;
     return true;
@@ -125,12 +129,16 @@ int64_t find_slot(const View &v, const int32_t *gram)
     }
 }
 
-int64_t find_key(const View &v, int32_t first)
+// Key of index `idx` for the prefix (its first plen tokens), or the empty
+// entry where it would go.  Keys never outnumber slots.
+int64_t find_key(const View &v, int idx, const int32_t *prefix)
 {
-    int64_t i = (int64_t)(hash_tokens(&first, 1) & (uint64_t)v.mask);
+    const int p = v.plen(idx);
+    const Key *keys = v.keys[idx];
+    int64_t i = (int64_t)(hash_tokens(prefix, p) & (uint64_t)v.mask);
     for (;;) {
-        const Key &k = v.keys[i];
-        if (k.head < 0 || k.first == first)
+        const Key &k = keys[i];
+        if (k.head < 0 || memcmp(v.slots[k.head].tok, prefix, sizeof(int32_t) * p) == 0)
             return i;
         i = (i + 1) & v.mask;
     }
@@ -145,8 +153,9 @@ bool tokens_less(const int32_t *a, const int32_t *b, int n)
     return false;
 }
 
-// retrieval order of two slots with the same first token: count
-// descending, then continuation ascending
+// Retrieval order of two slots that share a prefix: count descending, then
+// the tokens after the first in ascending order (for a shared prefix of any
+// length that is the order of the continuations).
 bool ranks_before(const View &v, int64_t a, int64_t b)
 {
     const Slot &x = v.slots[a], &y = v.slots[b];
@@ -155,7 +164,7 @@ bool ranks_before(const View &v, int64_t a, int64_t b)
     return tokens_less(x.tok + 1, y.tok + 1, v.n - 1);
 }
 
-// slot s (first token of key k) was just counted: keep k's best list exact
+// slot s of key k's chain was just counted: keep k's best list exact
 void refresh_top(const View &v, Key &k, int32_t s)
 {
     int pos = -1;
@@ -196,8 +205,8 @@ int ts_ngram_init(void *table, size_t bytes, int n, int64_t capacity)
     Slot *slots = reinterpret_cast<Slot *>(h + 1);
     Key *keys = reinterpret_cast<Key *>(slots + capacity);
     memset(slots, 0, sizeof(Slot) * (size_t)capacity);
-    memset(keys, 0, sizeof(Key) * (size_t)capacity);
-    for (int64_t i = 0; i < capacity; ++i)
+    memset(keys, 0, 2 * sizeof(Key) * (size_t)capacity);
+    for (int64_t i = 0; i < 2 * capacity; ++i)
         keys[i].head = -1;
     h->n = n;
     h->capacity = capacity;
@@ -246,58 +255,74 @@ int ts_ngram_update(void *table, size_t bytes, const int32_t *text, int64_t text
         const int32_t *g = text + e - (n - 1);
         const int64_t si = find_slot(v, g);
         Slot &s = v.slots[si];
-        Key &k = v.keys[find_key(v, g[0])];
+        Key *k[2] = {&v.keys[0][find_key(v, 0, g)], &v.keys[1][find_key(v, 1, g)]};
         if (s.count == 0) {
+            // the tokens first: an empty key found above is compared
+            // against its head slot's tokens from now on
             memset(s.tok, 0, sizeof(s.tok));
             memcpy(s.tok, g, sizeof(int32_t) * n);
-            if (k.head < 0) {
-                k.first = g[0];
-                k.n_top = 0;
-                ++v.hdr->keys;
+            for (int idx = 0; idx < 2; ++idx) {
+                if (k[idx]->head < 0) {
+                    k[idx]->n_top = 0;
+                    if (idx == 0)
+                        ++v.hdr->keys;
+                }
+                s.next[idx] = k[idx]->head;
+                k[idx]->head = si;
             }
-            s.next = k.head;
-            k.head = si;
             ++v.hdr->used;
         }
         ++s.count;
         ++v.hdr->total;
-        refresh_top(v, k, (int32_t)si);
+        refresh_top(v, *k[0], (int32_t)si);
+        refresh_top(v, *k[1], (int32_t)si);
     }
     return TS_OK;
 }
 
-int ts_ngram_topk(const void *table, size_t bytes, int32_t first, int k, int32_t *cont_out,
-                  int64_t *count_out, int *n_found)
+int ts_ngram_topk_prefix(const void *table, size_t bytes, const int32_t *prefix, int p, int k,
+                         int32_t *cont_out, int64_t *count_out, int *n_found)
 {
     View v;
-    if (!view_of(table, bytes, v) || k < 1 || k > kMaxK || !cont_out || !count_out || !n_found)
+    if (!view_of(table, bytes, v) || !prefix || p < 1 || p > v.n - 1 || k < 1 || k > kMaxK ||
+        !cont_out || !count_out || !n_found)
         return TS_ERR_INVALID_ARG;
-    const int m = v.n - 1;
+    const int m = v.n - p;   // continuation tokens per row
     for (int i = 0; i < k; ++i) {
         count_out[i] = 0;
         for (int j = 0; j < m; ++j)
             cont_out[(size_t)i * m + j] = -1;
     }
     *n_found = 0;
-    if (first < 0)
-        return TS_OK;
-    const Key &key = v.keys[find_key(v, first)];
+    for (int i = 0; i < p; ++i)
+        if (prefix[i] < 0)
+            return TS_OK;   // no such n-gram can be held
+    // an indexed prefix length walks (or reads the best list of) its own
+    // chain; any other walks the first-token chain and filters
+    const int idx = p == 1 ? 0 : (p == v.n - 1 ? 1 : 0);
+    const bool filter = p != v.plen(idx);
+    const Key &key = v.keys[idx][find_key(v, idx, prefix)];
     if (key.head < 0)
         return TS_OK;
-    // the best list holds the whole chain while it is not full, and the
-    // chain's best kTop once it is
-    if (k <= key.n_top || key.n_top < kTop) {
-        const int found = k < key.n_top ? k : key.n_top;
+    auto emit = [&](const int64_t *slots, int found) {
         for (int i = 0; i < found; ++i) {
-            const Slot &s = v.slots[key.top[i]];
+            const Slot &s = v.slots[slots[i]];
             count_out[i] = s.count;
-            memcpy(cont_out + (size_t)i * m, s.tok + 1, sizeof(int32_t) * m);
+            memcpy(cont_out + (size_t)i * m, s.tok + p, sizeof(int32_t) * m);
         }
         *n_found = found;
+    };
+    // the best list holds the whole chain while it is not full, and the
+    // chain's best kTop once it is
+    if (!filter && (k <= key.n_top || key.n_top < kTop)) {
+        int64_t top[kTop];
+        const int found = k < key.n_top ? k : key.n_top;
+        for (int i = 0; i < found; ++i)
+            top[i] = key.top[i];
+        emit(top, found);
         return TS_OK;
     }
-    // more than kTop asked of a longer chain: walk it, keeping the best k
-    // sorted in the same order
+    // walk the chain, keeping the best k sorted in the same order
     int found = 0;
     std::vector<int64_t> best;
     try {
@@ -305,9 +330,10 @@ int ts_ngram_topk(const void *table, size_t bytes, int32_t first, int k, int32_t
     } catch (const std::bad_alloc &) {
         return TS_ERR_WORKSPACE;
     }
-    auto before = [&](int64_t a, int64_t b) { return ranks_before(v, a, b); };
-    for (int64_t s = key.head; s >= 0; s = v.slots[s].next) {
-        if (found == k && !before(s, best[k - 1]))
+    for (int64_t s = key.head; s >= 0; s = v.slots[s].next[idx]) {
+        if (filter && memcmp(v.slots[s].tok, prefix, sizeof(int32_t) * p) != 0)
+            continue;
+        if (found == k && !ranks_before(v, s, best[k - 1]))
             continue;
         if (found < k) {
             best.push_back(s);
@@ -315,16 +341,17 @@ int ts_ngram_topk(const void *table, size_t bytes, int32_t first, int k, int32_t
         } else {
             best[k - 1] = s;
         }
-        for (int i = found - 1; i > 0 && before(best[i], best[i - 1]); --i)
+        for (int i = found - 1; i > 0 && ranks_before(v, best[i], best[i - 1]); --i)
             std::swap(best[i], best[i - 1]);
     }
-    for (int i = 0; i < found; ++i) {
-        const Slot &s = v.slots[best[i]];
-        count_out[i] = s.count;
-        memcpy(cont_out + (size_t)i * m, s.tok + 1, sizeof(int32_t) * m);
-    }
-    *n_found = found;
+    emit(best.data(), found);
     return TS_OK;
+}
+
+int ts_ngram_topk(const void *table, size_t bytes, int32_t first, int k, int32_t *cont_out,
+                  int64_t *count_out, int *n_found)
+{
+    return ts_ngram_topk_prefix(table, bytes, &first, 1, k, cont_out, count_out, n_found);
 }
 
 int ts_ngram_count(const void *table, size_t bytes, const int32_t *gram, int64_t *count)

@@ -11,8 +11,9 @@ generation of ultra-long text", aiboss88.com, "Parallel generation of
 multiple tokens and token reuse"; cloud.tencent.com article, the
 parallel-verification step of the method figure).  The pages fix neither n
 nor the retrieval order; the reading taken here: count every window of n
-tokens; the candidates for a first token are its n-grams by count,
-descending, ties by continuation in ascending token order.
+tokens; the candidates for a prefix (a first token, or the last n-1
+tokens) are the n-grams that start with it, by count, descending, ties by
+continuation in ascending token order.
 """
 from __future__ import annotations
 
@@ -41,5 +42,15 @@ def ngram_topk(counts, first, k):
     (continuation, count) pairs: count descending, then continuation
     ascending."""
     cands = [(g[1:], c) for g, c in counts.items() if g[0] == first]
+    cands.sort(key=lambda gc: (-gc[1], gc[0]))
+    return cands[:k]
+
+
+def ngram_topk_prefix(counts, prefix, k):
+    """The k most frequent n-grams that start with the tokens of `prefix`,
+    as (continuation, count) pairs in the same order as ngram_topk."""
+    p = len(prefix)
+    pre = tuple(int(x) for x in prefix)
+    cands = [(g[p:], c) for g, c in counts.items() if g[:p] == pre]
     cands.sort(key=lambda gc: (-gc[1], gc[0]))
     return cands[:k]

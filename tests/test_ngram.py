@@ -57,6 +57,9 @@ def test_oracle_golden_figure_example():
     assert diff == {tuple(enc(w)): 1 for w in g["new_windows"]}
     want2 = [(tuple(enc(cont)), cnt) for cont, cnt in g["topk_is_after"]]
     assert O.ngram_topk(c2, ids["is"], 3) == want2
+    pre = enc(["is", "the", "uncle"])
+    for cc, key in ((c, "next_after_is_the_uncle"), (c2, "next_after_is_the_uncle_after")):
+        assert O.ngram_topk_prefix(cc, pre, 5) == [(tuple(enc(t)), k) for t, k in g[key]]
 
 
 def test_oracle_update_counts_only_windows_ending_in_the_new_tokens():
@@ -75,6 +78,10 @@ def test_oracle_topk_order_breaks_ties_by_continuation():
     assert O.ngram_topk(c, 1, 10) == [((2, 3), 2), ((2, 9), 2), ((5, 5), 2), ((0, 0), 1)]
     assert O.ngram_topk(c, 1, 2) == [((2, 3), 2), ((2, 9), 2)]
     assert O.ngram_topk(c, 3, 4) == []
+    # a two-token prefix keeps only the n-grams that start with both tokens
+    assert O.ngram_topk_prefix(c, [1, 2], 10) == [((3,), 2), ((9,), 2)]
+    assert O.ngram_topk_prefix(c, [1], 10) == O.ngram_topk(c, 1, 10)
+    assert O.ngram_topk_prefix(c, [2, 1], 10) == []
 
 
 # ------------------------------------------------- the library's table
@@ -86,15 +93,25 @@ def L():
     return L
 
 
-def _same_as_oracle(tab, counts, n, firsts, ks=(1, 3, 16, 17, 50)):
+def _rows(cont, cnt):
+    return [(tuple(r), int(x)) for r, x in zip(cont.tolist(), cnt.tolist())]
+
+
+def _same_as_oracle(tab, counts, n, firsts, ks=(1, 3, 16, 17, 50), n_prefixes=12):
     assert tab.size() == (len(counts), sum(counts.values()))
     for g, c in counts.items():
         assert tab.count(g) == c
     for first in firsts:
         for k in ks:
-            cont, cnt = tab.topk(first, k)
-            want = O.ngram_topk(counts, first, k)
-            assert [(tuple(r), int(x)) for r, x in zip(cont.tolist(), cnt.tolist())] == want
+            assert _rows(*tab.topk(first, k)) == O.ngram_topk(counts, first, k)
+    # every prefix length, on prefixes that occur and one that does not
+    grams = sorted(counts)
+    for p in range(1, n):
+        picks = [grams[i][:p] for i in range(0, len(grams), max(1, len(grams) // n_prefixes))]
+        picks.append((10 ** 6,) * p)
+        for pre in picks:
+            for k in ks:
+                assert _rows(*tab.topk_prefix(pre, k)) == O.ngram_topk_prefix(counts, pre, k)
 
 
 @pytest.mark.parametrize("n,vocab,length,seed", [(2, 3, 400, 0), (3, 5, 1000, 1), (4, 8, 3000, 2),
@@ -134,6 +151,9 @@ def test_table_golden_figure_example(L):
     cont, cnt = tab.topk(ids["is"], 3)
     assert [(r, int(x)) for r, x in zip(cont.tolist(), cnt.tolist())] == \
         [(enc(c), k) for c, k in g["topk_is_after"]]
+    cont, cnt = tab.topk_prefix(enc(["is", "the", "uncle"]), 4)
+    assert [(r, int(x)) for r, x in zip(cont.tolist(), cnt.tolist())] == \
+        [(enc(c), k) for c, k in g["next_after_is_the_uncle_after"]]
 
 
 def test_table_full_is_all_or_nothing(L):
@@ -168,7 +188,7 @@ def test_table_rejects_invalid_calls(L):
     assert lib.ts_ngram_table_bytes(1, 16) == 0
     assert lib.ts_ngram_table_bytes(9, 16) == 0
     assert lib.ts_ngram_table_bytes(4, 24) == 0          # not a power of two
-    assert lib.ts_ngram_table_bytes(4, 16) == 64 + 16 * (48 + 80)
+    assert lib.ts_ngram_table_bytes(4, 16) == 64 + 16 * 216
     assert lib.ts_ngram_table_bytes(4, 1 << 32) == 0     # slot indices are int32
     with pytest.raises(ValueError):
         L.NgramTable(4, 12)
@@ -182,6 +202,10 @@ def test_table_rejects_invalid_calls(L):
         tab.topk(1, 0)
     with pytest.raises(L.TsError):
         tab.topk(1, 4097)
+    with pytest.raises(L.TsError):
+        tab.topk_prefix([1, 2, 3], 4)                     # prefix as long as n
+    with pytest.raises(L.TsError):
+        tab.topk_prefix([], 4)
     # an unformatted buffer is not a table
     import ctypes
     buf = np.zeros(200, dtype=np.uint64)
@@ -217,3 +241,29 @@ def test_table_best_lists_stay_exact_as_counts_grow(L):
                 assert [(tuple(r), int(x)) for r, x in zip(cont.tolist(), cnt.tolist())] == \
                     O.ngram_topk(counts, first, k)
     _same_as_oracle(tab, counts, n, firsts=range(3), ks=(16, 17, 81, 200))
+
+
+def test_table_next_token_lists_stay_exact_as_counts_grow(L):
+    # n = 3 over 40 tokens with a drifting skew: the frequent two-token
+    # prefixes gather far more than 16 next tokens, so their best lists (the
+    # second index) are displaced over and over; checked after every update
+    rng = np.random.default_rng(12)
+    n, vocab = 3, 40
+    parts = []
+    for shift in (0, 13, 27, 5):
+        w = 1.0 / (1.0 + ((np.arange(vocab) + shift) % vocab))
+        parts.append(rng.choice(vocab, 1500, p=w / w.sum()))
+    text = np.concatenate(parts).astype(np.int32)
+    tab = L.NgramTable(n, 1 << 14)
+    counts, done = {}, 0
+    watch = [(0, 0), (0, 1), (13, 13), (27, 27), (5, 5)]
+    while done < len(text):
+        cut = min(len(text), done + int(rng.integers(1, 50)))
+        tab.update(text[max(0, done - n + 1):cut], cut - done)
+        counts = O.ngram_update(counts, text[:cut].tolist(), cut - done, n)
+        done = cut
+        for pre in watch:
+            for k in (1, 5, 16):
+                assert _rows(*tab.topk_prefix(pre, k)) == O.ngram_topk_prefix(counts, pre, k)
+    assert max(len(O.ngram_topk_prefix(counts, pre, 100)) for pre in watch) > 16
+    _same_as_oracle(tab, counts, n, firsts=range(0, vocab, 3), ks=(16, 17, 40))
