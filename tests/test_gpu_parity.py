@@ -228,7 +228,9 @@ def test_select_llama8b_100k_spiked(oracle_mod):
 # ------------------------------- select from the verify attention's scores
 @pytest.mark.parametrize("hq,hkv,d,n_ctx,t,n_sink,budget", [
     (32, 8, 128, 32768, 40, 64, 4032),   # 128-position tcgen05 kernel, 160 rows
-    (16, 16, 128, 9001, 13, 16, 500),    # same kernel, G = 1, odd context
+    (32, 8, 128, 5000, 40, 64, 1000),    # same, last context tile partly filled (bulk copy)
+    (64, 8, 128, 4096, 24, 16, 500),     # same, G = 8: eight root rows, 192 rows
+    (16, 16, 128, 9001, 13, 16, 500),    # same kernel, G = 1, odd context (plain stores)
     (40, 8, 128, 6000, 40, 32, 1000),    # 64-position tcgen05 kernel (200 rows)
     (8, 2, 64, 3000, 13, 16, 240),       # mma.sync kernel (head_dim 64)
     (8, 2, 128, 1000, 4, 8, 100),        # mma.sync kernel (short context)
