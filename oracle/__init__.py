@@ -32,7 +32,9 @@ def build(force: bool = False) -> str:
 def _load():
     global _lib
     if _lib is None:
-        lib = ctypes.CDLL(build())
+        # a test that plants a mistake in the oracle loads its mutated build
+        # from TSO_MUTANT_LIB (tests/test_oracle_mutants.py)
+        lib = ctypes.CDLL(os.environ.get("TSO_MUTANT_LIB") or build())
         P = ctypes.c_void_p
         i32, i64, f64, f32 = ctypes.c_int, ctypes.c_int64, ctypes.c_double, ctypes.c_float
         lib.tso_tree_verify_attn.argtypes = [P, P, P, i64, i32, i32, i32, i32, i32, P, f64, P]
