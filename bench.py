@@ -4,11 +4,15 @@
 One step = one pass of the whole per-step hot path on the LLaMA3.1-8B
 100K-context workload (Hq=32, Hkv=8, D=128, n_ctx=102400, 40-node 3-ary
 tree):
-  1. ts_tree_verify_attn over the full cache (the headline call),
-  2. ts_kv_importance_select: 64 sinks + top-4032 into the partial cache,
+  1. ts_tree_verify_attn_root_scores over the full cache (the headline
+     call; it also leaves the root node's scores over the context),
+  2. ts_kv_select_from_scores: 64 sinks + top-4032 into the partial cache,
   3. the draft pass: ts_tree_verify_attn of a 4-node chain over that
      4096-row partial cache,
-  4. ts_penalize_accept over fp32 logits [40, 128256], window 1024.
+  4. ts_penalize_accept over fp32 logits [40, 128256], window 1024, on a
+     second stream beside 2 and 3.
+With --select-score-pass, 1 and 2 are ts_tree_verify_attn and
+ts_kv_importance_select (the select scores the context itself).
 The metric counts tree-verify calls: each step holds exactly one.
 
 Prints ONE JSON line (rank 0).  ``--impl reference`` times the fp64 CPU
