@@ -11,8 +11,10 @@
  * technical principles"; "From Hours to Minutes: Lossless Acceleration of
  * Ultra-Long Sequence Generation up to 100K Tokens", arxivlens.com,
  * "Technical Contribution").  This library implements the three kernels of
- * that step; the model around them (projections, LM head, draft heads) is
- * the caller's.
+ * that step (with a fused form in which the verify attention hands the root
+ * node's scores to the select) and, as host code, the n-gram reuse table;
+ * the model around them (projections, LM head, draft heads) is the
+ * caller's.
  *
  * Conventions for every entry point
  *  - Memory: the caller owns every buffer.  The library never allocates,
