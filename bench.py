@@ -120,6 +120,24 @@ def attn_traffic_record():
     return float(rec["dram_bytes_per_call"])
 
 
+def ngram_host_timing(L, n_tokens: int = 102400, steps: int = 2000, seed: int = 0) -> float:
+    """Host microseconds per verification step of the n-gram reuse table:
+    the step's accepted tokens (5: a depth-3 path and the bonus token) are
+    counted and the new root's 8 most frequent continuations fetched, on a
+    table that already holds the whole context (a Zipf(1.2) token stream
+    over the workload's 128256-token vocabulary, n = 4)."""
+    rng = np.random.default_rng(seed)
+    text = np.minimum(rng.zipf(1.2, n_tokens + 5 * steps), 128255).astype(np.int32)
+    tab = L.NgramTable(4, 1 << 18)   # fill limit 229376 n-grams
+    tab.update(text[:n_tokens])
+    t0 = time.perf_counter()
+    for s in range(steps):
+        end = n_tokens + 5 * (s + 1)
+        tab.update(text[end - 8:end], 5)
+        tab.topk(int(text[end - 1]), 8)
+    return (time.perf_counter() - t0) / steps * 1e6
+
+
 class ClockSampler:
     """SM clock and clock-event (throttle) reasons sampled during the timed
     region: NVML in a thread every 5 ms (read-only queries), else
@@ -442,6 +460,11 @@ def run_ours(args):
             "gpu_launches": int(launches_per_step * K),
             "clocks": clk.summary(),
         }
+        try:
+            out["ngram_host_us_per_step"] = round(ngram_host_timing(L), 2)
+        except Exception as e:   # host-side extra: never costs the GPU line
+            out["ngram_host_us_per_step"] = None
+            out["ngram_host_error"] = str(e)[:200]
         if not args.no_cpu_baseline:
             out["cpu_baseline"] = cpu_baseline(w)
     if world > 1:

@@ -76,3 +76,11 @@ def test_reference_arm_runs_on_rank_zero_only(monkeypatch):
     monkeypatch.setenv("WORLD_SIZE", "2")
     args = argparse.Namespace(steps=3, warmup=1, gpus=2, impl="reference")
     assert bench.run_reference(args) is None
+
+
+def test_ngram_host_timing_runs_on_the_cpu():
+    from lossless_ultra_long_b200 import build
+    build.build()
+    import lossless_ultra_long_b200 as L
+    us = bench.ngram_host_timing(L, n_tokens=3000, steps=50)
+    assert 0.0 < us < 1e5
