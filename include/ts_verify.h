@@ -326,6 +326,19 @@ TS_API int ts_ngram_size(const void *table, size_t table_bytes, int64_t *distinc
 TS_API unsigned long long ts_kernel_launch_count(void);
 
 /*
+ * Failure-detection self-test.  Every pipeline wait in this library's
+ * kernels is bounded (about one second of SM clock); a wait that runs out
+ * records TS_ERR_TIMEOUT in the workspace status word and the kernel ends
+ * without trapping, so the context stays usable.  This call launches one
+ * small CTA that takes that same bounded wait on a barrier nothing ever
+ * completes: about one second later it has recorded TS_ERR_TIMEOUT in
+ * `workspace` (read it with ts_workspace_status).  Diagnostic only; no
+ * page of the method has a counterpart.
+ *  workspace    device, >= 256 bytes, 256-byte aligned, zero-filled.
+ */
+TS_API int ts_selftest_bounded_wait(void *workspace, size_t workspace_bytes, void *stream);
+
+/*
  * Reads the status word of a workspace after the work queued on `stream`
  * has finished (this call synchronises `stream`).  Returns TS_OK or the
  * first device-side error recorded since the last clear; clears the word

@@ -28,7 +28,7 @@ EXPORTS = ("ts_status_string", "ts_version", "ts_tree_verify_attn_workspace_size
            "ts_kv_select_from_scores_workspace_size", "ts_kv_select_from_scores",
            "ts_ngram_table_bytes", "ts_ngram_init", "ts_ngram_update", "ts_ngram_topk",
            "ts_ngram_topk_prefix",
-           "ts_ngram_count", "ts_ngram_size")
+           "ts_ngram_count", "ts_ngram_size", "ts_selftest_bounded_wait")
 
 
 class TsError(RuntimeError):
@@ -79,6 +79,8 @@ def _lib():
         lib.ts_kernel_launch_count.argtypes = []
         lib.ts_workspace_status.restype = i32
         lib.ts_workspace_status.argtypes = [P, P, i32]
+        lib.ts_selftest_bounded_wait.restype = i32
+        lib.ts_selftest_bounded_wait.argtypes = [P, sz, P]
         lib.ts_ngram_table_bytes.restype = sz
         lib.ts_ngram_table_bytes.argtypes = [i32, i64]
         lib.ts_ngram_init.restype = i32
@@ -320,6 +322,17 @@ def penalize_accept(logits, window, penalty: float, parent, tree_tokens, argmax_
 def kernel_launch_count() -> int:
     """Kernels the library has launched in this process."""
     return int(_lib().ts_kernel_launch_count())
+
+
+def selftest_bounded_wait(workspace=None, stream=None):
+    """``ts_selftest_bounded_wait``: one CTA takes the kernels' bounded wait
+    on a barrier nothing completes; about a second later TS_ERR_TIMEOUT is
+    in the workspace's status word.  Returns the workspace."""
+    if workspace is None:
+        workspace = new_workspace(256)
+    _raise(_lib().ts_selftest_bounded_wait(_ptr(workspace), workspace.numel(), _stream(stream)),
+           "ts_selftest_bounded_wait")
+    return workspace
 
 
 def workspace_status(workspace, clear: bool = True, stream=None) -> int:

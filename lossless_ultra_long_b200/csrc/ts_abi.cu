@@ -321,6 +321,15 @@ int ts_penalize_accept(const float *logits, int n_tree, int vocab, const int32_t
     return e == cudaSuccess ? TS_OK : TS_ERR_CUDA;
 }
 
+int ts_selftest_bounded_wait(void *workspace, size_t workspace_bytes, void *stream)
+{
+    if (!workspace_ok(workspace, workspace_bytes, ts::kHeaderBytes))
+        return TS_ERR_WORKSPACE;
+    const cudaError_t e =
+        ts::selftest_bounded_wait_launch(workspace, static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? TS_OK : TS_ERR_CUDA;
+}
+
 int ts_workspace_status(const void *workspace, void *stream, int clear)
 {
     if (!workspace)

@@ -93,6 +93,10 @@ cudaError_t select_launch(const SelectArgs &a, int num_sms, cudaStream_t stream)
 cudaError_t select_score_pass_launch(const SelectArgs &a, float *out, int num_sms,
                                      cudaStream_t stream);
 
+// One CTA waits, with the kernels' bounded wait, on a barrier nothing
+// completes; the wait records TS_ERR_TIMEOUT after its bound.
+cudaError_t selftest_bounded_wait_launch(void *workspace, cudaStream_t stream);
+
 struct PenalizeArgs {
     const float *logits;
     int n_tree, vocab;
