@@ -173,3 +173,57 @@ def test_select_from_scores_accepts_4_byte_rows_for_ragged_contexts(lib):
     need = L.kv_select_from_scores_workspace_size()
     assert need > 0
     assert _from_scores_call(lib, rs=(1 << 20) + 4, n_ctx=999, ws_bytes=need - 1) == 3
+
+
+def test_header_is_plain_c_and_the_library_serves_a_c_program(lib, tmp_path):
+    """The public header compiles as C11 and as C++17, and a C program that
+    loads libtsverify.so with dlopen finds every declared entry point and
+    gets answers from the host-only ones (no device is touched)."""
+    import subprocess
+    from lossless_ultra_long_b200 import LIB_PATH
+    inc = os.path.dirname(HEADER)
+    names = declared_symbols()
+    prog = tmp_path / "abi_c.c"
+    prog.write_text(r"""
+#include <dlfcn.h>
+#include <stdio.h>
+#include <string.h>
+#include "ts_verify.h"
+static const char *names[] = {%s};
+int main(int argc, char **argv) {
+    void *h = dlopen(argv[1], RTLD_NOW | RTLD_LOCAL);
+    if (!h) { fprintf(stderr, "%%s\n", dlerror()); return 2; }
+    for (size_t i = 0; i < sizeof names / sizeof names[0]; ++i)
+        if (!dlsym(h, names[i])) { fprintf(stderr, "missing %%s\n", names[i]); return 3; }
+    int (*version)(void) = (int (*)(void))dlsym(h, "ts_version");
+    const char *(*status)(int) = (const char *(*)(int))dlsym(h, "ts_status_string");
+    size_t (*ng_bytes)(int, int64_t) = (size_t (*)(int, int64_t))dlsym(h, "ts_ngram_table_bytes");
+    int (*ng_init)(void *, size_t, int, int64_t) =
+        (int (*)(void *, size_t, int, int64_t))dlsym(h, "ts_ngram_init");
+    int (*ng_update)(void *, size_t, const int32_t *, int64_t, int64_t) =
+        (int (*)(void *, size_t, const int32_t *, int64_t, int64_t))dlsym(h, "ts_ngram_update");
+    int (*ng_topk)(const void *, size_t, int32_t, int, int32_t *, int64_t *, int *) =
+        (int (*)(const void *, size_t, int32_t, int, int32_t *, int64_t *, int *))
+            dlsym(h, "ts_ngram_topk");
+    if (version() < 100 || strlen(status(TS_ERR_WORKSPACE)) == 0) return 4;
+    static uint64_t table[(64 + 216 * 64) / 8];
+    const size_t nb = ng_bytes(2, 64);
+    if (nb != sizeof table || ng_init(table, nb, 2, 64) != TS_OK) return 5;
+    const int32_t text[] = {5, 7, 5, 7, 5, 9};
+    if (ng_update(table, nb, text, 6, 6) != TS_OK) return 6;
+    int32_t cont[2]; int64_t cnt[2]; int found = 0;
+    if (ng_topk(table, nb, 5, 2, cont, cnt, &found) != TS_OK) return 7;
+    /* bigrams after 5: (5,7) twice, (5,9) once */
+    if (found != 2 || cont[0] != 7 || cnt[0] != 2 || cont[1] != 9 || cnt[1] != 1) return 8;
+    puts("ok");
+    return 0;
+}
+""" % ", ".join('"%s"' % n for n in names))
+    for lang, std in (("c", "-std=c11"), ("c++", "-std=c++17")):
+        subprocess.run(["gcc", "-x", lang, std, "-fsyntax-only", "-Wall", "-Werror",
+                        "-I", inc, "-"], input=b'#include "ts_verify.h"\n', check=True)
+    exe = tmp_path / "abi_c"
+    subprocess.check_call(["gcc", "-std=c11", "-Wall", "-I", inc, str(prog), "-o", str(exe),
+                           "-ldl"])
+    r = subprocess.run([str(exe), LIB_PATH], capture_output=True, text=True, timeout=60)
+    assert r.returncode == 0 and r.stdout.strip() == "ok", (r.returncode, r.stderr)
