@@ -108,6 +108,7 @@ def test_c_program_runs_the_path_through_the_abi(tmp_path):
     subprocess.run(["gcc", "-std=c11", "-Wall", "-I", os.path.join(ROOT, "include"),
                     "-I", os.path.join(CUDA, "include"), str(src), "-o", str(exe),
                     "-L", libdir, "-l:libtsverify.so", "-Wl,-rpath," + libdir,
-                    "-L", os.path.join(CUDA, "lib64"), "-lcudart", "-lm"], check=True)
+                    "-L", os.path.join(CUDA, "lib64"), "-Wl,-rpath," + os.path.join(CUDA, "lib64"),
+                    "-lcudart", "-lm"], check=True)
     r = subprocess.run([str(exe)], capture_output=True, text=True, timeout=300)
     assert r.returncode == 0 and r.stdout.strip() == "ok", (r.returncode, r.stderr)
