@@ -45,8 +45,19 @@ def _load():
         lib.tso_gather_rows.argtypes = [P, i64, i32, i32, P, i32, P, i64]
         lib.tso_penalize_argmax.argtypes = [P, i32, i32, P, i32, f32, P, P]
         lib.tso_accept_longest.argtypes = [P, P, P, i32, P]
+        lib.tso_penalize_argmax_path.argtypes = [P, i32, i32, P, i32, f32, P, P, P, P]
+        lib.tso_accept_longest_random.argtypes = [P, P, P, i32, ctypes.c_uint64, P]
+        lib.tso_kv_commit_path.argtypes = [P, i64, i32, i32, i32, i32, P]
         _lib = lib
     return _lib
+
+
+def set_num_threads(n: int) -> None:
+    """Threads of the oracle's OpenMP loops from now on (in this process)."""
+    _load()
+    gomp = ctypes.CDLL("libgomp.so.1")
+    gomp.omp_set_num_threads.argtypes = [ctypes.c_int]
+    gomp.omp_set_num_threads(int(n))
 
 
 def _p(a: np.ndarray):
@@ -153,4 +164,45 @@ def accept_longest(parent, tokens, argmax) -> np.ndarray:
     rc = _load().tso_accept_longest(_p(parent), _p(tokens), _p(argmax), t, _p(out))
     if rc < 0:
         raise ValueError("oracle: invalid tree")
+    return out
+
+
+def penalize_argmax_path(logits, window, parent, tokens, penalty: float = 1.2,
+                         return_penalized: bool = False):
+    """int32 argmax ``[T]`` with each node's draft-path tokens in its window."""
+    logits = np.ascontiguousarray(logits, dtype=np.float32)
+    window, parent, tokens = _i32(window), _i32(parent), _i32(tokens)
+    t, vocab = logits.shape
+    am = np.empty(t, dtype=np.int32)
+    pen = np.empty_like(logits) if return_penalized else None
+    rc = _load().tso_penalize_argmax_path(_p(logits), t, vocab, _p(window), len(window),
+                                          float(np.float32(penalty)), _p(parent), _p(tokens),
+                                          _p(am), _p(pen) if pen is not None else None)
+    if rc != 0:
+        raise ValueError("oracle: invalid penalty arguments")
+    return (am, pen) if return_penalized else am
+
+
+def accept_longest_random(parent, tokens, argmax, r: int) -> np.ndarray:
+    """As :func:`accept_longest`, the kept node being the (r mod c)-th of the
+    c deepest valid nodes in index order."""
+    parent, tokens, argmax = _i32(parent), _i32(tokens), _i32(argmax)
+    t = len(parent)
+    out = np.full(2 + t, -1, dtype=np.int32)
+    rc = _load().tso_accept_longest_random(_p(parent), _p(tokens), _p(argmax), t,
+                                           ctypes.c_uint64(int(r) & (2 ** 64 - 1)), _p(out))
+    if rc < 0:
+        raise ValueError("oracle: invalid tree")
+    return out
+
+
+def kv_commit_path(cache, n_ctx: int, n_tree: int, accept) -> np.ndarray:
+    """A copy of one cache (bf16 bits [Hkv, kv_cap, D]) with the accepted
+    path's tree rows moved to n_ctx + 0 .. n_ctx + L."""
+    out = np.array(_u16(cache), copy=True)
+    accept = _i32(accept)
+    hkv, cap, d = out.shape
+    rc = _load().tso_kv_commit_path(_p(out), cap, hkv, d, int(n_ctx), int(n_tree), _p(accept))
+    if rc != 0:
+        raise ValueError("oracle: invalid commit arguments")
     return out

@@ -388,3 +388,145 @@ int tso_accept_longest(const int32_t *parent, const int32_t *tokens, const int32
     free(depth);
     return len;
 }
+
+/*
+ * Contextual penalty with each node's own draft path in its window, then
+ * the target argmax of every tree node (aiboss88 "Contextual penalty
+ * strategy": the penalty falls on recently generated tokens).  The logits of
+ * node i give the token that would follow i, and the tokens most recently
+ * generated before it are those of i's own draft path.  Reading: node i's
+ * window is the caller's window together with the tokens of the draft nodes
+ * on i's root path (i included; the root, the last accepted token, is
+ * already in the caller's window and its entry of `tokens` is not read),
+ * taken as one set.  Penalty and argmax rules as in tso_penalize_argmax.
+ * Returns 0, or -1 on invalid input (a window id or a draft token outside
+ * [0, V), or an invalid tree).
+ */
+int tso_penalize_argmax_path(const float *logits, int n_tree, int vocab, const int32_t *window,
+                             int window_len, float penalty, const int32_t *parent,
+                             const int32_t *tokens, int32_t *argmax, float *penalized)
+{
+    if (n_tree < 1 || vocab < 1 || window_len < 0 || !(penalty > 0.0f) ||
+        !tree_is_valid(parent, n_tree))
+        return -1;
+    for (int i = 1; i < n_tree; ++i)
+        if (tokens[i] < 0 || tokens[i] >= vocab)
+            return -1;
+    unsigned char *in_window = (unsigned char *)calloc((size_t)vocab, 1);
+    for (int w = 0; w < window_len; ++w) {
+        if (window[w] < 0 || window[w] >= vocab) {
+            free(in_window);
+            return -1;
+        }
+        in_window[window[w]] = 1;
+    }
+    unsigned char *mark = (unsigned char *)malloc((size_t)vocab);
+    for (int i = 0; i < n_tree; ++i) {
+        memcpy(mark, in_window, (size_t)vocab);
+        for (int a = i; a != 0; a = parent[a])
+            mark[tokens[a]] = 1;
+        float best = -INFINITY;
+        int32_t best_id = 0;
+        for (int id = 0; id < vocab; ++id) {
+            float x = logits[(int64_t)i * vocab + id];
+            if (mark[id])
+                x = x > 0.0f ? x / penalty : x * penalty;
+            if (penalized)
+                penalized[(int64_t)i * vocab + id] = x;
+            if (x != x)
+                x = -INFINITY;
+            if (x > best) {
+                best = x;
+                best_id = id;
+            }
+        }
+        argmax[i] = best_id;
+    }
+    free(mark);
+    free(in_window);
+    return 0;
+}
+
+/*
+ * Longest accepted path with a random choice among equally long valid paths
+ * (aiboss88 "Tree-based multi-candidate token verification": the longest
+ * valid n-gram is selected at random).  Validity as in tso_accept_longest.
+ * Reading: the deepest valid nodes are listed in ascending index (BFS)
+ * order; with c of them, the one at position (r mod c) is kept, r being a
+ * random 64-bit integer the caller draws.  Output as tso_accept_longest.
+ * Returns L, or -1 on invalid input.
+ */
+int tso_accept_longest_random(const int32_t *parent, const int32_t *tokens,
+                              const int32_t *argmax, int n_tree, uint64_t r, int32_t *out)
+{
+    if (!tree_is_valid(parent, n_tree))
+        return -1;
+    int *valid = (int *)malloc(sizeof(int) * (size_t)n_tree);
+    int *depth = (int *)malloc(sizeof(int) * (size_t)n_tree);
+    valid[0] = 1;
+    depth[0] = 0;
+    int deepest = 0;
+    for (int i = 1; i < n_tree; ++i) {
+        int p = parent[i];
+        valid[i] = valid[p] && tokens[i] == argmax[p];
+        depth[i] = depth[p] + 1;
+        if (valid[i] && depth[i] > deepest)
+            deepest = depth[i];
+    }
+    int count = 0;
+    for (int i = 0; i < n_tree; ++i)
+        count += valid[i] && depth[i] == deepest;
+    int pick = (int)(r % (uint64_t)count), best = 0;
+    for (int i = 0; i < n_tree; ++i)
+        if (valid[i] && depth[i] == deepest && pick-- == 0) {
+            best = i;
+            break;
+        }
+    const int len = depth[best];
+    int node = best;
+    for (int t = len; t >= 0; --t) {
+        out[2 + t] = node;
+        node = parent[node];
+    }
+    out[0] = len;
+    out[1] = argmax[best];
+    free(valid);
+    free(depth);
+    return len;
+}
+
+/*
+ * Commit of the accepted path into the cache (tencent parallel-verification
+ * figure: the candidates are verified against the full KV cache, the
+ * longest valid one is kept and the state is updated for the next step).
+ * The tree's K/V rows sit at n_ctx + node; after acceptance the accepted
+ * path's rows become the next context rows in path order: row n_ctx + j
+ * takes the row of path node path[j], j = 0 .. L (path[0] = 0, the root, at
+ * n_ctx already).  Rows past n_ctx + L are left as they were.  `accept` is
+ * the int32 {L, bonus, path[0..L]} of tso_accept_longest.  Operates on one
+ * cache (K or V) [Hkv, kv_cap, D] in place.  Returns 0, or -1 on invalid
+ * input.
+ */
+int tso_kv_commit_path(uint16_t *cache, int64_t kv_cap, int n_heads_kv, int head_dim, int n_ctx,
+                       int n_tree, const int32_t *accept)
+{
+    const int len = accept[0];
+    if (len < 0 || len >= n_tree || (int64_t)n_ctx + n_tree > kv_cap)
+        return -1;
+    for (int j = 0; j <= len; ++j)
+        if (accept[2 + j] < j || accept[2 + j] >= n_tree)
+            return -1;
+    uint16_t *rows = (uint16_t *)malloc(sizeof(uint16_t) * (size_t)(len + 1) * head_dim);
+    for (int g = 0; g < n_heads_kv; ++g) {
+        uint16_t *base = cache + (int64_t)g * kv_cap * head_dim;
+        /* every source row is read before any row is written */
+        for (int j = 0; j <= len; ++j)
+            memcpy(rows + (size_t)j * head_dim, base + ((int64_t)n_ctx + accept[2 + j]) * head_dim,
+                   sizeof(uint16_t) * head_dim);
+        for (int j = 0; j <= len; ++j)
+            memcpy(base + ((int64_t)n_ctx + j) * head_dim, rows + (size_t)j * head_dim,
+                   sizeof(uint16_t) * head_dim);
+    }
+    free(rows);
+    return 0;
+}

@@ -32,6 +32,15 @@ C_MUTANTS = {
                                        "return (x->pos < y->pos) - (x->pos > y->pos);"),
     "accept_ties_to_highest_index": ("if (valid[i] && depth[i] > depth[best])",
                                      "if (valid[i] && depth[i] >= depth[best])"),
+    "path_window_includes_root": ("for (int a = i; a != 0; a = parent[a])",
+                                  "for (int a = i; a >= 0; a = parent[a])"),
+    "path_window_without_self": ("for (int a = i; a != 0; a = parent[a])",
+                                 "for (int a = parent[i]; a > 0; a = parent[a])"),
+    "random_tie_off_by_one": ("int pick = (int)(r % (uint64_t)count), best = 0;",
+                              "int pick = (int)((r + 1) % (uint64_t)count), best = 0;"),
+    "commit_writes_rows_in_place": (
+        "memcpy(base + ((int64_t)n_ctx + j) * head_dim, rows + (size_t)j * head_dim,",
+        "memcpy(base + ((int64_t)n_ctx + accept[2 + j]) * head_dim, rows + (size_t)j * head_dim,"),
 }
 
 

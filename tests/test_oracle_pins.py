@@ -341,3 +341,125 @@ def test_accept_matches_exhaustive_path_search(oracle_mod):
         out = oracle_mod.accept_longest(parent, tokens, argmax)
         assert out[0] == best_len and out[1] == argmax[best_end], trial
         assert out[2 + best_len] == best_end
+
+
+# ------------------------------------------------- sampling variants, commit
+SAMPLING = os.path.join(GOLDEN, "sampling_cases.json")
+
+
+def test_path_window_golden_cases(oracle_mod):
+    for c in json.load(open(SAMPLING))["path_window"]:
+        lg = np.array(c["logits"], np.float32)
+        win = np.array(c["window"], np.int32)
+        am = oracle_mod.penalize_argmax_path(lg, win, c["parent"], c["tokens"], c["penalty"])
+        np.testing.assert_array_equal(am, c["argmax_with_path"], err_msg=c["name"])
+        np.testing.assert_array_equal(oracle_mod.penalize_argmax(lg, win, c["penalty"]),
+                                      c["argmax_window_only"], err_msg=c["name"])
+
+
+def test_path_window_is_the_window_with_each_path_added(oracle_mod):
+    """Per node, the result equals the plain penalty run with that node's
+    window widened by its draft-path tokens (collected here by walking the
+    parents), on random trees with small vocabularies (many collisions)."""
+    rng = np.random.default_rng(21)
+    for trial in range(40):
+        t = int(rng.integers(1, 20))
+        vocab = int(rng.integers(2, 40))
+        parent = np.array([-1] + [int(rng.integers(0, i)) for i in range(1, t)], np.int32)
+        tokens = rng.integers(0, vocab, size=t).astype(np.int32)
+        win = rng.integers(0, vocab, size=int(rng.integers(0, 8))).astype(np.int32)
+        lg = rng.normal(0, 2, size=(t, vocab)).astype(np.float32)
+        am = oracle_mod.penalize_argmax_path(lg, win, parent, tokens, 1.2)
+        for i in range(t):
+            path, a = [], i
+            while a != 0:
+                path.append(int(tokens[a]))
+                a = int(parent[a])
+            wi = np.concatenate([win, np.array(path, np.int32)])
+            assert am[i] == oracle_mod.penalize_argmax(lg[i:i + 1], wi, 1.2)[0], (trial, i)
+
+
+def test_path_window_single_node_equals_plain_penalty(oracle_mod):
+    rng = np.random.default_rng(22)
+    lg = rng.normal(0, 2, size=(1, 500)).astype(np.float32)
+    win = rng.integers(0, 500, size=50).astype(np.int32)
+    np.testing.assert_array_equal(
+        oracle_mod.penalize_argmax_path(lg, win, [-1], [7], 1.2),
+        oracle_mod.penalize_argmax(lg, win, 1.2))
+
+
+def test_path_window_rejects_out_of_vocab_tokens(oracle_mod):
+    with pytest.raises(ValueError):
+        oracle_mod.penalize_argmax_path(np.zeros((2, 8), np.float32), np.zeros(0, np.int32),
+                                        [-1, 0], [0, 8], 1.2)
+
+
+def test_random_tie_golden_case(oracle_mod):
+    c = json.load(open(SAMPLING))["random_tie"]
+    for r, exp in c["expected"].items():
+        out = oracle_mod.accept_longest_random(c["parent"], c["tokens"], c["argmax"], int(r))
+        np.testing.assert_array_equal(out[: len(exp)], exp, err_msg=r)
+        assert np.all(out[len(exp):] == -1)
+
+
+def test_random_tie_matches_exhaustive_path_search(oracle_mod):
+    """Random trees with few token values (many equally long valid paths):
+    for every r the kept path is the (r mod c)-th, in end-node order, of the
+    c longest root paths whose every step matches the parent's argmax, and
+    r = 0 is the deterministic lowest-index rule."""
+    rng = np.random.default_rng(23)
+    for trial in range(150):
+        t = int(rng.integers(1, 25))
+        parent = np.array([-1] + [int(rng.integers(0, i)) for i in range(1, t)], np.int32)
+        tokens = rng.integers(0, 2, size=t).astype(np.int32)
+        argmax = rng.integers(0, 2, size=t).astype(np.int32)
+        ends = {}
+        for end in range(t):
+            path, a = [], end
+            while a >= 0:
+                path.append(a)
+                a = int(parent[a])
+            path.reverse()
+            if all(tokens[path[s + 1]] == argmax[path[s]] for s in range(len(path) - 1)):
+                ends.setdefault(len(path) - 1, []).append(end)
+        best_len = max(ends)
+        best = sorted(ends[best_len])
+        for r in range(2 * len(best) + 1):
+            out = oracle_mod.accept_longest_random(parent, tokens, argmax, r)
+            end = best[r % len(best)]
+            assert out[0] == best_len and out[1] == argmax[end] and out[2 + best_len] == end
+        np.testing.assert_array_equal(oracle_mod.accept_longest_random(parent, tokens, argmax, 0),
+                                      oracle_mod.accept_longest(parent, tokens, argmax))
+
+
+def test_commit_golden_case(oracle_mod):
+    c = json.load(open(SAMPLING))["commit"]
+    cache = np.array(c["rows"], np.uint16)[None]
+    out = oracle_mod.kv_commit_path(cache, c["n_ctx"], c["n_tree"], c["accept"])
+    np.testing.assert_array_equal(out[0], np.array(c["expected_rows"], np.uint16))
+    np.testing.assert_array_equal(cache[0], np.array(c["rows"], np.uint16))   # input untouched
+
+
+def test_commit_moves_exactly_the_path_rows(oracle_mod):
+    """Random caches and accepted paths: rows n_ctx + j hold the old rows of
+    the path nodes, every other row is unchanged; L = 0 changes nothing."""
+    rng = np.random.default_rng(24)
+    for trial in range(30):
+        hkv, d, n_ctx, t = 3, 8, int(rng.integers(0, 20)), int(rng.integers(1, 30))
+        cap = n_ctx + t + int(rng.integers(0, 4))
+        cache = rng.integers(0, 65535, size=(hkv, cap, d)).astype(np.uint16)
+        parent = np.array([-1] + [int(rng.integers(0, i)) for i in range(1, t)], np.int32)
+        end = int(rng.integers(0, t))
+        path, a = [], end
+        while a >= 0:
+            path.append(a)
+            a = int(parent[a])
+        path.reverse()
+        acc = np.array([len(path) - 1, 0] + path, np.int32)
+        out = oracle_mod.kv_commit_path(cache, n_ctx, t, acc)
+        want = cache.copy()
+        for j, node in enumerate(path):
+            want[:, n_ctx + j] = cache[:, n_ctx + node]
+        np.testing.assert_array_equal(out, want)
+    cache = rng.integers(0, 65535, size=(2, 10, 4)).astype(np.uint16)
+    np.testing.assert_array_equal(oracle_mod.kv_commit_path(cache, 3, 5, [0, 1, 0]), cache)
