@@ -430,12 +430,12 @@ int tso_penalize_argmax_path(const float *logits, int n_tree, int vocab, const i
         for (int id = 0; id < vocab; ++id) {
             float x = logits[(int64_t)i * vocab + id];
             if (mark[id])
-                x = x > 0.0f ? x / penalty : x * penalty;
+                x = (x > 0.0f) ? (x / penalty) : (x * penalty);
             if (penalized)
                 penalized[(int64_t)i * vocab + id] = x;
             if (x != x)
                 x = -INFINITY;
-            if (x > best) {
+            if (best < x) {
                 best = x;
                 best_id = id;
             }
@@ -468,7 +468,7 @@ int tso_accept_longest_random(const int32_t *parent, const int32_t *tokens,
     int deepest = 0;
     for (int i = 1; i < n_tree; ++i) {
         int p = parent[i];
-        valid[i] = valid[p] && tokens[i] == argmax[p];
+        valid[i] = tokens[i] == argmax[p] && valid[p];
         depth[i] = depth[p] + 1;
         if (valid[i] && depth[i] > deepest)
             deepest = depth[i];

@@ -38,6 +38,11 @@ C_MUTANTS = {
                                  "for (int a = parent[i]; a > 0; a = parent[a])"),
     "random_tie_off_by_one": ("int pick = (int)(r % (uint64_t)count), best = 0;",
                               "int pick = (int)((r + 1) % (uint64_t)count), best = 0;"),
+    "path_penalty_sign_swapped": ("x = (x > 0.0f) ? (x / penalty) : (x * penalty);",
+                                  "x = (x > 0.0f) ? (x * penalty) : (x / penalty);"),
+    "path_argmax_ties_to_highest_id": ("if (best < x) {", "if (best <= x) {"),
+    "random_tie_validity_ignores_parent": ("valid[i] = tokens[i] == argmax[p] && valid[p];",
+                                           "valid[i] = tokens[i] == argmax[p];"),
     "commit_writes_rows_in_place": (
         "memcpy(base + ((int64_t)n_ctx + j) * head_dim, rows + (size_t)j * head_dim,",
         "memcpy(base + ((int64_t)n_ctx + accept[2 + j]) * head_dim, rows + (size_t)j * head_dim,"),
