@@ -46,6 +46,18 @@ AttnPlan attn_tc_plan(int n_heads_q, int n_heads_kv, int n_ctx, int n_tree, int 
 cudaError_t attn_tc_launch(const AttnArgs &a, const TreeMasks &masks, int num_sms,
                            cudaStream_t stream);
 
+// Split partials of the tcgen05 kernels (head_dim 128): acc fp32
+// [n_split, T*Hq, 128] after the workspace header, then (m, l, q, 0) fp32
+// [n_split, T*Hq, 4]: m in log2 units, l the sum of the bf16-rounded
+// weights relative to 2^m, q the sum of their squares.  The combine folds them; it recomputes exactly (fp32, CUDA
+// cores) every split whose int32 flag [n_split, Hkv] is set (flags may be
+// null: none), and the heavy splits of rows whose weight sits on too few
+// positions for bf16 weights.  split_positions: KV positions per split.
+size_t attn_exact_partial_bytes(int n_split, int n_heads_q, int n_tree);
+cudaError_t attn_exact_combine_launch(const AttnArgs &a, const TreeMasks &masks, int n_split,
+                                      int split_positions, const int32_t *flags,
+                                      cudaStream_t stream);
+
 // 128-position tiles, softmax spread over the four SM sub-partitions; up to
 // 192 query rows per KV head.
 bool attn_t128_eligible(int n_heads_q, int n_heads_kv, int head_dim, int n_ctx, int n_tree);
@@ -53,5 +65,8 @@ AttnPlan attn_t128_plan(int n_heads_q, int n_heads_kv, int n_ctx, int n_tree, in
 size_t attn_t128_workspace_bytes(int n_heads_q, int n_heads_kv, int n_ctx, int n_tree, int num_sms);
 cudaError_t attn_t128_launch(const AttnArgs &a, const TreeMasks &masks, int num_sms,
                              cudaStream_t stream);
+// whether that kernel writes a.root_scores itself (G <= 8 root rows inside
+// the first 16 TMEM lanes); otherwise it ignores them
+bool attn_t128_leaves_root_scores(const AttnArgs &a);
 
 }  // namespace ts

@@ -17,7 +17,7 @@ size_t attn_workspace_bytes(int n_heads_q, int n_heads_kv, int head_dim, int n_c
     size_t bytes = attn_mma_workspace_bytes(n_heads_q, n_heads_kv, head_dim, n_ctx, n_tree, num_sms);
     auto take = [&](const AttnPlan &p) {
         const size_t tc = kHeaderBytes +
-                          align_up(attn_partial_bytes(p.n_split, n_heads_q, head_dim, n_tree), 256);
+                          align_up(attn_exact_partial_bytes(p.n_split, n_heads_q, n_tree), 256);
         bytes = tc > bytes ? tc : bytes;
     };
     if (attn_t128_eligible(n_heads_q, n_heads_kv, head_dim, n_ctx, n_tree)) {
@@ -32,18 +32,24 @@ size_t attn_workspace_bytes(int n_heads_q, int n_heads_kv, int head_dim, int n_c
 cudaError_t attn_launch(const AttnArgs &a, const TreeMasks &masks, int num_sms,
                         cudaStream_t stream)
 {
-    if (a.scale_log2 > 0.f &&
-        attn_t128_eligible(a.n_heads_q, a.n_heads_kv, a.head_dim, a.n_ctx, a.n_tree))
-        return attn_t128_launch(a, masks, num_sms, stream);   // leaves root scores itself
     cudaError_t e;
     if (a.scale_log2 > 0.f &&
-        attn_tc_eligible(a.n_heads_q, a.n_heads_kv, a.head_dim, a.n_ctx, a.n_tree))
+        attn_t128_eligible(a.n_heads_q, a.n_heads_kv, a.head_dim, a.n_ctx, a.n_tree)) {
+        if (a.root_scores == nullptr || attn_t128_leaves_root_scores(a))
+            return attn_t128_launch(a, masks, num_sms, stream);   // leaves root scores itself
+        AttnArgs b = a;
+        b.root_scores = nullptr;
+        e = attn_t128_launch(b, masks, num_sms, stream);
+    } else if (a.scale_log2 > 0.f &&
+               attn_tc_eligible(a.n_heads_q, a.n_heads_kv, a.head_dim, a.n_ctx, a.n_tree)) {
         e = attn_tc_launch(a, masks, num_sms, stream);
-    else
+    } else {
         e = attn_mma_launch(a, masks, num_sms, stream);
+    }
     if (e != cudaSuccess || a.root_scores == nullptr || a.n_ctx == 0)
         return e;
-    // the other kernels do not leave root scores: the select's score pass does
+    // the other kernels (and the 128-position one on trees of fewer than
+    // four nodes) do not leave root scores: the select's score pass does
     SelectArgs sa = {};
     sa.q_last = a.q;   // node 0's rows [Hq, D]
     sa.k = a.k;

@@ -28,9 +28,14 @@
 // rows per thread (lanes t/4 and 8 + t/4 of the unit).
 //
 // CTA = (split, KV head), 16 warps, one CTA per SM:
-//   warp 0, 3   TMA producers of K and of V (two 64-column boxes of 128
-//               positions per tile, 128-byte swizzle).  The map's row extent
-//               is n_ctx + T, so rows past the tree tail arrive as zeros.
+//   warp 3      one lane is the TMA producer of K and V (two 64-column boxes
+//               of 128 positions per tile, 128-byte swizzle), K one tile
+//               ahead of V.  The map's row extent is n_ctx + T, so rows past
+//               the tree tail arrive as zeros.
+//   warp 0      when the call asks for the root node's scores and all of
+//               them sit in TMEM lane quarter 0 (the warp's own quarter),
+//               reads them out of S_0 each tile and stores them, so that no
+//               softmax warp carries that work; otherwise idle.
 //   warp 1      allocates TMEM; one lane issues the QK MMAs.  A block's S is
 //               released as soon as its softmax warps hold it in registers.
 //   warp 2      one lane issues the PV MMAs.
@@ -46,15 +51,26 @@
 // The reference max of a row is fixed at the first tile where the row sees
 // anything, and never moves, so the softmax warps need no per-tile
 // agreement with each other and no per-tile maximum at all.  fp32 has room
-// for it: a row's weights are at most its sum l, and while l <= 2^80 the
-// accumulated O^T stays below 2^80 * max|V|, far from overflow (a score
-// rise of about 55 nats inside one split would be needed to exceed it).  A
-// split in which some row's l ends above 2^80 (or not a number) raises a
+// for it: a row's weights are at most its sum l, and while l <= 2^63 the
+// accumulated O^T stays below 2^63 * max|V|, far from overflow (a score
+// rise of about 44 nats inside one split would be needed to exceed it).  A
+// split in which some row's l ends above 2^63 (or not a number) raises a
 // flag; the combine kernel then recomputes that split's partial for the
 // affected head exactly (fp32, online softmax on CUDA cores) instead of
 // reading it.
-// Each split leaves an unnormalised partial (acc, m, l) and its flag; the
-// combine kernel always runs.
+// Each split leaves an unnormalised partial (acc, m, l, q) and its flag;
+// the combine kernel always runs.
+//
+// P enters the PV product as one bf16 value and l sums those same rounded
+// values, so a row's output is an exact weighted mean of V with weights
+// perturbed by at most one bf16 rounding each.  Spread over many positions
+// those perturbations average out (the error falls like 1/sqrt of the
+// effective number of positions); on a row whose weight sits on a handful
+// of positions they do not.  The kernel therefore also keeps q, the sum of
+// the squared rounded weights, so that l^2 / q is the row's effective
+// number of positions.  The combine recomputes exactly (fp32, CUDA cores)
+// the splits that carry the weight of any row whose count over all splits
+// is below kNeffMin.
 //
 // Every wait is on an mbarrier and bounded (about a second): on expiry the
 // kernel records TS_ERR_TIMEOUT in the workspace status word, all roles
@@ -81,7 +97,15 @@ constexpr int kQCol = 192;                   // Q of block 0: 128 bf16 = 64 colu
 constexpr int kSCol = 256;                   // S_b: 128 columns from kSCol + 128 b
 constexpr int kTmemCols = 512;
 constexpr int kQ1Bytes = kBlockM * kD * 2;   // Q of block 1 in shared memory: 32 KB
-constexpr float kMaxRowSum = 1.2089258196146292e24f;   // 2^80: bound on a row's weight sum
+constexpr float kMaxRowSum = 9.223372036854775808e18f;   // 2^63: bound on a row's weight sum
+// Rows whose effective number of attended positions is below this are
+// recomputed exactly.  With each weight perturbed by one bf16 rounding
+// (relative spread 2^-8 / sqrt(3)), the output error of a row with n
+// effective positions has a standard deviation of about
+// 2^-8 / sqrt(3) * rms|v - o| / sqrt(n); at n = 64 and |v - o| ~ 1.4
+// (bf16 N(0,1) values) that is 4e-4, so even the largest of many such
+// errors stays inside 2e-3.
+constexpr float kNeffMin = 64.f;
 constexpr size_t kSmemLimit = 232448;        // dynamic shared memory per CTA
 
 struct Bars {
@@ -109,21 +133,24 @@ constexpr size_t kAuxBytes = (sizeof(Aux) + 1023) / 1024 * 1024;
 struct Layout {
     int r_pad;  // rows rounded up to 16: N of the PV product
     int stages_k, stages_v;
-    size_t q1_off, p_off, k_off, v_off, aux_off, rs_off, smem_bytes;
+    size_t q1_off, p_off, k_off, v_off, aux_off, smem_bytes;
 };
 
-// Shared memory that stages the root node's scores for bulk copies (two
-// tiles of the G root rows), when the call asks for them and every row of
-// them starts on a 16-byte boundary; 0 when they are stored directly.
-__host__ __device__ inline int t128_rs_bytes(const AttnArgs &a)
+// Rows per TMEM lane quarter in block 0 (rows 0..min(R, 128) - 1 cut into
+// four equal runs).
+__host__ __device__ inline int t128_rq0(int rows) { return ((rows < kBlockM ? rows : kBlockM) + 3) / 4; }
+
+// Whether warp 0 reads the root node's scores out of TMEM: the call asks for
+// them and the G root rows (rows 0..G-1) all fall in TMEM lanes 0..15 of
+// lane quarter 0, i.e. G <= 8 and G <= rq0.  For other shapes (trees of
+// fewer than four nodes) the launch leaves them to the select's score pass.
+__host__ __device__ inline bool t128_rs_warp0(const AttnArgs &a)
 {
-    const bool bulk = a.root_scores != nullptr &&
-                      (reinterpret_cast<uintptr_t>(a.root_scores) & 15) == 0 &&
-                      (a.n_ctx & 3) == 0;
-    return bulk ? 2 * (a.n_heads_q / a.n_heads_kv) * kTileN * 4 : 0;
+    const int G = a.n_heads_q / a.n_heads_kv;
+    return a.root_scores != nullptr && G <= 8 && G <= t128_rq0(G * a.n_tree);
 }
 
-__host__ __device__ inline Layout t128_layout(int rows, int rs_bytes)
+__host__ __device__ inline Layout t128_layout(int rows)
 {
     Layout L;
     L.r_pad = (rows + 15) / 16 * 16;
@@ -132,32 +159,33 @@ __host__ __device__ inline Layout t128_layout(int rows, int rs_bytes)
     // P^T: positions 0-63 then 64-127, each r_pad rows of 128 bytes; then
     // 1 KB that rows past the query rows are written to
     L.k_off = L.p_off + (size_t)L.r_pad * 256 + 1024;
-    const size_t fixed = 1024 + L.k_off + kAuxBytes + rs_bytes;
+    const size_t fixed = 1024 + L.k_off + kAuxBytes;
     int stages = (int)((kSmemLimit - fixed) / kStageBytes);
     stages = stages > 2 * kMaxStages ? 2 * kMaxStages : stages;
     L.stages_v = 2;
     L.stages_k = stages - 2 > kMaxStages ? kMaxStages : stages - 2;
     L.v_off = L.k_off + (size_t)L.stages_k * kStageBytes;
     L.aux_off = L.v_off + (size_t)L.stages_v * kStageBytes;
-    L.rs_off = L.aux_off + kAuxBytes;
-    L.smem_bytes = 1024 + L.rs_off + rs_bytes;
+    L.smem_bytes = 1024 + L.aux_off + kAuxBytes;
     return L;
 }
 
 // P = 2^(x * scale - m) for the 32 scores a thread holds of row A
 // (registers r[4j], r[4j + 1], j = 0..15) and, when TWO, of row B
 // (r[4j + 2], r[4j + 3]), packed to bf16 pairs; adds the sums of the rounded
-// values (what the PV product will use) to lA and lB.  Both rows advance
-// together, so each score register is dead once its pair is packed.
+// values (what the PV product will use) to lA and lB, and their squares to
+// qA and qB.  Both rows advance together, so each score register is dead
+// once its pair is packed.
 template <bool TWO>
 __device__ __forceinline__ void exp_pack_rows(const uint32_t (&r)[64], float scale, float neg_mA,
                                               float neg_mB, uint32_t (&pA)[16],
-                                              uint32_t (&pB)[16], float &lA, float &lB)
+                                              uint32_t (&pB)[16], float &lA, float &lB,
+                                              float &qA, float &qB)
 {
     const uint64_t sc2 = pack2(scale, scale);
     const uint64_t nA2 = pack2(neg_mA, neg_mA);
     const uint64_t nB2 = pack2(neg_mB, neg_mB);
-    uint64_t sA = 0ull, sB = 0ull;
+    uint64_t sA = 0ull, sB = 0ull, wA = 0ull, wB = 0ull;
 #pragma unroll
     for (int j = 0; j < 16; ++j) {
 #pragma unroll
@@ -174,18 +202,26 @@ __device__ __forceinline__ void exp_pack_rows(const uint32_t (&r)[64], float sca
             if (h) {
                 pB[j] = hb;
                 sB = add2(sB, e2);
+                wB = fma2(e2, e2, wB);
             } else {
                 pA[j] = hb;
                 sA = add2(sA, e2);
+                wA = fma2(e2, e2, wA);
             }
         }
     }
+    // a split whose rows keep l <= 2^63 has every sum of squares <= l^2 <=
+    // 2^126, inside the fp32 range (a larger l flags the split anyway)
     float a0, a1;
     unpack2(sA, a0, a1);
     lA += a0 + a1;
+    unpack2(wA, a0, a1);
+    qA += a0 + a1;
     if (TWO) {
         unpack2(sB, a0, a1);
         lB += a0 + a1;
+        unpack2(wB, a0, a1);
+        qB += a0 + a1;
     }
 }
 
@@ -242,8 +278,8 @@ attn_t128_kernel(const __grid_constant__ CUtensorMap tmap_k,
     const int rq0 = (R0 + 3) / 4, rq1 = (R1 + 3) / 4;  // rows per lane quarter
     const int u0 = (rq0 + 15) / 16, u1 = (rq1 + 15) / 16;
     const int U = u0 + u1;  // softmax warps per lane quarter (at most 3)
-    const int rs_bytes = t128_rs_bytes(a);
-    const Layout lay = t128_layout(R, rs_bytes);
+    const bool rs_warp0 = t128_rs_warp0(a);
+    const Layout lay = t128_layout(R);
     const int SK = lay.stages_k, SV = lay.stages_v, r_pad = lay.r_pad;
 
     extern __shared__ unsigned char smem_raw[];
@@ -276,7 +312,7 @@ attn_t128_kernel(const __grid_constant__ CUtensorMap tmap_k,
         }
         mbar_init(smem_addr(&bar->s_full[0]), 1);
         mbar_init(smem_addr(&bar->s_full[1]), 1);
-        mbar_init(smem_addr(&bar->s_free[0]), 4 * u0);
+        mbar_init(smem_addr(&bar->s_free[0]), 4 * u0 + (rs_warp0 ? 1 : 0));
         mbar_init(smem_addr(&bar->s_free[1]), u1 > 0 ? 4 * u1 : 1);
         mbar_init(smem_addr(&bar->sm_done), 4 * U);
         mbar_init(smem_addr(&bar->pv_done), 1);
@@ -293,7 +329,7 @@ attn_t128_kernel(const __grid_constant__ CUtensorMap tmap_k,
         tmem_alloc(smem_addr(&bar->tmem_base), kTmemCols);
         tmem_relinquish();
     }
-    if (warp == 0 && lane == 0) {
+    if (warp == 3 && lane == 0) {
         prefetch_tmap(&tmap_k);
         prefetch_tmap(&tmap_v);
     }
@@ -354,34 +390,94 @@ attn_t128_kernel(const __grid_constant__ CUtensorMap tmap_k,
     __syncthreads();
     tc_fence_after();
 
-    if (warp == 0 || warp == 3) {
-        // ----------------------------------------- TMA producers (K, V)
+    if (warp == 3) {
+        // ------------------------------------ TMA producer (K one tile ahead)
         if (lane == 0) {
-            const bool is_k = warp == 0;
-            const int ns = is_k ? SK : SV;
-            uint64_t *full = is_k ? bar->full_k : bar->full_v;
-            uint64_t *empty = is_k ? bar->empty_k : bar->empty_v;
-            unsigned char *ring = is_k ? sK : sV;
-            const void *tmap = is_k ? static_cast<const void *>(&tmap_k)
-                                    : static_cast<const void *>(&tmap_v);
-            int issued = 0;
-            for (int t = 0; t < n_tiles; ++t) {
-                const int s = t % ns;
-                if (t >= ns &&
-                    !wait_bounded(smem_addr(&empty[s]), ((t / ns) & 1) ^ 1, abort, hdr))
+            int nk = 0, nv = 0;   // tiles issued so far
+            // step i issues K(i), then V(i - 1): K is consumed a whole softmax
+            // pass before V, and each load waits only for its own ring slot
+            for (int i = 0; i <= n_tiles; ++i) {
+                bool ok = true;
+#pragma unroll 1
+                for (int which = 0; which < 2 && ok; ++which) {
+                    const bool is_k = which == 0;
+                    const int t = is_k ? i : i - 1;
+                    if (t < 0 || t >= n_tiles)
+                        continue;
+                    const int ns = is_k ? SK : SV;
+                    const int s = t % ns;
+                    uint64_t *full = is_k ? bar->full_k : bar->full_v;
+                    uint64_t *empty = is_k ? bar->empty_k : bar->empty_v;
+                    if (t >= ns &&
+                        !wait_bounded(smem_addr(&empty[s]), ((t / ns) & 1) ^ 1, abort, hdr)) {
+                        ok = false;
+                        break;
+                    }
+                    const uint32_t fb = smem_addr(&full[s]);
+                    mbar_arrive_expect_tx(fb, kStageBytes);
+                    const uint32_t dst = smem_addr((is_k ? sK : sV) + s * kStageBytes);
+                    const void *tmap = is_k ? static_cast<const void *>(&tmap_k)
+                                            : static_cast<const void *>(&tmap_v);
+                    const int pos0 = (t_begin + t) * kTileN;
+                    tma_load_3d(dst, tmap, 0, pos0, g, fb);
+                    tma_load_3d(dst + kBoxBytes, tmap, 64, pos0, g, fb);
+                    if (is_k)
+                        nk = t + 1;
+                    else
+                        nv = t + 1;
+                }
+                if (!ok)
                     break;
-                const uint32_t fb = smem_addr(&full[s]);
-                mbar_arrive_expect_tx(fb, kStageBytes);
-                const uint32_t dst = smem_addr(ring + s * kStageBytes);
-                const int pos0 = (t_begin + t) * kTileN;
-                tma_load_3d(dst, tmap, 0, pos0, g, fb);
-                tma_load_3d(dst + kBoxBytes, tmap, 64, pos0, g, fb);
-                issued = t + 1;
             }
             if (*abort) {
                 // let our own copies land before the CTA exits
-                for (int t = max(0, issued - ns); t < issued; ++t)
-                    wait_drain(smem_addr(&full[t % ns]), (t / ns) & 1);
+                for (int t = max(0, nk - SK); t < nk; ++t)
+                    wait_drain(smem_addr(&bar->full_k[t % SK]), (t / SK) & 1);
+                for (int t = max(0, nv - SV); t < nv; ++t)
+                    wait_drain(smem_addr(&bar->full_v[t % SV]), (t / SV) & 1);
+            }
+        }
+    } else if (warp == 0) {
+        // --------------------------- root node's scores out of S_0 (lanes 0..G-1)
+        if (rs_warp0) {
+            // one 16x256b load of lanes 0..15, the shape the softmax warps
+            // use: thread t holds lane t/4 (and 8 + t/4) at columns
+            // 8j + 2(t%4) + {0, 1}, so threads 0..4G-1 hold the G root rows
+            const int r = lane >> 2;          // root row of this thread (lanes 0..7)
+            const bool mine = r < G;
+            const int c0 = 2 * (lane & 3);
+            float *dst_row = a.root_scores + (size_t)(g * G + (mine ? r : 0)) * a.n_ctx;
+            const bool vec = ((reinterpret_cast<uintptr_t>(a.root_scores) | (uintptr_t)a.n_ctx * 4) &
+                              7) == 0;
+            for (int t = 0; t < n_tiles; ++t) {
+                if (!warp_wait_bounded(smem_addr(&bar->s_full[0]), t & 1, abort, hdr))
+                    break;
+                tc_fence_after();
+                const int pos0 = (t_begin + t) * kTileN;
+                uint32_t rr[64];
+                if (pos0 < a.n_ctx)
+                    tmem_ld16x256_x16(tmem + kSCol, rr);
+                // S_0 is read: QK of the next tile may overwrite it
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0)
+                    mbar_arrive(smem_addr(&bar->s_free[0]));
+                if (pos0 >= a.n_ctx || !mine)
+                    continue;   // a tile of the tree tail only, or not a root lane
+#pragma unroll
+                for (int jj = 0; jj < 16; ++jj) {
+                    const int p = pos0 + 8 * jj + c0;
+                    const float x0 = __uint_as_float(rr[4 * jj]) * a.scale_log2;
+                    const float x1 = __uint_as_float(rr[4 * jj + 1]) * a.scale_log2;
+                    if (vec && p + 1 < a.n_ctx) {
+                        *reinterpret_cast<float2 *>(dst_row + p) = make_float2(x0, x1);
+                    } else {
+                        if (p < a.n_ctx)
+                            dst_row[p] = x0;
+                        if (p + 1 < a.n_ctx)
+                            dst_row[p + 1] = x1;
+                    }
+                }
             }
         }
     } else if (warp == 1 || warp == 2) {
@@ -488,13 +584,7 @@ attn_t128_kernel(const __grid_constant__ CUtensorMap tmap_k,
         const int nvB = max(0, min(8, min(rqb - lb - 8, Rb - q * rqb - lb - 8)));
         const uint32_t p_addr = smem_addr(sP);
         const uint32_t p_scratch = p_addr + (uint32_t)r_pad * 256;
-        float mA = -INFINITY, mB = -INFINITY, lA = 0.f, lB = 0.f;
-        // root rows (node 0: rows 0..G-1) held by this thread and this warp;
-        // the first lane of a row's quad copies its staged scores out
-        const bool rootA = vA && nA < G, rootB = vB && nB < G;
-        const bool rs_warp =
-            a.root_scores != nullptr && __any_sync(0xffffffffu, rootA || rootB);
-        const bool rs_issue = rs_bytes != 0 && (lane & 3) == 0 && (rootA || rootB);
+        float mA = -INFINITY, mB = -INFINITY, lA = 0.f, lB = 0.f, qA = 0.f, qB = 0.f;
         bool ok = true;
         for (int t = 0; t < n_tiles; ++t) {
             if (!warp_wait_bounded(smem_addr(&bar->s_full[b]), t & 1, abort, hdr)) {
@@ -511,64 +601,6 @@ attn_t128_kernel(const __grid_constant__ CUtensorMap tmap_k,
                 mbar_arrive(smem_addr(&bar->s_free[b]));
             // raw scores; the scale (> 0) is applied inside the exponent
             const int pos0 = (t_begin + t) * kTileN;
-            // the root node's rows (0..G-1) leave their context scores, base
-            // 2, for the importance select
-            if (rs_warp && pos0 < a.n_ctx) {
-                if (rs_bytes != 0) {
-                    // staged in shared memory (one buffer per tile parity)
-                    // and written out by bulk copies, so that no global
-                    // store sits ahead of this warp's barrier arrivals
-                    const uint32_t buf =
-                        smem_addr(base + lay.rs_off) + (uint32_t)((t & 1) * G * kTileN * 4);
-                    if (rs_issue)
-                        bulk_wait_read<1>();   // the copy out of this buffer two tiles ago
-                    __syncwarp();
-#pragma unroll
-                    for (int h = 0; h < 2; ++h) {
-                        if (h ? rootB : rootA) {
-                            const uint32_t row =
-                                buf + (uint32_t)((h ? nB : nA) * kTileN * 4 + c0 * 4);
-#pragma unroll
-                            for (int jj = 0; jj < 16; ++jj)
-                                st_shared_v2(row + 32 * jj,
-                                             __float_as_uint(__uint_as_float(r[4 * jj + 2 * h]) *
-                                                             a.scale_log2),
-                                             __float_as_uint(__uint_as_float(r[4 * jj + 2 * h + 1]) *
-                                                             a.scale_log2));
-                        }
-                    }
-                    fence_proxy_async_smem();
-                    __syncwarp();
-                    if (rs_issue) {
-                        const uint32_t bytes = (uint32_t)min(kTileN, a.n_ctx - pos0) * 4;
-#pragma unroll
-                        for (int h = 0; h < 2; ++h) {
-                            const int n = h ? nB : nA;
-                            if (h ? rootB : rootA)
-                                bulk_store(a.root_scores + (size_t)(g * G + n) * a.n_ctx + pos0,
-                                           buf + (uint32_t)(n * kTileN * 4), bytes);
-                        }
-                        bulk_commit();
-                    }
-                } else {
-#pragma unroll
-                    for (int h = 0; h < 2; ++h) {
-                        if (h ? rootB : rootA) {
-                            float *dst = a.root_scores + (size_t)(g * G + (h ? nB : nA)) * a.n_ctx;
-#pragma unroll
-                            for (int jj = 0; jj < 16; ++jj) {
-#pragma unroll
-                                for (int e = 0; e < 2; ++e) {
-                                    const int pos = pos0 + 8 * jj + c0 + e;
-                                    if (pos < a.n_ctx)
-                                        dst[pos] =
-                                            __uint_as_float(r[4 * jj + 2 * h + e]) * a.scale_log2;
-                                }
-                            }
-                        }
-                    }
-                }
-            }
             if (pos0 + kTileN > a.n_ctx) {
                 // visibility of this thread's 32 positions (entry k = 2 jj + e
                 // is position pos0 + 8 jj + c0 + e) for its two rows
@@ -612,9 +644,9 @@ attn_t128_kernel(const __grid_constant__ CUtensorMap tmap_k,
                 const float nmA = mA == -INFINITY ? 0.f : -mA;
                 const float nmB = mB == -INFINITY ? 0.f : -mB;
                 if (hasB)
-                    exp_pack_rows<true>(r, a.scale_log2, nmA, nmB, pA, pB, lA, lB);
+                    exp_pack_rows<true>(r, a.scale_log2, nmA, nmB, pA, pB, lA, lB, qA, qB);
                 else if (hasA)
-                    exp_pack_rows<false>(r, a.scale_log2, nmA, nmB, pA, pB, lA, lB);
+                    exp_pack_rows<false>(r, a.scale_log2, nmA, nmB, pA, pB, lA, lB, qA, qB);
             }
             // P^T is free once PV(t-1) is done.  This warp saw PV(t-2) done
             // before writing P^T(t-1), and PV(t) waits for this warp, so
@@ -633,14 +665,15 @@ attn_t128_kernel(const __grid_constant__ CUtensorMap tmap_k,
             if (lane == 0)
                 mbar_arrive(smem_addr(&bar->sm_done));
         }
-        if (rs_issue)
-            bulk_wait_all();   // shared memory must outlive the copies out of it
         // ---- (m, l) of each row (four threads' partial sums), then O^T
-        lA += __shfl_xor_sync(0xffffffffu, lA, 1);
-        lB += __shfl_xor_sync(0xffffffffu, lB, 1);
-        lA += __shfl_xor_sync(0xffffffffu, lA, 2);
-        lB += __shfl_xor_sync(0xffffffffu, lB, 2);
-        // every weight of a row is at most its sum: a sum past 2^80 (or not a
+#pragma unroll
+        for (int o = 1; o <= 2; o <<= 1) {
+            lA += __shfl_xor_sync(0xffffffffu, lA, o);
+            lB += __shfl_xor_sync(0xffffffffu, lB, o);
+            qA += __shfl_xor_sync(0xffffffffu, qA, o);
+            qB += __shfl_xor_sync(0xffffffffu, qB, o);
+        }
+        // every weight of a row is at most its sum: a sum past 2^63 (or not a
         // number) flags the split for the exact recompute
         const bool over = (vA && !(lA <= kMaxRowSum)) || (vB && !(lB <= kMaxRowSum));
         if (__any_sync(0xffffffffu, over) && lane == 0)
@@ -652,11 +685,11 @@ attn_t128_kernel(const __grid_constant__ CUtensorMap tmap_k,
         auto orow_of = [&](int n) { return (n / G) * a.n_heads_q + g * G + n % G; };
         if (ok && (lane & 3) == 0) {
             if (vA)
-                *reinterpret_cast<float2 *>(ws_ml + ((size_t)split * rows_all + orow_of(nA)) * 2) =
-                    make_float2(mA, lA);
+                *reinterpret_cast<float4 *>(ws_ml + ((size_t)split * rows_all + orow_of(nA)) * 4) =
+                    make_float4(mA, lA, qA, 0.f);
             if (vB)
-                *reinterpret_cast<float2 *>(ws_ml + ((size_t)split * rows_all + orow_of(nB)) * 2) =
-                    make_float2(mB, lB);
+                *reinterpret_cast<float4 *>(ws_ml + ((size_t)split * rows_all + orow_of(nB)) * 4) =
+                    make_float4(mB, lB, qB, 0.f);
         }
         if (ok && warp_wait_bounded(smem_addr(&bar->o_final), 0, abort, hdr)) {
             tc_fence_after();
@@ -689,11 +722,13 @@ attn_t128_kernel(const __grid_constant__ CUtensorMap tmap_k,
 // fp32 from K and V by an online softmax over the split's visible
 // positions.  One warp; lane holds head dims 4 lane .. 4 lane + 3.  Used
 // only for splits whose flag says the kernel's fixed reference max ran out
-// of headroom.
+// of headroom, and for the splits that carry the weight of a row whose
+// weight sits on too few positions for one bf16 rounding of P.
 __device__ void split_partial_exact(const AttnArgs &a, unsigned long long anc, int g,
                                     const float (&q4)[4], int p0, int p1, float &m, float &l,
                                     float (&acc)[4])
 {
+    constexpr int kU = 8;   // positions per step: their loads and reductions overlap
     const int lane = threadIdx.x & 31;
     const __nv_bfloat16 *kh = a.k + (size_t)g * a.kv_cap * kD + 4 * lane;
     const __nv_bfloat16 *vh = a.v + (size_t)g * a.kv_cap * kD + 4 * lane;
@@ -702,42 +737,67 @@ __device__ void split_partial_exact(const AttnArgs &a, unsigned long long anc, i
 #pragma unroll
     for (int e = 0; e < 4; ++e)
         acc[e] = 0.f;
-    for (int pos = p0; pos < p1; ++pos) {
-        const int tp = pos - a.n_ctx;
-        if (tp >= 0 && !((anc >> tp) & 1ull))
-            continue;
-        const uint2 kb = *reinterpret_cast<const uint2 *>(kh + (size_t)pos * kD);
-        const float2 k01 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&kb.x));
-        const float2 k23 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&kb.y));
-        float dot = q4[0] * k01.x + q4[1] * k01.y + q4[2] * k23.x + q4[3] * k23.y;
+    for (int pos0 = p0; pos0 < p1; pos0 += kU) {
+        float sc[kU];
+        bool seen[kU];
+#pragma unroll
+        for (int u = 0; u < kU; ++u) {
+            const int pos = pos0 + u;
+            const int tp = pos - a.n_ctx;
+            seen[u] = pos < p1 && (tp < 0 || ((anc >> tp) & 1ull));
+            const uint2 kb = seen[u] ? *reinterpret_cast<const uint2 *>(kh + (size_t)pos * kD)
+                                     : make_uint2(0u, 0u);
+            const float2 k01 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&kb.x));
+            const float2 k23 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&kb.y));
+            sc[u] = q4[0] * k01.x + q4[1] * k01.y + q4[2] * k23.x + q4[3] * k23.y;
+        }
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1)
-            dot += __shfl_xor_sync(0xffffffffu, dot, o);
-        const float sc = dot * a.scale_log2;
-        if (sc > m) {
-            const float f = exp2f(m - sc);
+#pragma unroll
+            for (int u = 0; u < kU; ++u)
+                sc[u] += __shfl_xor_sync(0xffffffffu, sc[u], o);
+        float mx = -INFINITY;
+#pragma unroll
+        for (int u = 0; u < kU; ++u) {
+            sc[u] = seen[u] ? sc[u] * a.scale_log2 : -INFINITY;
+            mx = fmaxf(mx, sc[u]);
+        }
+        if (mx == -INFINITY)
+            continue;
+        if (mx > m) {
+            const float f = m == -INFINITY ? 0.f : exp2f(m - mx);
             l *= f;
 #pragma unroll
             for (int e = 0; e < 4; ++e)
                 acc[e] *= f;
-            m = sc;
+            m = mx;
         }
-        const float pw = exp2f(sc - m);
-        const uint2 vb = *reinterpret_cast<const uint2 *>(vh + (size_t)pos * kD);
-        const float2 v01 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&vb.x));
-        const float2 v23 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&vb.y));
-        l += pw;
-        acc[0] += pw * v01.x;
-        acc[1] += pw * v01.y;
-        acc[2] += pw * v23.x;
-        acc[3] += pw * v23.y;
+#pragma unroll
+        for (int u = 0; u < kU; ++u) {
+            if (!seen[u])
+                continue;
+            const float pw = exp2f(sc[u] - m);
+            const uint2 vb = *reinterpret_cast<const uint2 *>(vh + (size_t)(pos0 + u) * kD);
+            const float2 v01 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&vb.x));
+            const float2 v23 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&vb.y));
+            l += pw;
+            acc[0] += pw * v01.x;
+            acc[1] += pw * v01.y;
+            acc[2] += pw * v23.x;
+            acc[3] += pw * v23.y;
+        }
     }
 }
 
 // One warp per output row: out = sum_s 2^(m_s - M) acc_s / sum_s 2^(m_s - M) l_s
-// over the splits' partials, with flagged splits recomputed exactly.
+// over the splits' partials.  Recomputed exactly instead of read: splits
+// flagged for overflow, and, on a row whose effective number of positions
+// may be below kNeffMin (L^2 < kNeffMin * sum_s c_s^2 q_s with c_s =
+// 2^(m_s - M)), every split s whose c_s^2 q_s is above L^2 / (kNeffMin *
+// n_split) -- the remaining splits then add up to a bound of at least
+// kNeffMin on their own.
 __global__ void __launch_bounds__(256)
-attn_t128_combine_kernel(AttnArgs a, TreeMasks masks, int n_split, int tiles_per_split,
+attn_t128_combine_kernel(AttnArgs a, TreeMasks masks, int n_split, int split_positions,
                          const int32_t *__restrict__ flags)
 {
     const int rows_all = a.n_tree * a.n_heads_q;
@@ -750,77 +810,102 @@ attn_t128_combine_kernel(AttnArgs a, TreeMasks masks, int n_split, int tiles_per
     const float *ws_o =
         reinterpret_cast<const float *>(reinterpret_cast<const char *>(a.workspace) + kHeaderBytes);
     const float *ws_ml = ws_o + (size_t)n_split * rows_all * kD;
+    auto mlq_of = [&](int s) {
+        return __ldcg(reinterpret_cast<const float4 *>(ws_ml + ((size_t)s * rows_all + row) * 4));
+    };
+
+    // pass 1 over the (m, l, q) of every split: M, and L and the bound's
+    // denominator over the splits that are not flagged
     bool any = false;
-    for (int s = lane; s < n_split; s += 32)
-        any |= flags[s * a.n_heads_kv + g] != 0;
+    float M = -INFINITY;
+    auto flagged = [&](int s) { return flags != nullptr && flags[s * a.n_heads_kv + g] != 0; };
+    for (int s = lane; s < n_split; s += 32) {
+        const bool f = flagged(s);
+        any |= f;
+        if (!f)
+            M = fmaxf(M, mlq_of(s).x);
+    }
     any = __any_sync(0xffffffffu, any);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1)
+        M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+    // L^2 and the q sums reach 2^126 times the splits squared: the count is
+    // formed in fp64
+    double Lp = 0.0, Qp = 0.0;
+    if (M != -INFINITY) {
+        for (int s = lane; s < n_split; s += 32) {
+            if (flagged(s))
+                continue;
+            const float4 x = mlq_of(s);
+            const double c = x.x == -INFINITY ? 0.0 : (double)exp2f(x.x - M);
+            Lp += c * (double)x.y;
+            Qp += c * c * (double)x.z;
+        }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        Lp += __shfl_xor_sync(0xffffffffu, Lp, o);
+        Qp += __shfl_xor_sync(0xffffffffu, Qp, o);
+    }
+    const bool peaked = Lp * Lp < (double)kNeffMin * Qp;   // uniform across the warp
+    const double heavy = Lp * Lp / ((double)kNeffMin * n_split);
 
     float acc[4] = {0.f, 0.f, 0.f, 0.f};
     float L = 0.f;
-    if (!any) {
-        // one pass: splits in batches of kB whose loads are in flight
-        // together, folded into a running (M, L, acc)
+    if (!any && !peaked) {
+        // every partial is used as it is; M is known, so the splits are
+        // summed in batches of kB whose loads are in flight together
         constexpr int kB = 9;
-        float M = -INFINITY;
         for (int s0 = 0; s0 < n_split; s0 += kB) {
-            float2 ml[kB];
-            float4 x[kB];
+            float4 mlq[kB], x[kB];
 #pragma unroll
             for (int u = 0; u < kB; ++u) {
                 const int s = s0 + u;
                 if (s < n_split) {
-                    ml[u] = __ldcg(
-                        reinterpret_cast<const float2 *>(ws_ml + ((size_t)s * rows_all + row) * 2));
+                    mlq[u] = mlq_of(s);
                     x[u] = __ldcg(reinterpret_cast<const float4 *>(
                         ws_o + ((size_t)s * rows_all + row) * kD + 4 * lane));
                 } else {
-                    ml[u] = make_float2(-INFINITY, 0.f);
+                    mlq[u] = make_float4(-INFINITY, 0.f, 0.f, 0.f);
                     x[u] = make_float4(0.f, 0.f, 0.f, 0.f);
                 }
             }
-            float Mb = M;
-#pragma unroll
-            for (int u = 0; u < kB; ++u)
-                Mb = fmaxf(Mb, ml[u].x);
-            if (Mb == -INFINITY)
-                continue;
-            const float fa = M == -INFINITY ? 0.f : exp2f(M - Mb);
-            L *= fa;
-#pragma unroll
-            for (int e = 0; e < 4; ++e)
-                acc[e] *= fa;
 #pragma unroll
             for (int u = 0; u < kB; ++u) {
-                const float w = ml[u].x == -INFINITY ? 0.f : exp2f(ml[u].x - Mb);
-                L += w * ml[u].y;
+                const float w = mlq[u].x == -INFINITY ? 0.f : exp2f(mlq[u].x - M);
+                L += w * mlq[u].y;
                 acc[0] += w * x[u].x;
                 acc[1] += w * x[u].y;
                 acc[2] += w * x[u].z;
                 acc[3] += w * x[u].w;
             }
-            M = Mb;
         }
     } else {
-        // fold the splits one by one into a running (M, L, acc)
+        // fold the splits one by one into a running (Mr, L, acc), the
+        // flagged and the heavy ones recomputed
         const uint2 qb = *reinterpret_cast<const uint2 *>(a.q + (size_t)row * kD + 4 * lane);
         const float2 q01 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&qb.x));
         const float2 q23 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&qb.y));
         const float q4[4] = {q01.x, q01.y, q23.x, q23.y};
         const int total = a.n_ctx + a.n_tree;
-        float M = -INFINITY;
+        float Mr = -INFINITY;
         for (int s = 0; s < n_split; ++s) {
             float ms, ls, as[4];
-            if (flags[s * a.n_heads_kv + g]) {
-                const int p0 = s * tiles_per_split * kTileN;
-                const int p1 = min(p0 + tiles_per_split * kTileN, total);
+            const float4 x4 = mlq_of(s);
+            bool exact = flagged(s);
+            if (!exact && peaked && x4.x != -INFINITY) {
+                const double c = (double)exp2f(x4.x - M);
+                exact = c * c * (double)x4.z > heavy;
+            }
+            if (exact) {
+                const int p0 = s * split_positions;
+                const int p1 = min(p0 + split_positions, total);
                 split_partial_exact(a, masks.anc[node], g, q4, p0, p1, ms, ls, as);
             } else {
-                const float2 ml = __ldcg(
-                    reinterpret_cast<const float2 *>(ws_ml + ((size_t)s * rows_all + row) * 2));
                 const float4 x = __ldcg(reinterpret_cast<const float4 *>(
                     ws_o + ((size_t)s * rows_all + row) * kD + 4 * lane));
-                ms = ml.x;
-                ls = ml.y;
+                ms = x4.x;
+                ls = x4.y;
                 as[0] = x.x;
                 as[1] = x.y;
                 as[2] = x.z;
@@ -828,14 +913,14 @@ attn_t128_combine_kernel(AttnArgs a, TreeMasks masks, int n_split, int tiles_per
             }
             if (ms == -INFINITY)
                 continue;
-            const float Mn = fmaxf(M, ms);
-            const float fa = M == -INFINITY ? 0.f : exp2f(M - Mn);
+            const float Mn = fmaxf(Mr, ms);
+            const float fa = Mr == -INFINITY ? 0.f : exp2f(Mr - Mn);
             const float fb = exp2f(ms - Mn);
             L = L * fa + ls * fb;
 #pragma unroll
             for (int e = 0; e < 4; ++e)
                 acc[e] = acc[e] * fa + as[e] * fb;
-            M = Mn;
+            Mr = Mn;
         }
     }
     const float inv = 1.f / L;
@@ -843,11 +928,13 @@ attn_t128_combine_kernel(AttnArgs a, TreeMasks masks, int n_split, int tiles_per
         make_float4(acc[0] * inv, acc[1] * inv, acc[2] * inv, acc[3] * inv);
 }
 
-// Split partials (acc, m, l) after the header, then one int32 overflow flag
-// per (split, KV head).
+// Split partials (acc fp32 [n_split, T*Hq, D], then (m, l, q, 0) fp32
+// [n_split, T*Hq, 4]) after the header, then one int32 overflow flag per
+// (split, KV head).
+
 size_t flags_offset(int n_split, int n_heads_q, int n_tree)
 {
-    return kHeaderBytes + align_up(attn_partial_bytes(n_split, n_heads_q, kD, n_tree), 256);
+    return kHeaderBytes + align_up(attn_exact_partial_bytes(n_split, n_heads_q, n_tree), 256);
 }
 
 }  // namespace
@@ -886,7 +973,7 @@ cudaError_t attn_t128_launch(const AttnArgs &a, const TreeMasks &masks, int num_
     if (!encode_kv_map(&mk, a.k, rows, a.kv_cap, a.n_heads_kv, kTileN) ||
         !encode_kv_map(&mv, a.v, rows, a.kv_cap, a.n_heads_kv, kTileN))
         return cudaErrorInvalidValue;
-    const Layout lay = t128_layout((a.n_heads_q / a.n_heads_kv) * a.n_tree, t128_rs_bytes(a));
+    const Layout lay = t128_layout((a.n_heads_q / a.n_heads_kv) * a.n_tree);
     static const cudaError_t attr = cudaFuncSetAttribute(
         attn_t128_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemLimit);
     if (attr != cudaSuccess)
@@ -899,10 +986,25 @@ cudaError_t attn_t128_launch(const AttnArgs &a, const TreeMasks &masks, int num_
     if (e != cudaSuccess)
         return e;
     count_launches(1);
+    return attn_exact_combine_launch(a, masks, p.n_split, p.tiles_per_split * kTileN, flags,
+                                     stream);
+}
+
+bool attn_t128_leaves_root_scores(const AttnArgs &a) { return t128_rs_warp0(a); }
+
+size_t attn_exact_partial_bytes(int n_split, int n_heads_q, int n_tree)
+{
+    return (size_t)n_split * n_tree * n_heads_q * (kD + 4) * sizeof(float);
+}
+
+cudaError_t attn_exact_combine_launch(const AttnArgs &a, const TreeMasks &masks, int n_split,
+                                      int split_positions, const int32_t *flags,
+                                      cudaStream_t stream)
+{
     const int rows_all = a.n_tree * a.n_heads_q;
-    attn_t128_combine_kernel<<<(rows_all + 7) / 8, 256, 0, stream>>>(a, masks, p.n_split,
-                                                                      p.tiles_per_split, flags);
-    e = cudaGetLastError();
+    attn_t128_combine_kernel<<<(rows_all + 7) / 8, 256, 0, stream>>>(a, masks, n_split,
+                                                                      split_positions, flags);
+    const cudaError_t e = cudaGetLastError();
     if (e == cudaSuccess)
         count_launches(1);
     return e;

@@ -44,8 +44,10 @@
 //               rescale that row's O^T column.  At the end they write O^T.
 // TMEM: O^T in [0, kOCols), Q_b in 64 columns from kQCol0, S_b in 64
 // columns from kSCol0.
-// Each split leaves an unnormalised partial (acc, m, l) for the combine
-// kernel, or normalises in place when it is the only split.
+// Each split leaves an unnormalised partial (acc, m, l, q) for the combine
+// kernel; q is the sum of the squared bf16 weights, so that the combine can
+// recompute exactly the rows whose weight sits on too few positions for one
+// bf16 rounding of P each.
 //
 // Every wait is on an mbarrier and bounded (about a second): on expiry the
 // kernel records TS_ERR_TIMEOUT in the workspace status word, all roles
@@ -93,8 +95,6 @@ struct TcBarriers {
 
 struct TcAux {
     float factor[2][256];  // per-row O^T rescale factor of the tile (32-column reads)
-    float l[256];
-    float m[256];
     TcBarriers bar;
 };
 constexpr size_t kAuxBytes = (sizeof(TcAux) + 1023) / 1024 * 1024;
@@ -129,7 +129,7 @@ __host__ __device__ inline TcLayout tc_layout(int nb, int rows)
 // P = 2^(x * scale - m) for the 64 scores of one row, packed to bf16 pairs;
 // returns the sum of the rounded values (what the PV product will use).
 __device__ __forceinline__ float exp_pack_tile(const float (&x)[64], float scale, float neg_m,
-                                               uint32_t (&pk)[32])
+                                               uint32_t (&pk)[32], float &sq)
 {
     const uint64_t sc2 = pack2(scale, scale);
     const uint64_t nm2 = pack2(neg_m, neg_m);
@@ -137,7 +137,7 @@ __device__ __forceinline__ float exp_pack_tile(const float (&x)[64], float scale
 #pragma unroll
     for (int j = 0; j < 32; ++j)
         y[j] = fma2(pack2(x[2 * j], x[2 * j + 1]), sc2, nm2);
-    uint64_t ls2[4] = {0ull, 0ull, 0ull, 0ull};
+    uint64_t ls2[4] = {0ull, 0ull, 0ull, 0ull}, qs2[2] = {0ull, 0ull};
 #pragma unroll
     for (int j = 0; j < 32; ++j) {
         float y0, y1;
@@ -145,11 +145,15 @@ __device__ __forceinline__ float exp_pack_tile(const float (&x)[64], float scale
         __nv_bfloat162 h = __floats2bfloat162_rn(ex2(y0), ex2(y1));
         const uint32_t hb = *reinterpret_cast<uint32_t *>(&h);
         pk[j] = hb;
-        ls2[j & 3] = add2(ls2[j & 3],
-                          pack2(__uint_as_float(hb << 16), __uint_as_float(hb & 0xFFFF0000u)));
+        const uint64_t e2 = pack2(__uint_as_float(hb << 16), __uint_as_float(hb & 0xFFFF0000u));
+        ls2[j & 3] = add2(ls2[j & 3], e2);
+        qs2[j & 1] = fma2(e2, e2, qs2[j & 1]);
     }
     const uint64_t s01 = add2(add2(ls2[0], ls2[1]), add2(ls2[2], ls2[3]));
+    const uint64_t q01 = add2(qs2[0], qs2[1]);
     float a0, a1;
+    unpack2(q01, a0, a1);
+    sq = a0 + a1;
     unpack2(s01, a0, a1);
     return a0 + a1;
 }
@@ -385,7 +389,9 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_constant
             const int node = rr / G;
             const unsigned long long anc = masks.anc[node];
             const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
-            float m_ref = -INFINITY, l = 0.f;
+            // q: the sum of the squared rounded weights, rescaled with l
+            // (each weight is at most 2^8, so it cannot overflow)
+            float m_ref = -INFINITY, l = 0.f, q = 0.f;
             bool ok = true;
             for (int t = 0; t < n_tiles; ++t) {
                 const int buf = t & 1;
@@ -436,13 +442,16 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_constant
                     f = (m_ref == -INFINITY) ? 0.f : ex2(m_ref - mx);
                     m_ref = mx;
                     l *= f;
+                    q *= f * f;
                 }
                 aux->factor[buf][r] = f;
                 if (__any_sync(0xffffffffu, need) && lane == 0)
                     bar->rescale_tile[buf] = t + 1;
                 const float neg_m = m_ref == -INFINITY ? 0.f : -m_ref;
                 uint32_t pk[32];
-                l += exp_pack_tile(x, a.scale_log2, neg_m, pk);
+                float dq;
+                l += exp_pack_tile(x, a.scale_log2, neg_m, pk, dq);
+                q += dq;
                 // P^T(t) reuses the buffer of P^T(t-2): PV(t-2) must be done.
                 // PV(t-4), the buffer's previous user, finished before this
                 // warp wrote P^T(t-2), so pv_done[buf] has exactly one phase
@@ -473,13 +482,9 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_constant
                                                          kHeaderBytes) +
                                (size_t)n_split * rows_all * kD;
                 if (r < R) {
-                    aux->l[r] = l;
-                    if (n_split > 1) {
-                        const int orow = node * a.n_heads_q + g * G + r % G;
-                        *reinterpret_cast<float2 *>(ws_ml +
-                                                    ((size_t)split * rows_all + orow) * 2) =
-                            make_float2(m_ref, l);
-                    }
+                    const int orow = node * a.n_heads_q + g * G + r % G;
+                    *reinterpret_cast<float4 *>(ws_ml + ((size_t)split * rows_all + orow) * 4) =
+                        make_float4(m_ref, l, q, 0.f);
                 }
                 __syncwarp();
                 if (lane == 0)
@@ -540,11 +545,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_constant
                     const int rw = c + j;
                     if (rw < R) {
                         const int orow = (rw / G) * a.n_heads_q + g * G + rw % G;
-                        const float v = __uint_as_float(o[j]);
-                        if (n_split == 1)
-                            a.out[(size_t)orow * kD + d] = v / aux->l[rw];
-                        else
-                            ws_o[((size_t)split * rows_all + orow) * kD + d] = v;
+                        ws_o[((size_t)split * rows_all + orow) * kD + d] = __uint_as_float(o[j]);
                     }
                 }
             }
@@ -581,9 +582,9 @@ cudaError_t launch_nb(const AttnArgs &a, const TreeMasks &masks, const AttnPlan 
     if (e != cudaSuccess)
         return e;
     count_launches(1);
-    if (p.n_split == 1)
-        return cudaSuccess;
-    return attn_combine_launch(a, p.n_split, stream);
+    // no overflow flags: the reference max moves with the scores
+    return attn_exact_combine_launch(a, masks, p.n_split, p.tiles_per_split * kTileN, nullptr,
+                                     stream);
 }
 
 }  // namespace

@@ -180,6 +180,35 @@ def test_attn_score_jump_past_headroom(oracle_mod, hq, hkv, t):
     assert np.isfinite(got).all()
 
 
+def _key_ramp(w, lo=0.5, hi=30.0):
+    """K of the context scaled by a ramp from lo at position 0 to hi at the
+    last context position (tail rows unscaled), then rounded to bf16: the
+    scores grow along the context, so most rows put nearly all their weight
+    on a handful of late positions."""
+    q = I.gen_q(w)
+    k, v = I.gen_kv(w)
+    kf = I.bf16_bits_to_f32(k)
+    r = (lo + (hi - lo) * np.arange(w.n_ctx) / max(w.n_ctx - 1, 1)).astype(np.float32)
+    kf[:, : w.n_ctx] *= r[None, :, None]
+    return q, I.f32_to_bf16_bits(kf), v
+
+
+@pytest.mark.parametrize("hq,hkv,t,n_ctx", [(32, 8, 40, 8192), (32, 32, 40, 8192),
+                                            (40, 8, 40, 8192), (32, 8, 4, 20000)])
+def test_attn_peaked_key_ramp(oracle_mod, hq, hkv, t, n_ctx):
+    """Peaked attention (keys ramped 0.5 -> 30 along the context): a row's
+    weight sits on one to a few positions, where one bf16 rounding of P for
+    the PV product costs up to a few 1e-3.  Every row against the oracle,
+    within the same 2e-3."""
+    w = I.Workload("ramp", hq, hkv, 128, n_ctx, t, tree="chain" if t == 4 else "ternary",
+                   seed=11 + hq + t)
+    q, k, v = _key_ramp(w)
+    got = run_attn(q, k, v, w.n_ctx, w.parent())
+    want = oracle_mod.tree_verify_attn(q, k, v, w.n_ctx, w.parent())
+    err = np.abs(got - want).max()
+    assert err <= ATTN_TOL, f"{w.name}: max abs err {err}"
+
+
 def test_attn_draft_pass_over_partial_cache(oracle_mod):
     """Draft pass: a 4-node chain over a 4096-row compact cache (64 sinks + 4032)."""
     w = I.Workload("draft", 32, 8, 128, 4096, 4, tree="chain", seed=12)
