@@ -127,15 +127,20 @@ TS_API int ts_tree_verify_attn(const void *q, const void *k_cache, const void *v
  *    TS_NOALLOC_SCRATCH_BYTES is rejected with TS_ERR_SCRATCH_LIMIT before
  *    anything is launched (16 MiB covers, e.g., 32/8 heads, D 128, a 40-node
  *    tree at any context length).
- *  - Set-up: the first call on a device looks up the array's device address
- *    (cudaGetSymbolAddress) and caches it; make that first call outside any
- *    stream capture.
+ *  - Set-up: the first call on a device (and the first after that device's
+ *    context was reset) looks up the array's device address
+ *    (cudaGetSymbolAddress, with the device current) and keeps it for that
+ *    context; make that first call outside any stream capture.
  *  - Sharing: every call on a device uses the same array and it keeps the
  *    last call's contents; each call clears the part that must start at
  *    zero.  Calls whose work overlaps on the GPU (different streams, no
  *    ordering between them) race on the array and give wrong results:
  *    order them, or use ts_tree_verify_attn with separate workspaces.
- *  - Errors: as ts_tree_verify_attn, plus TS_ERR_SCRATCH_LIMIT.
+ *  - Errors: every argument is checked on the host first, with the same
+ *    results as ts_tree_verify_attn (an invalid call queues nothing);
+ *    TS_ERR_SCRATCH_LIMIT as above.  Conditions only the device can see (an
+ *    expired bounded wait) go to the status word of the array, which no
+ *    call clears: read and clear it with ts_noalloc_status.
  */
 #define TS_NOALLOC_SCRATCH_BYTES (16u << 20)
 TS_API int ts_tree_verify_attn_noalloc(const void *q, const void *k_cache, const void *v_cache,
@@ -143,6 +148,26 @@ TS_API int ts_tree_verify_attn_noalloc(const void *q, const void *k_cache, const
                                        int head_dim, int n_ctx, int n_tree,
                                        const int32_t *parent, float softmax_scale, float *out,
                                        void *stream);
+
+/*
+ * Device-side status of ts_tree_verify_attn_noalloc calls on the current
+ * device (no counterpart on the pages): waits for the work queued on
+ * `stream` (synchronises it), then returns TS_OK or the first device-side
+ * error those calls recorded since the status was last cleared, and clears
+ * it when `clear` is non-zero.  TS_ERR_CUDA if the read fails.
+ */
+TS_API int ts_noalloc_status(void *stream, int clear);
+
+/*
+ * Failure-detection self-test of the no-alloc scratch (no counterpart on the
+ * pages; diagnostic only): sets the array's hand-off tickets to non-zero
+ * values, as a call that ended early on the device could leave them, then
+ * launches the bounded-wait self-test of ts_selftest_bounded_wait on the
+ * array's header, so that about one second later TS_ERR_TIMEOUT is in the
+ * status word ts_noalloc_status reads.  The next ts_tree_verify_attn_noalloc
+ * call still computes correctly and leaves that status in place.
+ */
+TS_API int ts_noalloc_selftest(void *stream);
 
 /*
  * Dynamic partial-KV update: importance scores, sink + top-budget selection
@@ -253,6 +278,60 @@ TS_API int ts_penalize_accept(const float *logits, int n_tree, int vocab, const 
                        int window_len, float penalty, const int32_t *parent,
                        const int32_t *tree_tokens, int32_t *argmax_out, int32_t *accept_out,
                        void *workspace, size_t workspace_bytes, void *stream);
+
+/*
+ * ts_penalize_accept with the method's two randomised / contextual options
+ * ("TokenSwift's technical principles", aiboss88.com: "Contextual penalty
+ * strategy" -- the penalty falls on recently generated tokens -- and
+ * tree-based verification -- the longest valid candidate is selected at
+ * random).  flags = 0 gives exactly ts_penalize_accept.
+ *
+ *  TS_PENALIZE_PATH_TOKENS  node i's window is `window` together with the
+ *               tokens of the draft nodes on i's root path (i included; the
+ *               root's entry of tree_tokens is not read): the tokens that
+ *               precede the one node i's logits predict.  A draft token
+ *               outside [0, vocab) is ignored and flagged TS_ERR_DEVICE_ARG.
+ *  TS_ACCEPT_RANDOM_TIE     of the c deepest valid nodes, in ascending
+ *               index order, the one at position (random mod c) is kept
+ *               (instead of the first).  `random` is a random 64-bit
+ *               integer drawn by the caller; it is read only with this flag.
+ * Every other argument, the workspace and the outputs are as for
+ * ts_penalize_accept.  Unknown flag bits: TS_ERR_INVALID_ARG.
+ */
+#define TS_PENALIZE_PATH_TOKENS 1u
+#define TS_ACCEPT_RANDOM_TIE 2u
+TS_API int ts_penalize_accept_ex(const float *logits, int n_tree, int vocab,
+                                 const int32_t *window, int window_len, float penalty,
+                                 const int32_t *parent, const int32_t *tree_tokens,
+                                 unsigned flags, uint64_t random, int32_t *argmax_out,
+                                 int32_t *accept_out, void *workspace, size_t workspace_bytes,
+                                 void *stream);
+
+/*
+ * Commit of the accepted path: the tree rows of the nodes on the accepted
+ * path move to the context end, in path order, in both caches, so that the
+ * next step's context is n_ctx + L + 1 contiguous rows (tencent article,
+ * parallel-verification figure: the longest valid candidate is kept and
+ * updates the state for the next step).  For j = 1 .. L, row n_ctx + j of
+ * every KV head takes row n_ctx + path[j] (row n_ctx is the root already);
+ * other rows are not touched.  The path is read on the device, so the call
+ * can follow ts_penalize_accept on the same stream with no host round trip.
+ *
+ *  k_cache, v_cache  device bf16 [Hkv, kv_cap, D], modified in place.
+ *  kv_cap, n_heads_kv, head_dim  as for ts_tree_verify_attn (D 64 or 128).
+ *  n_ctx, n_tree     the verified step's context length and tree size;
+ *                    n_ctx + n_tree <= kv_cap.
+ *  accept            device int32 [2 + n_tree] as written by
+ *                    ts_penalize_accept: {L, bonus, path[0..L]}.  A result
+ *                    that is not a root path (L outside [0, n_tree), path[0]
+ *                    not 0, nodes not increasing or out of range) moves
+ *                    nothing and is flagged TS_ERR_DEVICE_ARG.
+ *  workspace         device, >= 256 bytes (the status header), 256-byte
+ *                    aligned, zero-filled.
+ */
+TS_API int ts_kv_commit_path(void *k_cache, void *v_cache, int64_t kv_cap, int n_heads_kv,
+                             int head_dim, int n_ctx, int n_tree, const int32_t *accept,
+                             void *workspace, size_t workspace_bytes, void *stream);
 
 /*
  * n-gram reuse table.  TokenSwift drafts with the frequencies of the

@@ -28,7 +28,11 @@ EXPORTS = ("ts_status_string", "ts_version", "ts_tree_verify_attn_workspace_size
            "ts_kv_select_from_scores_workspace_size", "ts_kv_select_from_scores",
            "ts_ngram_table_bytes", "ts_ngram_init", "ts_ngram_update", "ts_ngram_topk",
            "ts_ngram_topk_prefix",
-           "ts_ngram_count", "ts_ngram_size", "ts_selftest_bounded_wait")
+           "ts_ngram_count", "ts_ngram_size", "ts_selftest_bounded_wait",
+           "ts_penalize_accept_ex", "ts_kv_commit_path")
+
+TS_PENALIZE_PATH_TOKENS = 1
+TS_ACCEPT_RANDOM_TIE = 2
 
 
 class TsError(RuntimeError):
@@ -75,6 +79,11 @@ def _lib():
         lib.ts_penalize_accept_workspace_size.argtypes = [i32, i32]
         lib.ts_penalize_accept.restype = i32
         lib.ts_penalize_accept.argtypes = [P, i32, i32, P, i32, f32, P, P, P, P, P, sz, P]
+        lib.ts_penalize_accept_ex.restype = i32
+        lib.ts_penalize_accept_ex.argtypes = [P, i32, i32, P, i32, f32, P, P, ctypes.c_uint,
+                                              ctypes.c_uint64, P, P, P, sz, P]
+        lib.ts_kv_commit_path.restype = i32
+        lib.ts_kv_commit_path.argtypes = [P, P, i64, i32, i32, i32, i32, P, P, sz, P]
         lib.ts_kernel_launch_count.restype = ctypes.c_ulonglong
         lib.ts_kernel_launch_count.argtypes = []
         lib.ts_workspace_status.restype = i32
@@ -286,8 +295,13 @@ def penalize_accept_workspace_size(n_tree, vocab) -> int:
 
 
 def penalize_accept(logits, window, penalty: float, parent, tree_tokens, argmax_out=None,
-                    accept_out=None, workspace=None, stream=None, want_argmax: bool = True):
-    """Contextual penalty + per-node argmax + longest accepted path (``ts_penalize_accept``).
+                    accept_out=None, workspace=None, stream=None, want_argmax: bool = True,
+                    flags: int = 0, random: int = 0):
+    """Contextual penalty + per-node argmax + longest accepted path
+    (``ts_penalize_accept``; with ``flags`` -- TS_PENALIZE_PATH_TOKENS,
+    TS_ACCEPT_RANDOM_TIE -- ``ts_penalize_accept_ex``, ``random`` the
+    caller's random 64-bit integer for the choice among the deepest valid
+    nodes).
 
     Returns ``(accept [2 + T] int32, argmax [T] int32 or None)``.
     """
@@ -312,11 +326,38 @@ def penalize_accept(logits, window, penalty: float, parent, tree_tokens, argmax_
     par, par_p = _host_i32(parent)
     if len(par) != t:
         raise ValueError("parent must have one entry per tree node")
-    rc = _lib().ts_penalize_accept(_ptr(logits), t, vocab, wptr, wlen, float(penalty), par_p,
-                                   _ptr(tree_tokens), _ptr(argmax_out), _ptr(accept_out),
-                                   _ptr(workspace), workspace.numel(), _stream(stream))
-    _raise(rc, "ts_penalize_accept")
+    if flags == 0:
+        rc = _lib().ts_penalize_accept(_ptr(logits), t, vocab, wptr, wlen, float(penalty), par_p,
+                                       _ptr(tree_tokens), _ptr(argmax_out), _ptr(accept_out),
+                                       _ptr(workspace), workspace.numel(), _stream(stream))
+        _raise(rc, "ts_penalize_accept")
+    else:
+        rc = _lib().ts_penalize_accept_ex(
+            _ptr(logits), t, vocab, wptr, wlen, float(penalty), par_p, _ptr(tree_tokens),
+            int(flags), int(random) & (2 ** 64 - 1), _ptr(argmax_out), _ptr(accept_out),
+            _ptr(workspace), workspace.numel(), _stream(stream))
+        _raise(rc, "ts_penalize_accept_ex")
     return accept_out, argmax_out
+
+
+def kv_commit_path(k_cache, v_cache, n_ctx: int, n_tree: int, accept, workspace=None,
+                   stream=None):
+    """Moves the accepted path's tree rows to n_ctx + 0 .. n_ctx + L in both
+    caches, in place (``ts_kv_commit_path``); ``accept`` is the device
+    result of :func:`penalize_accept`."""
+    _check_dev("k_cache", k_cache, torch.bfloat16)
+    _check_dev("v_cache", v_cache, torch.bfloat16)
+    _check_dev("accept", accept, torch.int32)
+    hkv, cap, d = k_cache.shape
+    if v_cache.shape != k_cache.shape:
+        raise ValueError("k_cache / v_cache shapes disagree")
+    if workspace is None:
+        workspace = new_workspace(256, k_cache.device)
+    rc = _lib().ts_kv_commit_path(_ptr(k_cache), _ptr(v_cache), cap, hkv, d, int(n_ctx),
+                                  int(n_tree), _ptr(accept), _ptr(workspace), workspace.numel(),
+                                  _stream(stream))
+    _raise(rc, "ts_kv_commit_path")
+    return k_cache, v_cache
 
 
 def kernel_launch_count() -> int:

@@ -86,12 +86,12 @@ size_t ts_tree_verify_attn_workspace_size(int n_heads_q, int n_heads_kv, int hea
                                     current_num_sms());
 }
 
-namespace {
+extern "C++" {
+namespace ts {
 
-int attn_call(const void *q, const void *k_cache, const void *v_cache, int64_t kv_cap,
-              int n_heads_q, int n_heads_kv, int head_dim, int n_ctx, int n_tree,
-              const int32_t *parent, float softmax_scale, float *out, float *root_scores,
-              void *workspace, size_t workspace_bytes, void *stream)
+int attn_validate(const void *q, const void *k_cache, const void *v_cache, int64_t kv_cap,
+                  int n_heads_q, int n_heads_kv, int head_dim, int n_ctx, int n_tree,
+                  const int32_t *parent, float softmax_scale, const float *out)
 {
     if (!q || !k_cache || !v_cache || !out || !shape_ok(n_heads_q, n_heads_kv, head_dim))
         return TS_ERR_INVALID_ARG;
@@ -105,6 +105,23 @@ int attn_call(const void *q, const void *k_cache, const void *v_cache, int64_t k
         return TS_ERR_INVALID_ARG;
     if (!head_dim_supported(head_dim))
         return TS_ERR_UNSUPPORTED;
+    return TS_OK;
+}
+
+}  // namespace ts
+}  // extern "C++"
+
+namespace {
+
+int attn_call(const void *q, const void *k_cache, const void *v_cache, int64_t kv_cap,
+              int n_heads_q, int n_heads_kv, int head_dim, int n_ctx, int n_tree,
+              const int32_t *parent, float softmax_scale, float *out, float *root_scores,
+              void *workspace, size_t workspace_bytes, void *stream)
+{
+    const int st = ts::attn_validate(q, k_cache, v_cache, kv_cap, n_heads_q, n_heads_kv,
+                                     head_dim, n_ctx, n_tree, parent, softmax_scale, out);
+    if (st != TS_OK)
+        return st;
     const int sms = current_num_sms();
     const size_t need = ts::attn_workspace_bytes(n_heads_q, n_heads_kv, head_dim, n_ctx, n_tree, sms);
     if (!workspace_ok(workspace, workspace_bytes, need))
@@ -286,6 +303,19 @@ int ts_penalize_accept(const float *logits, int n_tree, int vocab, const int32_t
                        const int32_t *tree_tokens, int32_t *argmax_out, int32_t *accept_out,
                        void *workspace, size_t workspace_bytes, void *stream)
 {
+    return ts_penalize_accept_ex(logits, n_tree, vocab, window, window_len, penalty, parent,
+                                 tree_tokens, 0u, 0ull, argmax_out, accept_out, workspace,
+                                 workspace_bytes, stream);
+}
+
+int ts_penalize_accept_ex(const float *logits, int n_tree, int vocab, const int32_t *window,
+                          int window_len, float penalty, const int32_t *parent,
+                          const int32_t *tree_tokens, unsigned flags, uint64_t random,
+                          int32_t *argmax_out, int32_t *accept_out, void *workspace,
+                          size_t workspace_bytes, void *stream)
+{
+    if ((flags & ~(unsigned)(TS_PENALIZE_PATH_TOKENS | TS_ACCEPT_RANDOM_TIE)) != 0)
+        return TS_ERR_INVALID_ARG;
     if (!logits || !tree_tokens || !accept_out || n_tree < 1 || n_tree > TS_MAX_TREE || vocab < 1)
         return TS_ERR_INVALID_ARG;
     if (window_len < 0 || (window_len > 0 && !window) || !(penalty > 0.0f) || !isfinite(penalty))
@@ -316,8 +346,39 @@ int ts_penalize_accept(const float *logits, int n_tree, int vocab, const int32_t
     a.accept_out = accept_out;
     a.workspace = workspace;
     a.workspace_bytes = workspace_bytes;
+    a.flags = flags;
+    a.random = random;
     const cudaError_t e =
         ts::penalize_launch(a, tp, current_num_sms(), static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? TS_OK : TS_ERR_CUDA;
+}
+
+int ts_kv_commit_path(void *k_cache, void *v_cache, int64_t kv_cap, int n_heads_kv,
+                      int head_dim, int n_ctx, int n_tree, const int32_t *accept,
+                      void *workspace, size_t workspace_bytes, void *stream)
+{
+    if (!k_cache || !v_cache || !accept || n_heads_kv < 1 || n_ctx < 0 || n_tree < 1 ||
+        n_tree > TS_MAX_TREE)
+        return TS_ERR_INVALID_ARG;
+    if ((int64_t)n_ctx + n_tree > kv_cap)
+        return TS_ERR_INVALID_ARG;
+    if (!aligned(k_cache, 16) || !aligned(v_cache, 16) || !aligned(accept, 4))
+        return TS_ERR_INVALID_ARG;
+    if (!head_dim_supported(head_dim))
+        return TS_ERR_UNSUPPORTED;
+    if (!workspace_ok(workspace, workspace_bytes, ts::kHeaderBytes))
+        return TS_ERR_WORKSPACE;
+    ts::CommitArgs a;
+    a.k = static_cast<__nv_bfloat16 *>(k_cache);
+    a.v = static_cast<__nv_bfloat16 *>(v_cache);
+    a.kv_cap = kv_cap;
+    a.n_heads_kv = n_heads_kv;
+    a.head_dim = head_dim;
+    a.n_ctx = n_ctx;
+    a.n_tree = n_tree;
+    a.accept = accept;
+    a.workspace = workspace;
+    const cudaError_t e = ts::commit_launch(a, static_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? TS_OK : TS_ERR_CUDA;
 }
 

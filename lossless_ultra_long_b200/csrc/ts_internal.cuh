@@ -61,6 +61,11 @@ struct AttnArgs {
 
 size_t attn_workspace_bytes(int n_heads_q, int n_heads_kv, int head_dim, int n_ctx, int n_tree,
                             int num_sms);
+// Host-side checks of a verify-attention call's arguments (everything but
+// the workspace): TS_OK or the status the call returns.
+int attn_validate(const void *q, const void *k_cache, const void *v_cache, int64_t kv_cap,
+                  int n_heads_q, int n_heads_kv, int head_dim, int n_ctx, int n_tree,
+                  const int32_t *parent, float softmax_scale, const float *out);
 cudaError_t attn_launch(const AttnArgs &a, const TreeMasks &masks, int num_sms,
                         cudaStream_t stream);
 
@@ -108,7 +113,20 @@ struct PenalizeArgs {
     int32_t *accept_out;
     void *workspace;
     size_t workspace_bytes;
+    unsigned flags;              // TS_PENALIZE_PATH_TOKENS | TS_ACCEPT_RANDOM_TIE
+    unsigned long long random;   // r of the random choice among the deepest valid nodes
 };
+
+// Commit of the accepted path's tree rows into the context (one cache pair).
+struct CommitArgs {
+    __nv_bfloat16 *k;
+    __nv_bfloat16 *v;
+    int64_t kv_cap;
+    int n_heads_kv, head_dim, n_ctx, n_tree;
+    const int32_t *accept;   // device {L, bonus, path[0..L]}
+    void *workspace;
+};
+cudaError_t commit_launch(const CommitArgs &a, cudaStream_t stream);
 
 size_t penalize_workspace_bytes(int n_tree, int vocab);
 cudaError_t penalize_launch(const PenalizeArgs &a, const TreeParents &parents, int num_sms,
