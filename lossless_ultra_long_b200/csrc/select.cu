@@ -238,12 +238,20 @@ __device__ int block_exclusive_scan(int x, int *scratch, int &excl)
     return total;
 }
 
+// Radix select of the budget-th largest key in three passes over the
+// key bits: 11, 11 and 10 bits from the top.
+constexpr int kRadixBins = 2048;
+constexpr int kRadixPasses = 3;
+__host__ __device__ constexpr int radix_shift(int pass) { return pass == 0 ? 21 : pass == 1 ? 10 : 0; }
+__host__ __device__ constexpr uint32_t radix_mask(int pass) { return pass == 2 ? 1023u : 2047u; }
+
 struct alignas(16) P2Shared {
-    int hist[2][256];          // pass p uses hist[p & 1]
+    int hist[2][kRadixBins];   // pass p uses hist[p & 1]
     int scan[72];
     float head_w[kMaxGroup];   // 1 / (G * Z_h)
     float head_m[kMaxGroup];
     float2 slice_ml[kMaxGroup];  // this CTA's (max, sum) per head over its slice
+    float2 warp_ml[kP2Threads / 32][kMaxGroup];  // each warp's (max, sum) per head
     int counts[4];             // [0] equal-to-threshold, [1] kept
     int bcast[4];
 };
@@ -276,18 +284,80 @@ select_gather_kernel(SelectArgs a, int n_chunks, int slice, const float *__restr
     // per-chunk partials, or, for scores given by the caller, from this
     // cluster's own pass over them (each CTA its slice, summed across ranks)
     if (a.root_scores != nullptr) {
+        // every thread folds its positions of the slice into a running
+        // (max, sum of 2^(s - max)) per head in one pass; then the warp, the
+        // CTA and the cluster combine the pairs
+        float rm[kMaxGroup], rl[kMaxGroup];
+#pragma unroll
+        for (int h = 0; h < kMaxGroup; ++h) {
+            rm[h] = -INFINITY;
+            rl[h] = 0.f;
+        }
+        auto fold = [](float &m, float &l, float x) {
+            if (x > m) {
+                l = (m == -INFINITY ? 0.f : l * exp2f(m - x)) + 1.f;
+                m = x;
+            } else if (x != -INFINITY) {
+                l += exp2f(x - m);
+            }
+        };
+        if ((N & 3) == 0) {
+            for (int nb = p0 + 4 * tid; nb < p1; nb += 4 * kP2Threads) {
+                float4 sv[kMaxGroup];
+#pragma unroll
+                for (int h = 0; h < kMaxGroup; ++h)
+                    if (h < G)
+                        sv[h] = __ldcg(reinterpret_cast<const float4 *>(
+                            s_all + (size_t)(g * G + h) * N + nb));
+#pragma unroll
+                for (int h = 0; h < kMaxGroup; ++h)
+                    if (h < G) {
+                        const float mx = fmaxf(fmaxf(sv[h].x, sv[h].y), fmaxf(sv[h].z, sv[h].w));
+                        if (mx > rm[h]) {
+                            rl[h] = rm[h] == -INFINITY ? 0.f : rl[h] * exp2f(rm[h] - mx);
+                            rm[h] = mx;
+                        }
+                        if (mx != -INFINITY)
+                            rl[h] += exp2f(sv[h].x - rm[h]) + exp2f(sv[h].y - rm[h]) +
+                                     exp2f(sv[h].z - rm[h]) + exp2f(sv[h].w - rm[h]);
+                    }
+            }
+        } else {
+            for (int n = p0 + tid; n < p1; n += kP2Threads)
+#pragma unroll
+                for (int h = 0; h < kMaxGroup; ++h)
+                    if (h < G)
+                        fold(rm[h], rl[h], __ldcg(s_all + (size_t)(g * G + h) * N + n));
+        }
+        // warp: pairwise merge of (m, l)
+#pragma unroll
+        for (int h = 0; h < kMaxGroup; ++h) {
+            if (h >= G)
+                continue;
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) {
+                const float om = __shfl_xor_sync(0xffffffffu, rm[h], o);
+                const float ol = __shfl_xor_sync(0xffffffffu, rl[h], o);
+                const float mm = fmaxf(rm[h], om);
+                if (mm != -INFINITY) {
+                    rl[h] = (rm[h] == -INFINITY ? 0.f : rl[h] * exp2f(rm[h] - mm)) +
+                            (om == -INFINITY ? 0.f : ol * exp2f(om - mm));
+                    rm[h] = mm;
+                }
+            }
+            if (lane == 0)
+                sh.warp_ml[warp][h] = make_float2(rm[h], rl[h]);
+        }
+        __syncthreads();
+        // CTA: one warp per head over the 16 warps' pairs
         if (warp < G) {
-            const float *row = s_all + (size_t)(g * G + warp) * N;
-            float m = -INFINITY;
-            for (int n = p0 + lane; n < p1; n += 32)
-                m = fmaxf(m, __ldcg(row + n));
+            const float2 x = lane < kP2Threads / 32 ? sh.warp_ml[lane][warp]
+                                                    : make_float2(-INFINITY, 0.f);
+            float m = x.x;
 #pragma unroll
             for (int o = 16; o > 0; o >>= 1)
                 m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-            float l = 0.f;
-            if (m != -INFINITY)
-                for (int n = p0 + lane; n < p1; n += 32)
-                    l += exp2f(__ldcg(row + n) - m);
+            float l = (m == -INFINITY || x.x == -INFINITY) ? 0.f : x.y * exp2f(x.x - m);
 #pragma unroll
             for (int o = 16; o > 0; o >>= 1)
                 l += __shfl_xor_sync(0xffffffffu, l, o);
@@ -336,37 +406,75 @@ select_gather_kernel(SelectArgs a, int n_chunks, int slice, const float *__restr
     }
     __syncthreads();
 
+    const bool do_select = !keep_all && a.budget > 0;
+    // the first radix pass's histogram is built while the keys are formed
+    for (int b = tid; b < kRadixBins; b += kP2Threads)
+        sh.hist[0][b] = 0;
+    __syncthreads();
+    // adds one to the pass's bin of each candidate key (positions >= n_sink)
+    // whose higher digits match `prefix`; lanes with equal bins add once, by
+    // their leader (positive scores share their leading bits, so most lanes
+    // of a warp hit the same bin)
+    auto hist_add = [&](int *hist, bool in, uint32_t key, uint32_t prefix, uint32_t pmask,
+                        int pass) {
+        const bool hit = in && (key & pmask) == prefix;
+        const unsigned act = __ballot_sync(0xffffffffu, hit);
+        if (hit) {
+            const uint32_t bin = (key >> radix_shift(pass)) & radix_mask(pass);
+            const unsigned same = __match_any_sync(act, bin);
+            if (lane == __ffs(same) - 1)
+                atomicAdd(&hist[bin], __popc(same));
+        }
+    };
+
     // scores of this slice -> order-preserving keys in shared memory
     if ((N & 3) == 0) {
         // four consecutive positions per thread, one 16-byte load per head
-        // (the slice is a multiple of 4, so p0 and p1 are too)
-        for (int nb = p0 + 4 * tid; nb < p1; nb += 4 * kP2Threads) {
-            float4 sv[kMaxGroup];
-#pragma unroll
-            for (int h = 0; h < kMaxGroup; ++h)
-                if (h < G)
-                    sv[h] = __ldcg(reinterpret_cast<const float4 *>(
-                        s_all + (size_t)(g * G + h) * N + nb));
+        // (the slice is a multiple of 4, so p0 and p1 are too); every lane
+        // of a warp runs the same number of rounds
+        const int rounds = (p1 - p0 + 4 * kP2Threads - 1) / (4 * kP2Threads);
+        for (int it = 0; it < rounds; ++it) {
+            const int nb = p0 + 4 * (tid + it * kP2Threads);
+            const bool live = nb < p1;
             float sc[4] = {0.f, 0.f, 0.f, 0.f};
+            if (live) {
+                float4 sv[kMaxGroup];
 #pragma unroll
-            for (int h = 0; h < kMaxGroup; ++h)
-                if (h < G) {
-                    const float m = sh.head_m[h], wgt = sh.head_w[h];
-                    sc[0] += exp2f(sv[h].x - m) * wgt;
-                    sc[1] += exp2f(sv[h].y - m) * wgt;
-                    sc[2] += exp2f(sv[h].z - m) * wgt;
-                    sc[3] += exp2f(sv[h].w - m) * wgt;
-                }
-            *reinterpret_cast<uint4 *>(&keys[nb - p0]) =
-                make_uint4(order_key(sc[0]), order_key(sc[1]), order_key(sc[2]), order_key(sc[3]));
-            if (a.scores_out)
-                *reinterpret_cast<float4 *>(a.scores_out + (size_t)g * N + nb) =
-                    make_float4(sc[0], sc[1], sc[2], sc[3]);
+                for (int h = 0; h < kMaxGroup; ++h)
+                    if (h < G)
+                        sv[h] = __ldcg(reinterpret_cast<const float4 *>(
+                            s_all + (size_t)(g * G + h) * N + nb));
+#pragma unroll
+                for (int h = 0; h < kMaxGroup; ++h)
+                    if (h < G) {
+                        const float m = sh.head_m[h], wgt = sh.head_w[h];
+                        sc[0] += exp2f(sv[h].x - m) * wgt;
+                        sc[1] += exp2f(sv[h].y - m) * wgt;
+                        sc[2] += exp2f(sv[h].z - m) * wgt;
+                        sc[3] += exp2f(sv[h].w - m) * wgt;
+                    }
+            }
+            uint32_t kk[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e)
+                kk[e] = order_key(sc[e]);
+            if (live) {
+                *reinterpret_cast<uint4 *>(&keys[nb - p0]) = make_uint4(kk[0], kk[1], kk[2], kk[3]);
+                if (a.scores_out)
+                    *reinterpret_cast<float4 *>(a.scores_out + (size_t)g * N + nb) =
+                        make_float4(sc[0], sc[1], sc[2], sc[3]);
+            }
+            if (do_select)
+#pragma unroll
+                for (int e = 0; e < 4; ++e)
+                    hist_add(sh.hist[0], live && nb + e >= a.n_sink, kk[e], 0u, 0u, 0);
         }
     } else {
         // eight positions per thread per step so their loads are in flight together
         constexpr int kU = 8;
-        for (int nb = p0 + tid; nb < p1; nb += kP2Threads * kU) {
+        const int rounds = (p1 - p0 + kP2Threads * kU - 1) / (kP2Threads * kU);
+        for (int it = 0; it < rounds; ++it) {
+            const int nb = p0 + tid + it * kP2Threads * kU;
             float sc[kU];
 #pragma unroll
             for (int u = 0; u < kU; ++u)
@@ -386,65 +494,74 @@ select_gather_kernel(SelectArgs a, int n_chunks, int slice, const float *__restr
 #pragma unroll
             for (int u = 0; u < kU; ++u) {
                 const int n = nb + u * kP2Threads;
+                const uint32_t key = order_key(sc[u]);
                 if (n < p1) {
-                    keys[n - p0] = order_key(sc[u]);
+                    keys[n - p0] = key;
                     if (a.scores_out)
                         a.scores_out[(size_t)g * N + n] = sc[u];
                 }
+                if (do_select)
+                    hist_add(sh.hist[0], n < p1 && n >= a.n_sink, key, 0u, 0u, 0);
             }
         }
     }
     __syncthreads();
 
-    // exact radix select of the budget-th largest key over [n_sink, N)
+    // exact radix select of the budget-th largest key over [n_sink, N):
+    // three passes (11, 11, 10 bits), histograms summed over the cluster
+    // through distributed shared memory
     uint32_t prefix = 0u, pmask = 0u;
     int need = a.budget;
-    const bool do_select = !keep_all && a.budget > 0;
     if (do_select) {
         const int c0 = max(p0, a.n_sink);
-        for (int pass = 0; pass < 4; ++pass) {
-            const int shift = 24 - 8 * pass;
-            // this buffer was last read by other CTAs two passes ago, before
-            // they reached the previous pass's cluster barrier
+        for (int pass = 0; pass < kRadixPasses; ++pass) {
             int *hist = sh.hist[pass & 1];
-            for (int b = tid; b < 256; b += kP2Threads)
-                hist[b] = 0;
-            __syncthreads();
-            // positive scores share their leading bytes, so most lanes hit
-            // the same bin: lanes with equal bins add once, by their leader
-            for (int nb = c0 - (c0 - p0) % 32; nb < p1; nb += kP2Threads) {
-                const int n = nb + tid;
-                const bool in = n >= c0 && n < p1;
-                const uint32_t key = in ? keys[n - p0] : 0u;
-                const bool hit = in && (key & pmask) == prefix;
-                const unsigned act = __ballot_sync(0xffffffffu, hit);
-                if (hit) {
-                    const uint32_t bin = (key >> shift) & 255u;
-                    const unsigned same = __match_any_sync(act, bin);
-                    if ((lane) == __ffs(same) - 1)
-                        atomicAdd(&hist[bin], __popc(same));
+            if (pass > 0) {
+                // this buffer was last read by other CTAs two passes ago,
+                // before they reached the previous pass's cluster barrier
+                for (int b = tid; b < kRadixBins; b += kP2Threads)
+                    hist[b] = 0;
+                __syncthreads();
+                for (int nb = c0 - (c0 - p0) % 32; nb < p1; nb += kP2Threads) {
+                    const int n = nb + tid;
+                    const bool in = n >= c0 && n < p1;
+                    hist_add(hist, in, in ? keys[n - p0] : 0u, prefix, pmask, pass);
                 }
             }
             cluster.sync();
-            // Thread t looks at bin b = 255 - t; an inclusive scan over t is
-            // then a suffix sum over bins.  The digit is the bin with
-            // (keys in higher bins) < need <= (that count + its own keys).
-            const int b = 255 - tid;
-            int x = 0;
-            if (tid < 256)
-                for (int r = 0; r < n_ranks; ++r)
-                    x += cluster.map_shared_rank(hist, r)[b];
+            // thread t looks at bins 4t .. 4t + 3 from the top (bin
+            // 2047 - 4t - k): an exclusive scan over t counts the keys in
+            // higher bins; the digit is the bin with (keys above it) < need
+            // <= (that count + its own keys)
+            const int nbins = (int)radix_mask(pass) + 1;
+            int x[4] = {0, 0, 0, 0};
+            if (4 * tid < nbins) {
+                // bins nbins-4-4t .. nbins-1-4t: one 16-byte read per rank
+                const int q = (nbins - 4 - 4 * tid) / 4;
+                for (int r = 0; r < n_ranks; ++r) {
+                    const int4 v = reinterpret_cast<const int4 *>(cluster.map_shared_rank(hist, r))[q];
+                    x[0] += v.w;
+                    x[1] += v.z;
+                    x[2] += v.y;
+                    x[3] += v.x;
+                }
+            }
             int above;
-            block_exclusive_scan(x, sh.scan, above);
-            if (tid < 256 && above < need && need <= above + x) {
-                sh.bcast[0] = b;
-                sh.bcast[1] = above;
+            block_exclusive_scan(x[0] + x[1] + x[2] + x[3], sh.scan, above);
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                const int b = nbins - 1 - (4 * tid + k);
+                if (b >= 0 && above < need && need <= above + x[k]) {
+                    sh.bcast[0] = b;
+                    sh.bcast[1] = above;
+                }
+                above += x[k];
             }
             __syncthreads();   // the digit is in bcast
             const int d = sh.bcast[0];
             need -= sh.bcast[1];
-            prefix |= (uint32_t)d << shift;
-            pmask |= 255u << shift;
+            prefix |= (uint32_t)d << radix_shift(pass);
+            pmask |= radix_mask(pass) << radix_shift(pass);
             __syncthreads();
         }
     }
