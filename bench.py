@@ -10,7 +10,9 @@ tree):
   3. the draft pass: ts_tree_verify_attn of a 4-node chain over that
      4096-row partial cache,
   4. ts_penalize_accept over fp32 logits [40, 128256], window 1024, on a
-     second stream beside 2 and 3.
+     second stream beside 2 and 3,
+  5. ts_kv_commit_path: the accepted path's tree rows move to the end of
+     the context (after 3 and 4).
 With --select-score-pass, 1 and 2 are ts_tree_verify_attn and
 ts_kv_importance_select (the select scores the context itself).
 The metric counts tree-verify calls: each step holds exactly one.
@@ -41,7 +43,9 @@ UNIT = "calls/s"
 def parse():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=1000)
+    ap.add_argument("--steps", type=int, default=None,
+                    help="timed steps (default 1000; 3 for the reference arm, whose "
+                         "steps take seconds each)")
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -49,6 +53,14 @@ def parse():
     ap.add_argument("--select-score-pass", action="store_true",
                     help="the select scores the context with its own pass over K instead "
                          "of taking the root node's scores from the verify attention")
+    ap.add_argument("--no-sweep", action="store_true",
+                    help="skip the 14B-shape roofline sweep (context x tree size)")
+    ap.add_argument("--only", choices=["verify", "verify_plain", "select", "draft", "penalty",
+                                       "commit"],
+                    help="run one call of the step warmup + steps times, eagerly, and print "
+                         "its mean device time (for profiler captures of a single kernel)")
+    ap.add_argument("--breakdown", action="store_true",
+                    help="device time of each call of the step alone (eager, CUDA events)")
     return ap.parse_args()
 
 
@@ -94,13 +106,18 @@ def attn_flops(hq, d, n_ctx, t):
     return 4 * hq * t * d * (n_ctx + t)
 
 
-def measured_peaks():
+def measured_peaks(sustained=False):
+    """(HBM GB/s, dense bf16 TFLOP/s, source): the machine's measured copy
+    bandwidth and cuBLAS bf16 throughput (burst, or the seconds-long
+    sustained figure for a kernel timed inside a long loop), else the
+    fallback figures."""
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
         with open(p) as f:
             j = json.load(f)
-        return float(j["hbm_gbs"]), float(j["bf16_tflops"]), "measured"
-    return 6650.0, 1590.0, "fallback"
+        tf = j.get("bf16_tflops_sustained") if sustained else None
+        return float(j["hbm_gbs"]), float(tf or j["bf16_tflops"]), "measured"
+    return 6650.0, 1400.0 if sustained else 1590.0, "fallback"
 
 
 def attn_traffic_record():
@@ -236,7 +253,7 @@ class ClockSampler:
 class Step:
     """Device-resident buffers and the four ABI calls of one verification step."""
 
-    def __init__(self, torch, L, I, w, dev, fused=True):
+    def __init__(self, torch, L, I, w, dev, fused=True, want_scores=False):
         from_bits = lambda b: torch.from_numpy(np.ascontiguousarray(b).view(np.int16)).view(
             torch.bfloat16).to(dev)
         self.torch, self.L, self.w = torch, L, w
@@ -282,36 +299,59 @@ class Step:
             self.ws_sel = L.new_workspace(
                 L.kv_importance_select_workspace_size(hq, hkv, d, w.n_ctx), dev)
         self.ws_pen = L.new_workspace(L.penalize_accept_workspace_size(w.n_tree, w.vocab), dev)
+        self.ws_commit = L.new_workspace(256, dev)
+        # the importance scores the select ranks by, when a caller wants to see them
+        self.scores = (torch.empty((hkv, w.n_ctx), dtype=torch.float32, device=dev)
+                       if want_scores else None)
         self.side = torch.cuda.Stream(device=dev)
 
-    def attn(self):
+    def attn(self, root_scores=True):
         self.L.tree_verify_attn(self.q, self.k, self.v, self.w.n_ctx, self.parent, out=self.out,
-                                workspace=self.ws_attn, root_scores_out=self.rs)
+                                workspace=self.ws_attn,
+                                root_scores_out=self.rs if root_scores else None)
+
+    def select(self):
+        w, L = self.w, self.L
+        if self.fused:
+            L.kv_select_from_scores(self.rs, self.k, self.v, w.n_ctx, w.n_sink, w.budget,
+                                    k_partial=self.kp, v_partial=self.vp, idx_out=self.idx,
+                                    scores_out=self.scores, workspace=self.ws_sel)
+        else:
+            L.kv_importance_select(self.q[0], self.k, self.v, w.n_ctx, w.n_sink, w.budget,
+                                   k_partial=self.kp, v_partial=self.vp, idx_out=self.idx,
+                                   scores_out=self.scores, workspace=self.ws_sel)
+
+    def penalty(self):
+        w = self.w
+        self.L.penalize_accept(self.logits, self.window, w.penalty, self.parent, self.tokens,
+                               argmax_out=self.argmax, accept_out=self.accept,
+                               workspace=self.ws_pen)
+
+    def draft(self):
+        self.L.tree_verify_attn(self.dq, self.kp, self.vp, self.n_keep, self.draft_parent,
+                                out=self.dout, workspace=self.ws_draft)
+
+    def commit(self):
+        """The accepted path's tree rows become the context's next rows."""
+        w = self.w
+        self.L.kv_commit_path(self.k, self.v, w.n_ctx, w.n_tree, self.accept,
+                              workspace=self.ws_commit)
 
     def rest(self):
         """Select, then the draft pass over the partial cache it builds; the
         penalty/accept call depends on neither and runs beside them on a
-        second stream (the select's cluster kernel leaves most SMs idle)."""
-        w, L, torch = self.w, self.L, self.torch
+        second stream; the commit of the accepted path follows both."""
+        torch = self.torch
         main = torch.cuda.current_stream()
         self.side.wait_stream(main)   # fork: the side stream depends on what came before
-        if self.fused:
-            L.kv_select_from_scores(self.rs, self.k, self.v, w.n_ctx, w.n_sink, w.budget,
-                                    k_partial=self.kp, v_partial=self.vp, idx_out=self.idx,
-                                    workspace=self.ws_sel)
-        else:
-            L.kv_importance_select(self.q[0], self.k, self.v, w.n_ctx, w.n_sink, w.budget,
-                                   k_partial=self.kp, v_partial=self.vp, idx_out=self.idx,
-                                   workspace=self.ws_sel)
-        # enqueued after the select so that its cluster kernel starts first
-        # and the penalty CTAs fill the SMs it leaves
+        self.select()
+        # enqueued after the select so that its kernels start first and the
+        # penalty CTAs fill the SMs they leave
         with torch.cuda.stream(self.side):
-            L.penalize_accept(self.logits, self.window, w.penalty, self.parent, self.tokens,
-                              argmax_out=self.argmax, accept_out=self.accept,
-                              workspace=self.ws_pen)
-        L.tree_verify_attn(self.dq, self.kp, self.vp, self.n_keep, self.draft_parent,
-                           out=self.dout, workspace=self.ws_draft)
+            self.penalty()
+        self.draft()
         main.wait_stream(self.side)
+        self.commit()
 
     def step(self):
         self.attn()
@@ -425,10 +465,14 @@ def run_ours(args):
 
     out = None
     if rank == 0:
-        hbm, tflops, src = measured_peaks()
+        hbm, tflops, src = measured_peaks(sustained=True)
         attn_avg_s = statistics.mean(attn_ms) / 1e3
+        # the call's algorithmic bytes (K + V + Q + O); the fused call also
+        # writes the root node's scores, counted separately
         byts = attn_bytes(w.n_heads_q, w.n_heads_kv, w.head_dim, w.n_ctx, w.n_tree,
-                          root_scores=st.fused)
+                          root_scores=False)
+        score_bytes = (attn_bytes(w.n_heads_q, w.n_heads_kv, w.head_dim, w.n_ctx, w.n_tree,
+                                  root_scores=True) - byts) if st.fused else 0
         flops = attn_flops(w.n_heads_q, w.head_dim, w.n_ctx, w.n_tree)
         achieved = byts / attn_avg_s / 1e9
         value = job_throughput(K, world, ms_max)
@@ -443,7 +487,7 @@ def run_ours(args):
                        "tree": "3-ary BFS depth 3", "step": ("verify attn (leaving the root's scores) + importance "
                                 "select from them" if st.fused else "verify attn + importance "
                                 "select with its own score pass") + " (64+4032) + 4-node draft attn over the partial cache + penalty/accept "
-                       "(V=128256, W=1024); penalty/accept on a second stream beside the "
+                       "(V=128256, W=1024) + commit of the accepted path; penalty/accept on a second stream beside the "
                        "select and draft pass", "l2": "inputs larger than L2 (420 MB KV per step)",
                        "parallelism": f"replicas x{world}", "graphs": True,
                        "attn_timing": ("events inside the step graph, last %d steps" % kGraphs
@@ -453,8 +497,11 @@ def run_ours(args):
             "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": hbm,
                          "unit": "GB/s", "frac": round(achieved / hbm, 4),
                          "peak_source": src, "traffic": attn_traffic_record(),
-                         "algorithmic_bytes": byts,
-                         "tensor_frac": round(flops / attn_avg_s / 1e12 / tflops, 4)},
+                         "algorithmic_bytes": byts, "root_score_bytes": score_bytes,
+                         "frac_with_root_scores": round((byts + score_bytes) / attn_avg_s /
+                                                        1e9 / hbm, 4),
+                         "tensor_frac": round(flops / attn_avg_s / 1e12 / tflops, 4),
+                         "tensor_peak_tflops": tflops},
             "e2e": {"value": round(e2e_value, 2), "unit": UNIT,
                     "h2d_bytes_per_step": e2e["h2d"], "d2h_bytes_per_step": e2e["d2h"]},
             "gpu_launches": int(launches_per_step * K),
@@ -465,6 +512,9 @@ def run_ours(args):
         except Exception as e:   # host-side extra: never costs the GPU line
             out["ngram_host_us_per_step"] = None
             out["ngram_host_error"] = str(e)[:200]
+        if not args.no_sweep:
+            hbm_b, tf_b, _ = measured_peaks(sustained=False)
+            out["sweep"] = sweep_14b(torch, L, I, dev, hbm_b, tf_b)
         if not args.no_cpu_baseline:
             out["cpu_baseline"] = cpu_baseline(w)
     if world > 1:
@@ -474,6 +524,126 @@ def run_ours(args):
             del g_attn, g_rest
         dist.destroy_process_group()
     return out
+
+
+def _setup_single(args):
+    """Device, library and the step's buffers for the single-call modes."""
+    import torch
+    import lossless_ultra_long_b200 as L
+    from lossless_ultra_long_b200 import inputs as I
+    _, _, local = dist_env()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    L.library()
+    st = Step(torch, L, I, workload(), dev, fused=not args.select_score_pass)
+    return torch, L, st
+
+
+def _call_of(st, name):
+    return {"verify": lambda: st.attn(True), "verify_plain": lambda: st.attn(False),
+            "select": st.select, "draft": st.draft, "penalty": st.penalty,
+            "commit": st.commit}[name]
+
+
+def _prepare(st, name):
+    """Inputs a call reads that an earlier call of the step produces."""
+    if name in ("select", "draft"):
+        st.attn(True)
+    if name == "draft":
+        st.select()
+    if name == "commit":
+        st.penalty()
+
+
+def _time_call(torch, fn, warmup, steps):
+    """Mean device time (us) of fn over `steps` back-to-back calls after
+    `warmup` calls, CUDA events on the current stream."""
+    for _ in range(warmup):
+        fn()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(steps):
+        fn()
+    e1.record()
+    torch.cuda.synchronize()
+    return e0.elapsed_time(e1) * 1e3 / max(steps, 1)
+
+
+def run_only(args):
+    """One call of the step, run warmup + steps times eagerly (a short,
+    self-contained program for profiler captures of one kernel)."""
+    torch, L, st = _setup_single(args)
+    _prepare(st, args.only)
+    fn = _call_of(st, args.only)
+    us = _time_call(torch, fn, args.warmup, args.steps)
+    return {"mode": "only", "call": args.only, "workload": st.w.name, "steps": args.steps,
+            "warmup": args.warmup, "us_per_call": round(us, 2),
+            "launches": L.kernel_launch_count()}
+
+
+def run_breakdown(args):
+    """Device time of each call of the step alone (eager, back to back;
+    the verify call reads 420 MB per call, so it runs from HBM; the smaller
+    calls re-read inputs that may sit in L2)."""
+    torch, L, st = _setup_single(args)
+    w = st.w
+    st.attn(True)
+    st.select()
+    out = {"mode": "breakdown", "workload": w.name}
+    for name in ("verify", "verify_plain", "select", "draft", "penalty", "commit"):
+        out[name + "_us"] = round(_time_call(torch, _call_of(st, name), max(args.warmup, 3),
+                                             max(args.steps, 10)), 2)
+    return out
+
+
+def sweep_14b(torch, L, I, dev, hbm, tflops, warmup=10, calls=50):
+    """The 14B GQA roofline sweep: Hq 40, Hkv 8, D 128, contexts 4K-131K and
+    trees of 4 (a chain), 13 and 40 nodes.  Per point: the verify call's mean
+    device time over back-to-back calls that rotate over enough copies of the
+    KV cache that each call reads from HBM (3 x L2 at least), its algorithmic
+    bytes and flops, achieved GB/s and TFLOP/s and their fractions of the
+    measured peaks.  Inputs: seeded N(0, 1) bf16 drawn on the device."""
+    l2 = 126 * 2 ** 20
+    points = []
+    gen = torch.Generator(device=dev)
+    for n_ctx in I.SWEEP_CTX:
+        t_max = max(I.SWEEP_TREE)
+        hkv, hq, d = 8, 40, 128
+        kv_bytes = 2 * hkv * (n_ctx + t_max) * d * 2
+        n_sets = max(1, min(24, -(-3 * l2 // kv_bytes)))
+        gen.manual_seed(4000 + n_ctx)
+        sets = []
+        for _ in range(n_sets):
+            k = torch.randn((hkv, n_ctx + t_max, d), generator=gen, device=dev).to(torch.bfloat16)
+            v = torch.randn((hkv, n_ctx + t_max, d), generator=gen, device=dev).to(torch.bfloat16)
+            sets.append((k, v))
+        for t in I.SWEEP_TREE:
+            w = I.sweep14b(n_ctx, t)
+            parent = w.parent()
+            q = torch.randn((t, hq, d), generator=gen, device=dev).to(torch.bfloat16)
+            out = torch.empty((t, hq, d), dtype=torch.float32, device=dev)
+            ws = L.new_workspace(L.tree_verify_attn_workspace_size(hq, hkv, d, n_ctx, t), dev)
+            it = [0]
+
+            def call():
+                k, v = sets[it[0] % n_sets]
+                it[0] += 1
+                L.tree_verify_attn(q, k, v, n_ctx, parent, out=out, workspace=ws)
+
+            us = _time_call(torch, call, warmup, calls)
+            byts = attn_bytes(hq, hkv, d, n_ctx, t, root_scores=False)
+            flops = attn_flops(hq, d, n_ctx, t)
+            gbs = byts / (us * 1e-6) / 1e9
+            tfs = flops / (us * 1e-6) / 1e12
+            points.append({"n_ctx": n_ctx, "n_tree": t, "us": round(us, 2),
+                           "calls_per_s": round(1e6 / us, 1), "bytes": byts, "flops": flops,
+                           "gbs": round(gbs, 1), "hbm_frac": round(gbs / hbm, 4),
+                           "tflops": round(tfs, 1), "tensor_frac": round(tfs / tflops, 4)})
+        del sets
+        torch.cuda.empty_cache()
+    return {"workload": "qwen14b_gqa40x8_d128", "kv_sets_rotated": "ceil(3 x L2 / KV bytes), "
+            "at most 24", "calls_per_point": calls, "points": points}
 
 
 def run_e2e(torch, L, st, w, dev, stream, steps):
@@ -557,7 +727,7 @@ class OracleSample:
                        f"importance select of all {w.n_heads_kv} KV heads over "
                        f"{self.sel_positions} of {w.n_ctx} positions; {draft_rows} of "
                        f"{w.draft_tree * w.n_heads_q} draft-pass rows; penalty/argmax of "
-                       f"{pen_nodes} of {w.n_tree} nodes; acceptance; scaled to one step")
+                       f"{pen_nodes} of {w.n_tree} nodes; acceptance and commit; scaled to one step")
 
     def seconds_per_step(self):
         o, w = self.o, self.w
@@ -587,7 +757,11 @@ class OracleSample:
         t_pen = (time.perf_counter() - t0) * w.n_tree / self.pen_nodes
         am_full = np.resize(am, w.n_tree).astype(np.int32)
         t0 = time.perf_counter()
-        o.accept_longest(self.parent, self.tokens, am_full)
+        acc = o.accept_longest(self.parent, self.tokens, am_full)
+        # the commit touches the tree-tail rows only
+        lo, hi = w.n_ctx, w.n_ctx + w.n_tree
+        o.kv_commit_path(self.k[:, lo:hi], 0, w.n_tree, acc)
+        o.kv_commit_path(self.v[:, lo:hi], 0, w.n_tree, acc)
         t_acc = time.perf_counter() - t0
         return t_attn + t_sel + t_draft + t_pen + t_acc
 
@@ -596,24 +770,50 @@ def oracle_threads():
     return int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
 
 
+def cpu_model():
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return None
+
+
 def cpu_baseline(w):
-    """About 10-30 s of oracle work on the host cores (rank 0, N = 1 leg)."""
+    """About 10-30 s of oracle work on the host cores (rank 0, N = 1 leg):
+    a sampled step on all cores, and a smaller sample on one thread."""
+    import oracle
+    thr = oracle_threads()
     smp = OracleSample(w, attn_rows=160, sel_positions=w.n_ctx, draft_rows=128, pen_nodes=40)
     per_step = smp.seconds_per_step()
-    return {"value": round(1.0 / per_step, 6), "unit": UNIT, "cores": oracle_threads(),
-            "kind": "oracle", "sample": smp.sample, "seconds_per_step": round(per_step, 3)}
+    one = OracleSample(w, attn_rows=16, sel_positions=8192, draft_rows=16, pen_nodes=8)
+    oracle.set_num_threads(1)
+    try:
+        per_step_1 = one.seconds_per_step()
+    finally:
+        oracle.set_num_threads(thr)
+    return {"value": round(1.0 / per_step, 6), "unit": UNIT, "cores": thr,
+            "kind": "oracle", "sample": smp.sample, "seconds_per_step": round(per_step, 3),
+            "cpu_model": cpu_model(),
+            "one_thread": {"value": round(1.0 / per_step_1, 6), "unit": UNIT, "cores": 1,
+                           "sample": one.sample, "seconds_per_step": round(per_step_1, 3)}}
 
 
 def run_reference(args):
+    """The oracle timed on the host cores, whole steps: every verify row,
+    the importance select over the whole context with the gather, every
+    draft-pass row, the penalty/argmax of every node and the acceptance --
+    no sampling and no scaling.  Rank 0 only."""
     rank, world, _ = dist_env()
     if rank != 0:
         return None
     w = workload()
     K = max(1, args.steps)
     thr = oracle_threads()
-    smp = OracleSample(w, attn_rows=max(8, thr), sel_positions=8192,
-                       draft_rows=min(w.draft_tree * w.n_heads_q, max(8, thr)),
-                       pen_nodes=min(w.n_tree, max(8, thr)))
+    smp = OracleSample(w, attn_rows=w.n_tree * w.n_heads_q, sel_positions=w.n_ctx,
+                       draft_rows=w.draft_tree * w.n_heads_q, pen_nodes=w.n_tree)
     for _ in range(min(args.warmup, 1)):
         smp.seconds_per_step()
     secs = [smp.seconds_per_step() for _ in range(K)]
@@ -625,15 +825,26 @@ def run_reference(args):
             "data": "synthetic", "impl": "reference",
             "config": {"workload": w.name, "n_heads_q": w.n_heads_q, "n_heads_kv": w.n_heads_kv,
                        "head_dim": w.head_dim, "n_ctx": w.n_ctx, "n_tree": w.n_tree},
-            "cpu_baseline": {"value": val, "unit": UNIT, "cores": oracle_threads(),
-                             "kind": "oracle", "sample": smp.sample},
+            "cpu_baseline": {"value": val, "unit": UNIT, "cores": thr, "kind": "oracle",
+                             "sample": "whole steps: " + smp.sample.replace(
+                                 "; scaled to one step", ""),
+                             "cpu_model": cpu_model(), "warmup_steps": min(args.warmup, 1)},
             "e2e": {"value": val, "unit": UNIT, "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
 
 
 def main():
     args = parse()
-    out = run_reference(args) if args.impl == "reference" else run_ours(args)
+    if args.steps is None:
+        args.steps = 3 if args.impl == "reference" else 1000
+    if args.impl == "reference":
+        out = run_reference(args)
+    elif args.only:
+        out = run_only(args)
+    elif args.breakdown:
+        out = run_breakdown(args)
+    else:
+        out = run_ours(args)
     if out is not None:
         print(json.dumps(out), flush=True)
 
