@@ -133,24 +133,55 @@ constexpr size_t kAuxBytes = (sizeof(Aux) + 1023) / 1024 * 1024;
 struct Layout {
     int r_pad;  // rows rounded up to 16: N of the PV product
     int stages_k, stages_v;
-    size_t q1_off, p_off, k_off, v_off, aux_off, smem_bytes;
+    size_t q1_off, p_off, k_off, v_off, aux_off, rs_off, smem_bytes;
 };
 
 // Rows per TMEM lane quarter in block 0 (rows 0..min(R, 128) - 1 cut into
 // four equal runs).
 __host__ __device__ inline int t128_rq0(int rows) { return ((rows < kBlockM ? rows : kBlockM) + 3) / 4; }
 
-// Whether warp 0 reads the root node's scores out of TMEM: the call asks for
-// them and the G root rows (rows 0..G-1) all fall in TMEM lanes 0..15 of
-// lane quarter 0, i.e. G <= 8 and G <= rq0.  For other shapes (trees of
-// fewer than four nodes) the launch leaves them to the select's score pass.
+// With two blocks, block 1 holds rows 0..R1-1 (R1 = R - 128) and block 0
+// rows R1..R-1, so that the root node's rows sit in block 1, whose softmax
+// warps carry a quarter of a block-0 warp's exponentials at 160 rows.  P^T
+// row (and O^T column) n is block-0 row n for n < 128, block-1 row n - 128.
+__host__ __device__ inline int t128_row_of(int n, int R)
+{
+    return R > kBlockM ? (n < kBlockM ? (R - kBlockM) + n : n - kBlockM) : n;
+}
+
+// Whether warp 0 reads the root node's scores out of TMEM (one block: the G
+// root rows are TMEM lanes 0..G-1 of S_0, inside lanes 0..15, i.e. G <= 8
+// and G <= rq0).
 __host__ __device__ inline bool t128_rs_warp0(const AttnArgs &a)
 {
     const int G = a.n_heads_q / a.n_heads_kv;
-    return a.root_scores != nullptr && G <= 8 && G <= t128_rq0(G * a.n_tree);
+    const int R = G * a.n_tree;
+    return a.root_scores != nullptr && R <= kBlockM && G <= 8 && G <= t128_rq0(R);
 }
 
-__host__ __device__ inline Layout t128_layout(int rows)
+// Whether the block-1 softmax warp of lane quarter 0 stores the root node's
+// scores (two blocks: block 1's first quarter run, rows 0..rq1-1, holds the
+// G root rows when G <= rq1 and G <= 8, i.e. they are its first 16 lanes).
+__host__ __device__ inline bool t128_rs_block1(const AttnArgs &a)
+{
+    const int G = a.n_heads_q / a.n_heads_kv;
+    const int R = G * a.n_tree;
+    const int rq1 = (R - kBlockM + 3) / 4;
+    return a.root_scores != nullptr && R > kBlockM && G <= 8 && G <= rq1;
+}
+
+// Shared memory that stages the root node's scores for bulk copies (two
+// tiles of the G root rows) when block 1 stores them and every row starts
+// on a 16-byte boundary; 0 otherwise (plain stores, or warp 0).
+__host__ __device__ inline int t128_rs_bytes(const AttnArgs &a)
+{
+    const bool bulk = t128_rs_block1(a) &&
+                      (reinterpret_cast<uintptr_t>(a.root_scores) & 15) == 0 &&
+                      (a.n_ctx & 3) == 0;
+    return bulk ? 2 * (a.n_heads_q / a.n_heads_kv) * kTileN * 4 : 0;
+}
+
+__host__ __device__ inline Layout t128_layout(int rows, int rs_bytes)
 {
     Layout L;
     L.r_pad = (rows + 15) / 16 * 16;
@@ -159,14 +190,15 @@ __host__ __device__ inline Layout t128_layout(int rows)
     // P^T: positions 0-63 then 64-127, each r_pad rows of 128 bytes; then
     // 1 KB that rows past the query rows are written to
     L.k_off = L.p_off + (size_t)L.r_pad * 256 + 1024;
-    const size_t fixed = 1024 + L.k_off + kAuxBytes;
+    const size_t fixed = 1024 + L.k_off + kAuxBytes + rs_bytes;
     int stages = (int)((kSmemLimit - fixed) / kStageBytes);
     stages = stages > 2 * kMaxStages ? 2 * kMaxStages : stages;
     L.stages_v = 2;
     L.stages_k = stages - 2 > kMaxStages ? kMaxStages : stages - 2;
     L.v_off = L.k_off + (size_t)L.stages_k * kStageBytes;
     L.aux_off = L.v_off + (size_t)L.stages_v * kStageBytes;
-    L.smem_bytes = 1024 + L.aux_off + kAuxBytes;
+    L.rs_off = L.aux_off + kAuxBytes;
+    L.smem_bytes = 1024 + L.rs_off + rs_bytes;
     return L;
 }
 
@@ -279,7 +311,8 @@ attn_t128_kernel(const __grid_constant__ CUtensorMap tmap_k,
     const int u0 = (rq0 + 15) / 16, u1 = (rq1 + 15) / 16;
     const int U = u0 + u1;  // softmax warps per lane quarter (at most 3)
     const bool rs_warp0 = t128_rs_warp0(a);
-    const Layout lay = t128_layout(R);
+    const int rs_bytes = t128_rs_bytes(a);
+    const Layout lay = t128_layout(R, rs_bytes);
     const int SK = lay.stages_k, SV = lay.stages_v, r_pad = lay.r_pad;
 
     extern __shared__ unsigned char smem_raw[];
@@ -352,7 +385,7 @@ attn_t128_kernel(const __grid_constant__ CUtensorMap tmap_k,
         const bool valid = lane < rq0 && n < R0;
         uint32_t qv[64];
         if (valid) {
-            const uint4 *src = q_row(n);
+            const uint4 *src = q_row(t128_row_of(n, R));
 #pragma unroll
             for (int c = 0; c < 16; ++c) {
                 const uint4 u = src[c];
@@ -377,7 +410,7 @@ attn_t128_kernel(const __grid_constant__ CUtensorMap tmap_k,
         const int m = q * 32 + lane;  // A-tile row = TMEM lane of S_1
         const int n = kBlockM + q * rq1 + lane;
         const bool valid = lane < rq1 && n < R;
-        const uint4 *src = valid ? q_row(n) : nullptr;
+        const uint4 *src = valid ? q_row(t128_row_of(n, R)) : nullptr;
 #pragma unroll
         for (int c = 0; c < 16; ++c) {
             const uint4 u = valid ? src[c] : make_uint4(0u, 0u, 0u, 0u);
@@ -440,7 +473,7 @@ attn_t128_kernel(const __grid_constant__ CUtensorMap tmap_k,
     } else if (warp == 0) {
         // --------------------------- root node's scores out of S_0 (lanes 0..G-1)
         if (rs_warp0) {
-            // one 16x256b load of lanes 0..15, the shape the softmax warps
+            // one block only; one 16x256b load of lanes 0..15, the shape the softmax warps
             // use: thread t holds lane t/4 (and 8 + t/4) at columns
             // 8j + 2(t%4) + {0, 1}, so threads 0..4G-1 hold the G root rows
             const int r = lane >> 2;          // root row of this thread (lanes 0..7)
@@ -585,6 +618,12 @@ attn_t128_kernel(const __grid_constant__ CUtensorMap tmap_k,
         const uint32_t p_addr = smem_addr(sP);
         const uint32_t p_scratch = p_addr + (uint32_t)r_pad * 256;
         float mA = -INFINITY, mB = -INFINITY, lA = 0.f, lB = 0.f, qA = 0.f, qB = 0.f;
+        // root rows (rows 0..G-1) held by this thread and this warp (block 1
+        // only); the first lane of a row's quad copies its staged scores out
+        const bool rootA = b == 1 && vA && t128_row_of(nA, R) < G;
+        const bool rootB = b == 1 && vB && t128_row_of(nB, R) < G;
+        const bool rs_warp = t128_rs_block1(a) && __any_sync(0xffffffffu, rootA || rootB);
+        const bool rs_issue = rs_bytes != 0 && (lane & 3) == 0 && (rootA || rootB);
         bool ok = true;
         for (int t = 0; t < n_tiles; ++t) {
             if (!warp_wait_bounded(smem_addr(&bar->s_full[b]), t & 1, abort, hdr)) {
@@ -601,11 +640,70 @@ attn_t128_kernel(const __grid_constant__ CUtensorMap tmap_k,
                 mbar_arrive(smem_addr(&bar->s_free[b]));
             // raw scores; the scale (> 0) is applied inside the exponent
             const int pos0 = (t_begin + t) * kTileN;
+            // the root node's rows leave their context scores, base 2, for the
+            // importance select
+            if (rs_warp && pos0 < a.n_ctx) {
+                if (rs_bytes != 0) {
+                    // staged in shared memory (one buffer per tile parity) and
+                    // written out by bulk copies, so that no global store sits
+                    // ahead of this warp's barrier arrivals
+                    const uint32_t buf =
+                        smem_addr(base + lay.rs_off) + (uint32_t)((t & 1) * G * kTileN * 4);
+                    if (rs_issue)
+                        bulk_wait_read<1>();   // the copy out of this buffer two tiles ago
+                    __syncwarp();
+#pragma unroll
+                    for (int h = 0; h < 2; ++h) {
+                        if (h ? rootB : rootA) {
+                            const uint32_t row = buf + (uint32_t)(t128_row_of(h ? nB : nA, R) *
+                                                                      kTileN * 4 +
+                                                                  c0 * 4);
+#pragma unroll
+                            for (int jj = 0; jj < 16; ++jj)
+                                st_shared_v2(row + 32 * jj,
+                                             __float_as_uint(__uint_as_float(r[4 * jj + 2 * h]) *
+                                                             a.scale_log2),
+                                             __float_as_uint(__uint_as_float(r[4 * jj + 2 * h + 1]) *
+                                                             a.scale_log2));
+                        }
+                    }
+                    fence_proxy_async_smem();
+                    __syncwarp();
+                    if (rs_issue) {
+                        const uint32_t bytes = (uint32_t)min(kTileN, a.n_ctx - pos0) * 4;
+#pragma unroll
+                        for (int h = 0; h < 2; ++h) {
+                            const int m = t128_row_of(h ? nB : nA, R);
+                            if (h ? rootB : rootA)
+                                bulk_store(a.root_scores + (size_t)(g * G + m) * a.n_ctx + pos0,
+                                           buf + (uint32_t)(m * kTileN * 4), bytes);
+                        }
+                        bulk_commit();
+                    }
+                } else {
+#pragma unroll
+                    for (int h = 0; h < 2; ++h) {
+                        if (h ? rootB : rootA) {
+                            float *dst = a.root_scores +
+                                         (size_t)(g * G + t128_row_of(h ? nB : nA, R)) * a.n_ctx;
+#pragma unroll
+                            for (int jj = 0; jj < 16; ++jj)
+#pragma unroll
+                                for (int e = 0; e < 2; ++e) {
+                                    const int pos = pos0 + 8 * jj + c0 + e;
+                                    if (pos < a.n_ctx)
+                                        dst[pos] =
+                                            __uint_as_float(r[4 * jj + 2 * h + e]) * a.scale_log2;
+                                }
+                        }
+                    }
+                }
+            }
             if (pos0 + kTileN > a.n_ctx) {
                 // visibility of this thread's 32 positions (entry k = 2 jj + e
                 // is position pos0 + 8 jj + c0 + e) for its two rows
-                const unsigned long long ancA = masks.anc[vA ? nA / G : 0];
-                const unsigned long long ancB = masks.anc[vB ? nB / G : 0];
+                const unsigned long long ancA = masks.anc[vA ? t128_row_of(nA, R) / G : 0];
+                const unsigned long long ancB = masks.anc[vB ? t128_row_of(nB, R) / G : 0];
                 uint32_t visA = 0u, visB = 0u;
 #pragma unroll 1
                 for (int k = 0; k < 32; ++k) {
@@ -665,6 +763,8 @@ attn_t128_kernel(const __grid_constant__ CUtensorMap tmap_k,
             if (lane == 0)
                 mbar_arrive(smem_addr(&bar->sm_done));
         }
+        if (rs_issue)
+            bulk_wait_all();   // shared memory must outlive the copies out of it
         // ---- (m, l) of each row (four threads' partial sums), then O^T
 #pragma unroll
         for (int o = 1; o <= 2; o <<= 1) {
@@ -682,7 +782,11 @@ attn_t128_kernel(const __grid_constant__ CUtensorMap tmap_k,
         float *ws_o =
             reinterpret_cast<float *>(reinterpret_cast<char *>(a.workspace) + kHeaderBytes);
         float *ws_ml = ws_o + (size_t)n_split * rows_all * kD;
-        auto orow_of = [&](int n) { return (n / G) * a.n_heads_q + g * G + n % G; };
+        // P^T row n -> output row of the head group
+        auto orow_of = [&](int n) {
+            const int m = t128_row_of(n, R);
+            return (m / G) * a.n_heads_q + g * G + m % G;
+        };
         if (ok && (lane & 3) == 0) {
             if (vA)
                 *reinterpret_cast<float4 *>(ws_ml + ((size_t)split * rows_all + orow_of(nA)) * 4) =
@@ -973,7 +1077,7 @@ cudaError_t attn_t128_launch(const AttnArgs &a, const TreeMasks &masks, int num_
     if (!encode_kv_map(&mk, a.k, rows, a.kv_cap, a.n_heads_kv, kTileN) ||
         !encode_kv_map(&mv, a.v, rows, a.kv_cap, a.n_heads_kv, kTileN))
         return cudaErrorInvalidValue;
-    const Layout lay = t128_layout((a.n_heads_q / a.n_heads_kv) * a.n_tree);
+    const Layout lay = t128_layout((a.n_heads_q / a.n_heads_kv) * a.n_tree, t128_rs_bytes(a));
     static const cudaError_t attr = cudaFuncSetAttribute(
         attn_t128_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemLimit);
     if (attr != cudaSuccess)
@@ -990,7 +1094,10 @@ cudaError_t attn_t128_launch(const AttnArgs &a, const TreeMasks &masks, int num_
                                      stream);
 }
 
-bool attn_t128_leaves_root_scores(const AttnArgs &a) { return t128_rs_warp0(a); }
+bool attn_t128_leaves_root_scores(const AttnArgs &a)
+{
+    return t128_rs_warp0(a) || t128_rs_block1(a);
+}
 
 size_t attn_exact_partial_bytes(int n_split, int n_heads_q, int n_tree)
 {

@@ -302,25 +302,39 @@ select_gather_kernel(SelectArgs a, int n_chunks, int slice, const float *__restr
             }
         };
         if ((N & 3) == 0) {
-            for (int nb = p0 + 4 * tid; nb < p1; nb += 4 * kP2Threads) {
-                float4 sv[kMaxGroup];
+            // one head at a time, eight 16-byte loads in flight per thread
+            constexpr int kU = 8;
+            const int v0 = p0 / 4, v1 = p1 / 4;
 #pragma unroll
-                for (int h = 0; h < kMaxGroup; ++h)
-                    if (h < G)
-                        sv[h] = __ldcg(reinterpret_cast<const float4 *>(
-                            s_all + (size_t)(g * G + h) * N + nb));
+            for (int h = 0; h < kMaxGroup; ++h) {
+                if (h >= G)
+                    continue;
+                const float4 *row = reinterpret_cast<const float4 *>(s_all + (size_t)(g * G + h) * N);
+                for (int vb = v0 + tid; vb < v1; vb += kU * kP2Threads) {
+                    float4 sv[kU];
 #pragma unroll
-                for (int h = 0; h < kMaxGroup; ++h)
-                    if (h < G) {
-                        const float mx = fmaxf(fmaxf(sv[h].x, sv[h].y), fmaxf(sv[h].z, sv[h].w));
-                        if (mx > rm[h]) {
-                            rl[h] = rm[h] == -INFINITY ? 0.f : rl[h] * exp2f(rm[h] - mx);
-                            rm[h] = mx;
-                        }
-                        if (mx != -INFINITY)
-                            rl[h] += exp2f(sv[h].x - rm[h]) + exp2f(sv[h].y - rm[h]) +
-                                     exp2f(sv[h].z - rm[h]) + exp2f(sv[h].w - rm[h]);
+                    for (int u = 0; u < kU; ++u) {
+                        const int vi = vb + u * kP2Threads;
+                        sv[u] = vi < v1 ? __ldcg(row + vi)
+                                        : make_float4(-INFINITY, -INFINITY, -INFINITY, -INFINITY);
                     }
+                    float mx = -INFINITY;
+#pragma unroll
+                    for (int u = 0; u < kU; ++u)
+                        mx = fmaxf(mx, fmaxf(fmaxf(sv[u].x, sv[u].y), fmaxf(sv[u].z, sv[u].w)));
+                    if (mx == -INFINITY)
+                        continue;
+                    if (mx > rm[h]) {
+                        rl[h] = rm[h] == -INFINITY ? 0.f : rl[h] * exp2f(rm[h] - mx);
+                        rm[h] = mx;
+                    }
+                    float acc = 0.f;
+#pragma unroll
+                    for (int u = 0; u < kU; ++u)
+                        acc += exp2f(sv[u].x - rm[h]) + exp2f(sv[u].y - rm[h]) +
+                               exp2f(sv[u].z - rm[h]) + exp2f(sv[u].w - rm[h]);
+                    rl[h] += acc;
+                }
             }
         } else {
             for (int n = p0 + tid; n < p1; n += kP2Threads)
@@ -432,42 +446,60 @@ select_gather_kernel(SelectArgs a, int n_chunks, int slice, const float *__restr
         // four consecutive positions per thread, one 16-byte load per head
         // (the slice is a multiple of 4, so p0 and p1 are too); every lane
         // of a warp runs the same number of rounds
+        // two rounds per step, so that 2 G 16-byte loads are in flight
+        constexpr int kR = 2;
         const int rounds = (p1 - p0 + 4 * kP2Threads - 1) / (4 * kP2Threads);
-        for (int it = 0; it < rounds; ++it) {
-            const int nb = p0 + 4 * (tid + it * kP2Threads);
-            const bool live = nb < p1;
-            float sc[4] = {0.f, 0.f, 0.f, 0.f};
-            if (live) {
-                float4 sv[kMaxGroup];
+        float hm[kMaxGroup], hw[kMaxGroup];
+#pragma unroll
+        for (int h = 0; h < kMaxGroup; ++h) {
+            hm[h] = h < G ? sh.head_m[h] : 0.f;
+            hw[h] = h < G ? sh.head_w[h] : 0.f;
+        }
+        for (int it0 = 0; it0 < rounds; it0 += kR) {
+            float4 sv[kR][kMaxGroup];
+#pragma unroll
+            for (int r = 0; r < kR; ++r) {
+                const int nb = p0 + 4 * (tid + (it0 + r) * kP2Threads);
 #pragma unroll
                 for (int h = 0; h < kMaxGroup; ++h)
                     if (h < G)
-                        sv[h] = __ldcg(reinterpret_cast<const float4 *>(
-                            s_all + (size_t)(g * G + h) * N + nb));
-#pragma unroll
-                for (int h = 0; h < kMaxGroup; ++h)
-                    if (h < G) {
-                        const float m = sh.head_m[h], wgt = sh.head_w[h];
-                        sc[0] += exp2f(sv[h].x - m) * wgt;
-                        sc[1] += exp2f(sv[h].y - m) * wgt;
-                        sc[2] += exp2f(sv[h].z - m) * wgt;
-                        sc[3] += exp2f(sv[h].w - m) * wgt;
-                    }
+                        sv[r][h] = nb < p1 ? __ldcg(reinterpret_cast<const float4 *>(
+                                                 s_all + (size_t)(g * G + h) * N + nb))
+                                           : make_float4(0.f, 0.f, 0.f, 0.f);
             }
-            uint32_t kk[4];
 #pragma unroll
-            for (int e = 0; e < 4; ++e)
-                kk[e] = order_key(sc[e]);
-            if (live) {
-                *reinterpret_cast<uint4 *>(&keys[nb - p0]) = make_uint4(kk[0], kk[1], kk[2], kk[3]);
-                if (a.scores_out)
-                    *reinterpret_cast<float4 *>(a.scores_out + (size_t)g * N + nb) =
-                        make_float4(sc[0], sc[1], sc[2], sc[3]);
-            }
-            if (do_select)
+            for (int r = 0; r < kR; ++r) {
+                if (it0 + r >= rounds)
+                    break;   // uniform: every lane has the same rounds
+                const int nb = p0 + 4 * (tid + (it0 + r) * kP2Threads);
+                const bool live = nb < p1;
+                float sc[4] = {0.f, 0.f, 0.f, 0.f};
+                if (live) {
+#pragma unroll
+                    for (int h = 0; h < kMaxGroup; ++h)
+                        if (h < G) {
+                            sc[0] += exp2f(sv[r][h].x - hm[h]) * hw[h];
+                            sc[1] += exp2f(sv[r][h].y - hm[h]) * hw[h];
+                            sc[2] += exp2f(sv[r][h].z - hm[h]) * hw[h];
+                            sc[3] += exp2f(sv[r][h].w - hm[h]) * hw[h];
+                        }
+                }
+                uint32_t kk[4];
 #pragma unroll
                 for (int e = 0; e < 4; ++e)
-                    hist_add(sh.hist[0], live && nb + e >= a.n_sink, kk[e], 0u, 0u, 0);
+                    kk[e] = order_key(sc[e]);
+                if (live) {
+                    *reinterpret_cast<uint4 *>(&keys[nb - p0]) =
+                        make_uint4(kk[0], kk[1], kk[2], kk[3]);
+                    if (a.scores_out)
+                        *reinterpret_cast<float4 *>(a.scores_out + (size_t)g * N + nb) =
+                            make_float4(sc[0], sc[1], sc[2], sc[3]);
+                }
+                if (do_select)
+#pragma unroll
+                    for (int e = 0; e < 4; ++e)
+                        hist_add(sh.hist[0], live && nb + e >= a.n_sink, kk[e], 0u, 0u, 0);
+            }
         }
     } else {
         // eight positions per thread per step so their loads are in flight together
@@ -536,14 +568,21 @@ select_gather_kernel(SelectArgs a, int n_chunks, int slice, const float *__restr
             const int nbins = (int)radix_mask(pass) + 1;
             int x[4] = {0, 0, 0, 0};
             if (4 * tid < nbins) {
-                // bins nbins-4-4t .. nbins-1-4t: one 16-byte read per rank
+                // bins nbins-4-4t .. nbins-1-4t: one 16-byte read per rank,
+                // all ranks' reads in flight together
                 const int q = (nbins - 4 - 4 * tid) / 4;
-                for (int r = 0; r < n_ranks; ++r) {
-                    const int4 v = reinterpret_cast<const int4 *>(cluster.map_shared_rank(hist, r))[q];
-                    x[0] += v.w;
-                    x[1] += v.z;
-                    x[2] += v.y;
-                    x[3] += v.x;
+                int4 v[kClusterCtas];
+#pragma unroll
+                for (int r = 0; r < kClusterCtas; ++r)
+                    v[r] = r < n_ranks
+                               ? reinterpret_cast<const int4 *>(cluster.map_shared_rank(hist, r))[q]
+                               : make_int4(0, 0, 0, 0);
+#pragma unroll
+                for (int r = 0; r < kClusterCtas; ++r) {
+                    x[0] += v[r].w;
+                    x[1] += v[r].z;
+                    x[2] += v[r].y;
+                    x[3] += v[r].x;
                 }
             }
             int above;
