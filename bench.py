@@ -293,7 +293,8 @@ class Step:
         self.fused = fused
         if fused:
             self.rs = torch.empty((hq, w.n_ctx), dtype=torch.float32, device=dev)
-            self.ws_sel = L.new_workspace(L.kv_select_from_scores_workspace_size(), dev)
+            self.ws_sel = L.new_workspace(L.kv_select_from_scores_workspace_size(hq, hkv, w.n_ctx),
+                                          dev)
         else:
             self.rs = None
             self.ws_sel = L.new_workspace(

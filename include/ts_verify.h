@@ -29,8 +29,10 @@
  *    bounded wait) are recorded in the workspace's status word, read by
  *    ts_workspace_status().
  *  - Workspace: sized by the matching *_workspace_size() call, at least
- *    256-byte aligned, zero-filled once by the caller before first use
- *    (every call leaves it zero-filled again apart from the status word).
+ *    256-byte aligned, zero-filled once by the caller before first use.
+ *    Every call returns the counters and tickets it relies on to zero
+ *    before it ends; the rest of the workspace is scratch that each call
+ *    writes before it reads.
  *    Concurrent calls need distinct workspaces.
  *  - bf16 tensors are raw IEEE bfloat16 bit patterns; every device pointer
  *    must be 16-byte aligned.
@@ -232,9 +234,13 @@ TS_API int ts_tree_verify_attn_root_scores(const void *q, const void *k_cache,
  * top-budget selection and gather.  root_scores: device fp32 [n_heads_q,
  * n_ctx], read only.  The other arguments are as for
  * ts_kv_importance_select (no query rows, no scale); the workspace needs
- * ts_kv_select_from_scores_workspace_size() bytes.
+ * ts_kv_select_from_scores_workspace_size(n_heads_q, n_heads_kv, n_ctx)
+ * bytes for the current device (0 for an invalid shape): per-chunk head
+ * statistics, the importance scores when scores_out is NULL, per-head
+ * histograms and counters, and a candidate list of up to n_ctx entries per
+ * KV head.
  */
-TS_API size_t ts_kv_select_from_scores_workspace_size(void);
+TS_API size_t ts_kv_select_from_scores_workspace_size(int n_heads_q, int n_heads_kv, int n_ctx);
 TS_API int ts_kv_select_from_scores(const float *root_scores, const void *k_cache,
                                     const void *v_cache, int64_t kv_cap, int n_heads_q,
                                     int n_heads_kv, int head_dim, int n_ctx, int n_sink,

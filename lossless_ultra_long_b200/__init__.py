@@ -66,7 +66,7 @@ def _lib():
         lib.ts_tree_verify_attn_root_scores.argtypes = [P, P, P, i64, i32, i32, i32, i32, i32, P,
                                                         f32, P, P, P, sz, P]
         lib.ts_kv_select_from_scores_workspace_size.restype = sz
-        lib.ts_kv_select_from_scores_workspace_size.argtypes = []
+        lib.ts_kv_select_from_scores_workspace_size.argtypes = [i32, i32, i32]
         lib.ts_kv_select_from_scores.restype = i32
         lib.ts_kv_select_from_scores.argtypes = [P, P, P, i64, i32, i32, i32, i32, i32, i32, P, P,
                                                  P, P, i64, P, sz, P]
@@ -244,8 +244,8 @@ def kv_importance_select(q_last, k_cache, v_cache, n_ctx: int, n_sink: int, budg
     return idx_out, k_partial, v_partial, scores_out
 
 
-def kv_select_from_scores_workspace_size() -> int:
-    return int(_lib().ts_kv_select_from_scores_workspace_size())
+def kv_select_from_scores_workspace_size(n_heads_q, n_heads_kv, n_ctx) -> int:
+    return int(_lib().ts_kv_select_from_scores_workspace_size(n_heads_q, n_heads_kv, n_ctx))
 
 
 def kv_select_from_scores(root_scores, k_cache, v_cache, n_ctx: int, n_sink: int, budget: int,
@@ -280,7 +280,7 @@ def kv_select_from_scores(root_scores, k_cache, v_cache, n_ctx: int, n_sink: int
     if scores_out is not None:
         _check_dev("scores_out", scores_out, torch.float32)
     if workspace is None:
-        workspace = new_workspace(kv_select_from_scores_workspace_size(), dev)
+        workspace = new_workspace(kv_select_from_scores_workspace_size(hq, hkv, int(n_ctx)), dev)
     rc = _lib().ts_kv_select_from_scores(
         _ptr(root_scores), _ptr(k_cache), _ptr(v_cache), cap, hq, hkv, d, int(n_ctx),
         int(n_sink), int(budget), _ptr(scores_out), _ptr(idx_out), _ptr(k_partial),

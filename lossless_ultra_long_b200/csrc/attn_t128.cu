@@ -31,7 +31,9 @@
 //   warp 3      one lane is the TMA producer of K and V (two 64-column boxes
 //               of 128 positions per tile, 128-byte swizzle), K one tile
 //               ahead of V.  The map's row extent is n_ctx + T, so rows past
-//               the tree tail arrive as zeros.
+//               the tree tail arrive as zeros.  It starts as soon as the
+//               barriers exist, while the other warps put the query rows in
+//               place, so HBM is busy from the first microsecond.
 //   warp 0      when the call asks for the root node's scores and all of
 //               them sit in TMEM lane quarter 0 (the warp's own quarter),
 //               reads them out of S_0 each tile and stores them, so that no
@@ -43,8 +45,12 @@
 //               scale to base 2, ancestor mask on tiles that reach the tree
 //               tail, exponentiate against a per-row reference max, write
 //               the bf16 P^T rows.  l sums the bf16-rounded P so the
-//               normalisation matches what PV used.  At the end they write
-//               O^T (their lane quarters together cover all of D).
+//               normalisation matches what PV used.  At the end they read
+//               O^T (their lane quarters together cover all of D) into the
+//               freed K/V ring in output-row order and send each node's G
+//               rows to the workspace with one bulk copy: per-row stores
+//               from every SM at once took several microseconds per CTA,
+//               on the critical path of each split.
 // TMEM: O^T in [0, 192), Q_0 in [192, 256), S_0 in [256, 384), S_1 in
 // [384, 512).
 //
@@ -107,6 +113,11 @@ constexpr float kMaxRowSum = 9.223372036854775808e18f;   // 2^63: bound on a row
 // errors stays inside 2e-3.
 constexpr float kNeffMin = 64.f;
 constexpr size_t kSmemLimit = 232448;        // dynamic shared memory per CTA
+static_assert(kBlockM % 32 == 0, "a 32-column O^T chunk lies inside one query block");
+constexpr int kBarQuery = 1;                 // named barrier: query rows in place
+constexpr int kBarOut = 2;                   // named barrier: O^T staged in shared memory
+constexpr int kBarQLoads = 3;                // named barrier: the query loads are issued
+constexpr int kQLoadThreads = 32 * 9;        // warps 4-11 arrive, the producer warp waits
 
 struct Bars {
     uint64_t full_k[kMaxStages];
@@ -133,6 +144,7 @@ constexpr size_t kAuxBytes = (sizeof(Aux) + 1023) / 1024 * 1024;
 struct Layout {
     int r_pad;  // rows rounded up to 16: N of the PV product
     int stages_k, stages_v;
+    bool o_staged;  // the freed K/V ring holds every O row (fp32) for the write-out
     size_t q1_off, p_off, k_off, v_off, aux_off, rs_off, smem_bytes;
 };
 
@@ -196,6 +208,7 @@ __host__ __device__ inline Layout t128_layout(int rows, int rs_bytes)
     L.stages_v = 2;
     L.stages_k = stages - 2 > kMaxStages ? kMaxStages : stages - 2;
     L.v_off = L.k_off + (size_t)L.stages_k * kStageBytes;
+    L.o_staged = (size_t)rows * kD * 4 <= (size_t)(L.stages_k + L.stages_v) * kStageBytes;
     L.aux_off = L.v_off + (size_t)L.stages_v * kStageBytes;
     L.rs_off = L.aux_off + kAuxBytes;
     L.smem_bytes = 1024 + L.rs_off + rs_bytes;
@@ -357,6 +370,9 @@ attn_t128_kernel(const __grid_constant__ CUtensorMap tmap_k,
         bar->abort = 0u;
         bar->overflow = 0;
         fence_mbar_init();
+        // the combine kernel may take the SMs this grid leaves idle (and
+        // then each SM a split frees) and wait there for this grid's end
+        launch_dependents();
     }
     if (warp == 1) {
         tmem_alloc(smem_addr(&bar->tmem_base), kTmemCols);
@@ -371,6 +387,11 @@ attn_t128_kernel(const __grid_constant__ CUtensorMap tmap_k,
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = bar->tmem_base;
+    // The TMA producer (warp 3) starts streaming K and V as soon as the
+    // query rows' loads are on their way (ahead of the K/V requests, so
+    // that they are not queued behind a whole ring of tiles from every
+    // CTA); the other warps put the query rows in place meanwhile and meet
+    // at a named barrier of their own.
 
     // Query rows of this KV head into place: row n = node * G + (head - g*G).
     // Block 0 (rows 0..R0-1) into TMEM lanes (warps 4-7, 32x32b stores);
@@ -379,7 +400,9 @@ attn_t128_kernel(const __grid_constant__ CUtensorMap tmap_k,
         return reinterpret_cast<const uint4 *>(
             a.q + ((int64_t)(n / G) * a.n_heads_q + g * G + n % G) * kD);
     };
-    if (warp >= 4 && warp < 8) {
+    if (warp == 3) {
+        // producer: below, without the query barrier
+    } else if (warp >= 4 && warp < 8) {
         const int q = warp & 3;
         const int n = q * rq0 + lane;
         const bool valid = lane < rq0 && n < R0;
@@ -388,7 +411,7 @@ attn_t128_kernel(const __grid_constant__ CUtensorMap tmap_k,
             const uint4 *src = q_row(t128_row_of(n, R));
 #pragma unroll
             for (int c = 0; c < 16; ++c) {
-                const uint4 u = src[c];
+                const uint4 u = __ldg(src + c);
                 qv[4 * c] = u.x;
                 qv[4 * c + 1] = u.y;
                 qv[4 * c + 2] = u.z;
@@ -399,6 +422,7 @@ attn_t128_kernel(const __grid_constant__ CUtensorMap tmap_k,
             for (int c = 0; c < 64; ++c)
                 qv[c] = 0u;
         }
+        named_bar_arrive(kBarQLoads, kQLoadThreads);
         const uint32_t qa = tmem + ((uint32_t)(q * 32) << 16) + kQCol;
         uint32_t (&q0)[32] = *reinterpret_cast<uint32_t (*)[32]>(&qv[0]);
         uint32_t (&q1)[32] = *reinterpret_cast<uint32_t (*)[32]>(&qv[32]);
@@ -411,20 +435,30 @@ attn_t128_kernel(const __grid_constant__ CUtensorMap tmap_k,
         const int n = kBlockM + q * rq1 + lane;
         const bool valid = lane < rq1 && n < R;
         const uint4 *src = valid ? q_row(t128_row_of(n, R)) : nullptr;
+        // every load in flight before the first store (the stores could
+        // alias the loads as far as the compiler knows)
+        uint4 u[16];
 #pragma unroll
-        for (int c = 0; c < 16; ++c) {
-            const uint4 u = valid ? src[c] : make_uint4(0u, 0u, 0u, 0u);
+        for (int c = 0; c < 16; ++c)
+            u[c] = valid ? __ldg(src + c) : make_uint4(0u, 0u, 0u, 0u);
+        named_bar_arrive(kBarQLoads, kQLoadThreads);
+#pragma unroll
+        for (int c = 0; c < 16; ++c)
             *reinterpret_cast<uint4 *>(sQ1 + (c >> 3) * kBoxBytes + (m >> 3) * 1024 +
-                                       (m & 7) * 128 + (((c & 7) ^ (m & 7)) << 4)) = u;
-        }
+                                       (m & 7) * 128 + (((c & 7) ^ (m & 7)) << 4)) = u[c];
         fence_proxy_async_smem();
+    } else if (warp >= 8 && warp < 12) {
+        named_bar_arrive(kBarQLoads, kQLoadThreads);   // one block: no rows to load
     }
-    tc_fence_before();
-    __syncthreads();
-    tc_fence_after();
+    if (warp != 3) {
+        tc_fence_before();
+        named_bar_sync(kBarQuery, kThreads - 32);
+        tc_fence_after();
+    }
 
     if (warp == 3) {
         // ------------------------------------ TMA producer (K one tile ahead)
+        named_bar_sync(kBarQLoads, kQLoadThreads);
         if (lane == 0) {
             int nk = 0, nv = 0;   // tiles issued so far
             // step i issues K(i), then V(i - 1): K is consumed a whole softmax
@@ -795,19 +829,48 @@ attn_t128_kernel(const __grid_constant__ CUtensorMap tmap_k,
                 *reinterpret_cast<float4 *>(ws_ml + ((size_t)split * rows_all + orow_of(nB)) * 4) =
                     make_float4(mB, lB, qB, 0.f);
         }
-        if (ok && warp_wait_bounded(smem_addr(&bar->o_final), 0, abort, hdr)) {
+        // O^T out of TMEM.  Once the last PV is done the K/V ring is free:
+        // the rows are staged there in output order (row m = node * G + the
+        // head's index in the group, 512 bytes each), so that each node's G
+        // rows leave as one contiguous bulk copy instead of many small
+        // stores.
+        const bool have_o = ok && warp_wait_bounded(smem_addr(&bar->o_final), 0, abort, hdr);
+        const int d = 32 * q + lane;
+        if (have_o) {
             tc_fence_after();
-            const int d = 32 * q + lane;
+            const bool staged = lay.o_staged;
             for (int c = 32 * j; c < r_pad; c += 32 * U) {
                 uint32_t o[32];
                 tmem_ld32(tmem + o_lane + c, o);
+                const int nv = min(32, R - c);   // query rows among P^T rows c .. c+31
+                if (staged) {
+                    // a 32-row chunk lies inside one block, where the output
+                    // row is the P^T row plus a constant
+                    float *dst = reinterpret_cast<float *>(sK) + (size_t)t128_row_of(c, R) * kD + d;
 #pragma unroll
-                for (int jj = 0; jj < 32; ++jj) {
-                    const int n = c + jj;
-                    if (n < R)
-                        ws_o[((size_t)split * rows_all + orow_of(n)) * kD + d] =
-                            __uint_as_float(o[jj]);
+                    for (int jj = 0; jj < 32; ++jj)
+                        if (jj < nv)
+                            dst[jj * kD] = __uint_as_float(o[jj]);
+                } else {
+#pragma unroll
+                    for (int jj = 0; jj < 32; ++jj)
+                        if (jj < nv)
+                            ws_o[((size_t)split * rows_all + orow_of(c + jj)) * kD + d] =
+                                __uint_as_float(o[jj]);
                 }
+            }
+        }
+        if (lay.o_staged) {
+            fence_proxy_async_smem();
+            named_bar_sync(kBarOut, 128 * U);   // every softmax warp, whatever its path
+            // a warp that gave up set the abort flag before this barrier
+            if (!*abort && lane == 0) {
+                const int sw = warp - 4;   // 0 .. 4U-1
+                for (int node = sw; node < a.n_tree; node += 4 * U)
+                    bulk_store(ws_o + ((size_t)split * rows_all + (size_t)node * a.n_heads_q + g * G) * kD,
+                               smem_addr(sK) + (uint32_t)(node * G * kD * 4), (uint32_t)(G * kD * 4));
+                bulk_commit();
+                bulk_wait_all();   // the ring must outlive the copies out of it
             }
         }
     }
@@ -907,6 +970,9 @@ attn_t128_combine_kernel(AttnArgs a, TreeMasks masks, int n_split, int split_pos
     const int rows_all = a.n_tree * a.n_heads_q;
     const int row = blockIdx.x * 8 + (threadIdx.x >> 5);
     const int lane = threadIdx.x & 31;
+    // launched early (programmatic dependent launch): the split partials
+    // are complete only once the split grid has finished
+    grid_dependency_wait();
     if (row >= rows_all)
         return;
     const int head = row % a.n_heads_q, node = row / a.n_heads_q;
@@ -1109,9 +1175,20 @@ cudaError_t attn_exact_combine_launch(const AttnArgs &a, const TreeMasks &masks,
                                       cudaStream_t stream)
 {
     const int rows_all = a.n_tree * a.n_heads_q;
-    attn_t128_combine_kernel<<<(rows_all + 7) / 8, 256, 0, stream>>>(a, masks, n_split,
-                                                                      split_positions, flags);
-    const cudaError_t e = cudaGetLastError();
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((rows_all + 7) / 8);
+    cfg.blockDim = dim3(256);
+    cfg.dynamicSmemBytes = 0;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    cudaError_t e = cudaLaunchKernelEx(&cfg, attn_t128_combine_kernel, a, masks, n_split,
+                                       split_positions, flags);
+    if (e == cudaSuccess)
+        e = cudaGetLastError();
     if (e == cudaSuccess)
         count_launches(1);
     return e;

@@ -16,31 +16,34 @@
 //   of 64-row tiles (one producer lane, four MMA warps).  Writes s (fp32
 //   [Hq, n_ctx]) and a running (max, sum 2^(s-max)) per head and chunk.
 //   K is read once: Hkv * n_ctx * D * 2 bytes.
-// Pass 2 (one 8-CTA cluster per KV head): merges the chunk partials into
-//   the softmax max / normaliser of each head, forms
-//   score[n] = (1/G) sum_h 2^(s[h,n] - M_h) / Z_h for its slice of
-//   positions, keeps the order-preserving bit pattern of every score in
-//   shared memory, and finds the budget-th largest candidate exactly with a
-//   4 x 8-bit radix select whose histograms are summed over the cluster
-//   through distributed shared memory.  Positions are then compacted in
-//   ascending order (sinks, every key above the threshold, and the first
-//   keys equal to it in position order, so equal scores go to the lower
-//   position) and the kept K/V rows are copied with 16-byte loads.
-#include <cooperative_groups.h>
+// Selection (grids of chunks x Hkv, about two CTAs per SM, every head at
+//   once):
+//   1. per chunk, each head's (max, sum 2^(s-max)) -- only when the scores
+//      come from the caller; the score pass leaves them itself;
+//   2. the importance score[n] = (1/G) sum_h 2^(s[h,n] - M_h) / Z_h of the
+//      chunk's positions, written out, and a 4096-bin histogram of the top
+//      bits of the candidates' scores (non-negative floats order as their
+//      bit patterns), summed per head in global memory; the last chunk of a
+//      head to finish finds the bin holding the budget-th largest candidate;
+//   3. per chunk, the candidates above that bin are counted and those in it
+//      listed (score bits, position);
+//   4. one CTA per head finds the exact budget-th largest score among the
+//      listed ones (two radix passes over the remaining 19 bits) and, per
+//      chunk, how many positions are kept before it;
+//   5. per chunk, the kept positions -- sinks, every score above the
+//      threshold, and the first scores equal to it in position order, so
+//      equal scores go to the lower position -- are written in ascending
+//      order from the chunk's offset and their K/V rows copied with 16-byte
+//      loads.
 #include <math.h>
 
 #include "attn_common.cuh"
 #include "sm100.cuh"
 #include "ts_internal.cuh"
 
-namespace cg = cooperative_groups;
-
 namespace ts {
 namespace {
 
-constexpr int kClusterCtas = 8;
-constexpr int kP2Threads = 512;
-constexpr int kMaxSlice = 48 * 1024;   // positions per CTA held in shared memory
 constexpr int kMaxGroup = TS_MAX_SELECT_GROUP;
 
 // ------------------------------------------------------------------ pass 1
@@ -195,14 +198,73 @@ score_logits_kernel(const __grid_constant__ CUtensorMap tmap_k, SelectArgs a, in
     }
 }
 
-// ------------------------------------------------------------------ pass 2
-__device__ __forceinline__ uint32_t order_key(float f)
+// ------------------------------------------------------ the selection pipeline
+// Importance, threshold, compaction and gather for every KV head at once,
+// in five short kernels over (chunk of positions, KV head) grids that cover
+// the GPU.  Key of a position: the bit pattern of its importance, a sum of
+// non-negative terms, so keys order as the values do.
+constexpr int kSelThreads = 512;
+constexpr int kBins0 = 4096;   // first-level bins: key bits 30..19
+constexpr int kShift0 = 19;
+constexpr int kMaxChunks = 256;
+constexpr int kMaxChunkLen = 48 * 1024;   // a chunk's kept positions are listed in shared memory
+static_assert(kMaxChunks <= kSelThreads, "one chunk per thread in the offset scan");
+static_assert(kMaxGroup <= kSelThreads / 32, "one warp per head in the statistics merge");
+
+enum SelMode { kSelect = 0, kKeepAll = 1, kSinksOnly = 2 };
+
+struct SelInfo {
+    int digit0;    // the bin of the budget-th largest candidate key
+    int need0;     // how many keys of that bin are kept
+    int n_cand;    // keys of that bin, appended to the candidate list
+    uint32_t T;    // the budget-th largest candidate key
+    int need_eq;   // how many keys equal to T are kept (lowest positions first)
+    int pad[3];
+};
+
+struct SelWs {
+    float2 *part;      // [Hq, n_parts] per-chunk (max, sum 2^(s - max)) of each head
+    int n_parts;
+    float *imp;        // [Hkv, n_ctx] importance (scores_out or workspace)
+    int *hist;         // [Hkv, kBins0]
+    int *tick;         // [Hkv]
+    SelInfo *info;     // [Hkv]
+    int *above;        // [Hkv, NC] candidate keys above the threshold bin, per chunk
+    int2 *chunk;       // [Hkv, NC] (kept before the chunk, equal-to-T keys before it)
+    uint2 *cand;       // [Hkv, n_ctx] (key, position) of the threshold bin's keys
+};
+
+struct SelGeom {
+    int nc;      // chunks per head
+    int chunk;   // positions per chunk (a multiple of 4)
+};
+
+__device__ __forceinline__ float warp_max(float x)
 {
-    const uint32_t b = __float_as_uint(f);
-    return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1)
+        x = fmaxf(x, __shfl_xor_sync(0xffffffffu, x, o));
+    return x;
 }
 
-// exclusive scan of one int per thread over the block; returns the total
+__device__ __forceinline__ float warp_sum(float x)
+{
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1)
+        x += __shfl_xor_sync(0xffffffffu, x, o);
+    return x;
+}
+
+__device__ __forceinline__ int warp_isum(int x)
+{
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1)
+        x += __shfl_xor_sync(0xffffffffu, x, o);
+    return x;
+}
+
+// Exclusive scan of one int per thread over the block (any multiple of 32
+// threads up to 1024); returns the block total.  scratch: 65 ints.
 __device__ int block_exclusive_scan(int x, int *scratch, int &excl)
 {
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -218,7 +280,7 @@ __device__ int block_exclusive_scan(int x, int *scratch, int &excl)
     __syncthreads();
     if (warp == 0) {
         const int nw = blockDim.x / 32;
-        int w = lane < nw ? scratch[lane] : 0;
+        const int w = lane < nw ? scratch[lane] : 0;
         int wi = w;
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) {
@@ -238,228 +300,144 @@ __device__ int block_exclusive_scan(int x, int *scratch, int &excl)
     return total;
 }
 
-// Radix select of the budget-th largest key in three passes over the
-// key bits: 11, 11 and 10 bits from the top.
-constexpr int kRadixBins = 2048;
-constexpr int kRadixPasses = 3;
-__host__ __device__ constexpr int radix_shift(int pass) { return pass == 0 ? 21 : pass == 1 ? 10 : 0; }
-__host__ __device__ constexpr uint32_t radix_mask(int pass) { return pass == 2 ? 1023u : 2047u; }
-
-struct alignas(16) P2Shared {
-    int hist[2][kRadixBins];   // pass p uses hist[p & 1]
-    int scan[72];
-    float head_w[kMaxGroup];   // 1 / (G * Z_h)
-    float head_m[kMaxGroup];
-    float2 slice_ml[kMaxGroup];  // this CTA's (max, sum) per head over its slice
-    float2 warp_ml[kP2Threads / 32][kMaxGroup];  // each warp's (max, sum) per head
-    int counts[4];             // [0] equal-to-threshold, [1] kept
-    int bcast[4];
-};
-
-template <int D>
-__global__ void __launch_bounds__(kP2Threads, 1)
-select_gather_kernel(SelectArgs a, int n_chunks, int slice, const float *__restrict__ s_all)
+// Kernel 1 (scores given by the caller): per (chunk, KV head), each head of
+// the group's (max, sum of 2^(s - max)) over the chunk.
+__global__ void __launch_bounds__(kSelThreads)
+sel_stats_kernel(SelectArgs a, SelGeom geo, SelWs ws)
 {
-    cg::cluster_group cluster = cg::this_cluster();
-    extern __shared__ __align__(16) unsigned char dsm[];
-    P2Shared &sh = *reinterpret_cast<P2Shared *>(dsm);
-    uint32_t *keys = reinterpret_cast<uint32_t *>(dsm + sizeof(P2Shared));
-
-    const int rank = (int)cluster.block_rank();
-    const int n_ranks = (int)cluster.num_blocks();
-    const int g = blockIdx.y;
+    __shared__ float2 red[kSelThreads / 32];
+    const int c = blockIdx.x, g = blockIdx.y;
     const int G = a.n_heads_q / a.n_heads_kv;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int N = a.n_ctx;
-    const int p0 = min(rank * slice, N), p1 = min(p0 + slice, N);
-    const int64_t want = (int64_t)a.n_sink + a.budget;
-    const bool keep_all = want >= N;
-    const int n_keep = keep_all ? N : (int)want;
-
-    const float2 *part = reinterpret_cast<const float2 *>(
-        reinterpret_cast<const char *>(a.workspace) + kHeaderBytes +
-        (size_t)a.n_heads_q * N * sizeof(float));
-
-    // softmax max / normaliser per head of the group: from the score pass's
-    // per-chunk partials, or, for scores given by the caller, from this
-    // cluster's own pass over them (each CTA its slice, summed across ranks)
-    if (a.root_scores != nullptr) {
-        // every thread folds its positions of the slice into a running
-        // (max, sum of 2^(s - max)) per head in one pass; then the warp, the
-        // CTA and the cluster combine the pairs
-        float rm[kMaxGroup], rl[kMaxGroup];
-#pragma unroll
-        for (int h = 0; h < kMaxGroup; ++h) {
-            rm[h] = -INFINITY;
-            rl[h] = 0.f;
-        }
-        auto fold = [](float &m, float &l, float x) {
-            if (x > m) {
-                l = (m == -INFINITY ? 0.f : l * exp2f(m - x)) + 1.f;
-                m = x;
-            } else if (x != -INFINITY) {
-                l += exp2f(x - m);
-            }
-        };
+    const int p0 = min(c * geo.chunk, N), p1 = min(p0 + geo.chunk, N);
+    for (int h = 0; h < G; ++h) {
+        const float *row = a.root_scores + (size_t)(g * G + h) * N;
+        float m = -INFINITY, l = 0.f;
         if ((N & 3) == 0) {
-            // one head at a time, eight 16-byte loads in flight per thread
+            // the chunk is a multiple of 4 positions: 16-byte loads, all of
+            // this thread's loads in flight together
             constexpr int kU = 8;
             const int v0 = p0 / 4, v1 = p1 / 4;
+            for (int vb = v0 + tid; vb < v1; vb += kU * kSelThreads) {
+                float4 x[kU];
 #pragma unroll
-            for (int h = 0; h < kMaxGroup; ++h) {
-                if (h >= G)
-                    continue;
-                const float4 *row = reinterpret_cast<const float4 *>(s_all + (size_t)(g * G + h) * N);
-                for (int vb = v0 + tid; vb < v1; vb += kU * kP2Threads) {
-                    float4 sv[kU];
-#pragma unroll
-                    for (int u = 0; u < kU; ++u) {
-                        const int vi = vb + u * kP2Threads;
-                        sv[u] = vi < v1 ? __ldcg(row + vi)
-                                        : make_float4(-INFINITY, -INFINITY, -INFINITY, -INFINITY);
-                    }
-                    float mx = -INFINITY;
-#pragma unroll
-                    for (int u = 0; u < kU; ++u)
-                        mx = fmaxf(mx, fmaxf(fmaxf(sv[u].x, sv[u].y), fmaxf(sv[u].z, sv[u].w)));
-                    if (mx == -INFINITY)
-                        continue;
-                    if (mx > rm[h]) {
-                        rl[h] = rm[h] == -INFINITY ? 0.f : rl[h] * exp2f(rm[h] - mx);
-                        rm[h] = mx;
-                    }
-                    float acc = 0.f;
-#pragma unroll
-                    for (int u = 0; u < kU; ++u)
-                        acc += exp2f(sv[u].x - rm[h]) + exp2f(sv[u].y - rm[h]) +
-                               exp2f(sv[u].z - rm[h]) + exp2f(sv[u].w - rm[h]);
-                    rl[h] += acc;
+                for (int u = 0; u < kU; ++u) {
+                    const int vi = vb + u * kSelThreads;
+                    x[u] = vi < v1 ? __ldcg(reinterpret_cast<const float4 *>(row) + vi)
+                                   : make_float4(-INFINITY, -INFINITY, -INFINITY, -INFINITY);
                 }
+                float mx = -INFINITY;
+#pragma unroll
+                for (int u = 0; u < kU; ++u)
+                    mx = fmaxf(mx, fmaxf(fmaxf(x[u].x, x[u].y), fmaxf(x[u].z, x[u].w)));
+                if (mx == -INFINITY)
+                    continue;
+                if (mx > m) {
+                    l = m == -INFINITY ? 0.f : l * exp2f(m - mx);
+                    m = mx;
+                }
+                float acc = 0.f;
+#pragma unroll
+                for (int u = 0; u < kU; ++u)
+                    acc += exp2f(x[u].x - m) + exp2f(x[u].y - m) + exp2f(x[u].z - m) +
+                           exp2f(x[u].w - m);
+                l += acc;
             }
         } else {
-            for (int n = p0 + tid; n < p1; n += kP2Threads)
-#pragma unroll
-                for (int h = 0; h < kMaxGroup; ++h)
-                    if (h < G)
-                        fold(rm[h], rl[h], __ldcg(s_all + (size_t)(g * G + h) * N + n));
-        }
-        // warp: pairwise merge of (m, l)
-#pragma unroll
-        for (int h = 0; h < kMaxGroup; ++h) {
-            if (h >= G)
-                continue;
-#pragma unroll
-            for (int o = 16; o > 0; o >>= 1) {
-                const float om = __shfl_xor_sync(0xffffffffu, rm[h], o);
-                const float ol = __shfl_xor_sync(0xffffffffu, rl[h], o);
-                const float mm = fmaxf(rm[h], om);
-                if (mm != -INFINITY) {
-                    rl[h] = (rm[h] == -INFINITY ? 0.f : rl[h] * exp2f(rm[h] - mm)) +
-                            (om == -INFINITY ? 0.f : ol * exp2f(om - mm));
-                    rm[h] = mm;
+            for (int n = p0 + tid; n < p1; n += kSelThreads) {
+                const float x = __ldcg(row + n);
+                if (x > m) {
+                    l = (m == -INFINITY ? 0.f : l * exp2f(m - x)) + 1.f;
+                    m = x;
+                } else if (x != -INFINITY) {
+                    l += exp2f(x - m);
                 }
             }
+        }
+        // CTA: max, then the sums rescaled to it
+        const float wm = warp_max(m);
+        float wl = warp_sum(m == -INFINITY ? 0.f : l * exp2f(m - wm));
+        if (lane == 0)
+            red[warp] = make_float2(wm, wl);
+        __syncthreads();
+        if (warp == 0) {
+            const float2 r = lane < kSelThreads / 32 ? red[lane] : make_float2(-INFINITY, 0.f);
+            const float M = warp_max(r.x);
+            const float L = warp_sum(r.x == -INFINITY ? 0.f : r.y * exp2f(r.x - M));
             if (lane == 0)
-                sh.warp_ml[warp][h] = make_float2(rm[h], rl[h]);
+                ws.part[(size_t)(g * G + h) * ws.n_parts + c] = make_float2(M, L);
         }
         __syncthreads();
-        // CTA: one warp per head over the 16 warps' pairs
-        if (warp < G) {
-            const float2 x = lane < kP2Threads / 32 ? sh.warp_ml[lane][warp]
-                                                    : make_float2(-INFINITY, 0.f);
-            float m = x.x;
-#pragma unroll
-            for (int o = 16; o > 0; o >>= 1)
-                m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-            float l = (m == -INFINITY || x.x == -INFINITY) ? 0.f : x.y * exp2f(x.x - m);
-#pragma unroll
-            for (int o = 16; o > 0; o >>= 1)
-                l += __shfl_xor_sync(0xffffffffu, l, o);
-            if (lane == 0)
-                sh.slice_ml[warp] = make_float2(m, l);
-        }
-        cluster.sync();
-        if (warp < G) {
-            float M = -INFINITY;
-            float2 part_r[kClusterCtas];
-#pragma unroll
-            for (int r = 0; r < kClusterCtas; ++r) {
-                part_r[r] = r < n_ranks ? cluster.map_shared_rank(&sh.slice_ml[0], r)[warp]
-                                        : make_float2(-INFINITY, 0.f);
-                M = fmaxf(M, part_r[r].x);
-            }
-            float L = 0.f;
-#pragma unroll
-            for (int r = 0; r < kClusterCtas; ++r)
-                if (part_r[r].x != -INFINITY)
-                    L += part_r[r].y * exp2f(part_r[r].x - M);
-            if (lane == 0) {
-                sh.head_m[warp] = M;
-                sh.head_w[warp] = 1.f / ((float)G * L);
-            }
-        }
-    } else if (warp < G) {
-        const float2 *pp = part + (size_t)(g * G + warp) * n_chunks;
+    }
+}
+
+// Kernel 2: importance of the chunk's positions (group mean of the heads'
+// softmax weights), written out; a histogram of the candidate keys' top 12
+// bits, summed over the head's chunks; the last chunk of a head to finish
+// finds the bin holding the budget-th largest candidate.
+__global__ void __launch_bounds__(kSelThreads, 2)
+sel_keys_kernel(SelectArgs a, SelGeom geo, SelWs ws, const float *__restrict__ s_all, int mode,
+                int vec)
+{
+    __shared__ int hist[kBins0];
+    __shared__ float head_m[kMaxGroup], head_w[kMaxGroup];
+    __shared__ int scan[72];
+    __shared__ int is_last;
+    __shared__ int found[2];
+    const int c = blockIdx.x, g = blockIdx.y;
+    const int G = a.n_heads_q / a.n_heads_kv;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int N = a.n_ctx;
+    const int p0 = min(c * geo.chunk, N), p1 = min(p0 + geo.chunk, N);
+    const bool do_hist = mode == kSelect;
+    for (int b = tid; b < kBins0; b += kSelThreads)
+        hist[b] = 0;
+    if (warp < G) {
+        const float2 *pp = ws.part + (size_t)(g * G + warp) * ws.n_parts;
         float M = -INFINITY;
-        for (int c = lane; c < n_chunks; c += 32)
-            M = fmaxf(M, pp[c].x);
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1)
-            M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+        for (int i = lane; i < ws.n_parts; i += 32)
+            M = fmaxf(M, pp[i].x);
+        M = warp_max(M);
         float L = 0.f;
-        for (int c = lane; c < n_chunks; c += 32)
-            if (pp[c].x != -INFINITY)
-                L += pp[c].y * exp2f(pp[c].x - M);
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1)
-            L += __shfl_xor_sync(0xffffffffu, L, o);
+        for (int i = lane; i < ws.n_parts; i += 32)
+            if (pp[i].x != -INFINITY)
+                L += pp[i].y * exp2f(pp[i].x - M);
+        L = warp_sum(L);
         if (lane == 0) {
-            sh.head_m[warp] = M;
-            sh.head_w[warp] = 1.f / ((float)G * L);
+            head_m[warp] = M;
+            head_w[warp] = 1.f / ((float)G * L);
         }
     }
     __syncthreads();
-
-    const bool do_select = !keep_all && a.budget > 0;
-    // the first radix pass's histogram is built while the keys are formed
-    for (int b = tid; b < kRadixBins; b += kP2Threads)
-        sh.hist[0][b] = 0;
-    __syncthreads();
-    // adds one to the pass's bin of each candidate key (positions >= n_sink)
-    // whose higher digits match `prefix`; lanes with equal bins add once, by
-    // their leader (positive scores share their leading bits, so most lanes
-    // of a warp hit the same bin)
-    auto hist_add = [&](int *hist, bool in, uint32_t key, uint32_t prefix, uint32_t pmask,
-                        int pass) {
-        const bool hit = in && (key & pmask) == prefix;
-        const unsigned act = __ballot_sync(0xffffffffu, hit);
-        if (hit) {
-            const uint32_t bin = (key >> radix_shift(pass)) & radix_mask(pass);
+    float hm[kMaxGroup], hw[kMaxGroup];
+#pragma unroll
+    for (int h = 0; h < kMaxGroup; ++h) {
+        hm[h] = h < G ? head_m[h] : 0.f;
+        hw[h] = h < G ? head_w[h] : 0.f;
+    }
+    // lanes with equal bins add once, by their leader (positive scores
+    // share their leading bits, so many lanes of a warp hit the same bin)
+    auto hist_add = [&](bool in, uint32_t key) {
+        const unsigned act = __ballot_sync(0xffffffffu, in);
+        if (in) {
+            const uint32_t bin = key >> kShift0;
             const unsigned same = __match_any_sync(act, bin);
             if (lane == __ffs(same) - 1)
                 atomicAdd(&hist[bin], __popc(same));
         }
     };
-
-    // scores of this slice -> order-preserving keys in shared memory
-    if ((N & 3) == 0) {
-        // four consecutive positions per thread, one 16-byte load per head
-        // (the slice is a multiple of 4, so p0 and p1 are too); every lane
-        // of a warp runs the same number of rounds
-        // two rounds per step, so that 2 G 16-byte loads are in flight
-        constexpr int kR = 2;
-        const int rounds = (p1 - p0 + 4 * kP2Threads - 1) / (4 * kP2Threads);
-        float hm[kMaxGroup], hw[kMaxGroup];
-#pragma unroll
-        for (int h = 0; h < kMaxGroup; ++h) {
-            hm[h] = h < G ? sh.head_m[h] : 0.f;
-            hw[h] = h < G ? sh.head_w[h] : 0.f;
-        }
+    float *imp = ws.imp + (size_t)g * N;
+    if (vec) {
+        // four positions per thread and round; two CTAs per SM keep enough
+        // loads in flight
+        constexpr int kR = 1;
+        const int rounds = (p1 - p0 + 4 * kSelThreads - 1) / (4 * kSelThreads);
         for (int it0 = 0; it0 < rounds; it0 += kR) {
             float4 sv[kR][kMaxGroup];
 #pragma unroll
             for (int r = 0; r < kR; ++r) {
-                const int nb = p0 + 4 * (tid + (it0 + r) * kP2Threads);
+                const int nb = p0 + 4 * (tid + (it0 + r) * kSelThreads);
 #pragma unroll
                 for (int h = 0; h < kMaxGroup; ++h)
                     if (h < G)
@@ -471,7 +449,7 @@ select_gather_kernel(SelectArgs a, int n_chunks, int slice, const float *__restr
             for (int r = 0; r < kR; ++r) {
                 if (it0 + r >= rounds)
                     break;   // uniform: every lane has the same rounds
-                const int nb = p0 + 4 * (tid + (it0 + r) * kP2Threads);
+                const int nb = p0 + 4 * (tid + (it0 + r) * kSelThreads);
                 const bool live = nb < p1;
                 float sc[4] = {0.f, 0.f, 0.f, 0.f};
                 if (live) {
@@ -483,244 +461,388 @@ select_gather_kernel(SelectArgs a, int n_chunks, int slice, const float *__restr
                             sc[2] += exp2f(sv[r][h].z - hm[h]) * hw[h];
                             sc[3] += exp2f(sv[r][h].w - hm[h]) * hw[h];
                         }
+                    *reinterpret_cast<float4 *>(imp + nb) = make_float4(sc[0], sc[1], sc[2], sc[3]);
                 }
-                uint32_t kk[4];
-#pragma unroll
-                for (int e = 0; e < 4; ++e)
-                    kk[e] = order_key(sc[e]);
-                if (live) {
-                    *reinterpret_cast<uint4 *>(&keys[nb - p0]) =
-                        make_uint4(kk[0], kk[1], kk[2], kk[3]);
-                    if (a.scores_out)
-                        *reinterpret_cast<float4 *>(a.scores_out + (size_t)g * N + nb) =
-                            make_float4(sc[0], sc[1], sc[2], sc[3]);
-                }
-                if (do_select)
+                if (do_hist)
 #pragma unroll
                     for (int e = 0; e < 4; ++e)
-                        hist_add(sh.hist[0], live && nb + e >= a.n_sink, kk[e], 0u, 0u, 0);
+                        hist_add(live && nb + e >= a.n_sink, __float_as_uint(sc[e]));
             }
         }
     } else {
-        // eight positions per thread per step so their loads are in flight together
-        constexpr int kU = 8;
-        const int rounds = (p1 - p0 + kP2Threads * kU - 1) / (kP2Threads * kU);
+        const int rounds = (p1 - p0 + kSelThreads - 1) / kSelThreads;
         for (int it = 0; it < rounds; ++it) {
-            const int nb = p0 + tid + it * kP2Threads * kU;
-            float sc[kU];
-#pragma unroll
-            for (int u = 0; u < kU; ++u)
-                sc[u] = 0.f;
-            for (int h = 0; h < G; ++h) {
-                const float *row = s_all + (size_t)(g * G + h) * N;
-                float sv[kU];
-#pragma unroll
-                for (int u = 0; u < kU; ++u) {
-                    const int n = nb + u * kP2Threads;
-                    sv[u] = n < p1 ? __ldcg(row + n) : 0.f;
-                }
-#pragma unroll
-                for (int u = 0; u < kU; ++u)
-                    sc[u] += exp2f(sv[u] - sh.head_m[h]) * sh.head_w[h];
+            const int n = p0 + tid + it * kSelThreads;
+            float sc = 0.f;
+            if (n < p1) {
+                for (int h = 0; h < G; ++h)
+                    sc += exp2f(__ldcg(s_all + (size_t)(g * G + h) * N + n) - hm[h]) * hw[h];
+                imp[n] = sc;
             }
-#pragma unroll
-            for (int u = 0; u < kU; ++u) {
-                const int n = nb + u * kP2Threads;
-                const uint32_t key = order_key(sc[u]);
-                if (n < p1) {
-                    keys[n - p0] = key;
-                    if (a.scores_out)
-                        a.scores_out[(size_t)g * N + n] = sc[u];
-                }
-                if (do_select)
-                    hist_add(sh.hist[0], n < p1 && n >= a.n_sink, key, 0u, 0u, 0);
-            }
+            if (do_hist)
+                hist_add(n < p1 && n >= a.n_sink, __float_as_uint(sc));
         }
     }
+    if (!do_hist)
+        return;
     __syncthreads();
+    int *ghist = ws.hist + (size_t)g * kBins0;
+    for (int b = tid; b < kBins0; b += kSelThreads)
+        if (hist[b] != 0)
+            atomicAdd(&ghist[b], hist[b]);
+    __threadfence();
+    __syncthreads();
+    if (tid == 0)
+        is_last = atomicAdd(&ws.tick[g], 1) == geo.nc - 1;
+    __syncthreads();
+    if (!is_last)
+        return;
+    __threadfence();
+    // every chunk of this head has added its histogram: the digit is the
+    // bin b with (keys in higher bins) < budget <= (that count + its keys).
+    // Thread t holds bins 4095 - 8t .. 4088 - 8t (descending).
+    int x[8];
+    int sum = 0;
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+        x[k] = __ldcg(&ghist[kBins0 - 1 - (8 * tid + k)]);
+        sum += x[k];
+    }
+    int above;
+    block_exclusive_scan(sum, scan, above);
+    if (tid == 0)
+        found[0] = -1;
+    __syncthreads();
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+        if (above < a.budget && a.budget <= above + x[k]) {
+            found[0] = kBins0 - 1 - (8 * tid + k);
+            found[1] = a.budget - above;
+        }
+        above += x[k];
+    }
+    __syncthreads();
+    if (tid == 0) {
+        ws.info[g].digit0 = found[0];
+        ws.info[g].need0 = found[1];
+        ws.tick[g] = 0;
+    }
+    // the histogram is left zero for the next call
+    for (int b = tid; b < kBins0; b += kSelThreads)
+        ghist[b] = 0;
+}
 
-    // exact radix select of the budget-th largest key over [n_sink, N):
-    // three passes (11, 11, 10 bits), histograms summed over the cluster
-    // through distributed shared memory
-    uint32_t prefix = 0u, pmask = 0u;
-    int need = a.budget;
-    if (do_select) {
-        const int c0 = max(p0, a.n_sink);
-        for (int pass = 0; pass < kRadixPasses; ++pass) {
-            int *hist = sh.hist[pass & 1];
-            if (pass > 0) {
-                // this buffer was last read by other CTAs two passes ago,
-                // before they reached the previous pass's cluster barrier
-                for (int b = tid; b < kRadixBins; b += kP2Threads)
-                    hist[b] = 0;
-                __syncthreads();
-                for (int nb = c0 - (c0 - p0) % 32; nb < p1; nb += kP2Threads) {
-                    const int n = nb + tid;
-                    const bool in = n >= c0 && n < p1;
-                    hist_add(hist, in, in ? keys[n - p0] : 0u, prefix, pmask, pass);
-                }
+// Kernel 3: per chunk, the candidate keys above the threshold bin are
+// counted and those in it are appended (key, position) to the head's list.
+__global__ void __launch_bounds__(kSelThreads)
+sel_cand_kernel(SelectArgs a, SelGeom geo, SelWs ws)
+{
+    __shared__ int red[kSelThreads / 32];
+    const int c = blockIdx.x, g = blockIdx.y;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int N = a.n_ctx;
+    const int p0 = min(c * geo.chunk, N), p1 = min(p0 + geo.chunk, N);
+    const int digit0 = __ldcg(&ws.info[g].digit0);
+    const float *imp = ws.imp + (size_t)g * N;
+    uint2 *cand = ws.cand + (size_t)g * N;
+    int n_above = 0;
+    const int rounds = (p1 - p0 + kSelThreads - 1) / kSelThreads;
+    for (int it = 0; it < rounds; ++it) {
+        const int n = p0 + tid + it * kSelThreads;
+        const bool in = n < p1 && n >= a.n_sink;
+        const uint32_t key = in ? __float_as_uint(__ldcg(imp + n)) : 0u;
+        const int bin = (int)(key >> kShift0);
+        n_above += in && bin > digit0;
+        const bool hit = in && bin == digit0;
+        const unsigned m = __ballot_sync(0xffffffffu, hit);
+        if (m) {
+            int base = 0;
+            if (lane == 0)
+                base = atomicAdd(&ws.info[g].n_cand, __popc(m));
+            base = __shfl_sync(0xffffffffu, base, 0);
+            if (hit)
+                cand[base + __popc(m & ((1u << lane) - 1u))] = make_uint2(key, (uint32_t)n);
+        }
+    }
+    n_above = warp_isum(n_above);
+    if (lane == 0)
+        red[warp] = n_above;
+    __syncthreads();
+    if (warp == 0) {
+        int v = lane < kSelThreads / 32 ? red[lane] : 0;
+        v = warp_isum(v);
+        if (lane == 0)
+            ws.above[(size_t)g * geo.nc + c] = v;
+    }
+}
+
+// Kernel 4, one CTA per KV head: the exact budget-th largest key among the
+// candidates (two radix passes over their low 19 bits), then per chunk the
+// number of kept positions before it and of equal-to-threshold keys before
+// it, so that each chunk can place its kept positions on its own.
+__global__ void __launch_bounds__(kSelThreads)
+sel_thresh_kernel(SelectArgs a, SelGeom geo, SelWs ws, int mode)
+{
+    __shared__ int hist[1024];
+    __shared__ int scan[72];
+    __shared__ int found[2];
+    __shared__ int gtc[kMaxChunks], eqc[kMaxChunks];
+    const int g = blockIdx.x;
+    const int tid = threadIdx.x;
+    const int N = a.n_ctx;
+    SelInfo *inf = &ws.info[g];
+    uint32_t T = 0xFFFFFFFFu;   // nothing at or above: no candidate kept
+    int need_eq = 0;
+    int n_cand = 0;
+    if (mode == kSelect) {
+        n_cand = __ldcg(&inf->n_cand);
+        const int digit0 = __ldcg(&inf->digit0);
+        int need = __ldcg(&inf->need0);
+        const uint2 *cand = ws.cand + (size_t)g * N;
+        uint32_t prefix = (uint32_t)digit0 << kShift0;
+        uint32_t pmask = 0xFFFFFFFFu << kShift0;
+        for (int pass = 0; pass < 2; ++pass) {
+            const int shift = pass == 0 ? 9 : 0;
+            const int nb = pass == 0 ? 1024 : 512;
+            const uint32_t dmask = (uint32_t)nb - 1;
+            for (int b = tid; b < 1024; b += kSelThreads)
+                hist[b] = 0;
+            __syncthreads();
+            for (int i = tid; i < n_cand; i += kSelThreads) {
+                const uint32_t key = __ldcg(&cand[i].x);
+                if ((key & pmask) == prefix)
+                    atomicAdd(&hist[(key >> shift) & dmask], 1);
             }
-            cluster.sync();
-            // thread t looks at bins 4t .. 4t + 3 from the top (bin
-            // 2047 - 4t - k): an exclusive scan over t counts the keys in
-            // higher bins; the digit is the bin with (keys above it) < need
-            // <= (that count + its own keys)
-            const int nbins = (int)radix_mask(pass) + 1;
-            int x[4] = {0, 0, 0, 0};
-            if (4 * tid < nbins) {
-                // bins nbins-4-4t .. nbins-1-4t: one 16-byte read per rank,
-                // all ranks' reads in flight together
-                const int q = (nbins - 4 - 4 * tid) / 4;
-                int4 v[kClusterCtas];
-#pragma unroll
-                for (int r = 0; r < kClusterCtas; ++r)
-                    v[r] = r < n_ranks
-                               ? reinterpret_cast<const int4 *>(cluster.map_shared_rank(hist, r))[q]
-                               : make_int4(0, 0, 0, 0);
-#pragma unroll
-                for (int r = 0; r < kClusterCtas; ++r) {
-                    x[0] += v[r].w;
-                    x[1] += v[r].z;
-                    x[2] += v[r].y;
-                    x[3] += v[r].x;
-                }
+            __syncthreads();
+            // thread t holds bins nb-1-2t, nb-2-2t (descending)
+            int x0 = 0, x1 = 0;
+            if (2 * tid < nb) {
+                x0 = hist[nb - 1 - 2 * tid];
+                x1 = hist[nb - 2 - 2 * tid];
             }
             int above;
-            block_exclusive_scan(x[0] + x[1] + x[2] + x[3], sh.scan, above);
-#pragma unroll
-            for (int k = 0; k < 4; ++k) {
-                const int b = nbins - 1 - (4 * tid + k);
-                if (b >= 0 && above < need && need <= above + x[k]) {
-                    sh.bcast[0] = b;
-                    sh.bcast[1] = above;
+            block_exclusive_scan(x0 + x1, scan, above);
+            if (2 * tid < nb) {
+                if (above < need && need <= above + x0) {
+                    found[0] = nb - 1 - 2 * tid;
+                    found[1] = above;
+                } else if (above + x0 < need && need <= above + x0 + x1) {
+                    found[0] = nb - 2 - 2 * tid;
+                    found[1] = above + x0;
                 }
-                above += x[k];
             }
-            __syncthreads();   // the digit is in bcast
-            const int d = sh.bcast[0];
-            need -= sh.bcast[1];
-            prefix |= (uint32_t)d << radix_shift(pass);
-            pmask |= radix_mask(pass) << radix_shift(pass);
+            __syncthreads();
+            prefix |= (uint32_t)found[0] << shift;
+            pmask |= dmask << shift;
+            need -= found[1];
             __syncthreads();
         }
+        T = prefix;
+        need_eq = need;
     }
-    // prefix is now the threshold key; `need` keys equal to it are kept
-
-    // positions of this slice: how many equal the threshold (candidates only)
-    const int per_thread = (p1 - p0 + kP2Threads - 1) / kP2Threads;
-    const int q0 = p0 + tid * per_thread, q1 = min(q0 + per_thread, p1);
-    int my_eq = 0;
-    if (do_select)
-        for (int n = max(q0, a.n_sink); n < q1; ++n)
-            my_eq += keys[n - p0] == prefix;
-    int eq_excl;
-    const int eq_total = block_exclusive_scan(my_eq, sh.scan, eq_excl);
-    if (tid == 0)
-        sh.counts[0] = eq_total;
-    cluster.sync();
-    int eq_before = 0;
-    for (int r = 0; r < rank; ++r)
-        eq_before += *cluster.map_shared_rank(&sh.counts[0], r);
-
-    // kept flags -> counts -> ascending slots
-    auto kept = [&](int n, int &eq_rank) -> bool {
-        if (keep_all || n < a.n_sink)
-            return true;
-        if (!do_select)
-            return false;
-        const uint32_t key = keys[n - p0];
-        if (key > prefix)
-            return true;
-        if (key == prefix)
-            return eq_rank++ < need;
-        return false;
-    };
-    int my_kept = 0;
-    {
-        int eq_rank = eq_before + eq_excl;
-        for (int n = q0; n < q1; ++n)
-            my_kept += kept(n, eq_rank);
-    }
-    int kept_excl;
-    const int kept_total = block_exclusive_scan(my_kept, sh.scan, kept_excl);
-    if (tid == 0)
-        sh.counts[1] = kept_total;
-    cluster.sync();
-    int kept_before = 0;
-    for (int r = 0; r < rank; ++r)
-        kept_before += *cluster.map_shared_rank(&sh.counts[1], r);
-    cluster.sync();   // no CTA may exit while others read its shared memory
-
-    // write indices; reuse the key slots of kept positions to list them
-    int32_t *idx = a.idx_out + (size_t)g * n_keep;
-    {
-        int eq_rank = eq_before + eq_excl;
-        int slot = kept_before + kept_excl;
-        for (int n = q0; n < q1; ++n)
-            if (kept(n, eq_rank)) {
-                if (slot < n_keep)
-                    idx[slot] = n;
-                else
-                    record_status(reinterpret_cast<WorkspaceHeader *>(a.workspace),
-                                  TS_ERR_DEVICE_ARG);
-                ++slot;
-            }
+    // per chunk: candidates above T and equal to T
+    for (int i = tid; i < geo.nc; i += kSelThreads) {
+        gtc[i] = 0;
+        eqc[i] = 0;
     }
     __syncthreads();
+    if (mode == kSelect) {
+        const uint2 *cand = ws.cand + (size_t)g * N;
+        for (int i = tid; i < n_cand; i += kSelThreads) {
+            const uint2 kp = __ldcg(&cand[i]);
+            const int ch = (int)kp.y / geo.chunk;
+            if (kp.x > T)
+                atomicAdd(&gtc[ch], 1);
+            else if (kp.x == T)
+                atomicAdd(&eqc[ch], 1);
+        }
+    }
+    __syncthreads();
+    // kept before chunk c: sinks before it, keys above T before it, and of
+    // the equal keys the first need_eq in position order.  One chunk per
+    // thread (nc <= kMaxChunks <= kSelThreads): scan the equal counts, then
+    // the kept counts.
+    const int ch = tid;
+    const bool live = ch < geo.nc;
+    const int my_eq = live && mode == kSelect ? eqc[ch] : 0;
+    int eq_before;
+    block_exclusive_scan(my_eq, scan, eq_before);
+    int k = 0;
+    if (live) {
+        const int q0 = ch * geo.chunk, q1 = min(q0 + geo.chunk, N);
+        if (mode == kKeepAll) {
+            k = max(0, q1 - q0);
+        } else {
+            k = max(0, min(q1, a.n_sink) - q0);
+            if (mode == kSelect)
+                k += __ldcg(&ws.above[(size_t)g * geo.nc + ch]) + gtc[ch] +
+                     max(0, min(need_eq - eq_before, eqc[ch]));
+        }
+    }
+    int kept_before;
+    block_exclusive_scan(k, scan, kept_before);
+    if (live)
+        ws.chunk[(size_t)g * geo.nc + ch] = make_int2(kept_before, eq_before);
+    if (tid == 0) {
+        inf->T = T;
+        inf->need_eq = need_eq;
+        inf->n_cand = 0;   // the list is empty again for the next call
+    }
+}
 
-    // gather: kept rows of this slice are idx[kept_before .. kept_before + kept_total)
+// Kernel 5: each chunk writes its kept positions in ascending order from
+// its offset and copies their K and V rows into the partial cache.
+template <int D>
+__global__ void __launch_bounds__(kSelThreads)
+sel_gather_kernel(SelectArgs a, SelGeom geo, SelWs ws, int mode)
+{
+    extern __shared__ int list[];   // this chunk's kept positions
+    __shared__ int scan[72];
+    const int c = blockIdx.x, g = blockIdx.y;
+    const int tid = threadIdx.x;
+    const int N = a.n_ctx;
+    const int p0 = min(c * geo.chunk, N), p1 = min(p0 + geo.chunk, N);
+    const int2 ci = __ldcg(&ws.chunk[(size_t)g * geo.nc + c]);
+    const uint32_t T = __ldcg(&ws.info[g].T);
+    const int need_eq = __ldcg(&ws.info[g].need_eq);
+    const float *imp = ws.imp + (size_t)g * N;
+    const int64_t want = (int64_t)a.n_sink + a.budget;
+    const int n_keep = want < N ? (int)want : N;
+    // each thread a contiguous run of the chunk
+    const int per = (p1 - p0 + kSelThreads - 1) / kSelThreads;
+    const int q0 = p0 + tid * per, q1 = min(q0 + per, p1);
+    auto cls = [&](int n) -> int {   // 0 dropped, 1 kept, 2 equal to T
+        if (mode == kKeepAll || n < a.n_sink)
+            return 1;
+        if (mode != kSelect)
+            return 0;
+        const uint32_t key = __float_as_uint(__ldcg(imp + n));
+        return key > T ? 1 : (key == T ? 2 : 0);
+    };
+    int n_sure = 0, n_eq = 0;
+    for (int n = q0; n < q1; ++n) {
+        const int k = cls(n);
+        n_sure += k == 1;
+        n_eq += k == 2;
+    }
+    int sure_before, eq_before;
+    block_exclusive_scan(n_sure, scan, sure_before);
+    block_exclusive_scan(n_eq, scan, eq_before);
+    // equal keys are kept in position order: the first need_eq of the head
+    const int eqb = ci.y + eq_before;
+    int slot = sure_before + max(0, min(need_eq, eqb)) - max(0, min(need_eq, ci.y));
+    int eq_rank = eqb;
+    int32_t *idx = a.idx_out + (size_t)g * n_keep;
+    for (int n = q0; n < q1; ++n) {
+        const int k = cls(n);
+        const bool kept = k == 1 || (k == 2 && eq_rank++ < need_eq);
+        if (kept) {
+            const int out = ci.x + slot;
+            if (out < n_keep) {
+                idx[out] = n;
+                list[slot] = n;
+            } else {
+                record_status(reinterpret_cast<WorkspaceHeader *>(a.workspace), TS_ERR_DEVICE_ARG);
+            }
+            ++slot;
+        }
+    }
+    __syncthreads();
+    // rows: the chunk's kept count is the last thread's end slot
+    __shared__ int n_rows;
+    if (tid == kSelThreads - 1)
+        n_rows = min(slot, n_keep - ci.x);
+    __syncthreads();
+    const int rows = n_rows;
     constexpr int LPR = D / 8;   // lanes per row, 16 bytes each
     const __nv_bfloat16 *kh = a.k + (int64_t)g * a.kv_cap * D;
     const __nv_bfloat16 *vh = a.v + (int64_t)g * a.kv_cap * D;
     __nv_bfloat16 *kp = a.k_partial + (int64_t)g * a.partial_cap * D;
     __nv_bfloat16 *vp = a.v_partial + (int64_t)g * a.partial_cap * D;
-    const int rows_per_pass = kP2Threads / LPR;
+    const int rows_per_pass = kSelThreads / LPR;
     const int li = tid % LPR;
-    __threadfence_block();
-    const int my_rows = min(kept_total, n_keep - kept_before);
-    // eight rows per thread per step: their K and V loads are in flight together
-    constexpr int kG = 8;
-    for (int t0 = tid / LPR; t0 < my_rows; t0 += rows_per_pass * kG) {
+    constexpr int kG = 8;   // rows per thread per step, loads in flight together
+    for (int t0 = tid / LPR; t0 < rows; t0 += rows_per_pass * kG) {
         uint4 kv[kG], vv[kG];
-        int slot[kG];
-        bool ok[kG];
+        int nn[kG];
 #pragma unroll
         for (int u = 0; u < kG; ++u) {
             const int t = t0 + u * rows_per_pass;
-            slot[u] = kept_before + t;
-            const int n = t < my_rows ? __ldcg(&idx[slot[u]]) : -1;
-            ok[u] = n >= 0 && n < N;
-            const int nn = ok[u] ? n : 0;
-            kv[u] = *reinterpret_cast<const uint4 *>(kh + (int64_t)nn * D + li * 8);
-            vv[u] = *reinterpret_cast<const uint4 *>(vh + (int64_t)nn * D + li * 8);
+            nn[u] = t < rows ? list[t] : -1;
+            const int r = nn[u] >= 0 ? nn[u] : 0;
+            kv[u] = *reinterpret_cast<const uint4 *>(kh + (int64_t)r * D + li * 8);
+            vv[u] = *reinterpret_cast<const uint4 *>(vh + (int64_t)r * D + li * 8);
         }
 #pragma unroll
-        for (int u = 0; u < kG; ++u)
-            if (ok[u]) {
-                *reinterpret_cast<uint4 *>(kp + (int64_t)slot[u] * D + li * 8) = kv[u];
-                *reinterpret_cast<uint4 *>(vp + (int64_t)slot[u] * D + li * 8) = vv[u];
+        for (int u = 0; u < kG; ++u) {
+            const int t = t0 + u * rows_per_pass;
+            if (nn[u] >= 0) {
+                *reinterpret_cast<uint4 *>(kp + (int64_t)(ci.x + t) * D + li * 8) = kv[u];
+                *reinterpret_cast<uint4 *>(vp + (int64_t)(ci.x + t) * D + li * 8) = vv[u];
             }
+        }
     }
 }
 
+// --------------------------------------------------------------------- host
 struct SelPlan {
-    int chunk, n_chunks, slice;
+    int p1_chunk, p1_chunks;   // the score pass's chunks (its partials)
+    SelGeom geo;               // the selection's chunks
 };
 
 SelPlan make_sel_plan(int n_heads_kv, int n_ctx, int num_sms)
 {
     SelPlan p;
-    // three 64 KB-ring CTAs fit an SM: one wave of them over all heads
-    // (rounded down, so that no CTA waits for a second wave)
+    // score pass: three 64 KB-ring CTAs fit an SM, one wave over all heads
     int want = (num_sms * 3) / n_heads_kv;
     want = want < 1 ? 1 : want;
-    const int min_chunk = 512;
     int chunk = (n_ctx + want - 1) / want;
-    chunk = chunk < min_chunk ? min_chunk : chunk;
-    p.chunk = chunk;
-    p.n_chunks = (n_ctx + chunk - 1) / chunk;
-    p.slice = ((n_ctx + kClusterCtas - 1) / kClusterCtas + 3) / 4 * 4;
+    chunk = chunk < 512 ? 512 : chunk;
+    p.p1_chunk = chunk;
+    p.p1_chunks = (n_ctx + chunk - 1) / chunk;
+    // selection: about two CTAs per SM over all heads, chunks of at least
+    // 1024 positions, a multiple of 4, at most kMaxChunks per head
+    int nc = (2 * num_sms) / n_heads_kv;
+    nc = nc < 1 ? 1 : nc;
+    const int max_nc = (n_ctx + 1023) / 1024;
+    nc = nc > max_nc ? max_nc : nc;
+    const int min_nc = (n_ctx + kMaxChunkLen - 1) / kMaxChunkLen;
+    nc = nc < min_nc ? min_nc : nc;
+    nc = nc > kMaxChunks ? kMaxChunks : nc;
+    int sc = ((n_ctx + nc - 1) / nc + 3) / 4 * 4;
+    p.geo.chunk = sc;
+    p.geo.nc = (n_ctx + sc - 1) / sc;
     return p;
+}
+
+// Workspace: header, [score pass: s fp32 [Hq, n_ctx]], partials, importance,
+// histogram, tickets, info, per-chunk counts, candidates.
+struct SelOffsets {
+    size_t s, part, imp, hist, tick, info, above, chunk, cand, total;
+};
+
+SelOffsets sel_offsets(int n_heads_q, int n_heads_kv, int n_ctx, const SelPlan &p,
+                       bool score_pass)
+{
+    SelOffsets o;
+    size_t at = kHeaderBytes;
+    auto take = [&](size_t bytes) {
+        const size_t r = at;
+        at = align_up(at + bytes, 256);
+        return r;
+    };
+    const int n_parts = score_pass ? p.p1_chunks : p.geo.nc;
+    o.s = take(score_pass ? (size_t)n_heads_q * n_ctx * sizeof(float) : 0);
+    o.part = take((size_t)n_heads_q * n_parts * sizeof(float2));
+    o.imp = take((size_t)n_heads_kv * n_ctx * sizeof(float));
+    o.hist = take((size_t)n_heads_kv * kBins0 * sizeof(int));
+    o.tick = take((size_t)n_heads_kv * sizeof(int));
+    o.info = take((size_t)n_heads_kv * sizeof(SelInfo));
+    o.above = take((size_t)n_heads_kv * p.geo.nc * sizeof(int));
+    o.chunk = take((size_t)n_heads_kv * p.geo.nc * sizeof(int2));
+    o.cand = take((size_t)n_heads_kv * n_ctx * sizeof(uint2));
+    o.total = at;
+    return o;
 }
 
 template <int D>
@@ -735,9 +857,9 @@ cudaError_t launch_p1(const SelectArgs &a, const SelPlan &p, float *s_out, float
         score_logits_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (attr != cudaSuccess)
         return attr;
-    dim3 grid(p.n_chunks, a.n_heads_kv);
-    score_logits_kernel<D><<<grid, kP1Threads, smem, stream>>>(mk, a, p.chunk, p.n_chunks, s_out,
-                                                                part_out);
+    dim3 grid(p.p1_chunks, a.n_heads_kv);
+    score_logits_kernel<D><<<grid, kP1Threads, smem, stream>>>(mk, a, p.p1_chunk, p.p1_chunks,
+                                                                s_out, part_out);
     const cudaError_t e = cudaGetLastError();
     if (e == cudaSuccess)
         count_launches(1);
@@ -747,41 +869,66 @@ cudaError_t launch_p1(const SelectArgs &a, const SelPlan &p, float *s_out, float
 template <int D>
 cudaError_t launch_d(const SelectArgs &a, const SelPlan &p, cudaStream_t stream)
 {
-    // scores from the caller, or the score pass into the workspace
+    const bool score_pass = a.root_scores == nullptr;
+    const SelOffsets o = sel_offsets(a.n_heads_q, a.n_heads_kv, a.n_ctx, p, score_pass);
+    char *w = reinterpret_cast<char *>(a.workspace);
+    SelWs ws;
+    ws.part = reinterpret_cast<float2 *>(w + o.part);
+    ws.n_parts = score_pass ? p.p1_chunks : p.geo.nc;
+    ws.imp = a.scores_out ? a.scores_out : reinterpret_cast<float *>(w + o.imp);
+    ws.hist = reinterpret_cast<int *>(w + o.hist);
+    ws.tick = reinterpret_cast<int *>(w + o.tick);
+    ws.info = reinterpret_cast<SelInfo *>(w + o.info);
+    ws.above = reinterpret_cast<int *>(w + o.above);
+    ws.chunk = reinterpret_cast<int2 *>(w + o.chunk);
+    ws.cand = reinterpret_cast<uint2 *>(w + o.cand);
+    const int64_t want = (int64_t)a.n_sink + a.budget;
+    const int mode = want >= a.n_ctx ? kKeepAll : (a.budget == 0 ? kSinksOnly : kSelect);
+    const dim3 grid(p.geo.nc, a.n_heads_kv);
+
+    // scores: the caller's (then their per-chunk statistics here), or the
+    // score pass into the workspace (which leaves the statistics itself)
     const float *s_all = a.root_scores;
-    cudaError_t e = cudaSuccess;
-    if (s_all == nullptr) {
-        float *s_ws =
-            reinterpret_cast<float *>(reinterpret_cast<char *>(a.workspace) + kHeaderBytes);
-        e = launch_p1<D>(a, p, s_ws, reinterpret_cast<float2 *>(s_ws + (size_t)a.n_heads_q * a.n_ctx),
-                         stream);
+    cudaError_t e;
+    if (score_pass) {
+        float *s_ws = reinterpret_cast<float *>(w + o.s);
+        e = launch_p1<D>(a, p, s_ws, ws.part, stream);
         if (e != cudaSuccess)
             return e;
         s_all = s_ws;
-    }
-
-    const size_t smem = sizeof(P2Shared) + (size_t)p.slice * sizeof(uint32_t);
-    static const cudaError_t attr_ok = cudaFuncSetAttribute(
-        select_gather_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-        (int)(sizeof(P2Shared) + (size_t)kMaxSlice * sizeof(uint32_t)));
-    if (attr_ok != cudaSuccess)
-        return attr_ok;
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(kClusterCtas, a.n_heads_kv, 1);
-    cfg.blockDim = dim3(kP2Threads, 1, 1);
-    cfg.dynamicSmemBytes = smem;
-    cfg.stream = stream;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = kClusterCtas;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    e = cudaLaunchKernelEx(&cfg, select_gather_kernel<D>, a, p.n_chunks, p.slice, s_all);
-    if (e == cudaSuccess)
+    } else {
+        sel_stats_kernel<<<grid, kSelThreads, 0, stream>>>(a, p.geo, ws);
+        if ((e = cudaGetLastError()) != cudaSuccess)
+            return e;
         count_launches(1);
-    return e;
+    }
+    // 16-byte loads and stores when every row starts on a 16-byte boundary
+    const int vec = (a.n_ctx & 3) == 0 && reinterpret_cast<uintptr_t>(s_all) % 16 == 0 &&
+                    reinterpret_cast<uintptr_t>(ws.imp) % 16 == 0;
+    sel_keys_kernel<<<grid, kSelThreads, 0, stream>>>(a, p.geo, ws, s_all, mode, vec);
+    if ((e = cudaGetLastError()) != cudaSuccess)
+        return e;
+    count_launches(1);
+    if (mode == kSelect) {
+        sel_cand_kernel<<<grid, kSelThreads, 0, stream>>>(a, p.geo, ws);
+        if ((e = cudaGetLastError()) != cudaSuccess)
+            return e;
+        count_launches(1);
+    }
+    sel_thresh_kernel<<<a.n_heads_kv, kSelThreads, 0, stream>>>(a, p.geo, ws, mode);
+    if ((e = cudaGetLastError()) != cudaSuccess)
+        return e;
+    count_launches(1);
+    const size_t list_bytes = (size_t)p.geo.chunk * sizeof(int);
+    static const cudaError_t attr = cudaFuncSetAttribute(
+        sel_gather_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
+    if (attr != cudaSuccess)
+        return attr;
+    sel_gather_kernel<D><<<grid, kSelThreads, list_bytes, stream>>>(a, p.geo, ws, mode);
+    if ((e = cudaGetLastError()) != cudaSuccess)
+        return e;
+    count_launches(1);
+    return cudaSuccess;
 }
 
 }  // namespace
@@ -801,7 +948,9 @@ int select_supported(int n_heads_q, int n_heads_kv, int head_dim, int n_ctx)
         return 0;
     if (head_dim == 64 && G > 8)
         return 0;
-    return ((n_ctx + kClusterCtas - 1) / kClusterCtas + 3) / 4 * 4 <= kMaxSlice;
+    // a chunk's kept positions are listed in shared memory
+    const SelPlan p = make_sel_plan(n_heads_kv, n_ctx, 148);
+    return p.geo.chunk <= kMaxChunkLen;
 }
 
 size_t select_workspace_bytes(int n_heads_q, int n_heads_kv, int head_dim, int n_ctx,
@@ -809,9 +958,13 @@ size_t select_workspace_bytes(int n_heads_q, int n_heads_kv, int head_dim, int n
 {
     (void)head_dim;
     const SelPlan p = make_sel_plan(n_heads_kv, n_ctx, num_sms);
-    const size_t s_bytes = (size_t)n_heads_q * n_ctx * sizeof(float);
-    const size_t part = (size_t)n_heads_q * p.n_chunks * 2 * sizeof(float);
-    return kHeaderBytes + align_up(s_bytes + part, 256);
+    return sel_offsets(n_heads_q, n_heads_kv, n_ctx, p, true).total;
+}
+
+size_t select_from_scores_workspace_bytes(int n_heads_q, int n_heads_kv, int n_ctx, int num_sms)
+{
+    const SelPlan p = make_sel_plan(n_heads_kv, n_ctx, num_sms);
+    return sel_offsets(n_heads_q, n_heads_kv, n_ctx, p, false).total;
 }
 
 cudaError_t select_launch(const SelectArgs &a, int num_sms, cudaStream_t stream)

@@ -133,6 +133,33 @@ __device__ __forceinline__ void bulk_store(void *dst, uint32_t src, uint32_t byt
                  : "memory");
 }
 
+// Programmatic dependent launch: let the grid launched after this one (with
+// the programmatic-serialization attribute) be scheduled now; it waits in
+// grid_dependency_wait() until this grid has completed.
+__device__ __forceinline__ void launch_dependents()
+{
+    asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory");
+}
+
+// Wait until the grids this one depends on have completed and their memory
+// is visible (returns at once for a launch without the attribute).
+__device__ __forceinline__ void grid_dependency_wait()
+{
+    asm volatile("griddepcontrol.wait;\n" ::: "memory");
+}
+
+// Named barrier `id` (1..15) over `threads` threads (a multiple of 32).
+__device__ __forceinline__ void named_bar_sync(int id, int threads)
+{
+    asm volatile("bar.sync %0, %1;\n" ::"r"(id), "r"(threads) : "memory");
+}
+
+// Arrival (no wait) at named barrier `id` counted over `threads` threads.
+__device__ __forceinline__ void named_bar_arrive(int id, int threads)
+{
+    asm volatile("bar.arrive %0, %1;\n" ::"r"(id), "r"(threads) : "memory");
+}
+
 __device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;\n" ::: "memory"); }
 
 // until at most N of this thread's bulk groups still read shared memory

@@ -237,7 +237,12 @@ int ts_kv_importance_select(const void *q_last, const void *k_cache, const void 
     return e == cudaSuccess ? TS_OK : TS_ERR_CUDA;
 }
 
-size_t ts_kv_select_from_scores_workspace_size(void) { return ts::kHeaderBytes; }
+size_t ts_kv_select_from_scores_workspace_size(int n_heads_q, int n_heads_kv, int n_ctx)
+{
+    if (!shape_ok(n_heads_q, n_heads_kv, 64) || n_ctx < 1)
+        return 0;
+    return ts::select_from_scores_workspace_bytes(n_heads_q, n_heads_kv, n_ctx, current_num_sms());
+}
 
 int ts_kv_select_from_scores(const float *root_scores, const void *k_cache, const void *v_cache,
                              int64_t kv_cap, int n_heads_q, int n_heads_kv, int head_dim,
@@ -265,7 +270,9 @@ int ts_kv_select_from_scores(const float *root_scores, const void *k_cache, cons
         return TS_ERR_INVALID_ARG;
     if (!head_dim_supported(head_dim) || !ts::select_supported(n_heads_q, n_heads_kv, head_dim, n_ctx))
         return TS_ERR_UNSUPPORTED;
-    if (!workspace_ok(workspace, workspace_bytes, ts::kHeaderBytes))
+    const int sms = current_num_sms();
+    if (!workspace_ok(workspace, workspace_bytes,
+                      ts::select_from_scores_workspace_bytes(n_heads_q, n_heads_kv, n_ctx, sms)))
         return TS_ERR_WORKSPACE;
 
     ts::SelectArgs a = {};
@@ -286,8 +293,7 @@ int ts_kv_select_from_scores(const float *root_scores, const void *k_cache, cons
     a.workspace = workspace;
     a.workspace_bytes = workspace_bytes;
     a.root_scores = root_scores;
-    const cudaError_t e =
-        ts::select_launch(a, current_num_sms(), static_cast<cudaStream_t>(stream));
+    const cudaError_t e = ts::select_launch(a, sms, static_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? TS_OK : TS_ERR_CUDA;
 }
 

@@ -92,6 +92,7 @@ struct SelectArgs {
 
 size_t select_workspace_bytes(int n_heads_q, int n_heads_kv, int head_dim, int n_ctx,
                               int num_sms);
+size_t select_from_scores_workspace_bytes(int n_heads_q, int n_heads_kv, int n_ctx, int num_sms);
 int select_supported(int n_heads_q, int n_heads_kv, int head_dim, int n_ctx);
 cudaError_t select_launch(const SelectArgs &a, int num_sms, cudaStream_t stream);
 // The score pass alone: base-2 root scores fp32 [Hq, n_ctx] into `out`.

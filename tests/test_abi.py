@@ -168,9 +168,9 @@ def test_select_from_scores_rejects_on_host(lib, over, code):
 def test_select_from_scores_accepts_4_byte_rows_for_ragged_contexts(lib):
     # n_ctx not a multiple of 4: scores need only 4-byte alignment, so the
     # call passes every host check; it is not launched here (the workspace
-    # is one byte short of the header, the last check)
+    # is one byte short of its size, the last check)
     import lossless_ultra_long_b200 as L
-    need = L.kv_select_from_scores_workspace_size()
+    need = L.kv_select_from_scores_workspace_size(8, 2, 999)
     assert need > 0
     assert _from_scores_call(lib, rs=(1 << 20) + 4, n_ctx=999, ws_bytes=need - 1) == 3
 
