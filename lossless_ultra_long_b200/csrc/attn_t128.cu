@@ -984,16 +984,42 @@ attn_t128_combine_kernel(AttnArgs a, TreeMasks masks, int n_split, int split_pos
         return __ldcg(reinterpret_cast<const float4 *>(ws_ml + ((size_t)s * rows_all + row) * 4));
     };
 
-    // pass 1 over the (m, l, q) of every split: M, and L and the bound's
-    // denominator over the splits that are not flagged
+    // One round trip for the common case (at most kFastSplits splits): lane
+    // s reads split s's (m, l, q) and flag while every lane also reads its
+    // four columns of every split's acc, all loads in flight together.
+    auto flagged = [&](int s) { return flags != nullptr && flags[s * a.n_heads_kv + g] != 0; };
+    constexpr int kFastSplits = 24;
+    const bool fast = n_split <= kFastSplits;
+    float4 xs[kFastSplits];
+    float4 my = make_float4(-INFINITY, 0.f, 0.f, 0.f);
+    bool my_f = false;
+    if (fast) {
+        if (lane < n_split) {
+            my = mlq_of(lane);
+            my_f = flagged(lane);
+        }
+#pragma unroll
+        for (int u = 0; u < kFastSplits; ++u)
+            xs[u] = u < n_split ? __ldcg(reinterpret_cast<const float4 *>(
+                                      ws_o + ((size_t)u * rows_all + row) * kD + 4 * lane))
+                                : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+
+    // M, and L and the bound's denominator, over the splits that are not
+    // flagged
     bool any = false;
     float M = -INFINITY;
-    auto flagged = [&](int s) { return flags != nullptr && flags[s * a.n_heads_kv + g] != 0; };
-    for (int s = lane; s < n_split; s += 32) {
-        const bool f = flagged(s);
-        any |= f;
-        if (!f)
-            M = fmaxf(M, mlq_of(s).x);
+    if (fast) {
+        any = my_f;
+        if (!my_f)
+            M = my.x;
+    } else {
+        for (int s = lane; s < n_split; s += 32) {
+            const bool f = flagged(s);
+            any |= f;
+            if (!f)
+                M = fmaxf(M, mlq_of(s).x);
+        }
     }
     any = __any_sync(0xffffffffu, any);
 #pragma unroll
@@ -1003,13 +1029,21 @@ attn_t128_combine_kernel(AttnArgs a, TreeMasks masks, int n_split, int split_pos
     // formed in fp64
     double Lp = 0.0, Qp = 0.0;
     if (M != -INFINITY) {
-        for (int s = lane; s < n_split; s += 32) {
-            if (flagged(s))
-                continue;
-            const float4 x = mlq_of(s);
-            const double c = x.x == -INFINITY ? 0.0 : (double)exp2f(x.x - M);
-            Lp += c * (double)x.y;
-            Qp += c * c * (double)x.z;
+        if (fast) {
+            if (!my_f && my.x != -INFINITY) {
+                const double c = (double)exp2f(my.x - M);
+                Lp = c * (double)my.y;
+                Qp = c * c * (double)my.z;
+            }
+        } else {
+            for (int s = lane; s < n_split; s += 32) {
+                if (flagged(s))
+                    continue;
+                const float4 x = mlq_of(s);
+                const double c = x.x == -INFINITY ? 0.0 : (double)exp2f(x.x - M);
+                Lp += c * (double)x.y;
+                Qp += c * c * (double)x.z;
+            }
         }
     }
 #pragma unroll
@@ -1022,7 +1056,23 @@ attn_t128_combine_kernel(AttnArgs a, TreeMasks masks, int n_split, int split_pos
 
     float acc[4] = {0.f, 0.f, 0.f, 0.f};
     float L = 0.f;
-    if (!any && !peaked) {
+    if (!any && !peaked && fast) {
+        // every partial is used as it is: lane s's weight 2^(m_s - M) and
+        // its weighted l, passed to every lane
+        const float w_my = my.x == -INFINITY ? 0.f : exp2f(my.x - M);
+        const float wl_my = w_my * my.y;
+#pragma unroll
+        for (int u = 0; u < kFastSplits; ++u) {
+            if (u >= n_split)
+                break;
+            const float w = __shfl_sync(0xffffffffu, w_my, u);
+            L += __shfl_sync(0xffffffffu, wl_my, u);
+            acc[0] += w * xs[u].x;
+            acc[1] += w * xs[u].y;
+            acc[2] += w * xs[u].z;
+            acc[3] += w * xs[u].w;
+        }
+    } else if (!any && !peaked) {
         // every partial is used as it is; M is known, so the splits are
         // summed in batches of kB whose loads are in flight together
         constexpr int kB = 9;
@@ -1175,23 +1225,8 @@ cudaError_t attn_exact_combine_launch(const AttnArgs &a, const TreeMasks &masks,
                                       cudaStream_t stream)
 {
     const int rows_all = a.n_tree * a.n_heads_q;
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3((rows_all + 7) / 8);
-    cfg.blockDim = dim3(256);
-    cfg.dynamicSmemBytes = 0;
-    cfg.stream = stream;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    cudaError_t e = cudaLaunchKernelEx(&cfg, attn_t128_combine_kernel, a, masks, n_split,
-                                       split_positions, flags);
-    if (e == cudaSuccess)
-        e = cudaGetLastError();
-    if (e == cudaSuccess)
-        count_launches(1);
-    return e;
+    return launch_pdl(attn_t128_combine_kernel, dim3((rows_all + 7) / 8), dim3(256), 0, stream, a,
+                      masks, n_split, split_positions, flags);
 }
 
 }  // namespace ts

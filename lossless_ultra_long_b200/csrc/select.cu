@@ -17,24 +17,23 @@
 //   [Hq, n_ctx]) and a running (max, sum 2^(s-max)) per head and chunk.
 //   K is read once: Hkv * n_ctx * D * 2 bytes.
 // Selection (grids of chunks x Hkv, about two CTAs per SM, every head at
-//   once):
+//   once; each kernel a programmatic dependent of the one before):
 //   1. per chunk, each head's (max, sum 2^(s-max)) -- only when the scores
 //      come from the caller; the score pass leaves them itself;
 //   2. the importance score[n] = (1/G) sum_h 2^(s[h,n] - M_h) / Z_h of the
 //      chunk's positions, written out, and a 4096-bin histogram of the top
 //      bits of the candidates' scores (non-negative floats order as their
-//      bit patterns), summed per head in global memory; the last chunk of a
-//      head to finish finds the bin holding the budget-th largest candidate;
-//   3. per chunk, the candidates above that bin are counted and those in it
+//      bit patterns), summed per head in global memory;
+//   3. per chunk, the bin holding the budget-th largest candidate (from the
+//      head's histogram), the candidates above it counted and those in it
 //      listed (score bits, position);
-//   4. one CTA per head finds the exact budget-th largest score among the
-//      listed ones (two radix passes over the remaining 19 bits) and, per
-//      chunk, how many positions are kept before it;
-//   5. per chunk, the kept positions -- sinks, every score above the
-//      threshold, and the first scores equal to it in position order, so
-//      equal scores go to the lower position -- are written in ascending
-//      order from the chunk's offset and their K/V rows copied with 16-byte
-//      loads.
+//   4. per chunk, the exact budget-th largest score among the listed ones
+//      (two radix passes over the remaining 19 bits; every chunk of a head
+//      does this on its own, a few hundred keys) and the chunk's offset;
+//      then its kept positions -- sinks, every score above the threshold,
+//      and the first scores equal to it in position order, so equal scores
+//      go to the lower position -- written in ascending order and their
+//      K/V rows copied with 16-byte loads.
 #include <math.h>
 
 #include "attn_common.cuh"
@@ -208,6 +207,7 @@ constexpr int kBins0 = 4096;   // first-level bins: key bits 30..19
 constexpr int kShift0 = 19;
 constexpr int kMaxChunks = 256;
 constexpr int kMaxChunkLen = 48 * 1024;   // a chunk's kept positions are listed in shared memory
+static_assert(kMaxChunkLen < 65536, "per-chunk counts are packed in 16 bits");
 static_assert(kMaxChunks <= kSelThreads, "one chunk per thread in the offset scan");
 static_assert(kMaxGroup <= kSelThreads / 32, "one warp per head in the statistics merge");
 
@@ -216,22 +216,17 @@ enum SelMode { kSelect = 0, kKeepAll = 1, kSinksOnly = 2 };
 struct SelInfo {
     int digit0;    // the bin of the budget-th largest candidate key
     int need0;     // how many keys of that bin are kept
-    int n_cand;    // keys of that bin, appended to the candidate list
-    uint32_t T;    // the budget-th largest candidate key
-    int need_eq;   // how many keys equal to T are kept (lowest positions first)
-    int pad[3];
 };
 
 struct SelWs {
     float2 *part;      // [Hq, n_parts] per-chunk (max, sum 2^(s - max)) of each head
     int n_parts;
     float *imp;        // [Hkv, n_ctx] importance (scores_out or workspace)
-    int *hist;         // [Hkv, kBins0]
-    int *tick;         // [Hkv]
+    int *hist;         // [Hkv, kBins0] candidate keys per top-bits bin
     SelInfo *info;     // [Hkv]
-    int *above;        // [Hkv, NC] candidate keys above the threshold bin, per chunk
-    int2 *chunk;       // [Hkv, NC] (kept before the chunk, equal-to-T keys before it)
-    uint2 *cand;       // [Hkv, n_ctx] (key, position) of the threshold bin's keys
+    int2 *cnt;         // [Hkv, NC] per chunk: keys above the threshold bin, keys in it
+    uint2 *cand;       // [Hkv, n_ctx] (key, position) of the threshold bin's keys,
+                       // each chunk's from its own first position on
 };
 
 struct SelGeom {
@@ -301,90 +296,107 @@ __device__ int block_exclusive_scan(int x, int *scratch, int &excl)
 }
 
 // Kernel 1 (scores given by the caller): per (chunk, KV head), each head of
-// the group's (max, sum of 2^(s - max)) over the chunk.
+// the group's (max, sum of 2^(s - max)) over the chunk.  Every head's loads
+// of a round are in flight together; one reduction serves all heads.
+template <int GM>
 __global__ void __launch_bounds__(kSelThreads)
 sel_stats_kernel(SelectArgs a, SelGeom geo, SelWs ws)
 {
-    __shared__ float2 red[kSelThreads / 32];
+    __shared__ float2 red[kSelThreads / 32][GM];
     const int c = blockIdx.x, g = blockIdx.y;
     const int G = a.n_heads_q / a.n_heads_kv;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int N = a.n_ctx;
     const int p0 = min(c * geo.chunk, N), p1 = min(p0 + geo.chunk, N);
-    for (int h = 0; h < G; ++h) {
-        const float *row = a.root_scores + (size_t)(g * G + h) * N;
-        float m = -INFINITY, l = 0.f;
-        if ((N & 3) == 0) {
-            // the chunk is a multiple of 4 positions: 16-byte loads, all of
-            // this thread's loads in flight together
-            constexpr int kU = 8;
-            const int v0 = p0 / 4, v1 = p1 / 4;
-            for (int vb = v0 + tid; vb < v1; vb += kU * kSelThreads) {
-                float4 x[kU];
+    sm100::launch_dependents();
+    sm100::grid_dependency_wait();   // the scores come from the previous kernel
+    float m[GM], l[GM];
+#pragma unroll
+    for (int h = 0; h < GM; ++h) {
+        m[h] = -INFINITY;
+        l[h] = 0.f;
+    }
+    auto add = [&](int h, float x) {   // online (max, sum) of one head
+        if (x > m[h]) {
+            l[h] = (m[h] == -INFINITY ? 0.f : l[h] * exp2f(m[h] - x)) + 1.f;
+            m[h] = x;
+        } else if (x != -INFINITY) {
+            l[h] += exp2f(x - m[h]);
+        }
+    };
+    if ((N & 3) == 0) {
+        // 16-byte rows (the caller's rows are 16-byte aligned then)
+        constexpr int kU = 8 / GM;   // float4 per head and thread in flight
+        const int v0 = p0 / 4, v1 = p1 / 4;
+        for (int vb = v0 + tid; vb < v1; vb += kU * kSelThreads) {
+            float4 x[GM][kU];
+#pragma unroll
+            for (int h = 0; h < GM; ++h)
 #pragma unroll
                 for (int u = 0; u < kU; ++u) {
                     const int vi = vb + u * kSelThreads;
-                    x[u] = vi < v1 ? __ldcg(reinterpret_cast<const float4 *>(row) + vi)
-                                   : make_float4(-INFINITY, -INFINITY, -INFINITY, -INFINITY);
+                    x[h][u] = h < G && vi < v1
+                                  ? __ldcg(reinterpret_cast<const float4 *>(
+                                               a.root_scores + (size_t)(g * G + h) * N) + vi)
+                                  : make_float4(-INFINITY, -INFINITY, -INFINITY, -INFINITY);
                 }
+#pragma unroll
+            for (int h = 0; h < GM; ++h) {
                 float mx = -INFINITY;
 #pragma unroll
                 for (int u = 0; u < kU; ++u)
-                    mx = fmaxf(mx, fmaxf(fmaxf(x[u].x, x[u].y), fmaxf(x[u].z, x[u].w)));
+                    mx = fmaxf(mx, fmaxf(fmaxf(x[h][u].x, x[h][u].y), fmaxf(x[h][u].z, x[h][u].w)));
                 if (mx == -INFINITY)
                     continue;
-                if (mx > m) {
-                    l = m == -INFINITY ? 0.f : l * exp2f(m - mx);
-                    m = mx;
+                if (mx > m[h]) {
+                    l[h] = m[h] == -INFINITY ? 0.f : l[h] * exp2f(m[h] - mx);
+                    m[h] = mx;
                 }
                 float acc = 0.f;
 #pragma unroll
                 for (int u = 0; u < kU; ++u)
-                    acc += exp2f(x[u].x - m) + exp2f(x[u].y - m) + exp2f(x[u].z - m) +
-                           exp2f(x[u].w - m);
-                l += acc;
-            }
-        } else {
-            for (int n = p0 + tid; n < p1; n += kSelThreads) {
-                const float x = __ldcg(row + n);
-                if (x > m) {
-                    l = (m == -INFINITY ? 0.f : l * exp2f(m - x)) + 1.f;
-                    m = x;
-                } else if (x != -INFINITY) {
-                    l += exp2f(x - m);
-                }
+                    acc += exp2f(x[h][u].x - m[h]) + exp2f(x[h][u].y - m[h]) +
+                           exp2f(x[h][u].z - m[h]) + exp2f(x[h][u].w - m[h]);
+                l[h] += acc;
             }
         }
-        // CTA: max, then the sums rescaled to it
-        const float wm = warp_max(m);
-        float wl = warp_sum(m == -INFINITY ? 0.f : l * exp2f(m - wm));
+    } else {
+        for (int n = p0 + tid; n < p1; n += kSelThreads)
+#pragma unroll
+            for (int h = 0; h < GM; ++h)
+                if (h < G)
+                    add(h, __ldcg(a.root_scores + (size_t)(g * G + h) * N + n));
+    }
+    // warp, then CTA: the max, then the sums rescaled to it
+#pragma unroll
+    for (int h = 0; h < GM; ++h) {
+        const float wm = warp_max(m[h]);
+        const float wl = warp_sum(m[h] == -INFINITY ? 0.f : l[h] * exp2f(m[h] - wm));
         if (lane == 0)
-            red[warp] = make_float2(wm, wl);
-        __syncthreads();
-        if (warp == 0) {
-            const float2 r = lane < kSelThreads / 32 ? red[lane] : make_float2(-INFINITY, 0.f);
-            const float M = warp_max(r.x);
-            const float L = warp_sum(r.x == -INFINITY ? 0.f : r.y * exp2f(r.x - M));
-            if (lane == 0)
-                ws.part[(size_t)(g * G + h) * ws.n_parts + c] = make_float2(M, L);
-        }
-        __syncthreads();
+            red[warp][h] = make_float2(wm, wl);
+    }
+    __syncthreads();
+    if (warp < G) {
+        const float2 r = lane < kSelThreads / 32 ? red[lane][warp] : make_float2(-INFINITY, 0.f);
+        const float M = warp_max(r.x);
+        const float L = warp_sum(r.x == -INFINITY ? 0.f : r.y * exp2f(r.x - M));
+        if (lane == 0)
+            ws.part[(size_t)(g * G + warp) * ws.n_parts + c] = make_float2(M, L);
     }
 }
 
 // Kernel 2: importance of the chunk's positions (group mean of the heads'
-// softmax weights), written out; a histogram of the candidate keys' top 12
-// bits, summed over the head's chunks; the last chunk of a head to finish
-// finds the bin holding the budget-th largest candidate.
-__global__ void __launch_bounds__(kSelThreads, 2)
+// softmax weights), written out, and a histogram of the candidate keys'
+// top 12 bits added into the head's global histogram.  The score loads are
+// issued before the head statistics are merged, so that both are in flight
+// together.
+template <int GM>
+__global__ void __launch_bounds__(kSelThreads, GM == 4 ? 2 : 1)
 sel_keys_kernel(SelectArgs a, SelGeom geo, SelWs ws, const float *__restrict__ s_all, int mode,
                 int vec)
 {
     __shared__ int hist[kBins0];
-    __shared__ float head_m[kMaxGroup], head_w[kMaxGroup];
-    __shared__ int scan[72];
-    __shared__ int is_last;
-    __shared__ int found[2];
+    __shared__ float head_m[GM], head_w[GM];
     const int c = blockIdx.x, g = blockIdx.y;
     const int G = a.n_heads_q / a.n_heads_kv;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -393,16 +405,66 @@ sel_keys_kernel(SelectArgs a, SelGeom geo, SelWs ws, const float *__restrict__ s
     const bool do_hist = mode == kSelect;
     for (int b = tid; b < kBins0; b += kSelThreads)
         hist[b] = 0;
+    sm100::launch_dependents();
+    sm100::grid_dependency_wait();   // statistics and scores of the previous kernels
+    // one shared-memory atomic per key (grouping a warp's equal bins with
+    // a match instruction first measured slower)
+    auto hist_add = [&](bool in, uint32_t key) {
+        if (in)
+            atomicAdd(&hist[key >> kShift0], 1);
+    };
+    float *imp = ws.imp + (size_t)g * N;
+    constexpr int kR = 8 / GM;   // rounds of four positions per thread in flight
+    const int span = vec ? 4 * kSelThreads : kSelThreads;   // positions per round
+    const int rounds = (p1 - p0 + span - 1) / span;
+    float4 sv[kR][GM];
+    auto load = [&](int it0) {
+#pragma unroll
+        for (int r = 0; r < kR; ++r) {
+            if (vec) {
+                const int nb = p0 + 4 * (tid + (it0 + r) * kSelThreads);
+#pragma unroll
+                for (int h = 0; h < GM; ++h)
+                    sv[r][h] = h < G && it0 + r < rounds && nb < p1
+                                   ? __ldcg(reinterpret_cast<const float4 *>(
+                                         s_all + (size_t)(g * G + h) * N + nb))
+                                   : make_float4(0.f, 0.f, 0.f, 0.f);
+            } else {
+                const int n = p0 + tid + (it0 + r) * kSelThreads;
+#pragma unroll
+                for (int h = 0; h < GM; ++h)
+                    sv[r][h].x = h < G && it0 + r < rounds && n < p1
+                                     ? __ldcg(s_all + (size_t)(g * G + h) * N + n)
+                                     : 0.f;
+            }
+        }
+    };
+    load(0);
     if (warp < G) {
         const float2 *pp = ws.part + (size_t)(g * G + warp) * ws.n_parts;
         float M = -INFINITY;
-        for (int i = lane; i < ws.n_parts; i += 32)
-            M = fmaxf(M, pp[i].x);
+        float2 mine[2];
+#pragma unroll
+        for (int k = 0; k < 2; ++k) {
+            const int i = lane + 32 * k;
+            mine[k] = i < ws.n_parts ? __ldcg(pp + i) : make_float2(-INFINITY, 0.f);
+        }
+        for (int i = lane + 64; i < ws.n_parts; i += 32)
+            M = fmaxf(M, __ldcg(pp + i).x);
+#pragma unroll
+        for (int k = 0; k < 2; ++k)
+            M = fmaxf(M, mine[k].x);
         M = warp_max(M);
         float L = 0.f;
-        for (int i = lane; i < ws.n_parts; i += 32)
-            if (pp[i].x != -INFINITY)
-                L += pp[i].y * exp2f(pp[i].x - M);
+#pragma unroll
+        for (int k = 0; k < 2; ++k)
+            if (mine[k].x != -INFINITY)
+                L += mine[k].y * exp2f(mine[k].x - M);
+        for (int i = lane + 64; i < ws.n_parts; i += 32) {
+            const float2 x = __ldcg(pp + i);
+            if (x.x != -INFINITY)
+                L += x.y * exp2f(x.x - M);
+        }
         L = warp_sum(L);
         if (lane == 0) {
             head_m[warp] = M;
@@ -410,51 +472,26 @@ sel_keys_kernel(SelectArgs a, SelGeom geo, SelWs ws, const float *__restrict__ s
         }
     }
     __syncthreads();
-    float hm[kMaxGroup], hw[kMaxGroup];
+    float hm[GM], hw[GM];
 #pragma unroll
-    for (int h = 0; h < kMaxGroup; ++h) {
+    for (int h = 0; h < GM; ++h) {
         hm[h] = h < G ? head_m[h] : 0.f;
         hw[h] = h < G ? head_w[h] : 0.f;
     }
-    // lanes with equal bins add once, by their leader (positive scores
-    // share their leading bits, so many lanes of a warp hit the same bin)
-    auto hist_add = [&](bool in, uint32_t key) {
-        const unsigned act = __ballot_sync(0xffffffffu, in);
-        if (in) {
-            const uint32_t bin = key >> kShift0;
-            const unsigned same = __match_any_sync(act, bin);
-            if (lane == __ffs(same) - 1)
-                atomicAdd(&hist[bin], __popc(same));
-        }
-    };
-    float *imp = ws.imp + (size_t)g * N;
-    if (vec) {
-        // four positions per thread and round; two CTAs per SM keep enough
-        // loads in flight
-        constexpr int kR = 1;
-        const int rounds = (p1 - p0 + 4 * kSelThreads - 1) / (4 * kSelThreads);
-        for (int it0 = 0; it0 < rounds; it0 += kR) {
-            float4 sv[kR][kMaxGroup];
+    for (int it0 = 0; it0 < rounds; it0 += kR) {
+        if (it0 > 0)
+            load(it0);
 #pragma unroll
-            for (int r = 0; r < kR; ++r) {
-                const int nb = p0 + 4 * (tid + (it0 + r) * kSelThreads);
-#pragma unroll
-                for (int h = 0; h < kMaxGroup; ++h)
-                    if (h < G)
-                        sv[r][h] = nb < p1 ? __ldcg(reinterpret_cast<const float4 *>(
-                                                 s_all + (size_t)(g * G + h) * N + nb))
-                                           : make_float4(0.f, 0.f, 0.f, 0.f);
-            }
-#pragma unroll
-            for (int r = 0; r < kR; ++r) {
-                if (it0 + r >= rounds)
-                    break;   // uniform: every lane has the same rounds
+        for (int r = 0; r < kR; ++r) {
+            if (it0 + r >= rounds)
+                break;   // uniform: every lane has the same rounds
+            if (vec) {
                 const int nb = p0 + 4 * (tid + (it0 + r) * kSelThreads);
                 const bool live = nb < p1;
                 float sc[4] = {0.f, 0.f, 0.f, 0.f};
                 if (live) {
 #pragma unroll
-                    for (int h = 0; h < kMaxGroup; ++h)
+                    for (int h = 0; h < GM; ++h)
                         if (h < G) {
                             sc[0] += exp2f(sv[r][h].x - hm[h]) * hw[h];
                             sc[1] += exp2f(sv[r][h].y - hm[h]) * hw[h];
@@ -467,20 +504,19 @@ sel_keys_kernel(SelectArgs a, SelGeom geo, SelWs ws, const float *__restrict__ s
 #pragma unroll
                     for (int e = 0; e < 4; ++e)
                         hist_add(live && nb + e >= a.n_sink, __float_as_uint(sc[e]));
+            } else {
+                const int n = p0 + tid + (it0 + r) * kSelThreads;
+                float sc = 0.f;
+                if (n < p1) {
+#pragma unroll
+                    for (int h = 0; h < GM; ++h)
+                        if (h < G)
+                            sc += exp2f(sv[r][h].x - hm[h]) * hw[h];
+                    imp[n] = sc;
+                }
+                if (do_hist)
+                    hist_add(n < p1 && n >= a.n_sink, __float_as_uint(sc));
             }
-        }
-    } else {
-        const int rounds = (p1 - p0 + kSelThreads - 1) / kSelThreads;
-        for (int it = 0; it < rounds; ++it) {
-            const int n = p0 + tid + it * kSelThreads;
-            float sc = 0.f;
-            if (n < p1) {
-                for (int h = 0; h < G; ++h)
-                    sc += exp2f(__ldcg(s_all + (size_t)(g * G + h) * N + n) - hm[h]) * hw[h];
-                imp[n] = sc;
-            }
-            if (do_hist)
-                hist_add(n < p1 && n >= a.n_sink, __float_as_uint(sc));
         }
     }
     if (!do_hist)
@@ -490,17 +526,14 @@ sel_keys_kernel(SelectArgs a, SelGeom geo, SelWs ws, const float *__restrict__ s
     for (int b = tid; b < kBins0; b += kSelThreads)
         if (hist[b] != 0)
             atomicAdd(&ghist[b], hist[b]);
-    __threadfence();
-    __syncthreads();
-    if (tid == 0)
-        is_last = atomicAdd(&ws.tick[g], 1) == geo.nc - 1;
-    __syncthreads();
-    if (!is_last)
-        return;
-    __threadfence();
-    // every chunk of this head has added its histogram: the digit is the
-    // bin b with (keys in higher bins) < budget <= (that count + its keys).
-    // Thread t holds bins 4095 - 8t .. 4088 - 8t (descending).
+}
+
+// The threshold bin of head g from its global histogram: the bin b with
+// (candidates in higher bins) < budget <= (that count + its own).  Thread t
+// holds bins 4095 - 8t .. 4088 - 8t (descending).  found: 2 ints.
+__device__ void find_digit0(const int *ghist, int budget, int *scan, int *found)
+{
+    const int tid = threadIdx.x;
     int x[8];
     int sum = 0;
 #pragma unroll
@@ -510,59 +543,74 @@ sel_keys_kernel(SelectArgs a, SelGeom geo, SelWs ws, const float *__restrict__ s
     }
     int above;
     block_exclusive_scan(sum, scan, above);
-    if (tid == 0)
-        found[0] = -1;
-    __syncthreads();
 #pragma unroll
     for (int k = 0; k < 8; ++k) {
-        if (above < a.budget && a.budget <= above + x[k]) {
+        if (above < budget && budget <= above + x[k]) {
             found[0] = kBins0 - 1 - (8 * tid + k);
-            found[1] = a.budget - above;
+            found[1] = budget - above;
         }
         above += x[k];
     }
     __syncthreads();
-    if (tid == 0) {
-        ws.info[g].digit0 = found[0];
-        ws.info[g].need0 = found[1];
-        ws.tick[g] = 0;
-    }
-    // the histogram is left zero for the next call
-    for (int b = tid; b < kBins0; b += kSelThreads)
-        ghist[b] = 0;
 }
 
-// Kernel 3: per chunk, the candidate keys above the threshold bin are
-// counted and those in it are appended (key, position) to the head's list.
+// Kernel 3: per chunk, the threshold bin (found by every chunk from the
+// head's histogram), the candidate keys above it counted and those in it
+// listed at the chunk's own place in the candidate array.
+constexpr int kCandPer = 8;   // positions per thread and batch
 __global__ void __launch_bounds__(kSelThreads)
 sel_cand_kernel(SelectArgs a, SelGeom geo, SelWs ws)
 {
+    __shared__ int scan[72];
+    __shared__ int found[2];
     __shared__ int red[kSelThreads / 32];
     const int c = blockIdx.x, g = blockIdx.y;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int N = a.n_ctx;
     const int p0 = min(c * geo.chunk, N), p1 = min(p0 + geo.chunk, N);
-    const int digit0 = __ldcg(&ws.info[g].digit0);
     const float *imp = ws.imp + (size_t)g * N;
-    uint2 *cand = ws.cand + (size_t)g * N;
-    int n_above = 0;
-    const int rounds = (p1 - p0 + kSelThreads - 1) / kSelThreads;
-    for (int it = 0; it < rounds; ++it) {
-        const int n = p0 + tid + it * kSelThreads;
-        const bool in = n < p1 && n >= a.n_sink;
-        const uint32_t key = in ? __float_as_uint(__ldcg(imp + n)) : 0u;
-        const int bin = (int)(key >> kShift0);
-        n_above += in && bin > digit0;
-        const bool hit = in && bin == digit0;
-        const unsigned m = __ballot_sync(0xffffffffu, hit);
-        if (m) {
-            int base = 0;
-            if (lane == 0)
-                base = atomicAdd(&ws.info[g].n_cand, __popc(m));
-            base = __shfl_sync(0xffffffffu, base, 0);
-            if (hit)
-                cand[base + __popc(m & ((1u << lane) - 1u))] = make_uint2(key, (uint32_t)n);
+    uint2 *cand = ws.cand + (size_t)g * N + p0;
+    const int batches = (p1 - p0 + kCandPer * kSelThreads - 1) / (kCandPer * kSelThreads);
+    uint32_t key[kCandPer];
+    sm100::launch_dependents();
+    sm100::grid_dependency_wait();   // importance and histogram of the previous kernel
+    auto load = [&](int bt) {
+#pragma unroll
+        for (int i = 0; i < kCandPer; ++i) {
+            const int n = p0 + tid + (bt * kCandPer + i) * kSelThreads;
+            key[i] = n < p1 && n >= a.n_sink ? __float_as_uint(__ldcg(imp + n)) : 0xFFFFFFFFu;
         }
+    };
+    load(0);   // in flight while the histogram is read
+    if (tid == 0)
+        found[0] = -1;
+    find_digit0(ws.hist + (size_t)g * kBins0, a.budget, scan, found);
+    const int digit0 = found[0];
+    if (c == 0 && tid == 0) {
+        ws.info[g].digit0 = digit0;
+        ws.info[g].need0 = found[1];
+    }
+    int n_above = 0, base = 0;
+    for (int bt = 0; bt < batches; ++bt) {
+        if (bt > 0)
+            load(bt);
+        int hits = 0;
+#pragma unroll
+        for (int i = 0; i < kCandPer; ++i) {
+            if (key[i] == 0xFFFFFFFFu)
+                continue;   // outside the chunk, or a sink (scores are finite)
+            const int bin = (int)(key[i] >> kShift0);
+            n_above += bin > digit0;
+            hits += bin == digit0;
+        }
+        int before;
+        const int total = block_exclusive_scan(hits, scan, before);
+        int k = base + before;
+#pragma unroll
+        for (int i = 0; i < kCandPer; ++i)
+            if (key[i] != 0xFFFFFFFFu && (int)(key[i] >> kShift0) == digit0)
+                cand[k++] = make_uint2(key[i], (uint32_t)(p0 + tid + (bt * kCandPer + i) * kSelThreads));
+        base += total;
     }
     n_above = warp_isum(n_above);
     if (lane == 0)
@@ -572,101 +620,192 @@ sel_cand_kernel(SelectArgs a, SelGeom geo, SelWs ws)
         int v = lane < kSelThreads / 32 ? red[lane] : 0;
         v = warp_isum(v);
         if (lane == 0)
-            ws.above[(size_t)g * geo.nc + c] = v;
+            ws.cnt[(size_t)g * geo.nc + c] = make_int2(v, base);
     }
 }
 
-// Kernel 4, one CTA per KV head: the exact budget-th largest key among the
-// candidates (two radix passes over their low 19 bits), then per chunk the
-// number of kept positions before it and of equal-to-threshold keys before
-// it, so that each chunk can place its kept positions on its own.
-__global__ void __launch_bounds__(kSelThreads)
-sel_thresh_kernel(SelectArgs a, SelGeom geo, SelWs ws, int mode)
+// The exact threshold of head g and the offsets of chunk c, computed by
+// every chunk of the head on its own (a few hundred candidates in the
+// threshold bin, typically): the budget-th largest key among the
+// candidates (two radix passes over their low 19 bits, on a copy in shared
+// memory when it fits), then per chunk the number of kept positions before
+// it and of equal-to-threshold keys before it.
+constexpr int kCandSmem = 8 * 1024;   // candidates held in shared memory at most (64 KB)
+
+struct ThreshShared {
+    int hist[1024];
+    int scan[72];
+    int found[2];
+    uint32_t small[32];        // the keys of a thinly filled second-level bin
+    int n_small;
+    int seg[kMaxChunks];       // candidate offsets of the chunks
+    int gtc[kMaxChunks], eqc[kMaxChunks];
+    int2 ci;                   // this chunk: kept before it, equal-to-T keys before it
+    uint32_t T;                // the budget-th largest candidate key
+    int need_eq;               // keys equal to T that are kept (lowest positions first)
+};
+
+// Block-wide exact threshold over the n_cand candidates get(0 .. n_cand-1)
+// of bin digit0: a radix pass over bits 18..9 (1024 bins); if the bin it
+// finds holds at most 32 keys, warp 0 ranks them directly, else a second
+// pass over bits 8..0.  Then per chunk the candidates above T and equal to
+// T (sh.gtc, sh.eqc).  Leaves sh.T and sh.need_eq.
+template <typename Get>
+__device__ __forceinline__ void block_radix_threshold(Get get, int n_cand, int digit0, int need,
+                                                      const SelGeom &geo, ThreshShared &sh)
 {
-    __shared__ int hist[1024];
-    __shared__ int scan[72];
-    __shared__ int found[2];
-    __shared__ int gtc[kMaxChunks], eqc[kMaxChunks];
-    const int g = blockIdx.x;
+    const int tid = threadIdx.x, lane = tid & 31;
+    uint32_t prefix = (uint32_t)digit0 << kShift0;
+    uint32_t pmask = 0xFFFFFFFFu << kShift0;
+    bool done = false;
+    for (int pass = 0; pass < 2 && !done; ++pass) {
+        const int shift = pass == 0 ? 9 : 0;
+        const int nb = pass == 0 ? 1024 : 512;
+        const uint32_t dmask = (uint32_t)nb - 1;
+        for (int b = tid; b < 1024; b += kSelThreads)
+            sh.hist[b] = 0;
+        if (tid == 0)
+            sh.n_small = 0;
+        __syncthreads();
+        for (int i = tid; i < n_cand; i += kSelThreads) {
+            const uint32_t key = get(i).x;
+            if ((key & pmask) == prefix)
+                atomicAdd(&sh.hist[(key >> shift) & dmask], 1);
+        }
+        __syncthreads();
+        // thread t holds bins nb-1-2t, nb-2-2t (descending)
+        int x0 = 0, x1 = 0;
+        if (2 * tid < nb) {
+            x0 = sh.hist[nb - 1 - 2 * tid];
+            x1 = sh.hist[nb - 2 - 2 * tid];
+        }
+        int above;
+        block_exclusive_scan(x0 + x1, sh.scan, above);
+        if (2 * tid < nb) {
+            if (above < need && need <= above + x0) {
+                sh.found[0] = nb - 1 - 2 * tid;
+                sh.found[1] = above;
+            } else if (above + x0 < need && need <= above + x0 + x1) {
+                sh.found[0] = nb - 2 - 2 * tid;
+                sh.found[1] = above + x0;
+            }
+        }
+        __syncthreads();
+        const int digit = sh.found[0];
+        prefix |= (uint32_t)digit << shift;
+        pmask |= dmask << shift;
+        need -= sh.found[1];
+        if (pass == 0 && sh.hist[digit] <= 32) {
+            // few keys share the 22-bit prefix: list them and rank them in
+            // one warp
+            for (int i = tid; i < n_cand; i += kSelThreads) {
+                const uint32_t key = get(i).x;
+                if ((key & pmask) == prefix)
+                    sh.small[atomicAdd(&sh.n_small, 1)] = key;
+            }
+            __syncthreads();
+            if (tid < 32) {
+                const int m = sh.n_small;
+                const uint32_t mine = lane < m ? sh.small[lane] : 0u;
+                int gt = 0, ge = 0;
+                for (int j = 0; j < m; ++j) {
+                    const uint32_t kj = __shfl_sync(0xffffffffu, mine, j);
+                    gt += kj > mine;
+                    ge += kj >= mine;
+                }
+                if (lane < m && gt < need && need <= ge) {
+                    sh.T = mine;   // every writer holds the same key
+                    sh.need_eq = need - gt;
+                }
+            }
+            done = true;
+        } else if (pass == 1 && tid == 0) {
+            sh.T = prefix;
+            sh.need_eq = need;
+        }
+        __syncthreads();
+    }
+    const uint32_t T = sh.T;
+    for (int i = tid; i < n_cand; i += kSelThreads) {
+        const uint2 kp = get(i);
+        const int ch = (int)kp.y / geo.chunk;
+        if (kp.x > T)
+            atomicAdd(&sh.gtc[ch], 1);
+        else if (kp.x == T)
+            atomicAdd(&sh.eqc[ch], 1);
+    }
+    __syncthreads();
+}
+
+// The exact threshold of head g and the offsets of chunk c, found by every
+// chunk of the head on its own with the whole CTA (a few hundred
+// candidates in the threshold bin, typically).
+// The per-chunk counts (this thread's chunk), digit0 and need0 come loaded.
+__device__ void sel_threshold(const SelectArgs &a, const SelGeom &geo, const SelWs &ws, int mode,
+                              int g, int c, uint2 *cs, int cand_cap, ThreshShared &sh, int2 cn,
+                              int digit0, int need0)
+{
     const int tid = threadIdx.x;
     const int N = a.n_ctx;
-    SelInfo *inf = &ws.info[g];
-    uint32_t T = 0xFFFFFFFFu;   // nothing at or above: no candidate kept
-    int need_eq = 0;
-    int n_cand = 0;
-    if (mode == kSelect) {
-        n_cand = __ldcg(&inf->n_cand);
-        const int digit0 = __ldcg(&inf->digit0);
-        int need = __ldcg(&inf->need0);
-        const uint2 *cand = ws.cand + (size_t)g * N;
-        uint32_t prefix = (uint32_t)digit0 << kShift0;
-        uint32_t pmask = 0xFFFFFFFFu << kShift0;
-        for (int pass = 0; pass < 2; ++pass) {
-            const int shift = pass == 0 ? 9 : 0;
-            const int nb = pass == 0 ? 1024 : 512;
-            const uint32_t dmask = (uint32_t)nb - 1;
-            for (int b = tid; b < 1024; b += kSelThreads)
-                hist[b] = 0;
-            __syncthreads();
-            for (int i = tid; i < n_cand; i += kSelThreads) {
-                const uint32_t key = __ldcg(&cand[i].x);
-                if ((key & pmask) == prefix)
-                    atomicAdd(&hist[(key >> shift) & dmask], 1);
-            }
-            __syncthreads();
-            // thread t holds bins nb-1-2t, nb-2-2t (descending)
-            int x0 = 0, x1 = 0;
-            if (2 * tid < nb) {
-                x0 = hist[nb - 1 - 2 * tid];
-                x1 = hist[nb - 2 - 2 * tid];
-            }
-            int above;
-            block_exclusive_scan(x0 + x1, scan, above);
-            if (2 * tid < nb) {
-                if (above < need && need <= above + x0) {
-                    found[0] = nb - 1 - 2 * tid;
-                    found[1] = above;
-                } else if (above + x0 < need && need <= above + x0 + x1) {
-                    found[0] = nb - 2 - 2 * tid;
-                    found[1] = above + x0;
+    const bool sel = mode == kSelect;
+    const bool live = tid < geo.nc;
+    int seg_before;
+    const int n_cand = block_exclusive_scan(cn.y, sh.scan, seg_before);
+    if (live) {
+        sh.seg[tid] = seg_before;
+        sh.gtc[tid] = 0;
+        sh.eqc[tid] = 0;
+    }
+    if (tid == 0) {
+        sh.T = 0xFFFFFFFFu;   // nothing at or above: no candidate kept
+        sh.need_eq = 0;
+    }
+    __syncthreads();
+    const uint2 *gcand = ws.cand + (size_t)g * N;
+    // candidate i: chunk ch = the last with seg[ch] <= i, at its own place
+    auto cand_at = [&](int i) -> uint2 {
+        int lo = 0, hi = geo.nc - 1;
+        while (lo < hi) {
+            const int mid = (lo + hi + 1) >> 1;
+            if (sh.seg[mid] <= i)
+                lo = mid;
+            else
+                hi = mid - 1;
+        }
+        return __ldcg(gcand + (size_t)lo * geo.chunk + (i - sh.seg[lo]));
+    };
+    if (sel) {
+        if (n_cand <= cand_cap) {
+            for (int i0 = 0; i0 < n_cand; i0 += 4 * kSelThreads) {
+                uint2 v[4];
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                    const int i = i0 + tid + k * kSelThreads;
+                    v[k] = i < n_cand ? cand_at(i) : make_uint2(0u, 0u);
+                }
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                    const int i = i0 + tid + k * kSelThreads;
+                    if (i < n_cand)
+                        cs[i] = v[k];
                 }
             }
             __syncthreads();
-            prefix |= (uint32_t)found[0] << shift;
-            pmask |= dmask << shift;
-            need -= found[1];
-            __syncthreads();
-        }
-        T = prefix;
-        need_eq = need;
-    }
-    // per chunk: candidates above T and equal to T
-    for (int i = tid; i < geo.nc; i += kSelThreads) {
-        gtc[i] = 0;
-        eqc[i] = 0;
-    }
-    __syncthreads();
-    if (mode == kSelect) {
-        const uint2 *cand = ws.cand + (size_t)g * N;
-        for (int i = tid; i < n_cand; i += kSelThreads) {
-            const uint2 kp = __ldcg(&cand[i]);
-            const int ch = (int)kp.y / geo.chunk;
-            if (kp.x > T)
-                atomicAdd(&gtc[ch], 1);
-            else if (kp.x == T)
-                atomicAdd(&eqc[ch], 1);
+            // one code path per source of the candidates
+            block_radix_threshold([&](int i) { return cs[i]; }, n_cand, digit0, need0, geo, sh);
+        } else {
+            block_radix_threshold([&](int i) { return cand_at(i); }, n_cand, digit0, need0, geo,
+                                  sh);
         }
     }
-    __syncthreads();
-    // kept before chunk c: sinks before it, keys above T before it, and of
+    // kept before chunk ch: sinks before it, keys above T before it, and of
     // the equal keys the first need_eq in position order.  One chunk per
-    // thread (nc <= kMaxChunks <= kSelThreads): scan the equal counts, then
-    // the kept counts.
+    // thread: scan the equal counts, then the kept counts.
+    const int need_eq = sh.need_eq;
     const int ch = tid;
-    const bool live = ch < geo.nc;
-    const int my_eq = live && mode == kSelect ? eqc[ch] : 0;
+    const int my_eq = live && sel ? sh.eqc[ch] : 0;
     int eq_before;
-    block_exclusive_scan(my_eq, scan, eq_before);
+    block_exclusive_scan(my_eq, sh.scan, eq_before);
     int k = 0;
     if (live) {
         const int q0 = ch * geo.chunk, q1 = min(q0 + geo.chunk, N);
@@ -674,82 +813,136 @@ sel_thresh_kernel(SelectArgs a, SelGeom geo, SelWs ws, int mode)
             k = max(0, q1 - q0);
         } else {
             k = max(0, min(q1, a.n_sink) - q0);
-            if (mode == kSelect)
-                k += __ldcg(&ws.above[(size_t)g * geo.nc + ch]) + gtc[ch] +
-                     max(0, min(need_eq - eq_before, eqc[ch]));
+            if (sel)
+                k += cn.x + sh.gtc[ch] + max(0, min(need_eq - eq_before, my_eq));
         }
     }
     int kept_before;
-    block_exclusive_scan(k, scan, kept_before);
-    if (live)
-        ws.chunk[(size_t)g * geo.nc + ch] = make_int2(kept_before, eq_before);
-    if (tid == 0) {
-        inf->T = T;
-        inf->need_eq = need_eq;
-        inf->n_cand = 0;   // the list is empty again for the next call
-    }
+    block_exclusive_scan(k, sh.scan, kept_before);
+    if (ch == c)
+        sh.ci = make_int2(kept_before, eq_before);
+    __syncthreads();
 }
 
-// Kernel 5: each chunk writes its kept positions in ascending order from
-// its offset and copies their K and V rows into the partial cache.
+// Kernel 4: each chunk finds its head's threshold and its own offset, then
+// writes its kept positions in ascending order from that offset and copies
+// their K and V rows into the partial cache.  The first chunk of a head
+// leaves the head's histogram zero for the next call.
+constexpr int kGatherPer = 8;   // positions per thread held in registers
 template <int D>
-__global__ void __launch_bounds__(kSelThreads)
-sel_gather_kernel(SelectArgs a, SelGeom geo, SelWs ws, int mode)
+__global__ void __launch_bounds__(kSelThreads, 2)
+sel_gather_kernel(SelectArgs a, SelGeom geo, SelWs ws, int mode, int cand_cap)
 {
-    extern __shared__ int list[];   // this chunk's kept positions
-    __shared__ int scan[72];
+    extern __shared__ uint2 dyn[];   // cand_cap candidates, then this chunk's kept positions
+    __shared__ ThreshShared sh;
+    __shared__ int n_rows;
+    uint2 *cs = dyn;
+    int *list = reinterpret_cast<int *>(dyn + cand_cap);
     const int c = blockIdx.x, g = blockIdx.y;
     const int tid = threadIdx.x;
     const int N = a.n_ctx;
     const int p0 = min(c * geo.chunk, N), p1 = min(p0 + geo.chunk, N);
-    const int2 ci = __ldcg(&ws.chunk[(size_t)g * geo.nc + c]);
-    const uint32_t T = __ldcg(&ws.info[g].T);
-    const int need_eq = __ldcg(&ws.info[g].need_eq);
     const float *imp = ws.imp + (size_t)g * N;
+    sm100::launch_dependents();
+    sm100::grid_dependency_wait();   // candidates and counts of the previous kernel
+    const bool sel = mode == kSelect;
+    // the threshold's inputs first, so that they are not queued behind the
+    // chunk's keys
+    const int2 cn = tid < geo.nc && sel ? __ldcg(&ws.cnt[(size_t)g * geo.nc + tid])
+                                        : make_int2(0, 0);
+    const int digit0 = sel ? __ldcg(&ws.info[g].digit0) : 0;
+    const int need0 = sel ? __ldcg(&ws.info[g].need0) : 0;
+    // warp w owns positions [s0, s1) of the chunk, read coalesced in rounds
+    // of 32: position s0 + 32 r + lane
+    const int warp = tid >> 5, lane = tid & 31;
+    const int rounds = (p1 - p0 + kSelThreads - 1) / kSelThreads;
+    const int s0 = min(p0 + warp * 32 * rounds, p1), s1 = min(s0 + 32 * rounds, p1);
+    const bool in_regs = rounds <= kGatherPer && sel;
+    uint32_t key[kGatherPer];
+    if (in_regs) {
+#pragma unroll
+        for (int r = 0; r < kGatherPer; ++r) {
+            const int n = s0 + 32 * r + lane;
+            key[r] = r < rounds && n < s1 ? __float_as_uint(__ldcg(imp + n)) : 0u;
+        }
+    }
+    sel_threshold(a, geo, ws, mode, g, c, cs, cand_cap, sh, cn, digit0, need0);
+    if (c == 0 && sel) {
+        int *ghist = ws.hist + (size_t)g * kBins0;
+        for (int b = tid; b < kBins0; b += kSelThreads)
+            ghist[b] = 0;
+    }
+    const int2 ci = sh.ci;
+    const uint32_t T = sh.T;
+    const int need_eq = sh.need_eq;
     const int64_t want = (int64_t)a.n_sink + a.budget;
     const int n_keep = want < N ? (int)want : N;
-    // each thread a contiguous run of the chunk
-    const int per = (p1 - p0 + kSelThreads - 1) / kSelThreads;
-    const int q0 = p0 + tid * per, q1 = min(q0 + per, p1);
-    auto cls = [&](int n) -> int {   // 0 dropped, 1 kept, 2 equal to T
+    // 0 dropped, 1 kept, 2 equal to T
+    auto cls = [&](int r) -> int {
+        const int n = s0 + 32 * r + lane;
+        if (n >= s1)
+            return 0;
         if (mode == kKeepAll || n < a.n_sink)
             return 1;
-        if (mode != kSelect)
+        if (!sel)
             return 0;
-        const uint32_t key = __float_as_uint(__ldcg(imp + n));
-        return key > T ? 1 : (key == T ? 2 : 0);
+        const uint32_t k = in_regs ? key[r] : __float_as_uint(__ldcg(imp + n));
+        return k > T ? 1 : (k == T ? 2 : 0);
     };
+    // the warp's counts, then one scan over the warps (both counts packed:
+    // a chunk has at most kMaxChunkLen < 2^16 positions)
     int n_sure = 0, n_eq = 0;
-    for (int n = q0; n < q1; ++n) {
-        const int k = cls(n);
-        n_sure += k == 1;
-        n_eq += k == 2;
+    if (in_regs) {
+#pragma unroll
+        for (int r = 0; r < kGatherPer; ++r) {
+            const int k = r < rounds ? cls(r) : 0;
+            n_sure += __popc(__ballot_sync(0xffffffffu, k == 1));
+            n_eq += __popc(__ballot_sync(0xffffffffu, k == 2));
+        }
+    } else {
+        for (int r = 0; r < rounds; ++r) {
+            const int k = cls(r);
+            n_sure += __popc(__ballot_sync(0xffffffffu, k == 1));
+            n_eq += __popc(__ballot_sync(0xffffffffu, k == 2));
+        }
     }
-    int sure_before, eq_before;
-    block_exclusive_scan(n_sure, scan, sure_before);
-    block_exclusive_scan(n_eq, scan, eq_before);
+    int packed_before;
+    block_exclusive_scan(lane == 0 ? (n_sure | (n_eq << 16)) : 0, sh.scan, packed_before);
+    packed_before = __shfl_sync(0xffffffffu, packed_before, 0);
+    const int sure_before = packed_before & 0xFFFF, eq_before = packed_before >> 16;
     // equal keys are kept in position order: the first need_eq of the head
-    const int eqb = ci.y + eq_before;
+    int eqb = ci.y + eq_before;   // equal keys before this round's lane 0
     int slot = sure_before + max(0, min(need_eq, eqb)) - max(0, min(need_eq, ci.y));
-    int eq_rank = eqb;
     int32_t *idx = a.idx_out + (size_t)g * n_keep;
-    for (int n = q0; n < q1; ++n) {
-        const int k = cls(n);
-        const bool kept = k == 1 || (k == 2 && eq_rank++ < need_eq);
+    const unsigned lt = (1u << lane) - 1u;
+    auto place = [&](int r, int k) {
+        const unsigned eqm = __ballot_sync(0xffffffffu, k == 2);
+        const bool kept = k == 1 || (k == 2 && eqb + __popc(eqm & lt) < need_eq);
+        const unsigned km = __ballot_sync(0xffffffffu, kept);
         if (kept) {
-            const int out = ci.x + slot;
+            const int my = slot + __popc(km & lt);
+            const int out = ci.x + my;
+            const int n = s0 + 32 * r + lane;
             if (out < n_keep) {
                 idx[out] = n;
-                list[slot] = n;
+                list[my] = n;
             } else {
                 record_status(reinterpret_cast<WorkspaceHeader *>(a.workspace), TS_ERR_DEVICE_ARG);
             }
-            ++slot;
         }
+        eqb += __popc(eqm);
+        slot += __popc(km);
+    };
+    if (in_regs) {
+#pragma unroll
+        for (int r = 0; r < kGatherPer; ++r)
+            if (r < rounds)
+                place(r, cls(r));
+    } else {
+        for (int r = 0; r < rounds; ++r)
+            place(r, cls(r));
     }
-    __syncthreads();
     // rows: the chunk's kept count is the last thread's end slot
-    __shared__ int n_rows;
     if (tid == kSelThreads - 1)
         n_rows = min(slot, n_keep - ci.x);
     __syncthreads();
@@ -761,7 +954,7 @@ sel_gather_kernel(SelectArgs a, SelGeom geo, SelWs ws, int mode)
     __nv_bfloat16 *vp = a.v_partial + (int64_t)g * a.partial_cap * D;
     const int rows_per_pass = kSelThreads / LPR;
     const int li = tid % LPR;
-    constexpr int kG = 8;   // rows per thread per step, loads in flight together
+    constexpr int kG = 4;   // rows per thread per step, loads in flight together
     for (int t0 = tid / LPR; t0 < rows; t0 += rows_per_pass * kG) {
         uint4 kv[kG], vv[kG];
         int nn[kG];
@@ -816,9 +1009,9 @@ SelPlan make_sel_plan(int n_heads_kv, int n_ctx, int num_sms)
 }
 
 // Workspace: header, [score pass: s fp32 [Hq, n_ctx]], partials, importance,
-// histogram, tickets, info, per-chunk counts, candidates.
+// histograms, info, per-chunk counts and offsets, candidates.
 struct SelOffsets {
-    size_t s, part, imp, hist, tick, info, above, chunk, cand, total;
+    size_t s, part, imp, hist, info, cnt, cand, total;
 };
 
 SelOffsets sel_offsets(int n_heads_q, int n_heads_kv, int n_ctx, const SelPlan &p,
@@ -836,10 +1029,8 @@ SelOffsets sel_offsets(int n_heads_q, int n_heads_kv, int n_ctx, const SelPlan &
     o.part = take((size_t)n_heads_q * n_parts * sizeof(float2));
     o.imp = take((size_t)n_heads_kv * n_ctx * sizeof(float));
     o.hist = take((size_t)n_heads_kv * kBins0 * sizeof(int));
-    o.tick = take((size_t)n_heads_kv * sizeof(int));
     o.info = take((size_t)n_heads_kv * sizeof(SelInfo));
-    o.above = take((size_t)n_heads_kv * p.geo.nc * sizeof(int));
-    o.chunk = take((size_t)n_heads_kv * p.geo.nc * sizeof(int2));
+    o.cnt = take((size_t)n_heads_kv * p.geo.nc * sizeof(int2));
     o.cand = take((size_t)n_heads_kv * n_ctx * sizeof(uint2));
     o.total = at;
     return o;
@@ -877,10 +1068,8 @@ cudaError_t launch_d(const SelectArgs &a, const SelPlan &p, cudaStream_t stream)
     ws.n_parts = score_pass ? p.p1_chunks : p.geo.nc;
     ws.imp = a.scores_out ? a.scores_out : reinterpret_cast<float *>(w + o.imp);
     ws.hist = reinterpret_cast<int *>(w + o.hist);
-    ws.tick = reinterpret_cast<int *>(w + o.tick);
     ws.info = reinterpret_cast<SelInfo *>(w + o.info);
-    ws.above = reinterpret_cast<int *>(w + o.above);
-    ws.chunk = reinterpret_cast<int2 *>(w + o.chunk);
+    ws.cnt = reinterpret_cast<int2 *>(w + o.cnt);
     ws.cand = reinterpret_cast<uint2 *>(w + o.cand);
     const int64_t want = (int64_t)a.n_sink + a.budget;
     const int mode = want >= a.n_ctx ? kKeepAll : (a.budget == 0 ? kSinksOnly : kSelect);
@@ -889,7 +1078,12 @@ cudaError_t launch_d(const SelectArgs &a, const SelPlan &p, cudaStream_t stream)
     // scores: the caller's (then their per-chunk statistics here), or the
     // score pass into the workspace (which leaves the statistics itself)
     const float *s_all = a.root_scores;
+    const int G = a.n_heads_q / a.n_heads_kv;
+    const int GM = G <= 1 ? 1 : (G <= 2 ? 2 : (G <= 4 ? 4 : 8));
+    const dim3 block(kSelThreads);
     cudaError_t e;
+    // every kernel of the pipeline is launched as a programmatic dependent
+    // of the one before (it waits for it before reading its results)
     if (score_pass) {
         float *s_ws = reinterpret_cast<float *>(w + o.s);
         e = launch_p1<D>(a, p, s_ws, ws.part, stream);
@@ -897,37 +1091,42 @@ cudaError_t launch_d(const SelectArgs &a, const SelPlan &p, cudaStream_t stream)
             return e;
         s_all = s_ws;
     } else {
-        sel_stats_kernel<<<grid, kSelThreads, 0, stream>>>(a, p.geo, ws);
-        if ((e = cudaGetLastError()) != cudaSuccess)
+        e = GM == 1   ? launch_pdl(sel_stats_kernel<1>, grid, block, 0, stream, a, p.geo, ws)
+            : GM == 2 ? launch_pdl(sel_stats_kernel<2>, grid, block, 0, stream, a, p.geo, ws)
+            : GM == 4 ? launch_pdl(sel_stats_kernel<4>, grid, block, 0, stream, a, p.geo, ws)
+                      : launch_pdl(sel_stats_kernel<8>, grid, block, 0, stream, a, p.geo, ws);
+        if (e != cudaSuccess)
             return e;
-        count_launches(1);
     }
     // 16-byte loads and stores when every row starts on a 16-byte boundary
     const int vec = (a.n_ctx & 3) == 0 && reinterpret_cast<uintptr_t>(s_all) % 16 == 0 &&
                     reinterpret_cast<uintptr_t>(ws.imp) % 16 == 0;
-    sel_keys_kernel<<<grid, kSelThreads, 0, stream>>>(a, p.geo, ws, s_all, mode, vec);
-    if ((e = cudaGetLastError()) != cudaSuccess)
+    e = GM == 1   ? launch_pdl(sel_keys_kernel<1>, grid, block, 0, stream, a, p.geo, ws, s_all, mode, vec)
+        : GM == 2 ? launch_pdl(sel_keys_kernel<2>, grid, block, 0, stream, a, p.geo, ws, s_all, mode, vec)
+        : GM == 4 ? launch_pdl(sel_keys_kernel<4>, grid, block, 0, stream, a, p.geo, ws, s_all, mode, vec)
+                  : launch_pdl(sel_keys_kernel<8>, grid, block, 0, stream, a, p.geo, ws, s_all, mode, vec);
+    if (e != cudaSuccess)
         return e;
-    count_launches(1);
     if (mode == kSelect) {
-        sel_cand_kernel<<<grid, kSelThreads, 0, stream>>>(a, p.geo, ws);
-        if ((e = cudaGetLastError()) != cudaSuccess)
+        e = launch_pdl(sel_cand_kernel, grid, block, 0, stream, a, p.geo, ws);
+        if (e != cudaSuccess)
             return e;
-        count_launches(1);
     }
-    sel_thresh_kernel<<<a.n_heads_kv, kSelThreads, 0, stream>>>(a, p.geo, ws, mode);
-    if ((e = cudaGetLastError()) != cudaSuccess)
-        return e;
-    count_launches(1);
+    // dynamic shared memory: the candidates (as many as fit beside the
+    // chunk's list, up to kCandSmem), then the list
     const size_t list_bytes = (size_t)p.geo.chunk * sizeof(int);
+    constexpr size_t kDynMax = 96 * 1024;   // two CTAs per SM with the static part
+    size_t cap = list_bytes < kDynMax ? (kDynMax - list_bytes) / sizeof(uint2) : 0;
+    cap = cap > (size_t)kCandSmem ? (size_t)kCandSmem : cap;
+    const int cand_cap = (int)cap;
+    const size_t dyn = (size_t)cand_cap * sizeof(uint2) + list_bytes;
     static const cudaError_t attr = cudaFuncSetAttribute(
         sel_gather_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
     if (attr != cudaSuccess)
         return attr;
-    sel_gather_kernel<D><<<grid, kSelThreads, list_bytes, stream>>>(a, p.geo, ws, mode);
-    if ((e = cudaGetLastError()) != cudaSuccess)
+    e = launch_pdl(sel_gather_kernel<D>, grid, block, dyn, stream, a, p.geo, ws, mode, cand_cap);
+    if (e != cudaSuccess)
         return e;
-    count_launches(1);
     return cudaSuccess;
 }
 

@@ -27,6 +27,32 @@ inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 // Host-side count of kernel launches issued by the library.
 void count_launches(unsigned n);
 
+// Launch with programmatic stream serialization: the kernel may be
+// scheduled while the previous kernel on the stream is still running; it
+// must call griddepcontrol.wait before it touches that kernel's results (and
+// on every path, so that its own completion implies its predecessor's).
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                       cudaStream_t stream, Args... args)
+{
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    cudaError_t e = cudaLaunchKernelEx(&cfg, kernel, args...);
+    if (e == cudaSuccess)
+        e = cudaGetLastError();
+    if (e == cudaSuccess)
+        count_launches(1);
+    return e;
+}
+
 __device__ __forceinline__ void record_status(WorkspaceHeader *ws, uint32_t code)
 {
     atomicCAS(&ws->status, 0u, code);
