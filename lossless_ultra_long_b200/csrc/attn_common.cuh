@@ -12,6 +12,8 @@ namespace ts {
 struct AttnPlan {
     int n_split;          // KV splits per head
     int tiles_per_split;  // KV tiles each split streams
+    int node_groups = 1;      // tree-node groups, one CTA each per (split, head)
+    int nodes_per_group = 0;  // nodes of each group (the last may have fewer)
 };
 
 // The tcgen05 kernel feeds P to the PV product as one bf16 value; that is
@@ -39,13 +41,6 @@ cudaError_t attn_mma_launch(const AttnArgs &a, const TreeMasks &masks, int num_s
 bool encode_kv_map(CUtensorMap *m, const void *ptr, int rows, int64_t kv_cap, int n_heads_kv,
                    int box_rows, int head_dim = 128);
 
-bool attn_tc_eligible(int n_heads_q, int n_heads_kv, int head_dim, int n_ctx, int n_tree);
-// (the tcgen05 kernel also needs softmax_scale > 0: it takes the row max on
-// unscaled scores)
-AttnPlan attn_tc_plan(int n_heads_q, int n_heads_kv, int n_ctx, int n_tree, int num_sms);
-cudaError_t attn_tc_launch(const AttnArgs &a, const TreeMasks &masks, int num_sms,
-                           cudaStream_t stream);
-
 // Split partials of the tcgen05 kernels (head_dim 128): acc fp32
 // [n_split, T*Hq, 128] after the workspace header, then (m, l, q, 0) fp32
 // [n_split, T*Hq, 4]: m in log2 units, l the sum of the bf16-rounded
@@ -54,12 +49,15 @@ cudaError_t attn_tc_launch(const AttnArgs &a, const TreeMasks &masks, int num_sm
 // null: none), and the heavy splits of rows whose weight sits on too few
 // positions for bf16 weights.  split_positions: KV positions per split.
 size_t attn_exact_partial_bytes(int n_split, int n_heads_q, int n_tree);
+// flags: n_flag_groups int32 per (split, KV head), any of them set flags
+// the split of that head.
 cudaError_t attn_exact_combine_launch(const AttnArgs &a, const TreeMasks &masks, int n_split,
                                       int split_positions, const int32_t *flags,
-                                      cudaStream_t stream);
+                                      int n_flag_groups, cudaStream_t stream);
 
 // 128-position tiles, softmax spread over the four SM sub-partitions; up to
-// 192 query rows per KV head.
+// 192 query rows per KV head in one CTA, more split into groups of tree
+// nodes with one CTA each.
 bool attn_t128_eligible(int n_heads_q, int n_heads_kv, int head_dim, int n_ctx, int n_tree);
 AttnPlan attn_t128_plan(int n_heads_q, int n_heads_kv, int n_ctx, int n_tree, int num_sms);
 size_t attn_t128_workspace_bytes(int n_heads_q, int n_heads_kv, int n_ctx, int n_tree, int num_sms);

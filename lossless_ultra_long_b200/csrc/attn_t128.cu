@@ -164,20 +164,20 @@ __host__ __device__ inline int t128_row_of(int n, int R)
 // Whether warp 0 reads the root node's scores out of TMEM (one block: the G
 // root rows are TMEM lanes 0..G-1 of S_0, inside lanes 0..15, i.e. G <= 8
 // and G <= rq0).
-__host__ __device__ inline bool t128_rs_warp0(const AttnArgs &a)
+__host__ __device__ inline bool t128_rs_warp0(const AttnArgs &a, int T)
 {
     const int G = a.n_heads_q / a.n_heads_kv;
-    const int R = G * a.n_tree;
+    const int R = G * T;
     return a.root_scores != nullptr && R <= kBlockM && G <= 8 && G <= t128_rq0(R);
 }
 
 // Whether the block-1 softmax warp of lane quarter 0 stores the root node's
 // scores (two blocks: block 1's first quarter run, rows 0..rq1-1, holds the
 // G root rows when G <= rq1 and G <= 8, i.e. they are its first 16 lanes).
-__host__ __device__ inline bool t128_rs_block1(const AttnArgs &a)
+__host__ __device__ inline bool t128_rs_block1(const AttnArgs &a, int T)
 {
     const int G = a.n_heads_q / a.n_heads_kv;
-    const int R = G * a.n_tree;
+    const int R = G * T;
     const int rq1 = (R - kBlockM + 3) / 4;
     return a.root_scores != nullptr && R > kBlockM && G <= 8 && G <= rq1;
 }
@@ -185,9 +185,9 @@ __host__ __device__ inline bool t128_rs_block1(const AttnArgs &a)
 // Shared memory that stages the root node's scores for bulk copies (two
 // tiles of the G root rows) when block 1 stores them and every row starts
 // on a 16-byte boundary; 0 otherwise (plain stores, or warp 0).
-__host__ __device__ inline int t128_rs_bytes(const AttnArgs &a)
+__host__ __device__ inline int t128_rs_bytes(const AttnArgs &a, int T)
 {
-    const bool bulk = t128_rs_block1(a) &&
+    const bool bulk = t128_rs_block1(a, T) &&
                       (reinterpret_cast<uintptr_t>(a.root_scores) & 15) == 0 &&
                       (a.n_ctx & 3) == 0;
     return bulk ? 2 * (a.n_heads_q / a.n_heads_kv) * kTileN * 4 : 0;
@@ -314,17 +314,23 @@ __device__ __forceinline__ void store_p_half(uint32_t p_addr, uint32_t scratch, 
 __global__ void __launch_bounds__(kThreads, 1)
 attn_t128_kernel(const __grid_constant__ CUtensorMap tmap_k,
                  const __grid_constant__ CUtensorMap tmap_v, AttnArgs a, TreeMasks masks,
-                 int tiles_per_split, int n_split, int32_t *flags)
+                 int tiles_per_split, int n_split, int nodes_per_group, int32_t *flags)
 {
     const int G = a.n_heads_q / a.n_heads_kv;
-    const int R = G * a.n_tree;
+    // node group blockIdx.z: tree nodes node0 .. node0 + T - 1 (global node
+    // indices), its rows m = local node * G + head in group
+    const int node0 = blockIdx.z * nodes_per_group;
+    const int T = min(nodes_per_group, a.n_tree - node0);
+    if (node0 != 0)
+        a.root_scores = nullptr;   // the root node's rows live in group 0
+    const int R = G * T;
     const int NB = R > kBlockM ? 2 : 1;
     const int R0 = R < kBlockM ? R : kBlockM, R1 = R - R0;
     const int rq0 = (R0 + 3) / 4, rq1 = (R1 + 3) / 4;  // rows per lane quarter
     const int u0 = (rq0 + 15) / 16, u1 = (rq1 + 15) / 16;
     const int U = u0 + u1;  // softmax warps per lane quarter (at most 3)
-    const bool rs_warp0 = t128_rs_warp0(a);
-    const int rs_bytes = t128_rs_bytes(a);
+    const bool rs_warp0 = t128_rs_warp0(a, T);
+    const int rs_bytes = t128_rs_bytes(a, T);
     const Layout lay = t128_layout(R, rs_bytes);
     const int SK = lay.stages_k, SV = lay.stages_v, r_pad = lay.r_pad;
 
@@ -398,7 +404,7 @@ attn_t128_kernel(const __grid_constant__ CUtensorMap tmap_k,
     // block 1 (rows 128..R-1) into the shared-memory A tile (warps 8-11).
     auto q_row = [&](int n) {
         return reinterpret_cast<const uint4 *>(
-            a.q + ((int64_t)(n / G) * a.n_heads_q + g * G + n % G) * kD);
+            a.q + ((int64_t)(node0 + n / G) * a.n_heads_q + g * G + n % G) * kD);
     };
     if (warp == 3) {
         // producer: below, without the query barrier
@@ -656,7 +662,7 @@ attn_t128_kernel(const __grid_constant__ CUtensorMap tmap_k,
         // only); the first lane of a row's quad copies its staged scores out
         const bool rootA = b == 1 && vA && t128_row_of(nA, R) < G;
         const bool rootB = b == 1 && vB && t128_row_of(nB, R) < G;
-        const bool rs_warp = t128_rs_block1(a) && __any_sync(0xffffffffu, rootA || rootB);
+        const bool rs_warp = t128_rs_block1(a, T) && __any_sync(0xffffffffu, rootA || rootB);
         const bool rs_issue = rs_bytes != 0 && (lane & 3) == 0 && (rootA || rootB);
         bool ok = true;
         for (int t = 0; t < n_tiles; ++t) {
@@ -736,8 +742,8 @@ attn_t128_kernel(const __grid_constant__ CUtensorMap tmap_k,
             if (pos0 + kTileN > a.n_ctx) {
                 // visibility of this thread's 32 positions (entry k = 2 jj + e
                 // is position pos0 + 8 jj + c0 + e) for its two rows
-                const unsigned long long ancA = masks.anc[vA ? t128_row_of(nA, R) / G : 0];
-                const unsigned long long ancB = masks.anc[vB ? t128_row_of(nB, R) / G : 0];
+                const unsigned long long ancA = masks.anc[node0 + (vA ? t128_row_of(nA, R) / G : 0)];
+                const unsigned long long ancB = masks.anc[node0 + (vB ? t128_row_of(nB, R) / G : 0)];
                 uint32_t visA = 0u, visB = 0u;
 #pragma unroll 1
                 for (int k = 0; k < 32; ++k) {
@@ -819,7 +825,7 @@ attn_t128_kernel(const __grid_constant__ CUtensorMap tmap_k,
         // P^T row n -> output row of the head group
         auto orow_of = [&](int n) {
             const int m = t128_row_of(n, R);
-            return (m / G) * a.n_heads_q + g * G + m % G;
+            return (node0 + m / G) * a.n_heads_q + g * G + m % G;
         };
         if (ok && (lane & 3) == 0) {
             if (vA)
@@ -866,8 +872,8 @@ attn_t128_kernel(const __grid_constant__ CUtensorMap tmap_k,
             // a warp that gave up set the abort flag before this barrier
             if (!*abort && lane == 0) {
                 const int sw = warp - 4;   // 0 .. 4U-1
-                for (int node = sw; node < a.n_tree; node += 4 * U)
-                    bulk_store(ws_o + ((size_t)split * rows_all + (size_t)node * a.n_heads_q + g * G) * kD,
+                for (int node = sw; node < T; node += 4 * U)
+                    bulk_store(ws_o + ((size_t)split * rows_all + (size_t)(node0 + node) * a.n_heads_q + g * G) * kD,
                                smem_addr(sK) + (uint32_t)(node * G * kD * 4), (uint32_t)(G * kD * 4));
                 bulk_commit();
                 bulk_wait_all();   // the ring must outlive the copies out of it
@@ -882,7 +888,7 @@ attn_t128_kernel(const __grid_constant__ CUtensorMap tmap_k,
         tmem_dealloc(tmem, kTmemCols);
     }
     if (threadIdx.x == 0)
-        flags[split * a.n_heads_kv + g] = bar->overflow;
+        flags[(split * a.n_heads_kv + g) * gridDim.z + blockIdx.z] = bar->overflow;
 }
 
 // One split's partial (m, l, acc) of one query row, recomputed exactly in
@@ -965,7 +971,7 @@ __device__ void split_partial_exact(const AttnArgs &a, unsigned long long anc, i
 // kNeffMin on their own.
 __global__ void __launch_bounds__(256)
 attn_t128_combine_kernel(AttnArgs a, TreeMasks masks, int n_split, int split_positions,
-                         const int32_t *__restrict__ flags)
+                         const int32_t *__restrict__ flags, int n_flag_groups)
 {
     const int rows_all = a.n_tree * a.n_heads_q;
     const int row = blockIdx.x * 8 + (threadIdx.x >> 5);
@@ -987,7 +993,14 @@ attn_t128_combine_kernel(AttnArgs a, TreeMasks masks, int n_split, int split_pos
     // One round trip for the common case (at most kFastSplits splits): lane
     // s reads split s's (m, l, q) and flag while every lane also reads its
     // four columns of every split's acc, all loads in flight together.
-    auto flagged = [&](int s) { return flags != nullptr && flags[s * a.n_heads_kv + g] != 0; };
+    auto flagged = [&](int s) {
+        if (flags == nullptr)
+            return false;
+        bool f = false;
+        for (int z = 0; z < n_flag_groups; ++z)
+            f = f || flags[(s * a.n_heads_kv + g) * n_flag_groups + z] != 0;
+        return f;
+    };
     constexpr int kFastSplits = 24;
     const bool fast = n_split <= kFastSplits;
     float4 xs[kFastSplits];
@@ -1163,24 +1176,31 @@ size_t attn_t128_workspace_bytes(int n_heads_q, int n_heads_kv, int n_ctx, int n
 {
     const AttnPlan p = attn_t128_plan(n_heads_q, n_heads_kv, n_ctx, n_tree, num_sms);
     return flags_offset(p.n_split, n_heads_q, n_tree) +
-           align_up((size_t)p.n_split * n_heads_kv * sizeof(int32_t), 256);
+           align_up((size_t)p.n_split * n_heads_kv * p.node_groups * sizeof(int32_t), 256);
 }
 
 bool attn_t128_eligible(int n_heads_q, int n_heads_kv, int head_dim, int n_ctx, int n_tree)
 {
-    const int rows = (n_heads_q / n_heads_kv) * n_tree;
-    return head_dim == kD && rows <= kMaxRows && n_ctx >= kTcMinContext;
+    // a CTA takes whole tree nodes: one node's G rows must fit one block
+    const int G = n_heads_q / n_heads_kv;
+    return head_dim == kD && G <= kBlockM && n_ctx >= kTcMinContext;
 }
 
 AttnPlan attn_t128_plan(int n_heads_q, int n_heads_kv, int n_ctx, int n_tree, int num_sms)
 {
     AttnPlan p;
+    const int G = n_heads_q / n_heads_kv;
+    const int rows = G * n_tree;
+    // up to kMaxRows rows in one CTA; beyond that, groups of nodes of at
+    // most kBlockM rows (one 128-lane block each), one CTA per group
+    p.node_groups = rows <= kMaxRows ? 1 : (rows + kBlockM - 1) / kBlockM;
+    p.nodes_per_group = (n_tree + p.node_groups - 1) / p.node_groups;
+    p.node_groups = (n_tree + p.nodes_per_group - 1) / p.nodes_per_group;
     const int n_tiles = (n_ctx + n_tree + kTileN - 1) / kTileN;
-    int want = num_sms / n_heads_kv;
+    int want = num_sms / (n_heads_kv * p.node_groups);
     want = want < 1 ? 1 : (want > n_tiles ? n_tiles : want);
     p.tiles_per_split = (n_tiles + want - 1) / want;
     p.n_split = (n_tiles + p.tiles_per_split - 1) / p.tiles_per_split;
-    (void)n_heads_q;
     return p;
 }
 
@@ -1193,26 +1213,30 @@ cudaError_t attn_t128_launch(const AttnArgs &a, const TreeMasks &masks, int num_
     if (!encode_kv_map(&mk, a.k, rows, a.kv_cap, a.n_heads_kv, kTileN) ||
         !encode_kv_map(&mv, a.v, rows, a.kv_cap, a.n_heads_kv, kTileN))
         return cudaErrorInvalidValue;
-    const Layout lay = t128_layout((a.n_heads_q / a.n_heads_kv) * a.n_tree, t128_rs_bytes(a));
+    // the first node group is the largest and holds the root node
+    const int T0 = p.nodes_per_group;
+    const Layout lay = t128_layout((a.n_heads_q / a.n_heads_kv) * T0, t128_rs_bytes(a, T0));
     static const cudaError_t attr = cudaFuncSetAttribute(
         attn_t128_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemLimit);
     if (attr != cudaSuccess)
         return attr;
     int32_t *flags = reinterpret_cast<int32_t *>(
         reinterpret_cast<char *>(a.workspace) + flags_offset(p.n_split, a.n_heads_q, a.n_tree));
-    attn_t128_kernel<<<dim3(p.n_split, a.n_heads_kv), kThreads, lay.smem_bytes, stream>>>(
-        mk, mv, a, masks, p.tiles_per_split, p.n_split, flags);
+    attn_t128_kernel<<<dim3(p.n_split, a.n_heads_kv, p.node_groups), kThreads, lay.smem_bytes,
+                       stream>>>(mk, mv, a, masks, p.tiles_per_split, p.n_split, p.nodes_per_group,
+                                 flags);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess)
         return e;
     count_launches(1);
     return attn_exact_combine_launch(a, masks, p.n_split, p.tiles_per_split * kTileN, flags,
-                                     stream);
+                                     p.node_groups, stream);
 }
 
 bool attn_t128_leaves_root_scores(const AttnArgs &a)
 {
-    return t128_rs_warp0(a) || t128_rs_block1(a);
+    const AttnPlan p = attn_t128_plan(a.n_heads_q, a.n_heads_kv, a.n_ctx, a.n_tree, 148);
+    return t128_rs_warp0(a, p.nodes_per_group) || t128_rs_block1(a, p.nodes_per_group);
 }
 
 size_t attn_exact_partial_bytes(int n_split, int n_heads_q, int n_tree)
@@ -1222,11 +1246,11 @@ size_t attn_exact_partial_bytes(int n_split, int n_heads_q, int n_tree)
 
 cudaError_t attn_exact_combine_launch(const AttnArgs &a, const TreeMasks &masks, int n_split,
                                       int split_positions, const int32_t *flags,
-                                      cudaStream_t stream)
+                                      int n_flag_groups, cudaStream_t stream)
 {
     const int rows_all = a.n_tree * a.n_heads_q;
     return launch_pdl(attn_t128_combine_kernel, dim3((rows_all + 7) / 8), dim3(256), 0, stream, a,
-                      masks, n_split, split_positions, flags);
+                      masks, n_split, split_positions, flags, n_flag_groups);
 }
 
 }  // namespace ts
