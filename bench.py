@@ -130,7 +130,10 @@ def attn_traffic_record():
         rec = json.load(f)
     h = hashlib.sha256()
     for rel in rec.get("sources", []):
-        with open(os.path.join(ROOT, rel), "rb") as f:
+        path = os.path.join(ROOT, rel)
+        if not os.path.exists(path):
+            return None   # a source of the capture is gone: the record is stale
+        with open(path, "rb") as f:
             h.update(f.read())
     if h.hexdigest() != rec.get("sources_sha256"):
         return None

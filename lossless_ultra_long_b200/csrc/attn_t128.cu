@@ -1222,10 +1222,33 @@ cudaError_t attn_t128_launch(const AttnArgs &a, const TreeMasks &masks, int num_
         return attr;
     int32_t *flags = reinterpret_cast<int32_t *>(
         reinterpret_cast<char *>(a.workspace) + flags_offset(p.n_split, a.n_heads_q, a.n_tree));
-    attn_t128_kernel<<<dim3(p.n_split, a.n_heads_kv, p.node_groups), kThreads, lay.smem_bytes,
-                       stream>>>(mk, mv, a, masks, p.tiles_per_split, p.n_split, p.nodes_per_group,
-                                 flags);
-    cudaError_t e = cudaGetLastError();
+    cudaError_t e;
+    if (p.node_groups > 1 && p.node_groups <= 8) {
+        // the node groups of one (split, head) stream the same K/V tiles: as
+        // one cluster they start together on one GPC, so that the second
+        // read of each tile finds it in L2
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(p.n_split, a.n_heads_kv, p.node_groups);
+        cfg.blockDim = dim3(kThreads);
+        cfg.dynamicSmemBytes = lay.smem_bytes;
+        cfg.stream = stream;
+        cudaLaunchAttribute attr_c[1];
+        attr_c[0].id = cudaLaunchAttributeClusterDimension;
+        attr_c[0].val.clusterDim.x = 1;
+        attr_c[0].val.clusterDim.y = 1;
+        attr_c[0].val.clusterDim.z = p.node_groups;
+        cfg.attrs = attr_c;
+        cfg.numAttrs = 1;
+        e = cudaLaunchKernelEx(&cfg, attn_t128_kernel, mk, mv, a, masks, p.tiles_per_split,
+                               p.n_split, p.nodes_per_group, flags);
+        if (e == cudaSuccess)
+            e = cudaGetLastError();
+    } else {
+        attn_t128_kernel<<<dim3(p.n_split, a.n_heads_kv, p.node_groups), kThreads, lay.smem_bytes,
+                           stream>>>(mk, mv, a, masks, p.tiles_per_split, p.n_split,
+                                     p.nodes_per_group, flags);
+        e = cudaGetLastError();
+    }
     if (e != cudaSuccess)
         return e;
     count_launches(1);
