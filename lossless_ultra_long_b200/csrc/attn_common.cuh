@@ -41,26 +41,16 @@ cudaError_t attn_mma_launch(const AttnArgs &a, const TreeMasks &masks, int num_s
 bool encode_kv_map(CUtensorMap *m, const void *ptr, int rows, int64_t kv_cap, int n_heads_kv,
                    int box_rows, int head_dim = 128);
 
-// Split partials of the tcgen05 kernels (head_dim 128): acc fp32
-// [n_split, T*Hq, 128] after the workspace header, then (m, l, q, 0) fp32
-// [n_split, T*Hq, 4]: m in log2 units, l the sum of the bf16-rounded
-// weights relative to 2^m, q the sum of their squares.  The combine folds them; it recomputes exactly (fp32, CUDA
-// cores) every split whose int32 flag [n_split, Hkv] is set (flags may be
-// null: none), and the heavy splits of rows whose weight sits on too few
-// positions for bf16 weights.  split_positions: KV positions per split.
-size_t attn_exact_partial_bytes(int n_split, int n_heads_q, int n_tree);
-// flags: n_flag_groups int32 per (split, KV head), any of them set flags
-// the split of that head.
-cudaError_t attn_exact_combine_launch(const AttnArgs &a, const TreeMasks &masks, int n_split,
-                                      int split_positions, const int32_t *flags,
-                                      int n_flag_groups, cudaStream_t stream);
-
 // 128-position tiles, softmax spread over the four SM sub-partitions; up to
 // 192 query rows per KV head in one CTA, more split into groups of tree
-// nodes with one CTA each.
+// nodes with one CTA each.  The splits of a (head, group) take KV tiles at
+// run time and fold their partials themselves (one cooperative launch).
 bool attn_t128_eligible(int n_heads_q, int n_heads_kv, int head_dim, int n_ctx, int n_tree);
 AttnPlan attn_t128_plan(int n_heads_q, int n_heads_kv, int n_ctx, int n_tree, int num_sms);
 size_t attn_t128_workspace_bytes(int n_heads_q, int n_heads_kv, int n_ctx, int n_tree, int num_sms);
+// leading bytes of that workspace (header included) that must be zero when
+// a call starts; every call leaves them so
+size_t attn_t128_zeroed_bytes(int n_heads_q, int n_heads_kv, int n_ctx, int n_tree, int num_sms);
 cudaError_t attn_t128_launch(const AttnArgs &a, const TreeMasks &masks, int num_sms,
                              cudaStream_t stream);
 // whether that kernel writes a.root_scores itself (G <= 8 root rows inside

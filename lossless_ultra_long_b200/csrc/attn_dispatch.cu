@@ -57,6 +57,17 @@ size_t attn_workspace_bytes(int n_heads_q, int n_heads_kv, int head_dim, int n_c
     return bytes;
 }
 
+size_t attn_workspace_zeroed_bytes(int n_heads_q, int n_heads_kv, int head_dim, int n_ctx,
+                                   int n_tree, int num_sms)
+{
+    size_t bytes = kHeaderBytes;
+    if (attn_t128_eligible(n_heads_q, n_heads_kv, head_dim, n_ctx, n_tree)) {
+        const size_t t128 = attn_t128_zeroed_bytes(n_heads_q, n_heads_kv, n_ctx, n_tree, num_sms);
+        bytes = t128 > bytes ? t128 : bytes;
+    }
+    return bytes;
+}
+
 cudaError_t attn_launch(const AttnArgs &a, const TreeMasks &masks, int num_sms,
                         cudaStream_t stream)
 {

@@ -121,10 +121,13 @@ extern "C" int ts_tree_verify_attn_noalloc(const void *q, const void *k_cache,
         return TS_ERR_CUDA;
     }
     // the array keeps the previous call's contents: the hand-off tickets
-    // must start at zero; the status word is kept until the caller clears it
+    // and the kernel's counters must start at zero; the status word is kept
+    // until the caller clears it
     cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const size_t zeroed = ts::attn_workspace_zeroed_bytes(n_heads_q, n_heads_kv, head_dim, n_ctx,
+                                                          n_tree, ts::current_num_sms());
     if (cudaMemsetAsync(static_cast<unsigned char *>(scratch) + sizeof(uint32_t), 0,
-                        ts::kHeaderBytes - sizeof(uint32_t), s) != cudaSuccess) {
+                        zeroed - sizeof(uint32_t), s) != cudaSuccess) {
         cudaGetLastError();
         return TS_ERR_CUDA;
     }

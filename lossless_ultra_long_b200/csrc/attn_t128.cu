@@ -27,7 +27,7 @@
 // TMEM shape: four threads per row, 32 of the tile's 128 scores each, two
 // rows per thread (lanes t/4 and 8 + t/4 of the unit).
 //
-// CTA = (split, KV head), 16 warps, one CTA per SM:
+// CTA = (split, KV head, node group), 16 warps, one CTA per SM:
 //   warp 3      one lane is the TMA producer of K and V (two 64-column boxes
 //               of 128 positions per tile, 128-byte swizzle), K one tile
 //               ahead of V.  The map's row extent is n_ctx + T, so rows past
@@ -55,32 +55,45 @@
 // [384, 512).
 //
 // The reference max of a row is fixed at the first tile where the row sees
-// anything, and never moves, so the softmax warps need no per-tile
-// agreement with each other and no per-tile maximum at all.  fp32 has room
+// anything (that tile's max rounded up to an integer, in log2 units), and
+// never moves, so the softmax warps need no per-tile agreement with each
+// other and no per-tile maximum at all.  Being an integer, it scales every
+// weight by an exact power of two: the bf16-rounded weight of a position is
+// the same whichever split streams it, so the run-time hand-out of tiles to
+// splits moves results by fp32 summation order only.  fp32 has room
 // for it: a row's weights are at most its sum l, and while l <= 2^63 the
 // accumulated O^T stays below 2^63 * max|V|, far from overflow (a score
 // rise of about 44 nats inside one split would be needed to exceed it).  A
 // split in which some row's l ends above 2^63 (or not a number) raises a
-// flag; the combine kernel then recomputes that split's partial for the
-// affected head exactly (fp32, online softmax on CUDA cores) instead of
-// reading it.
-// Each split leaves an unnormalised partial (acc, m, l, q) and its flag;
-// the combine kernel always runs.
+// flag; the combine then recomputes that split's partial for the affected
+// head exactly (fp32, online softmax on CUDA cores) instead of reading it.
 //
-// P enters the PV product as one bf16 value and l sums those same rounded
-// values, so a row's output is an exact weighted mean of V with weights
-// perturbed by at most one bf16 rounding each.  Spread over many positions
-// those perturbations average out (the error falls like 1/sqrt of the
+// Work split: n_split CTAs per (KV head, node group), one per SM.  Each
+// starts on its own KV tile and then takes the next untaken tile of its
+// (head, group) from a counter in the workspace, so that splits which HBM
+// serves faster take more tiles and all end together (a fixed cut left the
+// slowest split several microseconds behind the mean).  An owner map
+// records which split streamed each tile.  Each split leaves an
+// unnormalised partial (acc, m, l, q) and its flag, counts itself in, and
+// once all splits of its (head, group) have arrived (the launch is
+// cooperative, so they are all resident) folds every n_split-th output row
+// of the group; no second kernel runs.
+//
+// P enters the PV product as one bf16 value while l sums the fp32 weights
+// (as FlashAttention kernels do), so a row's output is sum bf16(p) v /
+// sum p: every weight perturbed by at most one bf16 rounding (relative
+// 2^-8), the normalisation by none.  Spread over many positions those
+// perturbations average out (the error falls like rms|v| / sqrt of the
 // effective number of positions); on a row whose weight sits on a handful
 // of positions they do not.  The kernel therefore also keeps q, the sum of
-// the squared rounded weights, so that l^2 / q is the row's effective
-// number of positions.  The combine recomputes exactly (fp32, CUDA cores)
+// the squared weights, so that l^2 / q is the row's effective number of
+// positions.  The combine recomputes exactly (fp32, CUDA cores)
 // the splits that carry the weight of any row whose count over all splits
 // is below kNeffMin.
 //
-// Every wait is on an mbarrier and bounded (about a second): on expiry the
-// kernel records TS_ERR_TIMEOUT in the workspace status word, all roles
-// leave their loops, and TMEM is freed before the CTA exits.
+// Every wait is bounded (about a second): on expiry the kernel records
+// TS_ERR_TIMEOUT in the workspace status word, all roles leave their loops,
+// and TMEM is freed before the CTA exits.
 #include <math.h>
 
 #include "attn_common.cuh"
@@ -108,9 +121,9 @@ constexpr float kMaxRowSum = 9.223372036854775808e18f;   // 2^63: bound on a row
 // recomputed exactly.  With each weight perturbed by one bf16 rounding
 // (relative spread 2^-8 / sqrt(3)), the output error of a row with n
 // effective positions has a standard deviation of about
-// 2^-8 / sqrt(3) * rms|v - o| / sqrt(n); at n = 64 and |v - o| ~ 1.4
-// (bf16 N(0,1) values) that is 4e-4, so even the largest of many such
-// errors stays inside 2e-3.
+// 2^-8 / sqrt(3) * rms|v| / sqrt(n); at n = 64 and rms|v| ~ 1 (bf16
+// N(0,1) values) that is 2.8e-4, so even the largest of many such errors
+// stays inside 2e-3.
 constexpr float kNeffMin = 64.f;
 constexpr size_t kSmemLimit = 232448;        // dynamic shared memory per CTA
 static_assert(kBlockM % 32 == 0, "a 32-column O^T chunk lies inside one query block");
@@ -118,6 +131,7 @@ constexpr int kBarQuery = 1;                 // named barrier: query rows in pla
 constexpr int kBarOut = 2;                   // named barrier: O^T staged in shared memory
 constexpr int kBarQLoads = 3;                // named barrier: the query loads are issued
 constexpr int kQLoadThreads = 32 * 9;        // warps 4-11 arrive, the producer warp waits
+constexpr int kTileRing = 16;                // entries of the tile-index ring (> K/V lead)
 
 struct Bars {
     uint64_t full_k[kMaxStages];
@@ -131,6 +145,10 @@ struct Bars {
     uint64_t pv_issued[2];  // PV(t) is in the tensor queue (slot t & 1)
     uint64_t o_final;     // committed once, after the last PV
     uint64_t drain[2];    // each issuing thread's own MMAs, before TMEM is freed
+    // tile index of the CTA's t-th tile at [t % kTileRing], -1 after its
+    // last: written by the producer before the arrival on full_k of slot
+    // t, read by every role after its own wait for tile t
+    volatile int32_t tile_of[kTileRing];
     uint32_t tmem_base;
     uint32_t abort;
     int32_t overflow;     // some row exceeded its reference max by the headroom
@@ -145,7 +163,7 @@ struct Layout {
     int r_pad;  // rows rounded up to 16: N of the PV product
     int stages_k, stages_v;
     bool o_staged;  // the freed K/V ring holds every O row (fp32) for the write-out
-    size_t q1_off, p_off, k_off, v_off, aux_off, rs_off, smem_bytes;
+    size_t q1_off, p_off, k_off, v_off, aux_off, smem_bytes;
 };
 
 // Rows per TMEM lane quarter in block 0 (rows 0..min(R, 128) - 1 cut into
@@ -161,39 +179,20 @@ __host__ __device__ inline int t128_row_of(int n, int R)
     return R > kBlockM ? (n < kBlockM ? (R - kBlockM) + n : n - kBlockM) : n;
 }
 
-// Whether warp 0 reads the root node's scores out of TMEM (one block: the G
-// root rows are TMEM lanes 0..G-1 of S_0, inside lanes 0..15, i.e. G <= 8
-// and G <= rq0).
+// Whether warp 0 reads the root node's scores out of TMEM: they are rows
+// 0..G-1, which sit in the first lane-quarter run of the last block (block
+// 0 alone, or block 1: rows 0..rq_b-1 are TMEM lanes 0..rq_b-1), so the G
+// root rows are lanes 0..G-1, inside the first 16 lanes when G <= 8 and
+// G <= rq_b.  Warp 0 can read lane quarter 0, and is otherwise idle.
 __host__ __device__ inline bool t128_rs_warp0(const AttnArgs &a, int T)
 {
     const int G = a.n_heads_q / a.n_heads_kv;
     const int R = G * T;
-    return a.root_scores != nullptr && R <= kBlockM && G <= 8 && G <= t128_rq0(R);
+    const int rq = R > kBlockM ? (R - kBlockM + 3) / 4 : t128_rq0(R);
+    return a.root_scores != nullptr && G <= 8 && G <= rq;
 }
 
-// Whether the block-1 softmax warp of lane quarter 0 stores the root node's
-// scores (two blocks: block 1's first quarter run, rows 0..rq1-1, holds the
-// G root rows when G <= rq1 and G <= 8, i.e. they are its first 16 lanes).
-__host__ __device__ inline bool t128_rs_block1(const AttnArgs &a, int T)
-{
-    const int G = a.n_heads_q / a.n_heads_kv;
-    const int R = G * T;
-    const int rq1 = (R - kBlockM + 3) / 4;
-    return a.root_scores != nullptr && R > kBlockM && G <= 8 && G <= rq1;
-}
-
-// Shared memory that stages the root node's scores for bulk copies (two
-// tiles of the G root rows) when block 1 stores them and every row starts
-// on a 16-byte boundary; 0 otherwise (plain stores, or warp 0).
-__host__ __device__ inline int t128_rs_bytes(const AttnArgs &a, int T)
-{
-    const bool bulk = t128_rs_block1(a, T) &&
-                      (reinterpret_cast<uintptr_t>(a.root_scores) & 15) == 0 &&
-                      (a.n_ctx & 3) == 0;
-    return bulk ? 2 * (a.n_heads_q / a.n_heads_kv) * kTileN * 4 : 0;
-}
-
-__host__ __device__ inline Layout t128_layout(int rows, int rs_bytes)
+__host__ __device__ inline Layout t128_layout(int rows)
 {
     Layout L;
     L.r_pad = (rows + 15) / 16 * 16;
@@ -202,7 +201,7 @@ __host__ __device__ inline Layout t128_layout(int rows, int rs_bytes)
     // P^T: positions 0-63 then 64-127, each r_pad rows of 128 bytes; then
     // 1 KB that rows past the query rows are written to
     L.k_off = L.p_off + (size_t)L.r_pad * 256 + 1024;
-    const size_t fixed = 1024 + L.k_off + kAuxBytes + rs_bytes;
+    const size_t fixed = 1024 + L.k_off + kAuxBytes;
     int stages = (int)((kSmemLimit - fixed) / kStageBytes);
     stages = stages > 2 * kMaxStages ? 2 * kMaxStages : stages;
     L.stages_v = 2;
@@ -210,17 +209,17 @@ __host__ __device__ inline Layout t128_layout(int rows, int rs_bytes)
     L.v_off = L.k_off + (size_t)L.stages_k * kStageBytes;
     L.o_staged = (size_t)rows * kD * 4 <= (size_t)(L.stages_k + L.stages_v) * kStageBytes;
     L.aux_off = L.v_off + (size_t)L.stages_v * kStageBytes;
-    L.rs_off = L.aux_off + kAuxBytes;
-    L.smem_bytes = 1024 + L.rs_off + rs_bytes;
+    L.smem_bytes = 1024 + L.aux_off + kAuxBytes;
     return L;
 }
 
 // P = 2^(x * scale - m) for the 32 scores a thread holds of row A
 // (registers r[4j], r[4j + 1], j = 0..15) and, when TWO, of row B
-// (r[4j + 2], r[4j + 3]), packed to bf16 pairs; adds the sums of the rounded
-// values (what the PV product will use) to lA and lB, and their squares to
-// qA and qB.  Both rows advance together, so each score register is dead
-// once its pair is packed.
+// (r[4j + 2], r[4j + 3]), packed to bf16 pairs for the PV product; adds the
+// fp32 weights to lA and lB and their squares to qA and qB (summing the
+// rounded bf16 values instead costs two more instructions a pair, on the
+// path every tile waits for).  Both rows advance together, so each score
+// register is dead once its pair is packed.
 template <bool TWO>
 __device__ __forceinline__ void exp_pack_rows(const uint32_t (&r)[64], float scale, float neg_mA,
                                               float neg_mB, uint32_t (&pA)[16],
@@ -240,10 +239,10 @@ __device__ __forceinline__ void exp_pack_rows(const uint32_t (&r)[64], float sca
                                     sc2, h ? nB2 : nA2);
             float y0, y1;
             unpack2(y, y0, y1);
-            __nv_bfloat162 hv = __floats2bfloat162_rn(ex2(y0), ex2(y1));
+            const float x0 = ex2(y0), x1 = ex2(y1);
+            __nv_bfloat162 hv = __floats2bfloat162_rn(x0, x1);
             const uint32_t hb = *reinterpret_cast<uint32_t *>(&hv);
-            const uint64_t e2 =
-                pack2(__uint_as_float(hb << 16), __uint_as_float(hb & 0xFFFF0000u));
+            const uint64_t e2 = pack2(x0, x1);
             if (h) {
                 pB[j] = hb;
                 sB = add2(sB, e2);
@@ -311,10 +310,321 @@ __device__ __forceinline__ void store_p_half(uint32_t p_addr, uint32_t scratch, 
     }
 }
 
+// The kernel's workspace, after the 256-byte header.
+struct T128Sync {
+    int32_t *sync;    // [Hkv * groups][4]: tile counter, arrivals, finished combines, unused;
+                      // zero when a call starts, and again when it ends
+    float *part;      // split partials: acc fp32 [n_split][T*Hq][128], then
+                      // (m, l, q, 0) fp32 [n_split][T*Hq][4]
+    int32_t *flags;   // [n_split][Hkv * groups]: the split's reference max ran out of headroom
+    uint8_t *owner;   // [Hkv * groups][n_tiles]: the split that streamed each tile
+};
+
+// Adds positions p0 .. p1-1 of one query row to a running exact partial
+// (m, l, acc) of one split: fp32 online softmax on CUDA cores, one warp,
+// lane holding head dims 4 lane .. 4 lane + 3.  Used only for splits whose
+// flag says the fixed reference max ran out of headroom, and for the splits
+// that carry the weight of a row whose weight sits on too few positions for
+// one bf16 rounding of P.
+__device__ void split_partial_exact(const AttnArgs &a, unsigned long long anc, int g,
+                                    const float (&q4)[4], int p0, int p1, float &m, float &l,
+                                    float (&acc)[4])
+{
+    constexpr int kU = 8;   // positions per step: their loads and reductions overlap
+    const int lane = threadIdx.x & 31;
+    const __nv_bfloat16 *kh = a.k + (size_t)g * a.kv_cap * kD + 4 * lane;
+    const __nv_bfloat16 *vh = a.v + (size_t)g * a.kv_cap * kD + 4 * lane;
+    for (int pos0 = p0; pos0 < p1; pos0 += kU) {
+        float sc[kU];
+        bool seen[kU];
+#pragma unroll
+        for (int u = 0; u < kU; ++u) {
+            const int pos = pos0 + u;
+            const int tp = pos - a.n_ctx;
+            seen[u] = pos < p1 && (tp < 0 || ((anc >> tp) & 1ull));
+            const uint2 kb = seen[u] ? *reinterpret_cast<const uint2 *>(kh + (size_t)pos * kD)
+                                     : make_uint2(0u, 0u);
+            const float2 k01 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&kb.x));
+            const float2 k23 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&kb.y));
+            sc[u] = q4[0] * k01.x + q4[1] * k01.y + q4[2] * k23.x + q4[3] * k23.y;
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1)
+#pragma unroll
+            for (int u = 0; u < kU; ++u)
+                sc[u] += __shfl_xor_sync(0xffffffffu, sc[u], o);
+        float mx = -INFINITY;
+#pragma unroll
+        for (int u = 0; u < kU; ++u) {
+            sc[u] = seen[u] ? sc[u] * a.scale_log2 : -INFINITY;
+            mx = fmaxf(mx, sc[u]);
+        }
+        if (mx == -INFINITY)
+            continue;
+        if (mx > m) {
+            const float f = m == -INFINITY ? 0.f : exp2f(m - mx);
+            l *= f;
+#pragma unroll
+            for (int e = 0; e < 4; ++e)
+                acc[e] *= f;
+            m = mx;
+        }
+#pragma unroll
+        for (int u = 0; u < kU; ++u) {
+            if (!seen[u])
+                continue;
+            const float pw = exp2f(sc[u] - m);
+            const uint2 vb = *reinterpret_cast<const uint2 *>(vh + (size_t)(pos0 + u) * kD);
+            const float2 v01 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&vb.x));
+            const float2 v23 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&vb.y));
+            l += pw;
+            acc[0] += pw * v01.x;
+            acc[1] += pw * v01.y;
+            acc[2] += pw * v23.x;
+            acc[3] += pw * v23.y;
+        }
+    }
+}
+
+// One output row, by one warp: out = sum_s 2^(m_s - M) acc_s / sum_s
+// 2^(m_s - M) l_s over the n_split partials of its (KV head, node group)
+// gz.  Recomputed exactly instead of read: splits flagged for overflow,
+// and, on a row whose effective number of positions may be below kNeffMin
+// (L^2 < kNeffMin * sum_s c_s^2 q_s with c_s = 2^(m_s - M)), every split s
+// whose c_s^2 q_s is above L^2 / (kNeffMin * n_split) -- the remaining
+// splits then add up to a bound of at least kNeffMin on their own.  A
+// recomputed split covers the tiles the owner map gives it.
+__device__ __forceinline__ void t128_combine_row(const AttnArgs &a, const TreeMasks &masks, int row,
+                                              int g, int gz, int n_gz, int n_split,
+                                              const T128Sync &sy)
+{
+    const int rows_all = a.n_tree * a.n_heads_q;
+    const int lane = threadIdx.x & 31;
+    const int node = row / a.n_heads_q;
+    const int32_t *flags = sy.flags;
+    const float *ws_o = sy.part;
+    const float *ws_ml = ws_o + (size_t)n_split * rows_all * kD;
+    auto mlq_of = [&](int s) {
+        return __ldcg(reinterpret_cast<const float4 *>(ws_ml + ((size_t)s * rows_all + row) * 4));
+    };
+    auto flagged = [&](int s) { return __ldcg(flags + (size_t)s * n_gz + gz) != 0; };
+
+    // The common case (at most 2 kHalf splits): lane s reads split s's
+    // (m, l, q) and flag while every lane also reads its four columns of the
+    // acc of the first kHalf splits, all in flight together; the rest
+    // follow once M is known (two halves keep the registers below the
+    // kernel's budget).
+    constexpr int kHalf = 12;
+    const bool fast = n_split <= 2 * kHalf;
+    float4 xs[kHalf];
+    float4 my = make_float4(-INFINITY, 0.f, 0.f, 0.f);
+    bool my_f = false;
+    if (fast) {
+        if (lane < n_split) {
+            my = mlq_of(lane);
+            my_f = flagged(lane);
+        }
+#pragma unroll
+        for (int u = 0; u < kHalf; ++u)
+            xs[u] = u < n_split ? __ldcg(reinterpret_cast<const float4 *>(
+                                      ws_o + ((size_t)u * rows_all + row) * kD + 4 * lane))
+                                : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+
+    // M, and L and the bound's denominator, over the splits that are not
+    // flagged
+    bool any = false;
+    float M = -INFINITY;
+    if (fast) {
+        any = my_f;
+        if (!my_f)
+            M = my.x;
+    } else {
+        for (int s = lane; s < n_split; s += 32) {
+            const bool f = flagged(s);
+            any |= f;
+            if (!f)
+                M = fmaxf(M, mlq_of(s).x);
+        }
+    }
+    any = __any_sync(0xffffffffu, any);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1)
+        M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+    // L^2 and the q sums reach 2^126 times the splits squared: the count is
+    // formed in fp64
+    double Lp = 0.0, Qp = 0.0;
+    if (M != -INFINITY) {
+        if (fast) {
+            if (!my_f && my.x != -INFINITY) {
+                const double c = (double)exp2f(my.x - M);
+                Lp = c * (double)my.y;
+                Qp = c * c * (double)my.z;
+            }
+        } else {
+            for (int s = lane; s < n_split; s += 32) {
+                if (flagged(s))
+                    continue;
+                const float4 x = mlq_of(s);
+                const double c = x.x == -INFINITY ? 0.0 : (double)exp2f(x.x - M);
+                Lp += c * (double)x.y;
+                Qp += c * c * (double)x.z;
+            }
+        }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        Lp += __shfl_xor_sync(0xffffffffu, Lp, o);
+        Qp += __shfl_xor_sync(0xffffffffu, Qp, o);
+    }
+    const bool peaked = Lp * Lp < (double)kNeffMin * Qp;   // uniform across the warp
+    const double heavy = Lp * Lp / ((double)kNeffMin * n_split);
+
+    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+    float L = 0.f;
+    if (!any && !peaked && fast) {
+        // every partial is used as it is: lane s's weight 2^(m_s - M) and
+        // its weighted l, passed to every lane
+        const float w_my = my.x == -INFINITY ? 0.f : exp2f(my.x - M);
+        const float wl_my = w_my * my.y;
+        for (int h = 0; h < 2 && h * kHalf < n_split; ++h) {
+            if (h == 1) {
+#pragma unroll
+                for (int u = 0; u < kHalf; ++u)
+                    xs[u] = kHalf + u < n_split
+                                ? __ldcg(reinterpret_cast<const float4 *>(
+                                      ws_o + ((size_t)(kHalf + u) * rows_all + row) * kD + 4 * lane))
+                                : make_float4(0.f, 0.f, 0.f, 0.f);
+            }
+#pragma unroll
+            for (int u = 0; u < kHalf; ++u) {
+                const int sp = h * kHalf + u;
+                if (sp >= n_split)
+                    break;
+                const float w = __shfl_sync(0xffffffffu, w_my, sp);
+                L += __shfl_sync(0xffffffffu, wl_my, sp);
+                acc[0] += w * xs[u].x;
+                acc[1] += w * xs[u].y;
+                acc[2] += w * xs[u].z;
+                acc[3] += w * xs[u].w;
+            }
+        }
+    } else if (!any && !peaked) {
+        // every partial is used as it is; M is known, so the splits are
+        // summed in batches of kB whose loads are in flight together
+        constexpr int kB = 9;
+        for (int s0 = 0; s0 < n_split; s0 += kB) {
+            float4 mlq[kB], x[kB];
+#pragma unroll
+            for (int u = 0; u < kB; ++u) {
+                const int s = s0 + u;
+                if (s < n_split) {
+                    mlq[u] = mlq_of(s);
+                    x[u] = __ldcg(reinterpret_cast<const float4 *>(
+                        ws_o + ((size_t)s * rows_all + row) * kD + 4 * lane));
+                } else {
+                    mlq[u] = make_float4(-INFINITY, 0.f, 0.f, 0.f);
+                    x[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+                }
+            }
+#pragma unroll
+            for (int u = 0; u < kB; ++u) {
+                const float w = mlq[u].x == -INFINITY ? 0.f : exp2f(mlq[u].x - M);
+                L += w * mlq[u].y;
+                acc[0] += w * x[u].x;
+                acc[1] += w * x[u].y;
+                acc[2] += w * x[u].z;
+                acc[3] += w * x[u].w;
+            }
+        }
+    } else {
+        // fold the splits one by one into a running (Mr, L, acc), the
+        // flagged and the heavy ones recomputed
+        const uint2 qb = *reinterpret_cast<const uint2 *>(a.q + (size_t)row * kD + 4 * lane);
+        const float2 q01 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&qb.x));
+        const float2 q23 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&qb.y));
+        const float q4[4] = {q01.x, q01.y, q23.x, q23.y};
+        const int total = a.n_ctx + a.n_tree;
+        const int n_tiles_all = (total + kTileN - 1) / kTileN;
+        const uint8_t *own = sy.owner + (size_t)gz * n_tiles_all;
+        float Mr = -INFINITY;
+        for (int s = 0; s < n_split; ++s) {
+            float ms, ls, as[4];
+            const float4 x4 = mlq_of(s);
+            bool exact = flagged(s);
+            if (!exact && peaked && x4.x != -INFINITY) {
+                const double c = (double)exp2f(x4.x - M);
+                exact = c * c * (double)x4.z > heavy;
+            }
+            if (exact) {
+                ms = -INFINITY;
+                ls = 0.f;
+#pragma unroll
+                for (int e = 0; e < 4; ++e)
+                    as[e] = 0.f;
+                // the tiles this split streamed, 32 owner entries at a time
+                for (int t0 = 0; t0 < n_tiles_all; t0 += 32) {
+                    const int t = t0 + lane;
+                    uint32_t bits = __ballot_sync(0xffffffffu, t < n_tiles_all && own[t] == s);
+                    while (bits) {
+                        const int tt = t0 + __ffs(bits) - 1;
+                        bits &= bits - 1;
+                        split_partial_exact(a, masks.anc[node], g, q4, tt * kTileN,
+                                            min(tt * kTileN + kTileN, total), ms, ls, as);
+                    }
+                }
+            } else {
+                const float4 x = __ldcg(reinterpret_cast<const float4 *>(
+                    ws_o + ((size_t)s * rows_all + row) * kD + 4 * lane));
+                ms = x4.x;
+                ls = x4.y;
+                as[0] = x.x;
+                as[1] = x.y;
+                as[2] = x.z;
+                as[3] = x.w;
+            }
+            if (ms == -INFINITY)
+                continue;
+            const float Mn = fmaxf(Mr, ms);
+            const float fa = Mr == -INFINITY ? 0.f : exp2f(Mr - Mn);
+            const float fb = exp2f(ms - Mn);
+            L = L * fa + ls * fb;
+#pragma unroll
+            for (int e = 0; e < 4; ++e)
+                acc[e] = acc[e] * fa + as[e] * fb;
+            Mr = Mn;
+        }
+    }
+    const float inv = 1.f / L;
+    *reinterpret_cast<float4 *>(a.out + (size_t)row * kD + 4 * lane) =
+        make_float4(acc[0] * inv, acc[1] * inv, acc[2] * inv, acc[3] * inv);
+}
+
+// Bounded wait until the int32 at p (written by other CTAs) reaches
+// target, read with gpu-scope acquire; on expiry raises *abort and records
+// TS_ERR_TIMEOUT.
+__device__ __forceinline__ bool wait_count_bounded(const int32_t *p, int target,
+                                                   volatile uint32_t *abort, WorkspaceHeader *ws)
+{
+    const long long t0 = clock64();
+    for (;;) {
+        int32_t v;
+        asm volatile("ld.acquire.gpu.global.b32 %0, [%1];\n" : "=r"(v) : "l"(p) : "memory");
+        if (v >= target)
+            return true;
+        if (clock64() - t0 > kWaitCycles) {
+            *abort = 1u;
+            record_status(ws, TS_ERR_TIMEOUT);
+            return false;
+        }
+        __nanosleep(128);
+    }
+}
+
 __global__ void __launch_bounds__(kThreads, 1)
 attn_t128_kernel(const __grid_constant__ CUtensorMap tmap_k,
                  const __grid_constant__ CUtensorMap tmap_v, AttnArgs a, TreeMasks masks,
-                 int tiles_per_split, int n_split, int nodes_per_group, int32_t *flags)
+                 int n_split, int nodes_per_group, T128Sync sy)
 {
     const int G = a.n_heads_q / a.n_heads_kv;
     // node group blockIdx.z: tree nodes node0 .. node0 + T - 1 (global node
@@ -330,8 +640,7 @@ attn_t128_kernel(const __grid_constant__ CUtensorMap tmap_k,
     const int u0 = (rq0 + 15) / 16, u1 = (rq1 + 15) / 16;
     const int U = u0 + u1;  // softmax warps per lane quarter (at most 3)
     const bool rs_warp0 = t128_rs_warp0(a, T);
-    const int rs_bytes = t128_rs_bytes(a, T);
-    const Layout lay = t128_layout(R, rs_bytes);
+    const Layout lay = t128_layout(R);
     const int SK = lay.stages_k, SV = lay.stages_v, r_pad = lay.r_pad;
 
     extern __shared__ unsigned char smem_raw[];
@@ -350,8 +659,9 @@ attn_t128_kernel(const __grid_constant__ CUtensorMap tmap_k,
     const int split = blockIdx.x, g = blockIdx.y;
     const int total = a.n_ctx + a.n_tree;
     const int n_tiles_all = (total + kTileN - 1) / kTileN;
-    const int t_begin = split * tiles_per_split;
-    const int n_tiles = min(t_begin + tiles_per_split, n_tiles_all) - t_begin;
+    // (KV head, node group) of this CTA: its splits share one tile counter
+    // and one arrival count (sy.sync + 4 gz)
+    const int gz = g * gridDim.z + blockIdx.z;
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < SK; ++s) {
@@ -364,8 +674,9 @@ attn_t128_kernel(const __grid_constant__ CUtensorMap tmap_k,
         }
         mbar_init(smem_addr(&bar->s_full[0]), 1);
         mbar_init(smem_addr(&bar->s_full[1]), 1);
-        mbar_init(smem_addr(&bar->s_free[0]), 4 * u0 + (rs_warp0 ? 1 : 0));
-        mbar_init(smem_addr(&bar->s_free[1]), u1 > 0 ? 4 * u1 : 1);
+        // warp 0 also reads S of the last block when it stores the root scores
+        mbar_init(smem_addr(&bar->s_free[0]), 4 * u0 + (rs_warp0 && NB == 1 ? 1 : 0));
+        mbar_init(smem_addr(&bar->s_free[1]), (u1 > 0 ? 4 * u1 : 1) + (rs_warp0 && NB == 2 ? 1 : 0));
         mbar_init(smem_addr(&bar->sm_done), 4 * U);
         mbar_init(smem_addr(&bar->pv_done), 1);
         mbar_init(smem_addr(&bar->pv_issued[0]), 1);
@@ -464,77 +775,109 @@ attn_t128_kernel(const __grid_constant__ CUtensorMap tmap_k,
 
     if (warp == 3) {
         // ------------------------------------ TMA producer (K one tile ahead)
+        // Tiles are handed out at run time, from the end of the cache
+        // backwards: the split's own tile (n_tiles - 1 - split) first, then
+        // tile n_tiles - 1 - (n_split + k) for the k-th increment of the
+        // (head, group) counter, so that the splits of a head end together
+        // however HBM serves them, and the tree-tail tile (the one with
+        // ancestor masks) is taken first rather than last.  Each taken tile
+        // is recorded in the owner map (for the exact recompute of a split).
         named_bar_sync(kBarQLoads, kQLoadThreads);
         if (lane == 0) {
             int nk = 0, nv = 0;   // tiles issued so far
+            int uk = 0, uv = 0;   // ring entries used (the end marker included)
+            // k-th tile handed out -> its index (k < 0 once none is left)
+            auto tile_at = [&](int k) { return n_tiles_all - 1 - k; };
+            int32_t *ctr = sy.sync + 4 * gz;
+            int cur = tile_at(split);
+            int nxt = tile_at(n_split + atomicAdd(&ctr[0], 1));   // used one step later
+            int kend = -1;        // ring index of the end marker
+            uint8_t *owner = sy.owner + (size_t)gz * n_tiles_all;
             // step i issues K(i), then V(i - 1): K is consumed a whole softmax
             // pass before V, and each load waits only for its own ring slot
-            for (int i = 0; i <= n_tiles; ++i) {
-                bool ok = true;
-#pragma unroll 1
-                for (int which = 0; which < 2 && ok; ++which) {
-                    const bool is_k = which == 0;
-                    const int t = is_k ? i : i - 1;
-                    if (t < 0 || t >= n_tiles)
-                        continue;
-                    const int ns = is_k ? SK : SV;
-                    const int s = t % ns;
-                    uint64_t *full = is_k ? bar->full_k : bar->full_v;
-                    uint64_t *empty = is_k ? bar->empty_k : bar->empty_v;
-                    if (t >= ns &&
-                        !wait_bounded(smem_addr(&empty[s]), ((t / ns) & 1) ^ 1, abort, hdr)) {
-                        ok = false;
+            for (int i = 0;; ++i) {
+                if (kend < 0) {
+                    const int s = i % SK;
+                    if (i >= SK &&
+                        !wait_bounded(smem_addr(&bar->empty_k[s]), ((i / SK) & 1) ^ 1, abort, hdr))
+                        break;
+                    const uint32_t fb = smem_addr(&bar->full_k[s]);
+                    if (cur >= 0) {
+                        bar->tile_of[i % kTileRing] = cur;
+                        owner[cur] = (uint8_t)split;
+                        mbar_arrive_expect_tx(fb, kStageBytes);
+                        const uint32_t dst = smem_addr(sK + s * kStageBytes);
+                        tma_load_3d(dst, &tmap_k, 0, cur * kTileN, g, fb);
+                        tma_load_3d(dst + kBoxBytes, &tmap_k, 64, cur * kTileN, g, fb);
+                        nk = uk = i + 1;
+                        cur = nxt;
+                        if (cur >= 0)
+                            nxt = tile_at(n_split + atomicAdd(&ctr[0], 1));
+                    } else {
+                        // no tile left: the QK issuer passes the marker on
+                        bar->tile_of[i % kTileRing] = -1;
+                        mbar_arrive(fb);
+                        kend = i;
+                        uk = i + 1;
+                    }
+                }
+                if (i >= 1) {
+                    const int t = i - 1, s = t % SV;
+                    if (t >= SV &&
+                        !wait_bounded(smem_addr(&bar->empty_v[s]), ((t / SV) & 1) ^ 1, abort, hdr))
+                        break;
+                    const uint32_t fb = smem_addr(&bar->full_v[s]);
+                    if (t == kend) {
+                        mbar_arrive(fb);   // the PV issuer's end
+                        uv = t + 1;
                         break;
                     }
-                    const uint32_t fb = smem_addr(&full[s]);
                     mbar_arrive_expect_tx(fb, kStageBytes);
-                    const uint32_t dst = smem_addr((is_k ? sK : sV) + s * kStageBytes);
-                    const void *tmap = is_k ? static_cast<const void *>(&tmap_k)
-                                            : static_cast<const void *>(&tmap_v);
-                    const int pos0 = (t_begin + t) * kTileN;
-                    tma_load_3d(dst, tmap, 0, pos0, g, fb);
-                    tma_load_3d(dst + kBoxBytes, tmap, 64, pos0, g, fb);
-                    if (is_k)
-                        nk = t + 1;
-                    else
-                        nv = t + 1;
+                    const uint32_t dst = smem_addr(sV + s * kStageBytes);
+                    const int pos0 = bar->tile_of[t % kTileRing] * kTileN;
+                    tma_load_3d(dst, &tmap_v, 0, pos0, g, fb);
+                    tma_load_3d(dst + kBoxBytes, &tmap_v, 64, pos0, g, fb);
+                    nv = uv = t + 1;
                 }
-                if (!ok)
-                    break;
             }
             if (*abort) {
-                // let our own copies land before the CTA exits
-                for (int t = max(0, nk - SK); t < nk; ++t)
+                // let our own copies land before the CTA exits (those whose
+                // ring slot no later entry has taken)
+                for (int t = max(0, uk - SK); t < nk; ++t)
                     wait_drain(smem_addr(&bar->full_k[t % SK]), (t / SK) & 1);
-                for (int t = max(0, nv - SV); t < nv; ++t)
+                for (int t = max(0, uv - SV); t < nv; ++t)
                     wait_drain(smem_addr(&bar->full_v[t % SV]), (t / SV) & 1);
             }
         }
     } else if (warp == 0) {
-        // --------------------------- root node's scores out of S_0 (lanes 0..G-1)
+        // ------------------- root node's scores out of S_b, b the last block (lanes 0..G-1)
         if (rs_warp0) {
-            // one block only; one 16x256b load of lanes 0..15, the shape the softmax warps
+            // one 16x256b load of lanes 0..15, the shape the softmax warps
             // use: thread t holds lane t/4 (and 8 + t/4) at columns
             // 8j + 2(t%4) + {0, 1}, so threads 0..4G-1 hold the G root rows
+            const int bl = NB - 1;
             const int r = lane >> 2;          // root row of this thread (lanes 0..7)
             const bool mine = r < G;
             const int c0 = 2 * (lane & 3);
             float *dst_row = a.root_scores + (size_t)(g * G + (mine ? r : 0)) * a.n_ctx;
             const bool vec = ((reinterpret_cast<uintptr_t>(a.root_scores) | (uintptr_t)a.n_ctx * 4) &
                               7) == 0;
-            for (int t = 0; t < n_tiles; ++t) {
-                if (!warp_wait_bounded(smem_addr(&bar->s_full[0]), t & 1, abort, hdr))
+            for (int t = 0;; ++t) {
+                if (!warp_wait_bounded(smem_addr(&bar->s_full[bl]), t & 1, abort, hdr))
+                    break;
+                const int tile = bar->tile_of[t % kTileRing];
+                if (tile < 0)
                     break;
                 tc_fence_after();
-                const int pos0 = (t_begin + t) * kTileN;
+                const int pos0 = tile * kTileN;
                 uint32_t rr[64];
                 if (pos0 < a.n_ctx)
-                    tmem_ld16x256_x16(tmem + kSCol, rr);
-                // S_0 is read: QK of the next tile may overwrite it
+                    tmem_ld16x256_x16(tmem + kSCol + 128 * bl, rr);
+                // S_b is read: QK of the next tile may overwrite it
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0)
-                    mbar_arrive(smem_addr(&bar->s_free[0]));
+                    mbar_arrive(smem_addr(&bar->s_free[bl]));
                 if (pos0 >= a.n_ctx || !mine)
                     continue;   // a tile of the tree tail only, or not a root lane
 #pragma unroll
@@ -561,10 +904,21 @@ attn_t128_kernel(const __grid_constant__ CUtensorMap tmap_k,
                 const uint32_t idesc = idesc_bf16(kBlockM, kTileN, 0, 0);
                 const uint64_t kd0 = sdesc_sw128(smem_addr(sK), 16, 1024);
                 const uint64_t qd0 = sdesc_sw128(smem_addr(sQ1), 16, 1024);
-                for (int t = 0; t < n_tiles; ++t) {
+                for (int t = 0;; ++t) {
                     const int s = t % SK;
                     if (!wait_bounded(smem_addr(&bar->full_k[s]), (t / SK) & 1, abort, hdr))
                         break;
+                    if (bar->tile_of[t % kTileRing] < 0) {
+                        // no tile left: the readers of each S_b learn it from
+                        // a plain arrival, once they hold S_b(t-1)
+                        for (int b = 0; b < NB; ++b) {
+                            if (t > 0 &&
+                                !wait_bounded(smem_addr(&bar->s_free[b]), (t - 1) & 1, abort, hdr))
+                                break;
+                            mbar_arrive(smem_addr(&bar->s_full[b]));
+                        }
+                        break;
+                    }
                     // QK(t) enters the tensor queue after PV(t-2): the softmax
                     // warps wait for PV(t-2) before writing P^T(t-1), while
                     // S(t) is only read after they finish tile t-1.  PV(t)
@@ -609,10 +963,15 @@ attn_t128_kernel(const __grid_constant__ CUtensorMap tmap_k,
                 const uint64_t vd0 = sdesc_sw128(smem_addr(sV), kBoxBytes, 1024);
                 const uint64_t pd0 = sdesc_sw128(smem_addr(sP), 16, 1024);
                 const uint32_t p_half = (uint32_t)r_pad * 128;
-                for (int t = 0; t < n_tiles; ++t) {
+                for (int t = 0;; ++t) {
                     const int s = t % SV;
-                    if (!wait_bounded(smem_addr(&bar->full_v[s]), (t / SV) & 1, abort, hdr) ||
-                        !wait_bounded(smem_addr(&bar->sm_done), t & 1, abort, hdr))
+                    if (!wait_bounded(smem_addr(&bar->full_v[s]), (t / SV) & 1, abort, hdr))
+                        break;
+                    if (bar->tile_of[t % kTileRing] < 0) {
+                        mma_commit(smem_addr(&bar->o_final));   // after the last PV
+                        break;
+                    }
+                    if (!wait_bounded(smem_addr(&bar->sm_done), t & 1, abort, hdr))
                         break;
                     tc_fence_after();
                     const uint64_t vd = vd0 + (uint64_t)s * kStageStep;
@@ -625,8 +984,6 @@ attn_t128_kernel(const __grid_constant__ CUtensorMap tmap_k,
                         mma_ss_c<1>(tmem, vd + ((kk * 2048) >> 4),
                                     pd0 + (((kk >> 2) * p_half + (kk & 3) * 32) >> 4), idesc);
                     mma_commit(smem_addr(&bar->pv_done));
-                    if (t == n_tiles - 1)
-                        mma_commit(smem_addr(&bar->o_final));
                     mma_commit(smem_addr(&bar->empty_v[s]));
                     mbar_arrive(smem_addr(&bar->pv_issued[t & 1]));
                 }
@@ -658,18 +1015,15 @@ attn_t128_kernel(const __grid_constant__ CUtensorMap tmap_k,
         const uint32_t p_addr = smem_addr(sP);
         const uint32_t p_scratch = p_addr + (uint32_t)r_pad * 256;
         float mA = -INFINITY, mB = -INFINITY, lA = 0.f, lB = 0.f, qA = 0.f, qB = 0.f;
-        // root rows (rows 0..G-1) held by this thread and this warp (block 1
-        // only); the first lane of a row's quad copies its staged scores out
-        const bool rootA = b == 1 && vA && t128_row_of(nA, R) < G;
-        const bool rootB = b == 1 && vB && t128_row_of(nB, R) < G;
-        const bool rs_warp = t128_rs_block1(a, T) && __any_sync(0xffffffffu, rootA || rootB);
-        const bool rs_issue = rs_bytes != 0 && (lane & 3) == 0 && (rootA || rootB);
         bool ok = true;
-        for (int t = 0; t < n_tiles; ++t) {
+        for (int t = 0;; ++t) {
             if (!warp_wait_bounded(smem_addr(&bar->s_full[b]), t & 1, abort, hdr)) {
                 ok = false;
                 break;
             }
+            const int tile = bar->tile_of[t % kTileRing];
+            if (tile < 0)
+                break;
             tc_fence_after();
             uint32_t r[64];
             tmem_ld16x256_x16(s_addr, r);
@@ -679,66 +1033,7 @@ attn_t128_kernel(const __grid_constant__ CUtensorMap tmap_k,
             if (lane == 0)
                 mbar_arrive(smem_addr(&bar->s_free[b]));
             // raw scores; the scale (> 0) is applied inside the exponent
-            const int pos0 = (t_begin + t) * kTileN;
-            // the root node's rows leave their context scores, base 2, for the
-            // importance select
-            if (rs_warp && pos0 < a.n_ctx) {
-                if (rs_bytes != 0) {
-                    // staged in shared memory (one buffer per tile parity) and
-                    // written out by bulk copies, so that no global store sits
-                    // ahead of this warp's barrier arrivals
-                    const uint32_t buf =
-                        smem_addr(base + lay.rs_off) + (uint32_t)((t & 1) * G * kTileN * 4);
-                    if (rs_issue)
-                        bulk_wait_read<1>();   // the copy out of this buffer two tiles ago
-                    __syncwarp();
-#pragma unroll
-                    for (int h = 0; h < 2; ++h) {
-                        if (h ? rootB : rootA) {
-                            const uint32_t row = buf + (uint32_t)(t128_row_of(h ? nB : nA, R) *
-                                                                      kTileN * 4 +
-                                                                  c0 * 4);
-#pragma unroll
-                            for (int jj = 0; jj < 16; ++jj)
-                                st_shared_v2(row + 32 * jj,
-                                             __float_as_uint(__uint_as_float(r[4 * jj + 2 * h]) *
-                                                             a.scale_log2),
-                                             __float_as_uint(__uint_as_float(r[4 * jj + 2 * h + 1]) *
-                                                             a.scale_log2));
-                        }
-                    }
-                    fence_proxy_async_smem();
-                    __syncwarp();
-                    if (rs_issue) {
-                        const uint32_t bytes = (uint32_t)min(kTileN, a.n_ctx - pos0) * 4;
-#pragma unroll
-                        for (int h = 0; h < 2; ++h) {
-                            const int m = t128_row_of(h ? nB : nA, R);
-                            if (h ? rootB : rootA)
-                                bulk_store(a.root_scores + (size_t)(g * G + m) * a.n_ctx + pos0,
-                                           buf + (uint32_t)(m * kTileN * 4), bytes);
-                        }
-                        bulk_commit();
-                    }
-                } else {
-#pragma unroll
-                    for (int h = 0; h < 2; ++h) {
-                        if (h ? rootB : rootA) {
-                            float *dst = a.root_scores +
-                                         (size_t)(g * G + t128_row_of(h ? nB : nA, R)) * a.n_ctx;
-#pragma unroll
-                            for (int jj = 0; jj < 16; ++jj)
-#pragma unroll
-                                for (int e = 0; e < 2; ++e) {
-                                    const int pos = pos0 + 8 * jj + c0 + e;
-                                    if (pos < a.n_ctx)
-                                        dst[pos] =
-                                            __uint_as_float(r[4 * jj + 2 * h + e]) * a.scale_log2;
-                                }
-                        }
-                    }
-                }
-            }
+            const int pos0 = tile * kTileN;
             if (pos0 + kTileN > a.n_ctx) {
                 // visibility of this thread's 32 positions (entry k = 2 jj + e
                 // is position pos0 + 8 jj + c0 + e) for its two rows
@@ -761,9 +1056,9 @@ attn_t128_kernel(const __grid_constant__ CUtensorMap tmap_k,
                         r[4 * (k >> 1) + 2 + (k & 1)] = __float_as_uint(-INFINITY);
                 }
             }
-            // a row that has seen nothing yet takes this tile's max as its
-            // reference (its O^T column and l are still zero); afterwards
-            // the maxima are not needed
+            // a row that has seen nothing yet takes this tile's max, rounded
+            // up to an integer, as its reference (its O^T column and l are
+            // still zero); afterwards the maxima are not needed
             if (__any_sync(0xffffffffu, mA == -INFINITY || mB == -INFINITY)) {
                 const float xA = row_max(r, 0) * a.scale_log2;
                 const float xB = row_max(r, 2) * a.scale_log2;
@@ -772,9 +1067,9 @@ attn_t128_kernel(const __grid_constant__ CUtensorMap tmap_k,
                 yA = fmaxf(yA, __shfl_xor_sync(0xffffffffu, yA, 2));
                 yB = fmaxf(yB, __shfl_xor_sync(0xffffffffu, yB, 2));
                 if (mA == -INFINITY)
-                    mA = yA;
+                    mA = ceilf(yA);
                 if (mB == -INFINITY)
-                    mB = yB;
+                    mB = ceilf(yB);
             }
 
             uint32_t pA[16], pB[16];
@@ -803,8 +1098,6 @@ attn_t128_kernel(const __grid_constant__ CUtensorMap tmap_k,
             if (lane == 0)
                 mbar_arrive(smem_addr(&bar->sm_done));
         }
-        if (rs_issue)
-            bulk_wait_all();   // shared memory must outlive the copies out of it
         // ---- (m, l) of each row (four threads' partial sums), then O^T
 #pragma unroll
         for (int o = 1; o <= 2; o <<= 1) {
@@ -819,8 +1112,7 @@ attn_t128_kernel(const __grid_constant__ CUtensorMap tmap_k,
         if (__any_sync(0xffffffffu, over) && lane == 0)
             bar->overflow = 1;
         const int rows_all = a.n_tree * a.n_heads_q;
-        float *ws_o =
-            reinterpret_cast<float *>(reinterpret_cast<char *>(a.workspace) + kHeaderBytes);
+        float *ws_o = sy.part;
         float *ws_ml = ws_o + (size_t)n_split * rows_all * kD;
         // P^T row n -> output row of the head group
         auto orow_of = [&](int n) {
@@ -877,6 +1169,9 @@ attn_t128_kernel(const __grid_constant__ CUtensorMap tmap_k,
                                smem_addr(sK) + (uint32_t)(node * G * kD * 4), (uint32_t)(G * kD * 4));
                 bulk_commit();
                 bulk_wait_all();   // the ring must outlive the copies out of it
+                // the copies' writes, made by the async proxy, before the
+                // arrival below publishes them to the other splits
+                fence_proxy_async_global();
             }
         }
     }
@@ -887,287 +1182,52 @@ attn_t128_kernel(const __grid_constant__ CUtensorMap tmap_k,
         tc_fence_after();
         tmem_dealloc(tmem, kTmemCols);
     }
-    if (threadIdx.x == 0)
-        flags[(split * a.n_heads_kv + g) * gridDim.z + blockIdx.z] = bar->overflow;
-}
 
-// One split's partial (m, l, acc) of one query row, recomputed exactly in
-// fp32 from K and V by an online softmax over the split's visible
-// positions.  One warp; lane holds head dims 4 lane .. 4 lane + 3.  Used
-// only for splits whose flag says the kernel's fixed reference max ran out
-// of headroom, and for the splits that carry the weight of a row whose
-// weight sits on too few positions for one bf16 rounding of P.
-__device__ void split_partial_exact(const AttnArgs &a, unsigned long long anc, int g,
-                                    const float (&q4)[4], int p0, int p1, float &m, float &l,
-                                    float (&acc)[4])
-{
-    constexpr int kU = 8;   // positions per step: their loads and reductions overlap
-    const int lane = threadIdx.x & 31;
-    const __nv_bfloat16 *kh = a.k + (size_t)g * a.kv_cap * kD + 4 * lane;
-    const __nv_bfloat16 *vh = a.v + (size_t)g * a.kv_cap * kD + 4 * lane;
-    m = -INFINITY;
-    l = 0.f;
-#pragma unroll
-    for (int e = 0; e < 4; ++e)
-        acc[e] = 0.f;
-    for (int pos0 = p0; pos0 < p1; pos0 += kU) {
-        float sc[kU];
-        bool seen[kU];
-#pragma unroll
-        for (int u = 0; u < kU; ++u) {
-            const int pos = pos0 + u;
-            const int tp = pos - a.n_ctx;
-            seen[u] = pos < p1 && (tp < 0 || ((anc >> tp) & 1ull));
-            const uint2 kb = seen[u] ? *reinterpret_cast<const uint2 *>(kh + (size_t)pos * kD)
-                                     : make_uint2(0u, 0u);
-            const float2 k01 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&kb.x));
-            const float2 k23 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&kb.y));
-            sc[u] = q4[0] * k01.x + q4[1] * k01.y + q4[2] * k23.x + q4[3] * k23.y;
-        }
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1)
-#pragma unroll
-            for (int u = 0; u < kU; ++u)
-                sc[u] += __shfl_xor_sync(0xffffffffu, sc[u], o);
-        float mx = -INFINITY;
-#pragma unroll
-        for (int u = 0; u < kU; ++u) {
-            sc[u] = seen[u] ? sc[u] * a.scale_log2 : -INFINITY;
-            mx = fmaxf(mx, sc[u]);
-        }
-        if (mx == -INFINITY)
-            continue;
-        if (mx > m) {
-            const float f = m == -INFINITY ? 0.f : exp2f(m - mx);
-            l *= f;
-#pragma unroll
-            for (int e = 0; e < 4; ++e)
-                acc[e] *= f;
-            m = mx;
-        }
-#pragma unroll
-        for (int u = 0; u < kU; ++u) {
-            if (!seen[u])
-                continue;
-            const float pw = exp2f(sc[u] - m);
-            const uint2 vb = *reinterpret_cast<const uint2 *>(vh + (size_t)(pos0 + u) * kD);
-            const float2 v01 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&vb.x));
-            const float2 v23 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&vb.y));
-            l += pw;
-            acc[0] += pw * v01.x;
-            acc[1] += pw * v01.y;
-            acc[2] += pw * v23.x;
-            acc[3] += pw * v23.y;
-        }
+    // ---- combine.  Once every split of this (head, group) has arrived,
+    // each folds its share of the group's rows (rows split, split +
+    // n_split, ...; one warp each).  The launch is cooperative, so all
+    // splits are resident and the wait ends.
+    const int n_gz = a.n_heads_kv * gridDim.z;
+    int32_t *ctr = sy.sync + 4 * gz;
+    if (threadIdx.x == 0) {
+        sy.flags[(size_t)split * n_gz + gz] = bar->overflow;
+        __threadfence();   // partials, flag and owner entries before the arrival
+        atomicAdd(&ctr[1], 1);
+        wait_count_bounded(&ctr[1], n_split, abort, hdr);
+    }
+    __syncthreads();
+    if (!*abort) {
+        for (int m = split + warp * n_split; m < R; m += (kThreads / 32) * n_split)
+            t128_combine_row(a, masks, (node0 + m / G) * a.n_heads_q + g * G + m % G, g, gz, n_gz,
+                             n_split, sy);
+    }
+    __syncthreads();
+    if (threadIdx.x == 0 && atomicAdd(&ctr[2], 1) == n_split - 1) {
+        // every split of the group is past its wait and done taking tiles:
+        // the counters go back to zero for the next call
+        atomicExch(&ctr[0], 0);
+        atomicExch(&ctr[1], 0);
+        atomicExch(&ctr[2], 0);
     }
 }
 
-// One warp per output row: out = sum_s 2^(m_s - M) acc_s / sum_s 2^(m_s - M) l_s
-// over the splits' partials.  Recomputed exactly instead of read: splits
-// flagged for overflow, and, on a row whose effective number of positions
-// may be below kNeffMin (L^2 < kNeffMin * sum_s c_s^2 q_s with c_s =
-// 2^(m_s - M)), every split s whose c_s^2 q_s is above L^2 / (kNeffMin *
-// n_split) -- the remaining splits then add up to a bound of at least
-// kNeffMin on their own.
-__global__ void __launch_bounds__(256)
-attn_t128_combine_kernel(AttnArgs a, TreeMasks masks, int n_split, int split_positions,
-                         const int32_t *__restrict__ flags, int n_flag_groups)
+struct T128WsLayout {
+    size_t sync, part, flags, owner, total;
+};
+
+// header | counters (zero between calls) | partials | flags | owner map
+T128WsLayout t128_ws_layout(const AttnPlan &p, int n_heads_q, int n_heads_kv, int n_ctx,
+                            int n_tree)
 {
-    const int rows_all = a.n_tree * a.n_heads_q;
-    const int row = blockIdx.x * 8 + (threadIdx.x >> 5);
-    const int lane = threadIdx.x & 31;
-    // launched early (programmatic dependent launch): the split partials
-    // are complete only once the split grid has finished
-    grid_dependency_wait();
-    if (row >= rows_all)
-        return;
-    const int head = row % a.n_heads_q, node = row / a.n_heads_q;
-    const int g = head / (a.n_heads_q / a.n_heads_kv);
-    const float *ws_o =
-        reinterpret_cast<const float *>(reinterpret_cast<const char *>(a.workspace) + kHeaderBytes);
-    const float *ws_ml = ws_o + (size_t)n_split * rows_all * kD;
-    auto mlq_of = [&](int s) {
-        return __ldcg(reinterpret_cast<const float4 *>(ws_ml + ((size_t)s * rows_all + row) * 4));
-    };
-
-    // One round trip for the common case (at most kFastSplits splits): lane
-    // s reads split s's (m, l, q) and flag while every lane also reads its
-    // four columns of every split's acc, all loads in flight together.
-    auto flagged = [&](int s) {
-        if (flags == nullptr)
-            return false;
-        bool f = false;
-        for (int z = 0; z < n_flag_groups; ++z)
-            f = f || flags[(s * a.n_heads_kv + g) * n_flag_groups + z] != 0;
-        return f;
-    };
-    constexpr int kFastSplits = 24;
-    const bool fast = n_split <= kFastSplits;
-    float4 xs[kFastSplits];
-    float4 my = make_float4(-INFINITY, 0.f, 0.f, 0.f);
-    bool my_f = false;
-    if (fast) {
-        if (lane < n_split) {
-            my = mlq_of(lane);
-            my_f = flagged(lane);
-        }
-#pragma unroll
-        for (int u = 0; u < kFastSplits; ++u)
-            xs[u] = u < n_split ? __ldcg(reinterpret_cast<const float4 *>(
-                                      ws_o + ((size_t)u * rows_all + row) * kD + 4 * lane))
-                                : make_float4(0.f, 0.f, 0.f, 0.f);
-    }
-
-    // M, and L and the bound's denominator, over the splits that are not
-    // flagged
-    bool any = false;
-    float M = -INFINITY;
-    if (fast) {
-        any = my_f;
-        if (!my_f)
-            M = my.x;
-    } else {
-        for (int s = lane; s < n_split; s += 32) {
-            const bool f = flagged(s);
-            any |= f;
-            if (!f)
-                M = fmaxf(M, mlq_of(s).x);
-        }
-    }
-    any = __any_sync(0xffffffffu, any);
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1)
-        M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
-    // L^2 and the q sums reach 2^126 times the splits squared: the count is
-    // formed in fp64
-    double Lp = 0.0, Qp = 0.0;
-    if (M != -INFINITY) {
-        if (fast) {
-            if (!my_f && my.x != -INFINITY) {
-                const double c = (double)exp2f(my.x - M);
-                Lp = c * (double)my.y;
-                Qp = c * c * (double)my.z;
-            }
-        } else {
-            for (int s = lane; s < n_split; s += 32) {
-                if (flagged(s))
-                    continue;
-                const float4 x = mlq_of(s);
-                const double c = x.x == -INFINITY ? 0.0 : (double)exp2f(x.x - M);
-                Lp += c * (double)x.y;
-                Qp += c * c * (double)x.z;
-            }
-        }
-    }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-        Lp += __shfl_xor_sync(0xffffffffu, Lp, o);
-        Qp += __shfl_xor_sync(0xffffffffu, Qp, o);
-    }
-    const bool peaked = Lp * Lp < (double)kNeffMin * Qp;   // uniform across the warp
-    const double heavy = Lp * Lp / ((double)kNeffMin * n_split);
-
-    float acc[4] = {0.f, 0.f, 0.f, 0.f};
-    float L = 0.f;
-    if (!any && !peaked && fast) {
-        // every partial is used as it is: lane s's weight 2^(m_s - M) and
-        // its weighted l, passed to every lane
-        const float w_my = my.x == -INFINITY ? 0.f : exp2f(my.x - M);
-        const float wl_my = w_my * my.y;
-#pragma unroll
-        for (int u = 0; u < kFastSplits; ++u) {
-            if (u >= n_split)
-                break;
-            const float w = __shfl_sync(0xffffffffu, w_my, u);
-            L += __shfl_sync(0xffffffffu, wl_my, u);
-            acc[0] += w * xs[u].x;
-            acc[1] += w * xs[u].y;
-            acc[2] += w * xs[u].z;
-            acc[3] += w * xs[u].w;
-        }
-    } else if (!any && !peaked) {
-        // every partial is used as it is; M is known, so the splits are
-        // summed in batches of kB whose loads are in flight together
-        constexpr int kB = 9;
-        for (int s0 = 0; s0 < n_split; s0 += kB) {
-            float4 mlq[kB], x[kB];
-#pragma unroll
-            for (int u = 0; u < kB; ++u) {
-                const int s = s0 + u;
-                if (s < n_split) {
-                    mlq[u] = mlq_of(s);
-                    x[u] = __ldcg(reinterpret_cast<const float4 *>(
-                        ws_o + ((size_t)s * rows_all + row) * kD + 4 * lane));
-                } else {
-                    mlq[u] = make_float4(-INFINITY, 0.f, 0.f, 0.f);
-                    x[u] = make_float4(0.f, 0.f, 0.f, 0.f);
-                }
-            }
-#pragma unroll
-            for (int u = 0; u < kB; ++u) {
-                const float w = mlq[u].x == -INFINITY ? 0.f : exp2f(mlq[u].x - M);
-                L += w * mlq[u].y;
-                acc[0] += w * x[u].x;
-                acc[1] += w * x[u].y;
-                acc[2] += w * x[u].z;
-                acc[3] += w * x[u].w;
-            }
-        }
-    } else {
-        // fold the splits one by one into a running (Mr, L, acc), the
-        // flagged and the heavy ones recomputed
-        const uint2 qb = *reinterpret_cast<const uint2 *>(a.q + (size_t)row * kD + 4 * lane);
-        const float2 q01 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&qb.x));
-        const float2 q23 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&qb.y));
-        const float q4[4] = {q01.x, q01.y, q23.x, q23.y};
-        const int total = a.n_ctx + a.n_tree;
-        float Mr = -INFINITY;
-        for (int s = 0; s < n_split; ++s) {
-            float ms, ls, as[4];
-            const float4 x4 = mlq_of(s);
-            bool exact = flagged(s);
-            if (!exact && peaked && x4.x != -INFINITY) {
-                const double c = (double)exp2f(x4.x - M);
-                exact = c * c * (double)x4.z > heavy;
-            }
-            if (exact) {
-                const int p0 = s * split_positions;
-                const int p1 = min(p0 + split_positions, total);
-                split_partial_exact(a, masks.anc[node], g, q4, p0, p1, ms, ls, as);
-            } else {
-                const float4 x = __ldcg(reinterpret_cast<const float4 *>(
-                    ws_o + ((size_t)s * rows_all + row) * kD + 4 * lane));
-                ms = x4.x;
-                ls = x4.y;
-                as[0] = x.x;
-                as[1] = x.y;
-                as[2] = x.z;
-                as[3] = x.w;
-            }
-            if (ms == -INFINITY)
-                continue;
-            const float Mn = fmaxf(Mr, ms);
-            const float fa = Mr == -INFINITY ? 0.f : exp2f(Mr - Mn);
-            const float fb = exp2f(ms - Mn);
-            L = L * fa + ls * fb;
-#pragma unroll
-            for (int e = 0; e < 4; ++e)
-                acc[e] = acc[e] * fa + as[e] * fb;
-            Mr = Mn;
-        }
-    }
-    const float inv = 1.f / L;
-    *reinterpret_cast<float4 *>(a.out + (size_t)row * kD + 4 * lane) =
-        make_float4(acc[0] * inv, acc[1] * inv, acc[2] * inv, acc[3] * inv);
-}
-
-// Split partials (acc fp32 [n_split, T*Hq, D], then (m, l, q, 0) fp32
-// [n_split, T*Hq, 4]) after the header, then one int32 overflow flag per
-// (split, KV head).
-
-size_t flags_offset(int n_split, int n_heads_q, int n_tree)
-{
-    return kHeaderBytes + align_up(attn_exact_partial_bytes(n_split, n_heads_q, n_tree), 256);
+    const size_t n_gz = (size_t)n_heads_kv * p.node_groups;
+    const size_t n_tiles = (size_t)(n_ctx + n_tree + kTileN - 1) / kTileN;
+    T128WsLayout L;
+    L.sync = kHeaderBytes;
+    L.part = L.sync + align_up(n_gz * 4 * sizeof(int32_t), 256);
+    L.flags = L.part + align_up((size_t)p.n_split * n_tree * n_heads_q * (kD + 4) * sizeof(float), 256);
+    L.owner = L.flags + align_up((size_t)p.n_split * n_gz * sizeof(int32_t), 256);
+    L.total = L.owner + align_up(n_gz * n_tiles, 256);
+    return L;
 }
 
 }  // namespace
@@ -1175,8 +1235,13 @@ size_t flags_offset(int n_split, int n_heads_q, int n_tree)
 size_t attn_t128_workspace_bytes(int n_heads_q, int n_heads_kv, int n_ctx, int n_tree, int num_sms)
 {
     const AttnPlan p = attn_t128_plan(n_heads_q, n_heads_kv, n_ctx, n_tree, num_sms);
-    return flags_offset(p.n_split, n_heads_q, n_tree) +
-           align_up((size_t)p.n_split * n_heads_kv * p.node_groups * sizeof(int32_t), 256);
+    return t128_ws_layout(p, n_heads_q, n_heads_kv, n_ctx, n_tree).total;
+}
+
+size_t attn_t128_zeroed_bytes(int n_heads_q, int n_heads_kv, int n_ctx, int n_tree, int num_sms)
+{
+    const AttnPlan p = attn_t128_plan(n_heads_q, n_heads_kv, n_ctx, n_tree, num_sms);
+    return t128_ws_layout(p, n_heads_q, n_heads_kv, n_ctx, n_tree).part;
 }
 
 bool attn_t128_eligible(int n_heads_q, int n_heads_kv, int head_dim, int n_ctx, int n_tree)
@@ -1196,11 +1261,15 @@ AttnPlan attn_t128_plan(int n_heads_q, int n_heads_kv, int n_ctx, int n_tree, in
     p.node_groups = rows <= kMaxRows ? 1 : (rows + kBlockM - 1) / kBlockM;
     p.nodes_per_group = (n_tree + p.node_groups - 1) / p.node_groups;
     p.node_groups = (n_tree + p.nodes_per_group - 1) / p.nodes_per_group;
+    // one CTA per SM; the splits of a (head, group) take tiles at run time,
+    // each starting with its own, so there are at most as many as tiles
+    // (and at most 255: the owner map holds a byte per tile)
     const int n_tiles = (n_ctx + n_tree + kTileN - 1) / kTileN;
     int want = num_sms / (n_heads_kv * p.node_groups);
-    want = want < 1 ? 1 : (want > n_tiles ? n_tiles : want);
-    p.tiles_per_split = (n_tiles + want - 1) / want;
-    p.n_split = (n_tiles + p.tiles_per_split - 1) / p.tiles_per_split;
+    want = want < 1 ? 1 : want;
+    want = want > n_tiles ? n_tiles : want;
+    p.n_split = want > 255 ? 255 : want;
+    p.tiles_per_split = (n_tiles + p.n_split - 1) / p.n_split;   // on average
     return p;
 }
 
@@ -1215,65 +1284,44 @@ cudaError_t attn_t128_launch(const AttnArgs &a, const TreeMasks &masks, int num_
         return cudaErrorInvalidValue;
     // the first node group is the largest and holds the root node
     const int T0 = p.nodes_per_group;
-    const Layout lay = t128_layout((a.n_heads_q / a.n_heads_kv) * T0, t128_rs_bytes(a, T0));
+    const Layout lay = t128_layout((a.n_heads_q / a.n_heads_kv) * T0);
     static const cudaError_t attr = cudaFuncSetAttribute(
         attn_t128_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemLimit);
     if (attr != cudaSuccess)
         return attr;
-    int32_t *flags = reinterpret_cast<int32_t *>(
-        reinterpret_cast<char *>(a.workspace) + flags_offset(p.n_split, a.n_heads_q, a.n_tree));
-    cudaError_t e;
-    if (p.node_groups > 1 && p.node_groups <= 8) {
-        // the node groups of one (split, head) stream the same K/V tiles: as
-        // one cluster they start together on one GPC, so that the second
-        // read of each tile finds it in L2
-        cudaLaunchConfig_t cfg = {};
-        cfg.gridDim = dim3(p.n_split, a.n_heads_kv, p.node_groups);
-        cfg.blockDim = dim3(kThreads);
-        cfg.dynamicSmemBytes = lay.smem_bytes;
-        cfg.stream = stream;
-        cudaLaunchAttribute attr_c[1];
-        attr_c[0].id = cudaLaunchAttributeClusterDimension;
-        attr_c[0].val.clusterDim.x = 1;
-        attr_c[0].val.clusterDim.y = 1;
-        attr_c[0].val.clusterDim.z = p.node_groups;
-        cfg.attrs = attr_c;
-        cfg.numAttrs = 1;
-        e = cudaLaunchKernelEx(&cfg, attn_t128_kernel, mk, mv, a, masks, p.tiles_per_split,
-                               p.n_split, p.nodes_per_group, flags);
-        if (e == cudaSuccess)
-            e = cudaGetLastError();
-    } else {
-        attn_t128_kernel<<<dim3(p.n_split, a.n_heads_kv, p.node_groups), kThreads, lay.smem_bytes,
-                           stream>>>(mk, mv, a, masks, p.tiles_per_split, p.n_split,
-                                     p.nodes_per_group, flags);
+    const T128WsLayout wl = t128_ws_layout(p, a.n_heads_q, a.n_heads_kv, a.n_ctx, a.n_tree);
+    char *ws = reinterpret_cast<char *>(a.workspace);
+    T128Sync sy;
+    sy.sync = reinterpret_cast<int32_t *>(ws + wl.sync);
+    sy.part = reinterpret_cast<float *>(ws + wl.part);
+    sy.flags = reinterpret_cast<int32_t *>(ws + wl.flags);
+    sy.owner = reinterpret_cast<uint8_t *>(ws + wl.owner);
+    // cooperative: the splits of a head wait for one another before the
+    // combine, so every CTA must be resident at once (one per SM)
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(p.n_split, a.n_heads_kv, p.node_groups);
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = lay.smem_bytes;
+    cfg.stream = stream;
+    cudaLaunchAttribute at[1];
+    at[0].id = cudaLaunchAttributeCooperative;
+    at[0].val.cooperative = 1;
+    cfg.attrs = at;
+    cfg.numAttrs = 1;
+    cudaError_t e = cudaLaunchKernelEx(&cfg, attn_t128_kernel, mk, mv, a, masks, p.n_split,
+                                       p.nodes_per_group, sy);
+    if (e == cudaSuccess)
         e = cudaGetLastError();
-    }
     if (e != cudaSuccess)
         return e;
     count_launches(1);
-    return attn_exact_combine_launch(a, masks, p.n_split, p.tiles_per_split * kTileN, flags,
-                                     p.node_groups, stream);
+    return cudaSuccess;
 }
 
 bool attn_t128_leaves_root_scores(const AttnArgs &a)
 {
     const AttnPlan p = attn_t128_plan(a.n_heads_q, a.n_heads_kv, a.n_ctx, a.n_tree, 148);
-    return t128_rs_warp0(a, p.nodes_per_group) || t128_rs_block1(a, p.nodes_per_group);
-}
-
-size_t attn_exact_partial_bytes(int n_split, int n_heads_q, int n_tree)
-{
-    return (size_t)n_split * n_tree * n_heads_q * (kD + 4) * sizeof(float);
-}
-
-cudaError_t attn_exact_combine_launch(const AttnArgs &a, const TreeMasks &masks, int n_split,
-                                      int split_positions, const int32_t *flags,
-                                      int n_flag_groups, cudaStream_t stream)
-{
-    const int rows_all = a.n_tree * a.n_heads_q;
-    return launch_pdl(attn_t128_combine_kernel, dim3((rows_all + 7) / 8), dim3(256), 0, stream, a,
-                      masks, n_split, split_positions, flags, n_flag_groups);
+    return t128_rs_warp0(a, p.nodes_per_group);
 }
 
 }  // namespace ts

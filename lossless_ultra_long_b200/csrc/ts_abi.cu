@@ -13,8 +13,7 @@ static std::atomic<unsigned long long> g_launches{0};
 void count_launches(unsigned n) { g_launches.fetch_add(n, std::memory_order_relaxed); }
 }  // namespace ts
 
-namespace {
-
+namespace ts {
 int current_num_sms()
 {
     int dev = 0, n = 0;
@@ -25,6 +24,11 @@ int current_num_sms()
     }
     return n;
 }
+}  // namespace ts
+
+namespace {
+
+using ts::current_num_sms;
 
 bool aligned(const void *p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 

@@ -87,6 +87,13 @@ struct AttnArgs {
 
 size_t attn_workspace_bytes(int n_heads_q, int n_heads_kv, int head_dim, int n_ctx, int n_tree,
                             int num_sms);
+// Leading bytes of that workspace (header included) that must be zero when
+// a call starts (every call leaves them zero, unless it recorded a
+// device-side error).
+size_t attn_workspace_zeroed_bytes(int n_heads_q, int n_heads_kv, int head_dim, int n_ctx,
+                                   int n_tree, int num_sms);
+// SM count of the current device (148 when none can be queried).
+int current_num_sms();
 // Host-side checks of a verify-attention call's arguments (everything but
 // the workspace): TS_OK or the status the call returns.
 int attn_validate(const void *q, const void *k_cache, const void *v_cache, int64_t kv_cap,

@@ -267,7 +267,8 @@ def test_select_llama8b_100k_spiked(oracle_mod):
 def test_select_from_verify_attention_scores(oracle_mod, hq, hkv, d, n_ctx, t, n_sink, budget):
     """The verify attention leaves the root node's scores; the select run on
     them gives the oracle's importance and selection (same bars as the
-    select's own score pass), and the attention output is unchanged."""
+    select's own score pass), and the attention output is unchanged (up to
+    fp32 summation order)."""
     w = I.Workload("rs", hq, hkv, d, n_ctx, t, n_sink=n_sink, budget=budget,
                    seed=n_ctx + hq + t)
     q = I.gen_q(w)
@@ -279,7 +280,9 @@ def test_select_from_verify_attention_scores(oracle_mod, hq, hkv, d, n_ctx, t, n
     idx, kp, vp, sc = L.kv_select_from_scores(rs, dk, dv, n_ctx, n_sink, budget,
                                               want_scores=True)
     torch.cuda.synchronize()
-    assert torch.equal(plain, fused)
+    # the splits take KV tiles at run time, so two calls fold the same
+    # bf16 weights in different fp32 orders: equal up to summation order
+    assert (plain - fused).abs().max().item() <= 2e-5
     # root scores: log2(e) * q[0,h] . k[g,n] / sqrt(D) at sampled positions
     qf, kf = I.bf16_bits_to_f32(q).astype(np.float64), I.bf16_bits_to_f32(k).astype(np.float64)
     rng = np.random.default_rng(n_ctx)
