@@ -793,6 +793,10 @@ attn_t128_kernel(const __grid_constant__ CUtensorMap tmap_k,
             int nxt = tile_at(n_split + atomicAdd(&ctr[0], 1));   // used one step later
             int kend = -1;        // ring index of the end marker
             uint8_t *owner = sy.owner + (size_t)gz * n_tiles_all;
+            // K and V are read once per call: their L2 lines go first, so
+            // that the partials, the root scores and what the next kernels
+            // read stay in L2
+            const uint64_t pol = l2_evict_first_policy();
             // step i issues K(i), then V(i - 1): K is consumed a whole softmax
             // pass before V, and each load waits only for its own ring slot
             for (int i = 0;; ++i) {
@@ -807,8 +811,8 @@ attn_t128_kernel(const __grid_constant__ CUtensorMap tmap_k,
                         owner[cur] = (uint8_t)split;
                         mbar_arrive_expect_tx(fb, kStageBytes);
                         const uint32_t dst = smem_addr(sK + s * kStageBytes);
-                        tma_load_3d(dst, &tmap_k, 0, cur * kTileN, g, fb);
-                        tma_load_3d(dst + kBoxBytes, &tmap_k, 64, cur * kTileN, g, fb);
+                        tma_load_3d_hint(dst, &tmap_k, 0, cur * kTileN, g, fb, pol);
+                        tma_load_3d_hint(dst + kBoxBytes, &tmap_k, 64, cur * kTileN, g, fb, pol);
                         nk = uk = i + 1;
                         cur = nxt;
                         if (cur >= 0)
@@ -835,8 +839,8 @@ attn_t128_kernel(const __grid_constant__ CUtensorMap tmap_k,
                     mbar_arrive_expect_tx(fb, kStageBytes);
                     const uint32_t dst = smem_addr(sV + s * kStageBytes);
                     const int pos0 = bar->tile_of[t % kTileRing] * kTileN;
-                    tma_load_3d(dst, &tmap_v, 0, pos0, g, fb);
-                    tma_load_3d(dst + kBoxBytes, &tmap_v, 64, pos0, g, fb);
+                    tma_load_3d_hint(dst, &tmap_v, 0, pos0, g, fb, pol);
+                    tma_load_3d_hint(dst + kBoxBytes, &tmap_v, 64, pos0, g, fb, pol);
                     nv = uv = t + 1;
                 }
             }
