@@ -32,7 +32,8 @@
  *    256-byte aligned, zero-filled once by the caller before first use.
  *    Every call returns the counters and tickets it relies on to zero
  *    before it ends; the rest of the workspace is scratch that each call
- *    writes before it reads.
+ *    writes before it reads.  After a call that recorded a device-side
+ *    error in the status word, zero-fill the workspace again.
  *    Concurrent calls need distinct workspaces.
  *  - bf16 tensors are raw IEEE bfloat16 bit patterns; every device pointer
  *    must be 16-byte aligned.
@@ -105,6 +106,13 @@ TS_API int ts_version(void);
  *  softmax_scale  finite, usually 1/sqrt(D).
  *  out          device fp32 [n_tree, Hq, D], written entirely.
  *  workspace    device, >= ts_tree_verify_attn_workspace_size(...) bytes.
+ *
+ * With head_dim 128 and n_ctx >= 2048 the split-KV kernel hands tiles to
+ * its splits at run time, so two calls on the same inputs may fold the
+ * same bf16 weights in a different fp32 order: results agree to about
+ * 1e-5, not bit for bit.  That kernel is one cooperative launch (every CTA
+ * resident at once, one per SM); a launch the device cannot co-schedule
+ * returns TS_ERR_CUDA.
  */
 TS_API size_t ts_tree_verify_attn_workspace_size(int n_heads_q, int n_heads_kv, int head_dim,
                                           int n_ctx, int n_tree);
@@ -128,7 +136,8 @@ TS_API int ts_tree_verify_attn(const void *q, const void *k_cache, const void *v
  *  - Limit: a problem whose ts_tree_verify_attn_workspace_size() exceeds
  *    TS_NOALLOC_SCRATCH_BYTES is rejected with TS_ERR_SCRATCH_LIMIT before
  *    anything is launched (16 MiB covers, e.g., 32/8 heads, D 128, a 40-node
- *    tree at any context length).
+ *    tree up to about 73 million context positions: the scratch holds the
+ *    split partials and one byte per 128-position tile and KV head).
  *  - Set-up: the first call on a device (and the first after that device's
  *    context was reset) looks up the array's device address
  *    (cudaGetSymbolAddress, with the device current) and keeps it for that
