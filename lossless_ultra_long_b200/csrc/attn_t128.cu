@@ -59,8 +59,10 @@
 // never moves, so the softmax warps need no per-tile agreement with each
 // other and no per-tile maximum at all.  Being an integer, it scales every
 // weight by an exact power of two: the bf16-rounded weight of a position is
-// the same whichever split streams it, so the run-time hand-out of tiles to
-// splits moves results by fp32 summation order only.  fp32 has room
+// almost always the same whichever split streams it (the fp32 exponent
+// argument, formed against the split's reference, can round across a bf16
+// boundary the other way), so the run-time hand-out of tiles to splits
+// moves results by fp32 summation order and such rare flips (~1e-4).  fp32 has room
 // for it: a row's weights are at most its sum l, and while l <= 2^63 the
 // accumulated O^T stays below 2^63 * max|V|, far from overflow (a score
 // rise of about 44 nats inside one split would be needed to exceed it).  A
