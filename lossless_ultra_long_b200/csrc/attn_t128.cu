@@ -158,6 +158,7 @@ struct Bars {
 
 struct Aux {
     Bars bar;
+    unsigned long long anc[TS_MAX_TREE];   // the tree's ancestor masks, read on the tail tiles
 };
 constexpr size_t kAuxBytes = (sizeof(Aux) + 1023) / 1024 * 1024;
 
@@ -213,6 +214,37 @@ __host__ __device__ inline Layout t128_layout(int rows)
     L.aux_off = L.v_off + (size_t)L.stages_v * kStageBytes;
     L.smem_bytes = 1024 + L.aux_off + kAuxBytes;
     return L;
+}
+
+// Visibility of a thread's 32 positions of a tile that reaches the tree tail
+// (entry k = 2 jj + e is position pos0 + 8 jj + c0 + e) for a row with
+// ancestor mask anc: the tile's 128 positions as two 64-bit words (bit p
+// set iff position pos0 + p is a context position, p < d = n_ctx - pos0, or
+// a node of the row's root path, tree bit p - d of anc), shifted down by c0,
+// then bits 8 jj + e gathered into bit 2 jj + e.
+__device__ __noinline__ uint32_t t128_tail_vis(unsigned long long anc, int d, int n_tree, int c0)
+{
+    const unsigned long long tree = n_tree >= 64 ? anc : (anc & ((1ull << n_tree) - 1ull));
+    uint32_t vis = 0u;
+#pragma unroll
+    for (int w = 0; w < 2; ++w) {
+        const int nctx = min(max(d - 64 * w, 0), 64);
+        unsigned long long m = nctx == 64 ? ~0ull : ((1ull << nctx) - 1ull);
+        const int sft = 64 * w - d;   // tree bit of the word's bit 0
+        if (sft >= 0) {
+            if (sft < 64)
+                m |= tree >> sft;
+        } else if (-sft < 64) {
+            m |= tree << (-sft);
+        }
+        // bits 8 j and 8 j + 1 (j = 0..7) of the shifted word -> bits 2 j, 2 j + 1
+        unsigned long long x = (m >> c0) & 0x0303030303030303ull;
+        x = (x | (x >> 6)) & 0x000F000F000F000Full;
+        x = (x | (x >> 12)) & 0x000000FF000000FFull;
+        x = (x | (x >> 24)) & 0xFFFFull;
+        vis |= (uint32_t)x << (16 * w);
+    }
+    return vis;
 }
 
 // P = 2^(x * scale - m) for the 32 scores a thread holds of row A
@@ -768,6 +800,11 @@ attn_t128_kernel(const __grid_constant__ CUtensorMap tmap_k,
         fence_proxy_async_smem();
     } else if (warp >= 8 && warp < 12) {
         named_bar_arrive(kBarQLoads, kQLoadThreads);   // one block: no rows to load
+    } else if (warp == 0) {
+        // the ancestor masks into shared memory: the tail tiles read them per
+        // thread, which the kernel-parameter bank would serialise
+        for (int i = lane; i < a.n_tree; i += 32)
+            aux->anc[i] = masks.anc[i];
     }
     if (warp != 3) {
         tc_fence_before();
@@ -1043,17 +1080,12 @@ attn_t128_kernel(const __grid_constant__ CUtensorMap tmap_k,
             if (pos0 + kTileN > a.n_ctx) {
                 // visibility of this thread's 32 positions (entry k = 2 jj + e
                 // is position pos0 + 8 jj + c0 + e) for its two rows
-                const unsigned long long ancA = masks.anc[node0 + (vA ? t128_row_of(nA, R) / G : 0)];
-                const unsigned long long ancB = masks.anc[node0 + (vB ? t128_row_of(nB, R) / G : 0)];
-                uint32_t visA = 0u, visB = 0u;
-#pragma unroll 1
-                for (int k = 0; k < 32; ++k) {
-                    const int pos = pos0 + 8 * (k >> 1) + c0 + (k & 1);
-                    const int tp = pos - a.n_ctx;
-                    const bool in = pos < total;
-                    visA |= (uint32_t)(in && (tp < 0 || ((ancA >> tp) & 1ull))) << k;
-                    visB |= (uint32_t)(in && (tp < 0 || ((ancB >> tp) & 1ull))) << k;
-                }
+                const uint32_t visA =
+                    t128_tail_vis(aux->anc[node0 + (vA ? t128_row_of(nA, R) / G : 0)],
+                                  a.n_ctx - pos0, a.n_tree, c0);
+                const uint32_t visB =
+                    t128_tail_vis(aux->anc[node0 + (vB ? t128_row_of(nB, R) / G : 0)],
+                                  a.n_ctx - pos0, a.n_tree, c0);
 #pragma unroll
                 for (int k = 0; k < 32; ++k) {
                     if (!((visA >> k) & 1u))
