@@ -923,6 +923,15 @@ attn_t128_kernel(const __grid_constant__ CUtensorMap tmap_k,
                     mbar_arrive(smem_addr(&bar->s_free[bl]));
                 if (pos0 >= a.n_ctx || !mine)
                     continue;   // a tile of the tree tail only, or not a root lane
+                if (vec && pos0 + kTileN <= a.n_ctx) {
+                    // a whole context tile: no bounds, one 8-byte store per pair
+                    float2 *dst2 = reinterpret_cast<float2 *>(dst_row + pos0 + c0);
+#pragma unroll
+                    for (int jj = 0; jj < 16; ++jj)
+                        dst2[4 * jj] = make_float2(__uint_as_float(rr[4 * jj]) * a.scale_log2,
+                                                   __uint_as_float(rr[4 * jj + 1]) * a.scale_log2);
+                    continue;
+                }
 #pragma unroll
                 for (int jj = 0; jj < 16; ++jj) {
                     const int p = pos0 + 8 * jj + c0;
