@@ -611,10 +611,12 @@ def run_breakdown(args):
 def sweep_14b(torch, L, I, dev, hbm, tflops, warmup=10, calls=50):
     """The 14B GQA roofline sweep: Hq 40, Hkv 8, D 128, contexts 4K-131K and
     trees of 4 (a chain), 13 and 40 nodes.  Per point: the verify call's mean
-    device time over back-to-back calls that rotate over enough copies of the
-    KV cache that each call reads from HBM (3 x L2 at least), its algorithmic
-    bytes and flops, achieved GB/s and TFLOP/s and their fractions of the
-    measured peaks.  Inputs: seeded N(0, 1) bf16 drawn on the device."""
+    device time over back-to-back calls, replayed from a CUDA graph (so that
+    host launch cost does not time the short calls), that rotate over enough
+    copies of the KV cache that each call reads from HBM (3 x L2 at least),
+    its algorithmic bytes and flops, achieved GB/s and TFLOP/s and their
+    fractions of the measured peaks.  Inputs: seeded N(0, 1) bf16 drawn on
+    the device."""
     l2 = 126 * 2 ** 20
     points = []
     gen = torch.Generator(device=dev)
@@ -642,7 +644,9 @@ def sweep_14b(torch, L, I, dev, hbm, tflops, warmup=10, calls=50):
                 it[0] += 1
                 L.tree_verify_attn(q, k, v, n_ctx, parent, out=out, workspace=ws)
 
-            us = _time_call(torch, call, warmup, calls)
+            # one graph of a whole number of rotations, at least 10 calls
+            per_graph = n_sets * max(1, -(-10 // n_sets))
+            us = _time_call_graph(torch, call, warmup, calls, per_graph=per_graph)
             byts = attn_bytes(hq, hkv, d, n_ctx, t, root_scores=False)
             flops = attn_flops(hq, d, n_ctx, t)
             gbs = byts / (us * 1e-6) / 1e9
@@ -654,7 +658,8 @@ def sweep_14b(torch, L, I, dev, hbm, tflops, warmup=10, calls=50):
         del sets
         torch.cuda.empty_cache()
     return {"workload": "qwen14b_gqa40x8_d128", "kv_sets_rotated": "ceil(3 x L2 / KV bytes), "
-            "at most 24", "calls_per_point": calls, "points": points}
+            "at most 24", "calls_per_point": calls, "timing": "CUDA graph of whole rotations, "
+            "events around its replays", "points": points}
 
 
 def run_e2e(torch, L, st, w, dev, stream, steps):
