@@ -103,6 +103,27 @@ def test_attn_chain_equals_sequential_decode():
         np.testing.assert_allclose(chain[i], step[0], rtol=0, atol=2e-4)
 
 
+def test_attn_workspace_reused_across_calls(oracle_mod):
+    """One workspace, zero-filled once, serves calls of different shapes and
+    inputs back to back: the run-time tile counters, arrival counts and
+    flags a call relies on are back at zero when it ends, so every call
+    matches the oracle (a counter left over would skip or repeat tiles)."""
+    ws = L.new_workspace(max(L.tree_verify_attn_workspace_size(32, 8, 128, n, t)
+                             for n, t in ((5000, 40), (9000, 13), (3000, 4))))
+    for i, (n_ctx, t) in enumerate(((5000, 40), (9000, 13), (3000, 4), (5000, 40))):
+        w = I.Workload(f"reuse{i}", 32, 8, 128, n_ctx, t, tree="chain" if t == 4 else "ternary",
+                       seed=900 + i)
+        q = I.gen_q(w)
+        k, v = I.gen_kv(w)
+        got = L.tree_verify_attn(dev_bf16(q), dev_bf16(k), dev_bf16(v), n_ctx, w.parent(),
+                                 workspace=ws)
+        torch.cuda.synchronize()
+        want = oracle_mod.tree_verify_attn(q, k, v, n_ctx, w.parent())
+        err = np.abs(got.cpu().numpy().astype(np.float64) - want).max()
+        assert err <= ATTN_TOL, f"call {i} ({n_ctx}, {t}): max abs err {err}"
+    assert L.workspace_status(ws) == 0
+
+
 def test_attn_kv_cap_padding(oracle_mod):
     w = I.Workload("cap", 8, 2, 64, 777, 13, seed=9)
     _attn_full(oracle_mod, w, kv_cap=w.kv_rows + 91)
