@@ -665,8 +665,12 @@ def sweep_14b(torch, L, I, dev, hbm, tflops, warmup=10, calls=50):
 def run_e2e(torch, L, st, w, dev, stream, steps):
     """The same step through the Python API with host buffers: H2D of the
     step's new inputs (queries, the tree's own K/V rows, logits, window,
-    tree tokens, draft queries) from pinned memory, the four calls, D2H of
-    the results (outputs, accept, kept indices)."""
+    tree tokens, draft queries) from pinned memory, the calls, D2H of the
+    results (outputs, accept, kept indices), and a host wait for them every
+    step.  The penalty/accept inputs are uploaded on the stream that call
+    runs on, overlapping the verify attention.  After an eager warm-up the
+    calls and copies are captured once as a CUDA graph, replayed once per
+    step."""
     hq, hkv, d, t = w.n_heads_q, w.n_heads_kv, w.head_dim, w.n_tree
     pin = lambda x: x.cpu().pin_memory()
     h_q, h_dq = pin(st.q), pin(st.dq)
@@ -681,13 +685,18 @@ def run_e2e(torch, L, st, w, dev, stream, steps):
     d2h = sum(x.numel() * x.element_size() for x in (o_out, o_dout, o_acc, o_idx))
 
     def one():
+        # the penalty/accept call's inputs (the 20 MB of logits above all) go
+        # up on the side stream it runs on, so that their copy overlaps the
+        # verify attention, which does not need them; the attention's and
+        # the draft pass's inputs go up on the main stream
+        with torch.cuda.stream(st.side):
+            st.logits.copy_(h_lg, non_blocking=True)
+            st.window.copy_(h_win, non_blocking=True)
+            st.tokens.copy_(h_tok, non_blocking=True)
         st.q.copy_(h_q, non_blocking=True)
         st.dq.copy_(h_dq, non_blocking=True)
         st.k[:, w.n_ctx:w.n_ctx + t].copy_(h_kt, non_blocking=True)
         st.v[:, w.n_ctx:w.n_ctx + t].copy_(h_vt, non_blocking=True)
-        st.logits.copy_(h_lg, non_blocking=True)
-        st.window.copy_(h_win, non_blocking=True)
-        st.tokens.copy_(h_tok, non_blocking=True)
         st.step()
         o_out.copy_(st.out, non_blocking=True)
         o_dout.copy_(st.dout, non_blocking=True)
@@ -698,10 +707,32 @@ def run_e2e(torch, L, st, w, dev, stream, steps):
     with torch.cuda.stream(stream):
         for _ in range(3):
             one()
+    # the same calls and copies captured once as a CUDA graph: a step is then
+    # one launch, the host still waiting for each step's results
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream, capture_error_mode="thread_local"):
+        with torch.cuda.stream(st.side):
+            st.logits.copy_(h_lg, non_blocking=True)
+            st.window.copy_(h_win, non_blocking=True)
+            st.tokens.copy_(h_tok, non_blocking=True)
+        st.q.copy_(h_q, non_blocking=True)
+        st.dq.copy_(h_dq, non_blocking=True)
+        st.k[:, w.n_ctx:w.n_ctx + t].copy_(h_kt, non_blocking=True)
+        st.v[:, w.n_ctx:w.n_ctx + t].copy_(h_vt, non_blocking=True)
+        st.step()
+        o_out.copy_(st.out, non_blocking=True)
+        o_dout.copy_(st.dout, non_blocking=True)
+        o_acc.copy_(st.accept, non_blocking=True)
+        o_idx.copy_(st.idx, non_blocking=True)
+    with torch.cuda.stream(stream):
+        for _ in range(3):
+            g.replay()
+            stream.synchronize()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record(stream)
         for _ in range(steps):
-            one()
+            g.replay()
+            stream.synchronize()   # the host reads each step's results
         e1.record(stream)
     torch.cuda.synchronize()
     return {"ms_per_step": e0.elapsed_time(e1) / steps, "h2d": h2d, "d2h": d2h}
