@@ -737,6 +737,10 @@ attn_t128_kernel(const __grid_constant__ CUtensorMap tmap_k,
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
+    // launched as a programmatic dependent: everything above (barriers,
+    // TMEM, tensor maps) overlaps the previous kernel's tail; what follows
+    // reads its results (the query rows, the cache, the workspace counters)
+    grid_dependency_wait();
     const uint32_t tmem = bar->tmem_base;
     // The TMA producer (warp 3) starts streaming K and V as soon as the
     // query rows' loads are on their way (ahead of the K/V requests, so
@@ -1350,11 +1354,14 @@ cudaError_t attn_t128_launch(const AttnArgs &a, const TreeMasks &masks, int num_
     cfg.blockDim = dim3(kThreads);
     cfg.dynamicSmemBytes = lay.smem_bytes;
     cfg.stream = stream;
-    cudaLaunchAttribute at[1];
+    cudaLaunchAttribute at[2];
     at[0].id = cudaLaunchAttributeCooperative;
     at[0].val.cooperative = 1;
+    // and a programmatic dependent of the kernel before it in the stream
+    at[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    at[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = at;
-    cfg.numAttrs = 1;
+    cfg.numAttrs = 2;
     cudaError_t e = cudaLaunchKernelEx(&cfg, attn_t128_kernel, mk, mv, a, masks, p.n_split,
                                        p.nodes_per_group, sy);
     if (e == cudaSuccess)
