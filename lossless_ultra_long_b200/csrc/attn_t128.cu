@@ -721,8 +721,9 @@ attn_t128_kernel(const __grid_constant__ CUtensorMap tmap_k,
         bar->abort = 0u;
         bar->overflow = 0;
         fence_mbar_init();
-        // the combine kernel may take the SMs this grid leaves idle (and
-        // then each SM a split frees) and wait there for this grid's end
+        // the next kernel in the stream, when launched as a programmatic
+        // dependent, may take the SMs this grid leaves idle (and then each SM
+        // a split frees) and wait there for this grid's end
         launch_dependents();
     }
     if (warp == 1) {
