@@ -47,6 +47,9 @@ bool encode_kv_map(CUtensorMap *m, const void *ptr, int rows, int64_t kv_cap, in
 // run time and fold their partials themselves (one cooperative launch).
 bool attn_t128_eligible(int n_heads_q, int n_heads_kv, int head_dim, int n_ctx, int n_tree);
 AttnPlan attn_t128_plan(int n_heads_q, int n_heads_kv, int n_ctx, int n_tree, int num_sms);
+// whether its grid (one CTA per SM, all resident: a cooperative launch) fits
+// the device; more (KV head, node group) pairs than SMs go to the other kernel
+bool attn_t128_fits(int n_heads_q, int n_heads_kv, int n_ctx, int n_tree, int num_sms);
 size_t attn_t128_workspace_bytes(int n_heads_q, int n_heads_kv, int n_ctx, int n_tree, int num_sms);
 // leading bytes of that workspace (header included) that must be zero when
 // a call starts; every call leaves them so

@@ -73,7 +73,8 @@ cudaError_t attn_launch(const AttnArgs &a, const TreeMasks &masks, int num_sms,
 {
     cudaError_t e;
     if (a.scale_log2 > 0.f &&
-        attn_t128_eligible(a.n_heads_q, a.n_heads_kv, a.head_dim, a.n_ctx, a.n_tree)) {
+        attn_t128_eligible(a.n_heads_q, a.n_heads_kv, a.head_dim, a.n_ctx, a.n_tree) &&
+        attn_t128_fits(a.n_heads_q, a.n_heads_kv, a.n_ctx, a.n_tree, num_sms)) {
         if (a.root_scores == nullptr || attn_t128_leaves_root_scores(a))
             return attn_t128_launch(a, masks, num_sms, stream);   // leaves root scores itself
         AttnArgs b = a;

@@ -1325,6 +1325,12 @@ AttnPlan attn_t128_plan(int n_heads_q, int n_heads_kv, int n_ctx, int n_tree, in
     return p;
 }
 
+bool attn_t128_fits(int n_heads_q, int n_heads_kv, int n_ctx, int n_tree, int num_sms)
+{
+    const AttnPlan p = attn_t128_plan(n_heads_q, n_heads_kv, n_ctx, n_tree, num_sms);
+    return (long long)p.n_split * n_heads_kv * p.node_groups <= num_sms;
+}
+
 cudaError_t attn_t128_launch(const AttnArgs &a, const TreeMasks &masks, int num_sms,
                              cudaStream_t stream)
 {

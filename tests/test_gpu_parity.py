@@ -124,6 +124,20 @@ def test_attn_workspace_reused_across_calls(oracle_mod):
     assert L.workspace_status(ws) == 0
 
 
+def test_attn_more_groups_than_sms(oracle_mod):
+    """128 KV heads of 4 query heads and a 64-node tree: two node groups per
+    head need 256 resident CTAs, more than the SMs, so the call goes to the
+    other kernel instead of a cooperative launch that cannot be placed."""
+    w = I.Workload("wide", 512, 128, 128, 2048, 64, seed=31)
+    q = I.gen_q(w)
+    k, v = I.gen_kv(w)
+    got = run_attn(q, k, v, w.n_ctx, w.parent())
+    nodes, heads = sample_rows(w.n_tree, w.n_heads_q, 24, seed=31)
+    want = oracle_mod.tree_verify_attn_rows(q, k, v, w.n_ctx, w.parent(), nodes, heads)
+    err = np.abs(got[nodes, heads] - want).max()
+    assert err <= ATTN_TOL, f"max abs err {err}"
+
+
 def test_attn_kv_cap_padding(oracle_mod):
     w = I.Workload("cap", 8, 2, 64, 777, 13, seed=9)
     _attn_full(oracle_mod, w, kv_cap=w.kv_rows + 91)
