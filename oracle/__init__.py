@@ -47,6 +47,7 @@ def _load():
         lib.tso_accept_longest.argtypes = [P, P, P, i32, P]
         lib.tso_penalize_argmax_path.argtypes = [P, i32, i32, P, i32, f32, P, P, P, P]
         lib.tso_accept_longest_random.argtypes = [P, P, P, i32, ctypes.c_uint64, P]
+        lib.tso_sample_targets.argtypes = [P, P, i32, i32, f32, P]
         lib.tso_kv_commit_path.argtypes = [P, i64, i32, i32, i32, i32, P]
         _lib = lib
     return _lib
@@ -193,6 +194,22 @@ def accept_longest_random(parent, tokens, argmax, r: int) -> np.ndarray:
                                            ctypes.c_uint64(int(r) & (2 ** 64 - 1)), _p(out))
     if rc < 0:
         raise ValueError("oracle: invalid tree")
+    return out
+
+
+def sample_targets(penalized, gumbel, temperature: float) -> np.ndarray:
+    """int32 ``[T]``: per node the id maximising penalised / temperature + g
+    (binary32), the Gumbel-max draw from softmax(penalised / temperature)."""
+    penalized = np.ascontiguousarray(penalized, dtype=np.float32)
+    gumbel = np.ascontiguousarray(gumbel, dtype=np.float32)
+    if penalized.shape != gumbel.shape or penalized.ndim != 2:
+        raise ValueError("oracle: penalised logits and noise must both be [T, V]")
+    t, vocab = penalized.shape
+    out = np.empty(t, dtype=np.int32)
+    rc = _load().tso_sample_targets(_p(penalized), _p(gumbel), t, vocab,
+                                    float(np.float32(temperature)), _p(out))
+    if rc != 0:
+        raise ValueError("oracle: invalid temperature")
     return out
 
 

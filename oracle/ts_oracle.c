@@ -28,6 +28,7 @@
  *
  * Readings of points the pages leave open are stated at each function.
  */
+#include <float.h>
 #include <math.h>
 #include <stdint.h>
 #include <stdlib.h>
@@ -493,6 +494,51 @@ int tso_accept_longest_random(const int32_t *parent, const int32_t *tokens,
     free(valid);
     free(depth);
     return len;
+}
+
+/*
+ * Temperature acceptance: the target token of every tree node is a draw from
+ * the tempered distribution softmax(penalised logits / temperature) instead
+ * of its argmax (aiboss88 "Tree-based multi-candidate token verification":
+ * the output stays lossless, i.e. distributed as the target model's own
+ * sampling, while the choice gains diversity).  Reading: the draw is the
+ * Gumbel-max rule -- the id maximising penalised / temperature + g, with
+ * g[i][id] independent standard Gumbel noise drawn by the caller -- whose
+ * result is distributed exactly as that softmax.  A draft node is then valid
+ * when its parent is valid and its token equals the draw at its parent, so
+ * every accepted token is the target's own sample given the tokens before
+ * it; acceptance itself is tso_accept_longest (or _random) with the draws in
+ * place of the argmax.
+ *
+ * `penalized` is the fp32 output of tso_penalize_argmax (or _path).  Each
+ * node's score is computed in binary32, round-to-nearest, one rounding per
+ * operation: the quotient, then the sum with g, so that the integer decision
+ * is taken in the same precision as the path takes it.  The draw is the
+ * largest score, ties to the lowest id, a NaN counting as -inf.  Returns 0,
+ * or -1 when the temperature is not a finite positive number.
+ */
+int tso_sample_targets(const float *penalized, const float *gumbel, int n_tree, int vocab,
+                       float temperature, int32_t *target)
+{
+    if (n_tree < 0 || vocab < 1 || !(temperature > 0.0f) || !(temperature <= FLT_MAX))
+        return -1;
+    for (int i = 0; i < n_tree; ++i) {
+        float best = -INFINITY;
+        int32_t best_id = 0;
+        for (int id = 0; id < vocab; ++id) {
+            const int64_t at = (int64_t)i * vocab + id;
+            float z = penalized[at] / temperature;
+            z = z + gumbel[at];
+            if (z != z)
+                z = -INFINITY;
+            if (best < z) {
+                best = z;
+                best_id = id;
+            }
+        }
+        target[i] = best_id;
+    }
+    return 0;
 }
 
 /*

@@ -43,6 +43,11 @@ C_MUTANTS = {
     "path_argmax_ties_to_highest_id": ("if (best < x) {", "if (best <= x) {"),
     "random_tie_validity_ignores_parent": ("valid[i] = tokens[i] == argmax[p] && valid[p];",
                                            "valid[i] = tokens[i] == argmax[p];"),
+    "sample_multiplies_by_temperature": ("float z = penalized[at] / temperature;",
+                                         "float z = penalized[at] * temperature;"),
+    "sample_ignores_noise": ("z = z + gumbel[at];", "z = z + 0.0f;"),
+    "sample_subtracts_noise": ("z = z + gumbel[at];", "z = z - gumbel[at];"),
+    "sample_ties_to_highest_id": ("if (best < z) {", "if (best <= z) {"),
     "commit_writes_rows_in_place": (
         "memcpy(base + ((int64_t)n_ctx + j) * head_dim, rows + (size_t)j * head_dim,",
         "memcpy(base + ((int64_t)n_ctx + accept[2 + j]) * head_dim, rows + (size_t)j * head_dim,"),

@@ -432,6 +432,61 @@ def test_random_tie_matches_exhaustive_path_search(oracle_mod):
                                       oracle_mod.accept_longest(parent, tokens, argmax))
 
 
+def test_temperature_golden_cases(oracle_mod):
+    t = json.load(open(SAMPLING))["temperature"]
+    for c in t["draws"]:
+        got = oracle_mod.sample_targets(np.array(c["penalized"], np.float32),
+                                        np.array(c["gumbel"], np.float32), c["temperature"])
+        np.testing.assert_array_equal(got, c["expected"], err_msg=c["name"])
+    c = t["tree"]
+    pen = np.array(c["penalized"], np.float32)
+    draws = oracle_mod.sample_targets(pen, np.array(c["gumbel"], np.float32), c["temperature"])
+    np.testing.assert_array_equal(draws, c["expected_draws"])
+    out = oracle_mod.accept_longest(c["parent"], c["tokens"], draws)
+    np.testing.assert_array_equal(out[:len(c["expected_accept"])], c["expected_accept"])
+    greedy = oracle_mod.accept_longest(c["parent"], c["tokens"], np.argmax(pen, axis=1))
+    np.testing.assert_array_equal(greedy[:len(c["greedy_accept"])], c["greedy_accept"])
+
+
+@pytest.mark.parametrize("temperature", [0.5, 2.0])
+def test_temperature_draws_follow_the_tempered_softmax(oracle_mod, temperature):
+    """Gumbel-max: with independent standard Gumbel noise, the draw of each
+    row is distributed as softmax(logits / temperature).  200,000 rows of the
+    same five logits; every id's frequency within five standard errors of
+    the closed-form probability (numpy's own Gumbel generator, fp64
+    softmax)."""
+    n = 200_000
+    logits = np.array([1.0, 0.5, -0.3, 2.0, 1.2], np.float32)
+    g = np.random.default_rng(41).gumbel(size=(n, 5)).astype(np.float32)
+    draws = oracle_mod.sample_targets(np.tile(logits, (n, 1)), g, temperature)
+    z = logits.astype(np.float64) / temperature
+    p = np.exp(z - z.max())
+    p /= p.sum()
+    freq = np.bincount(draws, minlength=5) / n
+    se = np.sqrt(p * (1 - p) / n)
+    assert np.all(np.abs(freq - p) <= 5 * se + 1e-12), (freq, p)
+
+
+def test_temperature_one_without_noise_is_the_argmax(oracle_mod):
+    """temperature 1 divides exactly and zero noise adds nothing: the draw
+    is the penalised argmax (ties to the lowest id), on a workload's logits."""
+    w = I.TINY
+    lg = I.gen_logits(w)
+    lg[3, 17] = lg[3, 5] = 40.0   # a tie
+    am, pen = oracle_mod.penalize_argmax(lg, I.gen_window(w), w.penalty, return_penalized=True)
+    np.testing.assert_array_equal(oracle_mod.sample_targets(pen, np.zeros_like(pen), 1.0), am)
+    assert am[3] == 5
+
+
+def test_temperature_nan_is_never_drawn_and_bad_temperatures_rejected(oracle_mod):
+    pen = np.array([[np.nan, -5.0, -6.0], [1.0, np.nan, 0.0]], np.float32)
+    g = np.array([[0.0, 0.0, 0.5], [0.0, 0.0, np.nan]], np.float32)
+    np.testing.assert_array_equal(oracle_mod.sample_targets(pen, g, 1.0), [1, 0])
+    for bad in (0.0, -1.0, np.inf, np.nan):
+        with pytest.raises(ValueError):
+            oracle_mod.sample_targets(pen, g, bad)
+
+
 def test_commit_golden_case(oracle_mod):
     c = json.load(open(SAMPLING))["commit"]
     cache = np.array(c["rows"], np.uint16)[None]
