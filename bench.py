@@ -56,7 +56,7 @@ def parse():
     ap.add_argument("--no-sweep", action="store_true",
                     help="skip the 14B-shape roofline sweep (context x tree size)")
     ap.add_argument("--only", choices=["verify", "verify_plain", "select", "draft", "penalty",
-                                       "commit"],
+                                       "penalty_sample", "commit"],
                     help="run one call of the step warmup + steps times, eagerly, and print "
                          "its mean device time (for profiler captures of a single kernel)")
     ap.add_argument("--breakdown", action="store_true",
@@ -331,6 +331,22 @@ class Step:
                                argmax_out=self.argmax, accept_out=self.accept,
                                workspace=self.ws_pen)
 
+    def penalty_sample(self, temperature=0.8):
+        """The penalty call with temperature acceptance (the Gumbel-max
+        draw); the noise is drawn once, on the device, on first use."""
+        w = self.w
+        if getattr(self, "gumbel", None) is None:
+            gen = self.torch.Generator(device=self.logits.device)
+            gen.manual_seed(w.seed)
+            u = self.torch.rand(self.logits.shape, generator=gen, device=self.logits.device,
+                                dtype=self.torch.float64).clamp_min_(2.0 ** -1022)
+            self.gumbel = (-(-u.log()).log()).float()
+            del u
+        self.L.penalize_sample_accept(self.logits, self.gumbel, temperature, self.window,
+                                      w.penalty, self.parent, self.tokens,
+                                      target_out=self.argmax, accept_out=self.accept,
+                                      workspace=self.ws_pen)
+
     def draft(self):
         self.L.tree_verify_attn(self.dq, self.kp, self.vp, self.n_keep, self.draft_parent,
                                 out=self.dout, workspace=self.ws_draft)
@@ -528,7 +544,7 @@ def _setup_single(args):
 def _call_of(st, name):
     return {"verify": lambda: st.attn(True), "verify_plain": lambda: st.attn(False),
             "select": st.select, "draft": st.draft, "penalty": st.penalty,
-            "commit": st.commit}[name]
+            "penalty_sample": st.penalty_sample, "commit": st.commit}[name]
 
 
 def _prepare(st, name):
@@ -602,7 +618,9 @@ def run_breakdown(args):
     st.select()
     st.penalty()
     out = {"mode": "breakdown", "workload": w.name, "timing": "CUDA graph of 10 calls"}
-    for name in ("verify", "verify_plain", "select", "draft", "penalty", "commit"):
+    st.penalty_sample()   # draws the noise outside the timed graphs
+    for name in ("verify", "verify_plain", "select", "draft", "penalty", "penalty_sample",
+                 "commit"):
         out[name + "_us"] = round(_time_call_graph(torch, _call_of(st, name), args.warmup,
                                                    max(args.steps, 10)), 2)
     return out

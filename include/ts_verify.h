@@ -275,7 +275,8 @@ TS_API int ts_kv_select_from_scores(const float *root_scores, const void *k_cach
  * the lowest node index.
  *
  *  logits       device fp32 [n_tree, vocab]; not modified.
- *  n_tree       1 .. TS_MAX_TREE.   vocab >= 1.
+ *  n_tree       1 .. TS_MAX_TREE.   vocab 1 .. 16,777,216 (above:
+ *               TS_ERR_UNSUPPORTED).
  *  window       device int32 [window_len] (may be NULL when window_len is
  *               0); ids outside [0, vocab) are ignored and flagged as
  *               TS_ERR_DEVICE_ARG in the status word.
@@ -321,6 +322,44 @@ TS_API int ts_penalize_accept_ex(const float *logits, int n_tree, int vocab,
                                  unsigned flags, uint64_t random, int32_t *argmax_out,
                                  int32_t *accept_out, void *workspace, size_t workspace_bytes,
                                  void *stream);
+
+/*
+ * ts_penalize_accept_ex with temperature acceptance: the target token of
+ * every node is a draw from softmax(penalised logits / temperature) rather
+ * than its argmax ("TokenSwift's technical principles", aiboss88.com,
+ * tree-based verification: the output stays lossless -- every accepted
+ * token is what the target model itself would have sampled after the tokens
+ * before it -- and gains diversity).  The draw is the Gumbel-max rule:
+ * target[i] is the id maximising
+ *
+ *     score = penalised[i][id] / temperature + gumbel[i][id]
+ *
+ * computed in binary32 with round-to-nearest, one rounding per operation
+ * (the quotient, then the sum; never fused), ties to the lowest id, a NaN
+ * score counting as -inf.  With gumbel holding independent standard Gumbel
+ * draws (-log(-log u), u uniform on (0, 1)) the result is distributed
+ * exactly as that softmax.  A draft node is valid when its parent is valid
+ * and its token equals target[parent]; the accepted path and the flags are
+ * as for ts_penalize_accept_ex, with target in place of argmax (bonus =
+ * target at path[L]).  Temperature 1 with all-zero noise gives exactly
+ * ts_penalize_accept_ex.
+ *
+ *  gumbel       device fp32 [n_tree, vocab], 16-byte aligned; not
+ *               modified.  The caller draws it (and owns the generator).
+ *  temperature  finite, > 0.
+ *  vocab        1 .. 8,388,608 (above: TS_ERR_UNSUPPORTED).
+ *  target_out   device int32 [n_tree], or NULL.
+ * The other arguments, the workspace (ts_penalize_accept_workspace_size)
+ * and the errors are as for ts_penalize_accept_ex; a NULL or misaligned
+ * gumbel or a bad temperature: TS_ERR_INVALID_ARG.  The call reads
+ * 2 * n_tree * vocab * 4 bytes (logits and noise, each once).
+ */
+TS_API int ts_penalize_sample_accept(const float *logits, const float *gumbel, float temperature,
+                                     int n_tree, int vocab, const int32_t *window,
+                                     int window_len, float penalty, const int32_t *parent,
+                                     const int32_t *tree_tokens, unsigned flags, uint64_t random,
+                                     int32_t *target_out, int32_t *accept_out, void *workspace,
+                                     size_t workspace_bytes, void *stream);
 
 /*
  * Commit of the accepted path: the tree rows of the nodes on the accepted

@@ -29,7 +29,7 @@ EXPORTS = ("ts_status_string", "ts_version", "ts_tree_verify_attn_workspace_size
            "ts_ngram_table_bytes", "ts_ngram_init", "ts_ngram_update", "ts_ngram_topk",
            "ts_ngram_topk_prefix",
            "ts_ngram_count", "ts_ngram_size", "ts_selftest_bounded_wait",
-           "ts_penalize_accept_ex", "ts_kv_commit_path")
+           "ts_penalize_accept_ex", "ts_penalize_sample_accept", "ts_kv_commit_path")
 
 TS_PENALIZE_PATH_TOKENS = 1
 TS_ACCEPT_RANDOM_TIE = 2
@@ -82,6 +82,9 @@ def _lib():
         lib.ts_penalize_accept_ex.restype = i32
         lib.ts_penalize_accept_ex.argtypes = [P, i32, i32, P, i32, f32, P, P, ctypes.c_uint,
                                               ctypes.c_uint64, P, P, P, sz, P]
+        lib.ts_penalize_sample_accept.restype = i32
+        lib.ts_penalize_sample_accept.argtypes = [P, P, f32, i32, i32, P, i32, f32, P, P,
+                                                  ctypes.c_uint, ctypes.c_uint64, P, P, P, sz, P]
         lib.ts_kv_commit_path.restype = i32
         lib.ts_kv_commit_path.argtypes = [P, P, i64, i32, i32, i32, i32, P, P, sz, P]
         lib.ts_kernel_launch_count.restype = ctypes.c_ulonglong
@@ -338,6 +341,51 @@ def penalize_accept(logits, window, penalty: float, parent, tree_tokens, argmax_
             _ptr(workspace), workspace.numel(), _stream(stream))
         _raise(rc, "ts_penalize_accept_ex")
     return accept_out, argmax_out
+
+
+def penalize_sample_accept(logits, gumbel, temperature: float, window, penalty: float, parent,
+                           tree_tokens, target_out=None, accept_out=None, workspace=None,
+                           stream=None, want_target: bool = True, flags: int = 0,
+                           random: int = 0):
+    """Contextual penalty + per-node temperature draw + longest accepted path
+    (``ts_penalize_sample_accept``): node i's target token is the id
+    maximising penalised / temperature + gumbel[i] (binary32), the
+    Gumbel-max draw from softmax(penalised / temperature); ``gumbel`` is the
+    caller's standard Gumbel noise, fp32 ``[T, V]`` on the device.  ``flags``
+    and ``random`` as for :func:`penalize_accept`.
+
+    Returns ``(accept [2 + T] int32, target [T] int32 or None)``.
+    """
+    _check_dev("logits", logits, torch.float32)
+    _check_dev("gumbel", gumbel, torch.float32)
+    _check_dev("tree_tokens", tree_tokens, torch.int32)
+    t, vocab = logits.shape
+    if tuple(gumbel.shape) != (t, vocab):
+        raise ValueError("gumbel must have the logits' shape [T, V]")
+    dev = logits.device
+    if window is not None and window.numel() > 0:
+        _check_dev("window", window, torch.int32)
+        wlen, wptr = window.numel(), _ptr(window)
+    else:
+        wlen, wptr = 0, None
+    if accept_out is None:
+        accept_out = torch.empty(2 + t, dtype=torch.int32, device=dev)
+    if want_target and target_out is None:
+        target_out = torch.empty(t, dtype=torch.int32, device=dev)
+    _check_dev("accept_out", accept_out, torch.int32)
+    if target_out is not None:
+        _check_dev("target_out", target_out, torch.int32)
+    if workspace is None:
+        workspace = new_workspace(penalize_accept_workspace_size(t, vocab), dev)
+    par, par_p = _host_i32(parent)
+    if len(par) != t:
+        raise ValueError("parent must have one entry per tree node")
+    rc = _lib().ts_penalize_sample_accept(
+        _ptr(logits), _ptr(gumbel), float(temperature), t, vocab, wptr, wlen, float(penalty),
+        par_p, _ptr(tree_tokens), int(flags), int(random) & (2 ** 64 - 1), _ptr(target_out),
+        _ptr(accept_out), _ptr(workspace), workspace.numel(), _stream(stream))
+    _raise(rc, "ts_penalize_sample_accept")
+    return accept_out, target_out
 
 
 def kv_commit_path(k_cache, v_cache, n_ctx: int, n_tree: int, accept, workspace=None,

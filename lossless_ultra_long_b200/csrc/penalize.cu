@@ -18,7 +18,12 @@
 // (aiboss88, "Contextual penalty strategy": the recently generated tokens),
 // and the kept node is drawn among the deepest valid ones with a
 // caller-given random integer (aiboss88, tree-based verification: the
-// longest valid candidate is selected at random).
+// longest valid candidate is selected at random).  With caller-drawn
+// Gumbel noise (the kSample instance) each node's target token is the
+// draw from softmax(penalised / temperature) by the Gumbel-max rule -- the
+// largest penalised / temperature + g, in binary32 -- instead of the
+// argmax; the noise slice is bulk-copied beside the logits slice, so that
+// instance reads 2 * T * V * 4 bytes.
 #include <float.h>
 #include <limits.h>
 
@@ -34,12 +39,12 @@ constexpr int kBitWords = kMaxChunk / 32;
 constexpr int kMaxSplits = 1024;
 
 // Vocab entries per CTA (a multiple of 4): enough splits per node for one
-// wave of resident CTAs (ctas_per_sm on each SM), no more than kMaxChunk
+// wave of resident CTAs (ctas_per_sm on each SM), no more than max_chunk
 // entries each.
-int penalize_chunk(int n_tree, int vocab, int num_sms, int ctas_per_sm)
+int penalize_chunk(int n_tree, int vocab, int num_sms, int ctas_per_sm, int max_chunk)
 {
     int splits = (ctas_per_sm * num_sms) / (n_tree > 0 ? n_tree : 1);
-    const int need = (vocab + kMaxChunk - 1) / kMaxChunk;
+    const int need = (vocab + max_chunk - 1) / max_chunk;
     splits = splits < need ? need : splits;
     splits = splits > kMaxSplits ? kMaxSplits : (splits < 1 ? 1 : splits);
     int chunk = (vocab + splits - 1) / splits;
@@ -106,10 +111,25 @@ __device__ __forceinline__ void bulk_load(uint32_t dst, const void *src, uint32_
         : "memory");
 }
 
+// The score a node's id competes with: the penalised logit, or with the
+// temperature draw that divided by the temperature plus the id's noise
+// (one binary32 rounding per operation, never fused).
+template <bool kSample>
+__device__ __forceinline__ float draw_score(float y, float t, float g)
+{
+    if constexpr (kSample)
+        return __fadd_rn(__fdiv_rn(y, t), g);
+    else
+        return y;
+}
+
+template <bool kSample>
 __global__ void __launch_bounds__(kThreads)
 penalize_accept_kernel(PenalizeArgs a, TreeParents tree, int chunk, int n_chunks)
 {
-    extern __shared__ __align__(16) float xs[];   // this CTA's slice of the logits row
+    // this CTA's slice of the logits row, then (kSample) the same slice of
+    // the noise row at xs + chunk
+    extern __shared__ __align__(16) float xs[];
     __shared__ uint32_t bits[kBitWords];
     __shared__ Best warp_res[kThreads / 32];
     __shared__ int am[TS_MAX_TREE];
@@ -125,6 +145,7 @@ penalize_accept_kernel(PenalizeArgs a, TreeParents tree, int chunk, int n_chunks
     const int v0 = blockIdx.x * chunk;
     const int v1 = min(v0 + chunk, a.vocab);
     const float *row = a.logits + (int64_t)node * a.vocab;
+    const float *grow = kSample ? a.gumbel + (int64_t)node * a.vocab : nullptr;
     // rows and slices start on 16-byte boundaries and end on whole vectors
     const bool vec = (a.vocab & 3) == 0 && (reinterpret_cast<uintptr_t>(a.logits) & 15) == 0;
 
@@ -133,8 +154,11 @@ penalize_accept_kernel(PenalizeArgs a, TreeParents tree, int chunk, int n_chunks
         abort_flag = 0u;
         sm100::fence_mbar_init();
         const uint32_t bytes = (uint32_t)(v1 - v0) * 4u;
-        sm100::mbar_arrive_expect_tx(sm100::smem_addr(&landed), bytes);
+        sm100::mbar_arrive_expect_tx(sm100::smem_addr(&landed), kSample ? 2u * bytes : bytes);
         bulk_load(sm100::smem_addr(xs), row + v0, bytes, sm100::smem_addr(&landed));
+        if constexpr (kSample)   // chunk is a multiple of 4: 16-byte aligned
+            bulk_load(sm100::smem_addr(xs + chunk), grow + v0, bytes,
+                      sm100::smem_addr(&landed));
     }
     for (int w = tid; w < kBitWords; w += kThreads)
         bits[w] = 0u;
@@ -166,21 +190,28 @@ penalize_accept_kernel(PenalizeArgs a, TreeParents tree, int chunk, int n_chunks
     __syncthreads();
 
     const float p = a.penalty;
+    const float temp = a.temperature;
     Best b{-INFINITY, INT_MAX};
     if (vec) {
         if (sm100::wait_bounded(sm100::smem_addr(&landed), 0, &abort_flag, hdr)) {
             // two independent running bests (even and odd lanes of each
             // vector) halve the compare chain
             const float4 *x4 = reinterpret_cast<const float4 *>(xs);
+            const float4 *g4 = reinterpret_cast<const float4 *>(xs + chunk);
             Best b2{-INFINITY, INT_MAX};
             for (int u = tid; u < (v1 - v0) / 4; u += kThreads) {
                 const float4 q = x4[u];
+                float4 gq = make_float4(0.f, 0.f, 0.f, 0.f);
+                if constexpr (kSample)
+                    gq = g4[u];
                 const uint32_t word = bits[u >> 3] >> ((u & 7) * 4);
                 const float x[4] = {q.x, q.y, q.z, q.w};
+                const float g[4] = {gq.x, gq.y, gq.z, gq.w};
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
                     const float y = ((word >> e) & 1u) ? penalise(x[e], p) : x[e];
-                    consider(e & 1 ? b2 : b, y, v0 + 4 * u + e);
+                    consider(e & 1 ? b2 : b, draw_score<kSample>(y, temp, g[e]),
+                             v0 + 4 * u + e);
                 }
             }
             if (beats(b2.v, b2.i, b.v, b.i))
@@ -191,7 +222,7 @@ penalize_accept_kernel(PenalizeArgs a, TreeParents tree, int chunk, int n_chunks
             float x = __ldcs(row + v);
             if ((bits[(v - v0) >> 5] >> ((v - v0) & 31)) & 1u)
                 x = penalise(x, p);
-            consider(b, x, v);
+            consider(b, draw_score<kSample>(x, temp, kSample ? __ldcs(grow + v) : 0.f), v);
         }
     }
     b = warp_best(b);
@@ -321,23 +352,37 @@ penalize_accept_kernel(PenalizeArgs a, TreeParents tree, int chunk, int n_chunks
 
 }  // namespace
 
+int penalize_max_vocab(bool sample)
+{
+    return (sample ? kMaxChunk / 2 : kMaxChunk) * kMaxSplits;
+}
+
 size_t penalize_workspace_bytes(int n_tree, int vocab)
 {
     // room for the most splits any device gives (per-split results)
     return kHeaderBytes + align_up((size_t)kMaxSplits * n_tree * sizeof(Best), 256);
 }
 
-cudaError_t penalize_launch(const PenalizeArgs &a, const TreeParents &parents, int num_sms,
-                            cudaStream_t stream)
+namespace {
+
+template <bool kSample>
+cudaError_t penalize_launch_as(const PenalizeArgs &a, const TreeParents &parents, int num_sms,
+                               cudaStream_t stream)
 {
+    // dynamic shared memory: the logits slice, and the noise slice beside
+    // it; with two slices each is half as long, so that a CTA holds the same
+    // 64 KB and as many CTAs stay resident per SM
+    constexpr int kSlices = kSample ? 2 : 1;
+    constexpr int kSliceMax = kMaxChunk / kSlices;
     static int per_sm = 0;
     if (per_sm == 0) {
         int n = 0;
-        if (cudaFuncSetAttribute(penalize_accept_kernel,
+        if (cudaFuncSetAttribute(penalize_accept_kernel<kSample>,
                                  cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 kMaxChunk * (int)sizeof(float)) != cudaSuccess ||
-            cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, penalize_accept_kernel, kThreads,
-                                                          kMaxChunk * sizeof(float)) !=
+                                 kSlices * kSliceMax * (int)sizeof(float)) != cudaSuccess ||
+            cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, penalize_accept_kernel<kSample>,
+                                                          kThreads,
+                                                          kSlices * kSliceMax * sizeof(float)) !=
                 cudaSuccess ||
             n < 1) {
             cudaGetLastError();
@@ -345,15 +390,25 @@ cudaError_t penalize_launch(const PenalizeArgs &a, const TreeParents &parents, i
         }
         per_sm = n;
     }
-    const int chunk = penalize_chunk(a.n_tree, a.vocab, num_sms, per_sm);
+    const int chunk = penalize_chunk(a.n_tree, a.vocab, num_sms, per_sm, kSliceMax);
     const int n_chunks = (a.vocab + chunk - 1) / chunk;
     dim3 grid(n_chunks, a.n_tree);
-    penalize_accept_kernel<<<grid, kThreads, (size_t)chunk * sizeof(float), stream>>>(
-        a, parents, chunk, n_chunks);
+    penalize_accept_kernel<kSample>
+        <<<grid, kThreads, (size_t)kSlices * chunk * sizeof(float), stream>>>(a, parents, chunk,
+                                                                             n_chunks);
     const cudaError_t e = cudaGetLastError();
     if (e == cudaSuccess)
         count_launches(1);
     return e;
+}
+
+}  // namespace
+
+cudaError_t penalize_launch(const PenalizeArgs &a, const TreeParents &parents, int num_sms,
+                            cudaStream_t stream)
+{
+    return a.gumbel ? penalize_launch_as<true>(a, parents, num_sms, stream)
+                    : penalize_launch_as<false>(a, parents, num_sms, stream);
 }
 
 }  // namespace ts

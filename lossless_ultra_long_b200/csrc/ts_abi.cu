@@ -318,11 +318,16 @@ int ts_penalize_accept(const float *logits, int n_tree, int vocab, const int32_t
                                  workspace_bytes, stream);
 }
 
-int ts_penalize_accept_ex(const float *logits, int n_tree, int vocab, const int32_t *window,
-                          int window_len, float penalty, const int32_t *parent,
-                          const int32_t *tree_tokens, unsigned flags, uint64_t random,
-                          int32_t *argmax_out, int32_t *accept_out, void *workspace,
-                          size_t workspace_bytes, void *stream)
+namespace {
+
+// Both penalty entry points: gumbel == NULL takes the argmax, otherwise the
+// temperature draw.
+int penalize_accept_impl(const float *logits, const float *gumbel, float temperature,
+                         int n_tree, int vocab, const int32_t *window, int window_len,
+                         float penalty, const int32_t *parent, const int32_t *tree_tokens,
+                         unsigned flags, uint64_t random, int32_t *argmax_out,
+                         int32_t *accept_out, void *workspace, size_t workspace_bytes,
+                         void *stream)
 {
     if ((flags & ~(unsigned)(TS_PENALIZE_PATH_TOKENS | TS_ACCEPT_RANDOM_TIE)) != 0)
         return TS_ERR_INVALID_ARG;
@@ -332,7 +337,7 @@ int ts_penalize_accept_ex(const float *logits, int n_tree, int vocab, const int3
         return TS_ERR_INVALID_ARG;
     if (!tree_ok(parent, n_tree))
         return TS_ERR_INVALID_ARG;
-    if ((int64_t)n_tree * vocab > ((int64_t)1 << 40))
+    if (vocab > ts::penalize_max_vocab(gumbel != nullptr))
         return TS_ERR_UNSUPPORTED;
     if (!aligned(logits, 16) || !aligned(tree_tokens, 4) || !aligned(accept_out, 4) ||
         (window && !aligned(window, 4)) || (argmax_out && !aligned(argmax_out, 4)))
@@ -358,9 +363,38 @@ int ts_penalize_accept_ex(const float *logits, int n_tree, int vocab, const int3
     a.workspace_bytes = workspace_bytes;
     a.flags = flags;
     a.random = random;
+    a.gumbel = gumbel;
+    a.temperature = temperature;
     const cudaError_t e =
         ts::penalize_launch(a, tp, current_num_sms(), static_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? TS_OK : TS_ERR_CUDA;
+}
+
+}  // namespace
+
+int ts_penalize_accept_ex(const float *logits, int n_tree, int vocab, const int32_t *window,
+                          int window_len, float penalty, const int32_t *parent,
+                          const int32_t *tree_tokens, unsigned flags, uint64_t random,
+                          int32_t *argmax_out, int32_t *accept_out, void *workspace,
+                          size_t workspace_bytes, void *stream)
+{
+    return penalize_accept_impl(logits, nullptr, 1.0f, n_tree, vocab, window, window_len,
+                                penalty, parent, tree_tokens, flags, random, argmax_out,
+                                accept_out, workspace, workspace_bytes, stream);
+}
+
+int ts_penalize_sample_accept(const float *logits, const float *gumbel, float temperature,
+                              int n_tree, int vocab, const int32_t *window, int window_len,
+                              float penalty, const int32_t *parent, const int32_t *tree_tokens,
+                              unsigned flags, uint64_t random, int32_t *target_out,
+                              int32_t *accept_out, void *workspace, size_t workspace_bytes,
+                              void *stream)
+{
+    if (!gumbel || !aligned(gumbel, 16) || !(temperature > 0.0f) || !isfinite(temperature))
+        return TS_ERR_INVALID_ARG;
+    return penalize_accept_impl(logits, gumbel, temperature, n_tree, vocab, window, window_len,
+                                penalty, parent, tree_tokens, flags, random, target_out,
+                                accept_out, workspace, workspace_bytes, stream);
 }
 
 int ts_kv_commit_path(void *k_cache, void *v_cache, int64_t kv_cap, int n_heads_kv,

@@ -149,6 +149,8 @@ struct PenalizeArgs {
     size_t workspace_bytes;
     unsigned flags;              // TS_PENALIZE_PATH_TOKENS | TS_ACCEPT_RANDOM_TIE
     unsigned long long random;   // r of the random choice among the deepest valid nodes
+    const float *gumbel;         // [n_tree, vocab] noise of the temperature draw, or null (argmax)
+    float temperature;           // read only with gumbel
 };
 
 // Commit of the accepted path's tree rows into the context (one cache pair).
@@ -163,6 +165,9 @@ struct CommitArgs {
 cudaError_t commit_launch(const CommitArgs &a, cudaStream_t stream);
 
 size_t penalize_workspace_bytes(int n_tree, int vocab);
+// Largest vocabulary one penalty launch covers (its splits times the
+// longest slice a CTA stages); `sample`: with the temperature draw's noise.
+int penalize_max_vocab(bool sample);
 cudaError_t penalize_launch(const PenalizeArgs &a, const TreeParents &parents, int num_sms,
                             cudaStream_t stream);
 

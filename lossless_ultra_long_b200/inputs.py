@@ -16,6 +16,9 @@ Recipe (all seeds are numpy PCG64 ``default_rng`` SeedSequences):
   bf16 rounding.
 * Logits: fp32 normal with standard deviation 2.
 * Penalty window: ids drawn uniformly from ``[0, V)`` with replacement.
+* Gumbel noise (the temperature draw's randomness): ``-log(-log(u))`` with
+  ``u`` uniform on ``[0, 1)`` in fp64 (a zero replaced by the smallest
+  positive double), stored as fp32 ``[T, V]``.
 * Tree: a 3-ary tree in BFS order, ``parent[i] = (i - 1) // 3``; a chain is
   ``parent[i] = i - 1``.
 * Tree tokens: per node, with probability 0.7 one randomly chosen child gets
@@ -37,7 +40,7 @@ def _rng(seed: int, stream: int) -> np.random.Generator:
 
 
 # Per-tensor sub-streams so that any one tensor can be regenerated alone.
-_S_Q, _S_K, _S_V, _S_LOGITS, _S_WINDOW, _S_TOKENS, _S_SPIKE, _S_DRAFTQ = range(1, 9)
+_S_Q, _S_K, _S_V, _S_LOGITS, _S_WINDOW, _S_TOKENS, _S_SPIKE, _S_DRAFTQ, _S_GUMBEL = range(1, 10)
 
 
 def f32_to_bf16_bits(x: np.ndarray) -> np.ndarray:
@@ -170,6 +173,14 @@ def gen_kv(w: Workload, kv_cap: int | None = None) -> tuple[np.ndarray, np.ndarr
 def gen_logits(w: Workload) -> np.ndarray:
     """fp32 ``[T, V]`` with N(0, 2) entries (2 is the standard deviation)."""
     return _rng(w.seed, _S_LOGITS).normal(0.0, 2.0, size=(w.n_tree, w.vocab)).astype(np.float32)
+
+
+def gen_gumbel(w: Workload, draw: int = 0) -> np.ndarray:
+    """fp32 ``[T, V]`` standard Gumbel noise; ``draw`` selects an independent
+    draw for the same workload."""
+    u = _rng(w.seed * 1000 + draw, _S_GUMBEL).random(size=(w.n_tree, w.vocab))
+    u[u == 0.0] = np.finfo(np.float64).tiny
+    return (-np.log(-np.log(u))).astype(np.float32)
 
 
 def gen_window(w: Workload) -> np.ndarray:

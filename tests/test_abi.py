@@ -97,6 +97,21 @@ def test_select_and_penalize_reject_on_host(lib):
                                   1 << 20, None) == 1
     assert lib.ts_penalize_accept(a, 2, 100, a, 4, ctypes.c_float(1.2), pp, a, None, a, a,
                                   8, None) == 3
+    # vocabularies past what one launch covers
+    assert lib.ts_penalize_accept(a, 2, (1 << 24) + 1, a, 4, ctypes.c_float(1.2), pp, a, None,
+                                  a, a, 1 << 30, None) == 2
+    sample = lib.ts_penalize_sample_accept
+    sample.restype = ctypes.c_int
+    sample.argtypes = [P, P, ctypes.c_float, ctypes.c_int, ctypes.c_int, P, ctypes.c_int,
+                       ctypes.c_float, P, P, ctypes.c_uint, ctypes.c_uint64, P, P, P,
+                       ctypes.c_size_t, P]
+    assert sample(a, a, 1.0, 2, (1 << 23) + 1, a, 4, 1.2, pp, a, 0, 0, None, a, a, 1 << 30,
+                  None) == 2
+    # no noise, a bad temperature, unknown flags
+    assert sample(a, None, 1.0, 2, 100, a, 4, 1.2, pp, a, 0, 0, None, a, a, 1 << 30, None) == 1
+    for t in (0.0, -1.0, float("inf"), float("nan")):
+        assert sample(a, a, t, 2, 100, a, 4, 1.2, pp, a, 0, 0, None, a, a, 1 << 30, None) == 1
+    assert sample(a, a, 1.0, 2, 100, a, 4, 1.2, pp, a, 8, 0, None, a, a, 1 << 30, None) == 1
 
 
 def test_workspace_sizes_are_positive_and_zero_for_invalid(lib):

@@ -5,12 +5,17 @@ accepted path, through the C ABI, against the fp64/binary32 oracle.
   window (aiboss88, "Contextual penalty strategy");
 * TS_ACCEPT_RANDOM_TIE: the kept node is the (r mod c)-th of the c deepest
   valid nodes (aiboss88, tree-based verification: "randomly selected");
+* ts_penalize_sample_accept: temperature acceptance, each node's target
+  token the Gumbel-max draw from softmax(penalised / temperature) with
+  caller-drawn noise (aiboss88, tree-based verification: lossless, with
+  diversity);
 * ts_kv_commit_path: the accepted path's tree rows move to the context end
   (tencent, parallel-verification figure).
 
-All integer results are compared exactly: argmax, accepted length, bonus,
-path, and the committed cache rows bit for bit.
+All integer results are compared exactly: argmax, draws, accepted length,
+bonus, path, and the committed cache rows bit for bit.
 """
+import ctypes
 import json
 import os
 
@@ -128,6 +133,130 @@ def test_path_window_bad_token_sets_status():
     assert L.workspace_status(ws) == 6
     L.penalize_accept(lg, None, 1.2, [-1, 0], dev_i32([0, 99]), workspace=ws, flags=PATH)
     assert L.workspace_status(ws) == 0
+
+
+# ------------------------------------------------------- temperature draw
+def run_sample(logits, gumbel, temperature, window, penalty, parent, tokens, flags=0, r=0):
+    acc, tg = L.penalize_sample_accept(dev_f32(logits), dev_f32(gumbel), temperature,
+                                       dev_i32(window), penalty, parent, dev_i32(tokens),
+                                       flags=flags, random=r)
+    torch.cuda.synchronize()
+    return acc.cpu().numpy(), tg.cpu().numpy()
+
+
+def test_temperature_golden_cases():
+    t = json.load(open(GOLDEN))["temperature"]
+    none = np.zeros(0, np.int32)
+    for c in t["draws"]:
+        pen = np.array(c["penalized"], np.float32)
+        _, tg = run_sample(pen, np.array(c["gumbel"], np.float32), c["temperature"], none, 1.2,
+                           I.chain_tree(len(pen)), np.zeros(len(pen), np.int32))
+        np.testing.assert_array_equal(tg, c["expected"], err_msg=c["name"])
+    c = t["tree"]
+    acc, tg = run_sample(np.array(c["penalized"], np.float32), np.array(c["gumbel"], np.float32),
+                         c["temperature"], none, 1.2, c["parent"], c["tokens"])
+    np.testing.assert_array_equal(tg, c["expected_draws"])
+    np.testing.assert_array_equal(acc[:len(c["expected_accept"])], c["expected_accept"])
+
+
+@pytest.mark.parametrize("temperature", [0.6, 1.0, 1.7])
+@pytest.mark.parametrize("w", [I.TINY, I.LLAMA8B_32K, I.MHA7B_100K], ids=lambda w: w.name)
+def test_temperature_workloads(oracle_mod, w, temperature):
+    """The workloads' logits (planted maxima), window and seeded noise: the
+    draws against the oracle's, then tokens re-planted on the oracle's draws
+    so that the accepted path runs deep, with and without the random tie."""
+    parent = w.parent()
+    tokens, lg = I.gen_tree_tokens(w, parent, I.gen_logits(w))
+    win = I.gen_window(w)
+    g = I.gen_gumbel(w, draw=int(temperature * 10))
+    am, pen = oracle_mod.penalize_argmax(lg, win, w.penalty, return_penalized=True)
+    want = oracle_mod.sample_targets(pen, g, temperature)
+    assert (want != am).any()   # the draw is not the argmax
+    acc, tg = run_sample(lg, g, temperature, win, w.penalty, parent, tokens)
+    np.testing.assert_array_equal(tg, want)
+    np.testing.assert_array_equal(acc, oracle_mod.accept_longest(parent, tokens, want))
+    # every child carries its parent's draw: every node is valid, the leaves tie
+    deep = tokens.copy()
+    deep[1:] = want[parent[1:]]
+    for r in (0, 1, 7, 2 ** 64 - 1):
+        acc, tg = run_sample(lg, g, temperature, win, w.penalty, parent, deep, RAND, r)
+        np.testing.assert_array_equal(tg, want)
+        np.testing.assert_array_equal(acc, oracle_mod.accept_longest_random(parent, deep, want, r))
+    depth = np.zeros(len(parent), np.int64)
+    for i in range(1, len(parent)):
+        depth[i] = depth[parent[i]] + 1
+    assert acc[0] == depth.max()
+
+
+def test_temperature_with_path_window(oracle_mod):
+    w = I.LLAMA8B_32K
+    parent = w.parent()
+    lg = I.gen_logits(w)
+    win = I.gen_window(w)
+    tokens, lg = I.gen_tree_tokens(w, parent, lg)
+    tokens[1:] = np.argmax(lg[1:], axis=1).astype(np.int32)
+    g = I.gen_gumbel(w, draw=3)
+    _, pen = oracle_mod.penalize_argmax_path(lg, win, parent, tokens, w.penalty,
+                                             return_penalized=True)
+    want = oracle_mod.sample_targets(pen, g, 0.8)
+    acc, tg = run_sample(lg, g, 0.8, win, w.penalty, parent, tokens, PATH)
+    np.testing.assert_array_equal(tg, want)
+    np.testing.assert_array_equal(acc, oracle_mod.accept_longest(parent, tokens, want))
+
+
+def test_temperature_one_without_noise_is_the_argmax_call(oracle_mod):
+    w = I.LLAMA8B_32K
+    parent = w.parent()
+    tokens, lg = I.gen_tree_tokens(w, parent, I.gen_logits(w))
+    win = I.gen_window(w)
+    acc, tg = run_sample(lg, np.zeros_like(lg), 1.0, win, w.penalty, parent, tokens)
+    acc0, am0 = run_pen(lg, win, w.penalty, parent, tokens, 0)
+    np.testing.assert_array_equal(tg, am0)
+    np.testing.assert_array_equal(acc, acc0)
+    np.testing.assert_array_equal(tg, oracle_mod.penalize_argmax(lg, win, w.penalty))
+
+
+def test_temperature_ragged_vocab_and_nan(oracle_mod):
+    """A vocabulary that is not a multiple of 4 (the scalar route), NaN
+    logits and NaN noise, against the oracle."""
+    rng = np.random.default_rng(51)
+    t, vocab = 13, 1001
+    parent = I.bfs_tree(t)
+    lg = rng.normal(0, 2, size=(t, vocab)).astype(np.float32)
+    g = rng.gumbel(size=(t, vocab)).astype(np.float32)
+    lg[2, ::7] = np.nan
+    g[5, ::3] = np.nan
+    win = rng.integers(0, vocab, size=64).astype(np.int32)
+    tokens = rng.integers(0, vocab, size=t).astype(np.int32)
+    _, pen = oracle_mod.penalize_argmax(lg, win, 1.3, return_penalized=True)
+    want = oracle_mod.sample_targets(pen, g, 1.4)
+    tokens[1:] = want[parent[1:]]
+    acc, tg = run_sample(lg, g, 1.4, win, 1.3, parent, tokens)
+    np.testing.assert_array_equal(tg, want)
+    np.testing.assert_array_equal(acc, oracle_mod.accept_longest(parent, tokens, want))
+
+
+def test_temperature_rejects_bad_arguments():
+    lib = L.library()
+    lg = dev_f32(np.zeros((2, 8), np.float32))
+    g = dev_f32(np.zeros((2, 12), np.float32))
+    tok = dev_i32([0, 0])
+    acc = torch.empty(4, dtype=torch.int32, device="cuda")
+    ws = L.new_workspace(L.penalize_accept_workspace_size(2, 8))
+    par = np.array([-1, 0], np.int32)
+    P = ctypes.c_void_p
+
+    def call(gptr, temp):
+        return lib.ts_penalize_sample_accept(
+            P(lg.data_ptr()), gptr, temp, 2, 8, None, 0, 1.2, par.ctypes.data_as(P),
+            P(tok.data_ptr()), 0, 0, None, P(acc.data_ptr()), P(ws.data_ptr()), ws.numel(), None)
+
+    assert call(P(g.data_ptr()), 1.0) == 0
+    torch.cuda.synchronize()
+    assert call(None, 1.0) == 1
+    assert call(P(g.data_ptr() + 4), 1.0) == 1     # not 16-byte aligned
+    for bad in (0.0, -0.5, float("inf"), float("nan")):
+        assert call(P(g.data_ptr()), bad) == 1
 
 
 # ------------------------------------------------------------------ commit
