@@ -125,13 +125,38 @@ def _stream(stream):
     return ctypes.c_void_p(s.cuda_stream)
 
 
-def _check_dev(name, t, dtype):
+def _check_dev(name, t, dtype, device=None):
     if not isinstance(t, torch.Tensor) or not t.is_cuda:
         raise ValueError(f"{name} must be a CUDA tensor")
     if t.dtype != dtype:
         raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
     if not t.is_contiguous():
         raise ValueError(f"{name} must be contiguous")
+    if device is not None and t.device != device:
+        raise ValueError(f"{name} is on {t.device}, the call's other tensors on {device}")
+
+
+def _call_device(name, t):
+    """The device a call runs on: that of its first tensor, which must be the
+    current CUDA device (the kernels launch there, on its current stream)."""
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    cur = torch.cuda.current_device()
+    if t.device.index != cur:
+        raise ValueError(f"{name} is on {t.device} but the current device is cuda:{cur}")
+    return t.device
+
+
+def _ws_bytes(workspace, device):
+    """Size in bytes of a workspace, after checking that it is a contiguous
+    CUDA tensor on the call's device."""
+    if not isinstance(workspace, torch.Tensor) or not workspace.is_cuda:
+        raise ValueError("workspace must be a CUDA tensor")
+    if workspace.device != device:
+        raise ValueError(f"workspace is on {workspace.device}, the call's tensors on {device}")
+    if not workspace.is_contiguous():
+        raise ValueError("workspace must be contiguous")
+    return workspace.numel() * workspace.element_size()
 
 
 def _host_i32(a):
@@ -169,29 +194,30 @@ def tree_verify_attn(q, k_cache, v_cache, n_ctx: int, parent, out=None, workspac
     :func:`kv_select_from_scores`.
     """
     _check_dev("q", q, torch.bfloat16)
-    _check_dev("k_cache", k_cache, torch.bfloat16)
-    _check_dev("v_cache", v_cache, torch.bfloat16)
+    dev = _call_device("q", q)
+    _check_dev("k_cache", k_cache, torch.bfloat16, dev)
+    _check_dev("v_cache", v_cache, torch.bfloat16, dev)
     t, hq, d = q.shape
     hkv, cap, d2 = k_cache.shape
     if v_cache.shape != k_cache.shape or d2 != d:
         raise ValueError("k_cache / v_cache / q shapes disagree")
     if out is None:
-        out = torch.empty((t, hq, d), dtype=torch.float32, device=q.device)
-    _check_dev("out", out, torch.float32)
+        out = torch.empty((t, hq, d), dtype=torch.float32, device=dev)
+    _check_dev("out", out, torch.float32, dev)
     if workspace is None:
-        workspace = new_workspace(tree_verify_attn_workspace_size(hq, hkv, d, n_ctx, t), q.device)
+        workspace = new_workspace(tree_verify_attn_workspace_size(hq, hkv, d, n_ctx, t), dev)
     par, par_p = _host_i32(parent)
     if len(par) != t:
         raise ValueError("parent must have one entry per tree node")
     scale = float(d) ** -0.5 if softmax_scale is None else float(softmax_scale)
-    ws_bytes = workspace.numel() * workspace.element_size()
+    ws_bytes = _ws_bytes(workspace, dev)
     if root_scores_out is None:
         rc = _lib().ts_tree_verify_attn(_ptr(q), _ptr(k_cache), _ptr(v_cache), cap, hq, hkv, d,
                                         int(n_ctx), t, par_p, scale, _ptr(out), _ptr(workspace),
                                         ws_bytes, _stream(stream))
         _raise(rc, "ts_tree_verify_attn")
         return out
-    _check_dev("root_scores_out", root_scores_out, torch.float32)
+    _check_dev("root_scores_out", root_scores_out, torch.float32, dev)
     if tuple(root_scores_out.shape) != (hq, int(n_ctx)):
         raise ValueError("root_scores_out must be [Hq, n_ctx]")
     rc = _lib().ts_tree_verify_attn_root_scores(
@@ -216,12 +242,12 @@ def kv_importance_select(q_last, k_cache, v_cache, n_ctx: int, n_sink: int, budg
     Returns ``(idx [Hkv, n_keep] int32, k_partial, v_partial, scores or None)``.
     """
     _check_dev("q_last", q_last, torch.bfloat16)
-    _check_dev("k_cache", k_cache, torch.bfloat16)
-    _check_dev("v_cache", v_cache, torch.bfloat16)
+    dev = _call_device("q_last", q_last)
+    _check_dev("k_cache", k_cache, torch.bfloat16, dev)
+    _check_dev("v_cache", v_cache, torch.bfloat16, dev)
     hq, d = q_last.shape
     hkv, cap, d2 = k_cache.shape
     n_keep = min(n_ctx, n_sink + budget)
-    dev = q_last.device
     if k_partial is None:
         k_partial = torch.empty((hkv, n_keep, d), dtype=torch.bfloat16, device=dev)
     if v_partial is None:
@@ -233,16 +259,16 @@ def kv_importance_select(q_last, k_cache, v_cache, n_ctx: int, n_sink: int, budg
     for name, t, dt in (("k_partial", k_partial, torch.bfloat16),
                         ("v_partial", v_partial, torch.bfloat16),
                         ("idx_out", idx_out, torch.int32)):
-        _check_dev(name, t, dt)
+        _check_dev(name, t, dt, dev)
     if scores_out is not None:
-        _check_dev("scores_out", scores_out, torch.float32)
+        _check_dev("scores_out", scores_out, torch.float32, dev)
     if workspace is None:
         workspace = new_workspace(kv_importance_select_workspace_size(hq, hkv, d, n_ctx), dev)
     scale = float(d) ** -0.5 if softmax_scale is None else float(softmax_scale)
     rc = _lib().ts_kv_importance_select(
         _ptr(q_last), _ptr(k_cache), _ptr(v_cache), cap, hq, hkv, d, int(n_ctx), int(n_sink),
         int(budget), scale, _ptr(scores_out), _ptr(idx_out), _ptr(k_partial), _ptr(v_partial),
-        k_partial.shape[1], _ptr(workspace), workspace.numel(), _stream(stream))
+        k_partial.shape[1], _ptr(workspace), _ws_bytes(workspace, dev), _stream(stream))
     _raise(rc, "ts_kv_importance_select")
     return idx_out, k_partial, v_partial, scores_out
 
@@ -260,14 +286,14 @@ def kv_select_from_scores(root_scores, k_cache, v_cache, n_ctx: int, n_sink: int
     Returns ``(idx [Hkv, n_keep] int32, k_partial, v_partial, scores or None)``.
     """
     _check_dev("root_scores", root_scores, torch.float32)
-    _check_dev("k_cache", k_cache, torch.bfloat16)
-    _check_dev("v_cache", v_cache, torch.bfloat16)
+    dev = _call_device("root_scores", root_scores)
+    _check_dev("k_cache", k_cache, torch.bfloat16, dev)
+    _check_dev("v_cache", v_cache, torch.bfloat16, dev)
     hq, n = root_scores.shape
     if n != int(n_ctx):
         raise ValueError("root_scores must be [Hq, n_ctx]")
     hkv, cap, d = k_cache.shape
     n_keep = min(n_ctx, n_sink + budget)
-    dev = root_scores.device
     if k_partial is None:
         k_partial = torch.empty((hkv, n_keep, d), dtype=torch.bfloat16, device=dev)
     if v_partial is None:
@@ -279,15 +305,16 @@ def kv_select_from_scores(root_scores, k_cache, v_cache, n_ctx: int, n_sink: int
     for name, t, dt in (("k_partial", k_partial, torch.bfloat16),
                         ("v_partial", v_partial, torch.bfloat16),
                         ("idx_out", idx_out, torch.int32)):
-        _check_dev(name, t, dt)
+        _check_dev(name, t, dt, dev)
     if scores_out is not None:
-        _check_dev("scores_out", scores_out, torch.float32)
+        _check_dev("scores_out", scores_out, torch.float32, dev)
     if workspace is None:
         workspace = new_workspace(kv_select_from_scores_workspace_size(hq, hkv, int(n_ctx)), dev)
     rc = _lib().ts_kv_select_from_scores(
         _ptr(root_scores), _ptr(k_cache), _ptr(v_cache), cap, hq, hkv, d, int(n_ctx),
         int(n_sink), int(budget), _ptr(scores_out), _ptr(idx_out), _ptr(k_partial),
-        _ptr(v_partial), k_partial.shape[1], _ptr(workspace), workspace.numel(), _stream(stream))
+        _ptr(v_partial), k_partial.shape[1], _ptr(workspace), _ws_bytes(workspace, dev),
+        _stream(stream))
     _raise(rc, "ts_kv_select_from_scores")
     return idx_out, k_partial, v_partial, scores_out
 
@@ -309,11 +336,11 @@ def penalize_accept(logits, window, penalty: float, parent, tree_tokens, argmax_
     Returns ``(accept [2 + T] int32, argmax [T] int32 or None)``.
     """
     _check_dev("logits", logits, torch.float32)
-    _check_dev("tree_tokens", tree_tokens, torch.int32)
+    dev = _call_device("logits", logits)
+    _check_dev("tree_tokens", tree_tokens, torch.int32, dev)
     t, vocab = logits.shape
-    dev = logits.device
     if window is not None and window.numel() > 0:
-        _check_dev("window", window, torch.int32)
+        _check_dev("window", window, torch.int32, dev)
         wlen, wptr = window.numel(), _ptr(window)
     else:
         wlen, wptr = 0, None
@@ -321,9 +348,9 @@ def penalize_accept(logits, window, penalty: float, parent, tree_tokens, argmax_
         accept_out = torch.empty(2 + t, dtype=torch.int32, device=dev)
     if want_argmax and argmax_out is None:
         argmax_out = torch.empty(t, dtype=torch.int32, device=dev)
-    _check_dev("accept_out", accept_out, torch.int32)
+    _check_dev("accept_out", accept_out, torch.int32, dev)
     if argmax_out is not None:
-        _check_dev("argmax_out", argmax_out, torch.int32)
+        _check_dev("argmax_out", argmax_out, torch.int32, dev)
     if workspace is None:
         workspace = new_workspace(penalize_accept_workspace_size(t, vocab), dev)
     par, par_p = _host_i32(parent)
@@ -332,13 +359,14 @@ def penalize_accept(logits, window, penalty: float, parent, tree_tokens, argmax_
     if flags == 0:
         rc = _lib().ts_penalize_accept(_ptr(logits), t, vocab, wptr, wlen, float(penalty), par_p,
                                        _ptr(tree_tokens), _ptr(argmax_out), _ptr(accept_out),
-                                       _ptr(workspace), workspace.numel(), _stream(stream))
+                                       _ptr(workspace), _ws_bytes(workspace, dev),
+                                       _stream(stream))
         _raise(rc, "ts_penalize_accept")
     else:
         rc = _lib().ts_penalize_accept_ex(
             _ptr(logits), t, vocab, wptr, wlen, float(penalty), par_p, _ptr(tree_tokens),
             int(flags), int(random) & (2 ** 64 - 1), _ptr(argmax_out), _ptr(accept_out),
-            _ptr(workspace), workspace.numel(), _stream(stream))
+            _ptr(workspace), _ws_bytes(workspace, dev), _stream(stream))
         _raise(rc, "ts_penalize_accept_ex")
     return accept_out, argmax_out
 
@@ -357,14 +385,14 @@ def penalize_sample_accept(logits, gumbel, temperature: float, window, penalty: 
     Returns ``(accept [2 + T] int32, target [T] int32 or None)``.
     """
     _check_dev("logits", logits, torch.float32)
-    _check_dev("gumbel", gumbel, torch.float32)
-    _check_dev("tree_tokens", tree_tokens, torch.int32)
+    dev = _call_device("logits", logits)
+    _check_dev("gumbel", gumbel, torch.float32, dev)
+    _check_dev("tree_tokens", tree_tokens, torch.int32, dev)
     t, vocab = logits.shape
     if tuple(gumbel.shape) != (t, vocab):
         raise ValueError("gumbel must have the logits' shape [T, V]")
-    dev = logits.device
     if window is not None and window.numel() > 0:
-        _check_dev("window", window, torch.int32)
+        _check_dev("window", window, torch.int32, dev)
         wlen, wptr = window.numel(), _ptr(window)
     else:
         wlen, wptr = 0, None
@@ -372,9 +400,9 @@ def penalize_sample_accept(logits, gumbel, temperature: float, window, penalty: 
         accept_out = torch.empty(2 + t, dtype=torch.int32, device=dev)
     if want_target and target_out is None:
         target_out = torch.empty(t, dtype=torch.int32, device=dev)
-    _check_dev("accept_out", accept_out, torch.int32)
+    _check_dev("accept_out", accept_out, torch.int32, dev)
     if target_out is not None:
-        _check_dev("target_out", target_out, torch.int32)
+        _check_dev("target_out", target_out, torch.int32, dev)
     if workspace is None:
         workspace = new_workspace(penalize_accept_workspace_size(t, vocab), dev)
     par, par_p = _host_i32(parent)
@@ -383,7 +411,7 @@ def penalize_sample_accept(logits, gumbel, temperature: float, window, penalty: 
     rc = _lib().ts_penalize_sample_accept(
         _ptr(logits), _ptr(gumbel), float(temperature), t, vocab, wptr, wlen, float(penalty),
         par_p, _ptr(tree_tokens), int(flags), int(random) & (2 ** 64 - 1), _ptr(target_out),
-        _ptr(accept_out), _ptr(workspace), workspace.numel(), _stream(stream))
+        _ptr(accept_out), _ptr(workspace), _ws_bytes(workspace, dev), _stream(stream))
     _raise(rc, "ts_penalize_sample_accept")
     return accept_out, target_out
 
@@ -394,16 +422,17 @@ def kv_commit_path(k_cache, v_cache, n_ctx: int, n_tree: int, accept, workspace=
     caches, in place (``ts_kv_commit_path``); ``accept`` is the device
     result of :func:`penalize_accept`."""
     _check_dev("k_cache", k_cache, torch.bfloat16)
-    _check_dev("v_cache", v_cache, torch.bfloat16)
-    _check_dev("accept", accept, torch.int32)
+    dev = _call_device("k_cache", k_cache)
+    _check_dev("v_cache", v_cache, torch.bfloat16, dev)
+    _check_dev("accept", accept, torch.int32, dev)
     hkv, cap, d = k_cache.shape
     if v_cache.shape != k_cache.shape:
         raise ValueError("k_cache / v_cache shapes disagree")
     if workspace is None:
-        workspace = new_workspace(256, k_cache.device)
+        workspace = new_workspace(256, dev)
     rc = _lib().ts_kv_commit_path(_ptr(k_cache), _ptr(v_cache), cap, hkv, d, int(n_ctx),
-                                  int(n_tree), _ptr(accept), _ptr(workspace), workspace.numel(),
-                                  _stream(stream))
+                                  int(n_tree), _ptr(accept), _ptr(workspace),
+                                  _ws_bytes(workspace, dev), _stream(stream))
     _raise(rc, "ts_kv_commit_path")
     return k_cache, v_cache
 
@@ -419,13 +448,15 @@ def selftest_bounded_wait(workspace=None, stream=None):
     in the workspace's status word.  Returns the workspace."""
     if workspace is None:
         workspace = new_workspace(256)
-    _raise(_lib().ts_selftest_bounded_wait(_ptr(workspace), workspace.numel(), _stream(stream)),
+    nbytes = _ws_bytes(workspace, _call_device("workspace", workspace))
+    _raise(_lib().ts_selftest_bounded_wait(_ptr(workspace), nbytes, _stream(stream)),
            "ts_selftest_bounded_wait")
     return workspace
 
 
 def workspace_status(workspace, clear: bool = True, stream=None) -> int:
     """Device-side status word of a workspace (synchronises the stream)."""
+    _ws_bytes(workspace, _call_device("workspace", workspace))
     return int(_lib().ts_workspace_status(_ptr(workspace), _stream(stream), int(clear)))
 
 
